@@ -1,0 +1,329 @@
+"""Plain fp64 CPU oracle for SAS (Simple-Attention-Sparsification) gated
+block-sparse attention: decode step and block-sparse chunked prefill.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import
+this module.  The CUDA library never calls it, links it or reads its output;
+it shares no code, tables or helpers with ``gated_block_sparse_token_b200``.
+
+Everything here is computed in float64 with numpy, one (sequence, KV head)
+or (sequence, KV head, query block) at a time, in the order the method
+states its steps.  Inputs are the exact values the GPU receives (bf16 or
+fp32 numbers widened to float64).
+
+Sources (web pages describing the release; they print no formula, so every
+formula below is a reading, flagged ``ASSUMPTION``):
+
+* [aigc-0914] "Tencent released Simple-Attention-Sparsification, a method for
+  efficient sparse attention in Qwen3 models" (aigc.news, 2026-09-14), release
+  paragraph: KV block size 64 tokens, training Top-K 31 historical blocks,
+  gate hidden size 128, query projection Qproj, key block pooling
+  max + min + average, Q/K normalization enabled, gate RoPE enabled, training
+  length 32,768, default sparse decode budget 2,048 tokens (1,024 and 4,096
+  also usable); continuous gates act on the selected blocks.
+* [lmw-en] "Simple-Attention-Sparsification Text Generation Model: 12GB+
+  VRAM" (localmodelwatch, English), "Specifications and Configuration Table":
+  the same settings, and gate parameter counts 33.0M / 33.0M / 42.0M.
+* [lmw-ja] "Tencent、Qwen3向けSASスパースアテンションチェックポイント公開"
+  (localmodelwatch, Japanese), "スペック・構成表": the same tables.
+* [nedoborov] ai-news.nedoborov.com post of 2026-09-14 on the SAS release
+  (Russian), list of sparse-attention settings: block 64, Top-K 31, length
+  32,768, budget 2,048 with 1,024 / 4,096 usable without retraining.
+
+Readings fixed where the pages are silent (each also marked in code):
+
+R1  W_q is [128][128] per query head, W_k is [384][128] per KV head, no bias,
+    applied as row vector times matrix (x @ W).  The gate parameter counts
+    ([lmw-en] table) equal layers*(Hq*128*128 + Hkv*384*128) for the Qwen3
+    head layouts.
+R2  The query fed to Qproj is the per-head attention query (head_dim 128).
+R3  The pooled keys are the K cache values attention reads.
+R4  Pooled vector order is [max; min; avg] (word order of "max + min +
+    average").
+R5  Q/K normalization is RMSNorm x / sqrt(mean(x^2) + eps) * gamma, eps 1e-6,
+    applied after the projection and before RoPE.  The gain is one
+    128-vector per layer for q and one for k, shared by all heads: with
+    per-head gains the printed counts would read 33.2M, not 33.0M.
+R6  Gate RoPE is rotate-half (pairs i, i+64), theta_i = base^(-2i/128),
+    base 10000; key position = block index b, query position = current block
+    index c (decode) or query block index i (prefill).
+R7  Gate score s_{g,b} = (q~_g . k~_b) * gate_scale, gate_scale = 1/sqrt(128).
+R8  One block set per KV head, ranked by the mean over the G query heads of
+    the group of their gate scores.
+R9  Equal group scores: the lower block index wins.
+R10 The current block c = floor((L-1)/64) is always attended and never
+    scored; the query is token L-1, which is already in the cache.
+R11 With fewer historical blocks than Top-K, all of them are kept.
+R12 Inference weights every selected block 1 (the continuous gate is the
+    training path); a budget covering the context gives dense causal
+    attention.
+R13 Prefill gate query for query block i is the mean over the block's 64
+    token queries, per query head.
+R14 Attention logits use scale 1/sqrt(128); softmax in float64.
+
+Parity status: the gate formula as a whole (R1-R8) is pinned only by the
+invariants and hand-derived closed forms in tests/test_oracle.py, not by any
+value the pages print ("parity unpinned" against the pages for the exact gate
+arithmetic; the pages print no worked example).
+"""
+from __future__ import annotations
+
+import math
+import numpy as np
+
+BLOCK = 64          # KV block size in tokens  [aigc-0914], [lmw-en] table
+HEAD_DIM = 128      # Qwen3 head_dim (attention query/key width)
+GATE_HIDDEN = 128   # gate hidden size  [aigc-0914], [lmw-en] table
+POOL_DIM = 3 * HEAD_DIM   # max, min, avg stacked  (R4)
+
+
+# --------------------------------------------------------------------------
+# Step 1: key-block pooling ([aigc-0914] "key block pooling max + min +
+# average"; R3, R4).
+# --------------------------------------------------------------------------
+def pool_block(k_block: np.ndarray) -> np.ndarray:
+    """Pooled key of one complete 64-token block.
+
+    k_block: [64][128] keys of the block.  Returns [384] =
+    [per-dim max ; per-dim min ; per-dim mean].  ASSUMPTION R4 (order).
+    """
+    k_block = np.asarray(k_block, dtype=np.float64)
+    assert k_block.shape == (BLOCK, HEAD_DIM)
+    mx = k_block.max(axis=0)
+    mn = k_block.min(axis=0)
+    avg = k_block.sum(axis=0) / BLOCK
+    return np.concatenate([mx, mn, avg])
+
+
+# --------------------------------------------------------------------------
+# Step 2 pieces: Q/K normalisation and gate RoPE ([aigc-0914] "Q/K
+# normalization enabled", "gate RoPE enabled"; R5, R6).
+# --------------------------------------------------------------------------
+def rms_norm(x: np.ndarray, gamma: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * gamma.  ASSUMPTION R5."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / math.sqrt(float(np.mean(x * x)) + eps) * np.asarray(gamma, np.float64)
+
+
+def rope_rotate_half(x: np.ndarray, pos: int, base: float = 10000.0) -> np.ndarray:
+    """Rotary embedding of a 128-vector at integer position ``pos``.
+
+    Pairs (i, i+64), angle pos * base^(-2i/128):
+      y_i      = x_i cos - x_{i+64} sin
+      y_{i+64} = x_{i+64} cos + x_i sin
+    ASSUMPTION R6 (rotate-half convention, base 10000).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    half = x.shape[-1] // 2
+    i = np.arange(half, dtype=np.float64)
+    theta = base ** (-2.0 * i / x.shape[-1])
+    ang = float(pos) * theta
+    c, s = np.cos(ang), np.sin(ang)
+    lo, hi = x[:half], x[half:]
+    return np.concatenate([lo * c - hi * s, hi * c + lo * s])
+
+
+def gate_key(pooled: np.ndarray, w_k: np.ndarray, gamma_k: np.ndarray, pos: int,
+             eps: float = 1e-6, base: float = 10000.0) -> np.ndarray:
+    """k~_b = RoPE(RMSNorm(pooled @ W_k) , b).  W_k: [384][128].  R1, R5, R6."""
+    u = np.asarray(pooled, np.float64) @ np.asarray(w_k, np.float64)
+    return rope_rotate_half(rms_norm(u, gamma_k, eps), pos, base)
+
+
+def gate_query(q: np.ndarray, w_q: np.ndarray, gamma_q: np.ndarray, pos: int,
+               eps: float = 1e-6, base: float = 10000.0) -> np.ndarray:
+    """q~ = RoPE(RMSNorm(q @ W_q), pos) ("query projection Qproj").  W_q: [128][128].
+    R1, R2, R5, R6."""
+    v = np.asarray(q, np.float64) @ np.asarray(w_q, np.float64)
+    return rope_rotate_half(rms_norm(v, gamma_q, eps), pos, base)
+
+
+def gate_keys_for_sequence(k_seq: np.ndarray, num_blocks: int, w_k: np.ndarray,
+                           gamma_k: np.ndarray, eps: float = 1e-6,
+                           base: float = 10000.0) -> np.ndarray:
+    """Gate keys of blocks 0..num_blocks-1 of one (sequence, KV head).
+
+    k_seq: [>= 64*num_blocks][128].  Returns [num_blocks][128]."""
+    out = np.zeros((num_blocks, GATE_HIDDEN))
+    for b in range(num_blocks):
+        pooled = pool_block(k_seq[b * BLOCK:(b + 1) * BLOCK])
+        out[b] = gate_key(pooled, w_k, gamma_k, b, eps, base)
+    return out
+
+
+# --------------------------------------------------------------------------
+# Steps 2-3: gate scores and Top-K selection ([aigc-0914] "learns to rank
+# and select KV blocks", training Top-K 31, budget 2,048; [nedoborov] list).
+# --------------------------------------------------------------------------
+def gate_scores(q_group: np.ndarray, w_q_group: np.ndarray, gamma_q_group: np.ndarray,
+                gate_keys: np.ndarray, n_hist: int, q_pos: int,
+                gate_scale: float = 1.0 / math.sqrt(128.0), eps: float = 1e-6,
+                base: float = 10000.0):
+    """Per-head and group gate scores of the historical blocks 0..n_hist-1.
+
+    q_group:       [G][128] queries of the G query heads sharing a KV head.
+    w_q_group:     [G][128][128].   gamma_q_group: [G][128].
+    gate_keys:     [>= n_hist][128] k~ of the KV head.
+    Returns (s [G][n_hist], S [n_hist]) with s_{g,b} = q~_g . k~_b * scale
+    (R7) and S_b = mean_g s_{g,b} (R8).
+    """
+    G = q_group.shape[0]
+    s = np.zeros((G, n_hist))
+    for g in range(G):
+        qt = gate_query(q_group[g], w_q_group[g], gamma_q_group[g], q_pos, eps, base)
+        for b in range(n_hist):
+            s[g, b] = float(np.dot(qt, gate_keys[b])) * gate_scale
+    S = s.sum(axis=0) / G if n_hist else np.zeros(0)
+    return s, S
+
+
+def select_blocks(S: np.ndarray, n_hist: int, topk: int) -> list[int]:
+    """Ascending block list: the min(topk, n_hist) historical blocks with the
+    largest group score (ties -> lower index, R9), then the current block
+    ``n_hist`` (R10, R11).  Selection by a full sort of (-S_b, b)."""
+    order = sorted(range(n_hist), key=lambda b: (-float(S[b]), b))
+    kept = sorted(order[:min(topk, n_hist)])
+    return kept + [n_hist]
+
+
+def topk_for_budget(token_budget: int) -> int:
+    """Historical blocks kept for a token budget: budget/64 - 1 (the current
+    block takes the remaining 64 tokens: 31 + 1 = 2048/64)."""
+    assert token_budget % BLOCK == 0 and token_budget >= BLOCK
+    return token_budget // BLOCK - 1
+
+
+# --------------------------------------------------------------------------
+# Step 4: attention over the selected blocks (R12, R14).
+# --------------------------------------------------------------------------
+def attention_over_tokens(q: np.ndarray, k: np.ndarray, v: np.ndarray,
+                          token_ids, scale: float) -> np.ndarray:
+    """softmax(q . k_j * scale) weighted sum of v_j over the listed tokens,
+    two-pass (max, then exp-sum) in float64."""
+    idx = np.asarray(list(token_ids), dtype=np.int64)
+    logits = (k[idx].astype(np.float64) @ np.asarray(q, np.float64)) * scale
+    m = logits.max()
+    p = np.exp(logits - m)
+    return (p @ v[idx].astype(np.float64)) / p.sum()
+
+
+def selected_token_ids(blocks, seq_len: int):
+    """Token positions covered by the listed blocks, clipped to the context
+    (only the current block can be partial)."""
+    out = []
+    for b in blocks:
+        out.extend(range(b * BLOCK, min((b + 1) * BLOCK, seq_len)))
+    return out
+
+
+def decode_one_group(q_group, k_seq, v_seq, seq_len, gate_keys, w_q_group,
+                     gamma_q_group, token_budget, attn_scale=1.0 / math.sqrt(128.0),
+                     gate_scale=1.0 / math.sqrt(128.0), eps=1e-6, base=10000.0):
+    """Decode step of one (sequence, KV head): gate, select, attend.
+
+    q_group [G][128]: queries of token L-1 for the G heads of the group.
+    k_seq, v_seq [>= L][128]: the head's cache.  gate_keys [>= c][128].
+    Returns dict(out [G][128], sel (ascending list), s [G][c], S [c]).
+    """
+    c = (seq_len - 1) // BLOCK            # current block (R10)
+    s, S = gate_scores(q_group, w_q_group, gamma_q_group, gate_keys, c, c,
+                       gate_scale, eps, base)
+    sel = select_blocks(S, c, topk_for_budget(token_budget))
+    toks = selected_token_ids(sel, seq_len)
+    out = np.stack([attention_over_tokens(q_group[g], k_seq, v_seq, toks, attn_scale)
+                    for g in range(q_group.shape[0])])
+    return {"out": out, "sel": sel, "s": s, "S": S}
+
+
+def dense_causal_decode(q_group, k_seq, v_seq, seq_len,
+                        attn_scale=1.0 / math.sqrt(128.0)):
+    """Plain dense attention of token L-1 over tokens 0..L-1 (no gate, no
+    blocks); what a budget covering the whole context must reduce to."""
+    out = np.zeros((q_group.shape[0], HEAD_DIM))
+    for g in range(q_group.shape[0]):
+        logits = np.array([float(np.dot(q_group[g], k_seq[j])) for j in range(seq_len)]) * attn_scale
+        w = np.exp(logits - logits.max())
+        w /= w.sum()
+        acc = np.zeros(HEAD_DIM)
+        for j in range(seq_len):
+            acc += w[j] * np.asarray(v_seq[j], np.float64)
+        out[g] = acc
+    return out
+
+
+# --------------------------------------------------------------------------
+# Block-sparse chunked prefill (training setting: Top-K 31 over 32,768-token
+# sequences, [aigc-0914]; R13).
+# --------------------------------------------------------------------------
+def prefill_query_block(q_blk_group, k_seq, v_seq, i, gate_keys, w_q_group,
+                        gamma_q_group, topk, attn_scale=1.0 / math.sqrt(128.0),
+                        gate_scale=1.0 / math.sqrt(128.0), eps=1e-6, base=10000.0):
+    """One (sequence, KV head, query block i) of block-sparse causal prefill.
+
+    q_blk_group [G][64][128]: queries of block i for the G heads.
+    Gate query of head g = mean over the block's 64 queries (R13), placed at
+    position i; historical blocks 0..i-1 scored; top-min(topk, i) kept plus
+    the diagonal block i; token t of block i attends to all tokens of the
+    kept historical blocks and to tokens 64i..t of block i.
+    Returns dict(out [G][64][128], sel, S).
+    """
+    G = q_blk_group.shape[0]
+    qbar = q_blk_group.astype(np.float64).mean(axis=1)
+    _, S = gate_scores(qbar, w_q_group, gamma_q_group, gate_keys, i, i,
+                       gate_scale, eps, base)
+    sel = select_blocks(S, i, topk)
+    hist_toks = selected_token_ids(sel[:-1], (i + 1) * BLOCK)
+    out = np.zeros((G, BLOCK, HEAD_DIM))
+    for g in range(G):
+        for t in range(BLOCK):
+            toks = hist_toks + list(range(i * BLOCK, i * BLOCK + t + 1))
+            out[g, t] = attention_over_tokens(q_blk_group[g, t], k_seq, v_seq, toks, attn_scale)
+    return {"out": out, "sel": sel, "S": S}
+
+
+def dense_causal_prefill(q_seq, k_seq, v_seq, attn_scale=1.0 / math.sqrt(128.0)):
+    """Dense causal attention of every token of one head: [T][128] -> [T][128]."""
+    T = q_seq.shape[0]
+    logits = (q_seq.astype(np.float64) @ k_seq.astype(np.float64).T) * attn_scale
+    out = np.zeros((T, HEAD_DIM))
+    for t in range(T):
+        row = logits[t, :t + 1]
+        w = np.exp(row - row.max())
+        out[t] = (w @ v_seq[:t + 1].astype(np.float64)) / w.sum()
+    return out
+
+
+# --------------------------------------------------------------------------
+# Batched drivers (loops over sequences and KV heads) used by tests/bench.
+# Layouts: q [B][Hq][128]; contiguous cache [B][Hkv][cap][128]; gate weights
+# w_q [Hq][128][128], w_k [Hkv][384][128]; gains gamma_q [128] and gamma_k
+# [128], one each per layer (reading R5b: the printed parameter counts fit
+# one shared gain per layer, not one per head).  Query head g belongs to KV
+# head g // G (G = Hq / Hkv).
+# --------------------------------------------------------------------------
+def decode_step(q, k_cache, v_cache, seq_lens, w_q, gamma_q, w_k, gamma_k,
+                token_budget, gate_keys=None, pairs=None, eps=1e-6, base=10000.0):
+    """Full decode step for the listed (sequence, KV head) pairs (all if None).
+
+    gate_keys: optional precomputed [B][Hkv][>=c][128]; computed from the
+    cache when None.  Returns {(s, h): decode_one_group(...)}.
+    """
+    B, Hq = q.shape[0], q.shape[1]
+    Hkv = k_cache.shape[1]
+    G = Hq // Hkv
+    if pairs is None:
+        pairs = [(s, h) for s in range(B) for h in range(Hkv)]
+    res = {}
+    for (s, h) in pairs:
+        L = int(seq_lens[s])
+        c = (L - 1) // BLOCK
+        ks, vs = k_cache[s, h], v_cache[s, h]
+        if gate_keys is None:
+            gk = gate_keys_for_sequence(ks, c, w_k[h], gamma_k, eps, base)
+        else:
+            gk = np.asarray(gate_keys[s, h, :c], np.float64)
+        heads = slice(h * G, (h + 1) * G)
+        res[(s, h)] = decode_one_group(np.asarray(q[s, heads], np.float64), ks, vs, L, gk,
+                                       w_q[heads], np.tile(gamma_q, (G, 1)), token_budget,
+                                       eps=eps, base=base)
+    return res

@@ -1,0 +1,363 @@
+"""Pins for the fp64 CPU oracle, independent of the oracle's own code paths.
+
+Each check comes from something other than the oracle: a closed form derived
+by hand, an invariant of the mathematics, a brute-force search on tiny
+inputs, or a separately written dense-attention reduction.  The last test
+plants plausible mistakes in the oracle (on the CPU) and shows that the pins
+catch them.
+
+Sources: "Tencent released Simple-Attention-Sparsification ..." (aigc.news,
+2026-09-14), release paragraph, and "Simple-Attention-Sparsification Text
+Generation Model: 12GB+ VRAM" (localmodelwatch), "Specifications and
+Configuration Table": block 64, Top-K 31, gate hidden 128, Qproj, max + min +
+average pooling, Q/K normalization, gate RoPE, budgets 1,024/2,048/4,096.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+from oracle import sas_oracle as O
+
+EPS = 1e-6
+SCALE = 1.0 / math.sqrt(128.0)
+
+
+# ---------------------------------------------------------------- pooling
+def test_pool_closed_form():
+    # K[j][d] = 0.5 j - 0.25 d : max at j=63, min at j=0, mean at j=31.5
+    j = np.arange(64)[:, None]
+    d = np.arange(128)[None, :]
+    kb = 0.5 * j - 0.25 * d
+    p = O.pool_block(kb)
+    dd = np.arange(128)
+    assert np.array_equal(p[:128], 0.5 * 63 - 0.25 * dd)
+    assert np.array_equal(p[128:256], -0.25 * dd)
+    assert np.allclose(p[256:], 0.5 * 31.5 - 0.25 * dd, rtol=0, atol=1e-12)
+
+
+def test_pool_brute_force_random():
+    rng = np.random.default_rng(5)
+    kb = rng.standard_normal((64, 128)).astype(np.float32).astype(np.float64)
+    p = O.pool_block(kb)
+    for dim in (0, 17, 127):
+        col = [kb[t][dim] for t in range(64)]
+        m_hi = col[0]
+        m_lo = col[0]
+        tot = 0.0
+        for x in col:
+            m_hi = x if x > m_hi else m_hi
+            m_lo = x if x < m_lo else m_lo
+            tot += x
+        assert p[dim] == m_hi and p[128 + dim] == m_lo  # order-free: bit-exact
+        assert abs(p[256 + dim] - tot / 64) <= 1e-12
+
+
+# ---------------------------------------------------------------- RMSNorm
+def test_rmsnorm_unit_rms_and_scale_free():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal(128) * 3.0
+    y = O.rms_norm(x, np.ones(128), EPS)
+    ms = np.mean(x * x)
+    assert abs(math.sqrt(np.mean(y * y)) - math.sqrt(ms / (ms + EPS))) < 1e-12
+    y2 = O.rms_norm(7.0 * x, np.ones(128), EPS)
+    assert np.allclose(y, y2, rtol=1e-6, atol=0)
+    g = rng.standard_normal(128)
+    assert np.allclose(O.rms_norm(x, g, EPS), y * g, rtol=1e-14, atol=1e-14)
+
+
+# ---------------------------------------------------------------- RoPE
+def test_rope_pos0_identity_and_norm():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal(128)
+    assert np.allclose(O.rope_rotate_half(x, 0), x, atol=0, rtol=0)
+    y = O.rope_rotate_half(x, 1234)
+    assert abs(np.linalg.norm(y) - np.linalg.norm(x)) < 1e-10
+
+
+def test_rope_closed_form_basis_vectors():
+    # pair (0, 64) turns at 1 rad per position; pair (1, 65) at 10000^(-1/64)
+    e = np.eye(128)
+    for pos in (0, 1, 5, 511, 2047):
+        y0 = O.rope_rotate_half(e[0], pos)
+        exp0 = math.cos(pos) * e[0] + math.sin(pos) * e[64]
+        assert np.allclose(y0, exp0, atol=1e-12)
+        y64 = O.rope_rotate_half(e[64], pos)
+        assert np.allclose(y64, -math.sin(pos) * e[0] + math.cos(pos) * e[64], atol=1e-12)
+        th1 = 10000.0 ** (-2.0 / 128.0)
+        y1 = O.rope_rotate_half(e[1], pos)
+        assert np.allclose(y1, math.cos(pos * th1) * e[1] + math.sin(pos * th1) * e[65], atol=1e-12)
+
+
+def test_rope_relative_position_invariance():
+    rng = np.random.default_rng(3)
+    x, y = rng.standard_normal(128), rng.standard_normal(128)
+    a = np.dot(O.rope_rotate_half(x, 40), O.rope_rotate_half(y, 13))
+    b = np.dot(O.rope_rotate_half(x, 40 + 300), O.rope_rotate_half(y, 13 + 300))
+    assert abs(a - b) < 1e-9 * max(1.0, abs(a))
+
+
+# ---------------------------------------------------------------- gate, hand-derived closed form
+def _closed_form_inputs(c):
+    """Blocks whose dim 64 alternates +1 / -3 (max 1, min -3, avg -1), all other
+    dims 0; W_k sends max(dim64) -> u_64, min(dim64) -> u_0, avg(dim64) -> u_1;
+    W_q = I; q = e_0; gains 1."""
+    n = c
+    k = np.zeros((64 * (c + 1), 128))
+    k[0::2, 64] = 1.0
+    k[1::2, 64] = -3.0
+    w_k = np.zeros((384, 128))
+    w_k[64, 64] = 1.0            # max part
+    w_k[128 + 64, 0] = 1.0       # min part
+    w_k[256 + 64, 1] = 1.0       # avg part
+    w_q = np.eye(128)[None]
+    q = np.zeros((1, 128))
+    q[0, 0] = 1.0
+    return n, k, w_k, w_q, q
+
+
+def test_gate_scores_closed_form():
+    # u = 1 e64 - 3 e0 - 1 e1 ; |u|^2/128 = 11/128 ; RoPE at b; q~ = a(cos c e0 + sin c e64)
+    # s_b = a * kn * (-3 cos(c-b) + sin(c-b) + 0) * scale   (pair (1,65) meets q~ = 0)
+    c = 9
+    n, k, w_k, w_q, q = _closed_form_inputs(c)
+    gk = O.gate_keys_for_sequence(k, n, w_k, np.ones(128), EPS)
+    s, S = O.gate_scores(q, w_q, np.ones((1, 128)), gk, n, c, SCALE, EPS)
+    a = 1.0 / math.sqrt(1.0 / 128 + EPS)
+    kn = 1.0 / math.sqrt(11.0 / 128 + EPS)
+    for b in range(n):
+        want = a * kn * (-3.0 * math.cos(c - b) + math.sin(c - b)) * SCALE
+        assert abs(s[0, b] - want) < 1e-12, (b, s[0, b], want)
+        assert S[b] == s[0, b]
+
+
+def test_gate_group_score_is_mean_over_heads():
+    rng = np.random.default_rng(4)
+    G, c = 4, 12
+    k = rng.standard_normal((64 * (c + 1), 128))
+    w_k = rng.standard_normal((384, 128)) / math.sqrt(384)
+    gk = O.gate_keys_for_sequence(k, c, w_k, np.ones(128), EPS)
+    q = rng.standard_normal((G, 128))
+    w_q = rng.standard_normal((G, 128, 128)) / math.sqrt(128)
+    s, S = O.gate_scores(q, w_q, np.ones((G, 128)), gk, c, c, SCALE, EPS)
+    for g in range(G):
+        s1, _ = O.gate_scores(q[g:g + 1], w_q[g:g + 1], np.ones((1, 128)), gk, c, c, SCALE, EPS)
+        assert np.allclose(s1[0], s[g], atol=1e-14)
+    assert np.allclose(S, s.mean(axis=0), atol=1e-14)
+
+
+def test_gate_scores_invariant_to_positive_key_scale():
+    rng = np.random.default_rng(6)
+    c = 10
+    k = rng.standard_normal((64 * (c + 1), 128))
+    w_k = rng.standard_normal((384, 128)) / math.sqrt(384)
+    q = rng.standard_normal((2, 128))
+    w_q = rng.standard_normal((2, 128, 128)) / math.sqrt(128)
+    g1 = O.gate_keys_for_sequence(k, c, w_k, np.ones(128), EPS)
+    g2 = O.gate_keys_for_sequence(3.0 * k, c, w_k, np.ones(128), EPS)
+    s1, _ = O.gate_scores(q, w_q, np.ones((2, 128)), g1, c, c, SCALE, EPS)
+    s2, _ = O.gate_scores(q, w_q, np.ones((2, 128)), g2, c, c, SCALE, EPS)
+    assert np.allclose(s1, s2, rtol=1e-5, atol=1e-7)
+
+
+def test_gate_query_shift_invariance():
+    # shifting query and key positions together leaves the score unchanged
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal(128)
+    w_q = rng.standard_normal((128, 128)) / math.sqrt(128)
+    pooled = rng.standard_normal(384)
+    w_k = rng.standard_normal((384, 128)) / math.sqrt(384)
+    s1 = np.dot(O.gate_query(q, w_q, np.ones(128), 50), O.gate_key(pooled, w_k, np.ones(128), 20))
+    s2 = np.dot(O.gate_query(q, w_q, np.ones(128), 950), O.gate_key(pooled, w_k, np.ones(128), 920))
+    assert abs(s1 - s2) < 1e-9 * max(1.0, abs(s1))
+
+
+# ---------------------------------------------------------------- Top-K selection
+def _dominance_ok(S, sel_hist, n):
+    rest = [b for b in range(n) if b not in sel_hist]
+    return all((S[b] > S[r]) or (S[b] == S[r] and b < r) for b in sel_hist for r in rest)
+
+
+@pytest.mark.parametrize("n,topk", [(0, 3), (1, 3), (5, 3), (6, 6), (8, 3), (8, 1), (7, 7), (9, 4)])
+def test_select_brute_force_tiny(n, topk):
+    rng = np.random.default_rng(100 + 10 * n + topk)
+    for trial in range(20):
+        S = rng.integers(-3, 4, size=n).astype(np.float64) * 0.5  # many ties
+        if trial % 2:
+            S = S + rng.standard_normal(n) * 1e-3
+        sel = O.select_blocks(S, n, topk)
+        assert sel[-1] == n and sel == sorted(sel) and len(set(sel)) == len(sel)
+        want_k = min(topk, n)
+        cands = [list(c) for c in itertools.combinations(range(n), want_k) if _dominance_ok(S, c, n)]
+        assert len(cands) == 1
+        assert sel[:-1] == cands[0]
+
+
+@pytest.mark.parametrize("L", [1, 63, 64, 65, 128, 4096, 4097, 32768])
+@pytest.mark.parametrize("budget", [64, 1024, 2048, 4096])
+def test_selected_count(L, budget):
+    c = (L - 1) // 64
+    S = np.random.default_rng(L + budget).standard_normal(c)
+    sel = O.select_blocks(S, c, O.topk_for_budget(budget))
+    assert len(sel) == min(budget // 64, c + 1)
+
+
+def test_topk_for_budget_matches_training_setting():
+    # 31 historical + current = 2048/64 (release settings)
+    assert O.topk_for_budget(2048) == 31
+    assert O.topk_for_budget(1024) == 15 and O.topk_for_budget(4096) == 63
+
+
+# ---------------------------------------------------------------- attention reductions
+def _rand_group(rng, L, G=4):
+    k = rng.standard_normal((L, 128))
+    v = rng.standard_normal((L, 128))
+    q = rng.standard_normal((G, 128))
+    w_q = rng.standard_normal((G, 128, 128)) / math.sqrt(128)
+    w_k = rng.standard_normal((384, 128)) / math.sqrt(384)
+    return k, v, q, w_q, w_k
+
+
+@pytest.mark.parametrize("L", [1, 64, 65, 300, 1000])
+def test_budget_covering_context_is_dense_causal(L):
+    rng = np.random.default_rng(L)
+    k, v, q, w_q, w_k = _rand_group(rng, L)
+    c = (L - 1) // 64
+    gk = O.gate_keys_for_sequence(k, c, w_k, np.ones(128), EPS)
+    budget = 64 * (c + 1)
+    r = O.decode_one_group(q, k, v, L, gk, w_q, np.ones((4, 128)), budget)
+    assert r["sel"] == list(range(c + 1))
+    dense = O.dense_causal_decode(q, k, v, L)
+    assert np.max(np.abs(r["out"] - dense)) < 1e-12
+
+
+def test_equal_values_and_zero_query():
+    rng = np.random.default_rng(11)
+    L = 700
+    k, v, q, w_q, w_k = _rand_group(rng, L)
+    c = (L - 1) // 64
+    gk = O.gate_keys_for_sequence(k, c, w_k, np.ones(128), EPS)
+    vconst = np.tile(rng.standard_normal(128), (L, 1))
+    r = O.decode_one_group(q, k, vconst, L, gk, w_q, np.ones((4, 128)), 256)
+    assert np.allclose(r["out"], vconst[0][None, :], atol=1e-12)
+    # q = 0 for attention -> plain mean of the selected tokens' values
+    toks = O.selected_token_ids(r["sel"], L)
+    z = O.attention_over_tokens(np.zeros(128), k, v, toks, SCALE)
+    assert np.allclose(z, v[toks].mean(axis=0), atol=1e-12)
+
+
+def test_budget_64_attends_current_block_only():
+    rng = np.random.default_rng(12)
+    L = 1000
+    k, v, q, w_q, w_k = _rand_group(rng, L)
+    c = (L - 1) // 64
+    gk = O.gate_keys_for_sequence(k, c, w_k, np.ones(128), EPS)
+    r = O.decode_one_group(q, k, v, L, gk, w_q, np.ones((4, 128)), 64)
+    assert r["sel"] == [c]
+    lo = 64 * c
+    for g in range(4):
+        logits = (k[lo:L] @ q[g]) * SCALE
+        w = np.exp(logits - logits.max())
+        assert np.allclose(r["out"][g], (w @ v[lo:L]) / w.sum(), atol=1e-12)
+
+
+def test_closed_form_selection_ranks_by_relative_position():
+    # with the closed-form gate above, block b's score is f(c-b); Top-K must
+    # follow the ranking of f over the offsets
+    c = 20
+    n, k, w_k, w_q, q = _closed_form_inputs(c)
+    L = 64 * c + 1
+    v = np.zeros_like(k)
+    gk = O.gate_keys_for_sequence(k, n, w_k, np.ones(128), EPS)
+    r = O.decode_one_group(q, k[:L], v[:L], L, gk, w_q, np.ones((1, 128)), 64 * 6)
+    f = [(-3.0 * math.cos(c - b) + math.sin(c - b), b) for b in range(c)]
+    want = sorted(b for _, b in sorted(f, key=lambda t: (-t[0], t[1]))[:5])
+    assert r["sel"] == want + [c]
+
+
+# ---------------------------------------------------------------- prefill
+def test_prefill_full_budget_is_dense_causal():
+    rng = np.random.default_rng(13)
+    nb, G = 4, 2
+    T = 64 * nb
+    q = rng.standard_normal((G, T, 128))
+    k = rng.standard_normal((T, 128))
+    v = rng.standard_normal((T, 128))
+    w_q = rng.standard_normal((G, 128, 128)) / math.sqrt(128)
+    w_k = rng.standard_normal((384, 128)) / math.sqrt(384)
+    gk = O.gate_keys_for_sequence(k, nb, w_k, np.ones(128), EPS)
+    dense = [O.dense_causal_prefill(q[g], k, v) for g in range(G)]
+    for i in range(nb):
+        r = O.prefill_query_block(q[:, 64 * i:64 * (i + 1)], k, v, i, gk, w_q,
+                                  np.ones((G, 128)), topk=nb)
+        assert r["sel"] == list(range(i + 1))
+        for g in range(G):
+            assert np.max(np.abs(r["out"][g] - dense[g][64 * i:64 * (i + 1)])) < 1e-12
+
+
+def test_prefill_gate_query_is_block_mean():
+    rng = np.random.default_rng(14)
+    nb, G, i = 6, 2, 5
+    T = 64 * nb
+    q = rng.standard_normal((G, T, 128))
+    k = rng.standard_normal((T, 128))
+    v = rng.standard_normal((T, 128))
+    w_q = rng.standard_normal((G, 128, 128)) / math.sqrt(128)
+    w_k = rng.standard_normal((384, 128)) / math.sqrt(384)
+    gk = O.gate_keys_for_sequence(k, nb, w_k, np.ones(128), EPS)
+    r = O.prefill_query_block(q[:, 64 * i:64 * (i + 1)], k, v, i, gk, w_q, np.ones((G, 128)), topk=2)
+    qbar = q[:, 64 * i:64 * (i + 1)].mean(axis=1)
+    _, S = O.gate_scores(qbar, w_q, np.ones((G, 128)), gk, i, i, SCALE, EPS)
+    assert np.allclose(r["S"], S, atol=1e-14)
+    assert len(r["sel"]) == 3 and r["sel"][-1] == i
+    # token 0 of the query block sees the kept blocks plus itself only
+    toks = O.selected_token_ids(r["sel"][:-1], 64 * i) + [64 * i]
+    ref = O.attention_over_tokens(q[0, 64 * i], k, v, toks, SCALE)
+    assert np.allclose(r["out"][0, 0], ref, atol=1e-12)
+
+
+# ---------------------------------------------------------------- planted mistakes
+def test_pins_catch_planted_mistakes(monkeypatch):
+    """Plant plausible mistakes in the oracle (CPU) and show a pin fails."""
+    good_rope = O.rope_rotate_half
+
+    def rope_wrong_sign(x, pos, base=10000.0):
+        return good_rope(x, -pos, base)
+
+    monkeypatch.setattr(O, "rope_rotate_half", rope_wrong_sign)
+    with pytest.raises(AssertionError):
+        test_gate_scores_closed_form()
+    monkeypatch.setattr(O, "rope_rotate_half", good_rope)
+
+    good_pool = O.pool_block
+
+    def pool_swapped(kb):
+        p = good_pool(kb)
+        return np.concatenate([p[128:256], p[:128], p[256:]])
+
+    monkeypatch.setattr(O, "pool_block", pool_swapped)
+    with pytest.raises(AssertionError):
+        test_gate_scores_closed_form()
+    monkeypatch.setattr(O, "pool_block", good_pool)
+
+    good_select = O.select_blocks
+
+    def select_high_index_ties(S, n, topk):
+        order = sorted(range(n), key=lambda b: (-float(S[b]), -b))
+        return sorted(order[:min(topk, n)]) + [n]
+
+    monkeypatch.setattr(O, "select_blocks", select_high_index_ties)
+    with pytest.raises(AssertionError):
+        test_select_brute_force_tiny(8, 3)
+    monkeypatch.setattr(O, "select_blocks", good_select)
+
+    good_attn = O.attention_over_tokens
+
+    def attn_no_scale(q, k, v, toks, scale):
+        return good_attn(q, k, v, toks, 1.0)
+
+    monkeypatch.setattr(O, "attention_over_tokens", attn_no_scale)
+    with pytest.raises(AssertionError):
+        test_budget_covering_context_is_dense_causal(300)
+    monkeypatch.setattr(O, "attention_over_tokens", good_attn)
