@@ -1,0 +1,469 @@
+"""Benchmark of the SAS decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: Qwen3-4B-shaped decode layer, batch 8, 32 query / 8 KV heads,
+head_dim 128, context 32,768 for every sequence, token budget 2,048
+(31 historical blocks + the current block), bf16 K/V with per-block mean
+offsets (seeded, synthetic).  A step is one pass of the whole decode path
+over the batch: pooling + gate key of the just-completed current block
+(sas_pool_keys) and the fused gate / Top-K / block-sparse attention launch
+(sas_decode_step).  Steps rotate over R layers with their own caches, so the
+selected working set (R x ~85 MB) is far larger than the 126 MB L2.
+
+Metric: decode steps/s per layer (whole job: summed over ranks), achieved
+HBM GB/s of the dominant kernel against the measured B200 copy bandwidth.
+
+Multi-GPU: one process per GPU (torchrun); every rank decodes its own
+independent batch (weak scaling, no collective on the data path); the only
+collectives are the barrier and the max-reduce of the timings.
+
+--impl reference times the CPU oracle (the plain fp64 restatement of the
+method) on a bounded sample of the same workload: each step is one (sequence,
+KV head) pair of the batch, reported as steps/s of the whole batch.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode steps/s per layer at 32k ctx; achieved HBM GB/s vs B200 peak"
+UNIT = "steps/s"
+WORKLOAD = "qwen3_4b_decode_b8_ctx32768_budget2048"
+BATCH, HQ, HKV, CTX, BUDGET = 8, 32, 8, 32768, 2048
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=400)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- measured peaks, clocks
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.reader.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                sm.append(float(f[2]))
+                smax = float(f[3])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[6:10]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- algorithmic bytes
+def decode_bytes(seq_lens, hq, hkv, budget, kv_elem=2):
+    """Bytes the fused decode step must move: selected K/V tokens, the fp32 gate
+    key of every historical block, q and out of every head, W_q once."""
+    G = hq // hkv
+    tot = 0
+    for L in seq_lens:
+        c = (L - 1) // 64
+        m = min(budget // 64 - 1, c)
+        cur_tokens = L - 64 * c
+        per_pair = (m * 64 + cur_tokens) * 128 * kv_elem * 2 + c * 128 * 4 + 2 * G * 128 * 2
+        tot += hkv * per_pair
+    return tot + hq * 128 * 128 * 2
+
+
+def pool_bytes(batch, hkv):
+    """Bytes of pooling the current block: its K tile, W_k once, the gate key."""
+    return batch * hkv * (64 * 128 * 2 + 128 * 4) + hkv * 384 * 128 * 2
+
+
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_block_sparse_token_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the fused decode kernel from the committed ncu
+    summary, if it was taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "decode_step_qwen3_4b_32k.md")
+    if not os.path.exists(p):
+        return None
+    want = source_digest()
+    digest, traffic = None, None
+    for line in open(p):
+        if line.startswith("source_digest:"):
+            digest = line.split(":", 1)[1].strip()
+        if line.startswith("dram_bytes_per_launch:"):
+            traffic = float(line.split(":", 1)[1].strip())
+    return traffic if digest == want else None
+
+
+# ---------------------------------------------------------------- our arm
+def build_layers(R, rank, device):
+    import torch
+    from gated_block_sparse_token_b200 import sas
+    from gated_block_sparse_token_b200.workloads import make_decode_inputs, qwen3_4b_32k
+
+    cfg = sas.Config(HQ, HKV, token_budget=BUDGET)
+    layers = []
+    for li in range(R):
+        spec = qwen3_4b_32k(batch=BATCH, seq_len=CTX, seed=1000 * (rank + 1) + li)
+        inp = make_decode_inputs(spec, device)
+        kv = sas.KvCache(inp["k"], inp["v"], inp["seq_lens"])
+        mg = spec.cap // 64
+        gk = torch.zeros(BATCH, HKV, mg, 128, dtype=torch.float32, device=device)
+        ws = sas.make_workspace(cfg, device)
+        sas.pool_keys(cfg, kv, inp["w_k"], inp["gamma_k"], gk, ws)  # prefill-time keys (untimed)
+        cur = torch.full((BATCH,), (CTX - 1) // 64, dtype=torch.int32, device=device)
+        out = torch.empty(BATCH, HQ, 128, dtype=torch.bfloat16, device=device)
+        layers.append(dict(inp=inp, kv=kv, gk=gk, ws=ws, cur=cur, out=out))
+    return cfg, layers
+
+
+def step(cfg, L, stream=None, q=None):
+    """One decode step of one layer: pool the just-completed current block, then
+    the fused gate / Top-K / sparse-attention launch."""
+    from gated_block_sparse_token_b200 import sas
+    inp = L["inp"]
+    sas.pool_keys(cfg, L["kv"], inp["w_k"], inp["gamma_k"], L["gk"], L["ws"], blk_begin=L["cur"],
+                  num_blocks=1, stream=stream)
+    sas.decode_step(cfg, inp["q"] if q is None else q, L["kv"], inp["w_q"], inp["gamma_q"], L["gk"],
+                    L["out"], L["ws"], stream=stream)
+
+
+def decode_only(cfg, L, stream=None):
+    from gated_block_sparse_token_b200 import sas
+    inp = L["inp"]
+    sas.decode_step(cfg, inp["q"], L["kv"], inp["w_q"], inp["gamma_q"], L["gk"], L["out"], L["ws"],
+                    stream=stream)
+
+
+def capture(fn, n, layers, stream, offset=0):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            fn(layers[(offset + i) % len(layers)], stream)
+    return g
+
+
+def run_graphs(graphs_plan):
+    for g, reps in graphs_plan:
+        for _ in range(reps):
+            g.replay()
+
+
+def plan(fn, K, layers, stream, chunk=512):
+    """Graphs that replay exactly K steps (rotating over the layers)."""
+    R = len(layers)
+    chunk = max(R, (min(chunk, K) // R) * R) if K >= R else K
+    out = []
+    if K // chunk:
+        out.append((capture(fn, chunk, layers, stream), K // chunk))
+    rem = K - (K // chunk) * chunk
+    if rem:
+        out.append((capture(fn, rem, layers, stream), 1))
+    return out
+
+
+def timed(graphs, world, stream):
+    import torch
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run_graphs(graphs)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+
+
+def cpu_baseline(seconds):
+    """The oracle as it stands, single-threaded, on a bounded sample of the
+    workload: decode steps of individual (sequence, KV head) pairs."""
+    r = reference_sample(seconds_budget=seconds)
+    return {"value": r["value"], "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": r["sample"]}
+
+
+def run_ours(args):
+    import torch
+    from gated_block_sparse_token_b200 import sas
+
+    rank, world, local = dist_setup(args.gpus)
+    device = torch.device("cuda", local)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.cpu_seconds)   # before any pool could fork after CUDA use
+    cfg, layers = build_layers(args.layers, rank, device)
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for L in layers:       # first calls (one-time set-up) outside capture
+            step(cfg, L, stream)
+    torch.cuda.synchronize()
+
+    fn = lambda L, st: step(cfg, L, st)  # noqa: E731
+    warm = plan(fn, args.warmup, layers, stream)
+    main = plan(fn, args.steps, layers, stream)
+    run_graphs(warm)
+    torch.cuda.synchronize()
+    clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.3)
+    t = timed(main, world, stream)
+    clocks = clk.stop()
+    for L in layers:
+        if sas.get_device_status(L["ws"], stream) != sas.SAS_OK:
+            raise RuntimeError("device status not OK after the timed run")
+
+    # dominant kernel alone (same rotation), for the roofline
+    dk = plan(lambda L, st: decode_only(cfg, L, st), args.steps, layers, stream)
+    run_graphs(plan(lambda L, st: decode_only(cfg, L, st), min(args.warmup, 200), layers, stream))
+    t_dec = timed(dk, world, stream)
+    del dk
+
+    # end to end through the public API: pinned host q in, host out back, every step
+    q_host = [L["inp"]["q"].cpu().pin_memory() for L in layers]
+    out_host = torch.empty(BATCH, HQ, 128, dtype=torch.bfloat16).pin_memory()
+    q_dev = torch.empty_like(layers[0]["inp"]["q"])
+    ke = args.e2e_steps
+    with torch.cuda.stream(stream):
+        for i in range(min(50, ke)):
+            L = layers[i % len(layers)]
+            q_dev.copy_(q_host[i % len(layers)], non_blocking=True)
+            step(cfg, L, stream, q=q_dev)
+            out_host.copy_(L["out"], non_blocking=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(ke):
+            L = layers[i % len(layers)]
+            q_dev.copy_(q_host[i % len(layers)], non_blocking=True)
+            step(cfg, L, stream, q=q_dev)
+            out_host.copy_(L["out"], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+
+    if rank != 0:
+        return
+    peak, peak_kind = measured_peaks()
+    dbytes = decode_bytes([CTX] * BATCH, HQ, HKV, BUDGET)
+    pbytes = pool_bytes(BATCH, HKV)
+    dec_s = t_dec / args.steps
+    achieved = dbytes / dec_s / 1e9
+    step_s = t / args.steps
+    value = world * args.steps / t
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded normal K/V with per-block offsets, random-init gate weights)",
+        "config": {"workload": WORKLOAD, "batch_per_gpu": BATCH, "q_heads": HQ, "kv_heads": HKV,
+                   "head_dim": 128, "context": CTX, "token_budget": BUDGET,
+                   "layers_rotated": args.layers,
+                   "l2": f"inputs larger than L2: {args.layers} layer caches rotated, "
+                         f"{args.layers * (dbytes + pbytes) / 1e6:.0f} MB touched per rotation",
+                   "parallelism": f"replicas x{world} (independent batches)"},
+        "hbm_gbs_step": round((dbytes + pbytes) / step_s / 1e9, 1),
+        "roofline": {"kernel": "decode_cluster_kernel (sas_decode_step)", "bound": "hbm",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+                     "bytes_per_launch": dbytes, "avg_launch_us": round(dec_s * 1e6, 3),
+                     "traffic": profiled_traffic()},
+        "e2e": {"value": round(world * ke / t_e2e, 2), "unit": UNIT,
+                "h2d_bytes_per_step": BATCH * HQ * 128 * 2, "d2h_bytes_per_step": BATCH * HQ * 128 * 2},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- reference arm (CPU oracle)
+def reference_sample(seconds_budget=None, steps=None):
+    """Time oracle decode steps of single (sequence, KV head) pairs of the
+    workload (gate keys of the historical blocks precomputed by the oracle,
+    untimed; the step pools the current block, gates, selects and attends)."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_limits
+
+    from gated_block_sparse_token_b200.workloads import qwen3_4b_32k, make_decode_inputs, logical_kv
+    from oracle import sas_oracle as O
+
+    spec = qwen3_4b_32k(batch=1, seq_len=CTX, seed=1)
+    # one sequence of the same shape, generated on the host
+    inp = make_decode_inputs(spec, "cpu")
+    G = HQ // HKV
+    q = inp["q"].double().numpy()
+    wq = inp["w_q"].double().numpy()
+    wk = inp["w_k"].double().numpy()
+    ones = np.ones(128)
+    c = (CTX - 1) // 64
+    pairs = []
+    for h in range(HKV):
+        ks, vs = logical_kv(inp, 0, h, CTX)
+        keys = O.gate_keys_for_sequence(ks, c, wk[h], ones)
+        pairs.append((h, ks, vs, keys))
+    done = 0
+    t0 = time.perf_counter()
+    with threadpool_limits(limits=1):
+        while True:
+            h, ks, vs, keys = pairs[done % HKV]
+            O.gate_key(O.pool_block(ks[64 * c:64 * c + 64]), wk[h], ones, c)
+            O.decode_one_group(q[0, h * G:(h + 1) * G], ks, vs, CTX, keys, wq[h * G:(h + 1) * G],
+                               np.tile(ones, (G, 1)), BUDGET)
+            done += 1
+            el = time.perf_counter() - t0
+            if (steps is not None and done >= steps) or (seconds_budget is not None and el >= seconds_budget):
+                break
+    per_pair = el / done
+    return {"value": 1.0 / (per_pair * BATCH * HKV), "elapsed": el, "pairs": done,
+            "sample": f"{done} (sequence, KV head) decode steps of the workload in {el:.1f} s, "
+                      f"1 thread; a full step is {BATCH * HKV} pairs"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    warm = reference_sample(steps=max(1, min(args.warmup, 3)))
+    del warm
+    r = reference_sample(steps=args.steps)
+    value = r["value"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": WORKLOAD, "batch_per_gpu": BATCH, "q_heads": HQ, "kv_heads": HKV,
+                   "head_dim": 128, "context": CTX, "token_budget": BUDGET},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": r["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    run_ours(args)
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,373 @@
+// libsas C ABI: host-side validation, TMA tensor-map encoding and kernel
+// dispatch.  Every entry point validates on the host, enqueues on the given
+// stream and returns; nothing here allocates or synchronises except
+// sas_get_device_status.
+#include <math.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "sas.h"
+#include "sas_internal.h"
+
+namespace sas {
+cudaError_t prepare_decode_kernels();
+}
+
+namespace {
+
+using sas::kDim;
+
+constexpr int32_t kAbiVersion = 1;
+constexpr size_t kStatusBytes = 256;  // status word + padding
+constexpr int kMaxBudget = 16384;
+constexpr int kMaxGateBlocks = 16384;
+constexpr int kClusterSize = 8;
+constexpr int kStages = 2;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::once_flag g_once;
+cudaError_t g_prep_err = cudaSuccess;
+EncodeTiledFn g_encode = nullptr;
+
+cudaError_t prepare() {
+  std::call_once(g_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000,
+                                                     cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || fn == nullptr) {
+      g_prep_err = (e != cudaSuccess) ? e : cudaErrorSymbolNotFound;
+      return;
+    }
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    g_prep_err = sas::prepare_decode_kernels();
+  });
+  return g_prep_err;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool finite_pos(float x) { return isfinite(x) && x > 0.f; }
+
+sas_status check_config(const sas_config* c) {
+  if (c == nullptr) return SAS_ERR_INVALID_ARG;
+  if (c->block_size != 64 || c->gate_hidden != 128) return SAS_ERR_INVALID_ARG;
+  if (c->head_dim != 128) return SAS_ERR_UNSUPPORTED;
+  if (c->num_q_heads < 1 || c->num_kv_heads < 1) return SAS_ERR_INVALID_ARG;
+  if (c->num_q_heads % c->num_kv_heads != 0) return SAS_ERR_INVALID_ARG;
+  if (c->num_q_heads / c->num_kv_heads > sas::kMaxGroup) return SAS_ERR_UNSUPPORTED;
+  if (c->token_budget < 64 || c->token_budget % 64 != 0) return SAS_ERR_INVALID_ARG;
+  if (c->token_budget > kMaxBudget) return SAS_ERR_UNSUPPORTED;
+  if (!finite_pos(c->rope_base) || !finite_pos(c->attn_scale) || !finite_pos(c->gate_scale))
+    return SAS_ERR_INVALID_ARG;
+  if (!isfinite(c->norm_eps) || c->norm_eps < 0.f) return SAS_ERR_INVALID_ARG;
+  if (c->kv_dtype != SAS_DTYPE_BF16 && c->kv_dtype != SAS_DTYPE_F32) return SAS_ERR_INVALID_ARG;
+  if (c->out_dtype != SAS_DTYPE_BF16 && c->out_dtype != SAS_DTYPE_F32) return SAS_ERR_INVALID_ARG;
+  return SAS_OK;
+}
+
+sas_status check_ws(const sas_config* cfg, void* ws, size_t ws_bytes) {
+  if (ws == nullptr || !aligned(ws, 16)) return SAS_ERR_WORKSPACE;
+  if (ws_bytes < sas_workspace_bytes(cfg, 0, 0)) return SAS_ERR_WORKSPACE;
+  return SAS_OK;
+}
+
+sas_status check_kv(const sas_config* cfg, const sas_kv* kv) {
+  if (kv == nullptr) return SAS_ERR_INVALID_ARG;
+  if (kv->batch < 0) return SAS_ERR_INVALID_ARG;
+  if (kv->batch == 0) return SAS_OK;
+  if (kv->k == nullptr || kv->v == nullptr || kv->seq_lens == nullptr) return SAS_ERR_INVALID_ARG;
+  if (!aligned(kv->k, 16) || !aligned(kv->v, 16) || !aligned(kv->seq_lens, 4))
+    return SAS_ERR_INVALID_ARG;
+  long long rows;
+  if (kv->block_table != nullptr) {
+    if (!aligned(kv->block_table, 4) || kv->num_pages < 1 || kv->max_blocks_per_seq < 1)
+      return SAS_ERR_INVALID_ARG;
+    rows = static_cast<long long>(kv->num_pages) * cfg->num_kv_heads * 64;
+  } else {
+    if (kv->capacity < 64 || kv->capacity % 64 != 0) return SAS_ERR_INVALID_ARG;
+    rows = static_cast<long long>(kv->batch) * cfg->num_kv_heads * kv->capacity;
+  }
+  if (rows > 0x7fffffffLL) return SAS_ERR_UNSUPPORTED;  // TMA row coordinate is int32
+  return SAS_OK;
+}
+
+sas::KvView make_view(const sas_config* cfg, const sas_kv* kv) {
+  sas::KvView v{};
+  v.k = kv->k;
+  v.v = kv->v;
+  v.block_table = kv->block_table;
+  v.seq_lens = kv->seq_lens;
+  v.hkv = cfg->num_kv_heads;
+  v.capacity = kv->capacity;
+  v.num_pages = kv->num_pages;
+  v.max_blocks_per_seq = kv->max_blocks_per_seq;
+  return v;
+}
+
+// 2-D view [rows][128] of a bf16 K or V cache, 64x64 boxes, 128-byte swizzle.
+bool encode_kv_map(CUtensorMap* m, const void* ptr, long long rows) {
+  memset(m, 0, sizeof(*m));
+  if (g_encode == nullptr) return false;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(kDim * 2)};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim,
+                              gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+long long kv_rows(const sas_config* cfg, const sas_kv* kv) {
+  return kv->block_table != nullptr
+             ? static_cast<long long>(kv->num_pages) * cfg->num_kv_heads * 64
+             : static_cast<long long>(kv->batch) * cfg->num_kv_heads * kv->capacity;
+}
+
+void fill_common(sas::DecodeParams& p, const sas_config* cfg, int mg) {
+  p.hq = cfg->num_q_heads;
+  p.hkv = cfg->num_kv_heads;
+  p.G = cfg->num_q_heads / cfg->num_kv_heads;
+  p.max_sel = cfg->token_budget / 64;
+  p.topk = p.max_sel - 1;
+  p.mg = mg;
+  p.rope_base = cfg->rope_base;
+  p.eps = cfg->norm_eps;
+  p.attn_scale_log2 = cfg->attn_scale * 1.4426950408889634f;
+  p.gate_scale = cfg->gate_scale;
+  p.sm = sas::plan_decode_smem(p.G, mg, kClusterSize, kStages, p.max_sel,
+                               cfg->kv_dtype == SAS_DTYPE_F32);
+}
+
+sas_status launch_result(cudaError_t e) {
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SAS_ERR_CUDA;
+  }
+  return SAS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t sas_abi_version(void) { return kAbiVersion; }
+
+const char* sas_status_string(sas_status s) {
+  switch (s) {
+    case SAS_OK: return "ok";
+    case SAS_ERR_INVALID_ARG: return "invalid argument";
+    case SAS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SAS_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case SAS_ERR_CUDA: return "CUDA runtime error";
+    case SAS_ERR_DEVICE_BOUNDS: return "device-detected out-of-range length, page or block index";
+    case SAS_ERR_TIMEOUT: return "bounded device wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t sas_workspace_bytes(const sas_config* cfg, int32_t batch, int32_t max_seq_len) {
+  (void)cfg;
+  (void)batch;
+  (void)max_seq_len;
+  return kStatusBytes;
+}
+
+sas_status sas_reset_device_status(void* ws, sas_stream_t stream) {
+  if (ws == nullptr || !aligned(ws, 16)) return SAS_ERR_WORKSPACE;
+  return launch_result(cudaMemsetAsync(ws, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_get_device_status(const void* ws, sas_stream_t stream, sas_status* out) {
+  if (ws == nullptr || out == nullptr || !aligned(ws, 16)) return SAS_ERR_INVALID_ARG;
+  uint32_t word = 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return SAS_ERR_CUDA;
+  }
+  if (word & sas::kStatusBounds)
+    *out = SAS_ERR_DEVICE_BOUNDS;
+  else if (word & sas::kStatusTimeout)
+    *out = SAS_ERR_TIMEOUT;
+  else
+    *out = SAS_OK;
+  return SAS_OK;
+}
+
+sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv, const int32_t* blk_begin,
+                         int32_t num_blocks, const void* w_k, const float* gamma_k,
+                         float* gate_keys, int32_t max_gate_blocks, float* pooled_raw, void* ws,
+                         size_t ws_bytes, sas_stream_t stream) {
+  sas_status st = check_config(cfg);
+  if (st != SAS_OK) return st;
+  if ((st = check_kv(cfg, kv)) != SAS_OK) return st;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != SAS_OK) return st;
+  if (num_blocks < 0 || max_gate_blocks < 1 || max_gate_blocks > kMaxGateBlocks)
+    return SAS_ERR_INVALID_ARG;
+  if (kv->batch == 0 || num_blocks == 0) return SAS_OK;
+  if (w_k == nullptr || gamma_k == nullptr || gate_keys == nullptr) return SAS_ERR_INVALID_ARG;
+  if (!aligned(w_k, 16) || !aligned(gamma_k, 4) || !aligned(gate_keys, 16) ||
+      (pooled_raw != nullptr && !aligned(pooled_raw, 4)) ||
+      (blk_begin != nullptr && !aligned(blk_begin, 4)))
+    return SAS_ERR_INVALID_ARG;
+  if (kv->batch > 65535) return SAS_ERR_UNSUPPORTED;
+  if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
+  sas::PoolParams p{};
+  p.hkv = cfg->num_kv_heads;
+  p.mg = max_gate_blocks;
+  p.num_blocks = num_blocks;
+  p.rope_base = cfg->rope_base;
+  p.eps = cfg->norm_eps;
+  p.kv = make_view(cfg, kv);
+  p.blk_begin = blk_begin;
+  p.w_k = static_cast<const __nv_bfloat16*>(w_k);
+  p.gamma_k = gamma_k;
+  p.gate_keys = gate_keys;
+  p.pooled_raw = pooled_raw;
+  p.status = static_cast<uint32_t*>(ws);
+  return launch_result(sas::launch_pool(cfg->kv_dtype == SAS_DTYPE_F32, p, kv->batch,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_gate_scores(const sas_config* cfg, const void* q, const int32_t* seq_lens,
+                           int32_t batch, const void* w_q, const float* gamma_q,
+                           const float* gate_keys, int32_t max_gate_blocks, float* head_scores,
+                           float* group_scores, void* ws, size_t ws_bytes, sas_stream_t stream) {
+  sas_status st = check_config(cfg);
+  if (st != SAS_OK) return st;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != SAS_OK) return st;
+  if (batch < 0 || max_gate_blocks < 1 || max_gate_blocks > kMaxGateBlocks) return SAS_ERR_INVALID_ARG;
+  if (batch == 0) return SAS_OK;
+  if (q == nullptr || seq_lens == nullptr || w_q == nullptr || gamma_q == nullptr ||
+      gate_keys == nullptr || group_scores == nullptr)
+    return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 4) || !aligned(seq_lens, 4) || !aligned(w_q, 16) || !aligned(gamma_q, 4) ||
+      !aligned(gate_keys, 16) || !aligned(group_scores, 4) ||
+      (head_scores != nullptr && !aligned(head_scores, 4)))
+    return SAS_ERR_INVALID_ARG;
+  if (static_cast<long long>(batch) * cfg->num_kv_heads > 65535) return SAS_ERR_UNSUPPORTED;
+  if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
+  sas::DecodeParams p{};
+  fill_common(p, cfg, max_gate_blocks);
+  if (p.sm.total > 227 * 1024) return SAS_ERR_UNSUPPORTED;
+  p.q = q;
+  p.w_q = static_cast<const __nv_bfloat16*>(w_q);
+  p.gamma_q = gamma_q;
+  p.gate_keys = gate_keys;
+  p.kv.seq_lens = seq_lens;
+  p.kv.hkv = cfg->num_kv_heads;
+  p.head_scores = head_scores;
+  p.group_scores = group_scores;
+  p.status = static_cast<uint32_t*>(ws);
+  CUtensorMap dummy;
+  memset(&dummy, 0, sizeof(dummy));
+  return launch_result(sas::launch_decode(sas::kModeGate, cfg->kv_dtype == SAS_DTYPE_F32, false,
+                                          kClusterSize, kStages, p, dummy, dummy, batch,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_topk_blocks(const sas_config* cfg, const float* group_scores,
+                           const int32_t* seq_lens, int32_t batch, int32_t max_gate_blocks,
+                           int32_t* sel_idx, int32_t* sel_count, void* ws, size_t ws_bytes,
+                           sas_stream_t stream) {
+  sas_status st = check_config(cfg);
+  if (st != SAS_OK) return st;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != SAS_OK) return st;
+  if (batch < 0 || max_gate_blocks < 1 || max_gate_blocks > kMaxGateBlocks) return SAS_ERR_INVALID_ARG;
+  if (batch == 0) return SAS_OK;
+  if (group_scores == nullptr || seq_lens == nullptr || sel_idx == nullptr || sel_count == nullptr)
+    return SAS_ERR_INVALID_ARG;
+  if (!aligned(group_scores, 4) || !aligned(seq_lens, 4) || !aligned(sel_idx, 4) ||
+      !aligned(sel_count, 4))
+    return SAS_ERR_INVALID_ARG;
+  if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
+  sas::TopkParams p{};
+  p.hkv = cfg->num_kv_heads;
+  p.max_sel = cfg->token_budget / 64;
+  p.topk = p.max_sel - 1;
+  p.mg = max_gate_blocks;
+  p.group_scores = group_scores;
+  p.seq_lens = seq_lens;
+  p.sel_idx = sel_idx;
+  p.sel_count = sel_count;
+  p.status = static_cast<uint32_t*>(ws);
+  return launch_result(sas::launch_topk(p, batch, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static sas_status attention_call(int mode, const sas_config* cfg, const void* q, const sas_kv* kv,
+                                 const void* w_q, const float* gamma_q, const float* gate_keys,
+                                 int32_t max_gate_blocks, void* out, int32_t* sel_idx,
+                                 int32_t* sel_count, float* group_scores, void* ws,
+                                 size_t ws_bytes, sas_stream_t stream) {
+  sas_status st = check_config(cfg);
+  if (st != SAS_OK) return st;
+  if ((st = check_kv(cfg, kv)) != SAS_OK) return st;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != SAS_OK) return st;
+  if (kv->batch == 0) return SAS_OK;
+  if (q == nullptr || out == nullptr || !aligned(q, 4) || !aligned(out, 4)) return SAS_ERR_INVALID_ARG;
+  if (mode == sas::kModeFused) {
+    if (max_gate_blocks < 1 || max_gate_blocks > kMaxGateBlocks) return SAS_ERR_INVALID_ARG;
+    if (w_q == nullptr || gamma_q == nullptr || gate_keys == nullptr) return SAS_ERR_INVALID_ARG;
+    if (!aligned(w_q, 16) || !aligned(gamma_q, 4) || !aligned(gate_keys, 16)) return SAS_ERR_INVALID_ARG;
+    if ((sel_idx != nullptr && !aligned(sel_idx, 4)) || (sel_count != nullptr && !aligned(sel_count, 4)) ||
+        (group_scores != nullptr && !aligned(group_scores, 4)))
+      return SAS_ERR_INVALID_ARG;
+  } else {
+    if (sel_idx == nullptr || sel_count == nullptr || !aligned(sel_idx, 4) || !aligned(sel_count, 4))
+      return SAS_ERR_INVALID_ARG;
+    max_gate_blocks = 1;
+  }
+  if (static_cast<long long>(kv->batch) * cfg->num_kv_heads > 65535) return SAS_ERR_UNSUPPORTED;
+  if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
+  sas::DecodeParams p{};
+  fill_common(p, cfg, max_gate_blocks);
+  if (p.sm.total > 227 * 1024) return SAS_ERR_UNSUPPORTED;
+  p.q = q;
+  p.w_q = static_cast<const __nv_bfloat16*>(w_q);
+  p.gamma_q = gamma_q;
+  p.gate_keys = gate_keys;
+  p.kv = make_view(cfg, kv);
+  p.group_scores = group_scores;
+  p.sel_idx = sel_idx;
+  p.sel_count = sel_count;
+  p.out = out;
+  p.status = static_cast<uint32_t*>(ws);
+  const bool f32_kv = cfg->kv_dtype == SAS_DTYPE_F32;
+  CUtensorMap tmk, tmv;
+  memset(&tmk, 0, sizeof(tmk));
+  memset(&tmv, 0, sizeof(tmv));
+  if (!f32_kv) {
+    const long long rows = kv_rows(cfg, kv);
+    if (!encode_kv_map(&tmk, kv->k, rows) || !encode_kv_map(&tmv, kv->v, rows)) return SAS_ERR_CUDA;
+  }
+  return launch_result(sas::launch_decode(mode, f32_kv, cfg->out_dtype == SAS_DTYPE_F32,
+                                          kClusterSize, kStages, p, tmk, tmv, kv->batch,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const sas_kv* kv,
+                             const int32_t* sel_idx, const int32_t* sel_count, void* out,
+                             void* ws, size_t ws_bytes, sas_stream_t stream) {
+  return attention_call(sas::kModeAttend, cfg, q, kv, nullptr, nullptr, nullptr, 0, out,
+                        const_cast<int32_t*>(sel_idx), const_cast<int32_t*>(sel_count), nullptr,
+                        ws, ws_bytes, stream);
+}
+
+sas_status sas_decode_step(const sas_config* cfg, const void* q, const sas_kv* kv, const void* w_q,
+                           const float* gamma_q, const float* gate_keys, int32_t max_gate_blocks,
+                           void* out, int32_t* sel_idx, int32_t* sel_count, float* group_scores,
+                           void* ws, size_t ws_bytes, sas_stream_t stream) {
+  return attention_call(sas::kModeFused, cfg, q, kv, w_q, gamma_q, gate_keys, max_gate_blocks, out,
+                        sel_idx, sel_count, group_scores, ws, ws_bytes, stream);
+}
+
+}  // extern "C"

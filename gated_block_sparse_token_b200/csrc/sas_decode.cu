@@ -1,0 +1,867 @@
+// SAS decode kernels: gate scores, Top-K block selection and block-sparse
+// flash-decoding attention, as one thread-block cluster per (sequence, KV
+// head).
+//
+// Method (release pages: "Tencent released Simple-Attention-Sparsification
+// ..." aigc.news 2026-09-14, release paragraph; "Simple-Attention-
+// Sparsification Text Generation Model: 12GB+ VRAM", "Specifications and
+// Configuration Table"): a 128-wide gate scores every historical 64-token
+// block from the Qproj-projected query and the projected, Q/K-normalised,
+// RoPE'd max+min+average pooled keys; the top blocks under the token budget
+// plus the current block are attended.
+//
+// Work split of one cluster of CS CTAs (128 threads each) for (s, h):
+//   phase 0  each CTA computes 128/CS columns of v_g = q_g @ W_q[g] for the G
+//            query heads of the group and stores them into every CTA of the
+//            cluster (distributed shared memory); RMSNorm + RoPE -> q~_g.
+//   phase 1  each CTA streams 1/CS of the gate keys k~_b (TMA bulk copies
+//            into a ring of 16 KiB stage slots) and scores its blocks.
+//   phase 2  every CTA gathers all group scores through DSMEM and runs the
+//            same radix select (exact, ties -> lower index), so all CTAs
+//            hold the same ascending block list without another barrier.
+//   phase 3  CTA r attends to list entries j = r (mod CS): K and V tiles come
+//            in by 2-D TMA (128-byte swizzle) and each warp runs flash-
+//            decoding over 16 tokens of every tile with bf16 mma.sync
+//            (GQA group as the M=16 rows, fp32 accumulate, online softmax).
+//   phase 4  the 4*CS per-warp partials (m, l, o) are merged through DSMEM;
+//            CTA r writes 128/CS output columns.
+// The CTA that owns the current block (always selected) prefetches its
+// tiles before the selection finishes.
+#include <cooperative_groups.h>
+
+#include <type_traits>
+
+#include "sas_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace sas {
+
+namespace {
+
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* raw) {
+  const uint32_t a = smem_u32(raw);
+  return raw + (((a + 1023u) & ~1023u) - a);
+}
+
+// Exclusive prefix sum of v over the kThreads threads (thread order).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* scan) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) scan[warp] = inc;
+  __syncthreads();
+  int off = 0;
+  for (int w = 0; w < warp; ++w) off += scan[w];
+  __syncthreads();
+  return off + inc - v;
+}
+
+// Top-K selection (pages: training Top-K 31 under the 2,048-token budget).
+// Keeps the min(topk, n) largest of sall[0..n) -- ties go to the lower index
+// -- lists them ascending in sel[], appends the current block `cur` and
+// returns the count.  Exact radix select on order-preserving 32-bit keys
+// (four 8-bit passes), then an index-ordered compaction.  Called by all
+// kThreads threads of the CTA; overwrites sall with the keys.
+__device__ int select_blocks(float* sall, int n, int topk, int cur, int* sel, uint32_t* hist,
+                             int* scan) {
+  const int tid = threadIdx.x;
+  if (n <= topk) {
+    for (int i = tid; i < n; i += kThreads) sel[i] = i;
+    if (tid == 0) sel[n] = cur;
+    __syncthreads();
+    return n + 1;
+  }
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sall);
+  for (int i = tid; i < n; i += kThreads) keys[i] = order_key(sall[i]);
+  for (int i = tid; i < 512; i += kThreads) hist[i] = 0u;
+  __syncthreads();
+  uint32_t prefix = 0u;
+  int remaining = topk;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    const uint32_t hmask = (pass == 0) ? 0u : (0xFFFFFFFFu << (shift + 8));
+    uint32_t* hcur = hist + (pass & 1) * 256;
+    uint32_t* hnext = hist + ((pass + 1) & 1) * 256;
+    for (int i = tid; i < n; i += kThreads) {
+      const uint32_t k = keys[i];
+      if ((k & hmask) == prefix) atomicAdd(&hcur[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // lane l owns bins 255-8l .. 248-8l, so lane order is descending key order
+      uint32_t cnt[8];
+      uint32_t tot = 0u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = hcur[255 - 8 * tid - j];
+        tot += cnt[j];
+      }
+      uint32_t inc = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (tid >= o) inc += y;
+      }
+      const uint32_t exc = inc - tot;
+      const uint32_t want = static_cast<uint32_t>(remaining);
+      if (exc < want && want <= inc) {
+        uint32_t run = exc;
+        bool done = false;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (!done) {
+            if (run + cnt[j] >= want) {
+              scan[8] = 255 - 8 * tid - j;
+              scan[9] = static_cast<int>(want - run);
+              done = true;
+            } else {
+              run += cnt[j];
+            }
+          }
+        }
+      }
+    }
+    for (int i = tid; i < 256; i += kThreads) hnext[i] = 0u;
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(scan[8]) << shift;
+    remaining = scan[9];
+  }
+  // prefix is now the exact key of the topk-th largest score; keep every key
+  // above it and the first `remaining` keys equal to it, in index order.
+  const uint32_t thr = prefix;
+  const int take_eq = remaining;
+  const int per = (n + kThreads - 1) / kThreads;
+  const int lo = min(n, tid * per);
+  const int hi = min(n, lo + per);
+  int ceq = 0;
+  for (int i = lo; i < hi; ++i) ceq += (keys[i] == thr) ? 1 : 0;
+  const int eq_before = block_exclusive_scan(ceq, scan);
+  int cnt = 0;
+  int eqs = eq_before;
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t k = keys[i];
+    if (k > thr) {
+      ++cnt;
+    } else if (k == thr) {
+      if (eqs < take_eq) ++cnt;
+      ++eqs;
+    }
+  }
+  int pos = block_exclusive_scan(cnt, scan);
+  eqs = eq_before;
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t k = keys[i];
+    bool take = false;
+    if (k > thr) {
+      take = true;
+    } else if (k == thr) {
+      take = eqs < take_eq;
+      ++eqs;
+    }
+    if (take) sel[pos++] = i;
+  }
+  if (tid == 0) sel[topk] = cur;
+  __syncthreads();
+  return topk + 1;
+}
+
+__device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc) {
+  acc = fmaf(a.x, b.x, acc);
+  acc = fmaf(a.y, b.y, acc);
+  acc = fmaf(a.z, b.z, acc);
+  acc = fmaf(a.w, b.w, acc);
+  return acc;
+}
+
+}  // namespace
+
+template <typename T, typename OutT, int CS, int NST, int MODE>
+__global__ void __launch_bounds__(kThreads, 4)
+    decode_cluster_kernel(const __grid_constant__ DecodeParams p,
+                          const __grid_constant__ CUtensorMap tmk,
+                          const __grid_constant__ CUtensorMap tmv) {
+  constexpr bool kF32 = std::is_same<T, float>::value;
+  constexpr int kDpc = kDim / CS;                // output / W_q columns per CTA
+  constexpr int kTilesPerBlock = kF32 ? 4 : 2;   // 16 KiB tiles per K+V block
+  static_assert(kDpc % 8 == 0, "cluster size must divide 128 into 16-byte slices");
+
+  cg::cluster_group cluster = cg::this_cluster();
+  cluster_arrive_relaxed();  // matched by cluster_wait() before the first DSMEM store
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int pair = blockIdx.y;
+  const int s = pair / p.hkv;
+  const int h = pair - s * p.hkv;
+  const int G = p.G;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align_smem_1024(smem_raw);
+  uint8_t* slots = base + p.sm.slots;
+  float* sslice = reinterpret_cast<float*>(base + p.sm.sslice);
+  __nv_bfloat16* wq_s = reinterpret_cast<__nv_bfloat16*>(base + p.sm.u_wq);
+  float* qs = reinterpret_cast<float*>(base + p.sm.u_qs);
+  float* sall = reinterpret_cast<float*>(base + p.sm.u_sall);
+  int* sel = reinterpret_cast<int*>(base + p.sm.u_sel);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base + p.sm.u_hist);
+  int* scan = reinterpret_cast<int*>(base + p.sm.u_scan);
+  float* qv = reinterpret_cast<float*>(base + p.sm.qv);
+  float* qbar = reinterpret_cast<float*>(base + p.sm.qbar);
+  float* qatt = reinterpret_cast<float*>(base + p.sm.qatt);
+  float* pm = reinterpret_cast<float*>(base + p.sm.pml);
+  float* pl = pm + kWarps * kMaxGroup;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + p.sm.bars);
+  float* po = reinterpret_cast<float*>(slots);  // [4][G][128], after the last tile
+
+  // ------------------------------------------------------------ validation
+  const int L = p.kv.seq_lens[s];
+  bool err = (L < 1);
+  const int c = err ? 0 : (L - 1) / kBlock;  // current block
+  if (MODE != kModeAttend && c > p.mg) err = true;
+  if (MODE == kModeFused && !err) {
+    for (int b = tid; b <= c; b += kThreads)
+      if (p.kv.block_row(s, h, b) < 0) err = true;
+  }
+  int m = 0;  // entries of the block list (current block last)
+  if (MODE == kModeAttend && !err) {
+    int mm = p.sel_count[pair];
+    if (mm < 1 || mm > p.max_sel) {
+      err = true;
+    } else {
+      const int32_t* si = p.sel_idx + static_cast<size_t>(pair) * p.max_sel;
+      for (int j = tid; j < mm; j += kThreads) {
+        const int b = si[j];
+        sel[j] = b;
+        if (b < 0 || b > c) err = true;
+        if (j == mm - 1 && b != c) err = true;
+        if (j > 0 && si[j - 1] >= b) err = true;
+        if (p.kv.block_row(s, h, b) < 0) err = true;
+      }
+      m = mm;
+    }
+  }
+  const bool bad = __syncthreads_or(err) != 0;
+  if (bad && rank == 0 && tid == 0) raise_status(p.status, kStatusBounds);
+  const int n = bad ? 0 : c;  // historical blocks
+  if (MODE == kModeFused) m = bad ? 0 : min(p.topk, n) + 1;
+  if (MODE == kModeAttend && bad) m = 0;
+
+  const int nb_per = (n + CS - 1) / CS;
+  const int b_lo = min(n, rank * nb_per);
+  const int b_hi = min(n, b_lo + nb_per);
+  const int nchunks = (MODE == kModeAttend) ? 0 : (b_hi - b_lo + kGkChunk - 1) / kGkChunk;
+  const int cnt_mine = (rank < m) ? (m - 1 - rank) / CS + 1 : 0;
+  const bool own_cur = (m > 0) && ((m - 1) % CS == rank);
+
+  // list entry e of this CTA -> block id (the current block first if owned)
+  auto entry_block = [&](int e) -> int {
+    int j;
+    if (own_cur)
+      j = (e == 0) ? (m - 1) : rank + (e - 1) * CS;
+    else
+      j = rank + e * CS;
+    return (j == m - 1) ? c : sel[j];
+  };
+
+  // ------------------------------------------------------------ tile ring
+  // Tile t lives in slot t % NST, phase (t / NST) & 1.  Tiles 0..nchunks-1
+  // are gate-key chunks, then kTilesPerBlock tiles per list entry.  Thread 0
+  // issues tile t once tile t - NST has been released by every thread.
+  int issued = 0;  // meaningful in thread 0 only
+  auto issue = [&](int t) {
+    const int slot = t % NST;
+    uint8_t* dst = slots + slot * kTileBytes;
+    if (t < nchunks) {
+      const int b0 = b_lo + t * kGkChunk;
+      const int cntb = min(kGkChunk, b_hi - b0);
+      const uint32_t bytes = static_cast<uint32_t>(cntb) * kDim * 4u;
+      mbar_arrive_expect_tx(&bars[slot], bytes);
+      bulk_g2s(dst, p.gate_keys + (static_cast<size_t>(pair) * p.mg + b0) * kDim, bytes,
+               &bars[slot]);
+      return;
+    }
+    const int k = t - nchunks;
+    const int e = k / kTilesPerBlock;
+    const int part = k - e * kTilesPerBlock;
+    const long long row0 = p.kv.block_row(s, h, entry_block(e));
+    mbar_arrive_expect_tx(&bars[slot], kTileBytes);
+    if constexpr (kF32) {
+      const float* src = static_cast<const float*>(part < 2 ? p.kv.k : p.kv.v) +
+                         (row0 + (part & 1) * 32) * kDim;
+      bulk_g2s(dst, src, kTileBytes, &bars[slot]);
+    } else {
+      const CUtensorMap* map = (part == 0) ? &tmk : &tmv;
+      tma_load_2d(dst, map, 0, static_cast<int>(row0), &bars[slot]);
+      tma_load_2d(dst + 8192, map, 64, static_cast<int>(row0), &bars[slot]);
+    }
+  };
+  auto pump = [&](int consumed, int known) {
+    if (tid != 0) return;
+    fence_proxy_async_smem();
+    while (issued < known && issued < consumed + NST) issue(issued++);
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < NST; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // before the selection only the gate-key chunks and the current block are known
+  int known = nchunks + ((MODE == kModeAttend) ? kTilesPerBlock * cnt_mine
+                                               : (own_cur ? kTilesPerBlock : 0));
+  pump(0, known);
+
+  // ------------------------------------------------------------ phase 0: gate query
+  if (MODE != kModeAttend) {
+    if (!bad) {
+      const T* qg = static_cast<const T*>(p.q) +
+                    (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim;
+      for (int i = tid; i < G * kDim; i += kThreads) qs[i] = to_float(qg[i]);
+      constexpr int kVec = kDpc / 8;
+      for (int it = tid; it < G * kDim * kVec; it += kThreads) {
+        const int g = it / (kDim * kVec);
+        const int rem = it - g * kDim * kVec;
+        const int i = rem / kVec;
+        const int ch = rem - i * kVec;
+        const uint4 w = *reinterpret_cast<const uint4*>(
+            p.w_q + (static_cast<size_t>(h * G + g) * kDim + i) * kDim + rank * kDpc + ch * 8);
+        *reinterpret_cast<uint4*>(wq_s + (static_cast<size_t>(g) * kDim + i) * kDpc + ch * 8) = w;
+      }
+    }
+    __syncthreads();
+    cluster_wait();  // every CTA of the cluster is running
+    if (!bad) {
+      for (int o = tid; o < G * kDpc; o += kThreads) {
+        const int g = o / kDpc;
+        const int j = o - g * kDpc;
+        const float* qrow = qs + g * kDim;
+        const __nv_bfloat16* wcol = wq_s + static_cast<size_t>(g) * kDim * kDpc + j;
+        float acc = 0.f;
+#pragma unroll 16
+        for (int i = 0; i < kDim; ++i) acc = fmaf(qrow[i], __bfloat162float(wcol[i * kDpc]), acc);
+#pragma unroll
+        for (int r = 0; r < CS; ++r) cluster.map_shared_rank(qv, r)[g * kDim + rank * kDpc + j] = acc;
+      }
+    }
+  } else {
+    cluster_wait();
+  }
+  cluster.sync();  // #1: every CTA holds all of v
+
+  if (MODE != kModeAttend) {
+    if (!bad) {
+      // Q normalisation (RMSNorm, gain gamma_q) and gate RoPE at position c.
+      for (int g = warp; g < G; g += kWarps) {
+        float x[4];
+        float ss = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          x[k] = qv[g * kDim + lane + 32 * k];
+          ss = fmaf(x[k], x[k], ss);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = 1.f / sqrtf(ss / kDim + p.eps);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) x[k] = x[k] * inv * p.gamma_q[lane + 32 * k];
+        float c0, s0, c1, s1;
+        rope_cos_sin(lane, c, p.rope_base, c0, s0);
+        rope_cos_sin(lane + 32, c, p.rope_base, c1, s1);
+        qv[g * kDim + lane] = x[0] * c0 - x[2] * s0;
+        qv[g * kDim + lane + 64] = x[2] * c0 + x[0] * s0;
+        qv[g * kDim + lane + 32] = x[1] * c1 - x[3] * s1;
+        qv[g * kDim + lane + 96] = x[3] * c1 + x[1] * s1;
+      }
+    }
+    __syncthreads();
+    if (MODE == kModeFused && !bad) {
+      // S_b = mean_g(q~_g . k~_b) * scale = (scale/G * sum_g q~_g) . k~_b
+      const float f = p.gate_scale / static_cast<float>(G);
+      for (int d = tid; d < kDim; d += kThreads) {
+        float a = 0.f;
+        for (int g = 0; g < G; ++g) a += qv[g * kDim + d];
+        qbar[d] = a * f;
+      }
+    }
+    __syncthreads();
+
+    // ---------------------------------------------------------- phase 1: scores
+    const int grp = lane >> 3;  // 4 blocks per warp at a time, 8 lanes per block
+    const int sub = lane & 7;   // lane covers dims sub*16 .. sub*16+15
+    const int rot = sub >> 1;   // chunk rotation: conflict-free 16-byte loads
+    float4 qr[4];
+    if (MODE == kModeFused) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        qr[i] = *reinterpret_cast<const float4*>(qbar + sub * 16 + ((i + rot) & 3) * 4);
+    }
+    for (int ci = 0; ci < nchunks; ++ci) {
+      const int slot = ci % NST;
+      const bool ok = mbar_wait(&bars[slot], (ci / NST) & 1, p.status);
+      const int b0 = b_lo + ci * kGkChunk;
+      const int cntb = min(kGkChunk, b_hi - b0);
+      const float* gk = reinterpret_cast<const float*>(slots + slot * kTileBytes);
+#pragma unroll
+      for (int it = 0; it < kGkChunk / 16; ++it) {
+        const int bb = it * 16 + warp * 4 + grp;
+        const bool act = ok && bb < cntb;
+        const float* row = gk + bb * kDim + sub * 16;
+        float S = 0.f;
+        if (MODE == kModeFused) {
+          float acc = 0.f;
+          if (act) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              acc = dot4(qr[i], *reinterpret_cast<const float4*>(row + ((i + rot) & 3) * 4), acc);
+          }
+          acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+          acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+          S = acc;
+        } else {
+          for (int g = 0; g < G; ++g) {
+            float acc = 0.f;
+            if (act) {
+              const float* qrow = qv + g * kDim + sub * 16;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int ch = ((i + rot) & 3) * 4;
+                acc = dot4(*reinterpret_cast<const float4*>(qrow + ch),
+                           *reinterpret_cast<const float4*>(row + ch), acc);
+              }
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+            const float sg = acc * p.gate_scale;
+            S += sg;
+            if (act && sub == 0 && p.head_scores != nullptr)
+              p.head_scores[(static_cast<size_t>(s) * p.hq + h * G + g) * p.mg + b0 + bb] = sg;
+          }
+          S = S / static_cast<float>(G);
+        }
+        if (act && sub == 0) {
+          sslice[b0 - b_lo + bb] = S;
+          if (p.group_scores != nullptr)
+            p.group_scores[static_cast<size_t>(pair) * p.mg + b0 + bb] = S;
+        }
+      }
+      __syncthreads();
+      pump(ci + 1, known);
+    }
+  }
+  if (MODE == kModeGate) return;  // no DSMEM access after barrier #1
+
+  // ------------------------------------------------------------ phase 2: Top-K
+  if (MODE == kModeFused) {
+    cluster.sync();  // #2: all score slices written
+    if (!bad) {
+      for (int b = tid; b < n; b += kThreads) {
+        const int r = b / nb_per;
+        sall[b] = cluster.map_shared_rank(sslice, r)[b - r * nb_per];
+      }
+    }
+    __syncthreads();
+    if (!bad) {
+      const int mm = select_blocks(sall, n, p.topk, c, sel, hist, scan);
+      (void)mm;  // == m by construction
+      if (rank == 0) {
+        if (p.sel_idx != nullptr)
+          for (int j = tid; j < m; j += kThreads)
+            p.sel_idx[static_cast<size_t>(pair) * p.max_sel + j] = sel[j];
+        if (p.sel_count != nullptr && tid == 0) p.sel_count[pair] = m;
+      }
+    } else if (rank == 0 && tid == 0 && p.sel_count != nullptr) {
+      p.sel_count[pair] = 0;
+    }
+    known = nchunks + kTilesPerBlock * cnt_mine;
+    pump(nchunks, known);
+  }
+
+  // ------------------------------------------------------------ phase 3: attention
+  const int tq = lane & 3, gq = lane >> 2;
+  float m_run = -INFINITY, l_run = 0.f;  // bf16 path: head gq of this warp
+  float o_acc[16][2];                      // bf16 path: O[gq][8nt + 2tq + e]
+  float fm[kMaxGroup], fl[kMaxGroup], fo[kMaxGroup][4];  // fp32 path
+  uint32_t qa0[8], qa2[8];
+  if constexpr (!kF32) {
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) o_acc[nt][0] = o_acc[nt][1] = 0.f;
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) +
+                                (static_cast<size_t>(s) * p.hq + h * G + min(gq, G - 1)) * kDim;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      qa0[ks] = (gq < G && !bad) ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq) : 0u;
+      qa2[ks] =
+          (gq < G && !bad) ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * tq) : 0u;
+    }
+  } else {
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g) {
+      fm[g] = -INFINITY;
+      fl[g] = 0.f;
+      fo[g][0] = fo[g][1] = fo[g][2] = fo[g][3] = 0.f;
+    }
+    if (!bad) {
+      const float* qg = static_cast<const float*>(p.q) +
+                        (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim;
+      for (int i = tid; i < G * kDim; i += kThreads) qatt[i] = qg[i];
+    }
+    __syncthreads();
+  }
+  const float sl2 = p.attn_scale_log2;
+
+  for (int e = 0; e < cnt_mine; ++e) {
+    const int b = entry_block(e);
+    const int nvalid = (b == c) ? (L - b * kBlock) : kBlock;
+    const int t0 = nchunks + e * kTilesPerBlock;
+    if constexpr (!kF32) {
+      // ---- K tile: S = q K^T for this warp's 16 tokens
+      const int slotK = t0 % NST;
+      bool ok = mbar_wait(&bars[slotK], (t0 / NST) & 1, p.status);
+      float sacc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      if (ok) {
+        const uint32_t kbase = smem_u32(slots + slotK * kTileBytes);
+        const int mat = lane >> 3;
+        const int tok = 16 * warp + (mat >> 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4(kbase + swz_tile_offset(tok, 2 * ks + (mat & 1)), r0, r1, r2, r3);
+          mma_rows0_7(sacc[0][0], sacc[0][1], qa0[ks], qa2[ks], r0, r1);
+          mma_rows0_7(sacc[1][0], sacc[1][1], qa0[ks], qa2[ks], r2, r3);
+        }
+      }
+      __syncthreads();
+      pump(t0 + 1, known);
+      // ---- online softmax (per warp, head gq)
+      float x[2][2];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int tl = 16 * warp + 8 * nt + 2 * tq + q;
+          x[nt][q] = (tl < nvalid) ? sacc[nt][q] * sl2 : -INFINITY;
+          mx = fmaxf(mx, x[nt][q]);
+        }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      const float mnew = fmaxf(m_run, mx);
+      const float alpha = (mnew == -INFINITY) ? 1.f : exp2f(m_run - mnew);
+      float pr[2][2];
+      float psum = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          pr[nt][q] = (x[nt][q] == -INFINITY) ? 0.f : exp2f(x[nt][q] - mnew);
+          psum += pr[nt][q];
+        }
+      l_run = l_run * alpha + psum;
+      m_run = mnew;
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        o_acc[nt][0] *= alpha;
+        o_acc[nt][1] *= alpha;
+      }
+      const uint32_t pa0 = pack_bf16x2(pr[0][0], pr[0][1]);
+      const uint32_t pa2 = pack_bf16x2(pr[1][0], pr[1][1]);
+      // ---- V tile: O += P V
+      const int t1 = t0 + 1;
+      const int slotV = t1 % NST;
+      ok = mbar_wait(&bars[slotV], (t1 / NST) & 1, p.status);
+      if (ok) {
+        uint8_t* vtile = slots + slotV * kTileBytes;
+        if (nvalid < kBlock) {
+          // rows past the context may hold anything (even NaN): zero this
+          // warp's invalid rows so that P = 0 there gives exactly 0
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int idx = it * 32 + lane;
+            const int row = 16 * warp + (idx >> 4);
+            const int ch = idx & 15;
+            if (row >= nvalid)
+              *reinterpret_cast<uint4*>(vtile + (ch >> 3) * 8192 + row * 128 + (ch & 7) * 16) =
+                  make_uint4(0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();  // the slot is refilled by TMA later
+          __syncwarp();
+        }
+        const uint32_t vbase = smem_u32(vtile);
+        const int mat = lane >> 3;
+        const int tok = 16 * warp + (mat & 1) * 8 + (lane & 7);
+#pragma unroll
+        for (int np = 0; np < 8; ++np) {
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4_trans(vbase + swz_tile_offset(tok, 2 * np + (mat >> 1)), r0, r1, r2, r3);
+          mma_rows0_7(o_acc[2 * np][0], o_acc[2 * np][1], pa0, pa2, r0, r1);
+          mma_rows0_7(o_acc[2 * np + 1][0], o_acc[2 * np + 1][1], pa0, pa2, r2, r3);
+        }
+      }
+      __syncthreads();
+      pump(t1 + 1, known);
+    } else {
+      // ---- fp32 K/V: SIMT path (small parity configurations)
+      const int half = warp >> 1;  // tokens 0..31 in tile t0 (t0+2 for V), 32..63 in t0+1
+      const int tK = t0 + half;
+      bool ok = mbar_wait(&bars[t0 % NST], (t0 / NST) & 1, p.status);
+      ok = mbar_wait(&bars[(t0 + 1) % NST], ((t0 + 1) / NST) & 1, p.status) && ok;
+      const int tt = lane >> 1, hh = lane & 1;
+      const int tl = 16 * warp + tt;
+      float lg[kMaxGroup];
+#pragma unroll
+      for (int g = 0; g < kMaxGroup; ++g) lg[g] = 0.f;
+      if (ok) {
+        const float* krow =
+            reinterpret_cast<const float*>(slots + (tK % NST) * kTileBytes) + (tl & 31) * kDim + hh * 64;
+        for (int i = 0; i < 64; ++i) {
+          const int d = (i + tt) & 63;
+          const float kv = krow[d];
+#pragma unroll
+          for (int g = 0; g < kMaxGroup; ++g)
+            if (g < G) lg[g] = fmaf(qatt[g * kDim + hh * 64 + d], kv, lg[g]);
+        }
+      }
+      __syncthreads();
+      pump(t0 + 2, known);
+      float pg[kMaxGroup];
+#pragma unroll
+      for (int g = 0; g < kMaxGroup; ++g) {
+        float xv = lg[g] + __shfl_xor_sync(0xffffffffu, lg[g], 1);
+        xv = (tl < nvalid) ? xv * sl2 : -INFINITY;
+        float mx = xv;
+#pragma unroll
+        for (int o = 2; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float mnew = fmaxf(fm[g], mx);
+        const float alpha = (mnew == -INFINITY) ? 1.f : exp2f(fm[g] - mnew);
+        pg[g] = (xv == -INFINITY) ? 0.f : exp2f(xv - mnew);
+        float ps = pg[g];
+#pragma unroll
+        for (int o = 2; o < 32; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        fl[g] = fl[g] * alpha + ps;
+        fm[g] = mnew;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) fo[g][k] *= alpha;
+      }
+      const int t2 = t0 + 2;
+      ok = mbar_wait(&bars[t2 % NST], (t2 / NST) & 1, p.status);
+      ok = mbar_wait(&bars[(t2 + 1) % NST], ((t2 + 1) / NST) & 1, p.status) && ok;
+      if (ok) {
+        float* vt = reinterpret_cast<float*>(slots + ((t2 + half) % NST) * kTileBytes);
+        if (nvalid < kBlock) {
+          for (int it = 0; it < 16; ++it) {
+            const int idx = it * 32 + lane;
+            const int row = 16 * warp + (idx >> 5);
+            if (row >= nvalid)
+              *reinterpret_cast<float4*>(vt + (row & 31) * kDim + (idx & 31) * 4) =
+                  make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        for (int tk = 0; tk < 16; ++tk) {
+          const float4 v4 =
+              *reinterpret_cast<const float4*>(vt + ((16 * warp + tk) & 31) * kDim + 4 * lane);
+#pragma unroll
+          for (int g = 0; g < kMaxGroup; ++g) {
+            const float pv = __shfl_sync(0xffffffffu, pg[g], 2 * tk);
+            if (g < G) {
+              fo[g][0] = fmaf(pv, v4.x, fo[g][0]);
+              fo[g][1] = fmaf(pv, v4.y, fo[g][1]);
+              fo[g][2] = fmaf(pv, v4.z, fo[g][2]);
+              fo[g][3] = fmaf(pv, v4.w, fo[g][3]);
+            }
+          }
+        }
+      }
+      __syncthreads();
+      pump(t0 + 4, known);
+    }
+  }
+
+  // per-warp partials (the stage slots are free: every issued tile was consumed)
+  if constexpr (!kF32) {
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    if (gq < G) {
+      if (tq == 0) {
+        pm[warp * kMaxGroup + gq] = m_run;
+        pl[warp * kMaxGroup + gq] = l_run;
+      }
+      float* dst = po + (static_cast<size_t>(warp) * G + gq) * kDim;
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt)
+        *reinterpret_cast<float2*>(dst + 8 * nt + 2 * tq) = make_float2(o_acc[nt][0], o_acc[nt][1]);
+    }
+  } else {
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g) {
+      if (g < G) {
+        if (lane == 0) {
+          pm[warp * kMaxGroup + g] = fm[g];
+          pl[warp * kMaxGroup + g] = fl[g];
+        }
+        *reinterpret_cast<float4*>(po + (static_cast<size_t>(warp) * G + g) * kDim + 4 * lane) =
+            make_float4(fo[g][0], fo[g][1], fo[g][2], fo[g][3]);
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ phase 4: merge
+  cluster.sync();  // #3: all partials written
+  {
+    OutT* out = static_cast<OutT*>(p.out);
+    for (int it = tid; it < G * kDpc; it += kThreads) {
+      const int g = it / kDpc;
+      const int d = rank * kDpc + (it - g * kDpc);
+      float res = 0.f;
+      if (!bad) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < CS; ++r) {
+          const float* rpm = cluster.map_shared_rank(pm, r);
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) M = fmaxf(M, rpm[w * kMaxGroup + g]);
+        }
+        float den = 0.f, num = 0.f;
+#pragma unroll
+        for (int r = 0; r < CS; ++r) {
+          const float* rpm = cluster.map_shared_rank(pm, r);
+          const float* rpl = cluster.map_shared_rank(pl, r);
+          const float* rpo = cluster.map_shared_rank(po, r);
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) {
+            const float mw = rpm[w * kMaxGroup + g];
+            if (mw != -INFINITY) {
+              const float f = exp2f(mw - M);
+              den = fmaf(rpl[w * kMaxGroup + g], f, den);
+              num = fmaf(rpo[(static_cast<size_t>(w) * G + g) * kDim + d], f, num);
+            }
+          }
+        }
+        res = num / den;
+      }
+      out[(static_cast<size_t>(s) * p.hq + h * G + g) * kDim + d] = from_float<OutT>(res);
+    }
+  }
+  cluster.sync();  // #4: no CTA leaves while its partials may still be read
+}
+
+// ------------------------------------------------------------ Top-K kernel
+__global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ TopkParams p) {
+  const int pair = blockIdx.x;
+  const int s = pair / p.hkv;
+  const int tid = threadIdx.x;
+  extern __shared__ uint8_t smem_raw[];
+  float* sall = reinterpret_cast<float*>(smem_raw);
+  int* sel = reinterpret_cast<int*>(smem_raw + (p.mg * 4 + 15) / 16 * 16);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(sel) +
+                                               (p.max_sel * 4 + 15) / 16 * 16);
+  int* scan = reinterpret_cast<int*>(hist + 512);
+  const int L = p.seq_lens[s];
+  if (L < 1 || (L - 1) / kBlock > p.mg) {
+    if (tid == 0) {
+      raise_status(p.status, kStatusBounds);
+      p.sel_count[pair] = 0;
+    }
+    return;
+  }
+  const int c = (L - 1) / kBlock;
+  for (int b = tid; b < c; b += kThreads) sall[b] = p.group_scores[static_cast<size_t>(pair) * p.mg + b];
+  __syncthreads();
+  const int m = select_blocks(sall, c, p.topk, c, sel, hist, scan);
+  for (int j = tid; j < m; j += kThreads) p.sel_idx[static_cast<size_t>(pair) * p.max_sel + j] = sel[j];
+  if (tid == 0) p.sel_count[pair] = m;
+}
+
+size_t topk_smem_bytes(int mg, int max_sel) {
+  return static_cast<size_t>((mg * 4 + 15) / 16 * 16 + (max_sel * 4 + 15) / 16 * 16 + 512 * 4 + 16 * 4);
+}
+
+// ------------------------------------------------------------ launchers
+namespace {
+
+template <typename T, typename OutT, int CS, int NST, int MODE>
+cudaError_t launch_cluster(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                           int batch, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CS, static_cast<unsigned>(batch * p.hkv), 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(p.sm.total);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_cluster_kernel<T, OutT, CS, NST, MODE>, p, tmk, tmv);
+}
+
+template <typename T, typename OutT, int CS, int NST, int MODE>
+cudaError_t set_attrs() {
+  auto k = decode_cluster_kernel<T, OutT, CS, NST, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e != cudaSuccess) return e;
+  if (CS > 8) e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
+}
+
+template <int MODE>
+cudaError_t dispatch_types(bool f32_kv, bool f32_out, int cs, int nst, const DecodeParams& p,
+                           const CUtensorMap& tmk, const CUtensorMap& tmv, int batch,
+                           cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  if (cs != 8 || nst != 2) return cudaErrorInvalidValue;
+  if (!f32_kv && !f32_out) return launch_cluster<bf, bf, 8, 2, MODE>(p, tmk, tmv, batch, st);
+  if (!f32_kv && f32_out) return launch_cluster<bf, float, 8, 2, MODE>(p, tmk, tmv, batch, st);
+  if (f32_kv && !f32_out) return launch_cluster<float, bf, 8, 2, MODE>(p, tmk, tmv, batch, st);
+  return launch_cluster<float, float, 8, 2, MODE>(p, tmk, tmv, batch, st);
+}
+
+template <int MODE>
+cudaError_t attrs_for_mode() {
+  using bf = __nv_bfloat16;
+  cudaError_t e;
+  if ((e = set_attrs<bf, bf, 8, 2, MODE>()) != cudaSuccess) return e;
+  if ((e = set_attrs<bf, float, 8, 2, MODE>()) != cudaSuccess) return e;
+  if ((e = set_attrs<float, bf, 8, 2, MODE>()) != cudaSuccess) return e;
+  return set_attrs<float, float, 8, 2, MODE>();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(int mode, bool f32_kv, bool f32_out, int cs, int nst,
+                          const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                          int batch, cudaStream_t stream) {
+  switch (mode) {
+    case kModeGate:
+      return dispatch_types<kModeGate>(f32_kv, false, cs, nst, p, tmk, tmv, batch, stream);
+    case kModeAttend:
+      return dispatch_types<kModeAttend>(f32_kv, f32_out, cs, nst, p, tmk, tmv, batch, stream);
+    default:
+      return dispatch_types<kModeFused>(f32_kv, f32_out, cs, nst, p, tmk, tmv, batch, stream);
+  }
+}
+
+cudaError_t launch_topk(const TopkParams& p, int batch, cudaStream_t stream) {
+  const size_t smem = topk_smem_bytes(p.mg, p.max_sel);
+  topk_kernel<<<static_cast<unsigned>(batch * p.hkv), kThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t prepare_decode_kernels() {
+  cudaError_t e;
+  if ((e = attrs_for_mode<kModeGate>()) != cudaSuccess) return e;
+  if ((e = attrs_for_mode<kModeAttend>()) != cudaSuccess) return e;
+  if ((e = attrs_for_mode<kModeFused>()) != cudaSuccess) return e;
+  return cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+}
+
+}  // namespace sas

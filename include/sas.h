@@ -1,0 +1,218 @@
+/*
+ * sas.h -- C ABI of libsas: SAS (Simple-Attention-Sparsification) gated
+ * Top-K KV-block selection feeding block-sparse GQA attention, for NVIDIA
+ * B200 (sm_100a).
+ *
+ * What the method fixes (release pages: "Tencent released
+ * Simple-Attention-Sparsification, a method for efficient sparse attention
+ * in Qwen3 models", aigc.news 2026-09-14, release paragraph; "Simple-Attention-
+ * Sparsification Text Generation Model: 12GB+ VRAM", localmodelwatch,
+ * "Specifications and Configuration Table"):
+ *   KV block size 64 tokens; gate hidden size 128; query projection "Qproj";
+ *   key block pooling max + min + average; Q/K normalization; gate RoPE;
+ *   Top-K of historical blocks under a 1,024 / 2,048 (default) / 4,096-token
+ *   budget, the current block always kept (31 + 1 = 2,048 / 64).
+ *
+ * Readings of what the pages leave open (one per item, used by every entry
+ * point):
+ *   - gate weights: W_q [128][128] per query head, W_k [384][128] per KV head,
+ *     bf16, applied as x @ W (row vector times matrix), no bias; one RMSNorm
+ *     gain [128] for q and one for k per layer (the printed parameter counts
+ *     33.0M / 42.0M fit exactly this layout);
+ *   - pooled key of block b = [max ; min ; mean] over its 64 tokens, per dim;
+ *   - k~_b = RoPE(RMSNorm(pooled_b @ W_k) * gamma_k, position b);
+ *     q~_g = RoPE(RMSNorm(q_g @ W_q[g]) * gamma_q, position c), c the current
+ *     block index floor((L-1)/64); RMSNorm x / sqrt(mean(x^2) + eps);
+ *     RoPE rotate-half, pairs (i, i+64), angle pos * base^(-2i/128);
+ *   - s_{g,b} = (q~_g . k~_b) * gate_scale; group score S_b = mean over the
+ *     G = Hq/Hkv query heads of a KV head; one block set per KV head;
+ *   - selection: the min(budget/64 - 1, c) historical blocks of largest S
+ *     (ties: lower index), plus block c, listed in ascending order;
+ *   - attention: softmax(q . k_j * attn_scale) over every token j <= L-1 of
+ *     the selected blocks, each selected block weighted 1.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are caller-owned DEVICE memory; the library never
+ *     allocates, frees or synchronises (except sas_get_device_status, which
+ *     synchronises the given stream).
+ *   - Every call validates its arguments on the host, enqueues its kernels on
+ *     `stream` and returns.  Host-detected problems return an error code and
+ *     enqueue nothing.  A failed launch returns SAS_ERR_CUDA.
+ *   - Problems only the device can see (a sequence length beyond the cache,
+ *     a page id out of range, a selected block beyond the current block)
+ *     skip the affected (sequence, KV head), write zeros to its outputs and
+ *     set a bit in the status word at the start of `ws`; read it with
+ *     sas_get_device_status.  No device-side trap or assert is used.
+ *   - Every bounded device wait that runs out (1 s) sets SAS_ERR_TIMEOUT's
+ *     bit in the same status word and the kernel returns.
+ *   - The first call that launches kernels performs one-time set-up (kernel
+ *     attributes, driver entry point for tensor maps); make it before any
+ *     CUDA stream capture.
+ *   - Layouts are row-major C arrays; the shapes below use
+ *     B = batch, Hq/Hkv = query/KV heads, D = 128, MG = max_gate_blocks.
+ */
+#ifndef SAS_H_
+#define SAS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SAS_API __attribute__((visibility("default")))
+#else
+#define SAS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t.  NULL means the legacy default stream. */
+typedef struct CUstream_st* sas_stream_t;
+
+typedef enum {
+  SAS_OK = 0,
+  SAS_ERR_INVALID_ARG = 1,   /* a host-checked argument is wrong */
+  SAS_ERR_UNSUPPORTED = 2,   /* valid request this build does not handle */
+  SAS_ERR_WORKSPACE = 3,     /* ws NULL, misaligned or smaller than needed */
+  SAS_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  SAS_ERR_DEVICE_BOUNDS = 5, /* device saw an out-of-range length/page/index */
+  SAS_ERR_TIMEOUT = 6        /* a bounded device wait ran out */
+} sas_status;
+
+typedef enum { SAS_DTYPE_BF16 = 0, SAS_DTYPE_F32 = 1 } sas_dtype;
+
+typedef struct {
+  int32_t num_q_heads;   /* Hq >= 1 */
+  int32_t num_kv_heads;  /* Hkv >= 1, Hq % Hkv == 0, 1 <= Hq/Hkv <= 8 */
+  int32_t head_dim;      /* must be 128 */
+  int32_t block_size;    /* must be 64 (KV block size of the method) */
+  int32_t gate_hidden;   /* must be 128 (gate hidden size of the method) */
+  int32_t token_budget;  /* multiple of 64, 64 .. 16384; default 2048 */
+  float rope_base;       /* gate RoPE base, > 0; default 10000 */
+  float norm_eps;        /* RMSNorm epsilon, >= 0; default 1e-6 */
+  float attn_scale;      /* attention logit scale, > 0; default 1/sqrt(128) */
+  float gate_scale;      /* gate score scale, > 0; default 1/sqrt(128) */
+  int32_t kv_dtype;      /* sas_dtype of q, K and V (and of prefill Q) */
+  int32_t out_dtype;     /* sas_dtype of the attention output */
+} sas_config;
+
+/* KV cache description (device pointers, caller-owned). */
+typedef struct {
+  const void* k;               /* keys, kv_dtype, 16-byte aligned */
+  const void* v;               /* values, same layout as k */
+  const int32_t* block_table;  /* NULL: contiguous layout [B][Hkv][capacity][D].
+                                  Else paged layout [num_pages][Hkv][64][D] and
+                                  block_table [B][max_blocks_per_seq] holds the
+                                  page id of each 64-token block. */
+  const int32_t* seq_lens;     /* [B] context length L_s >= 1 of each sequence,
+                                  including the token being decoded */
+  int32_t batch;               /* B >= 0 (0: nothing to do) */
+  int32_t capacity;            /* contiguous: tokens per (seq, head), multiple
+                                  of 64; paged: ignored */
+  int32_t num_pages;           /* paged: pages in the pool; contiguous: ignored */
+  int32_t max_blocks_per_seq;  /* paged: row length of block_table */
+} sas_kv;
+
+/* Bytes of device workspace `ws` every entry point below needs for this
+ * configuration (status word plus any scratch).  max_seq_len is the largest
+ * L_s (decode) or T (prefill) of the calls that will use it. */
+SAS_API size_t sas_workspace_bytes(const sas_config* cfg, int32_t batch, int32_t max_seq_len);
+
+/* Zero the status word at the start of ws (cudaMemsetAsync on `stream`). */
+SAS_API sas_status sas_reset_device_status(void* ws, sas_stream_t stream);
+
+/* Synchronise `stream`, read the status word of ws and return it as a
+ * sas_status in *out (SAS_OK, SAS_ERR_DEVICE_BOUNDS or SAS_ERR_TIMEOUT; bounds
+ * wins when both bits are set). */
+SAS_API sas_status sas_get_device_status(const void* ws, sas_stream_t stream, sas_status* out);
+
+SAS_API const char* sas_status_string(sas_status s);
+
+/* ABI version of this header; bumped on any signature or layout change. */
+SAS_API int32_t sas_abi_version(void);
+
+/*
+ * Pooling and gate keys (pages: "key block pooling max + min + average",
+ * "Q/K normalization", "gate RoPE"; gate hidden 128).
+ *
+ * For each sequence s and KV head h, pools blocks
+ *   b = blk_begin[s] .. blk_begin[s] + num_blocks - 1
+ * (blk_begin may be NULL: 0 for every sequence), skipping blocks that are not
+ * complete (64*(b+1) > L_s) or have b >= max_gate_blocks, and writes
+ *   gate_keys[s][h][b][:] = RoPE(RMSNorm(P_b @ W_k[h]) * gamma_k, b)   (fp32)
+ *   pooled_raw[s][h][b][:] = P_b = [max ; min ; mean]                 (fp32,
+ *   optional, NULL to skip).
+ * Call it for new complete blocks as tokens are appended (incremental), or
+ * with blk_begin NULL and num_blocks = L/64 after a prefill.
+ *   w_k       bf16 [Hkv][384][128]     gamma_k  fp32 [128]
+ *   gate_keys fp32 [B][Hkv][MG][128]   pooled_raw fp32 [B][Hkv][MG][384]
+ */
+SAS_API sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv,
+                         const int32_t* blk_begin, int32_t num_blocks,
+                         const void* w_k, const float* gamma_k,
+                         float* gate_keys, int32_t max_gate_blocks,
+                         float* pooled_raw, void* ws, size_t ws_bytes,
+                         sas_stream_t stream);
+
+/*
+ * Gate scores of every historical block (pages: gate "learns to rank and
+ * select KV blocks"; query projection Qproj).
+ *   q            kv_dtype [B][Hq][128]  query of token L_s - 1
+ *   w_q          bf16 [Hq][128][128]    gamma_q fp32 [128]
+ *   gate_keys    fp32 [B][Hkv][MG][128] (from sas_pool_keys)
+ *   head_scores  fp32 [B][Hq][MG]  s_{g,b} for b < c_s (optional, NULL)
+ *   group_scores fp32 [B][Hkv][MG] S_b for b < c_s
+ * Entries b >= c_s are left untouched.  Requires c_s <= MG.
+ */
+SAS_API sas_status sas_gate_scores(const sas_config* cfg, const void* q, const int32_t* seq_lens,
+                           int32_t batch, const void* w_q, const float* gamma_q,
+                           const float* gate_keys, int32_t max_gate_blocks,
+                           float* head_scores, float* group_scores,
+                           void* ws, size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * Top-K block selection under the token budget (pages: training Top-K 31,
+ * default budget 2,048; 1,024 and 4,096 usable without retraining).
+ *   group_scores fp32 [B][Hkv][MG]
+ *   sel_idx   int32 [B][Hkv][budget/64]: ascending block ids, the current
+ *             block c_s last; entries past sel_count are left untouched
+ *   sel_count int32 [B][Hkv] = min(budget/64, c_s + 1)
+ */
+SAS_API sas_status sas_topk_blocks(const sas_config* cfg, const float* group_scores,
+                           const int32_t* seq_lens, int32_t batch, int32_t max_gate_blocks,
+                           int32_t* sel_idx, int32_t* sel_count,
+                           void* ws, size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * Block-sparse flash-decoding attention over given block lists (the sparse
+ * decode backend the pages name for inference).
+ *   q    kv_dtype [B][Hq][128]
+ *   sel_idx / sel_count as produced by sas_topk_blocks (any ascending list of
+ *   blocks <= c_s whose last entry is c_s is accepted)
+ *   out  out_dtype [B][Hq][128]
+ */
+SAS_API sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const sas_kv* kv,
+                             const int32_t* sel_idx, const int32_t* sel_count,
+                             void* out, void* ws, size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * Fused decode step: gate query, scores, Top-K and block-sparse attention in
+ * one launch (one thread-block cluster per (sequence, KV head); the cluster's
+ * CTAs split the gate keys and the selected blocks and merge through
+ * distributed shared memory).
+ *   sel_idx, sel_count, group_scores: optional outputs (NULL to skip), layouts
+ *   as above.
+ */
+SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const sas_kv* kv,
+                           const void* w_q, const float* gamma_q,
+                           const float* gate_keys, int32_t max_gate_blocks,
+                           void* out, int32_t* sel_idx, int32_t* sel_count,
+                           float* group_scores, void* ws, size_t ws_bytes,
+                           sas_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* SAS_H_ */

@@ -1,0 +1,142 @@
+"""Shared helpers of the parity tests: run the library on a workload, run the
+CPU oracle on chosen (sequence, KV head) pairs, and compare with the
+tolerances of the acceptance bar (block sets exact up to a 1e-3 tie window,
+gate scores 1e-3 relative with a floor, outputs 1e-2 max-abs)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from gated_block_sparse_token_b200 import sas
+from gated_block_sparse_token_b200.workloads import BLOCK, logical_kv
+from oracle import sas_oracle as O
+
+OUT_ATOL = 1e-2        # attention outputs, bf16 storage / fp32 accumulate
+SCORE_RTOL = 1e-3      # gate scores and gate keys, relative ...
+SCORE_FLOOR = 1e-3     # ... to max(|x|, 1e-3 * max|x|): the pure relative form is ill-posed near 0
+TIE_RTOL = 1e-3        # K-th vs (K+1)-th oracle score window for set mismatches
+
+
+def config_for(spec, budget, out_dtype="bf16"):
+    return sas.Config(spec.hq, spec.hkv, token_budget=budget, kv_dtype=spec.kv_dtype,
+                      out_dtype=out_dtype)
+
+
+def kv_of(inputs):
+    return sas.KvCache(inputs["k"], inputs["v"], inputs["seq_lens"], inputs["block_table"])
+
+
+def gate_key_rows(spec):
+    return spec.cap // BLOCK
+
+
+def run_pool(inputs, cfg, ws, gate_keys=None, pooled_raw=None, blk_begin=None, num_blocks=None):
+    spec = inputs["spec"]
+    dev = inputs["q"].device
+    mg = gate_key_rows(spec)
+    if gate_keys is None:
+        gate_keys = torch.zeros(spec.batch, spec.hkv, mg, 128, dtype=torch.float32, device=dev)
+    sas.pool_keys(cfg, kv_of(inputs), inputs["w_k"], inputs["gamma_k"], gate_keys, ws,
+                  blk_begin=blk_begin, num_blocks=num_blocks, pooled_raw=pooled_raw)
+    return gate_keys
+
+
+def run_decode_step(inputs, cfg, ws, gate_keys):
+    spec = inputs["spec"]
+    dev = inputs["q"].device
+    B = spec.batch
+    mg = gate_keys.shape[2]
+    out = torch.full((B, spec.hq, 128), float("nan"), dtype=sas.out_dtype(cfg), device=dev)
+    sel_idx = torch.full((B, spec.hkv, cfg.max_sel), -1, dtype=torch.int32, device=dev)
+    sel_count = torch.full((B, spec.hkv), -1, dtype=torch.int32, device=dev)
+    group_scores = torch.full((B, spec.hkv, mg), float("nan"), dtype=torch.float32, device=dev)
+    sas.decode_step(cfg, inputs["q"], kv_of(inputs), inputs["w_q"], inputs["gamma_q"], gate_keys,
+                    out, ws, sel_idx=sel_idx, sel_count=sel_count, group_scores=group_scores)
+    return {"out": out, "sel_idx": sel_idx, "sel_count": sel_count, "group_scores": group_scores}
+
+
+def oracle_pairs(inputs, budget, pairs):
+    """Oracle decode step (gate keys recomputed from K) for the listed pairs."""
+    spec = inputs["spec"]
+    G = spec.hq // spec.hkv
+    q = inputs["q"].double().cpu().numpy()
+    wq = inputs["w_q"].double().cpu().numpy()
+    wk = inputs["w_k"].double().cpu().numpy()
+    gq = inputs["gamma_q"].double().cpu().numpy()
+    gk = inputs["gamma_k"].double().cpu().numpy()
+    res = {}
+    for (s, h) in pairs:
+        L = int(spec.seq_lens[s])
+        ks, vs = logical_kv(inputs, s, h, L)
+        c = (L - 1) // BLOCK
+        keys = O.gate_keys_for_sequence(ks, c, wk[h], gk)
+        r = O.decode_one_group(q[s, h * G:(h + 1) * G], ks, vs, L, keys, wq[h * G:(h + 1) * G],
+                               np.tile(gq, (G, 1)), budget)
+        r["gate_keys"] = keys
+        r["k"], r["v"], r["L"] = ks, vs, L
+        res[(s, h)] = r
+    return res
+
+
+def assert_close_rel(got, want, what, rtol=SCORE_RTOL, floor=SCORE_FLOOR):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    if want.size == 0:
+        return
+    scale = np.maximum(np.abs(want), floor * np.max(np.abs(want)))
+    err = np.abs(got - want) / scale
+    i = int(np.argmax(err))
+    assert err.flat[i] <= rtol, f"{what}: rel err {err.flat[i]:.3g} at {i} (got {got.flat[i]}, want {want.flat[i]})"
+
+
+def assert_selection(gpu_sel, oracle_sel, S, topk, what=""):
+    """Exact block sets, except blocks swapped inside the K-th/(K+1)-th window."""
+    gpu_sel = [int(x) for x in gpu_sel]
+    assert len(gpu_sel) == len(oracle_sel), (what, gpu_sel, oracle_sel)
+    assert gpu_sel == sorted(gpu_sel) and len(set(gpu_sel)) == len(gpu_sel), (what, gpu_sel)
+    assert gpu_sel[-1] == oracle_sel[-1], (what, gpu_sel[-1], oracle_sel[-1])
+    if gpu_sel == oracle_sel:
+        return False
+    n = len(S)
+    K = min(topk, n)
+    order = sorted(range(n), key=lambda b: (-float(S[b]), b))
+    sK = float(S[order[K - 1]])
+    sK1 = float(S[order[K]]) if K < n else -math.inf
+    scale = max(abs(sK), SCORE_FLOOR * float(np.max(np.abs(S))))
+    assert abs(sK - sK1) <= TIE_RTOL * scale, f"{what}: set mismatch outside the tie window"
+    for b in set(gpu_sel) ^ set(oracle_sel):
+        assert abs(float(S[b]) - sK) <= TIE_RTOL * scale, f"{what}: block {b} outside the tie window"
+    return True
+
+
+def check_pairs(inputs, cfg, gpu, oracle, gate_keys=None, out_atol=OUT_ATOL):
+    """Compare a fused decode step's outputs with the oracle on the given pairs."""
+    spec = inputs["spec"]
+    G = spec.hq // spec.hkv
+    topk = cfg.max_sel - 1
+    out = gpu["out"].float().cpu().numpy()
+    sel_idx = gpu["sel_idx"].cpu().numpy()
+    sel_count = gpu["sel_count"].cpu().numpy()
+    gs = gpu["group_scores"].cpu().numpy()
+    gkeys = None if gate_keys is None else gate_keys.cpu().numpy()
+    for (s, h), r in oracle.items():
+        tag = f"{spec.name} s={s} h={h} budget={cfg.token_budget}"
+        c = len(r["S"])
+        if gkeys is not None:
+            assert_close_rel(gkeys[s, h, :c], r["gate_keys"], tag + " gate keys")
+        assert_close_rel(gs[s, h, :c], r["S"], tag + " group scores")
+        m = int(sel_count[s, h])
+        sel = list(sel_idx[s, h, :m])
+        swapped = assert_selection(sel, r["sel"], r["S"], topk, tag)
+        want = r["out"]
+        if swapped:  # an accepted tie swap: attend over the GPU's set
+            toks = O.selected_token_ids(sel, r["L"])
+            qg = inputs["q"][s, h * G:(h + 1) * G].double().cpu().numpy()
+            want = np.stack([O.attention_over_tokens(qg[g], r["k"], r["v"], toks, cfg.attn_scale)
+                             for g in range(G)])
+        got = out[s, h * G:(h + 1) * G]
+        err = float(np.max(np.abs(got - want)))
+        assert np.all(np.isfinite(got)) and err <= out_atol, f"{tag}: out max-abs err {err}"

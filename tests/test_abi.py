@@ -1,0 +1,180 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the
+header declares, the ctypes mirrors match the C struct layouts (checked
+against a gcc build of the header), and host-side validation rejects bad
+arguments before touching CUDA."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+import torch
+
+from gated_block_sparse_token_b200 import build as B
+from gated_block_sparse_token_b200 import sas
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sas.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return sas.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"^SAS_API\s+[\w\s\*]+?\b(sas_\w+)\(", src, flags=re.M)
+
+
+def test_header_declares_all_entry_points():
+    names = set(declared_functions())
+    want = {"sas_pool_keys", "sas_gate_scores", "sas_topk_blocks", "sas_sparse_decode",
+            "sas_decode_step", "sas_workspace_bytes", "sas_get_device_status",
+            "sas_reset_device_status", "sas_status_string", "sas_abi_version"}
+    assert want <= names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", sas.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (sas_\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(L, name)
+
+
+def test_library_needs_no_driver_at_load():
+    out = subprocess.run(["ldd", sas.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libtorch" not in out
+
+
+def test_struct_layout_matches_header():
+    prog = r'''
+#include <stdio.h>
+#include <stddef.h>
+#include "sas.h"
+#define O(T, f) printf("%s.%s %zu\n", #T, #f, offsetof(T, f))
+int main(void) {
+  printf("sizeof.sas_config %zu\nsizeof.sas_kv %zu\n", sizeof(sas_config), sizeof(sas_kv));
+  O(sas_config, token_budget); O(sas_config, rope_base); O(sas_config, gate_scale);
+  O(sas_config, kv_dtype); O(sas_config, out_dtype);
+  O(sas_kv, block_table); O(sas_kv, seq_lens); O(sas_kv, batch); O(sas_kv, capacity);
+  O(sas_kv, num_pages); O(sas_kv, max_blocks_per_seq);
+  return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(prog)
+        subprocess.run(["gcc", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
+        lines = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = dict(l.split() for l in lines if l.strip())
+    assert int(got["sizeof.sas_config"]) == ctypes.sizeof(sas._Config)
+    assert int(got["sizeof.sas_kv"]) == ctypes.sizeof(sas._Kv)
+    for key, val in got.items():
+        if key.startswith("sizeof"):
+            continue
+        struct, fieldname = key.split(".")
+        cls = sas._Config if struct == "sas_config" else sas._Kv
+        assert getattr(cls, fieldname).offset == int(val), key
+
+
+def test_abi_version_and_status_strings(L):
+    assert sas.abi_version() >= 1
+    for st in range(7):
+        assert len(sas.status_string(st)) > 0
+    assert sas.status_string(sas.SAS_OK) == "ok"
+
+
+# Host validation.  Every call below must fail in the host checks, which come
+# before any CUDA call; pointers are dummies that are never dereferenced.
+# Skipped where a GPU is present so that a validation bug can never launch a
+# kernel on dummy pointers.
+nogpu = pytest.mark.skipif(torch.cuda.is_available(), reason="host validation runs on CPU-only hosts")
+FAKE = 0x100000  # 16-byte aligned dummy address
+
+
+def _cfg(**kw):
+    base = dict(num_q_heads=32, num_kv_heads=8, token_budget=2048)
+    base.update(kw)
+    return sas.Config(**base)
+
+
+def _kv(batch=2, cap=4096, **kw):
+    k = sas._Kv(FAKE, FAKE, None, FAKE, batch, cap, 0, 0)
+    for key, val in kw.items():
+        setattr(k, key, val)
+    return k
+
+
+def _decode(L, cfg, kv=None, ws_bytes=256, ws=FAKE, q=FAKE, out=FAKE, mg=64):
+    c = cfg.c()
+    kv = kv or _kv()
+    return L.sas_decode_step(ctypes.byref(c), q, ctypes.byref(kv), FAKE, FAKE, FAKE, mg, out,
+                             None, None, None, ws, ws_bytes, None)
+
+
+@nogpu
+@pytest.mark.parametrize("kw,status", [
+    (dict(head_dim=64), sas.SAS_ERR_UNSUPPORTED),
+    (dict(block_size=32), sas.SAS_ERR_INVALID_ARG),
+    (dict(gate_hidden=64), sas.SAS_ERR_INVALID_ARG),
+    (dict(token_budget=100), sas.SAS_ERR_INVALID_ARG),
+    (dict(token_budget=0), sas.SAS_ERR_INVALID_ARG),
+    (dict(token_budget=32768), sas.SAS_ERR_UNSUPPORTED),
+    (dict(num_q_heads=30), sas.SAS_ERR_INVALID_ARG),
+    (dict(num_q_heads=72, num_kv_heads=8), sas.SAS_ERR_UNSUPPORTED),
+    (dict(attn_scale=0.0), sas.SAS_ERR_INVALID_ARG),
+    (dict(gate_scale=float("nan")), sas.SAS_ERR_INVALID_ARG),
+    (dict(norm_eps=-1.0), sas.SAS_ERR_INVALID_ARG),
+    (dict(rope_base=-5.0), sas.SAS_ERR_INVALID_ARG),
+])
+def test_config_validation(L, kw, status):
+    assert _decode(L, _cfg(**kw)) == status
+
+
+@nogpu
+def test_workspace_and_pointer_validation(L):
+    cfg = _cfg()
+    assert _decode(L, cfg, ws_bytes=8) == sas.SAS_ERR_WORKSPACE
+    assert _decode(L, cfg, ws=0) == sas.SAS_ERR_WORKSPACE
+    assert _decode(L, cfg, ws=FAKE + 4) == sas.SAS_ERR_WORKSPACE
+    assert _decode(L, cfg, kv=_kv(cap=1000)) == sas.SAS_ERR_INVALID_ARG
+    assert _decode(L, cfg, kv=_kv(k=FAKE + 2)) == sas.SAS_ERR_INVALID_ARG
+    assert _decode(L, cfg, kv=_kv(seq_lens=None)) == sas.SAS_ERR_INVALID_ARG
+    assert _decode(L, cfg, kv=_kv(batch=-1)) == sas.SAS_ERR_INVALID_ARG
+    # a paged cache needs pages and a block-table width
+    assert _decode(L, cfg, kv=_kv(block_table=FAKE, num_pages=0, max_blocks_per_seq=4)) == sas.SAS_ERR_INVALID_ARG
+    # TMA row coordinates are 32-bit
+    assert _decode(L, cfg, kv=_kv(batch=4096, cap=1 << 20)) == sas.SAS_ERR_UNSUPPORTED
+    assert _decode(L, cfg, q=0) == sas.SAS_ERR_INVALID_ARG
+    assert _decode(L, cfg, mg=0) == sas.SAS_ERR_INVALID_ARG
+
+
+@nogpu
+def test_empty_batch_is_a_no_op(L):
+    assert _decode(L, _cfg(), kv=_kv(batch=0)) == sas.SAS_OK
+
+
+@nogpu
+def test_other_entry_points_validate(L):
+    c = _cfg(token_budget=96).c()
+    kv = _kv()
+    assert L.sas_pool_keys(ctypes.byref(c), ctypes.byref(kv), None, 4, FAKE, FAKE, FAKE, 64, None,
+                           FAKE, 256, None) == sas.SAS_ERR_INVALID_ARG
+    c = _cfg().c()
+    assert L.sas_pool_keys(ctypes.byref(c), ctypes.byref(kv), None, -1, FAKE, FAKE, FAKE, 64, None,
+                           FAKE, 256, None) == sas.SAS_ERR_INVALID_ARG
+    assert L.sas_gate_scores(ctypes.byref(c), FAKE, FAKE, 2, FAKE, FAKE, FAKE, 64, None, None,
+                             FAKE, 256, None) == sas.SAS_ERR_INVALID_ARG
+    assert L.sas_topk_blocks(ctypes.byref(c), FAKE, FAKE, 2, 64, FAKE, None, FAKE, 256,
+                             None) == sas.SAS_ERR_INVALID_ARG
+    assert L.sas_sparse_decode(ctypes.byref(c), FAKE, ctypes.byref(kv), None, FAKE, FAKE, FAKE,
+                               256, None) == sas.SAS_ERR_INVALID_ARG
+    st = ctypes.c_int(0)
+    assert L.sas_get_device_status(None, None, ctypes.byref(st)) == sas.SAS_ERR_INVALID_ARG
+    assert L.sas_reset_device_status(None, None) == sas.SAS_ERR_WORKSPACE

@@ -1,0 +1,290 @@
+"""GPU parity of the decode path against the CPU oracle, through the C ABI.
+
+Small shapes span several gate-key chunks, several selected blocks per CTA
+and ragged current blocks; the full-size workloads (Qwen3-4B 32k batch 8,
+Qwen3-8B ragged batch 32, Qwen3-14B paged 128k) are checked on sampled
+(sequence, KV head) pairs the oracle computes one by one."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from gated_block_sparse_token_b200 import sas
+from gated_block_sparse_token_b200.workloads import (DecodeSpec, make_decode_inputs, qwen3_4b_32k,
+                                                     qwen3_8b_ragged, qwen3_14b_paged_128k,
+                                                     tiny_decode, logical_kv)
+from oracle import sas_oracle as O
+
+import sas_testlib as T
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _all_pairs(spec):
+    return [(s, h) for s in range(spec.batch) for h in range(spec.hkv)]
+
+
+def _run_and_check(spec, budget, out_dtype="bf16", pairs=None, out_atol=T.OUT_ATOL):
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, budget, out_dtype)
+    ws = sas.make_workspace(cfg, DEV)
+    gk = T.run_pool(inp, cfg, ws)
+    gpu = T.run_decode_step(inp, cfg, ws, gk)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    pairs = pairs or _all_pairs(spec)
+    orc = T.oracle_pairs(inp, budget, pairs)
+    T.check_pairs(inp, cfg, gpu, orc, gate_keys=gk, out_atol=out_atol)
+    return inp, cfg, gpu, orc
+
+
+SMALL = [
+    # name, B, hq, hkv, lens, budget, dtype
+    ("g4_multi_tile", 2, 8, 2, [4096, 2500], 1024, "bf16"),
+    ("g4_ragged_tail", 3, 4, 1, [65, 1000, 2049], 256, "bf16"),
+    ("g5_qwen14b_heads", 2, 10, 2, [3000, 4097], 512, "bf16"),
+    ("g8", 1, 8, 1, [1800], 320, "bf16"),
+    ("g1", 2, 2, 2, [777, 64], 128, "bf16"),
+    ("budget64_current_only", 2, 8, 2, [1000, 3], 64, "bf16"),
+    ("single_token", 1, 4, 1, [1], 2048, "bf16"),
+    ("full_first_block", 1, 4, 1, [64], 2048, "bf16"),
+    ("budget_covers_context", 2, 8, 2, [1500, 640], 2048, "bf16"),
+    ("long_slices", 1, 4, 1, [20000], 1024, "bf16"),
+    ("f32_small", 2, 8, 2, [1500, 333], 512, "f32"),
+]
+
+
+@pytest.mark.parametrize("name,B,hq,hkv,lens,budget,dt", SMALL, ids=[s[0] for s in SMALL])
+def test_decode_step_small(name, B, hq, hkv, lens, budget, dt):
+    spec = DecodeSpec(name, B, hq, hkv, lens, (budget,), kv_dtype=dt, block_offset_std=0.5, seed=11)
+    _run_and_check(spec, budget, out_atol=(2e-4 if dt == "f32" else T.OUT_ATOL),
+                   out_dtype=("f32" if dt == "f32" else "bf16"))
+
+
+def test_decode_step_f32_out_from_bf16_cache():
+    spec = DecodeSpec("bf16_to_f32", 2, 8, 2, [3000, 1234], (512,), seed=12)
+    _run_and_check(spec, 512, out_dtype="f32")
+
+
+def test_paged_small():
+    spec = DecodeSpec("paged_small", 2, 8, 2, [2000, 4096], (512,), paged=True, capacity=4096, seed=13)
+    _run_and_check(spec, 512)
+
+
+def test_tiny_config_full():
+    """One sequence, one KV head, G 4, 4,096 tokens, budget 1,024, fp32 Q/K/V."""
+    spec = tiny_decode()
+    _run_and_check(spec, 1024, out_dtype="f32", out_atol=2e-4)
+
+
+def test_budget_covering_context_equals_dense():
+    spec = DecodeSpec("dense", 2, 8, 2, [1200, 2048], (2048,), seed=14)
+    inp, cfg, gpu, _ = _run_and_check(spec, 2048)
+    out = gpu["out"].float().cpu().numpy()
+    q = inp["q"].double().cpu().numpy()
+    for s in range(2):
+        for h in range(2):
+            ks, vs = logical_kv(inp, s, h, spec.seq_lens[s])
+            dense = O.dense_causal_decode(q[s, 4 * h:4 * h + 4], ks, vs, spec.seq_lens[s])
+            assert np.max(np.abs(out[s, 4 * h:4 * h + 4] - dense)) <= T.OUT_ATOL
+
+
+def test_values_past_context_are_ignored():
+    """NaN in cache rows past L (the unwritten tail of the current block) must
+    not reach the output."""
+    spec = DecodeSpec("nan_tail", 2, 8, 2, [1000, 2050], (512,), capacity=4096, seed=15)
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, 512)
+    ws = sas.make_workspace(cfg, DEV)
+    gk = T.run_pool(inp, cfg, ws)
+    for s, L in enumerate(spec.seq_lens):
+        inp["k"][s, :, L:] = float("nan")
+        inp["v"][s, :, L:] = float("nan")
+    gpu = T.run_decode_step(inp, cfg, ws, gk)
+    orc = T.oracle_pairs(inp, 512, _all_pairs(spec))
+    T.check_pairs(inp, cfg, gpu, orc, gate_keys=gk)
+
+
+def test_pool_keys_vs_oracle_and_raw_pooling():
+    spec = DecodeSpec("pool", 2, 8, 2, [3000, 700], (512,), capacity=4096, block_offset_std=0.5, seed=16)
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, 512)
+    ws = sas.make_workspace(cfg, DEV)
+    mg = T.gate_key_rows(spec)
+    raw = torch.zeros(2, 2, mg, 384, dtype=torch.float32, device=DEV)
+    gk = T.run_pool(inp, cfg, ws, pooled_raw=raw)
+    torch.cuda.synchronize()
+    gk, raw = gk.cpu().numpy(), raw.cpu().numpy()
+    wk = inp["w_k"].double().cpu().numpy()
+    for s in range(2):
+        for h in range(2):
+            L = spec.seq_lens[s]
+            ks, _ = logical_kv(inp, s, h, L)
+            nfull = L // 64
+            want = O.gate_keys_for_sequence(ks, nfull, wk[h], np.ones(128))
+            T.assert_close_rel(gk[s, h, :nfull], want, f"gate keys s={s} h={h}")
+            assert np.all(gk[s, h, nfull:] == 0), "incomplete blocks must not be pooled"
+            for b in range(nfull):
+                p = O.pool_block(ks[64 * b:64 * b + 64])
+                assert np.array_equal(raw[s, h, b, :256], p[:256])  # max, min exact
+                assert np.allclose(raw[s, h, b, 256:], p[256:], rtol=1e-6, atol=1e-7)
+
+
+def test_incremental_pooling_matches_full_pooling():
+    spec = DecodeSpec("incr", 2, 8, 2, [4096, 3000], (512,), capacity=4096, seed=17)
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, 512)
+    ws = sas.make_workspace(cfg, DEV)
+    full = T.run_pool(inp, cfg, ws)
+    # pool the first part, then the rest block by block from per-sequence starts
+    part = torch.zeros_like(full)
+    T.run_pool(inp, cfg, ws, gate_keys=part, num_blocks=20)
+    begin = torch.full((2,), 20, dtype=torch.int32, device=DEV)
+    for _ in range(50):
+        T.run_pool(inp, cfg, ws, gate_keys=part, blk_begin=begin, num_blocks=1)
+        begin += 1
+    torch.cuda.synchronize()
+    assert torch.equal(part, full)
+
+
+def test_gate_scores_entry_point():
+    spec = DecodeSpec("gate", 3, 10, 2, [4000, 129, 2500], (1024,), capacity=4096, seed=18)
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, 1024)
+    ws = sas.make_workspace(cfg, DEV)
+    gk = T.run_pool(inp, cfg, ws)
+    mg = gk.shape[2]
+    head = torch.full((3, 10, mg), float("nan"), device=DEV)
+    group = torch.full((3, 2, mg), float("nan"), device=DEV)
+    sas.gate_scores(cfg, inp["q"], inp["seq_lens"], inp["w_q"], inp["gamma_q"], gk, group, ws,
+                    head_scores=head)
+    torch.cuda.synchronize()
+    orc = T.oracle_pairs(inp, 1024, _all_pairs(spec))
+    head, group = head.cpu().numpy(), group.cpu().numpy()
+    for (s, h), r in orc.items():
+        c = len(r["S"])
+        T.assert_close_rel(group[s, h, :c], r["S"], f"group s={s} h={h}")
+        T.assert_close_rel(head[s, 5 * h:5 * h + 5, :c], r["s"], f"head s={s} h={h}")
+
+
+@pytest.mark.parametrize("budget", [64, 256, 1024, 4096])
+def test_topk_exact_with_ties(budget):
+    """Selection on given scores must equal the full-sort rule exactly, ties
+    included (scores drawn from a handful of values)."""
+    g = torch.Generator().manual_seed(budget)
+    B, hkv, mg = 3, 4, 2048
+    lens = torch.tensor([1, 2000, 131072 // 64], dtype=torch.int32)
+    lens = torch.tensor([1, 2000, 64 * 2047 + 5], dtype=torch.int32)
+    scores = (torch.randint(-4, 5, (B, hkv, mg), generator=g).float() * 0.25)
+    scores[1, 1] += torch.randn(mg, generator=g) * 1e-3
+    scores[2, 3] = torch.randn(mg, generator=g)
+    cfg = sas.Config(4 * hkv, hkv, token_budget=budget)
+    ws = sas.make_workspace(cfg, DEV)
+    sel = torch.full((B, hkv, budget // 64), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.full((B, hkv), -1, dtype=torch.int32, device=DEV)
+    sas.topk_blocks(cfg, scores.to(DEV), lens.to(DEV), sel, cnt, ws)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    for s in range(B):
+        c = (int(lens[s]) - 1) // 64
+        for h in range(hkv):
+            want = O.select_blocks(scores[s, h, :c].double().numpy(), c, budget // 64 - 1)
+            assert int(cnt[s, h]) == len(want)
+            assert list(sel[s, h, :len(want)]) == want, (s, h)
+
+
+def test_sparse_decode_given_blocks():
+    spec = DecodeSpec("given", 2, 8, 2, [3000, 2100], (512,), capacity=4096, seed=19)
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, 512)
+    ws = sas.make_workspace(cfg, DEV)
+    orc = T.oracle_pairs(inp, 512, _all_pairs(spec))
+    sel = torch.full((2, 2, 8), -1, dtype=torch.int32)
+    cnt = torch.zeros((2, 2), dtype=torch.int32)
+    for (s, h), r in orc.items():
+        sel[s, h, :len(r["sel"])] = torch.tensor(r["sel"], dtype=torch.int32)
+        cnt[s, h] = len(r["sel"])
+    out = torch.full((2, 8, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
+    sas.sparse_decode(cfg, inp["q"], T.kv_of(inp), sel.to(DEV), cnt.to(DEV), out, ws)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    out = out.float().cpu().numpy()
+    for (s, h), r in orc.items():
+        assert np.max(np.abs(out[s, 4 * h:4 * h + 4] - r["out"])) <= T.OUT_ATOL
+
+
+def test_device_bounds_are_reported_not_faulted():
+    """A sequence longer than its cache, and a block table entry outside the
+    page pool, are caught by the kernels' own checks (no access is issued):
+    status bit set, that (seq, head) zeroed, the others still correct."""
+    spec = DecodeSpec("bounds", 2, 8, 2, [1000, 2000], (512,), capacity=2048, seed=20)
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, 512)
+    ws = sas.make_workspace(cfg, DEV)
+    gk = T.run_pool(inp, cfg, ws)
+    torch.cuda.synchronize()
+    inp["seq_lens"][1] = 5000  # beyond capacity 2048
+    gpu = T.run_decode_step(inp, cfg, ws, gk)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_ERR_DEVICE_BOUNDS
+    assert torch.all(gpu["out"][1] == 0)
+    assert int(gpu["sel_count"][1, 0]) == 0
+    inp["seq_lens"][1] = 2000
+    orc = T.oracle_pairs(inp, 512, [(0, 0), (0, 1)])
+    T.check_pairs(inp, cfg, gpu, orc)
+    # paged: a page id past the pool
+    spec = DecodeSpec("bounds_paged", 2, 8, 2, [1000, 2000], (512,), paged=True, capacity=2048, seed=21)
+    inp = make_decode_inputs(spec, DEV)
+    ws = sas.make_workspace(cfg, DEV)
+    gk = T.run_pool(inp, cfg, ws)
+    torch.cuda.synchronize()
+    inp["block_table"][0, 3] = 10 ** 6
+    gpu = T.run_decode_step(inp, cfg, ws, gk)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_ERR_DEVICE_BOUNDS
+    assert torch.all(gpu["out"][0] == 0)
+    sas.reset_device_status(ws)
+    assert sas.get_device_status(ws) == sas.SAS_OK
+
+
+# ------------------------------------------------------------ full-size workloads
+def test_qwen3_4b_32k_full_size():
+    spec = qwen3_4b_32k()
+    _run_and_check(spec, 2048, pairs=[(0, 0), (3, 5), (7, 7), (5, 2)])
+
+
+@pytest.mark.parametrize("budget", [1024, 2048, 4096])
+def test_qwen3_8b_ragged_full_size(budget):
+    spec = qwen3_8b_ragged()
+    _run_and_check(spec, budget, pairs=[(0, 0), (13, 4), (31, 7)])
+
+
+def test_qwen3_14b_paged_128k_incremental():
+    """Pool all but the last 256 tokens, then append them 64 at a time (one
+    pooling call per completed block) and decode at 131,072."""
+    spec = qwen3_14b_paged_128k()
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, 4096)
+    ws = sas.make_workspace(cfg, DEV)
+    full_len = spec.seq_lens[0]
+    start = full_len - spec.appended
+    lens = inp["seq_lens"].clone()
+    inp["seq_lens"].fill_(start)
+    gk = T.run_pool(inp, cfg, ws)
+    begin = torch.full((spec.batch,), start // 64, dtype=torch.int32, device=DEV)
+    for t in range(64, spec.appended + 1, 64):
+        inp["seq_lens"].fill_(start + t)
+        T.run_pool(inp, cfg, ws, gate_keys=gk, blk_begin=begin, num_blocks=1)
+        begin += 1
+    inp["seq_lens"].copy_(lens)
+    ref = T.run_pool(inp, cfg, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(gk, ref)
+    gpu = T.run_decode_step(inp, cfg, ws, gk)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    orc = T.oracle_pairs(inp, 4096, [(0, 0), (9, 3), (15, 7)])
+    T.check_pairs(inp, cfg, gpu, orc, gate_keys=gk)
