@@ -268,14 +268,17 @@ def plan(fn, K, layers, stream, chunk=512):
 
 
 def timed(graphs, world, stream):
+    """Device time of replaying `graphs` (CUDAGraph.replay launches on the
+    current stream, so replays and events both go to `stream`)."""
     import torch
     barrier(world)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    run_graphs(graphs)
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        run_graphs(graphs)
+        e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     return max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
@@ -309,7 +312,8 @@ def run_ours(args):
     fn = lambda L, st: step(cfg, L, st)  # noqa: E731
     warm = plan(fn, args.warmup, layers, stream)
     main = plan(fn, args.steps, layers, stream)
-    run_graphs(warm)
+    with torch.cuda.stream(stream):
+        run_graphs(warm)
     torch.cuda.synchronize()
     clk = ClockSampler(local)
     clk.start()
@@ -322,7 +326,8 @@ def run_ours(args):
 
     # dominant kernel alone (same rotation), for the roofline
     dk = plan(lambda L, st: decode_only(cfg, L, st), args.steps, layers, stream)
-    run_graphs(plan(lambda L, st: decode_only(cfg, L, st), min(args.warmup, 200), layers, stream))
+    with torch.cuda.stream(stream):
+        run_graphs(plan(lambda L, st: decode_only(cfg, L, st), min(args.warmup, 200), layers, stream))
     t_dec = timed(dk, world, stream)
     del dk
 

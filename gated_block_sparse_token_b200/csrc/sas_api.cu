@@ -12,6 +12,7 @@
 
 namespace sas {
 cudaError_t prepare_decode_kernels();
+cudaError_t prepare_pool_kernels();
 }
 
 namespace {
@@ -46,6 +47,7 @@ cudaError_t prepare() {
     }
     g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     g_prep_err = sas::prepare_decode_kernels();
+    if (g_prep_err == cudaSuccess) g_prep_err = sas::prepare_pool_kernels();
   });
   return g_prep_err;
 }
@@ -125,6 +127,22 @@ bool encode_kv_map(CUtensorMap* m, const void* ptr, long long rows) {
   return r == CUDA_SUCCESS;
 }
 
+// 2-D view [Hq*128][128] of bf16 W_q; one box = the 128 rows of one query
+// head restricted to the 128/CS columns a cluster CTA projects.
+bool encode_wq_map(CUtensorMap* m, const void* w_q, int hq) {
+  memset(m, 0, sizeof(*m));
+  if (g_encode == nullptr) return false;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(hq) * kDim};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(kDim * 2)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kDim / kClusterSize), static_cast<cuuint32_t>(kDim)};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w_q), gdim,
+                              gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 long long kv_rows(const sas_config* cfg, const sas_kv* kv) {
   return kv->block_table != nullptr
              ? static_cast<long long>(kv->num_pages) * cfg->num_kv_heads * 64
@@ -144,6 +162,20 @@ void fill_common(sas::DecodeParams& p, const sas_config* cfg, int mg) {
   p.gate_scale = cfg->gate_scale;
   p.sm = sas::plan_decode_smem(p.G, mg, kClusterSize, kStages, p.max_sel,
                                cfg->kv_dtype == SAS_DTYPE_F32);
+  sas::fill_rope_table(p.rope, cfg->rope_base);
+}
+
+bool plan_ok(const sas::DecodeParams& p) {
+  return p.sm.total <= 227 * 1024 && sas::decode_smem_aligned(p.sm, p.G, kDim / kClusterSize);
+}
+
+unsigned long long* trace_region(void* ws) {
+#ifdef SAS_PHASE_TRACE
+  return reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ws) + kStatusBytes);
+#else
+  (void)ws;
+  return nullptr;
+#endif
 }
 
 sas_status launch_result(cudaError_t e) {
@@ -177,7 +209,11 @@ size_t sas_workspace_bytes(const sas_config* cfg, int32_t batch, int32_t max_seq
   (void)cfg;
   (void)batch;
   (void)max_seq_len;
+#ifdef SAS_PHASE_TRACE
+  return kStatusBytes + static_cast<size_t>(sas::kTraceCtas) * sas::kTraceSlots * 8;
+#else
   return kStatusBytes;
+#endif
 }
 
 sas_status sas_reset_device_status(void* ws, sas_stream_t stream) {
@@ -227,6 +263,7 @@ sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv, const int32_t*
   p.num_blocks = num_blocks;
   p.rope_base = cfg->rope_base;
   p.eps = cfg->norm_eps;
+  sas::fill_rope_table(p.rope, cfg->rope_base);
   p.kv = make_view(cfg, kv);
   p.blk_begin = blk_begin;
   p.w_k = static_cast<const __nv_bfloat16*>(w_k);
@@ -250,7 +287,7 @@ sas_status sas_gate_scores(const sas_config* cfg, const void* q, const int32_t* 
   if (q == nullptr || seq_lens == nullptr || w_q == nullptr || gamma_q == nullptr ||
       gate_keys == nullptr || group_scores == nullptr)
     return SAS_ERR_INVALID_ARG;
-  if (!aligned(q, 4) || !aligned(seq_lens, 4) || !aligned(w_q, 16) || !aligned(gamma_q, 4) ||
+  if (!aligned(q, 16) || !aligned(seq_lens, 4) || !aligned(w_q, 16) || !aligned(gamma_q, 16) ||
       !aligned(gate_keys, 16) || !aligned(group_scores, 4) ||
       (head_scores != nullptr && !aligned(head_scores, 4)))
     return SAS_ERR_INVALID_ARG;
@@ -258,7 +295,7 @@ sas_status sas_gate_scores(const sas_config* cfg, const void* q, const int32_t* 
   if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
   sas::DecodeParams p{};
   fill_common(p, cfg, max_gate_blocks);
-  if (p.sm.total > 227 * 1024) return SAS_ERR_UNSUPPORTED;
+  if (!plan_ok(p)) return SAS_ERR_UNSUPPORTED;
   p.q = q;
   p.w_q = static_cast<const __nv_bfloat16*>(w_q);
   p.gamma_q = gamma_q;
@@ -268,10 +305,12 @@ sas_status sas_gate_scores(const sas_config* cfg, const void* q, const int32_t* 
   p.head_scores = head_scores;
   p.group_scores = group_scores;
   p.status = static_cast<uint32_t*>(ws);
-  CUtensorMap dummy;
+  p.trace = trace_region(ws);
+  CUtensorMap dummy, tmw;
   memset(&dummy, 0, sizeof(dummy));
+  if (!encode_wq_map(&tmw, w_q, cfg->num_q_heads)) return SAS_ERR_CUDA;
   return launch_result(sas::launch_decode(sas::kModeGate, cfg->kv_dtype == SAS_DTYPE_F32, false,
-                                          kClusterSize, kStages, p, dummy, dummy, batch,
+                                          kClusterSize, kStages, p, dummy, dummy, tmw, batch,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -313,11 +352,11 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
   if ((st = check_kv(cfg, kv)) != SAS_OK) return st;
   if ((st = check_ws(cfg, ws, ws_bytes)) != SAS_OK) return st;
   if (kv->batch == 0) return SAS_OK;
-  if (q == nullptr || out == nullptr || !aligned(q, 4) || !aligned(out, 4)) return SAS_ERR_INVALID_ARG;
+  if (q == nullptr || out == nullptr || !aligned(q, 16) || !aligned(out, 4)) return SAS_ERR_INVALID_ARG;
   if (mode == sas::kModeFused) {
     if (max_gate_blocks < 1 || max_gate_blocks > kMaxGateBlocks) return SAS_ERR_INVALID_ARG;
     if (w_q == nullptr || gamma_q == nullptr || gate_keys == nullptr) return SAS_ERR_INVALID_ARG;
-    if (!aligned(w_q, 16) || !aligned(gamma_q, 4) || !aligned(gate_keys, 16)) return SAS_ERR_INVALID_ARG;
+    if (!aligned(w_q, 16) || !aligned(gamma_q, 16) || !aligned(gate_keys, 16)) return SAS_ERR_INVALID_ARG;
     if ((sel_idx != nullptr && !aligned(sel_idx, 4)) || (sel_count != nullptr && !aligned(sel_count, 4)) ||
         (group_scores != nullptr && !aligned(group_scores, 4)))
       return SAS_ERR_INVALID_ARG;
@@ -330,7 +369,7 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
   if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
   sas::DecodeParams p{};
   fill_common(p, cfg, max_gate_blocks);
-  if (p.sm.total > 227 * 1024) return SAS_ERR_UNSUPPORTED;
+  if (!plan_ok(p)) return SAS_ERR_UNSUPPORTED;
   p.q = q;
   p.w_q = static_cast<const __nv_bfloat16*>(w_q);
   p.gamma_q = gamma_q;
@@ -341,16 +380,19 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
   p.sel_count = sel_count;
   p.out = out;
   p.status = static_cast<uint32_t*>(ws);
+  p.trace = trace_region(ws);
   const bool f32_kv = cfg->kv_dtype == SAS_DTYPE_F32;
-  CUtensorMap tmk, tmv;
+  CUtensorMap tmk, tmv, tmw;
   memset(&tmk, 0, sizeof(tmk));
   memset(&tmv, 0, sizeof(tmv));
+  memset(&tmw, 0, sizeof(tmw));
   if (!f32_kv) {
     const long long rows = kv_rows(cfg, kv);
     if (!encode_kv_map(&tmk, kv->k, rows) || !encode_kv_map(&tmv, kv->v, rows)) return SAS_ERR_CUDA;
   }
+  if (mode == sas::kModeFused && !encode_wq_map(&tmw, w_q, cfg->num_q_heads)) return SAS_ERR_CUDA;
   return launch_result(sas::launch_decode(mode, f32_kv, cfg->out_dtype == SAS_DTYPE_F32,
-                                          kClusterSize, kStages, p, tmk, tmv, kv->batch,
+                                          kClusterSize, kStages, p, tmk, tmv, tmw, kv->batch,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -11,20 +11,24 @@
 // plus the current block are attended.
 //
 // Work split of one cluster of CS CTAs (128 threads each) for (s, h):
+//   start    every load that does not depend on the sequence length (q, the
+//            CTA's W_q column slice, gains, RoPE frequencies) is issued first.
 //   phase 0  each CTA computes 128/CS columns of v_g = q_g @ W_q[g] for the G
 //            query heads of the group and stores them into every CTA of the
 //            cluster (distributed shared memory); RMSNorm + RoPE -> q~_g.
 //   phase 1  each CTA streams 1/CS of the gate keys k~_b (TMA bulk copies
-//            into a ring of 16 KiB stage slots) and scores its blocks.
-//   phase 2  every CTA gathers all group scores through DSMEM and runs the
-//            same radix select (exact, ties -> lower index), so all CTAs
-//            hold the same ascending block list without another barrier.
+//            into a ring of 16 KiB stage slots), scores its blocks and stores
+//            each score into every CTA of the cluster.
+//   phase 2  every CTA runs the same exact selection on the full score list
+//            (value buckets, exact ranking inside the boundary bucket, ties to
+//            the lower index), so all CTAs hold the same ascending block list.
 //   phase 3  CTA r attends to list entries j = r (mod CS): K and V tiles come
-//            in by 2-D TMA (128-byte swizzle) and each warp runs flash-
-//            decoding over 16 tokens of every tile with bf16 mma.sync
-//            (GQA group as the M=16 rows, fp32 accumulate, online softmax).
-//   phase 4  the 4*CS per-warp partials (m, l, o) are merged through DSMEM;
-//            CTA r writes 128/CS output columns.
+//            in by 2-D TMA (128-byte swizzle); each warp runs flash-decoding
+//            over 16 tokens of every tile on bf16 mma.sync (the GQA group as
+//            the M=16 rows, fp32 accumulate, online softmax).
+//   phase 4  each CTA folds its 4 warps' partials (m, l, o) and stores the
+//            128/CS-column slices into the owning CTAs; after one cluster
+//            barrier CTA r merges the CS partials of its columns locally.
 // The CTA that owns the current block (always selected) prefetches its
 // tiles before the selection finishes.
 #include <cooperative_groups.h>
@@ -36,6 +40,21 @@
 namespace cg = cooperative_groups;
 
 namespace sas {
+
+// Phase-trace hook: thread 0 of each CTA stamps the global timer at phase
+// boundaries (tracing builds only).
+#ifdef SAS_PHASE_TRACE
+#define SAS_TRACE(k)                                                                        \
+  do {                                                                                      \
+    const unsigned cta_ = blockIdx.y * gridDim.x + blockIdx.x;                              \
+    if (p.trace != nullptr && threadIdx.x == 0 && cta_ < static_cast<unsigned>(kTraceCtas)) \
+      p.trace[cta_ * kTraceSlots + (k)] = global_timer_ns();                               \
+  } while (0)
+#else
+#define SAS_TRACE(k) \
+  do {               \
+  } while (0)
+#endif
 
 namespace {
 
@@ -62,108 +81,141 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scan) {
 }
 
 // Top-K selection (pages: training Top-K 31 under the 2,048-token budget).
-// Keeps the min(topk, n) largest of sall[0..n) -- ties go to the lower index
+// Keeps the min(topk, n) largest of vals[0..n) -- ties go to the lower index
 // -- lists them ascending in sel[], appends the current block `cur` and
-// returns the count.  Exact radix select on order-preserving 32-bit keys
-// (four 8-bit passes), then an index-ordered compaction.  Called by all
-// kThreads threads of the CTA; overwrites sall with the keys.
-__device__ int select_blocks(float* sall, int n, int topk, int cur, int* sel, uint32_t* hist,
-                             int* scan) {
-  const int tid = threadIdx.x;
+// returns the count.  Exact: scores map to order-preserving 32-bit keys,
+// which are spread over kSelBins buckets by a monotone map (the leading 10
+// bits of key - min key); the
+// bucket holding the topk-th key is found from the histogram, everything
+// above it is kept, and inside it the members are ranked exactly by
+// (key descending, index ascending).  Called by all kThreads threads;
+// overwrites vals with the keys.
+__device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
+                             uint32_t* selbits, int* scan) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (topk <= 0) {  // a 64-token budget keeps the current block only
+    if (tid == 0) sel[0] = cur;
+    __syncthreads();
+    return 1;
+  }
   if (n <= topk) {
     for (int i = tid; i < n; i += kThreads) sel[i] = i;
     if (tid == 0) sel[n] = cur;
     __syncthreads();
     return n + 1;
   }
-  uint32_t* keys = reinterpret_cast<uint32_t*>(sall);
-  for (int i = tid; i < n; i += kThreads) keys[i] = order_key(sall[i]);
-  for (int i = tid; i < 512; i += kThreads) hist[i] = 0u;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int i = tid; i < n; i += kThreads) {
+    const uint32_t k = order_key(vals[i]);
+    keys[i] = k;
+    lo = min(lo, k);
+    hi = max(hi, k);
+  }
+  for (int i = tid; i < kSelBins; i += kThreads) hist[i] = 0u;
+  for (int i = tid; i < (n + 31) / 32; i += kThreads) selbits[i] = 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    scan[warp] = static_cast<int>(lo);
+    scan[4 + warp] = static_cast<int>(hi);
+  }
+  if (tid == 0) scan[10] = 0;
   __syncthreads();
-  uint32_t prefix = 0u;
-  int remaining = topk;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    const uint32_t hmask = (pass == 0) ? 0u : (0xFFFFFFFFu << (shift + 8));
-    uint32_t* hcur = hist + (pass & 1) * 256;
-    uint32_t* hnext = hist + ((pass + 1) & 1) * 256;
-    for (int i = tid; i < n; i += kThreads) {
-      const uint32_t k = keys[i];
-      if ((k & hmask) == prefix) atomicAdd(&hcur[(k >> shift) & 255u], 1u);
-    }
-    __syncthreads();
-    if (tid < 32) {
-      // lane l owns bins 255-8l .. 248-8l, so lane order is descending key order
-      uint32_t cnt[8];
-      uint32_t tot = 0u;
+  lo = static_cast<uint32_t>(scan[0]);
+  hi = static_cast<uint32_t>(scan[4]);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        cnt[j] = hcur[255 - 8 * tid - j];
-        tot += cnt[j];
-      }
-      uint32_t inc = tot;
+  for (int w = 1; w < kWarps; ++w) {
+    lo = min(lo, static_cast<uint32_t>(scan[w]));
+    hi = max(hi, static_cast<uint32_t>(scan[4 + w]));
+  }
+  // monotone bucket map: the top 10 significant bits of (key - lo)
+  const uint32_t span = hi - lo;
+  const int shift = max(0, 32 - __clz(static_cast<int>(span | 1u)) - 10);
+  auto bin_of = [&](uint32_t k) -> int { return static_cast<int>((k - lo) >> shift); };
+  for (int i = tid; i < n; i += kThreads) atomicAdd(&hist[bin_of(keys[i])], 1u);
+  __syncthreads();
+  // thread t owns buckets kSelBins-1-8t .. kSelBins-8-8t (descending order)
+  static_assert(kSelBins == 8 * kThreads, "bucket ownership");
+  uint32_t cnt[8];
+  int tot = 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (tid >= o) inc += y;
-      }
-      const uint32_t exc = inc - tot;
-      const uint32_t want = static_cast<uint32_t>(remaining);
-      if (exc < want && want <= inc) {
-        uint32_t run = exc;
-        bool done = false;
+  for (int j = 0; j < 8; ++j) {
+    cnt[j] = hist[kSelBins - 1 - 8 * tid - j];
+    tot += static_cast<int>(cnt[j]);
+  }
+  const int excl = block_exclusive_scan(tot, scan);
+  if (excl < topk && topk <= excl + tot) {
+    int run = excl;
+    bool done = false;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (!done) {
-            if (run + cnt[j] >= want) {
-              scan[8] = 255 - 8 * tid - j;
-              scan[9] = static_cast<int>(want - run);
-              done = true;
-            } else {
-              run += cnt[j];
-            }
-          }
+    for (int j = 0; j < 8; ++j) {
+      if (!done) {
+        if (run + static_cast<int>(cnt[j]) >= topk) {
+          scan[8] = kSelBins - 1 - 8 * tid - j;
+          scan[9] = topk - run;  // members of the boundary bucket to keep
+          done = true;
+        } else {
+          run += static_cast<int>(cnt[j]);
         }
       }
     }
-    for (int i = tid; i < 256; i += kThreads) hnext[i] = 0u;
-    __syncthreads();
-    prefix |= static_cast<uint32_t>(scan[8]) << shift;
-    remaining = scan[9];
   }
-  // prefix is now the exact key of the topk-th largest score; keep every key
-  // above it and the first `remaining` keys equal to it, in index order.
-  const uint32_t thr = prefix;
-  const int take_eq = remaining;
+  __syncthreads();
+  const int bstar = scan[8];
+  const int take = scan[9];
+  int* cand = reinterpret_cast<int*>(hist);  // the histogram is no longer needed
+  for (int i = tid; i < n; i += kThreads) {
+    if (bin_of(keys[i]) == bstar) {
+      const int pos = atomicAdd(&scan[10], 1);
+      if (pos < kSelCand) cand[pos] = i;
+    }
+  }
+  __syncthreads();
+  const int nc = scan[10];
+  if (nc <= kSelCand) {
+    for (int ci = warp; ci < nc; ci += kWarps) {
+      const int i = cand[ci];
+      const uint32_t ki = keys[i];
+      int r = 0;
+      for (int cj = lane; cj < nc; cj += 32) {
+        const int j = cand[cj];
+        const uint32_t kj = keys[j];
+        r += (kj > ki || (kj == ki && j < i)) ? 1 : 0;
+      }
+      r = __reduce_add_sync(0xffffffffu, r);
+      if (lane == 0 && r < take) atomicOr(&selbits[i >> 5], 1u << (i & 31));
+    }
+  } else {
+    // a crowded boundary bucket (many equal scores): rank against all members
+    for (int i = tid; i < n; i += kThreads) {
+      const uint32_t ki = keys[i];
+      if (bin_of(ki) != bstar) continue;
+      int r = 0;
+      for (int j = 0; j < n; ++j) {
+        const uint32_t kj = keys[j];
+        r += (bin_of(kj) == bstar && (kj > ki || (kj == ki && j < i))) ? 1 : 0;
+      }
+      if (r < take) atomicOr(&selbits[i >> 5], 1u << (i & 31));
+    }
+  }
+  __syncthreads();
+  // ascending list: everything above the boundary bucket plus the marked members
   const int per = (n + kThreads - 1) / kThreads;
-  const int lo = min(n, tid * per);
-  const int hi = min(n, lo + per);
-  int ceq = 0;
-  for (int i = lo; i < hi; ++i) ceq += (keys[i] == thr) ? 1 : 0;
-  const int eq_before = block_exclusive_scan(ceq, scan);
-  int cnt = 0;
-  int eqs = eq_before;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t k = keys[i];
-    if (k > thr) {
-      ++cnt;
-    } else if (k == thr) {
-      if (eqs < take_eq) ++cnt;
-      ++eqs;
-    }
+  const int i0 = min(n, tid * per);
+  const int i1 = min(n, i0 + per);
+  int cntk = 0;
+  for (int i = i0; i < i1; ++i) {
+    const int b = bin_of(keys[i]);
+    cntk += (b > bstar || (b == bstar && ((selbits[i >> 5] >> (i & 31)) & 1u))) ? 1 : 0;
   }
-  int pos = block_exclusive_scan(cnt, scan);
-  eqs = eq_before;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t k = keys[i];
-    bool take = false;
-    if (k > thr) {
-      take = true;
-    } else if (k == thr) {
-      take = eqs < take_eq;
-      ++eqs;
-    }
-    if (take) sel[pos++] = i;
+  int pos = block_exclusive_scan(cntk, scan);
+  for (int i = i0; i < i1; ++i) {
+    const int b = bin_of(keys[i]);
+    if (b > bstar || (b == bstar && ((selbits[i >> 5] >> (i & 31)) & 1u))) sel[pos++] = i;
   }
   if (tid == 0) sel[topk] = cur;
   __syncthreads();
@@ -184,14 +236,16 @@ template <typename T, typename OutT, int CS, int NST, int MODE>
 __global__ void __launch_bounds__(kThreads, 4)
     decode_cluster_kernel(const __grid_constant__ DecodeParams p,
                           const __grid_constant__ CUtensorMap tmk,
-                          const __grid_constant__ CUtensorMap tmv) {
+                          const __grid_constant__ CUtensorMap tmv,
+                          const __grid_constant__ CUtensorMap tmw) {
   constexpr bool kF32 = std::is_same<T, float>::value;
-  constexpr int kDpc = kDim / CS;                // output / W_q columns per CTA
-  constexpr int kTilesPerBlock = kF32 ? 4 : 2;   // 16 KiB tiles per K+V block
+  constexpr int kDpc = kDim / CS;               // output / W_q columns per CTA
+  constexpr int kTilesPerBlock = kF32 ? 4 : 2;  // 16 KiB tiles per K+V block
   static_assert(kDpc % 8 == 0, "cluster size must divide 128 into 16-byte slices");
 
   cg::cluster_group cluster = cg::this_cluster();
   cluster_arrive_relaxed();  // matched by cluster_wait() before the first DSMEM store
+  SAS_TRACE(0);
   const int rank = static_cast<int>(cluster.block_rank());
   const int pair = blockIdx.y;
   const int s = pair / p.hkv;
@@ -202,20 +256,49 @@ __global__ void __launch_bounds__(kThreads, 4)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align_smem_1024(smem_raw);
   uint8_t* slots = base + p.sm.slots;
-  float* sslice = reinterpret_cast<float*>(base + p.sm.sslice);
-  __nv_bfloat16* wq_s = reinterpret_cast<__nv_bfloat16*>(base + p.sm.u_wq);
-  float* qs = reinterpret_cast<float*>(base + p.sm.u_qs);
-  float* sall = reinterpret_cast<float*>(base + p.sm.u_sall);
-  int* sel = reinterpret_cast<int*>(base + p.sm.u_sel);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(base + p.sm.u_hist);
-  int* scan = reinterpret_cast<int*>(base + p.sm.u_scan);
-  float* qv = reinterpret_cast<float*>(base + p.sm.qv);
+  int* sel = reinterpret_cast<int*>(base + p.sm.sel);
+  T* qraw = reinterpret_cast<T*>(base + p.sm.qraw);
   float* qbar = reinterpret_cast<float*>(base + p.sm.qbar);
-  float* qatt = reinterpret_cast<float*>(base + p.sm.qatt);
   float* pm = reinterpret_cast<float*>(base + p.sm.pml);
   float* pl = pm + kWarps * kMaxGroup;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + p.sm.bars);
+  float* qv = reinterpret_cast<float*>(base + p.sm.r_qv);
+  __nv_bfloat16* wq_s = reinterpret_cast<__nv_bfloat16*>(base + p.sm.r_wq);
+  float* gam_s = reinterpret_cast<float*>(base + p.sm.gam);
+  uint64_t* bar_pro = bars + NST;  // prologue copies: q, W_q slice, gamma_q
+  float* inbox_o = reinterpret_cast<float*>(base + p.sm.r_inbox);  // [CS][G][kDpc]
+  float* inbox_ml = inbox_o + CS * G * kDpc;                         // [CS][G][2]
+  float* keys = reinterpret_cast<float*>(base + p.sm.r_keys);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(base + p.sm.r_hist);
+  uint32_t* selbits = reinterpret_cast<uint32_t*>(base + p.sm.r_selbits);
+  int* scan = reinterpret_cast<int*>(base + p.sm.r_scan);
   float* po = reinterpret_cast<float*>(slots);  // [4][G][128], after the last tile
+
+  // ------------------------------------------------------------ prologue copies
+  // Everything that does not depend on the sequence length is requested
+  // first, asynchronously: q of the group (bulk), the W_q column slice of
+  // this CTA (one 2-D TMA box per head) and gamma_q (bulk).
+  if (tid == 0) {
+    for (int i = 0; i <= NST; ++i) mbar_init(&bars[i], 1);
+    fence_mbar_init();
+    const uint32_t qbytes = static_cast<uint32_t>(G * kDim * sizeof(T));
+    uint32_t tx = qbytes;
+    if (MODE != kModeAttend) tx += static_cast<uint32_t>(G * kDim * kDpc * 2 + kDim * 4);
+    mbar_arrive_expect_tx(bar_pro, tx);
+    bulk_g2s(qraw, static_cast<const T*>(p.q) + (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim,
+             qbytes, bar_pro);
+    if (MODE != kModeAttend) {
+      for (int g = 0; g < G; ++g)
+        tma_load_2d(wq_s + static_cast<size_t>(g) * kDim * kDpc, &tmw, rank * kDpc, (h * G + g) * kDim,
+                    bar_pro);
+      bulk_g2s(gam_s, p.gamma_q, kDim * 4, bar_pro);
+    }
+  }
+  double th0 = 0.0, th1 = 0.0;
+  if (MODE != kModeAttend) {
+    th0 = p.rope.theta_over_pi[lane];
+    th1 = p.rope.theta_over_pi[lane + 32];
+  }
 
   // ------------------------------------------------------------ validation
   const int L = p.kv.seq_lens[s];
@@ -228,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   }
   int m = 0;  // entries of the block list (current block last)
   if (MODE == kModeAttend && !err) {
-    int mm = p.sel_count[pair];
+    const int mm = p.sel_count[pair];
     if (mm < 1 || mm > p.max_sel) {
       err = true;
     } else {
@@ -305,56 +388,44 @@ __global__ void __launch_bounds__(kThreads, 4)
     while (issued < known && issued < consumed + NST) issue(issued++);
   };
 
-  if (tid == 0) {
-    for (int i = 0; i < NST; ++i) mbar_init(&bars[i], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
   // before the selection only the gate-key chunks and the current block are known
   int known = nchunks + ((MODE == kModeAttend) ? kTilesPerBlock * cnt_mine
                                                : (own_cur ? kTilesPerBlock : 0));
   pump(0, known);
+  SAS_TRACE(1);
 
   // ------------------------------------------------------------ phase 0: gate query
-  if (MODE != kModeAttend) {
-    if (!bad) {
-      const T* qg = static_cast<const T*>(p.q) +
-                    (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim;
-      for (int i = tid; i < G * kDim; i += kThreads) qs[i] = to_float(qg[i]);
-      constexpr int kVec = kDpc / 8;
-      for (int it = tid; it < G * kDim * kVec; it += kThreads) {
-        const int g = it / (kDim * kVec);
-        const int rem = it - g * kDim * kVec;
-        const int i = rem / kVec;
-        const int ch = rem - i * kVec;
-        const uint4 w = *reinterpret_cast<const uint4*>(
-            p.w_q + (static_cast<size_t>(h * G + g) * kDim + i) * kDim + rank * kDpc + ch * 8);
-        *reinterpret_cast<uint4*>(wq_s + (static_cast<size_t>(g) * kDim + i) * kDpc + ch * 8) = w;
-      }
-    }
-    __syncthreads();
-    cluster_wait();  // every CTA of the cluster is running
-    if (!bad) {
-      for (int o = tid; o < G * kDpc; o += kThreads) {
-        const int g = o / kDpc;
-        const int j = o - g * kDpc;
-        const float* qrow = qs + g * kDim;
-        const __nv_bfloat16* wcol = wq_s + static_cast<size_t>(g) * kDim * kDpc + j;
-        float acc = 0.f;
+  const bool pro_ok = mbar_wait(bar_pro, 0, p.status);
+  cluster_wait();  // every CTA of the cluster is running
+  if (MODE != kModeAttend && !bad && pro_ok) {
+    // two threads per output column (rows 0..63 and 64..127), combined by shuffle
+    for (int o = tid; o < 2 * G * kDpc; o += kThreads) {
+      const int half = o & 1;
+      const int oc = o >> 1;
+      const int g = oc / kDpc;
+      const int j = oc - g * kDpc;
+      const T* qrow = qraw + g * kDim + half * 64;
+      const __nv_bfloat16* wcol = wq_s + (static_cast<size_t>(g) * kDim + half * 64) * kDpc + j;
+      float acc = 0.f;
 #pragma unroll 16
-        for (int i = 0; i < kDim; ++i) acc = fmaf(qrow[i], __bfloat162float(wcol[i * kDpc]), acc);
+      for (int i = 0; i < 64; ++i)
+        acc = fmaf(to_float(qrow[i]), __bfloat162float(wcol[i * kDpc]), acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      if (half == 0) {
 #pragma unroll
         for (int r = 0; r < CS; ++r) cluster.map_shared_rank(qv, r)[g * kDim + rank * kDpc + j] = acc;
       }
     }
-  } else {
-    cluster_wait();
   }
   cluster.sync();  // #1: every CTA holds all of v
+  SAS_TRACE(2);
 
   if (MODE != kModeAttend) {
     if (!bad) {
       // Q normalisation (RMSNorm, gain gamma_q) and gate RoPE at position c.
+      float c0, s0, c1, s1;
+      rope_cos_sin(th0, c, c0, s0);
+      rope_cos_sin(th1, c, c1, s1);
       for (int g = warp; g < G; g += kWarps) {
         float x[4];
         float ss = 0.f;
@@ -367,10 +438,7 @@ __global__ void __launch_bounds__(kThreads, 4)
         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
         const float inv = 1.f / sqrtf(ss / kDim + p.eps);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) x[k] = x[k] * inv * p.gamma_q[lane + 32 * k];
-        float c0, s0, c1, s1;
-        rope_cos_sin(lane, c, p.rope_base, c0, s0);
-        rope_cos_sin(lane + 32, c, p.rope_base, c1, s1);
+        for (int k = 0; k < 4; ++k) x[k] = x[k] * inv * gam_s[lane + 32 * k];
         qv[g * kDim + lane] = x[0] * c0 - x[2] * s0;
         qv[g * kDim + lane + 64] = x[2] * c0 + x[0] * s0;
         qv[g * kDim + lane + 32] = x[1] * c1 - x[3] * s1;
@@ -422,6 +490,9 @@ __global__ void __launch_bounds__(kThreads, 4)
           acc += __shfl_xor_sync(0xffffffffu, acc, 2);
           acc += __shfl_xor_sync(0xffffffffu, acc, 4);
           S = acc;
+          // every CTA of the cluster receives every score (lane `sub` -> rank sub)
+          if (act)
+            for (int r = sub; r < CS; r += 8) cluster.map_shared_rank(keys, r)[b0 + bb] = S;
         } else {
           for (int g = 0; g < G; ++g) {
             float acc = 0.f;
@@ -444,31 +515,22 @@ __global__ void __launch_bounds__(kThreads, 4)
           }
           S = S / static_cast<float>(G);
         }
-        if (act && sub == 0) {
-          sslice[b0 - b_lo + bb] = S;
-          if (p.group_scores != nullptr)
-            p.group_scores[static_cast<size_t>(pair) * p.mg + b0 + bb] = S;
-        }
+        if (act && sub == 0 && p.group_scores != nullptr)
+          p.group_scores[static_cast<size_t>(pair) * p.mg + b0 + bb] = S;
       }
       __syncthreads();
       pump(ci + 1, known);
     }
   }
+  SAS_TRACE(3);
   if (MODE == kModeGate) return;  // no DSMEM access after barrier #1
 
   // ------------------------------------------------------------ phase 2: Top-K
   if (MODE == kModeFused) {
-    cluster.sync();  // #2: all score slices written
+    cluster.sync();  // #2: every score of the (seq, head) is in every CTA
+    SAS_TRACE(4);
     if (!bad) {
-      for (int b = tid; b < n; b += kThreads) {
-        const int r = b / nb_per;
-        sall[b] = cluster.map_shared_rank(sslice, r)[b - r * nb_per];
-      }
-    }
-    __syncthreads();
-    if (!bad) {
-      const int mm = select_blocks(sall, n, p.topk, c, sel, hist, scan);
-      (void)mm;  // == m by construction
+      select_blocks(keys, n, p.topk, c, sel, hist, selbits, scan);
       if (rank == 0) {
         if (p.sel_idx != nullptr)
           for (int j = tid; j < m; j += kThreads)
@@ -480,6 +542,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
     known = nchunks + kTilesPerBlock * cnt_mine;
     pump(nchunks, known);
+    SAS_TRACE(5);
   }
 
   // ------------------------------------------------------------ phase 3: attention
@@ -491,13 +554,11 @@ __global__ void __launch_bounds__(kThreads, 4)
   if constexpr (!kF32) {
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) o_acc[nt][0] = o_acc[nt][1] = 0.f;
-    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) +
-                                (static_cast<size_t>(s) * p.hq + h * G + min(gq, G - 1)) * kDim;
+    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(qraw) + min(gq, G - 1) * kDim;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      qa0[ks] = (gq < G && !bad) ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq) : 0u;
-      qa2[ks] =
-          (gq < G && !bad) ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * tq) : 0u;
+      qa0[ks] = (gq < G) ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq) : 0u;
+      qa2[ks] = (gq < G) ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * tq) : 0u;
     }
   } else {
 #pragma unroll
@@ -506,12 +567,6 @@ __global__ void __launch_bounds__(kThreads, 4)
       fl[g] = 0.f;
       fo[g][0] = fo[g][1] = fo[g][2] = fo[g][3] = 0.f;
     }
-    if (!bad) {
-      const float* qg = static_cast<const float*>(p.q) +
-                        (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim;
-      for (int i = tid; i < G * kDim; i += kThreads) qatt[i] = qg[i];
-    }
-    __syncthreads();
   }
   const float sl2 = p.attn_scale_log2;
 
@@ -607,6 +662,7 @@ __global__ void __launch_bounds__(kThreads, 4)
       pump(t1 + 1, known);
     } else {
       // ---- fp32 K/V: SIMT path (small parity configurations)
+      const float* qatt = reinterpret_cast<const float*>(qraw);
       const int half = warp >> 1;  // tokens 0..31 in tile t0 (t0+2 for V), 32..63 in t0+1
       const int tK = t0 + half;
       bool ok = mbar_wait(&bars[t0 % NST], (t0 / NST) & 1, p.status);
@@ -617,8 +673,8 @@ __global__ void __launch_bounds__(kThreads, 4)
 #pragma unroll
       for (int g = 0; g < kMaxGroup; ++g) lg[g] = 0.f;
       if (ok) {
-        const float* krow =
-            reinterpret_cast<const float*>(slots + (tK % NST) * kTileBytes) + (tl & 31) * kDim + hh * 64;
+        const float* krow = reinterpret_cast<const float*>(slots + (tK % NST) * kTileBytes) +
+                            (tl & 31) * kDim + hh * 64;
         for (int i = 0; i < 64; ++i) {
           const int d = (i + tt) & 63;
           const float kv = krow[d];
@@ -683,7 +739,9 @@ __global__ void __launch_bounds__(kThreads, 4)
       pump(t0 + 4, known);
     }
   }
+  SAS_TRACE(6);
 
+  // ------------------------------------------------------------ phase 4: merge
   // per-warp partials (the stage slots are free: every issued tile was consumed)
   if constexpr (!kF32) {
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
@@ -711,45 +769,64 @@ __global__ void __launch_bounds__(kThreads, 4)
       }
     }
   }
-
-  // ------------------------------------------------------------ phase 4: merge
-  cluster.sync();  // #3: all partials written
+  __syncthreads();
+  // fold the 4 warps; thread d owns column d of every head and sends it to
+  // the CTA that writes that column
+  {
+    const int d = tid;
+    const int dst = d / kDpc;
+    const int dd = d - dst * kDpc;
+    float* rin_o = cluster.map_shared_rank(inbox_o, dst);
+    float* rin_ml = cluster.map_shared_rank(inbox_ml, dst);
+    for (int g = 0; g < G; ++g) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, pm[w * kMaxGroup + g]);
+      float lsum = 0.f, osum = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+          const float f = exp2f(pm[w * kMaxGroup + g] - M);
+          lsum = fmaf(pl[w * kMaxGroup + g], f, lsum);
+          osum = fmaf(po[(static_cast<size_t>(w) * G + g) * kDim + d], f, osum);
+        }
+      }
+      rin_o[(rank * G + g) * kDpc + dd] = osum;
+      if (dd == 0) {
+        rin_ml[(rank * G + g) * 2 + 0] = M;
+        rin_ml[(rank * G + g) * 2 + 1] = lsum;
+      }
+    }
+  }
+  cluster.sync();  // #3: every partial of this CTA's columns has arrived
+  SAS_TRACE(7);
   {
     OutT* out = static_cast<OutT*>(p.out);
     for (int it = tid; it < G * kDpc; it += kThreads) {
       const int g = it / kDpc;
-      const int d = rank * kDpc + (it - g * kDpc);
+      const int dd = it - g * kDpc;
       float res = 0.f;
       if (!bad) {
         float M = -INFINITY;
 #pragma unroll
-        for (int r = 0; r < CS; ++r) {
-          const float* rpm = cluster.map_shared_rank(pm, r);
-#pragma unroll
-          for (int w = 0; w < kWarps; ++w) M = fmaxf(M, rpm[w * kMaxGroup + g]);
-        }
+        for (int r = 0; r < CS; ++r) M = fmaxf(M, inbox_ml[(r * G + g) * 2]);
         float den = 0.f, num = 0.f;
 #pragma unroll
         for (int r = 0; r < CS; ++r) {
-          const float* rpm = cluster.map_shared_rank(pm, r);
-          const float* rpl = cluster.map_shared_rank(pl, r);
-          const float* rpo = cluster.map_shared_rank(po, r);
-#pragma unroll
-          for (int w = 0; w < kWarps; ++w) {
-            const float mw = rpm[w * kMaxGroup + g];
-            if (mw != -INFINITY) {
-              const float f = exp2f(mw - M);
-              den = fmaf(rpl[w * kMaxGroup + g], f, den);
-              num = fmaf(rpo[(static_cast<size_t>(w) * G + g) * kDim + d], f, num);
-            }
+          const float mr = inbox_ml[(r * G + g) * 2];
+          if (mr != -INFINITY) {
+            const float f = exp2f(mr - M);
+            den = fmaf(inbox_ml[(r * G + g) * 2 + 1], f, den);
+            num = fmaf(inbox_o[(r * G + g) * kDpc + dd], f, num);
           }
         }
         res = num / den;
       }
-      out[(static_cast<size_t>(s) * p.hq + h * G + g) * kDim + d] = from_float<OutT>(res);
+      out[(static_cast<size_t>(s) * p.hq + h * G + g) * kDim + rank * kDpc + dd] =
+          from_float<OutT>(res);
     }
   }
-  cluster.sync();  // #4: no CTA leaves while its partials may still be read
+  SAS_TRACE(8);
 }
 
 // ------------------------------------------------------------ Top-K kernel
@@ -757,12 +834,16 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
   const int pair = blockIdx.x;
   const int s = pair / p.hkv;
   const int tid = threadIdx.x;
-  extern __shared__ uint8_t smem_raw[];
-  float* sall = reinterpret_cast<float*>(smem_raw);
-  int* sel = reinterpret_cast<int*>(smem_raw + (p.mg * 4 + 15) / 16 * 16);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(sel) +
-                                               (p.max_sel * 4 + 15) / 16 * 16);
-  int* scan = reinterpret_cast<int*>(hist + 512);
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  float* vals = reinterpret_cast<float*>(smem_raw);
+  uint8_t* q = smem_raw + (p.mg * 4 + 15) / 16 * 16;
+  int* sel = reinterpret_cast<int*>(q);
+  q += (p.max_sel * 4 + 15) / 16 * 16;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(q);
+  q += kSelBins * 4;
+  uint32_t* selbits = reinterpret_cast<uint32_t*>(q);
+  q += ((p.mg + 31) / 32 * 4 + 15) / 16 * 16;
+  int* scan = reinterpret_cast<int*>(q);
   const int L = p.seq_lens[s];
   if (L < 1 || (L - 1) / kBlock > p.mg) {
     if (tid == 0) {
@@ -772,15 +853,16 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
     return;
   }
   const int c = (L - 1) / kBlock;
-  for (int b = tid; b < c; b += kThreads) sall[b] = p.group_scores[static_cast<size_t>(pair) * p.mg + b];
+  for (int b = tid; b < c; b += kThreads) vals[b] = p.group_scores[static_cast<size_t>(pair) * p.mg + b];
   __syncthreads();
-  const int m = select_blocks(sall, c, p.topk, c, sel, hist, scan);
+  const int m = select_blocks(vals, c, p.topk, c, sel, hist, selbits, scan);
   for (int j = tid; j < m; j += kThreads) p.sel_idx[static_cast<size_t>(pair) * p.max_sel + j] = sel[j];
   if (tid == 0) p.sel_count[pair] = m;
 }
 
 size_t topk_smem_bytes(int mg, int max_sel) {
-  return static_cast<size_t>((mg * 4 + 15) / 16 * 16 + (max_sel * 4 + 15) / 16 * 16 + 512 * 4 + 16 * 4);
+  return static_cast<size_t>((mg * 4 + 15) / 16 * 16 + (max_sel * 4 + 15) / 16 * 16 + kSelBins * 4 +
+                             ((mg + 31) / 32 * 4 + 15) / 16 * 16 + 16 * 4);
 }
 
 // ------------------------------------------------------------ launchers
@@ -788,7 +870,7 @@ namespace {
 
 template <typename T, typename OutT, int CS, int NST, int MODE>
 cudaError_t launch_cluster(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                           int batch, cudaStream_t stream) {
+                           const CUtensorMap& tmw, int batch, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CS, static_cast<unsigned>(batch * p.hkv), 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -801,7 +883,7 @@ cudaError_t launch_cluster(const DecodeParams& p, const CUtensorMap& tmk, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_cluster_kernel<T, OutT, CS, NST, MODE>, p, tmk, tmv);
+  return cudaLaunchKernelEx(&cfg, decode_cluster_kernel<T, OutT, CS, NST, MODE>, p, tmk, tmv, tmw);
 }
 
 template <typename T, typename OutT, int CS, int NST, int MODE>
@@ -815,14 +897,14 @@ cudaError_t set_attrs() {
 
 template <int MODE>
 cudaError_t dispatch_types(bool f32_kv, bool f32_out, int cs, int nst, const DecodeParams& p,
-                           const CUtensorMap& tmk, const CUtensorMap& tmv, int batch,
-                           cudaStream_t st) {
+                           const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap& tmw,
+                           int batch, cudaStream_t st) {
   using bf = __nv_bfloat16;
   if (cs != 8 || nst != 2) return cudaErrorInvalidValue;
-  if (!f32_kv && !f32_out) return launch_cluster<bf, bf, 8, 2, MODE>(p, tmk, tmv, batch, st);
-  if (!f32_kv && f32_out) return launch_cluster<bf, float, 8, 2, MODE>(p, tmk, tmv, batch, st);
-  if (f32_kv && !f32_out) return launch_cluster<float, bf, 8, 2, MODE>(p, tmk, tmv, batch, st);
-  return launch_cluster<float, float, 8, 2, MODE>(p, tmk, tmv, batch, st);
+  if (!f32_kv && !f32_out) return launch_cluster<bf, bf, 8, 2, MODE>(p, tmk, tmv, tmw, batch, st);
+  if (!f32_kv && f32_out) return launch_cluster<bf, float, 8, 2, MODE>(p, tmk, tmv, tmw, batch, st);
+  if (f32_kv && !f32_out) return launch_cluster<float, bf, 8, 2, MODE>(p, tmk, tmv, tmw, batch, st);
+  return launch_cluster<float, float, 8, 2, MODE>(p, tmk, tmv, tmw, batch, st);
 }
 
 template <int MODE>
@@ -839,14 +921,14 @@ cudaError_t attrs_for_mode() {
 
 cudaError_t launch_decode(int mode, bool f32_kv, bool f32_out, int cs, int nst,
                           const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                          int batch, cudaStream_t stream) {
+                          const CUtensorMap& tmw, int batch, cudaStream_t stream) {
   switch (mode) {
     case kModeGate:
-      return dispatch_types<kModeGate>(f32_kv, false, cs, nst, p, tmk, tmv, batch, stream);
+      return dispatch_types<kModeGate>(f32_kv, false, cs, nst, p, tmk, tmv, tmw, batch, stream);
     case kModeAttend:
-      return dispatch_types<kModeAttend>(f32_kv, f32_out, cs, nst, p, tmk, tmv, batch, stream);
+      return dispatch_types<kModeAttend>(f32_kv, f32_out, cs, nst, p, tmk, tmv, tmw, batch, stream);
     default:
-      return dispatch_types<kModeFused>(f32_kv, f32_out, cs, nst, p, tmk, tmv, batch, stream);
+      return dispatch_types<kModeFused>(f32_kv, f32_out, cs, nst, p, tmk, tmv, tmw, batch, stream);
   }
 }
 

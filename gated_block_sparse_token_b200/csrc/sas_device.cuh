@@ -189,15 +189,20 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Gate RoPE factors for pair index i (0..63) at integer position pos:
-// angle = pos * base^(-2i/128), evaluated in double precision.
-__device__ __forceinline__ void rope_cos_sin(int i, int pos, float base, float& c, float& s) {
-  const double theta = pow(static_cast<double>(base), -2.0 * i / static_cast<double>(kDim));
-  double sd, cd;
-  sincos(static_cast<double>(pos) * theta, &sd, &cd);
-  c = static_cast<float>(cd);
-  s = static_cast<float>(sd);
+// Gate RoPE factors at integer position pos for a pair whose frequency is
+// theta = base^(-2i/128), given as theta_over_pi = theta / pi (double, from the
+// host).  The angle is pos * theta; with a = pos * theta / pi, a - 2*floor(a/2)
+// is exact in double, so sincospif sees a reduced argument in [0, 2).
+__device__ __forceinline__ void rope_cos_sin(double theta_over_pi, int pos, float& c, float& s) {
+  const double a = static_cast<double>(pos) * theta_over_pi;
+  const double r = a - 2.0 * floor(0.5 * a);
+  sincospif(static_cast<float>(r), &s, &c);
 }
+
+// Frequencies of the 64 rotate-half pairs, divided by pi (host-computed).
+struct RopeTable {
+  double theta_over_pi[64];
+};
 
 // KV cache addressing: row (in the [rows][128] view of K or V) of the first
 // token of block b of (sequence s, KV head h); -1 if the block lies outside

@@ -15,24 +15,31 @@ namespace sas {
 enum DecodeMode : int { kModeGate = 0, kModeAttend = 1, kModeFused = 2 };
 
 // Byte offsets (from a 1024-byte aligned base) of the shared-memory regions
-// of the cluster decode kernel.  `u_*` regions share one union: the gate
-// weights slice and raw query are dead before the selection arrays are used.
+// of the cluster decode kernel.  Region R is reused across phases:
+//   phases 0-1  [ qv | wq | qs ]
+//   phases 2-4  [ inbox | keys | hist | selbits | scan ]
+// inbox (written by other CTAs after the attention phase) covers at least
+// qv, and keys (written by other CTAs during their phase 1) starts past the
+// inbox, so no remote write can land on data this CTA still reads.
+constexpr int kSelBins = 1024;  // value buckets of the Top-K selection
+constexpr int kSelCand = 256;   // candidates ranked exactly in the boundary bucket
+
 struct DecodeSmem {
-  int slots;   // NST stage slots of 16 KiB (gate-key chunks, then K/V tiles)
-  int sslice;  // fp32 [slice_cap]  this CTA's share of the group scores
-  int u_wq;    // bf16 [G][128][dpc] W_q column slice          (phase 0)
-  int u_qs;    // fp32 [G][128] query staged for the gate GEMV (phase 0)
-  int u_sall;  // fp32 [mg] all group scores of the (seq, head) (phase 2)
-  int u_sel;   // int32 [max_sel] selected blocks             (phase 2, 3)
-  int u_hist;  // uint32 [2][256] radix histograms            (phase 2)
-  int u_scan;  // int32 [16] scan scratch
-  int qv;      // fp32 [G][128] gate query v, then q~ in place
-  int qbar;    // fp32 [128] group-mean gate query (fused mode)
-  int qatt;    // fp32 [G][128] attention query (fp32 K/V only)
-  int pml;     // fp32 m[4][8], l[4][8] per-warp softmax state
-  int bars;    // uint64 [NST] mbarriers
-  int total;   // bytes to request, including alignment slack
-  int slice_cap;
+  int slots;     // NST stage slots of 16 KiB (gate-key chunks, then K/V tiles)
+  int sel;       // int32 [max_sel] selected blocks (phases 2-3)
+  int qraw;      // T [G][128] query as stored (bf16 or fp32), bulk copy
+  int qbar;      // fp32 [128] group-mean gate query (fused mode)
+  int pml;       // fp32 m[4][8], l[4][8] per-warp softmax state
+  int bars;      // uint64 [NST] mbarriers
+  int r_qv;      // fp32 [G][128] gate query v, then q~ in place   (phases 0-1)
+  int r_wq;      // bf16 [G][128][dpc] W_q column slice (TMA)       (phase 0)
+  int gam;       // fp32 [128] gamma_q (bulk copy)
+  int r_inbox;   // fp32 [CS][G][dpc] o, then [CS][G][2] (m, l)     (phases 3-4)
+  int r_keys;    // fp32 scores -> uint32 keys [mg]                 (phases 1-2)
+  int r_hist;    // uint32 [kSelBins], then int32 candidates        (phase 2)
+  int r_selbits; // uint32 [(mg + 31) / 32]                         (phase 2)
+  int r_scan;    // int32 [16]                                      (phase 2)
+  int total;     // bytes to request, including alignment slack
 };
 
 inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, bool f32_kv) {
@@ -44,37 +51,43 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
     off += bytes;
     return o;
   };
+  auto up16 = [](int x) { return (x + 15) / 16 * 16; };
   const int dpc = kDim / cs;
-  p.slice_cap = (std::max(mg, 1) + cs - 1) / cs;
+  mg = std::max(mg, 1);
   p.slots = take(nst * kTileBytes, 1024);
-  p.sslice = take(p.slice_cap * 4, 16);
-  // union region
-  const int ustart = (off + 15) / 16 * 16;
-  const int wq_bytes = G * kDim * dpc * 2;
-  const int qs_bytes = G * kDim * 4;
-  p.u_wq = ustart;
-  p.u_qs = ustart + wq_bytes;
-  const int part_a = wq_bytes + qs_bytes;
-  int o2 = ustart;
-  p.u_sall = o2;
-  o2 += (std::max(mg, 1) * 4 + 15) / 16 * 16;
-  p.u_sel = o2;
-  o2 += (max_sel * 4 + 15) / 16 * 16;
-  p.u_hist = o2;
-  o2 += 512 * 4;
-  p.u_scan = o2;
-  o2 += 16 * 4;
-  off = ustart + std::max(part_a, o2 - ustart);
-  p.qv = take(G * kDim * 4, 16);
+  p.sel = take(max_sel * 4, 16);
+  p.qraw = take(G * kDim * (f32_kv ? 4 : 2), 16);
   p.qbar = take(kDim * 4, 16);
-  p.qatt = f32_kv ? take(G * kDim * 4, 16) : 0;
   p.pml = take(2 * kWarps * kMaxGroup * 4, 16);
-  p.bars = take(nst * 8, 8);
-  p.total = off + 1024;
+  p.gam = take(kDim * 4, 16);
+  p.bars = take((nst + 1) * 8, 8);  // ring slots + the prologue barrier
+  auto up128 = [](int x) { return (x + 127) / 128 * 128; };
+  const int r = up128(off);
+  // phases 0-1 (the W_q slice is a tensor-TMA destination: 128-byte aligned)
+  p.r_qv = r;
+  p.r_wq = up128(r + G * kDim * 4);
+  const int end01 = p.r_wq + up16(G * kDim * dpc * 2);
+  // phases 2-4
+  p.r_inbox = r;
+  p.r_keys = r + up16(cs * G * (dpc + 2) * 4);
+  p.r_hist = p.r_keys + up16(mg * 4);
+  p.r_selbits = p.r_hist + up16(std::max(kSelBins, kSelCand) * 4);
+  p.r_scan = p.r_selbits + up16((mg + 31) / 32 * 4);
+  const int end24 = p.r_scan + 16 * 4;
+  p.total = std::max(end01, end24) + 1024;
   return p;
 }
 
+// TMA destinations of the plan: tensor boxes need 128-byte (swizzled: 1024-
+// byte) aligned shared addresses, bulk copies 16-byte ones.
+inline bool decode_smem_aligned(const DecodeSmem& p, int G, int dpc) {
+  return p.slots % 1024 == 0 && p.r_wq % 128 == 0 && (G * kDim * dpc * 2) % 128 == 0 &&
+         p.qraw % 16 == 0 && p.gam % 16 == 0 && p.bars % 8 == 0;
+}
+
 struct DecodeParams {
+  RopeTable rope;
+  unsigned long long* trace;  // phase timestamps (tracing builds only), else null
   int hq, hkv, G;
   int topk;     // historical blocks kept: budget/64 - 1
   int max_sel;  // budget/64
@@ -104,6 +117,7 @@ struct TopkParams {
 };
 
 struct PoolParams {
+  RopeTable rope;
   int hkv, mg, num_blocks;
   float rope_base, eps;
   KvView kv;
@@ -116,15 +130,22 @@ struct PoolParams {
 };
 
 constexpr int kPoolBlocksPerCta = 8;
+constexpr int kPoolWkBytes = kPool * kDim * 2;  // W_k of one KV head, bf16 (96 KiB)
+
+// Phase-trace builds (-DSAS_PHASE_TRACE) record per-CTA timestamps after the
+// status word; ordinary builds compile the hooks out.
+constexpr int kTraceSlots = 16;
+constexpr int kTraceCtas = 4096;
 
 // Launchers (return the cudaError_t of the launch).
 cudaError_t launch_decode(int mode, bool f32_kv, bool f32_out, int cs, int nst,
                           const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                          int batch, cudaStream_t stream);
+                          const CUtensorMap& tmw, int batch, cudaStream_t stream);
 cudaError_t launch_topk(const TopkParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_pool(bool f32_kv, const PoolParams& p, int batch, cudaStream_t stream);
 size_t topk_smem_bytes(int mg, int max_sel);
 size_t pool_smem_bytes();
+void fill_rope_table(RopeTable& t, float base);
 
 // One-time per-process set-up of kernel attributes.
 cudaError_t prepare_kernels();

@@ -16,7 +16,8 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsas.so")
+# SAS_LIBRARY selects another build of the same ABI (e.g. the phase-trace build).
+LIB_PATH = os.environ.get("SAS_LIBRARY", os.path.join(_HERE, "libsas.so"))
 
 SAS_OK = 0
 SAS_ERR_INVALID_ARG = 1

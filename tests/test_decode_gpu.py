@@ -175,11 +175,13 @@ def test_topk_exact_with_ties(budget):
     included (scores drawn from a handful of values)."""
     g = torch.Generator().manual_seed(budget)
     B, hkv, mg = 3, 4, 2048
-    lens = torch.tensor([1, 2000, 131072 // 64], dtype=torch.int32)
     lens = torch.tensor([1, 2000, 64 * 2047 + 5], dtype=torch.int32)
     scores = (torch.randint(-4, 5, (B, hkv, mg), generator=g).float() * 0.25)
     scores[1, 1] += torch.randn(mg, generator=g) * 1e-3
     scores[2, 3] = torch.randn(mg, generator=g)
+    scores[2, 0] = 0.5                      # all equal: index order decides
+    scores[2, 1, 100:300] = float("-inf")   # extreme values next to ordinary ones
+    scores[2, 2, 7] = 3.0e38
     cfg = sas.Config(4 * hkv, hkv, token_budget=budget)
     ws = sas.make_workspace(cfg, DEV)
     sel = torch.full((B, hkv, budget // 64), -1, dtype=torch.int32, device=DEV)

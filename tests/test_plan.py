@@ -1,0 +1,63 @@
+"""Host-side checks of the decode kernel's shared-memory plan (no GPU): every
+TMA destination is aligned as the copy requires, regions that are live at the
+same time do not overlap, and the remote writes of other CTAs (scores during
+their phase 1, merge partials after their attention phase) never land on a
+region this CTA may still be reading."""
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "gated_block_sparse_token_b200", "csrc")
+
+
+@pytest.fixture(scope="module")
+def plans():
+    with tempfile.TemporaryDirectory() as d:
+        exe = os.path.join(d, "plan_check")
+        subprocess.run(["/usr/local/cuda/bin/nvcc", "-std=c++17", "-I", CSRC, "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "native", "plan_check.cu"), "-o", exe], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    rows = []
+    for line in out.splitlines():
+        rows.append({k: int(v) for k, v in (f.split("=") for f in line.split())})
+    return rows
+
+
+def test_plan_alignment_and_overlap(plans):
+    CS, dpc = 8, 16
+    assert len(plans) == 8 * 8 * 5 * 2
+    for p in plans:
+        G, mg, ms = p["G"], max(p["mg"], 1), p["budget"] // 64
+        tag = str(p)
+        assert p["ok"] == 1, tag
+        assert p["slots"] % 1024 == 0 and p["r_wq"] % 128 == 0, tag
+        assert p["qraw"] % 16 == 0 and p["gam"] % 16 == 0 and p["bars"] % 8 == 0, tag
+        # fixed regions, in order, disjoint
+        fixed = [("slots", 2 * 16384), ("sel", 4 * ms), ("qraw", G * 128 * (4 if p["f32"] else 2)),
+                 ("qbar", 512), ("pml", 256), ("gam", 512), ("bars", 24)]
+        for (a, sa), (b, _) in zip(fixed, fixed[1:]):
+            assert p[a] + sa <= p[b], (tag, a, b)
+        r = p["r_qv"]
+        assert p["bars"] + 24 <= r, tag
+        # phase 0-1 layout: qv then the W_q slice
+        qv_end = r + G * 128 * 4
+        assert qv_end <= p["r_wq"], tag
+        # phase 2-4 layout: inbox first, covering qv entirely
+        inbox_end = p["r_inbox"] + CS * G * (dpc + 2) * 4
+        assert p["r_inbox"] == r and inbox_end >= qv_end, tag
+        # scores pushed by other CTAs during their phase 1 must not touch qv
+        assert p["r_keys"] >= inbox_end and p["r_keys"] >= qv_end, tag
+        assert p["r_hist"] >= p["r_keys"] + 4 * mg, tag
+        assert p["r_selbits"] >= p["r_hist"] + 4 * 1024, tag
+        assert p["r_scan"] >= p["r_selbits"] + 4 * ((mg + 31) // 32), tag
+        end = max(p["r_wq"] + G * 128 * dpc * 2, p["r_scan"] + 64)
+        assert p["total"] >= end + 1024, tag
+
+
+def test_plan_fits_four_ctas_per_sm_at_the_benchmark_shape(plans):
+    # Qwen3-4B, 32k context: G = 4, 512 gate-key rows, budget 2,048, bf16
+    p = next(q for q in plans if q["G"] == 4 and q["mg"] == 512 and q["budget"] == 2048 and q["f32"] == 0)
+    assert 4 * (p["total"] + 1024) <= 228 * 1024
