@@ -19,7 +19,7 @@ namespace {
 
 using sas::kDim;
 
-constexpr int32_t kAbiVersion = 1;
+constexpr int32_t kAbiVersion = 2;
 constexpr size_t kStatusBytes = 256;  // status word + padding
 constexpr int kMaxBudget = 16384;
 constexpr int kMaxGateBlocks = 16384;
@@ -137,6 +137,22 @@ bool encode_wq_map(CUtensorMap* m, const void* w_q, int hq) {
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(kDim / kClusterSize), static_cast<cuuint32_t>(kDim)};
   const cuuint32_t estride[2] = {1, 1};
   const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w_q), gdim,
+                              gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 2-D view [Hkv*384][128] of bf16 W_k; one box = 128 rows x the 128/CS
+// columns a cluster CTA projects.
+bool encode_wk_map(CUtensorMap* m, const void* w_k, int hkv) {
+  memset(m, 0, sizeof(*m));
+  if (g_encode == nullptr) return false;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(hkv) * sas::kPool};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(kDim * 2)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kDim / kClusterSize), 128};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w_k), gdim,
                               gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -310,7 +326,7 @@ sas_status sas_gate_scores(const sas_config* cfg, const void* q, const int32_t* 
   memset(&dummy, 0, sizeof(dummy));
   if (!encode_wq_map(&tmw, w_q, cfg->num_q_heads)) return SAS_ERR_CUDA;
   return launch_result(sas::launch_decode(sas::kModeGate, cfg->kv_dtype == SAS_DTYPE_F32, false,
-                                          kClusterSize, kStages, p, dummy, dummy, tmw, batch,
+                                          kClusterSize, kStages, p, dummy, dummy, tmw, dummy, batch,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -343,10 +359,11 @@ sas_status sas_topk_blocks(const sas_config* cfg, const float* group_scores,
 }
 
 static sas_status attention_call(int mode, const sas_config* cfg, const void* q, const sas_kv* kv,
-                                 const void* w_q, const float* gamma_q, const float* gate_keys,
-                                 int32_t max_gate_blocks, void* out, int32_t* sel_idx,
-                                 int32_t* sel_count, float* group_scores, void* ws,
-                                 size_t ws_bytes, sas_stream_t stream) {
+                                 const void* w_q, const float* gamma_q, const void* w_k,
+                                 const float* gamma_k, float* gate_keys, int32_t max_gate_blocks,
+                                 void* out, int32_t* sel_idx, int32_t* sel_count,
+                                 float* group_scores, void* ws, size_t ws_bytes,
+                                 sas_stream_t stream) {
   sas_status st = check_config(cfg);
   if (st != SAS_OK) return st;
   if ((st = check_kv(cfg, kv)) != SAS_OK) return st;
@@ -357,6 +374,8 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
     if (max_gate_blocks < 1 || max_gate_blocks > kMaxGateBlocks) return SAS_ERR_INVALID_ARG;
     if (w_q == nullptr || gamma_q == nullptr || gate_keys == nullptr) return SAS_ERR_INVALID_ARG;
     if (!aligned(w_q, 16) || !aligned(gamma_q, 16) || !aligned(gate_keys, 16)) return SAS_ERR_INVALID_ARG;
+    if ((w_k == nullptr) != (gamma_k == nullptr)) return SAS_ERR_INVALID_ARG;
+    if (w_k != nullptr && (!aligned(w_k, 16) || !aligned(gamma_k, 16))) return SAS_ERR_INVALID_ARG;
     if ((sel_idx != nullptr && !aligned(sel_idx, 4)) || (sel_count != nullptr && !aligned(sel_count, 4)) ||
         (group_scores != nullptr && !aligned(group_scores, 4)))
       return SAS_ERR_INVALID_ARG;
@@ -374,6 +393,8 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
   p.w_q = static_cast<const __nv_bfloat16*>(w_q);
   p.gamma_q = gamma_q;
   p.gate_keys = gate_keys;
+  p.gamma_k = (mode == sas::kModeFused) ? gamma_k : nullptr;
+  p.gate_keys_out = gate_keys;
   p.kv = make_view(cfg, kv);
   p.group_scores = group_scores;
   p.sel_idx = sel_idx;
@@ -382,34 +403,38 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
   p.status = static_cast<uint32_t*>(ws);
   p.trace = trace_region(ws);
   const bool f32_kv = cfg->kv_dtype == SAS_DTYPE_F32;
-  CUtensorMap tmk, tmv, tmw;
+  CUtensorMap tmk, tmv, tmw, tmwk;
   memset(&tmk, 0, sizeof(tmk));
   memset(&tmv, 0, sizeof(tmv));
   memset(&tmw, 0, sizeof(tmw));
+  memset(&tmwk, 0, sizeof(tmwk));
   if (!f32_kv) {
     const long long rows = kv_rows(cfg, kv);
     if (!encode_kv_map(&tmk, kv->k, rows) || !encode_kv_map(&tmv, kv->v, rows)) return SAS_ERR_CUDA;
   }
   if (mode == sas::kModeFused && !encode_wq_map(&tmw, w_q, cfg->num_q_heads)) return SAS_ERR_CUDA;
+  if (p.gamma_k != nullptr && !encode_wk_map(&tmwk, w_k, cfg->num_kv_heads)) return SAS_ERR_CUDA;
   return launch_result(sas::launch_decode(mode, f32_kv, cfg->out_dtype == SAS_DTYPE_F32,
-                                          kClusterSize, kStages, p, tmk, tmv, tmw, kv->batch,
+                                          kClusterSize, kStages, p, tmk, tmv, tmw, tmwk, kv->batch,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const sas_kv* kv,
                              const int32_t* sel_idx, const int32_t* sel_count, void* out,
                              void* ws, size_t ws_bytes, sas_stream_t stream) {
-  return attention_call(sas::kModeAttend, cfg, q, kv, nullptr, nullptr, nullptr, 0, out,
-                        const_cast<int32_t*>(sel_idx), const_cast<int32_t*>(sel_count), nullptr,
-                        ws, ws_bytes, stream);
+  return attention_call(sas::kModeAttend, cfg, q, kv, nullptr, nullptr, nullptr, nullptr, nullptr,
+                        0, out, const_cast<int32_t*>(sel_idx), const_cast<int32_t*>(sel_count),
+                        nullptr, ws, ws_bytes, stream);
 }
 
 sas_status sas_decode_step(const sas_config* cfg, const void* q, const sas_kv* kv, const void* w_q,
-                           const float* gamma_q, const float* gate_keys, int32_t max_gate_blocks,
-                           void* out, int32_t* sel_idx, int32_t* sel_count, float* group_scores,
-                           void* ws, size_t ws_bytes, sas_stream_t stream) {
-  return attention_call(sas::kModeFused, cfg, q, kv, w_q, gamma_q, gate_keys, max_gate_blocks, out,
-                        sel_idx, sel_count, group_scores, ws, ws_bytes, stream);
+                           const float* gamma_q, const void* w_k, const float* gamma_k,
+                           float* gate_keys, int32_t max_gate_blocks, void* out,
+                           int32_t* sel_idx, int32_t* sel_count, float* group_scores, void* ws,
+                           size_t ws_bytes, sas_stream_t stream) {
+  return attention_call(sas::kModeFused, cfg, q, kv, w_q, gamma_q, w_k, gamma_k, gate_keys,
+                        max_gate_blocks, out, sel_idx, sel_count, group_scores, ws, ws_bytes,
+                        stream);
 }
 
 }  // extern "C"

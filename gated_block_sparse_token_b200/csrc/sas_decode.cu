@@ -84,15 +84,22 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scan) {
 // Keeps the min(topk, n) largest of vals[0..n) -- ties go to the lower index
 // -- lists them ascending in sel[], appends the current block `cur` and
 // returns the count.  Exact: scores map to order-preserving 32-bit keys,
-// which are spread over kSelBins buckets by a monotone map (the leading 10
-// bits of key - min key); the
-// bucket holding the topk-th key is found from the histogram, everything
-// above it is kept, and inside it the members are ranked exactly by
-// (key descending, index ascending).  Called by all kThreads threads;
-// overwrites vals with the keys.
+// which fall into kSelBins buckets by a monotone map (the leading 10 bits of
+// key - min key); the bucket holding the topk-th key is found from the
+// histogram, every bucket above it is kept, and the members of that bucket
+// are ranked exactly by (key descending, index ascending).  One warp does the
+// work with ballots and warp reductions (no CTA barrier inside); all threads
+// of the CTA call it and meet at the final barrier.  Overwrites vals with keys.
 __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
-                             uint32_t* selbits, int* scan) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+                             uint32_t* selbits, int* scan, unsigned long long* tr = nullptr) {
+#ifdef SAS_PHASE_TRACE
+#define SEL_TRACE(k, v) \
+  if (tr != nullptr && threadIdx.x == 0) tr[k] = (v)
+#else
+#define SEL_TRACE(k, v)
+#endif
+  (void)scan;
+  const int tid = threadIdx.x, lane = tid & 31;
   if (topk <= 0) {  // a 64-token budget keeps the current block only
     if (tid == 0) sel[0] = cur;
     __syncthreads();
@@ -104,120 +111,114 @@ __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, ui
     __syncthreads();
     return n + 1;
   }
-  uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-  for (int i = tid; i < n; i += kThreads) {
-    const uint32_t k = order_key(vals[i]);
-    keys[i] = k;
-    lo = min(lo, k);
-    hi = max(hi, k);
-  }
-  for (int i = tid; i < kSelBins; i += kThreads) hist[i] = 0u;
-  for (int i = tid; i < (n + 31) / 32; i += kThreads) selbits[i] = 0u;
+  if (tid < 32) {
+    const unsigned full = 0xffffffffu;
+    const unsigned lt = (1u << lane) - 1u;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (int i = lane; i < n; i += 32) {
+      const uint32_t k = order_key(vals[i]);
+      keys[i] = k;
+      lo = min(lo, k);
+      hi = max(hi, k);
+    }
+    for (int i = lane; i < kSelBins; i += 32) hist[i] = 0u;
+    for (int i = lane; i < (n + 31) / 32; i += 32) selbits[i] = 0u;
+    lo = __reduce_min_sync(full, lo);
+    hi = __reduce_max_sync(full, hi);
+    const int shift = max(0, 32 - __clz(static_cast<int>((hi - lo) | 1u)) - 10);
+    __syncwarp();
+    SEL_TRACE(0, global_timer_ns());
+    for (int i = lane; i < n; i += 32) atomicAdd(&hist[(keys[i] - lo) >> shift], 1u);
+    __syncwarp();
+    SEL_TRACE(1, global_timer_ns());
+    // buckets in descending order, 32 groups of 32: lane g sums group g
+    uint32_t gsum = 0u;
+    for (int g = 0; g < kSelBins / 32; ++g) {
+      const uint32_t v = __reduce_add_sync(full, hist[kSelBins - 1 - 32 * g - lane]);
+      if (lane == g) gsum = v;
+    }
+    uint32_t ginc = gsum;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-  }
-  if (lane == 0) {
-    scan[warp] = static_cast<int>(lo);
-    scan[4 + warp] = static_cast<int>(hi);
-  }
-  if (tid == 0) scan[10] = 0;
-  __syncthreads();
-  lo = static_cast<uint32_t>(scan[0]);
-  hi = static_cast<uint32_t>(scan[4]);
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(full, ginc, o);
+      if (lane >= o) ginc += y;
+    }
+    const uint32_t want = static_cast<uint32_t>(topk);
+    const unsigned hitg = __ballot_sync(full, ginc - gsum < want && want <= ginc);
+    const int gstar = __ffs(hitg) - 1;
+    const uint32_t gexcl = __shfl_sync(full, ginc - gsum, gstar);
+    const uint32_t bc = hist[kSelBins - 1 - 32 * gstar - lane];  // lane i: i-th bucket of the group
+    uint32_t binc = bc;
 #pragma unroll
-  for (int w = 1; w < kWarps; ++w) {
-    lo = min(lo, static_cast<uint32_t>(scan[w]));
-    hi = max(hi, static_cast<uint32_t>(scan[4 + w]));
-  }
-  // monotone bucket map: the top 10 significant bits of (key - lo)
-  const uint32_t span = hi - lo;
-  const int shift = max(0, 32 - __clz(static_cast<int>(span | 1u)) - 10);
-  auto bin_of = [&](uint32_t k) -> int { return static_cast<int>((k - lo) >> shift); };
-  for (int i = tid; i < n; i += kThreads) atomicAdd(&hist[bin_of(keys[i])], 1u);
-  __syncthreads();
-  // thread t owns buckets kSelBins-1-8t .. kSelBins-8-8t (descending order)
-  static_assert(kSelBins == 8 * kThreads, "bucket ownership");
-  uint32_t cnt[8];
-  int tot = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    cnt[j] = hist[kSelBins - 1 - 8 * tid - j];
-    tot += static_cast<int>(cnt[j]);
-  }
-  const int excl = block_exclusive_scan(tot, scan);
-  if (excl < topk && topk <= excl + tot) {
-    int run = excl;
-    bool done = false;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (!done) {
-        if (run + static_cast<int>(cnt[j]) >= topk) {
-          scan[8] = kSelBins - 1 - 8 * tid - j;
-          scan[9] = topk - run;  // members of the boundary bucket to keep
-          done = true;
-        } else {
-          run += static_cast<int>(cnt[j]);
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(full, binc, o);
+      if (lane >= o) binc += y;
+    }
+    const unsigned hitb = __ballot_sync(full, gexcl + binc - bc < want && want <= gexcl + binc);
+    const int lstar = __ffs(hitb) - 1;
+    const uint32_t bstar = static_cast<uint32_t>(kSelBins - 1 - 32 * gstar - lstar);
+    const int take = static_cast<int>(want - gexcl - __shfl_sync(full, binc - bc, lstar));
+    __syncwarp();
+    SEL_TRACE(2, global_timer_ns());
+    // members of the boundary bucket (the histogram is no longer needed)
+    int* cand = reinterpret_cast<int*>(hist);
+    int nc = 0;
+    for (int base = 0; base < n; base += 32) {
+      const int i = base + lane;
+      const bool in = i < n && ((keys[i] - lo) >> shift) == bstar;
+      const unsigned bal = __ballot_sync(full, in);
+      if (in) {
+        const int pos = nc + __popc(bal & lt);
+        if (pos < kSelCand) cand[pos] = i;
+      }
+      nc += __popc(bal);
+    }
+    __syncwarp();
+    SEL_TRACE(3, global_timer_ns());
+    SEL_TRACE(5, static_cast<unsigned long long>(nc));
+    if (nc <= kSelCand) {
+      for (int ci = lane; ci < nc; ci += 32) {
+        const int i = cand[ci];
+        const uint32_t ki = keys[i];
+        int r = 0;
+        for (int cj = 0; cj < nc; ++cj) {
+          const int j = cand[cj];
+          const uint32_t kj = keys[j];
+          r += (kj > ki || (kj == ki && j < i)) ? 1 : 0;
         }
+        if (r < take) atomicOr(&selbits[i >> 5], 1u << (i & 31));
+      }
+    } else {
+      // a crowded boundary bucket (many equal scores): rank against all members
+      for (int i = lane; i < n; i += 32) {
+        const uint32_t ki = keys[i];
+        if (((ki - lo) >> shift) != bstar) continue;
+        int r = 0;
+        for (int j = 0; j < n; ++j) {
+          const uint32_t kj = keys[j];
+          r += (((kj - lo) >> shift) == bstar && (kj > ki || (kj == ki && j < i))) ? 1 : 0;
+        }
+        if (r < take) atomicOr(&selbits[i >> 5], 1u << (i & 31));
       }
     }
-  }
-  __syncthreads();
-  const int bstar = scan[8];
-  const int take = scan[9];
-  int* cand = reinterpret_cast<int*>(hist);  // the histogram is no longer needed
-  for (int i = tid; i < n; i += kThreads) {
-    if (bin_of(keys[i]) == bstar) {
-      const int pos = atomicAdd(&scan[10], 1);
-      if (pos < kSelCand) cand[pos] = i;
-    }
-  }
-  __syncthreads();
-  const int nc = scan[10];
-  if (nc <= kSelCand) {
-    for (int ci = warp; ci < nc; ci += kWarps) {
-      const int i = cand[ci];
-      const uint32_t ki = keys[i];
-      int r = 0;
-      for (int cj = lane; cj < nc; cj += 32) {
-        const int j = cand[cj];
-        const uint32_t kj = keys[j];
-        r += (kj > ki || (kj == ki && j < i)) ? 1 : 0;
+    __syncwarp();
+    SEL_TRACE(4, global_timer_ns());
+    // ascending list: every bucket above the boundary plus the marked members
+    int pos = 0;
+    for (int base = 0; base < n; base += 32) {
+      const int i = base + lane;
+      bool keep = false;
+      if (i < n) {
+        const uint32_t b = (keys[i] - lo) >> shift;
+        keep = b > bstar || (b == bstar && ((selbits[i >> 5] >> (i & 31)) & 1u));
       }
-      r = __reduce_add_sync(0xffffffffu, r);
-      if (lane == 0 && r < take) atomicOr(&selbits[i >> 5], 1u << (i & 31));
+      const unsigned bal = __ballot_sync(full, keep);
+      if (keep) sel[pos + __popc(bal & lt)] = i;
+      pos += __popc(bal);
     }
-  } else {
-    // a crowded boundary bucket (many equal scores): rank against all members
-    for (int i = tid; i < n; i += kThreads) {
-      const uint32_t ki = keys[i];
-      if (bin_of(ki) != bstar) continue;
-      int r = 0;
-      for (int j = 0; j < n; ++j) {
-        const uint32_t kj = keys[j];
-        r += (bin_of(kj) == bstar && (kj > ki || (kj == ki && j < i))) ? 1 : 0;
-      }
-      if (r < take) atomicOr(&selbits[i >> 5], 1u << (i & 31));
-    }
+    if (lane == 0) sel[topk] = cur;
   }
-  __syncthreads();
-  // ascending list: everything above the boundary bucket plus the marked members
-  const int per = (n + kThreads - 1) / kThreads;
-  const int i0 = min(n, tid * per);
-  const int i1 = min(n, i0 + per);
-  int cntk = 0;
-  for (int i = i0; i < i1; ++i) {
-    const int b = bin_of(keys[i]);
-    cntk += (b > bstar || (b == bstar && ((selbits[i >> 5] >> (i & 31)) & 1u))) ? 1 : 0;
-  }
-  int pos = block_exclusive_scan(cntk, scan);
-  for (int i = i0; i < i1; ++i) {
-    const int b = bin_of(keys[i]);
-    if (b > bstar || (b == bstar && ((selbits[i >> 5] >> (i & 31)) & 1u))) sel[pos++] = i;
-  }
-  if (tid == 0) sel[topk] = cur;
   __syncthreads();
   return topk + 1;
 }
@@ -237,7 +238,8 @@ __global__ void __launch_bounds__(kThreads, 4)
     decode_cluster_kernel(const __grid_constant__ DecodeParams p,
                           const __grid_constant__ CUtensorMap tmk,
                           const __grid_constant__ CUtensorMap tmv,
-                          const __grid_constant__ CUtensorMap tmw) {
+                          const __grid_constant__ CUtensorMap tmw,
+                          const __grid_constant__ CUtensorMap tmwk) {
   constexpr bool kF32 = std::is_same<T, float>::value;
   constexpr int kDpc = kDim / CS;               // output / W_q columns per CTA
   constexpr int kTilesPerBlock = kF32 ? 4 : 2;  // 16 KiB tiles per K+V block
@@ -265,7 +267,14 @@ __global__ void __launch_bounds__(kThreads, 4)
   float* qv = reinterpret_cast<float*>(base + p.sm.r_qv);
   __nv_bfloat16* wq_s = reinterpret_cast<__nv_bfloat16*>(base + p.sm.r_wq);
   float* gam_s = reinterpret_cast<float*>(base + p.sm.gam);
-  uint64_t* bar_pro = bars + NST;  // prologue copies: q, W_q slice, gamma_q
+  uint64_t* bar_pro = bars + NST;     // prologue copies: q, W_q slice, gamma_q (, gamma_k)
+  uint64_t* bar_p = bars + NST + 1;   // pooled current block has arrived (cluster scope)
+  uint64_t* bar_wk = bars + NST + 2;  // W_k column slice has arrived
+  float* pool_p = reinterpret_cast<float*>(base + p.sm.r_pool_p);
+  float* pool_u = reinterpret_cast<float*>(base + p.sm.r_pool_u);
+  __nv_bfloat16* wk_s = reinterpret_cast<__nv_bfloat16*>(base + p.sm.r_wk);
+  float* gamk_s = reinterpret_cast<float*>(base + p.sm.gamk);
+  const bool pool_on = (MODE == kModeFused) && (p.gamma_k != nullptr);
   float* inbox_o = reinterpret_cast<float*>(base + p.sm.r_inbox);  // [CS][G][kDpc]
   float* inbox_ml = inbox_o + CS * G * kDpc;                         // [CS][G][2]
   float* keys = reinterpret_cast<float*>(base + p.sm.r_keys);
@@ -279,11 +288,12 @@ __global__ void __launch_bounds__(kThreads, 4)
   // first, asynchronously: q of the group (bulk), the W_q column slice of
   // this CTA (one 2-D TMA box per head) and gamma_q (bulk).
   if (tid == 0) {
-    for (int i = 0; i <= NST; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < NST + 3; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
     const uint32_t qbytes = static_cast<uint32_t>(G * kDim * sizeof(T));
     uint32_t tx = qbytes;
     if (MODE != kModeAttend) tx += static_cast<uint32_t>(G * kDim * kDpc * 2 + kDim * 4);
+    if (pool_on) tx += kDim * 4;
     mbar_arrive_expect_tx(bar_pro, tx);
     bulk_g2s(qraw, static_cast<const T*>(p.q) + (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim,
              qbytes, bar_pro);
@@ -293,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 4)
                     bar_pro);
       bulk_g2s(gam_s, p.gamma_q, kDim * 4, bar_pro);
     }
+    if (pool_on) bulk_g2s(gamk_s, p.gamma_k, kDim * 4, bar_pro);
   }
   double th0 = 0.0, th1 = 0.0;
   if (MODE != kModeAttend) {
@@ -330,6 +341,8 @@ __global__ void __launch_bounds__(kThreads, 4)
   const bool bad = __syncthreads_or(err) != 0;
   if (bad && rank == 0 && tid == 0) raise_status(p.status, kStatusBounds);
   const int n = bad ? 0 : c;  // historical blocks
+  // the decoded token completes block c: pool it into gate-key row c
+  const bool do_pool = pool_on && !bad && (L % kBlock == 0) && (c < p.mg);
   if (MODE == kModeFused) m = bad ? 0 : min(p.topk, n) + 1;
   if (MODE == kModeAttend && bad) m = 0;
 
@@ -530,7 +543,14 @@ __global__ void __launch_bounds__(kThreads, 4)
     cluster.sync();  // #2: every score of the (seq, head) is in every CTA
     SAS_TRACE(4);
     if (!bad) {
-      select_blocks(keys, n, p.topk, c, sel, hist, selbits, scan);
+#ifdef SAS_PHASE_TRACE
+      unsigned long long* tr = (p.trace != nullptr && blockIdx.y * gridDim.x + blockIdx.x < kTraceCtas)
+                                   ? p.trace + (blockIdx.y * gridDim.x + blockIdx.x) * kTraceSlots + 10
+                                   : nullptr;
+#else
+      unsigned long long* tr = nullptr;
+#endif
+      select_blocks(keys, n, p.topk, c, sel, hist, selbits, scan, tr);
       if (rank == 0) {
         if (p.sel_idx != nullptr)
           for (int j = tid; j < m; j += kThreads)
@@ -542,6 +562,12 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
     known = nchunks + kTilesPerBlock * cnt_mine;
     pump(nchunks, known);
+    if (do_pool && tid == 0) {
+      // this CTA's 16 columns of W_k[h] (384 rows as three 128-row boxes)
+      mbar_arrive_expect_tx(bar_wk, kPool * kDpc * 2);
+      for (int part = 0; part < 3; ++part)
+        tma_load_2d(wk_s + part * 128 * kDpc, &tmwk, rank * kDpc, h * kPool + part * 128, bar_wk);
+    }
     SAS_TRACE(5);
   }
 
@@ -591,8 +617,33 @@ __global__ void __launch_bounds__(kThreads, 4)
           mma_rows0_7(sacc[1][0], sacc[1][1], qa0[ks], qa2[ks], r2, r3);
         }
       }
+      const bool pool_here = do_pool && own_cur && e == 0;
+      if (pool_here) {
+        // key-block pooling (max, min, mean over the 64 tokens) of the
+        // current block straight from its K tile, sent to every CTA
+        const uint8_t* kt = slots + slotK * kTileBytes;
+        const int d = tid, jc = d >> 3, el = d & 7;
+        float mx = -INFINITY, mn = INFINITY, sm = 0.f;
+        for (int t = 0; t < kBlock; ++t) {
+          const float x = __bfloat162float(
+              *reinterpret_cast<const __nv_bfloat16*>(kt + swz_tile_offset(t, jc) + el * 2));
+          mx = fmaxf(mx, x);
+          mn = fminf(mn, x);
+          sm += x;
+        }
+        sm *= (1.f / kBlock);
+#pragma unroll
+        for (int r = 0; r < CS; ++r) {
+          float* dst = cluster.map_shared_rank(pool_p, r);
+          dst[d] = mx;
+          dst[kDim + d] = mn;
+          dst[2 * kDim + d] = sm;
+        }
+        fence_acq_rel_cluster();
+      }
       __syncthreads();
       pump(t0 + 1, known);
+      if (pool_here && tid < CS) mbar_remote_arrive(bar_p, tid);
       // ---- online softmax (per warp, head gq)
       float x[2][2];
       float mx = -INFINITY;
@@ -683,8 +734,31 @@ __global__ void __launch_bounds__(kThreads, 4)
             if (g < G) lg[g] = fmaf(qatt[g * kDim + hh * 64 + d], kv, lg[g]);
         }
       }
+      const bool pool_here = do_pool && own_cur && e == 0;
+      if (pool_here) {
+        const int d = tid;
+        const float* k0 = reinterpret_cast<const float*>(slots + (t0 % NST) * kTileBytes);
+        const float* k1 = reinterpret_cast<const float*>(slots + ((t0 + 1) % NST) * kTileBytes);
+        float mx = -INFINITY, mn = INFINITY, sm = 0.f;
+        for (int t = 0; t < kBlock; ++t) {
+          const float x = (t < 32 ? k0 : k1)[(t & 31) * kDim + d];
+          mx = fmaxf(mx, x);
+          mn = fminf(mn, x);
+          sm += x;
+        }
+        sm *= (1.f / kBlock);
+#pragma unroll
+        for (int r = 0; r < CS; ++r) {
+          float* dst = cluster.map_shared_rank(pool_p, r);
+          dst[d] = mx;
+          dst[kDim + d] = mn;
+          dst[2 * kDim + d] = sm;
+        }
+        fence_acq_rel_cluster();
+      }
       __syncthreads();
       pump(t0 + 2, known);
+      if (pool_here && tid < CS) mbar_remote_arrive(bar_p, tid);
       float pg[kMaxGroup];
 #pragma unroll
       for (int g = 0; g < kMaxGroup; ++g) {
@@ -798,6 +872,32 @@ __global__ void __launch_bounds__(kThreads, 4)
       }
     }
   }
+  if (do_pool) {
+    // u = P @ W_k[h] for this CTA's 16 columns; slices and their sums of
+    // squares go to CTA 0, which normalises and rotates after barrier #3
+    const bool okp = mbar_wait_cluster(bar_p, 0, p.status);
+    const bool okw = mbar_wait(bar_wk, 0, p.status);
+    const int j = tid & (kDpc - 1);
+    const int rg = tid / kDpc;  // kThreads / kDpc row groups
+    constexpr int kRowsPer = kPool / (kThreads / kDpc);
+    float acc = 0.f;
+    if (okp && okw) {
+      for (int r = rg * kRowsPer; r < (rg + 1) * kRowsPer; ++r)
+        acc = fmaf(pool_p[r], __bfloat162float(wk_s[r * kDpc + j]), acc);
+    }
+    qbar[tid] = acc;  // qbar (dead since the scores) holds the row-group sums
+    __syncthreads();
+    if (tid < kDpc) {
+      float u = 0.f;
+      for (int g = 0; g < kThreads / kDpc; ++g) u += qbar[g * kDpc + tid];
+      float sq = u * u;
+#pragma unroll
+      for (int o = kDpc / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0x0000ffffu, sq, o);
+      float* dst = cluster.map_shared_rank(pool_u, 0);
+      dst[rank * 17 + tid] = u;
+      if (tid == 0) dst[rank * 17 + 16] = sq;
+    }
+  }
   cluster.sync();  // #3: every partial of this CTA's columns has arrived
   SAS_TRACE(7);
   {
@@ -825,6 +925,20 @@ __global__ void __launch_bounds__(kThreads, 4)
       out[(static_cast<size_t>(s) * p.hq + h * G + g) * kDim + rank * kDpc + dd] =
           from_float<OutT>(res);
     }
+  }
+  if (do_pool && rank == 0) {
+    // RMSNorm (gain gamma_k) and gate RoPE at position c of the pooled block
+    const int d = tid;
+    float ss = 0.f;
+#pragma unroll
+    for (int r = 0; r < CS; ++r) ss += pool_u[r * 17 + 16];
+    const float x = pool_u[(d / kDpc) * 17 + (d % kDpc)] * (1.f / sqrtf(ss / kDim + p.eps)) * gamk_s[d];
+    qbar[d] = x;
+    __syncthreads();
+    float cs, sn;
+    rope_cos_sin(p.rope.theta_over_pi[d & 63], c, cs, sn);
+    const float y = (d < 64) ? qbar[d] * cs - qbar[d + 64] * sn : qbar[d] * cs + qbar[d - 64] * sn;
+    p.gate_keys_out[(static_cast<size_t>(pair) * p.mg + c) * kDim + d] = y;
   }
   SAS_TRACE(8);
 }
@@ -870,7 +984,8 @@ namespace {
 
 template <typename T, typename OutT, int CS, int NST, int MODE>
 cudaError_t launch_cluster(const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                           const CUtensorMap& tmw, int batch, cudaStream_t stream) {
+                           const CUtensorMap& tmw, const CUtensorMap& tmwk, int batch,
+                           cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CS, static_cast<unsigned>(batch * p.hkv), 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -883,7 +998,8 @@ cudaError_t launch_cluster(const DecodeParams& p, const CUtensorMap& tmk, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_cluster_kernel<T, OutT, CS, NST, MODE>, p, tmk, tmv, tmw);
+  return cudaLaunchKernelEx(&cfg, decode_cluster_kernel<T, OutT, CS, NST, MODE>, p, tmk, tmv, tmw,
+                            tmwk);
 }
 
 template <typename T, typename OutT, int CS, int NST, int MODE>
@@ -898,13 +1014,13 @@ cudaError_t set_attrs() {
 template <int MODE>
 cudaError_t dispatch_types(bool f32_kv, bool f32_out, int cs, int nst, const DecodeParams& p,
                            const CUtensorMap& tmk, const CUtensorMap& tmv, const CUtensorMap& tmw,
-                           int batch, cudaStream_t st) {
+                           const CUtensorMap& tmwk, int batch, cudaStream_t st) {
   using bf = __nv_bfloat16;
   if (cs != 8 || nst != 2) return cudaErrorInvalidValue;
-  if (!f32_kv && !f32_out) return launch_cluster<bf, bf, 8, 2, MODE>(p, tmk, tmv, tmw, batch, st);
-  if (!f32_kv && f32_out) return launch_cluster<bf, float, 8, 2, MODE>(p, tmk, tmv, tmw, batch, st);
-  if (f32_kv && !f32_out) return launch_cluster<float, bf, 8, 2, MODE>(p, tmk, tmv, tmw, batch, st);
-  return launch_cluster<float, float, 8, 2, MODE>(p, tmk, tmv, tmw, batch, st);
+  if (!f32_kv && !f32_out) return launch_cluster<bf, bf, 8, 2, MODE>(p, tmk, tmv, tmw, tmwk, batch, st);
+  if (!f32_kv && f32_out) return launch_cluster<bf, float, 8, 2, MODE>(p, tmk, tmv, tmw, tmwk, batch, st);
+  if (f32_kv && !f32_out) return launch_cluster<float, bf, 8, 2, MODE>(p, tmk, tmv, tmw, tmwk, batch, st);
+  return launch_cluster<float, float, 8, 2, MODE>(p, tmk, tmv, tmw, tmwk, batch, st);
 }
 
 template <int MODE>
@@ -921,14 +1037,15 @@ cudaError_t attrs_for_mode() {
 
 cudaError_t launch_decode(int mode, bool f32_kv, bool f32_out, int cs, int nst,
                           const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                          const CUtensorMap& tmw, int batch, cudaStream_t stream) {
+                          const CUtensorMap& tmw, const CUtensorMap& tmwk, int batch,
+                          cudaStream_t stream) {
   switch (mode) {
     case kModeGate:
-      return dispatch_types<kModeGate>(f32_kv, false, cs, nst, p, tmk, tmv, tmw, batch, stream);
+      return dispatch_types<kModeGate>(f32_kv, false, cs, nst, p, tmk, tmv, tmw, tmwk, batch, stream);
     case kModeAttend:
-      return dispatch_types<kModeAttend>(f32_kv, f32_out, cs, nst, p, tmk, tmv, tmw, batch, stream);
+      return dispatch_types<kModeAttend>(f32_kv, f32_out, cs, nst, p, tmk, tmv, tmw, tmwk, batch, stream);
     default:
-      return dispatch_types<kModeFused>(f32_kv, f32_out, cs, nst, p, tmk, tmv, tmw, batch, stream);
+      return dispatch_types<kModeFused>(f32_kv, f32_out, cs, nst, p, tmk, tmv, tmw, tmwk, batch, stream);
   }
 }
 

@@ -17,7 +17,9 @@ enum DecodeMode : int { kModeGate = 0, kModeAttend = 1, kModeFused = 2 };
 // Byte offsets (from a 1024-byte aligned base) of the shared-memory regions
 // of the cluster decode kernel.  Region R is reused across phases:
 //   phases 0-1  [ qv | wq | qs ]
-//   phases 2-4  [ inbox | keys | hist | selbits | scan ]
+//   phases 2-4  [ inbox | pool P | pool u | keys | hist | selbits | scan ]
+//               with the W_k slice of the fused pooling over keys.. once the
+//               selection is done
 // inbox (written by other CTAs after the attention phase) covers at least
 // qv, and keys (written by other CTAs during their phase 1) starts past the
 // inbox, so no remote write can land on data this CTA still reads.
@@ -35,6 +37,10 @@ struct DecodeSmem {
   int r_wq;      // bf16 [G][128][dpc] W_q column slice (TMA)       (phase 0)
   int gam;       // fp32 [128] gamma_q (bulk copy)
   int r_inbox;   // fp32 [CS][G][dpc] o, then [CS][G][2] (m, l)     (phases 3-4)
+  int r_pool_p;  // fp32 [384] pooled current block (fused pooling)  (phases 3-4)
+  int r_pool_u;  // fp32 [CS][17] projected slices + sum of squares  (phases 3-4)
+  int r_wk;      // bf16 [384][dpc] W_k column slice (TMA)           (phases 3-4)
+  int gamk;      // fp32 [128] gamma_k (bulk copy, fused pooling)
   int r_keys;    // fp32 scores -> uint32 keys [mg]                 (phases 1-2)
   int r_hist;    // uint32 [kSelBins], then int32 candidates        (phase 2)
   int r_selbits; // uint32 [(mg + 31) / 32]                         (phase 2)
@@ -60,7 +66,8 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
   p.qbar = take(kDim * 4, 16);
   p.pml = take(2 * kWarps * kMaxGroup * 4, 16);
   p.gam = take(kDim * 4, 16);
-  p.bars = take((nst + 1) * 8, 8);  // ring slots + the prologue barrier
+  p.gamk = take(kDim * 4, 16);
+  p.bars = take((nst + 3) * 8, 8);  // ring slots, prologue, pooled P ready, W_k slice
   auto up128 = [](int x) { return (x + 127) / 128 * 128; };
   const int r = up128(off);
   // phases 0-1 (the W_q slice is a tensor-TMA destination: 128-byte aligned)
@@ -69,11 +76,14 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
   const int end01 = p.r_wq + up16(G * kDim * dpc * 2);
   // phases 2-4
   p.r_inbox = r;
-  p.r_keys = r + up16(cs * G * (dpc + 2) * 4);
+  p.r_pool_p = r + up16(cs * G * (dpc + 2) * 4);
+  p.r_pool_u = p.r_pool_p + up16(kPool * 4);
+  p.r_keys = up128(p.r_pool_u + up16(cs * 17 * 4));
+  p.r_wk = p.r_keys;
   p.r_hist = p.r_keys + up16(mg * 4);
   p.r_selbits = p.r_hist + up16(std::max(kSelBins, kSelCand) * 4);
   p.r_scan = p.r_selbits + up16((mg + 31) / 32 * 4);
-  const int end24 = p.r_scan + 16 * 4;
+  const int end24 = std::max(p.r_scan + 16 * 4, p.r_wk + kPool * dpc * 2);
   p.total = std::max(end01, end24) + 1024;
   return p;
 }
@@ -82,7 +92,8 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
 // byte) aligned shared addresses, bulk copies 16-byte ones.
 inline bool decode_smem_aligned(const DecodeSmem& p, int G, int dpc) {
   return p.slots % 1024 == 0 && p.r_wq % 128 == 0 && (G * kDim * dpc * 2) % 128 == 0 &&
-         p.qraw % 16 == 0 && p.gam % 16 == 0 && p.bars % 8 == 0;
+         p.r_wk % 128 == 0 && p.qraw % 16 == 0 && p.gam % 16 == 0 && p.gamk % 16 == 0 &&
+         p.bars % 8 == 0;
 }
 
 struct DecodeParams {
@@ -97,6 +108,8 @@ struct DecodeParams {
   const __nv_bfloat16* w_q;
   const float* gamma_q;
   const float* gate_keys;
+  const float* gamma_k;  // fused pooling of a completed current block (null: off)
+  float* gate_keys_out;  // same array as gate_keys, written at row c when pooling
   KvView kv;
   float* head_scores;
   float* group_scores;
@@ -140,7 +153,8 @@ constexpr int kTraceCtas = 4096;
 // Launchers (return the cudaError_t of the launch).
 cudaError_t launch_decode(int mode, bool f32_kv, bool f32_out, int cs, int nst,
                           const DecodeParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
-                          const CUtensorMap& tmw, int batch, cudaStream_t stream);
+                          const CUtensorMap& tmw, const CUtensorMap& tmwk, int batch,
+                          cudaStream_t stream);
 cudaError_t launch_topk(const TopkParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_pool(bool f32_kv, const PoolParams& p, int batch, cudaStream_t stream);
 size_t topk_smem_bytes(int mg, int max_sel);

@@ -78,7 +78,7 @@ def lib() -> ctypes.CDLL:
             "sas_gate_scores": (ctypes.c_int, [cfgp, vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, sz, vp]),
             "sas_topk_blocks": (ctypes.c_int, [cfgp, vp, vp, i32, i32, vp, vp, vp, sz, vp]),
             "sas_sparse_decode": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, sz, vp]),
-            "sas_decode_step": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
+            "sas_decode_step": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -220,12 +220,15 @@ def sparse_decode(cfg: Config, q, kv: KvCache, sel_idx, sel_count, out, ws, stre
 
 
 def decode_step(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out, ws, sel_idx=None,
-                sel_count=None, group_scores=None, stream=None) -> None:
+                sel_count=None, group_scores=None, w_k=None, gamma_k=None, stream=None) -> None:
+    """sas_decode_step.  With w_k / gamma_k the step also pools the block the
+    decoded token completes into gate_keys (see include/sas.h)."""
     c, k = cfg.c(), kv.c()
     _check(lib().sas_decode_step(ctypes.byref(c), _ptr(q), ctypes.byref(k), _ptr(w_q),
-                                 _ptr(gamma_q), _ptr(gate_keys), int(gate_keys.shape[2]), _ptr(out),
-                                 _ptr(sel_idx), _ptr(sel_count), _ptr(group_scores), _ptr(ws),
-                                 ws.numel(), _stream(stream)), "sas_decode_step")
+                                 _ptr(gamma_q), _ptr(w_k), _ptr(gamma_k), _ptr(gate_keys),
+                                 int(gate_keys.shape[2]), _ptr(out), _ptr(sel_idx), _ptr(sel_count),
+                                 _ptr(group_scores), _ptr(ws), ws.numel(), _stream(stream)),
+           "sas_decode_step")
 
 
 def out_dtype(cfg: Config) -> torch.dtype:

@@ -201,15 +201,22 @@ SAS_API sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const
  * one launch (one thread-block cluster per (sequence, KV head); the cluster's
  * CTAs split the gate keys and the selected blocks and merge through
  * distributed shared memory).
+ *   q, w_q, gamma_q, gate_keys as for sas_gate_scores (q and gamma_q 16-byte
+ *   aligned); out as for sas_sparse_decode.
+ *   w_k, gamma_k: optional (both NULL or both set).  When set, and the decoded
+ *   token completes its block (L_s % 64 == 0) and c_s < max_gate_blocks, the
+ *   step also writes gate_keys[s][h][c_s] -- the gate key of that block, as
+ *   sas_pool_keys computes it -- so decoding maintains the gate keys without
+ *   a separate launch.  Row c_s is not read by the same step.
  *   sel_idx, sel_count, group_scores: optional outputs (NULL to skip), layouts
  *   as above.
  */
 SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const sas_kv* kv,
-                           const void* w_q, const float* gamma_q,
-                           const float* gate_keys, int32_t max_gate_blocks,
-                           void* out, int32_t* sel_idx, int32_t* sel_count,
-                           float* group_scores, void* ws, size_t ws_bytes,
-                           sas_stream_t stream);
+                                   const void* w_q, const float* gamma_q, const void* w_k,
+                                   const float* gamma_k, float* gate_keys,
+                                   int32_t max_gate_blocks, void* out, int32_t* sel_idx,
+                                   int32_t* sel_count, float* group_scores, void* ws,
+                                   size_t ws_bytes, sas_stream_t stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

@@ -43,7 +43,7 @@ def run_pool(inputs, cfg, ws, gate_keys=None, pooled_raw=None, blk_begin=None, n
     return gate_keys
 
 
-def run_decode_step(inputs, cfg, ws, gate_keys):
+def run_decode_step(inputs, cfg, ws, gate_keys, pool=False):
     spec = inputs["spec"]
     dev = inputs["q"].device
     B = spec.batch
@@ -53,7 +53,8 @@ def run_decode_step(inputs, cfg, ws, gate_keys):
     sel_count = torch.full((B, spec.hkv), -1, dtype=torch.int32, device=dev)
     group_scores = torch.full((B, spec.hkv, mg), float("nan"), dtype=torch.float32, device=dev)
     sas.decode_step(cfg, inputs["q"], kv_of(inputs), inputs["w_q"], inputs["gamma_q"], gate_keys,
-                    out, ws, sel_idx=sel_idx, sel_count=sel_count, group_scores=group_scores)
+                    out, ws, sel_idx=sel_idx, sel_count=sel_count, group_scores=group_scores,
+                    w_k=inputs["w_k"] if pool else None, gamma_k=inputs["gamma_k"] if pool else None)
     return {"out": out, "sel_idx": sel_idx, "sel_count": sel_count, "group_scores": group_scores}
 
 

@@ -114,8 +114,8 @@ def _kv(batch=2, cap=4096, **kw):
 def _decode(L, cfg, kv=None, ws_bytes=256, ws=FAKE, q=FAKE, out=FAKE, mg=64):
     c = cfg.c()
     kv = kv or _kv()
-    return L.sas_decode_step(ctypes.byref(c), q, ctypes.byref(kv), FAKE, FAKE, FAKE, mg, out,
-                             None, None, None, ws, ws_bytes, None)
+    return L.sas_decode_step(ctypes.byref(c), q, ctypes.byref(kv), FAKE, FAKE, None, None, FAKE, mg,
+                             out, None, None, None, ws, ws_bytes, None)
 
 
 @nogpu
@@ -152,7 +152,13 @@ def test_workspace_and_pointer_validation(L):
     # TMA row coordinates are 32-bit
     assert _decode(L, cfg, kv=_kv(batch=4096, cap=1 << 20)) == sas.SAS_ERR_UNSUPPORTED
     assert _decode(L, cfg, q=0) == sas.SAS_ERR_INVALID_ARG
+    assert _decode(L, cfg, q=FAKE + 4) == sas.SAS_ERR_INVALID_ARG   # q is bulk-copied: 16 bytes
     assert _decode(L, cfg, mg=0) == sas.SAS_ERR_INVALID_ARG
+    c = cfg.c()
+    kv = _kv()
+    # fused pooling needs both W_k and gamma_k
+    assert L.sas_decode_step(ctypes.byref(c), FAKE, ctypes.byref(kv), FAKE, FAKE, FAKE, None, FAKE, 64,
+                             FAKE, None, None, None, FAKE, 256, None) == sas.SAS_ERR_INVALID_ARG
 
 
 @nogpu

@@ -132,6 +132,44 @@ def test_pool_keys_vs_oracle_and_raw_pooling():
                 assert np.allclose(raw[s, h, b, 256:], p[256:], rtol=1e-6, atol=1e-7)
 
 
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_decode_step_pools_the_completed_block(dt):
+    """With W_k / gamma_k the fused step writes the gate key of the block the
+    decoded token completes (L % 64 == 0) and leaves other rows alone."""
+    spec = DecodeSpec("fused_pool_" + dt, 4, 8, 2, [4096, 2048, 2049, 64], (512,), kv_dtype=dt,
+                      capacity=4096, block_offset_std=0.5, seed=22)
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, 512, "f32" if dt == "f32" else "bf16")
+    ws = sas.make_workspace(cfg, DEV)
+    ref = T.run_pool(inp, cfg, ws)           # every complete block, by the pooling kernel
+    gk = ref.clone()
+    for s, L in enumerate(spec.seq_lens):
+        gk[s, :, (L - 1) // 64] = 0.0          # forget the current block's row
+    gpu = T.run_decode_step(inp, cfg, ws, gk, pool=True)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    wk = inp["w_k"].double().cpu().numpy()
+    for s, L in enumerate(spec.seq_lens):
+        c = (L - 1) // 64
+        for h in range(2):
+            row = gk[s, h, c].cpu().numpy()
+            if L % 64 == 0:
+                ks, _ = logical_kv(inp, s, h, L)
+                want = O.gate_key(O.pool_block(ks[64 * c:64 * c + 64]), wk[h], np.ones(128), c)
+                T.assert_close_rel(row, want, f"fused pooled key s={s} h={h}")
+                # same fp32 arithmetic in another accumulation order (384-term dot products)
+                T.assert_close_rel(row, ref[s, h, c].cpu().numpy(), "fused vs pooling kernel",
+                                   rtol=2e-4)
+            else:
+                assert np.all(row == 0), "an incomplete block must not be pooled"
+    for s, L in enumerate(spec.seq_lens):  # every other row untouched
+        c = (L - 1) // 64
+        keep = [b for b in range(gk.shape[2]) if b != c]
+        assert torch.equal(gk[s, :, keep], ref[s, :, keep])
+    orc = T.oracle_pairs(inp, 512, _all_pairs(spec))
+    T.check_pairs(inp, cfg, gpu, orc, out_atol=(2e-4 if dt == "f32" else T.OUT_ATOL))
+
+
 def test_incremental_pooling_matches_full_pooling():
     spec = DecodeSpec("incr", 2, 8, 2, [4096, 3000], (512,), capacity=4096, seed=17)
     inp = make_decode_inputs(spec, DEV)
