@@ -79,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "sas_topk_blocks": (ctypes.c_int, [cfgp, vp, vp, i32, i32, vp, vp, vp, sz, vp]),
             "sas_sparse_decode": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
+            "sas_decode_step_static": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -229,6 +230,20 @@ def decode_step(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out, ws, s
                                  int(gate_keys.shape[2]), _ptr(out), _ptr(sel_idx), _ptr(sel_count),
                                  _ptr(group_scores), _ptr(ws), ws.numel(), _stream(stream)),
            "sas_decode_step")
+
+
+def decode_step_static(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out, sel_idx=None,
+                       sel_count=None, group_scores=None, w_k=None, gamma_k=None, status_out=None,
+                       stream=None) -> None:
+    """sas_decode_step_static: the same step with no workspace argument, for
+    callers that cannot allocate; status_out (optional device uint32/int32
+    tensor) receives the call's status bits."""
+    c, k = cfg.c(), kv.c()
+    _check(lib().sas_decode_step_static(ctypes.byref(c), _ptr(q), ctypes.byref(k), _ptr(w_q),
+                                        _ptr(gamma_q), _ptr(w_k), _ptr(gamma_k), _ptr(gate_keys),
+                                        int(gate_keys.shape[2]), _ptr(out), _ptr(sel_idx),
+                                        _ptr(sel_count), _ptr(group_scores), _ptr(status_out),
+                                        _stream(stream)), "sas_decode_step_static")
 
 
 def out_dtype(cfg: Config) -> torch.dtype:

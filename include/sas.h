@@ -218,6 +218,31 @@ SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const s
                                    int32_t* sel_count, float* group_scores, void* ws,
                                    size_t ws_bytes, sas_stream_t stream);
 
+/*
+ * Allocation-free variant of sas_decode_step.  The release pages have no
+ * counterpart: this exists for callers that cannot allocate device memory
+ * (a serving loop that must not allocate after warm-up, a plugin whose host
+ * framework owns all GPU memory, a C caller without an allocator) and so
+ * cannot provide the workspace `ws`.
+ *   Same arguments and results as sas_decode_step, minus ws / ws_bytes.  The
+ *   scratch (the device status word) lives in a 256-byte file-scope device
+ *   array of the library that every GPU loading the library keeps until exit.
+ *   status_out: optional device uint32; receives the status bits of this call
+ *   (bit 0: out-of-range length / page / block, bit 1: a bounded wait timed
+ *   out; 0 when clean).
+ *   The first call on a device looks up the array's device address; make it
+ *   before any CUDA stream capture.  Every call clears the status word first;
+ *   calls that overlap on the GPU share the array and race on it.  A build
+ *   whose scratch need exceeds 256 bytes is refused with SAS_ERR_WORKSPACE.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+SAS_API sas_status sas_decode_step_static(const sas_config* cfg, const void* q, const sas_kv* kv,
+                                          const void* w_q, const float* gamma_q, const void* w_k,
+                                          const float* gamma_k, float* gate_keys,
+                                          int32_t max_gate_blocks, void* out, int32_t* sel_idx,
+                                          int32_t* sel_count, float* group_scores,
+                                          uint32_t* status_out, sas_stream_t stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif
