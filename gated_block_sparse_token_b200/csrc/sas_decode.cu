@@ -116,11 +116,23 @@ __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, ui
     const unsigned lt = (1u << lane) - 1u;
     uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
     uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-    for (int i = lane; i < n; i += 32) {
-      const uint32_t k = order_key(vals[i]);
-      keys[i] = k;
-      lo = min(lo, k);
-      hi = max(hi, k);
+    for (int base = 0; base < n; base += 128) {
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + 32 * u + lane;
+        v[u] = (i < n) ? vals[i] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + 32 * u + lane;
+        if (i < n) {
+          const uint32_t k = order_key(v[u]);
+          keys[i] = k;
+          lo = min(lo, k);
+          hi = max(hi, k);
+        }
+      }
     }
     for (int i = lane; i < kSelBins; i += 32) hist[i] = 0u;
     for (int i = lane; i < (n + 31) / 32; i += 32) selbits[i] = 0u;
@@ -129,11 +141,22 @@ __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, ui
     const int shift = max(0, 32 - __clz(static_cast<int>((hi - lo) | 1u)) - 10);
     __syncwarp();
     SEL_TRACE(0, global_timer_ns());
-    for (int i = lane; i < n; i += 32) atomicAdd(&hist[(keys[i] - lo) >> shift], 1u);
+    for (int base = 0; base < n; base += 128) {
+      uint32_t kk[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + 32 * u + lane;
+        kk[u] = (i < n) ? keys[i] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (base + 32 * u + lane < n) atomicAdd(&hist[(kk[u] - lo) >> shift], 1u);
+    }
     __syncwarp();
     SEL_TRACE(1, global_timer_ns());
     // buckets in descending order, 32 groups of 32: lane g sums group g
     uint32_t gsum = 0u;
+#pragma unroll 8
     for (int g = 0; g < kSelBins / 32; ++g) {
       const uint32_t v = __reduce_add_sync(full, hist[kSelBins - 1 - 32 * g - lane]);
       if (lane == g) gsum = v;
@@ -164,15 +187,24 @@ __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, ui
     // members of the boundary bucket (the histogram is no longer needed)
     int* cand = reinterpret_cast<int*>(hist);
     int nc = 0;
-    for (int base = 0; base < n; base += 32) {
-      const int i = base + lane;
-      const bool in = i < n && ((keys[i] - lo) >> shift) == bstar;
-      const unsigned bal = __ballot_sync(full, in);
-      if (in) {
-        const int pos = nc + __popc(bal & lt);
-        if (pos < kSelCand) cand[pos] = i;
+    for (int base = 0; base < n; base += 128) {
+      uint32_t kk[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + 32 * u + lane;
+        kk[u] = (i < n) ? keys[i] : 0u;
       }
-      nc += __popc(bal);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + 32 * u + lane;
+        const bool in = i < n && ((kk[u] - lo) >> shift) == bstar;
+        const unsigned bal = __ballot_sync(full, in);
+        if (in) {
+          const int pos = nc + __popc(bal & lt);
+          if (pos < kSelCand) cand[pos] = i;
+        }
+        nc += __popc(bal);
+      }
     }
     __syncwarp();
     SEL_TRACE(3, global_timer_ns());
@@ -206,16 +238,26 @@ __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, ui
     SEL_TRACE(4, global_timer_ns());
     // ascending list: every bucket above the boundary plus the marked members
     int pos = 0;
-    for (int base = 0; base < n; base += 32) {
-      const int i = base + lane;
-      bool keep = false;
-      if (i < n) {
-        const uint32_t b = (keys[i] - lo) >> shift;
-        keep = b > bstar || (b == bstar && ((selbits[i >> 5] >> (i & 31)) & 1u));
+    for (int base = 0; base < n; base += 128) {
+      uint32_t kk[4], sb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + 32 * u + lane;
+        kk[u] = (i < n) ? keys[i] : 0u;
+        sb[u] = (i < n) ? selbits[i >> 5] : 0u;
       }
-      const unsigned bal = __ballot_sync(full, keep);
-      if (keep) sel[pos + __popc(bal & lt)] = i;
-      pos += __popc(bal);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + 32 * u + lane;
+        bool keep = false;
+        if (i < n) {
+          const uint32_t b = (kk[u] - lo) >> shift;
+          keep = b > bstar || (b == bstar && ((sb[u] >> (i & 31)) & 1u));
+        }
+        const unsigned bal = __ballot_sync(full, keep);
+        if (keep) sel[pos + __popc(bal & lt)] = i;
+        pos += __popc(bal);
+      }
     }
     if (lane == 0) sel[topk] = cur;
   }
@@ -405,6 +447,12 @@ __global__ void __launch_bounds__(kThreads, 4)
   int known = nchunks + ((MODE == kModeAttend) ? kTilesPerBlock * cnt_mine
                                                : (own_cur ? kTilesPerBlock : 0));
   pump(0, known);
+  if (tid == 0 && nchunks > NST) {
+    // the ring holds NST chunks: ask L2 for the rest of this CTA's gate keys now
+    const int b0 = b_lo + NST * kGkChunk;
+    prefetch_l2(p.gate_keys + (static_cast<size_t>(pair) * p.mg + b0) * kDim,
+                static_cast<uint32_t>(b_hi - b0) * kDim * 4u);
+  }
   SAS_TRACE(1);
 
   // ------------------------------------------------------------ phase 0: gate query
@@ -419,10 +467,11 @@ __global__ void __launch_bounds__(kThreads, 4)
       const int j = oc - g * kDpc;
       const T* qrow = qraw + g * kDim + half * 64;
       const __nv_bfloat16* wcol = wq_s + (static_cast<size_t>(g) * kDim + half * 64) * kDpc + j;
-      float acc = 0.f;
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 16
       for (int i = 0; i < 64; ++i)
-        acc = fmaf(to_float(qrow[i]), __bfloat162float(wcol[i * kDpc]), acc);
+        a4[i & 3] = fmaf(to_float(qrow[i]), __bfloat162float(wcol[i * kDpc]), a4[i & 3]);
+      float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       if (half == 0) {
 #pragma unroll
@@ -624,6 +673,7 @@ __global__ void __launch_bounds__(kThreads, 4)
         const uint8_t* kt = slots + slotK * kTileBytes;
         const int d = tid, jc = d >> 3, el = d & 7;
         float mx = -INFINITY, mn = INFINITY, sm = 0.f;
+#pragma unroll 16
         for (int t = 0; t < kBlock; ++t) {
           const float x = __bfloat162float(
               *reinterpret_cast<const __nv_bfloat16*>(kt + swz_tile_offset(t, jc) + el * 2));
@@ -882,8 +932,12 @@ __global__ void __launch_bounds__(kThreads, 4)
     constexpr int kRowsPer = kPool / (kThreads / kDpc);
     float acc = 0.f;
     if (okp && okw) {
-      for (int r = rg * kRowsPer; r < (rg + 1) * kRowsPer; ++r)
-        acc = fmaf(pool_p[r], __bfloat162float(wk_s[r * kDpc + j]), acc);
+      float a2[2] = {0.f, 0.f};
+#pragma unroll 16
+      for (int r = 0; r < kRowsPer; ++r)
+        a2[r & 1] = fmaf(pool_p[rg * kRowsPer + r], __bfloat162float(wk_s[(rg * kRowsPer + r) * kDpc + j]),
+                         a2[r & 1]);
+      acc = a2[0] + a2[1];
     }
     qbar[tid] = acc;  // qbar (dead since the scores) holds the row-group sums
     __syncthreads();

@@ -150,6 +150,18 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Ask L2 to fetch `bytes` contiguous bytes from global memory (no shared
+// memory involved, nothing to wait for).  src 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Prefetch the 128-byte line holding `p` into L2 (load/store unit path, so it
+// does not queue behind the TMA copies of the same SM).
+__device__ __forceinline__ void prefetch_line_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // 2-D tiled tensor copy (box given by the tensor map) at element coordinates
 // (x = innermost, y = row) into this CTA's shared memory.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
