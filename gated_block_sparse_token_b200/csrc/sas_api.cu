@@ -13,6 +13,7 @@
 namespace sas {
 cudaError_t prepare_decode_kernels();
 cudaError_t prepare_pool_kernels();
+cudaError_t prepare_prefill_kernels();
 }
 
 namespace {
@@ -48,6 +49,7 @@ cudaError_t prepare() {
     g_encode = reinterpret_cast<EncodeTiledFn>(fn);
     g_prep_err = sas::prepare_decode_kernels();
     if (g_prep_err == cudaSuccess) g_prep_err = sas::prepare_pool_kernels();
+    if (g_prep_err == cudaSuccess) g_prep_err = sas::prepare_prefill_kernels();
   });
   return g_prep_err;
 }
@@ -194,6 +196,21 @@ unsigned long long* trace_region(void* ws) {
 #endif
 }
 
+size_t ws_header_bytes() {
+#ifdef SAS_PHASE_TRACE
+  return kStatusBytes + static_cast<size_t>(sas::kTraceCtas) * sas::kTraceSlots * 8;
+#else
+  return kStatusBytes;
+#endif
+}
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t prefill_scratch_bytes(size_t batch, int hq, int hkv, size_t nblk, int max_sel) {
+  return up256(batch * hq * nblk * kDim * 4) + up256(batch * hkv * nblk * max_sel * 4) +
+         up256(batch * hkv * nblk * 4);
+}
+
 sas_status launch_result(cudaError_t e) {
   if (e != cudaSuccess) {
     (void)cudaGetLastError();
@@ -222,14 +239,15 @@ const char* sas_status_string(sas_status s) {
 }
 
 size_t sas_workspace_bytes(const sas_config* cfg, int32_t batch, int32_t max_seq_len) {
-  (void)cfg;
-  (void)batch;
-  (void)max_seq_len;
-#ifdef SAS_PHASE_TRACE
-  return kStatusBytes + static_cast<size_t>(sas::kTraceCtas) * sas::kTraceSlots * 8;
-#else
-  return kStatusBytes;
-#endif
+  size_t bytes = ws_header_bytes();
+  if (cfg != nullptr && batch > 0 && max_seq_len > 0 && cfg->num_kv_heads > 0 &&
+      cfg->num_q_heads > 0 && cfg->token_budget >= 64) {
+    // prefill scratch: gate queries, block lists and their lengths
+    const size_t nblk = static_cast<size_t>((max_seq_len + 63) / 64);
+    bytes += prefill_scratch_bytes(batch, cfg->num_q_heads, cfg->num_kv_heads, nblk,
+                                   cfg->token_budget / 64);
+  }
+  return bytes;
 }
 
 sas_status sas_reset_device_status(void* ws, sas_stream_t stream) {
@@ -417,6 +435,104 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
   return launch_result(sas::launch_decode(mode, f32_kv, cfg->out_dtype == SAS_DTYPE_F32,
                                           kClusterSize, kStages, p, tmk, tmv, tmw, tmwk, kv->batch,
                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const void* k,
+                                    const void* v, int32_t batch, int32_t seq_len,
+                                    const void* w_q, const float* gamma_q, const void* w_k,
+                                    const float* gamma_k, float* gate_keys,
+                                    int32_t max_gate_blocks, void* out, int32_t* sel_idx,
+                                    int32_t* sel_count, void* ws, size_t ws_bytes,
+                                    sas_stream_t stream) {
+  sas_status st = check_config(cfg);
+  if (st != SAS_OK) return st;
+  if (batch < 0 || seq_len < 0) return SAS_ERR_INVALID_ARG;
+  if (batch == 0 || seq_len == 0) return SAS_OK;
+  if (cfg->kv_dtype != SAS_DTYPE_BF16 || cfg->out_dtype != SAS_DTYPE_BF16) return SAS_ERR_UNSUPPORTED;
+  const int G = cfg->num_q_heads / cfg->num_kv_heads;
+  if (G % 2 != 0) return SAS_ERR_UNSUPPORTED;  // the tensor-core tile pairs two query heads
+  if (seq_len % 64 != 0) return SAS_ERR_UNSUPPORTED;
+  if (cfg->token_budget / 64 > sas::kPfMaxSel) return SAS_ERR_UNSUPPORTED;
+  const int nblk = seq_len / 64;
+  if (max_gate_blocks < nblk || max_gate_blocks > kMaxGateBlocks) return SAS_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || v == nullptr || w_q == nullptr || gamma_q == nullptr ||
+      w_k == nullptr || gamma_k == nullptr || gate_keys == nullptr || out == nullptr)
+    return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(w_q, 16) ||
+      !aligned(gamma_q, 16) || !aligned(w_k, 16) || !aligned(gamma_k, 16) ||
+      !aligned(gate_keys, 16) || !aligned(out, 16) || (sel_idx != nullptr && !aligned(sel_idx, 4)) ||
+      (sel_count != nullptr && !aligned(sel_count, 4)))
+    return SAS_ERR_INVALID_ARG;
+  if (ws == nullptr || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
+  if (ws_bytes < sas_workspace_bytes(cfg, batch, seq_len)) return SAS_ERR_WORKSPACE;
+  const long long qrows = static_cast<long long>(batch) * cfg->num_q_heads * seq_len;
+  if (qrows > 0x7fffffffLL) return SAS_ERR_UNSUPPORTED;
+  if (static_cast<long long>(batch) * cfg->num_kv_heads * nblk * (G / 2) > 0x7fffffffLL)
+    return SAS_ERR_UNSUPPORTED;
+  if (batch > 65535 || cfg->num_q_heads > 65535) return SAS_ERR_UNSUPPORTED;
+  if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  // 1. pooled gate keys of every block
+  sas_kv kv{};
+  kv.k = k;
+  kv.v = v;
+  kv.block_table = nullptr;
+  kv.seq_lens = nullptr;  // every sequence has seq_len tokens
+  kv.batch = batch;
+  kv.capacity = seq_len;
+  sas::PoolParams pp{};
+  pp.hkv = cfg->num_kv_heads;
+  pp.mg = max_gate_blocks;
+  pp.num_blocks = nblk;
+  pp.rope_base = cfg->rope_base;
+  pp.eps = cfg->norm_eps;
+  sas::fill_rope_table(pp.rope, cfg->rope_base);
+  pp.kv = make_view(cfg, &kv);
+  pp.blk_begin = nullptr;
+  pp.w_k = static_cast<const __nv_bfloat16*>(w_k);
+  pp.gamma_k = gamma_k;
+  pp.gate_keys = gate_keys;
+  pp.pooled_raw = nullptr;
+  pp.status = static_cast<uint32_t*>(ws);
+  cudaError_t e = sas::launch_pool(false, pp, batch, s);
+  if (e != cudaSuccess) return launch_result(e);
+
+  // 2-4. gate queries, selection, tensor-core block-sparse attention
+  sas::PrefillParams p{};
+  sas::fill_rope_table(p.rope, cfg->rope_base);
+  p.batch = batch;
+  p.hq = cfg->num_q_heads;
+  p.hkv = cfg->num_kv_heads;
+  p.G = G;
+  p.T = seq_len;
+  p.nblk = nblk;
+  p.max_sel = cfg->token_budget / 64;
+  p.topk = p.max_sel - 1;
+  p.mg = max_gate_blocks;
+  p.eps = cfg->norm_eps;
+  p.attn_scale_log2 = cfg->attn_scale * 1.4426950408889634f;
+  p.gate_scale = cfg->gate_scale;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.w_q = static_cast<const __nv_bfloat16*>(w_q);
+  p.gamma_q = gamma_q;
+  p.gate_keys = gate_keys;
+  uint8_t* scratch = static_cast<uint8_t*>(ws) + ws_header_bytes();
+  p.qt = reinterpret_cast<float*>(scratch);
+  scratch += up256(static_cast<size_t>(batch) * p.hq * nblk * kDim * 4);
+  p.sel = reinterpret_cast<int32_t*>(scratch);
+  scratch += up256(static_cast<size_t>(batch) * p.hkv * nblk * p.max_sel * 4);
+  p.cnt = reinterpret_cast<int32_t*>(scratch);
+  p.sel_out = sel_idx;
+  p.cnt_out = sel_count;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.status = static_cast<uint32_t*>(ws);
+  CUtensorMap tmq, tmk, tmv;
+  if (!encode_kv_map(&tmq, q, qrows) ||
+      !encode_kv_map(&tmk, k, static_cast<long long>(batch) * p.hkv * seq_len) ||
+      !encode_kv_map(&tmv, v, static_cast<long long>(batch) * p.hkv * seq_len))
+    return SAS_ERR_CUDA;
+  return launch_result(sas::launch_prefill(p, tmq, tmk, tmv, s));
 }
 
 sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const sas_kv* kv,

@@ -142,6 +142,26 @@ struct PoolParams {
   uint32_t* status;
 };
 
+struct PrefillParams {
+  RopeTable rope;
+  int batch, hq, hkv, G, T, nblk, topk, max_sel, mg;
+  float eps, attn_scale_log2, gate_scale;
+  const __nv_bfloat16* q;     // [B][Hq][T][128]
+  const __nv_bfloat16* w_q;   // [Hq][128][128]
+  const float* gamma_q;       // [128]
+  const float* gate_keys;     // [B][Hkv][mg][128]
+  float* qt;                  // workspace: gate queries [B][Hq][nblk][128]
+  int32_t* sel;               // workspace: block lists [B][Hkv][nblk][max_sel]
+  int32_t* cnt;               // workspace: list lengths [B][Hkv][nblk]
+  int32_t* sel_out;           // optional copies of the lists
+  int32_t* cnt_out;
+  __nv_bfloat16* out;         // [B][Hq][T][128]
+  uint32_t* status;
+};
+
+constexpr int kPfQb = 16;      // query blocks per gate-query CTA
+constexpr int kPfMaxSel = 64;  // prefill budget up to 4,096 tokens (two CTAs per SM)
+
 constexpr int kPoolBlocksPerCta = 8;
 constexpr int kPoolWkBytes = kPool * kDim * 2;  // W_k of one KV head, bf16 (96 KiB)
 
@@ -160,6 +180,9 @@ cudaError_t launch_pool(bool f32_kv, const PoolParams& p, int batch, cudaStream_
 size_t topk_smem_bytes(int mg, int max_sel);
 size_t pool_smem_bytes();
 void fill_rope_table(RopeTable& t, float base);
+cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                           const CUtensorMap& tmv, cudaStream_t stream);
+size_t prefill_attn_smem_bytes(int max_sel);
 
 // One-time per-process set-up of kernel attributes.
 cudaError_t prepare_kernels();

@@ -38,7 +38,7 @@ __global__ void __launch_bounds__(kThreads) pool_keys_kernel(const __grid_consta
   __shared__ float xn[kDim];
   __shared__ float ssq[kWarps];
 
-  const int L = p.kv.seq_lens[s];
+  const int L = (p.kv.seq_lens != nullptr) ? p.kv.seq_lens[s] : p.kv.capacity;  // prefill: full length
   const int first = p.blk_begin != nullptr ? p.blk_begin[s] : 0;
   const int b0 = first + static_cast<int>(blockIdx.x) * NB;
   const int b_end = first + p.num_blocks;

@@ -80,6 +80,7 @@ def lib() -> ctypes.CDLL:
             "sas_sparse_decode": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step_static": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]),
+            "sas_prefill_block_sparse": (ctypes.c_int, [cfgp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -244,6 +245,20 @@ def decode_step_static(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out
                                         int(gate_keys.shape[2]), _ptr(out), _ptr(sel_idx),
                                         _ptr(sel_count), _ptr(group_scores), _ptr(status_out),
                                         _stream(stream)), "sas_decode_step_static")
+
+
+def prefill_block_sparse(cfg: Config, q, k, v, w_q, gamma_q, w_k, gamma_k, gate_keys, out, ws,
+                         sel_idx=None, sel_count=None, stream=None) -> None:
+    """sas_prefill_block_sparse: q [B][Hq][T][128], k / v [B][Hkv][T][128] (bf16),
+    out like q; writes gate_keys [B][Hkv][MG][128]; ws from
+    make_workspace(cfg, device, batch=B, max_seq_len=T)."""
+    c = cfg.c()
+    B, T = int(q.shape[0]), int(q.shape[2])
+    _check(lib().sas_prefill_block_sparse(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), B, T, _ptr(w_q),
+                                          _ptr(gamma_q), _ptr(w_k), _ptr(gamma_k), _ptr(gate_keys),
+                                          int(gate_keys.shape[2]), _ptr(out), _ptr(sel_idx),
+                                          _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),
+           "sas_prefill_block_sparse")
 
 
 def out_dtype(cfg: Config) -> torch.dtype:

@@ -139,3 +139,36 @@ def logical_kv(inputs: dict, s: int, h: int, length: int):
         ks = k[pages, h].reshape(nb * BLOCK, DIM)
         vs = v[pages, h].reshape(nb * BLOCK, DIM)
     return (ks[:length].double().cpu().numpy(), vs[:length].double().cpu().numpy())
+
+
+@dataclass
+class PrefillSpec:
+    name: str
+    batch: int
+    hq: int
+    hkv: int
+    seq_len: int
+    token_budget: int = 2048
+    seed: int = 4
+
+
+def qwen3_8b_prefill_32k(batch: int = 4, seq_len: int = 32768, seed: int = 4) -> PrefillSpec:
+    """Qwen3-8B head layout (32 query / 8 KV heads), batch 4, causal 32,768-token
+    prefill, Top-K 31 + the diagonal block (2,048-token budget)."""
+    return PrefillSpec(f"qwen3_8b_prefill_b{batch}_{seq_len // 1024}k", batch, 32, 8, seq_len, 2048, seed)
+
+
+def make_prefill_inputs(spec: PrefillSpec, device="cpu") -> dict:
+    """q [B][Hq][T][128], k / v [B][Hkv][T][128] ~ N(0,1) in bf16; gate weights as
+    for decode.  Draw order: q, K, V, W_q, W_k."""
+    g = torch.Generator(device=device).manual_seed(spec.seed)
+    B, hq, hkv, T = spec.batch, spec.hq, spec.hkv, spec.seq_len
+    out = {"spec": spec}
+    out["q"] = _randn((B, hq, T, DIM), g, device).to(torch.bfloat16)
+    out["k"] = _randn((B, hkv, T, DIM), g, device).to(torch.bfloat16)
+    out["v"] = _randn((B, hkv, T, DIM), g, device).to(torch.bfloat16)
+    out["w_q"] = _randn((hq, DIM, DIM), g, device, 1.0 / math.sqrt(DIM)).to(torch.bfloat16)
+    out["w_k"] = _randn((hkv, 3 * DIM, DIM), g, device, 1.0 / math.sqrt(3 * DIM)).to(torch.bfloat16)
+    out["gamma_q"] = torch.ones(DIM, dtype=torch.float32, device=device)
+    out["gamma_k"] = torch.ones(DIM, dtype=torch.float32, device=device)
+    return out

@@ -219,6 +219,36 @@ SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const s
                                    size_t ws_bytes, sas_stream_t stream);
 
 /*
+ * Block-sparse chunked prefill (pages: training Top-K 31 historical blocks
+ * over 32,768-token sequences, 64-token blocks, gate with Qproj, Q/K
+ * normalisation and gate RoPE).  For every 64-token query block i of every
+ * sequence and KV head: gate query = per-head mean of the block's 64 queries
+ * through Qproj, RMSNorm and RoPE at position i; group scores against the
+ * gate keys of blocks b < i; the min(budget/64 - 1, i) best blocks plus block
+ * i; token t of block i attends to all tokens of the kept blocks and to
+ * tokens 64i..t of its own block.
+ *   q      bf16 [B][Hq][T][128]      k, v bf16 [B][Hkv][T][128]
+ *   out    bf16 [B][Hq][T][128]      (all 16-byte aligned)
+ *   w_q, gamma_q, w_k, gamma_k as for the decode entry points.
+ *   gate_keys fp32 [B][Hkv][MG][128] (output): rows 0..T/64-1 are written, so
+ *   decoding can continue from them.  MG >= T/64.
+ *   sel_idx int32 [B][Hkv][T/64][budget/64], sel_count int32 [B][Hkv][T/64]:
+ *   optional outputs (NULL to skip), the block list of every query block.
+ *   ws: 256-byte aligned, at least sas_workspace_bytes(cfg, B, T) bytes
+ *   (gate queries and block lists live there).
+ * This build requires bf16 inputs and output, an even GQA group size
+ * (the tensor-core tile holds two query heads), T a multiple of 64 and a
+ * budget of at most 4,096 tokens; other requests return SAS_ERR_UNSUPPORTED.
+ */
+SAS_API sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const void* k,
+                                            const void* v, int32_t batch, int32_t seq_len,
+                                            const void* w_q, const float* gamma_q,
+                                            const void* w_k, const float* gamma_k,
+                                            float* gate_keys, int32_t max_gate_blocks, void* out,
+                                            int32_t* sel_idx, int32_t* sel_count, void* ws,
+                                            size_t ws_bytes, sas_stream_t stream);
+
+/*
  * Allocation-free variant of sas_decode_step.  The release pages have no
  * counterpart: this exists for callers that cannot allocate device memory
  * (a serving loop that must not allocate after warm-up, a plugin whose host

@@ -1,0 +1,102 @@
+"""GPU parity of the block-sparse chunked prefill (tcgen05 attention) against
+the CPU oracle, through the C ABI: gate keys of every block, the block list of
+every query block (exact up to the tie window), and the attention output of
+every token (bf16 storage, 1e-2 max-abs)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from gated_block_sparse_token_b200 import sas
+from gated_block_sparse_token_b200.workloads import PrefillSpec, make_prefill_inputs, qwen3_8b_prefill_32k
+from oracle import sas_oracle as O
+
+import sas_testlib as T
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _run(spec):
+    inp = make_prefill_inputs(spec, DEV)
+    B, Tn = spec.batch, spec.seq_len
+    nblk = Tn // 64
+    cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget)
+    ws = sas.make_workspace(cfg, DEV, batch=B, max_seq_len=Tn)
+    gk = torch.zeros(B, spec.hkv, nblk, 128, dtype=torch.float32, device=DEV)
+    out = torch.full((B, spec.hq, Tn, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
+    sel = torch.full((B, spec.hkv, nblk, cfg.max_sel), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.full((B, spec.hkv, nblk), -1, dtype=torch.int32, device=DEV)
+    sas.prefill_block_sparse(cfg, inp["q"], inp["k"], inp["v"], inp["w_q"], inp["gamma_q"], inp["w_k"],
+                             inp["gamma_k"], gk, out, ws, sel_idx=sel, sel_count=cnt)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    return inp, cfg, gk, out, sel, cnt
+
+
+def _check(spec, inp, cfg, gk, out, sel, cnt, triples):
+    G = spec.hq // spec.hkv
+    topk = cfg.max_sel - 1
+    wq = inp["w_q"].double().cpu().numpy()
+    wk = inp["w_k"].double().cpu().numpy()
+    ones = np.ones(128)
+    gk_h, out_h, sel_h, cnt_h = gk.cpu().numpy(), out.float().cpu().numpy(), sel.cpu().numpy(), cnt.cpu().numpy()
+    cache = {}
+    for (s, h, i) in triples:
+        if (s, h) not in cache:
+            ks = inp["k"][s, h].double().cpu().numpy()
+            vs = inp["v"][s, h].double().cpu().numpy()
+            keys = O.gate_keys_for_sequence(ks, spec.seq_len // 64, wk[h], ones)
+            T.assert_close_rel(gk_h[s, h], keys, f"prefill gate keys s={s} h={h}")
+            cache[(s, h)] = (ks, vs, keys)
+        ks, vs, keys = cache[(s, h)]
+        qb = inp["q"][s, h * G:(h + 1) * G, 64 * i:64 * (i + 1)].double().cpu().numpy()
+        r = O.prefill_query_block(qb, ks, vs, i, keys, wq[h * G:(h + 1) * G], np.tile(ones, (G, 1)), topk)
+        m = int(cnt_h[s, h, i])
+        got_sel = list(sel_h[s, h, i, :m])
+        tag = f"{spec.name} s={s} h={h} i={i}"
+        swapped = T.assert_selection(got_sel, r["sel"], r["S"], topk, tag)
+        want = r["out"]
+        if swapped:
+            hist = O.selected_token_ids(got_sel[:-1], 64 * (i + 1))
+            want = np.stack([np.stack([O.attention_over_tokens(qb[g, t], ks, vs, hist + list(range(64 * i, 64 * i + t + 1)),
+                                                                 cfg.attn_scale) for t in range(64)]) for g in range(G)])
+        got = out_h[s, h * G:(h + 1) * G, 64 * i:64 * (i + 1)]
+        err = float(np.max(np.abs(got - want)))
+        assert np.all(np.isfinite(got)) and err <= T.OUT_ATOL, f"{tag}: out max-abs err {err}"
+
+
+def test_prefill_small_all_blocks():
+    spec = PrefillSpec("pf_small", 1, 4, 2, 1024, token_budget=256, seed=41)
+    res = _run(spec)
+    triples = [(0, h, i) for h in range(2) for i in range(16)]
+    _check(spec, *res, triples)
+
+
+def test_prefill_budget_covering_context_is_dense_causal():
+    spec = PrefillSpec("pf_dense", 2, 4, 1, 512, token_budget=1024, seed=42)
+    inp, cfg, gk, out, sel, cnt = _run(spec)
+    q = inp["q"].double().cpu().numpy()
+    outh = out.float().cpu().numpy()
+    for s in range(2):
+        ks = inp["k"][s, 0].double().cpu().numpy()
+        vs = inp["v"][s, 0].double().cpu().numpy()
+        for g in range(4):
+            dense = O.dense_causal_prefill(q[s, g], ks, vs)
+            err = float(np.max(np.abs(outh[s, g] - dense)))
+            assert err <= T.OUT_ATOL, (s, g, err)
+    assert torch.equal(cnt.cpu(), torch.arange(1, 9, dtype=torch.int32).repeat(2, 1, 1))
+
+
+def test_prefill_eight_query_heads_per_kv_head():
+    spec = PrefillSpec("pf_g8", 1, 8, 1, 768, token_budget=320, seed=43)
+    res = _run(spec)
+    _check(spec, *res, [(0, 0, i) for i in range(12)])
+
+
+def test_prefill_qwen3_8b_32k_full_size():
+    spec = qwen3_8b_prefill_32k()
+    res = _run(spec)
+    triples = [(0, 0, 0), (0, 0, 30), (1, 3, 31), (2, 5, 200), (3, 7, 511), (3, 2, 64)]
+    _check(spec, *res, triples)
