@@ -56,6 +56,10 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-batch", type=int, default=4)
+    ap.add_argument("--prefill-steps", type=int, default=5)
+    ap.add_argument("--skip-prefill", action="store_true")
+    ap.add_argument("--prefill-only", action="store_true")
     return ap.parse_args()
 
 
@@ -176,6 +180,78 @@ def decode_bytes(seq_lens, hq, hkv, budget, kv_elem=2, pool=True):
     return tot
 
 
+def prefill_flops(nblk, hq, hkv, budget, batch):
+    """Tensor FLOPs of the block-sparse prefill attention, counted as full
+    64x64 tiles: per (sequence, query head, query block i) min(topk, i) + 1
+    blocks, each 2*64*64*128 for Q K^T and as much for P V."""
+    topk = budget // 64 - 1
+    pairs = sum(min(topk, i) + 1 for i in range(nblk))
+    return batch * hq * pairs * 4 * 64 * 64 * 128
+
+
+def measured_tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained"]), "measured sustained bf16"
+    return 1400.0, "fallback sustained bf16"
+
+
+def run_prefill(args, device, world):
+    """Block-sparse chunked prefill, Qwen3-8B heads, 32,768 tokens per sequence,
+    Top-K 31 + diagonal: one sas_prefill_block_sparse call per step (pooling,
+    gate queries, selection, tcgen05 attention)."""
+    import torch
+    from gated_block_sparse_token_b200 import sas
+    from gated_block_sparse_token_b200.workloads import make_prefill_inputs, qwen3_8b_prefill_32k
+
+    spec = qwen3_8b_prefill_32k(batch=args.prefill_batch)
+    inp = make_prefill_inputs(spec, device)
+    B, T = spec.batch, spec.seq_len
+    nblk = T // 64
+    cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget)
+    ws = sas.make_workspace(cfg, device, batch=B, max_seq_len=T)
+    gk = torch.zeros(B, spec.hkv, nblk, 128, dtype=torch.float32, device=device)
+    out = torch.empty(B, spec.hq, T, 128, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.Stream(device)
+
+    def call():
+        sas.prefill_block_sparse(cfg, inp["q"], inp["k"], inp["v"], inp["w_q"], inp["gamma_q"], inp["w_k"],
+                                 inp["gamma_k"], gk, out, ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            call()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.prefill_steps):
+            call()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.prefill_steps, world)
+    if sas.get_device_status(ws, stream) != sas.SAS_OK:
+        raise RuntimeError("device status not OK after the prefill run")
+    flops = prefill_flops(nblk, spec.hq, spec.hkv, spec.token_budget, B)
+    peak, kind = measured_tensor_peak()
+    achieved = flops / t / 1e12
+    return {"workload": spec.name, "batch_per_gpu": B, "seq_len": T, "q_heads": spec.hq,
+            "kv_heads": spec.hkv, "token_budget": spec.token_budget, "steps": args.prefill_steps,
+            "ms_per_step": round(t * 1e3, 4), "tokens_per_s": round(world * B * T / t, 1),
+            "launches_per_step": 4,
+            "roofline": {"kernel": "prefill_attn_kernel (tcgen05)", "bound": "tensor",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": kind,
+                         "flops_per_step": flops,
+                         "note": "FLOPs over the whole prefill call (pooling, gate, selection and "
+                                 "attention launches): a lower bound on the attention kernel's rate"}}
+
+
 def source_digest():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_block_sparse_token_b200", "csrc")
@@ -291,6 +367,11 @@ def run_ours(args):
 
     rank, world, local = dist_setup(args.gpus)
     device = torch.device("cuda", local)
+    if args.prefill_only:
+        pf = run_prefill(args, device, world)
+        if rank == 0:
+            print(json.dumps({"impl": "ours", "prefill": pf}), flush=True)
+        return
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_seconds)   # before any pool could fork after CUDA use
@@ -347,6 +428,10 @@ def run_ours(args):
         barrier(world)
     t_e2e = max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
 
+    del layers, main, warm
+    torch.cuda.empty_cache()
+    pf = None if args.skip_prefill else run_prefill(args, device, world)
+
     if rank != 0:
         return
     peak, peak_kind = measured_peaks()
@@ -379,6 +464,8 @@ def run_ours(args):
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if pf is not None:
+        line["prefill"] = pf
     print(json.dumps(line), flush=True)
 
 
