@@ -527,6 +527,7 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
   p.cnt_out = sel_count;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.status = static_cast<uint32_t*>(ws);
+  p.trace = trace_region(ws);
   CUtensorMap tmq, tmk, tmv;
   if (!encode_kv_map(&tmq, q, qrows) ||
       !encode_kv_map(&tmk, k, static_cast<long long>(batch) * p.hkv * seq_len) ||

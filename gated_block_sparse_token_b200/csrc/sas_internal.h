@@ -157,6 +157,7 @@ struct PrefillParams {
   int32_t* cnt_out;
   __nv_bfloat16* out;         // [B][Hq][T][128]
   uint32_t* status;
+  unsigned long long* trace;  // per-CTA timings (tracing builds only), else null
 };
 
 constexpr int kPfQb = 16;      // query blocks per gate-query CTA

@@ -172,19 +172,45 @@ size_t prefill_select_smem_bytes(int nblk, int max_sel) {
 // ------------------------------------------------------------ tcgen05 attention
 // 160 threads: warps 0-3 own one query row each per thread (softmax, O
 // rescaling, epilogue); warp 4 lane 0 issues the TMA copies and the MMAs.
-// Shared memory (1024-aligned): Q 32 KiB | K ring 2 x 16 KiB | V ring 2 x 16 KiB
-// | P 16 KiB | barriers | block list.  Tensor memory: S double buffer
-// (2 x 64 columns) and O (128 columns), 256 columns in all.
+// Shared memory (1024-aligned): Q 32 KiB | K ring 3 x 16 KiB | V ring 2 x 16 KiB
+// | barriers | block list.  Tensor memory, 256 columns: two S buffers of 64
+// fp32 columns and O (128 columns).  The softmax writes P_e as bf16 pairs over
+// the first 32 columns of S buffer e % 2, and P V reads it from there (A
+// operand in tensor memory), so P never goes through shared memory and the
+// softmax of tile e + 1 does not wait for P V of tile e.
+//
+// Per tile e (m tiles, ascending block ids, the diagonal block last):
+//   QK_e    S[e%2] = Q K_e^T          needs K_e and P V_{e-2} done (S[e%2] free)
+//   soft_e  P_e = exp2(S log2e/sqrt(d) - m), into S[e%2]; O *= alpha when the
+//           running maximum grew by more than 2^8 (then after P V_{e-1})
+//   PV_e    O += P_e V_e              needs soft_e and V_e
+// The issuer runs PV_e, waits for it, then QK_{e+2}; soft_{e+1} overlaps both.
 constexpr int kPfAttnThreads = 160;
 constexpr uint32_t kPfTmemCols = 256;
-constexpr int kPfSmemQ = 0, kPfSmemK = 32768, kPfSmemV = 65536, kPfSmemP = 98304,
-              kPfSmemBars = 114688;
-enum { kBarQ = 0, kBarK0 = 1, kBarV0 = 3, kBarS0 = 5, kBarSfree0 = 7, kBarP = 9, kBarO = 10,
-       kNumPfBars = 11 };
+constexpr int kPfKStages = 3, kPfVStages = 2;
+constexpr int kPfSmemQ = 0, kPfSmemK = 32768, kPfSmemV = kPfSmemK + kPfKStages * 16384,
+              kPfSmemBars = kPfSmemV + kPfVStages * 16384;
+enum { kBarQ = 0, kBarK0 = 1, kBarV0 = kBarK0 + kPfKStages, kBarS0 = kBarV0 + kPfVStages,
+       kBarP0 = kBarS0 + 2, kBarO = kBarP0 + 2, kNumPfBars = kBarO + 1 };
 
 size_t prefill_attn_smem_bytes(int max_sel) {
   return static_cast<size_t>(kPfSmemBars + kNumPfBars * 8 + 16 + max_sel * 4);
 }
+
+// Tracing builds: the issuer and softmax thread 0 add up the SM cycles they
+// spend in each wait and phase; CTA k < kTraceCtas writes them to slots of
+// trace row k.  Ordinary builds compile the hooks out.
+#ifdef SAS_PHASE_TRACE
+#define PF_TIC(v) const long long v = clock64()
+#define PF_TOC(acc, v) (acc) += clock64() - (v)
+#else
+#define PF_TIC(v) \
+  do {            \
+  } while (0)
+#define PF_TOC(acc, v) \
+  do {                 \
+  } while (0)
+#endif
 
 __global__ void __launch_bounds__(kPfAttnThreads, 2)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p,
@@ -201,6 +227,12 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
   const int s = idx % p.batch;
   const int i = p.nblk - 1 - idx / p.batch;  // longest block lists first
   const int g0 = h * p.G + 2 * pair;
+#ifdef SAS_PHASE_TRACE
+  unsigned long long* trc =
+      (p.trace != nullptr && blockIdx.x < static_cast<unsigned>(kTraceCtas)) ? p.trace + blockIdx.x * kTraceSlots : nullptr;
+  const unsigned long long t_start = global_timer_ns();
+  long long acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#endif
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw;
@@ -228,7 +260,7 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
   }
   if (tid == 0 && !misaligned) {
     for (int b = 0; b < kNumPfBars; ++b)
-      mbar_init(&bars[b], (b == kBarSfree0 || b == kBarSfree0 + 1 || b == kBarP) ? 128u : 1u);
+      mbar_init(&bars[b], (b == kBarP0 || b == kBarP0 + 1) ? 128u : 1u);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -245,15 +277,21 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
   uint8_t* sQ = base + kPfSmemQ;
   uint8_t* sK = base + kPfSmemK;
   uint8_t* sV = base + kPfSmemV;
-  uint8_t* sP = base + kPfSmemP;
   const float sl2 = p.attn_scale_log2;
 
   if (warp == 4) {
     if (lane == 0 && m > 0) {
       // ---------------------------------------------------- producer / MMA issuer
-      const uint32_t idesc_qk = umma_idesc_bf16(128, 64, false, false);
-      const uint32_t idesc_pv = umma_idesc_bf16(128, 128, false, true);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
+#ifdef SAS_PHASE_TRACE
+      const long long t_prod0 = clock64();
+#endif
+      constexpr uint32_t idesc_qk = umma_idesc_bf16(128, 64, false, false);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 128, false, true);
+      // descriptors of the stage-0 operands; later k-steps and stages add
+      // their byte offset >> 4 to the start-address field
+      const uint64_t dQ = umma_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK = umma_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV = umma_desc_sw128(smem_u32(sV), 8192, 1024);
       const int rowq0 = static_cast<int>((static_cast<size_t>(s) * p.hq + g0) * p.T) + kBlock * i;
       const int rowq1 = rowq0 + p.T;
       const int rowkv = static_cast<int>((static_cast<size_t>(s) * p.hkv + h) * p.T);
@@ -263,108 +301,128 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
       tma_load_2d(sQ + 16384, &tmq, 64, rowq0, &bars[kBarQ]);
       tma_load_2d(sQ + 24576, &tmq, 64, rowq1, &bars[kBarQ]);
       auto load_k = [&](int e) {
-        const int st = e & 1;
+        const int st = e % kPfKStages;
         mbar_arrive_expect_tx(&bars[kBarK0 + st], 16384);
         const int row = rowkv + kBlock * sel_s[e];
         tma_load_2d(sK + st * 16384, &tmk, 0, row, &bars[kBarK0 + st]);
         tma_load_2d(sK + st * 16384 + 8192, &tmk, 64, row, &bars[kBarK0 + st]);
       };
       auto load_v = [&](int e) {
-        const int st = e & 1;
+        const int st = e % kPfVStages;
         mbar_arrive_expect_tx(&bars[kBarV0 + st], 16384);
         const int row = rowkv + kBlock * sel_s[e];
         tma_load_2d(sV + st * 16384, &tmv, 0, row, &bars[kBarV0 + st]);
         tma_load_2d(sV + st * 16384 + 8192, &tmv, 64, row, &bars[kBarV0 + st]);
       };
-      auto issue_qk = [&](int e) {
-        const int st = e & 1;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = umma_desc_sw128(aQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t b = umma_desc_sw128(aK + st * 16384 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-          umma_bf16_ss(tmem + st * 64, a, b, idesc_qk, kk > 0);
-        }
-        umma_commit(&bars[kBarS0 + st]);
-      };
-      load_k(0);
-      load_v(0);
-      if (m > 1) {
-        load_k(1);
-        load_v(1);
-      }
-      mbar_wait(&bars[kBarQ], 0, p.status);
-      mbar_wait(&bars[kBarK0], 0, p.status);
-      tc_fence_after_sync();
-      issue_qk(0);
-      for (int e = 0; e < m; ++e) {
-        if (e + 1 < m) {
-          mbar_wait(&bars[kBarK0 + ((e + 1) & 1)], ((e + 1) >> 1) & 1, p.status);
-          if (e >= 1) mbar_wait(&bars[kBarSfree0 + ((e + 1) & 1)], ((e - 1) >> 1) & 1, p.status);
-          tc_fence_after_sync();
-          issue_qk(e + 1);
-        }
-        if (e + 2 < m) {
-          mbar_wait(&bars[kBarS0 + (e & 1)], (e >> 1) & 1, p.status);  // QK_e done: K slot free
-          load_k(e + 2);
-        }
-        mbar_wait(&bars[kBarP], e & 1, p.status);
-        mbar_wait(&bars[kBarV0 + (e & 1)], (e >> 1) & 1, p.status);
+      auto issue_qk = [&](int e) {  // K_e has landed, S[e % 2] is free
+        const int st = e % kPfKStages;
+        PF_TIC(tk);
+        mbar_wait(&bars[kBarK0 + st], (e / kPfKStages) & 1, p.status);
+        PF_TOC(acc[3], tk);
         tc_fence_after_sync();
+        PF_TIC(tiq);
+        const uint64_t dk = dK + static_cast<uint64_t>(st * (16384 >> 4));
+        const uint32_t d_tmem = tmem + (e & 1) * 64;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t a = umma_desc_sw128(aP + kk * 32, 16, 1024);
-          const uint64_t b = umma_desc_sw128(aV + (e & 1) * 16384 + kk * 2048, 8192, 1024);
-          umma_bf16_ss(tmem + 128, a, b, idesc_pv, e > 0 || kk > 0);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ss(d_tmem, dQ + static_cast<uint64_t>(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4),
+                       dk + static_cast<uint64_t>(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0);
+        umma_commit(&bars[kBarS0 + (e & 1)]);
+        PF_TOC(acc[6], tiq);
+      };
+      for (int e = 0; e < m && e < kPfKStages; ++e) load_k(e);
+      for (int e = 0; e < m && e < kPfVStages; ++e) load_v(e);
+      PF_TIC(tq);
+      mbar_wait(&bars[kBarQ], 0, p.status);
+      PF_TOC(acc[4], tq);
+      issue_qk(0);
+      if (m > 1) issue_qk(1);
+      for (int e = 0; e < m; ++e) {
+        // P_e written (and so S_e read, Q K_e done: its K slot is free)
+        PF_TIC(tp);
+        mbar_wait(&bars[kBarP0 + (e & 1)], (e >> 1) & 1, p.status);
+        PF_TOC(acc[0], tp);
+        if (e + kPfKStages < m) load_k(e + kPfKStages);
+        PF_TIC(tv);
+        mbar_wait(&bars[kBarV0 + e % kPfVStages], (e / kPfVStages) & 1, p.status);
+        PF_TOC(acc[1], tv);
+        tc_fence_after_sync();
+        PF_TIC(tip);
+        const uint32_t aP = tmem + (e & 1) * 64;
+        const uint64_t dv = dV + static_cast<uint64_t>((e % kPfVStages) * (16384 >> 4));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16_ts(tmem + 128, aP + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                       e > 0 || kk > 0);
         umma_commit(&bars[kBarO]);
+        PF_TOC(acc[5], tip);
         if (e + 2 < m) {
-          mbar_wait(&bars[kBarO], e & 1, p.status);  // PV_e done: V slot free
-          load_v(e + 2);
+          PF_TIC(to);
+          mbar_wait(&bars[kBarO], e & 1, p.status);  // P V_e done: V slot and S[e % 2] free
+          PF_TOC(acc[2], to);
+          if (e + kPfVStages < m) load_v(e + kPfVStages);
+          issue_qk(e + 2);
         }
       }
       mbar_wait(&bars[kBarO], (m - 1) & 1, p.status);  // nothing of ours in flight at teardown
+#ifdef SAS_PHASE_TRACE
+      if (trc != nullptr) {
+        for (int k = 0; k < 5; ++k) trc[2 + k] = static_cast<unsigned long long>(acc[k]);
+        trc[12] = static_cast<unsigned long long>(acc[5]);
+        trc[13] = static_cast<unsigned long long>(acc[6]);
+        trc[14] = static_cast<unsigned long long>(clock64() - t_prod0);
+      }
+#endif
     }
   } else {
     // ------------------------------------------------------ softmax / epilogue
     const int r = tid;            // query row: head g0 + (r >> 6), token r & 63
     const int t = r & 63;
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;  // running maximum in log2 units, row sum
     for (int e = 0; e < m; ++e) {
+      PF_TIC(ts);
       mbar_wait(&bars[kBarS0 + (e & 1)], (e >> 1) & 1, p.status);
+      PF_TOC(acc[5], ts);
+      PF_TIC(tc);
       tc_fence_after_sync();
       float sv[64];
       tmem_ld32(tl + (e & 1) * 64, sv);
       tmem_ld32(tl + (e & 1) * 64 + 32, sv + 32);
       tmem_wait_ld();
-      tc_fence_before_sync();
-      mbar_arrive(&bars[kBarSfree0 + (e & 1)]);
-      const bool diag = (sel_s[e] == i);
-      float mx = -INFINITY;
+      if (e == m - 1) {  // the diagonal block: causal mask
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const float x = (diag && j > t) ? -INFINITY : sv[j] * sl2;
-        sv[j] = x;
-        mx = fmaxf(mx, x);
+        for (int j = 0; j < 64; ++j)
+          if (j > t) sv[j] = -INFINITY;
       }
+      float mx0 = fmax3(sv[0], sv[1], sv[2]), mx1 = fmax3(sv[3], sv[4], sv[5]);
+#pragma unroll
+      for (int j = 6; j < 62; j += 4) {
+        mx0 = fmax3(mx0, sv[j], sv[j + 1]);
+        mx1 = fmax3(mx1, sv[j + 2], sv[j + 3]);
+      }
+      const float mx = fmax3(mx0, mx1, fmaxf(sv[62], sv[63])) * sl2;
       const float m_new = fmaxf(m_run, mx);
       // rescale O only when the running maximum grows by more than 2^8:
       // probabilities stay below 256 in between, exact after normalisation
       const bool resc = (m_new > m_run + 8.f);
       const float m_use = resc ? m_new : m_run;
-      float rs = 0.f;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[32];
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const float pj = (sv[j] == -INFINITY) ? 0.f : exp2f(sv[j] - m_use);
-        sv[j] = pj;
-        rs += pj;
+      for (int j = 0; j < 64; j += 2) {
+        const float p0 = exp2_approx(fmaf(sv[j], sl2, -m_use));
+        const float p1 = exp2_approx(fmaf(sv[j + 1], sl2, -m_use));
+        rs[(j >> 1) & 3] += p0 + p1;
+        pk[j >> 1] = pack_bf16x2(p0, p1);
       }
-      if (e > 0) {
-        mbar_wait(&bars[kBarO], (e - 1) & 1, p.status);  // PV_{e-1} done: O and P free
-        tc_fence_after_sync();
-      }
-      const float alpha = resc ? exp2f(m_run - m_use) : 1.f;
+      const float alpha = exp2_approx(m_run - m_use);
       if (e > 0 && __any_sync(0xffffffffu, resc)) {
+#ifdef SAS_PHASE_TRACE
+        acc[7] += 1;
+#endif
+        mbar_wait(&bars[kBarO], (e - 1) & 1, p.status);  // P V_{e-1} done: O is stable
+        tc_fence_after_sync();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           float o[32];
@@ -374,24 +432,18 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
           for (int k = 0; k < 32; ++k) o[k] *= alpha;
           tmem_st32(tl + 128 + 32 * c, o);
         }
-        tmem_wait_st();
       }
-      l_run = l_run * alpha + rs;
-      m_run = m_use;
-      // P row r as bf16, 128-byte swizzled (chunk jc of row r at jc ^ (r & 7))
-#pragma unroll
-      for (int jc = 0; jc < 8; ++jc) {
-        uint4 pk;
-        pk.x = pack_bf16x2(sv[8 * jc + 0], sv[8 * jc + 1]);
-        pk.y = pack_bf16x2(sv[8 * jc + 2], sv[8 * jc + 3]);
-        pk.z = pack_bf16x2(sv[8 * jc + 4], sv[8 * jc + 5]);
-        pk.w = pack_bf16x2(sv[8 * jc + 6], sv[8 * jc + 7]);
-        *reinterpret_cast<uint4*>(sP + r * 128 + ((jc ^ (r & 7)) << 4)) = pk;
-      }
-      fence_proxy_async_smem();
+      tmem_st32(tl + (e & 1) * 64, pk);
+      tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(&bars[kBarP]);
+      mbar_arrive(&bars[kBarP0 + (e & 1)]);
+      PF_TOC(acc[6], tc);
+      l_run = l_run * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+      m_run = m_use;
     }
+#ifdef SAS_PHASE_TRACE
+    if (trc != nullptr && tid == 0) trc[11] = global_timer_ns();  // end of the tile loop
+#endif
     // epilogue: O / l, bf16, one row per thread
     __nv_bfloat16* dst = p.out + ((static_cast<size_t>(s) * p.hq + g0 + (r >> 6)) * p.T +
                                   static_cast<size_t>(i) * kBlock + t) * kDim;
@@ -422,6 +474,16 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
   __syncthreads();
   tc_fence_after_sync();
   if (warp == 0) tmem_dealloc(tmem, kPfTmemCols);
+#ifdef SAS_PHASE_TRACE
+  if (trc != nullptr && tid == 0) {
+    trc[0] = t_start;
+    trc[1] = global_timer_ns();
+    trc[7] = static_cast<unsigned long long>(acc[5]);
+    trc[8] = static_cast<unsigned long long>(acc[6]);
+    trc[9] = static_cast<unsigned long long>(acc[7]);
+    trc[10] = static_cast<unsigned long long>(m);
+  }
+#endif
 }
 
 // ------------------------------------------------------------ launchers
