@@ -87,7 +87,6 @@ __global__ void __launch_bounds__(kThreads, 4)
   static_assert(kDpc % 8 == 0, "cluster size must divide 128 into 16-byte slices");
 
   cg::cluster_group cluster = cg::this_cluster();
-  cluster_arrive_relaxed();  // matched by cluster_wait() before the first DSMEM store
   SAS_TRACE(0);
   const int rank = static_cast<int>(cluster.block_rank());
   const int pair = blockIdx.y;
@@ -111,6 +110,14 @@ __global__ void __launch_bounds__(kThreads, 4)
   uint64_t* bar_pro = bars + NST;     // prologue copies: q, W_q slice, gamma_q (, gamma_k)
   uint64_t* bar_p = bars + NST + 1;   // pooled current block has arrived (cluster scope)
   uint64_t* bar_wk = bars + NST + 2;  // W_k column slice has arrived
+  // Cluster exchanges: the sender stores into the receiver's shared memory
+  // with st.async, which completes the bytes on the receiver's barrier; the
+  // receiver registers the bytes it expects (its own single arrival).
+  uint64_t* bar_sc = bars + NST + 3;  // rank 0: the scores of every CTA
+  uint64_t* bar_sel = bars + NST + 4; // ranks > 0: the block list from rank 0
+  uint64_t* bar_v = bars + NST + 5;   // the gate query v (a slice from each CTA)
+  uint64_t* bar_m = bars + NST + 6;   // attention partials of this CTA's columns
+  uint64_t* bar_u = bars + NST + 7;   // rank 0: projected pooled slices
   float* pool_p = reinterpret_cast<float*>(base + p.sm.r_pool_p);
   float* pool_u = reinterpret_cast<float*>(base + p.sm.r_pool_u);
   __nv_bfloat16* wk_s = reinterpret_cast<__nv_bfloat16*>(base + p.sm.r_wk);
@@ -129,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   // first, asynchronously: q of the group (bulk), the W_q column slice of
   // this CTA (one 2-D TMA box per head) and gamma_q (bulk).
   if (tid == 0) {
-    for (int i = 0; i < NST + 3; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < NST + 8; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
     const uint32_t qbytes = static_cast<uint32_t>(G * kDim * sizeof(T));
     uint32_t tx = qbytes;
@@ -146,6 +153,9 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
     if (pool_on) bulk_g2s(gamk_s, p.gamma_k, kDim * 4, bar_pro);
   }
+  // thread 0 arrives after its barrier initialisation: no CTA of the cluster
+  // passes cluster_wait() (and stores into this one) before it
+  cluster_arrive_relaxed();
   double th0 = 0.0, th1 = 0.0;
   if (MODE != kModeAttend) {
     th0 = p.rope.theta_over_pi[lane];
@@ -193,6 +203,22 @@ __global__ void __launch_bounds__(kThreads, 4)
   const int nchunks = (MODE == kModeAttend) ? 0 : (b_hi - b_lo + kGkChunk - 1) / kGkChunk;
   const int cnt_mine = (rank < m) ? (m - 1 - rank) / CS + 1 : 0;
   const bool own_cur = (m > 0) && ((m - 1) % CS == rank);
+
+  // bytes this CTA will receive from the cluster (bad is uniform over it)
+  if (tid == 0) {
+    if (MODE != kModeAttend && !bad) mbar_arrive_expect_tx(bar_v, static_cast<uint32_t>(G * kDim * 4));
+    if (MODE == kModeFused && !bad) {
+      if (rank == 0)
+        mbar_arrive_expect_tx(bar_sc, static_cast<uint32_t>(n * 4));
+      else
+        mbar_arrive_expect_tx(bar_sel, static_cast<uint32_t>(m * 4));
+    }
+    if (do_pool) {
+      mbar_arrive_expect_tx(bar_p, kPool * 4);
+      if (rank == 0) mbar_arrive_expect_tx(bar_u, CS * 17 * 4);
+    }
+    if (MODE != kModeGate) mbar_arrive_expect_tx(bar_m, static_cast<uint32_t>(CS * G * (kDpc + 2) * 4));
+  }
 
   // list entry e of this CTA -> block id (the current block first if owned)
   auto entry_block = [&](int e) -> int {
@@ -257,8 +283,9 @@ __global__ void __launch_bounds__(kThreads, 4)
   // ------------------------------------------------------------ phase 0: gate query
   const bool pro_ok = mbar_wait(bar_pro, 0, p.status);
   cluster_wait();  // every CTA of the cluster is running
-  if (MODE != kModeAttend && !bad && pro_ok) {
-    // two threads per output column (rows 0..63 and 64..127), combined by shuffle
+  if (MODE != kModeAttend && !bad) {
+    // two threads per output column (rows 0..63 and 64..127), combined by
+    // shuffle; every CTA of the cluster receives every column
     for (int o = tid; o < 2 * G * kDpc; o += kThreads) {
       const int half = o & 1;
       const int oc = o >> 1;
@@ -267,18 +294,21 @@ __global__ void __launch_bounds__(kThreads, 4)
       const T* qrow = qraw + g * kDim + half * 64;
       const __nv_bfloat16* wcol = wq_s + (static_cast<size_t>(g) * kDim + half * 64) * kDpc + j;
       float a4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (pro_ok) {
 #pragma unroll 16
-      for (int i = 0; i < 64; ++i)
-        a4[i & 3] = fmaf(to_float(qrow[i]), __bfloat162float(wcol[i * kDpc]), a4[i & 3]);
+        for (int i = 0; i < 64; ++i)
+          a4[i & 3] = fmaf(to_float(qrow[i]), __bfloat162float(wcol[i * kDpc]), a4[i & 3]);
+      }
       float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       if (half == 0) {
 #pragma unroll
-        for (int r = 0; r < CS; ++r) cluster.map_shared_rank(qv, r)[g * kDim + rank * kDpc + j] = acc;
+        for (int r = 0; r < CS; ++r)
+          st_async_f32(dsmem_addr(qv + g * kDim + rank * kDpc + j, r), acc, dsmem_addr(bar_v, r));
       }
     }
+    mbar_wait_cluster(bar_v, 0, p.status);  // every column of v is here
   }
-  cluster.sync();  // #1: every CTA holds all of v
   SAS_TRACE(2);
 
   if (MODE != kModeAttend) {
@@ -351,9 +381,8 @@ __global__ void __launch_bounds__(kThreads, 4)
           acc += __shfl_xor_sync(0xffffffffu, acc, 2);
           acc += __shfl_xor_sync(0xffffffffu, acc, 4);
           S = acc;
-          // every CTA of the cluster receives every score (lane `sub` -> rank sub)
-          if (act)
-            for (int r = sub; r < CS; r += 8) cluster.map_shared_rank(keys, r)[b0 + bb] = S;
+          // rank 0 of the cluster receives every score and selects
+          if (sub == 0 && bb < cntb) st_async_f32(dsmem_addr(keys + b0 + bb, 0), S, dsmem_addr(bar_sc, 0));
         } else {
           for (int g = 0; g < G; ++g) {
             float acc = 0.f;
@@ -384,38 +413,65 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
   }
   SAS_TRACE(3);
-  if (MODE == kModeGate) return;  // no DSMEM access after barrier #1
+  if (MODE == kModeGate) return;  // everything sent to this CTA (v) has arrived
 
   // ------------------------------------------------------------ phase 2: Top-K
+  // Rank 0 selects once for the cluster: every CTA signals rank 0 when its
+  // scores are in (release / acquire at cluster scope), rank 0 ranks them
+  // and sends the block list to every other CTA the same way.
   if (MODE == kModeFused) {
-    cluster.sync();  // #2: every score of the (seq, head) is in every CTA
     SAS_TRACE(4);
+    auto issue_wk = [&]() {
+      // this CTA's 16 columns of W_k[h] (384 rows as three 128-row boxes);
+      // they land over the key region, unused from here on
+      if (do_pool && tid == 0) {
+        mbar_arrive_expect_tx(bar_wk, kPool * kDpc * 2);
+        for (int part = 0; part < 3; ++part)
+          tma_load_2d(wk_s + part * 128 * kDpc, &tmwk, rank * kDpc, h * kPool + part * 128, bar_wk);
+      }
+    };
+    bool list_ok = true;
     if (!bad) {
-#ifdef SAS_PHASE_TRACE
-      unsigned long long* tr = (p.trace != nullptr && blockIdx.y * gridDim.x + blockIdx.x < kTraceCtas)
-                                   ? p.trace + (blockIdx.y * gridDim.x + blockIdx.x) * kTraceSlots + 10
-                                   : nullptr;
-#else
-      unsigned long long* tr = nullptr;
-#endif
-      select_blocks(keys, n, p.topk, c, sel, hist, selbits, scan, tr);
       if (rank == 0) {
-        if (p.sel_idx != nullptr)
-          for (int j = tid; j < m; j += kThreads)
-            p.sel_idx[static_cast<size_t>(pair) * p.max_sel + j] = sel[j];
-        if (p.sel_count != nullptr && tid == 0) p.sel_count[pair] = m;
+        list_ok = mbar_wait_cluster(bar_sc, 0, p.status);
+        SAS_TRACE(9);  // rank 0: every score of the cluster is in
+#ifdef SAS_PHASE_TRACE
+        unsigned long long* tr = (p.trace != nullptr && blockIdx.y * gridDim.x + blockIdx.x < kTraceCtas)
+                                     ? p.trace + (blockIdx.y * gridDim.x + blockIdx.x) * kTraceSlots + 10
+                                     : nullptr;
+#else
+        unsigned long long* tr = nullptr;
+#endif
+        list_ok = __syncthreads_and(list_ok) != 0;
+        if (list_ok) {
+          select_blocks(keys, n, p.topk, c, sel, hist, selbits, scan, tr);
+        } else {  // scores missing (timeout, in the status word): a valid stand-in list
+          for (int j = tid; j < m; j += kThreads) sel[j] = c;
+          __syncthreads();
+        }
+        for (int j = tid; j < m; j += kThreads) {
+          const int b = sel[j];
+          for (int r = 1; r < CS; ++r)
+            st_async_u32(dsmem_addr(sel + j, r), static_cast<uint32_t>(b), dsmem_addr(bar_sel, r));
+          if (p.sel_idx != nullptr) p.sel_idx[static_cast<size_t>(pair) * p.max_sel + j] = b;
+        }
+        if (p.sel_count != nullptr && tid == 0) p.sel_count[pair] = list_ok ? m : 0;
+        issue_wk();
+      } else {
+        issue_wk();
+        list_ok = mbar_wait_cluster(bar_sel, 0, p.status);
       }
     } else if (rank == 0 && tid == 0 && p.sel_count != nullptr) {
       p.sel_count[pair] = 0;
     }
+    // a list that never came (timeout, already in the status word) is not
+    // read: the current block, always valid, stands in for every entry
+    if (__syncthreads_and(list_ok) == 0) {
+      for (int j = tid; j < m; j += kThreads) sel[j] = c;
+      __syncthreads();
+    }
     known = nchunks + kTilesPerBlock * cnt_mine;
     pump(nchunks, known);
-    if (do_pool && tid == 0) {
-      // this CTA's 16 columns of W_k[h] (384 rows as three 128-row boxes)
-      mbar_arrive_expect_tx(bar_wk, kPool * kDpc * 2);
-      for (int part = 0; part < 3; ++part)
-        tma_load_2d(wk_s + part * 128 * kDpc, &tmwk, rank * kDpc, h * kPool + part * 128, bar_wk);
-    }
     SAS_TRACE(5);
   }
 
@@ -483,16 +539,14 @@ __global__ void __launch_bounds__(kThreads, 4)
         sm *= (1.f / kBlock);
 #pragma unroll
         for (int r = 0; r < CS; ++r) {
-          float* dst = cluster.map_shared_rank(pool_p, r);
-          dst[d] = mx;
-          dst[kDim + d] = mn;
-          dst[2 * kDim + d] = sm;
+          const uint32_t rb = dsmem_addr(bar_p, r);
+          st_async_f32(dsmem_addr(pool_p + d, r), mx, rb);
+          st_async_f32(dsmem_addr(pool_p + kDim + d, r), mn, rb);
+          st_async_f32(dsmem_addr(pool_p + 2 * kDim + d, r), sm, rb);
         }
-        fence_acq_rel_cluster();
       }
       __syncthreads();
       pump(t0 + 1, known);
-      if (pool_here && tid < CS) mbar_remote_arrive(bar_p, tid);
       // ---- online softmax (per warp, head gq)
       float x[2][2];
       float mx = -INFINITY;
@@ -598,16 +652,14 @@ __global__ void __launch_bounds__(kThreads, 4)
         sm *= (1.f / kBlock);
 #pragma unroll
         for (int r = 0; r < CS; ++r) {
-          float* dst = cluster.map_shared_rank(pool_p, r);
-          dst[d] = mx;
-          dst[kDim + d] = mn;
-          dst[2 * kDim + d] = sm;
+          const uint32_t rb = dsmem_addr(bar_p, r);
+          st_async_f32(dsmem_addr(pool_p + d, r), mx, rb);
+          st_async_f32(dsmem_addr(pool_p + kDim + d, r), mn, rb);
+          st_async_f32(dsmem_addr(pool_p + 2 * kDim + d, r), sm, rb);
         }
-        fence_acq_rel_cluster();
       }
       __syncthreads();
       pump(t0 + 2, known);
-      if (pool_here && tid < CS) mbar_remote_arrive(bar_p, tid);
       float pg[kMaxGroup];
 #pragma unroll
       for (int g = 0; g < kMaxGroup; ++g) {
@@ -699,8 +751,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     const int d = tid;
     const int dst = d / kDpc;
     const int dd = d - dst * kDpc;
-    float* rin_o = cluster.map_shared_rank(inbox_o, dst);
-    float* rin_ml = cluster.map_shared_rank(inbox_ml, dst);
+    const uint32_t rb = dsmem_addr(bar_m, dst);
     for (int g = 0; g < G; ++g) {
       float M = -INFINITY;
 #pragma unroll
@@ -714,17 +765,17 @@ __global__ void __launch_bounds__(kThreads, 4)
           osum = fmaf(po[(static_cast<size_t>(w) * G + g) * kDim + d], f, osum);
         }
       }
-      rin_o[(rank * G + g) * kDpc + dd] = osum;
+      st_async_f32(dsmem_addr(inbox_o + (rank * G + g) * kDpc + dd, dst), osum, rb);
       if (dd == 0) {
-        rin_ml[(rank * G + g) * 2 + 0] = M;
-        rin_ml[(rank * G + g) * 2 + 1] = lsum;
+        st_async_f32(dsmem_addr(inbox_ml + (rank * G + g) * 2 + 0, dst), M, rb);
+        st_async_f32(dsmem_addr(inbox_ml + (rank * G + g) * 2 + 1, dst), lsum, rb);
       }
     }
   }
   if (do_pool) {
     // u = P @ W_k[h] for this CTA's 16 columns; slices and their sums of
-    // squares go to CTA 0, which normalises and rotates after barrier #3
-    const bool okp = mbar_wait_cluster(bar_p, 0, p.status);
+    // squares go to CTA 0, which normalises and rotates once all have come
+    const bool okp = mbar_wait_cluster(bar_p, 0, p.status);  // the pooled block
     const bool okw = mbar_wait(bar_wk, 0, p.status);
     const int j = tid & (kDpc - 1);
     const int rg = tid / kDpc;  // kThreads / kDpc row groups
@@ -746,12 +797,13 @@ __global__ void __launch_bounds__(kThreads, 4)
       float sq = u * u;
 #pragma unroll
       for (int o = kDpc / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0x0000ffffu, sq, o);
-      float* dst = cluster.map_shared_rank(pool_u, 0);
-      dst[rank * 17 + tid] = u;
-      if (tid == 0) dst[rank * 17 + 16] = sq;
+      const uint32_t rb = dsmem_addr(bar_u, 0);
+      st_async_f32(dsmem_addr(pool_u + rank * 17 + tid, 0), u, rb);
+      if (tid == 0) st_async_f32(dsmem_addr(pool_u + rank * 17 + 16, 0), sq, rb);
     }
   }
-  cluster.sync();  // #3: every partial of this CTA's columns has arrived
+  mbar_wait_cluster(bar_m, 0, p.status);  // every partial of this CTA's columns
+  __syncthreads();                         // qbar is reused below
   SAS_TRACE(7);
   {
     OutT* out = static_cast<OutT*>(p.out);
@@ -781,6 +833,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   }
   if (do_pool && rank == 0) {
     // RMSNorm (gain gamma_k) and gate RoPE at position c of the pooled block
+    mbar_wait_cluster(bar_u, 0, p.status);
     const int d = tid;
     float ss = 0.f;
 #pragma unroll

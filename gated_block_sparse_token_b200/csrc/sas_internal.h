@@ -19,10 +19,11 @@ enum DecodeMode : int { kModeGate = 0, kModeAttend = 1, kModeFused = 2 };
 //   phases 0-1  [ qv | wq | qs ]
 //   phases 2-4  [ inbox | pool P | pool u | keys | hist | selbits | scan ]
 //               with the W_k slice of the fused pooling over keys.. once the
-//               selection is done
+//               selection is done (rank 0) or the scores are sent (others)
 // inbox (written by other CTAs after the attention phase) covers at least
-// qv, and keys (written by other CTAs during their phase 1) starts past the
-// inbox, so no remote write can land on data this CTA still reads.
+// qv, and keys (written by the other CTAs of the cluster into rank 0 during
+// their phase 1) starts past the inbox, so no remote write can land on data
+// this CTA still reads.
 constexpr int kSelBins = 1024;  // value buckets of the Top-K selection
 constexpr int kSelCand = 256;   // candidates ranked exactly in the boundary bucket
 
@@ -41,7 +42,7 @@ struct DecodeSmem {
   int r_pool_u;  // fp32 [CS][17] projected slices + sum of squares  (phases 3-4)
   int r_wk;      // bf16 [384][dpc] W_k column slice (TMA)           (phases 3-4)
   int gamk;      // fp32 [128] gamma_k (bulk copy, fused pooling)
-  int r_keys;    // fp32 scores -> uint32 keys [mg]                 (phases 1-2)
+  int r_keys;    // fp32 scores -> uint32 keys [mg] (rank 0)        (phases 1-2)
   int r_hist;    // uint32 [kSelBins], then int32 candidates        (phase 2)
   int r_selbits; // uint32 [(mg + 31) / 32]                         (phase 2)
   int r_scan;    // int32 [16]                                      (phase 2)
@@ -67,7 +68,9 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
   p.pml = take(2 * kWarps * kMaxGroup * 4, 16);
   p.gam = take(kDim * 4, 16);
   p.gamk = take(kDim * 4, 16);
-  p.bars = take((nst + 3) * 8, 8);  // ring slots, prologue, pooled P ready, W_k slice
+  // ring slots, prologue, pooled P, W_k slice, scores (rank 0), list, v,
+  // attention partials, pooled slices (rank 0)
+  p.bars = take((nst + 8) * 8, 8);
   auto up128 = [](int x) { return (x + 127) / 128 * 128; };
   const int r = up128(off);
   // phases 0-1 (the W_q slice is a tensor-TMA destination: 128-byte aligned)

@@ -6,23 +6,6 @@
 namespace sas {
 namespace {
 
-// Exclusive prefix sum of v over the kThreads threads (thread order).
-__device__ __forceinline__ int block_exclusive_scan(int v, int* scan) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += y;
-  }
-  if (lane == 31) scan[warp] = inc;
-  __syncthreads();
-  int off = 0;
-  for (int w = 0; w < warp; ++w) off += scan[w];
-  __syncthreads();
-  return off + inc - v;
-}
-
 // Top-K selection (pages: training Top-K 31 under the 2,048-token budget).
 // Keeps the min(topk, n) largest of vals[0..n) -- ties go to the lower index
 // -- lists them ascending in sel[], appends the current block `cur` and
@@ -30,9 +13,14 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scan) {
 // which fall into kSelBins buckets by a monotone map (the leading 10 bits of
 // key - min key); the bucket holding the topk-th key is found from the
 // histogram, every bucket above it is kept, and the members of that bucket
-// are ranked exactly by (key descending, index ascending).  One warp does the
-// work with ballots and warp reductions (no CTA barrier inside); all threads
-// of the CTA call it and meet at the final barrier.  Overwrites vals with keys.
+// are ranked exactly by (key descending, index ascending).
+//
+// All kThreads threads take part; thread t owns the contiguous index range
+// [t * per, (t + 1) * per) with per a multiple of 4 (16-byte key loads), so
+// the final ascending list comes from one block-wide prefix sum.  vals must
+// be 16-byte aligned with room for ceil(n / 4) * 4 entries; it is
+// overwritten with the keys.  hist needs kSelBins words, selbits
+// ceil(n / 32) words, scan 16 words.
 __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
                              uint32_t* selbits, int* scan, unsigned long long* tr = nullptr) {
 #ifdef SAS_PHASE_TRACE
@@ -41,8 +29,9 @@ __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, ui
 #else
 #define SEL_TRACE(k, v)
 #endif
-  (void)scan;
-  const int tid = threadIdx.x, lane = tid & 31;
+  static_assert(kThreads == 128 && kSelBins == 8 * kThreads, "one thread per 8 histogram bins");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned full = 0xffffffffu;
   if (topk <= 0) {  // a 64-token budget keeps the current block only
     if (tid == 0) sel[0] = cur;
     __syncthreads();
@@ -54,160 +43,185 @@ __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, ui
     __syncthreads();
     return n + 1;
   }
-  if (tid < 32) {
-    const unsigned full = 0xffffffffu;
-    const unsigned lt = (1u << lane) - 1u;
-    uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
-    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-    for (int base = 0; base < n; base += 128) {
-      float v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + 32 * u + lane;
-        v[u] = (i < n) ? vals[i] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + 32 * u + lane;
-        if (i < n) {
-          const uint32_t k = order_key(v[u]);
-          keys[i] = k;
-          lo = min(lo, k);
-          hi = max(hi, k);
-        }
-      }
-    }
-    for (int i = lane; i < kSelBins; i += 32) hist[i] = 0u;
-    for (int i = lane; i < (n + 31) / 32; i += 32) selbits[i] = 0u;
-    lo = __reduce_min_sync(full, lo);
-    hi = __reduce_max_sync(full, hi);
-    const int shift = max(0, 32 - __clz(static_cast<int>((hi - lo) | 1u)) - 10);
-    __syncwarp();
-    SEL_TRACE(0, global_timer_ns());
-    for (int base = 0; base < n; base += 128) {
-      uint32_t kk[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + 32 * u + lane;
-        kk[u] = (i < n) ? keys[i] : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (base + 32 * u + lane < n) atomicAdd(&hist[(kk[u] - lo) >> shift], 1u);
-    }
-    __syncwarp();
-    SEL_TRACE(1, global_timer_ns());
-    // buckets in descending order, 32 groups of 32: lane g sums group g
-    uint32_t gsum = 0u;
-#pragma unroll 8
-    for (int g = 0; g < kSelBins / 32; ++g) {
-      const uint32_t v = __reduce_add_sync(full, hist[kSelBins - 1 - 32 * g - lane]);
-      if (lane == g) gsum = v;
-    }
-    uint32_t ginc = gsum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(full, ginc, o);
-      if (lane >= o) ginc += y;
-    }
-    const uint32_t want = static_cast<uint32_t>(topk);
-    const unsigned hitg = __ballot_sync(full, ginc - gsum < want && want <= ginc);
-    const int gstar = __ffs(hitg) - 1;
-    const uint32_t gexcl = __shfl_sync(full, ginc - gsum, gstar);
-    const uint32_t bc = hist[kSelBins - 1 - 32 * gstar - lane];  // lane i: i-th bucket of the group
-    uint32_t binc = bc;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(full, binc, o);
-      if (lane >= o) binc += y;
-    }
-    const unsigned hitb = __ballot_sync(full, gexcl + binc - bc < want && want <= gexcl + binc);
-    const int lstar = __ffs(hitb) - 1;
-    const uint32_t bstar = static_cast<uint32_t>(kSelBins - 1 - 32 * gstar - lstar);
-    const int take = static_cast<int>(want - gexcl - __shfl_sync(full, binc - bc, lstar));
-    __syncwarp();
-    SEL_TRACE(2, global_timer_ns());
-    // members of the boundary bucket (the histogram is no longer needed)
-    int* cand = reinterpret_cast<int*>(hist);
-    int nc = 0;
-    for (int base = 0; base < n; base += 128) {
-      uint32_t kk[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + 32 * u + lane;
-        kk[u] = (i < n) ? keys[i] : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + 32 * u + lane;
-        const bool in = i < n && ((kk[u] - lo) >> shift) == bstar;
-        const unsigned bal = __ballot_sync(full, in);
-        if (in) {
-          const int pos = nc + __popc(bal & lt);
-          if (pos < kSelCand) cand[pos] = i;
-        }
-        nc += __popc(bal);
-      }
-    }
-    __syncwarp();
-    SEL_TRACE(3, global_timer_ns());
-    SEL_TRACE(5, static_cast<unsigned long long>(nc));
-    if (nc <= kSelCand) {
-      for (int ci = lane; ci < nc; ci += 32) {
-        const int i = cand[ci];
-        const uint32_t ki = keys[i];
-        int r = 0;
-        for (int cj = 0; cj < nc; ++cj) {
-          const int j = cand[cj];
-          const uint32_t kj = keys[j];
-          r += (kj > ki || (kj == ki && j < i)) ? 1 : 0;
-        }
-        if (r < take) atomicOr(&selbits[i >> 5], 1u << (i & 31));
-      }
+  uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
+  const int per = (n + 4 * kThreads - 1) / (4 * kThreads) * 4;
+  const int i0 = tid * per;
+  const int i1 = min(n, i0 + per);
+
+  // ---- keys, their range; clear the histogram, the marks and the counter
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int i = i0; i < i1; i += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(vals + i);
+    uint4 k;
+    k.x = order_key(v.x);
+    k.y = order_key(v.y);
+    k.z = order_key(v.z);
+    k.w = order_key(v.w);
+    if (i + 3 < n) {
+      *reinterpret_cast<uint4*>(keys + i) = k;
+      lo = min(min(lo, min(k.x, k.y)), min(k.z, k.w));
+      hi = max(max(hi, max(k.x, k.y)), max(k.z, k.w));
     } else {
-      // a crowded boundary bucket (many equal scores): rank against all members
-      for (int i = lane; i < n; i += 32) {
-        const uint32_t ki = keys[i];
-        if (((ki - lo) >> shift) != bstar) continue;
-        int r = 0;
-        for (int j = 0; j < n; ++j) {
-          const uint32_t kj = keys[j];
-          r += (((kj - lo) >> shift) == bstar && (kj > ki || (kj == ki && j < i))) ? 1 : 0;
-        }
-        if (r < take) atomicOr(&selbits[i >> 5], 1u << (i & 31));
+      const uint32_t kk[4] = {k.x, k.y, k.z, k.w};
+      for (int u = 0; u < n - i; ++u) {
+        keys[i + u] = kk[u];
+        lo = min(lo, kk[u]);
+        hi = max(hi, kk[u]);
       }
     }
-    __syncwarp();
-    SEL_TRACE(4, global_timer_ns());
-    // ascending list: every bucket above the boundary plus the marked members
-    int pos = 0;
-    for (int base = 0; base < n; base += 128) {
-      uint32_t kk[4], sb[4];
+  }
+  *reinterpret_cast<uint4*>(hist + 8 * tid) = make_uint4(0u, 0u, 0u, 0u);
+  *reinterpret_cast<uint4*>(hist + 8 * tid + 4) = make_uint4(0u, 0u, 0u, 0u);
+  for (int w = tid; w < (n + 31) / 32; w += kThreads) selbits[w] = 0u;
+  lo = __reduce_min_sync(full, lo);
+  hi = __reduce_max_sync(full, hi);
+  if (lane == 0) {
+    scan[warp] = static_cast<int>(lo);
+    scan[4 + warp] = static_cast<int>(hi);
+  }
+  if (tid == 0) scan[10] = 0;  // candidate counter
+  __syncthreads();
+  lo = min(min(static_cast<uint32_t>(scan[0]), static_cast<uint32_t>(scan[1])),
+           min(static_cast<uint32_t>(scan[2]), static_cast<uint32_t>(scan[3])));
+  hi = max(max(static_cast<uint32_t>(scan[4]), static_cast<uint32_t>(scan[5])),
+           max(static_cast<uint32_t>(scan[6]), static_cast<uint32_t>(scan[7])));
+  const int shift = max(0, 32 - __clz(static_cast<int>((hi - lo) | 1u)) - 10);
+  SEL_TRACE(0, global_timer_ns());
+
+  // ---- histogram of buckets
+  for (int i = i0; i < i1; ++i) atomicAdd(&hist[(keys[i] - lo) >> shift], 1u);
+  __syncthreads();
+  SEL_TRACE(1, global_timer_ns());
+
+  // ---- boundary bucket: thread t sums buckets 1023-8t .. 1016-8t (descending)
+  const int hb = kSelBins - 8 * (tid + 1);
+  const uint4 h0 = *reinterpret_cast<const uint4*>(hist + hb);
+  const uint4 h1 = *reinterpret_cast<const uint4*>(hist + hb + 4);
+  const uint32_t hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+  const int want = topk;
+  {
+    int sum = 0;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + 32 * u + lane;
-        kk[u] = (i < n) ? keys[i] : 0u;
-        sb[u] = (i < n) ? selbits[i >> 5] : 0u;
-      }
+    for (int j = 0; j < 8; ++j) sum += static_cast<int>(hv[j]);
+    int inc = sum;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + 32 * u + lane;
-        bool keep = false;
-        if (i < n) {
-          const uint32_t b = (kk[u] - lo) >> shift;
-          keep = b > bstar || (b == bstar && ((sb[u] >> (i & 31)) & 1u));
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(full, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) scan[12 + warp] = inc;
+    __syncthreads();
+    int excl = inc - sum;
+    for (int w = 0; w < warp; ++w) excl += scan[12 + w];
+    if (excl < want && want <= excl + sum) {
+      int cum = excl;
+#pragma unroll
+      for (int j = 7; j >= 0; --j) {
+        const int hj = static_cast<int>(hv[j]);
+        if (cum < want && want <= cum + hj) {
+          scan[8] = hb + j;      // the boundary bucket
+          scan[9] = want - cum;  // members of it to keep
         }
-        const unsigned bal = __ballot_sync(full, keep);
-        if (keep) sel[pos + __popc(bal & lt)] = i;
-        pos += __popc(bal);
+        cum += hj;
       }
     }
-    if (lane == 0) sel[topk] = cur;
+  }
+  __syncthreads();
+  const uint32_t bstar = static_cast<uint32_t>(scan[8]);
+  const int take = scan[9];
+  SEL_TRACE(2, global_timer_ns());
+
+  // ---- members of the boundary bucket, with their keys (the histogram is done)
+  int* cand = reinterpret_cast<int*>(hist);
+  uint32_t* candk = hist + kSelCand;
+  {
+    int cnt = 0;
+    for (int i = i0; i < i1; ++i) cnt += (((keys[i] - lo) >> shift) == bstar) ? 1 : 0;
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(full, inc, o);
+      if (lane >= o) inc += y;
+    }
+    int base = 0;
+    if (lane == 31 && inc > 0) base = atomicAdd(&scan[10], inc);
+    base = __shfl_sync(full, base, 31);
+    int pos = base + inc - cnt;
+    if (cnt > 0) {
+      for (int i = i0; i < i1; ++i) {
+        const uint32_t k = keys[i];
+        if (((k - lo) >> shift) == bstar) {
+          if (pos < kSelCand) {
+            cand[pos] = i;
+            candk[pos] = k;
+          }
+          ++pos;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int nc = scan[10];
+  SEL_TRACE(3, global_timer_ns());
+  SEL_TRACE(5, static_cast<unsigned long long>(nc));
+
+  // ---- exact rank inside the boundary bucket: (key descending, index ascending)
+  if (nc <= kSelCand) {
+    for (int ci = tid; ci < nc; ci += kThreads) {
+      const int i = cand[ci];
+      const uint32_t ki = candk[ci];
+      int r = 0;
+#pragma unroll 4
+      for (int cj = 0; cj < nc; ++cj) {
+        const uint32_t kj = candk[cj];
+        r += (kj > ki || (kj == ki && cand[cj] < i)) ? 1 : 0;
+      }
+      if (r < take) atomicOr(&selbits[i >> 5], 1u << (i & 31));
+    }
+  } else {
+    // a crowded boundary bucket (many equal scores): rank against all members
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t ki = keys[i];
+      if (((ki - lo) >> shift) != bstar) continue;
+      int r = 0;
+      for (int j = 0; j < n; ++j) {
+        const uint32_t kj = keys[j];
+        r += (((kj - lo) >> shift) == bstar && (kj > ki || (kj == ki && j < i))) ? 1 : 0;
+      }
+      if (r < take) atomicOr(&selbits[i >> 5], 1u << (i & 31));
+    }
+  }
+  __syncthreads();
+  SEL_TRACE(4, global_timer_ns());
+
+  // ---- ascending list: every bucket above the boundary plus the marked members
+  {
+    int cnt = 0;
+    for (int i = i0; i < i1; ++i) {
+      const uint32_t b = (keys[i] - lo) >> shift;
+      cnt += (b > bstar || (b == bstar && ((selbits[i >> 5] >> (i & 31)) & 1u))) ? 1 : 0;
+    }
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(full, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) scan[12 + warp] = inc;
+    __syncthreads();
+    int pos = inc - cnt;
+    for (int w = 0; w < warp; ++w) pos += scan[12 + w];
+    if (cnt > 0) {
+      for (int i = i0; i < i1; ++i) {
+        const uint32_t b = (keys[i] - lo) >> shift;
+        if (b > bstar || (b == bstar && ((selbits[i >> 5] >> (i & 31)) & 1u))) sel[pos++] = i;
+      }
+    }
+    if (tid == 0) sel[topk] = cur;
   }
   __syncthreads();
   return topk + 1;
 }
-
 
 }  // namespace
 }  // namespace sas
