@@ -64,18 +64,25 @@ def parse():
 
 
 # ---------------------------------------------------------------- distributed plumbing
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend=None):
+    """One process per GPU from the torchrun environment (RANK, LOCAL_RANK,
+    WORLD_SIZE, MASTER_ADDR/PORT).  NCCL on GPUs; gloo when asked (the CPU
+    tests of this plumbing).  The group carries only the barrier and the
+    max-reduce of timings."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    backend = backend or "nccl"
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return rank, world, local
 
@@ -87,13 +94,21 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """The largest of the ranks' values (timings are max over ranks)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank, world, seconds_max):
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's time."""
+    return world * units_per_rank / seconds_max
 
 
 # ---------------------------------------------------------------- measured peaks, clocks
@@ -242,7 +257,7 @@ def run_prefill(args, device, world):
     achieved = flops / t / 1e12
     return {"workload": spec.name, "batch_per_gpu": B, "seq_len": T, "q_heads": spec.hq,
             "kv_heads": spec.hkv, "token_budget": spec.token_budget, "steps": args.prefill_steps,
-            "ms_per_step": round(t * 1e3, 4), "tokens_per_s": round(world * B * T / t, 1),
+            "ms_per_step": round(t * 1e3, 4), "tokens_per_s": round(job_throughput(B * T, world, t), 1),
             "launches_per_step": 4,
             "roofline": {"kernel": "prefill_attn_kernel (tcgen05)", "bound": "tensor",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
@@ -439,7 +454,7 @@ def run_ours(args):
     dec_s = t_dec / args.steps
     achieved = dbytes / dec_s / 1e9
     step_s = t / args.steps
-    value = world * args.steps / t
+    value = job_throughput(args.steps, world, t)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 5),
@@ -457,7 +472,7 @@ def run_ours(args):
                      "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
                      "bytes_per_launch": dbytes, "avg_launch_us": round(dec_s * 1e6, 3),
                      "traffic": profiled_traffic()},
-        "e2e": {"value": round(world * ke / t_e2e, 2), "unit": UNIT,
+        "e2e": {"value": round(job_throughput(ke, world, t_e2e), 2), "unit": UNIT,
                 "h2d_bytes_per_step": BATCH * HQ * 128 * 2, "d2h_bytes_per_step": BATCH * HQ * 128 * 2},
         "gpu_launches": args.steps,
         "clocks": clocks,
@@ -522,7 +537,7 @@ def run_reference(args):
     r = reference_sample(steps=args.steps)
     value = r["value"]
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 / value, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
