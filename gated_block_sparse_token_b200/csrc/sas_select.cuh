@@ -6,6 +6,228 @@
 namespace sas {
 namespace {
 
+// Phase stamps of the selection (tracing builds only).
+#ifdef SAS_PHASE_TRACE
+#define SEL_TRACE(k, v) \
+  if (tr != nullptr && threadIdx.x == 0) tr[k] = (v)
+#else
+#define SEL_TRACE(k, v)
+#endif
+
+// Exact Top-K of n <= 4 * kThreads scores (every decode context up to 32,768
+// tokens), the short path: each thread keeps the keys of indices
+// 4t .. 4t+3 in registers; buckets are linear in the score value between the
+// finite minimum and maximum (monotone in key order: NaN and -inf fall in
+// bucket 0, +inf in the last), so the boundary bucket holds few members; the
+// kept set is a bit mask, turned into the ascending list by one warp.
+// Requires topk >= 1 and n > topk; same result as the general path.
+__device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
+                            uint32_t* selmask, int* scan, unsigned long long* tr) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned full = 0xffffffffu;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
+  const int i0 = 4 * tid;
+  float x[4];
+  uint32_t k[4];
+  bool valid[4];
+  {
+    const float4 v = (i0 < n) ? *reinterpret_cast<const float4*>(vals + i0) : make_float4(0.f, 0.f, 0.f, 0.f);
+    x[0] = v.x;
+    x[1] = v.y;
+    x[2] = v.z;
+    x[3] = v.w;
+  }
+  float fmn = INFINITY, fmx = -INFINITY;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    valid[u] = (i0 + u) < n;
+    k[u] = order_key(x[u]);
+    if (valid[u] && isfinite(x[u])) {
+      fmn = fminf(fmn, x[u]);
+      fmx = fmaxf(fmx, x[u]);
+    }
+  }
+  if (i0 + 3 < n) {
+    *reinterpret_cast<uint4*>(keys + i0) = make_uint4(k[0], k[1], k[2], k[3]);
+  } else {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (valid[u]) keys[i0 + u] = k[u];
+  }
+  *reinterpret_cast<uint4*>(hist + 8 * tid) = make_uint4(0u, 0u, 0u, 0u);
+  *reinterpret_cast<uint4*>(hist + 8 * tid + 4) = make_uint4(0u, 0u, 0u, 0u);
+  const int words = (n + 31) / 32;  // mask words (selmask holds this many)
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    fmn = fminf(fmn, __shfl_xor_sync(full, fmn, o));
+    fmx = fmaxf(fmx, __shfl_xor_sync(full, fmx, o));
+  }
+  float* red = reinterpret_cast<float*>(scan);
+  if (lane == 0) {
+    red[warp] = fmn;
+    red[4 + warp] = fmx;
+  }
+  if (tid == 0) scan[10] = 0;  // candidate counter
+  __syncthreads();
+  fmn = fminf(fminf(red[0], red[1]), fminf(red[2], red[3]));
+  fmx = fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]));
+  SEL_TRACE(0, global_timer_ns());
+  const float span = fmx - fmn;
+  const float scale = (span > 0.f && isfinite(span)) ? static_cast<float>(kSelBins - 1) / span : 0.f;
+  int bk[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    int b = 0;
+    if (isfinite(x[u]))
+      b = min(kSelBins - 1, static_cast<int>((x[u] - fmn) * scale));
+    else if (x[u] > 0.f)
+      b = kSelBins - 1;  // +inf; NaN and -inf stay in bucket 0
+    bk[u] = b;
+    if (valid[u]) atomicAdd(&hist[b], 1u);
+  }
+  __syncthreads();
+  SEL_TRACE(1, global_timer_ns());
+
+  // ---- boundary bucket: thread t sums buckets 1023-8t .. 1016-8t (descending)
+  const int hb = kSelBins - 8 * (tid + 1);
+  {
+    const uint4 h0 = *reinterpret_cast<const uint4*>(hist + hb);
+    const uint4 h1 = *reinterpret_cast<const uint4*>(hist + hb + 4);
+    const int hv[8] = {static_cast<int>(h0.x), static_cast<int>(h0.y), static_cast<int>(h0.z),
+                       static_cast<int>(h0.w), static_cast<int>(h1.x), static_cast<int>(h1.y),
+                       static_cast<int>(h1.z), static_cast<int>(h1.w)};
+    const int sum = ((hv[0] + hv[1]) + (hv[2] + hv[3])) + ((hv[4] + hv[5]) + (hv[6] + hv[7]));
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(full, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) scan[12 + warp] = inc;
+    __syncthreads();
+    int excl = inc - sum;
+    for (int w = 0; w < warp; ++w) excl += scan[12 + w];
+    if (excl < topk && topk <= excl + sum) {
+      int cum = excl;
+#pragma unroll
+      for (int j = 7; j >= 0; --j) {
+        if (cum < topk && topk <= cum + hv[j]) {
+          scan[8] = hb + j;      // the boundary bucket
+          scan[9] = topk - cum;  // members of it to keep
+        }
+        cum += hv[j];
+      }
+    }
+  }
+  __syncthreads();
+  const int bstar = scan[8];
+  const int take = scan[9];
+  SEL_TRACE(2, global_timer_ns());
+
+  // ---- kept-above bits (one 32-bit word per 8 threads) and boundary members
+  int* cand = reinterpret_cast<int*>(hist);
+  uint32_t* candk = hist + kSelCand;
+  {
+    uint32_t bits = 0u;
+    int cnt = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (valid[u] && bk[u] > bstar) bits |= 1u << (4 * (tid & 7) + u);
+      cnt += (valid[u] && bk[u] == bstar) ? 1 : 0;
+    }
+    bits |= __shfl_xor_sync(full, bits, 1);
+    bits |= __shfl_xor_sync(full, bits, 2);
+    bits |= __shfl_xor_sync(full, bits, 4);
+    if ((tid & 7) == 0 && (tid >> 3) < words) selmask[tid >> 3] = bits;
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(full, inc, o);
+      if (lane >= o) inc += y;
+    }
+    int base = 0;
+    if (lane == 31 && inc > 0) base = atomicAdd(&scan[10], inc);
+    base = __shfl_sync(full, base, 31);
+    int pos = base + inc - cnt;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (valid[u] && bk[u] == bstar) {
+        if (pos < kSelCand) {
+          cand[pos] = i0 + u;
+          candk[pos] = k[u];
+        }
+        ++pos;
+      }
+    }
+  }
+  __syncthreads();
+  const int nc = scan[10];
+  SEL_TRACE(3, global_timer_ns());
+  SEL_TRACE(5, static_cast<unsigned long long>(nc));
+
+  // ---- exact rank inside the boundary bucket: (key descending, index ascending)
+  if (nc <= kSelCand) {
+    for (int ci = tid; ci < nc; ci += kThreads) {
+      const int i = cand[ci];
+      const uint32_t ki = candk[ci];
+      int r = 0;
+      for (int cj = 0; cj < nc; ++cj) {
+        const uint32_t kj = candk[cj];
+        r += (kj > ki || (kj == ki && cand[cj] < i)) ? 1 : 0;
+      }
+      if (r < take) atomicOr(&selmask[i >> 5], 1u << (i & 31));
+    }
+  } else {
+    // a crowded boundary bucket (many equal scores): rank against all members
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (!(valid[u] && bk[u] == bstar)) continue;
+      const int i = i0 + u;
+      int r = 0;
+      for (int j = 0; j < n; ++j) {
+        const uint32_t kj = keys[j];
+        if (kj > k[u] || (kj == k[u] && j < i)) {
+          // member of the boundary bucket? (recomputed from the key's value)
+          const float xj = __uint_as_float((kj & 0x80000000u) ? (kj & 0x7FFFFFFFu) : ~kj);
+          int bj = 0;
+          if (kj == 0u)
+            bj = 0;
+          else if (isfinite(xj))
+            bj = min(kSelBins - 1, static_cast<int>((xj - fmn) * scale));
+          else if (xj > 0.f)
+            bj = kSelBins - 1;
+          r += (bj == bstar) ? 1 : 0;
+        }
+      }
+      if (r < take) atomicOr(&selmask[i >> 5], 1u << (i & 31));
+    }
+  }
+  __syncthreads();
+  SEL_TRACE(4, global_timer_ns());
+
+  // ---- ascending list from the mask (one warp: lane w owns word w)
+  if (warp == 0) {
+    const uint32_t wmask = (lane < words) ? selmask[lane] : 0u;
+    const int c = __popc(wmask);
+    int inc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(full, inc, o);
+      if (lane >= o) inc += y;
+    }
+    int pos = inc - c;
+    uint32_t mm = wmask;
+    while (mm != 0u) {
+      const int b = __ffs(mm) - 1;
+      sel[pos++] = 32 * lane + b;
+      mm &= mm - 1u;
+    }
+    if (lane == 0) sel[topk] = cur;
+  }
+  __syncthreads();
+  return topk + 1;
+}
+
 // Top-K selection (pages: training Top-K 31 under the 2,048-token budget).
 // Keeps the min(topk, n) largest of vals[0..n) -- ties go to the lower index
 // -- lists them ascending in sel[], appends the current block `cur` and
@@ -23,12 +245,6 @@ namespace {
 // ceil(n / 32) words, scan 16 words.
 __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
                              uint32_t* selbits, int* scan, unsigned long long* tr = nullptr) {
-#ifdef SAS_PHASE_TRACE
-#define SEL_TRACE(k, v) \
-  if (tr != nullptr && threadIdx.x == 0) tr[k] = (v)
-#else
-#define SEL_TRACE(k, v)
-#endif
   static_assert(kThreads == 128 && kSelBins == 8 * kThreads, "one thread per 8 histogram bins");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned full = 0xffffffffu;
@@ -43,6 +259,7 @@ __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, ui
     __syncthreads();
     return n + 1;
   }
+  if (n <= 4 * kThreads) return select_small(vals, n, topk, cur, sel, hist, selbits, scan, tr);
   uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
   const int per = (n + 4 * kThreads - 1) / (4 * kThreads) * 4;
   const int i0 = tid * per;

@@ -236,6 +236,39 @@ def test_topk_exact_with_ties(budget):
             assert list(sel[s, h, :len(want)]) == want, (s, h)
 
 
+@pytest.mark.parametrize("budget", [1024, 2048, 4096, 16384])
+def test_topk_exact_up_to_512_blocks(budget):
+    """Up to 512 historical blocks (contexts to 32k) take the short selection
+    path: value-linear buckets, a bit mask, a crowded-bucket fallback.  Ties,
+    equal scores, infinities and a span that overflows fp32 must still give
+    the full-sort rule exactly."""
+    g = torch.Generator().manual_seed(budget + 7)
+    B, hkv, mg = 2, 4, 512
+    lens = torch.tensor([64 * 257 + 1, 64 * 512], dtype=torch.int32)   # 257 and 511 blocks
+    scores = torch.randn(B, hkv, mg, generator=g)
+    scores[:, 0] = torch.randint(-4, 5, (B, mg), generator=g).float() * 0.25   # 9 values, many ties
+    scores[:, 1] = -1.25                                                     # all equal
+    scores[0, 2, 3] = float("inf")
+    scores[0, 2, 50:60] = float("-inf")
+    scores[1, 2, 10] = 3.0e38
+    scores[1, 2, 11] = -3.0e38                                               # max - min overflows
+    scores[1, 3, 200:220] = 2.0                                              # a tied plateau at the top
+    cfg = sas.Config(4 * hkv, hkv, token_budget=budget)
+    ws = sas.make_workspace(cfg, DEV)
+    sel = torch.full((B, hkv, budget // 64), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.full((B, hkv), -1, dtype=torch.int32, device=DEV)
+    sas.topk_blocks(cfg, scores.to(DEV), lens.to(DEV), sel, cnt, ws)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    for s in range(B):
+        c = (int(lens[s]) - 1) // 64
+        for h in range(hkv):
+            want = O.select_blocks(scores[s, h, :c].double().numpy(), c, budget // 64 - 1)
+            assert int(cnt[s, h]) == len(want)
+            assert list(sel[s, h, :len(want)]) == want, (s, h)
+
+
 def test_sparse_decode_given_blocks():
     spec = DecodeSpec("given", 2, 8, 2, [3000, 2100], (512,), capacity=4096, seed=19)
     inp = make_decode_inputs(spec, DEV)
