@@ -132,10 +132,22 @@ __global__ void __launch_bounds__(kThreads, 4)
   float* po = reinterpret_cast<float*>(slots);  // [4][G][128], after the last tile
 
   // ------------------------------------------------------------ prologue copies
-  // Everything that does not depend on the sequence length is requested
-  // first, asynchronously: q of the group (bulk), the W_q column slice of
-  // this CTA (one 2-D TMA box per head) and gamma_q (bulk).
+  // Thread 0 loads the sequence length first (one request per CTA: every CTA
+  // of the grid reads the same few bytes) and, while it is in flight,
+  // requests everything that does not depend on it, asynchronously: q of the
+  // group (bulk), gamma_q (bulk) and the W_q column slice of this CTA (one 2-D
+  // TMA box per head).
+  int* len_s = reinterpret_cast<int*>(qbar);  // qbar is written only after the validation
   if (tid == 0) {
+    const int L0 = p.kv.seq_lens[s];
+    // the descriptors of the maps this mode uses are fetched while the plain
+    // copies go out
+    if (MODE != kModeAttend) prefetch_tensormap(&tmw);
+    if constexpr (!kF32 && MODE != kModeGate) {
+      prefetch_tensormap(&tmk);
+      prefetch_tensormap(&tmv);
+    }
+    if (pool_on) prefetch_tensormap(&tmwk);
     for (int i = 0; i < NST + 8; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
     const uint32_t qbytes = static_cast<uint32_t>(G * kDim * sizeof(T));
@@ -145,14 +157,16 @@ __global__ void __launch_bounds__(kThreads, 4)
     mbar_arrive_expect_tx(bar_pro, tx);
     bulk_g2s(qraw, static_cast<const T*>(p.q) + (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim,
              qbytes, bar_pro);
+    if (MODE != kModeAttend) bulk_g2s(gam_s, p.gamma_q, kDim * 4, bar_pro);
+    if (pool_on) bulk_g2s(gamk_s, p.gamma_k, kDim * 4, bar_pro);
     if (MODE != kModeAttend) {
       for (int g = 0; g < G; ++g)
         tma_load_2d(wq_s + static_cast<size_t>(g) * kDim * kDpc, &tmw, rank * kDpc, (h * G + g) * kDim,
                     bar_pro);
-      bulk_g2s(gam_s, p.gamma_q, kDim * 4, bar_pro);
     }
-    if (pool_on) bulk_g2s(gamk_s, p.gamma_k, kDim * 4, bar_pro);
+    *len_s = L0;
   }
+  SAS_TRACE(16);  // thread 0: prologue copies requested
   // thread 0 arrives after its barrier initialisation: no CTA of the cluster
   // passes cluster_wait() (and stores into this one) before it
   cluster_arrive_relaxed();
@@ -163,7 +177,8 @@ __global__ void __launch_bounds__(kThreads, 4)
   }
 
   // ------------------------------------------------------------ validation
-  const int L = p.kv.seq_lens[s];
+  __syncthreads();
+  const int L = *len_s;
   bool err = (L < 1);
   const int c = err ? 0 : (L - 1) / kBlock;  // current block
   if (MODE != kModeAttend && c > p.mg) err = true;
@@ -190,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
   }
   const bool bad = __syncthreads_or(err) != 0;
+  SAS_TRACE(17);  // length read and validated
   if (bad && rank == 0 && tid == 0) raise_status(p.status, kStatusBounds);
   const int n = bad ? 0 : c;  // historical blocks
   // the decoded token completes block c: pool it into gate-key row c
@@ -449,6 +465,7 @@ __global__ void __launch_bounds__(kThreads, 4)
           for (int j = tid; j < m; j += kThreads) sel[j] = c;
           __syncthreads();
         }
+        SAS_TRACE(18);  // rank 0: list ready
         for (int j = tid; j < m; j += kThreads) {
           const int b = sel[j];
           for (int r = 1; r < CS; ++r)
@@ -456,6 +473,7 @@ __global__ void __launch_bounds__(kThreads, 4)
           if (p.sel_idx != nullptr) p.sel_idx[static_cast<size_t>(pair) * p.max_sel + j] = b;
         }
         if (p.sel_count != nullptr && tid == 0) p.sel_count[pair] = list_ok ? m : 0;
+        SAS_TRACE(19);  // rank 0: list sent
         issue_wk();
       } else {
         issue_wk();
@@ -471,6 +489,7 @@ __global__ void __launch_bounds__(kThreads, 4)
       __syncthreads();
     }
     known = nchunks + kTilesPerBlock * cnt_mine;
+    SAS_TRACE(20);  // list in hand
     pump(nchunks, known);
     SAS_TRACE(5);
   }

@@ -171,7 +171,7 @@ constexpr int kPoolWkBytes = kPool * kDim * 2;  // W_k of one KV head, bf16 (96 
 
 // Phase-trace builds (-DSAS_PHASE_TRACE) record per-CTA timestamps after the
 // status word; ordinary builds compile the hooks out.
-constexpr int kTraceSlots = 16;
+constexpr int kTraceSlots = 24;
 constexpr int kTraceCtas = 4096;
 
 // Launchers (return the cudaError_t of the launch).
