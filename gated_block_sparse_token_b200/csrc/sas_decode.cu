@@ -499,16 +499,14 @@ __global__ void __launch_bounds__(kThreads, 4)
   float m_run = -INFINITY, l_run = 0.f;  // bf16 path: head gq of this warp
   float o_acc[16][2];                      // bf16 path: O[gq][8nt + 2tq + e]
   float fm[kMaxGroup], fl[kMaxGroup], fo[kMaxGroup][4];  // fp32 path
-  uint32_t qa0[8], qa2[8];
+  // bf16 path: this lane's q fragments (head gq, columns 16ks + 2tq (+8)) are
+  // read from shared memory at each K tile rather than held in registers
+  const uint32_t* qfrag = reinterpret_cast<const uint32_t*>(
+      reinterpret_cast<const __nv_bfloat16*>(qraw) + min(gq, G - 1) * kDim + 2 * tq);
+  const bool qlive = gq < G;
   if constexpr (!kF32) {
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) o_acc[nt][0] = o_acc[nt][1] = 0.f;
-    const __nv_bfloat16* qrow = reinterpret_cast<const __nv_bfloat16*>(qraw) + min(gq, G - 1) * kDim;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      qa0[ks] = (gq < G) ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq) : 0u;
-      qa2[ks] = (gq < G) ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * tq) : 0u;
-    }
   } else {
 #pragma unroll
     for (int g = 0; g < kMaxGroup; ++g) {
@@ -518,6 +516,51 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
   }
   const float sl2 = p.attn_scale_log2;
+
+  if (do_pool && own_cur) {
+    // key-block pooling (max, min, mean over the 64 tokens) of the current
+    // block, straight from its K tile (list entry 0 of this CTA, already
+    // requested), sent to every CTA of the cluster
+    const int t0 = nchunks;
+    float mx = -INFINITY, mn = INFINITY, sm = 0.f;
+    const int d = tid;
+    if constexpr (!kF32) {
+      const bool ok = mbar_wait(&bars[t0 % NST], (t0 / NST) & 1, p.status);
+      const uint8_t* kt = slots + (t0 % NST) * kTileBytes;
+      const int jc = d >> 3, el = d & 7;
+      if (ok) {
+#pragma unroll 8
+        for (int t = 0; t < kBlock; ++t) {
+          const float x = __bfloat162float(
+              *reinterpret_cast<const __nv_bfloat16*>(kt + swz_tile_offset(t, jc) + el * 2));
+          mx = fmaxf(mx, x);
+          mn = fminf(mn, x);
+          sm += x;
+        }
+      }
+    } else {
+      bool ok = mbar_wait(&bars[t0 % NST], (t0 / NST) & 1, p.status);
+      ok = mbar_wait(&bars[(t0 + 1) % NST], ((t0 + 1) / NST) & 1, p.status) && ok;
+      const float* k0 = reinterpret_cast<const float*>(slots + (t0 % NST) * kTileBytes);
+      const float* k1 = reinterpret_cast<const float*>(slots + ((t0 + 1) % NST) * kTileBytes);
+      if (ok) {
+        for (int t = 0; t < kBlock; ++t) {
+          const float x = (t < 32 ? k0 : k1)[(t & 31) * kDim + d];
+          mx = fmaxf(mx, x);
+          mn = fminf(mn, x);
+          sm += x;
+        }
+      }
+    }
+    sm *= (1.f / kBlock);
+#pragma unroll
+    for (int r = 0; r < CS; ++r) {
+      const uint32_t rb = dsmem_addr(bar_p, r);
+      st_async_f32(dsmem_addr(pool_p + d, r), mx, rb);
+      st_async_f32(dsmem_addr(pool_p + kDim + d, r), mn, rb);
+      st_async_f32(dsmem_addr(pool_p + 2 * kDim + d, r), sm, rb);
+    }
+  }
 
   for (int e = 0; e < cnt_mine; ++e) {
     const int b = entry_block(e);
@@ -536,32 +579,10 @@ __global__ void __launch_bounds__(kThreads, 4)
         for (int ks = 0; ks < 8; ++ks) {
           uint32_t r0, r1, r2, r3;
           ldsm_x4(kbase + swz_tile_offset(tok, 2 * ks + (mat & 1)), r0, r1, r2, r3);
-          mma_rows0_7(sacc[0][0], sacc[0][1], qa0[ks], qa2[ks], r0, r1);
-          mma_rows0_7(sacc[1][0], sacc[1][1], qa0[ks], qa2[ks], r2, r3);
-        }
-      }
-      const bool pool_here = do_pool && own_cur && e == 0;
-      if (pool_here) {
-        // key-block pooling (max, min, mean over the 64 tokens) of the
-        // current block straight from its K tile, sent to every CTA
-        const uint8_t* kt = slots + slotK * kTileBytes;
-        const int d = tid, jc = d >> 3, el = d & 7;
-        float mx = -INFINITY, mn = INFINITY, sm = 0.f;
-#pragma unroll 16
-        for (int t = 0; t < kBlock; ++t) {
-          const float x = __bfloat162float(
-              *reinterpret_cast<const __nv_bfloat16*>(kt + swz_tile_offset(t, jc) + el * 2));
-          mx = fmaxf(mx, x);
-          mn = fminf(mn, x);
-          sm += x;
-        }
-        sm *= (1.f / kBlock);
-#pragma unroll
-        for (int r = 0; r < CS; ++r) {
-          const uint32_t rb = dsmem_addr(bar_p, r);
-          st_async_f32(dsmem_addr(pool_p + d, r), mx, rb);
-          st_async_f32(dsmem_addr(pool_p + kDim + d, r), mn, rb);
-          st_async_f32(dsmem_addr(pool_p + 2 * kDim + d, r), sm, rb);
+          const uint32_t qa0 = qlive ? qfrag[8 * ks] : 0u;      // q[16ks + 2tq], [+1]
+          const uint32_t qa2 = qlive ? qfrag[8 * ks + 4] : 0u;  // q[16ks + 8 + 2tq], [+1]
+          mma_rows0_7(sacc[0][0], sacc[0][1], qa0, qa2, r0, r1);
+          mma_rows0_7(sacc[1][0], sacc[1][1], qa0, qa2, r2, r3);
         }
       }
       __syncthreads();
@@ -654,27 +675,6 @@ __global__ void __launch_bounds__(kThreads, 4)
 #pragma unroll
           for (int g = 0; g < kMaxGroup; ++g)
             if (g < G) lg[g] = fmaf(qatt[g * kDim + hh * 64 + d], kv, lg[g]);
-        }
-      }
-      const bool pool_here = do_pool && own_cur && e == 0;
-      if (pool_here) {
-        const int d = tid;
-        const float* k0 = reinterpret_cast<const float*>(slots + (t0 % NST) * kTileBytes);
-        const float* k1 = reinterpret_cast<const float*>(slots + ((t0 + 1) % NST) * kTileBytes);
-        float mx = -INFINITY, mn = INFINITY, sm = 0.f;
-        for (int t = 0; t < kBlock; ++t) {
-          const float x = (t < 32 ? k0 : k1)[(t & 31) * kDim + d];
-          mx = fmaxf(mx, x);
-          mn = fminf(mn, x);
-          sm += x;
-        }
-        sm *= (1.f / kBlock);
-#pragma unroll
-        for (int r = 0; r < CS; ++r) {
-          const uint32_t rb = dsmem_addr(bar_p, r);
-          st_async_f32(dsmem_addr(pool_p + d, r), mx, rb);
-          st_async_f32(dsmem_addr(pool_p + kDim + d, r), mn, rb);
-          st_async_f32(dsmem_addr(pool_p + 2 * kDim + d, r), sm, rb);
         }
       }
       __syncthreads();

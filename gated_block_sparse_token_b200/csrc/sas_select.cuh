@@ -228,7 +228,7 @@ __device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uin
   return topk + 1;
 }
 
-// Top-K selection (pages: training Top-K 31 under the 2,048-token budget).
+// Top-K selection, general path (pages: training Top-K 31 under the 2,048-token budget).
 // Keeps the min(topk, n) largest of vals[0..n) -- ties go to the lower index
 // -- lists them ascending in sel[], appends the current block `cur` and
 // returns the count.  Exact: scores map to order-preserving 32-bit keys,
@@ -243,23 +243,11 @@ __device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uin
 // be 16-byte aligned with room for ceil(n / 4) * 4 entries; it is
 // overwritten with the keys.  hist needs kSelBins words, selbits
 // ceil(n / 32) words, scan 16 words.
-__device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
-                             uint32_t* selbits, int* scan, unsigned long long* tr = nullptr) {
+__device__ __noinline__ int select_large(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
+                                         uint32_t* selbits, int* scan, unsigned long long* tr) {
   static_assert(kThreads == 128 && kSelBins == 8 * kThreads, "one thread per 8 histogram bins");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned full = 0xffffffffu;
-  if (topk <= 0) {  // a 64-token budget keeps the current block only
-    if (tid == 0) sel[0] = cur;
-    __syncthreads();
-    return 1;
-  }
-  if (n <= topk) {
-    for (int i = tid; i < n; i += kThreads) sel[i] = i;
-    if (tid == 0) sel[n] = cur;
-    __syncthreads();
-    return n + 1;
-  }
-  if (n <= 4 * kThreads) return select_small(vals, n, topk, cur, sel, hist, selbits, scan, tr);
   uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
   const int per = (n + 4 * kThreads - 1) / (4 * kThreads) * 4;
   const int i0 = tid * per;
@@ -438,6 +426,28 @@ __device__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, ui
   }
   __syncthreads();
   return topk + 1;
+}
+
+
+// Entry point: trivial budgets, then the short path (n <= 512) inline, the
+// general path out of line (it is rare, and keeping its code out of the
+// caller keeps the caller's instruction footprint small).
+__device__ __forceinline__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
+                                             uint32_t* selbits, int* scan, unsigned long long* tr = nullptr) {
+  const int tid = threadIdx.x;
+  if (topk <= 0) {  // a 64-token budget keeps the current block only
+    if (tid == 0) sel[0] = cur;
+    __syncthreads();
+    return 1;
+  }
+  if (n <= topk) {
+    for (int i = tid; i < n; i += kThreads) sel[i] = i;
+    if (tid == 0) sel[n] = cur;
+    __syncthreads();
+    return n + 1;
+  }
+  if (n <= 4 * kThreads) return select_small(vals, n, topk, cur, sel, hist, selbits, scan, tr);
+  return select_large(vals, n, topk, cur, sel, hist, selbits, scan, tr);
 }
 
 }  // namespace
