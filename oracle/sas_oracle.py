@@ -60,6 +60,11 @@ R12 Inference weights every selected block 1 (the continuous gate is the
 R13 Prefill gate query for query block i is the mean over the block's 64
     token queries, per query head.
 R14 Attention logits use scale 1/sqrt(128); softmax in float64.
+R18 Gated inference mode (a variant of R12; "continuous gates act on the
+    selected blocks", [aigc-0914] release paragraph): the logits of every
+    token of a selected historical block b, for query head g, get the
+    additive bias log(sigmoid(s_{g,b})) with s_{g,b} the head's gate score
+    (R7); the current block gets 0.  Gates equal to 1 reduce it to R12.
 
 Parity status: the gate formula as a whole (R1-R8) is pinned only by the
 invariants and hand-derived closed forms in tests/test_oracle.py, not by any
@@ -196,12 +201,27 @@ def topk_for_budget(token_budget: int) -> int:
 # --------------------------------------------------------------------------
 # Step 4: attention over the selected blocks (R12, R14).
 # --------------------------------------------------------------------------
+GATE_SELECT_ONLY = 0       # R12: selected blocks weighted 1
+GATE_LOGSIGMOID_BIAS = 1   # R18: + log(sigmoid(s_{g,b})) on block b's logits
+
+
+def log_sigmoid(x: float) -> float:
+    """log(1 / (1 + exp(-x))), evaluated without overflow for either sign."""
+    x = float(x)
+    if x >= 0.0:
+        return -math.log1p(math.exp(-x))
+    return x - math.log1p(math.exp(x))
+
+
 def attention_over_tokens(q: np.ndarray, k: np.ndarray, v: np.ndarray,
-                          token_ids, scale: float) -> np.ndarray:
-    """softmax(q . k_j * scale) weighted sum of v_j over the listed tokens,
-    two-pass (max, then exp-sum) in float64."""
+                          token_ids, scale: float, bias=None) -> np.ndarray:
+    """softmax(q . k_j * scale + bias_j) weighted sum of v_j over the listed
+    tokens, two-pass (max, then exp-sum) in float64.  bias: None, or one
+    additive logit term per listed token (the gated mode, R18)."""
     idx = np.asarray(list(token_ids), dtype=np.int64)
     logits = (k[idx].astype(np.float64) @ np.asarray(q, np.float64)) * scale
+    if bias is not None:
+        logits = logits + np.asarray(bias, np.float64)
     m = logits.max()
     p = np.exp(logits - m)
     return (p @ v[idx].astype(np.float64)) / p.sum()
@@ -216,13 +236,26 @@ def selected_token_ids(blocks, seq_len: int):
     return out
 
 
+def gated_token_bias(s_g, blocks, seq_len: int, cur: int):
+    """The gated mode's logit bias for one query head (R18), one entry per
+    token of selected_token_ids(blocks, seq_len): log(sigmoid(s_g[b])) for a
+    historical block b, 0 for the current block."""
+    out = []
+    for b in blocks:
+        n = min((b + 1) * BLOCK, seq_len) - b * BLOCK
+        out.extend([0.0 if b == cur else log_sigmoid(s_g[b])] * n)
+    return out
+
+
 def decode_one_group(q_group, k_seq, v_seq, seq_len, gate_keys, w_q_group,
                      gamma_q_group, token_budget, attn_scale=1.0 / math.sqrt(128.0),
-                     gate_scale=1.0 / math.sqrt(128.0), eps=1e-6, base=10000.0):
+                     gate_scale=1.0 / math.sqrt(128.0), eps=1e-6, base=10000.0,
+                     gate_mode=GATE_SELECT_ONLY):
     """Decode step of one (sequence, KV head): gate, select, attend.
 
     q_group [G][128]: queries of token L-1 for the G heads of the group.
     k_seq, v_seq [>= L][128]: the head's cache.  gate_keys [>= c][128].
+    gate_mode: GATE_SELECT_ONLY (R12) or GATE_LOGSIGMOID_BIAS (R18).
     Returns dict(out [G][128], sel (ascending list), s [G][c], S [c]).
     """
     c = (seq_len - 1) // BLOCK            # current block (R10)
@@ -230,9 +263,13 @@ def decode_one_group(q_group, k_seq, v_seq, seq_len, gate_keys, w_q_group,
                        gate_scale, eps, base)
     sel = select_blocks(S, c, topk_for_budget(token_budget))
     toks = selected_token_ids(sel, seq_len)
-    out = np.stack([attention_over_tokens(q_group[g], k_seq, v_seq, toks, attn_scale)
-                    for g in range(q_group.shape[0])])
-    return {"out": out, "sel": sel, "s": s, "S": S}
+    outs = []
+    for g in range(q_group.shape[0]):
+        bias = None
+        if gate_mode == GATE_LOGSIGMOID_BIAS:
+            bias = gated_token_bias(s[g], sel, seq_len, c)
+        outs.append(attention_over_tokens(q_group[g], k_seq, v_seq, toks, attn_scale, bias))
+    return {"out": np.stack(outs), "sel": sel, "s": s, "S": S}
 
 
 def dense_causal_decode(q_group, k_seq, v_seq, seq_len,
@@ -302,7 +339,8 @@ def dense_causal_prefill(q_seq, k_seq, v_seq, attn_scale=1.0 / math.sqrt(128.0))
 # head g // G (G = Hq / Hkv).
 # --------------------------------------------------------------------------
 def decode_step(q, k_cache, v_cache, seq_lens, w_q, gamma_q, w_k, gamma_k,
-                token_budget, gate_keys=None, pairs=None, eps=1e-6, base=10000.0):
+                token_budget, gate_keys=None, pairs=None, eps=1e-6, base=10000.0,
+                gate_mode=GATE_SELECT_ONLY):
     """Full decode step for the listed (sequence, KV head) pairs (all if None).
 
     gate_keys: optional precomputed [B][Hkv][>=c][128]; computed from the
@@ -325,5 +363,5 @@ def decode_step(q, k_cache, v_cache, seq_lens, w_q, gamma_q, w_k, gamma_k,
         heads = slice(h * G, (h + 1) * G)
         res[(s, h)] = decode_one_group(np.asarray(q[s, heads], np.float64), ks, vs, L, gk,
                                        w_q[heads], np.tile(gamma_q, (G, 1)), token_budget,
-                                       eps=eps, base=base)
+                                       eps=eps, base=base, gate_mode=gate_mode)
     return res

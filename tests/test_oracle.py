@@ -317,6 +317,76 @@ def test_prefill_gate_query_is_block_mean():
     assert np.allclose(r["out"][0, 0], ref, atol=1e-12)
 
 
+# ---------------------------------------------------------------- gated inference mode (R18)
+def _gated_case(gate_scale=SCALE):
+    """Two heads, one complete historical block and the query token (L = 65).
+    Block 0's keys are a*e1, so the pooled block projects (W_k maps max, min
+    and mean of dim 1 to output 0) onto k~_0 = sqrt(128) e0 after RMSNorm;
+    W_q = I and q_g = +-b e0 give q~_g = +-sqrt(128) (cos 1 e0 + sin 1 e64) at
+    query position 1, so s_g = +-sqrt(128) cos(1) * sqrt(128) * gate_scale.
+    Every attention logit is 0 (q _|_ keys, current key 0)."""
+    a, b, L = 1.5, 2.0, 65
+    rng = np.random.default_rng(3)
+    k = np.zeros((L, 128))
+    k[:64, 1] = a
+    v = np.zeros((L, 128))
+    v0 = rng.standard_normal(128)
+    v1 = rng.standard_normal(128)
+    v[:64] = v0
+    v[64] = v1
+    w_k = np.zeros((384, 128))
+    w_k[1, 0] = w_k[129, 0] = w_k[257, 0] = 1.0
+    gk = O.gate_keys_for_sequence(k, 1, w_k, np.ones(128))
+    q = np.zeros((2, 128))
+    q[0, 0], q[1, 0] = b, -b
+    w_q = np.stack([np.eye(128)] * 2)
+    gam = np.ones((2, 128))
+    res = {}
+    for mode in (O.GATE_SELECT_ONLY, O.GATE_LOGSIGMOID_BIAS):
+        res[mode] = O.decode_one_group(q, k, v, L, gk, w_q, gam, 2048, gate_scale=gate_scale,
+                                       gate_mode=mode)
+    eps = 1e-6  # RMSNorm epsilon (R5)
+    kn = 3 * a / math.sqrt((3 * a) ** 2 / 128 + eps)   # |k~_0|
+    qn = b / math.sqrt(b ** 2 / 128 + eps)             # |q~_g|
+    s = np.array([1.0, -1.0]) * qn * math.cos(1.0) * kn * gate_scale
+    return res, s, v0, v1
+
+
+def test_gated_mode_closed_form():
+    """out_g = (64 sigmoid(s_g) v0 + v1) / (64 sigmoid(s_g) + 1): the bias is
+    log(sigmoid(s_g)) per head on the historical block only."""
+    res, s, v0, v1 = _gated_case()
+    r = res[O.GATE_LOGSIGMOID_BIAS]
+    assert r["sel"] == [0, 1]
+    assert np.allclose(r["s"][:, 0], s, rtol=1e-12, atol=1e-12)
+    for g in range(2):
+        w = 64.0 / (1.0 + math.exp(-s[g]))
+        want = (w * v0 + v1) / (w + 1.0)
+        assert np.allclose(r["out"][g], want, rtol=1e-12, atol=1e-12), g
+    plain = res[O.GATE_SELECT_ONLY]["out"]
+    assert np.allclose(plain, (64.0 * v0 + v1) / 65.0, rtol=1e-12, atol=1e-12)
+    assert not np.allclose(r["out"][0], plain[0])
+
+
+def test_gated_mode_saturated_gates():
+    """Gates near 1 reduce the gated mode to select-only (R12); gates near 0
+    leave the current block alone."""
+    res, s, v0, v1 = _gated_case(gate_scale=1e3)
+    assert s[0] > 700 and s[1] < -700
+    assert np.allclose(res[O.GATE_LOGSIGMOID_BIAS]["out"][0], res[O.GATE_SELECT_ONLY]["out"][0],
+                       rtol=1e-12, atol=1e-12)
+    assert np.allclose(res[O.GATE_LOGSIGMOID_BIAS]["out"][1], v1, rtol=1e-12, atol=1e-12)
+
+
+def test_log_sigmoid_values():
+    assert O.log_sigmoid(0.0) == pytest.approx(-math.log(2.0), abs=1e-15)
+    for x in (-50.0, -3.0, -0.5, 0.25, 4.0):
+        assert O.log_sigmoid(x) == pytest.approx(math.log(1.0 / (1.0 + math.exp(-x))), rel=1e-12, abs=1e-300)
+    assert O.log_sigmoid(60.0) == pytest.approx(-math.exp(-60.0), rel=1e-12)
+    assert O.log_sigmoid(-800.0) == pytest.approx(-800.0)
+    assert -1e-300 < O.log_sigmoid(800.0) <= 0.0
+
+
 # ---------------------------------------------------------------- planted mistakes
 def test_pins_catch_planted_mistakes(monkeypatch):
     """Plant plausible mistakes in the oracle (CPU) and show a pin fails."""
@@ -354,10 +424,32 @@ def test_pins_catch_planted_mistakes(monkeypatch):
 
     good_attn = O.attention_over_tokens
 
-    def attn_no_scale(q, k, v, toks, scale):
-        return good_attn(q, k, v, toks, 1.0)
+    def attn_no_scale(q, k, v, toks, scale, bias=None):
+        return good_attn(q, k, v, toks, 1.0, bias)
 
     monkeypatch.setattr(O, "attention_over_tokens", attn_no_scale)
     with pytest.raises(AssertionError):
         test_budget_covering_context_is_dense_causal(300)
     monkeypatch.setattr(O, "attention_over_tokens", good_attn)
+
+    # gated mode: log(1 - sigmoid) instead of log(sigmoid); the gate itself
+    # instead of its log; a bias on the current block too
+    good_ls = O.log_sigmoid
+    monkeypatch.setattr(O, "log_sigmoid", lambda x: good_ls(-x))
+    with pytest.raises(AssertionError):
+        test_gated_mode_closed_form()
+    monkeypatch.setattr(O, "log_sigmoid", lambda x: math.exp(good_ls(x)))
+    with pytest.raises(AssertionError):
+        test_gated_mode_closed_form()
+    monkeypatch.setattr(O, "log_sigmoid", good_ls)
+
+    good_bias = O.gated_token_bias
+
+    def bias_on_current_too(s_g, blocks, seq_len, cur):
+        b = good_bias(s_g, blocks, seq_len, cur)
+        return [x if x != 0.0 else good_ls(0.0) for x in b]
+
+    monkeypatch.setattr(O, "gated_token_bias", bias_on_current_too)
+    with pytest.raises(AssertionError):
+        test_gated_mode_closed_form()
+    monkeypatch.setattr(O, "gated_token_bias", good_bias)
