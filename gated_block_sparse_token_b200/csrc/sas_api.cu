@@ -20,7 +20,7 @@ namespace {
 
 using sas::kDim;
 
-constexpr int32_t kAbiVersion = 2;
+constexpr int32_t kAbiVersion = 3;
 constexpr size_t kStatusBytes = 256;  // status word + padding
 constexpr int kMaxBudget = 16384;
 constexpr int kMaxGateBlocks = 16384;
@@ -72,6 +72,8 @@ sas_status check_config(const sas_config* c) {
   if (!isfinite(c->norm_eps) || c->norm_eps < 0.f) return SAS_ERR_INVALID_ARG;
   if (c->kv_dtype != SAS_DTYPE_BF16 && c->kv_dtype != SAS_DTYPE_F32) return SAS_ERR_INVALID_ARG;
   if (c->out_dtype != SAS_DTYPE_BF16 && c->out_dtype != SAS_DTYPE_F32) return SAS_ERR_INVALID_ARG;
+  if (c->gate_mode != SAS_GATE_SELECT_ONLY && c->gate_mode != SAS_GATE_LOGSIGMOID_BIAS)
+    return SAS_ERR_INVALID_ARG;
   return SAS_OK;
 }
 
@@ -178,8 +180,9 @@ void fill_common(sas::DecodeParams& p, const sas_config* cfg, int mg) {
   p.eps = cfg->norm_eps;
   p.attn_scale_log2 = cfg->attn_scale * 1.4426950408889634f;
   p.gate_scale = cfg->gate_scale;
+  p.gated = cfg->gate_mode == SAS_GATE_LOGSIGMOID_BIAS ? 1 : 0;
   p.sm = sas::plan_decode_smem(p.G, mg, kClusterSize, kStages, p.max_sel,
-                               cfg->kv_dtype == SAS_DTYPE_F32);
+                               cfg->kv_dtype == SAS_DTYPE_F32, p.gated != 0);
   sas::fill_rope_table(p.rope, cfg->rope_base);
 }
 
@@ -400,6 +403,8 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
   } else {
     if (sel_idx == nullptr || sel_count == nullptr || !aligned(sel_idx, 4) || !aligned(sel_count, 4))
       return SAS_ERR_INVALID_ARG;
+    // the gated mode needs the gate query and keys, which this call has not
+    if (cfg->gate_mode != SAS_GATE_SELECT_ONLY) return SAS_ERR_UNSUPPORTED;
     max_gate_blocks = 1;
   }
   if (static_cast<long long>(kv->batch) * cfg->num_kv_heads > 65535) return SAS_ERR_UNSUPPORTED;
@@ -445,6 +450,7 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
                                     int32_t* sel_count, void* ws, size_t ws_bytes,
                                     sas_stream_t stream) {
   sas_status st = check_config(cfg);
+  if (st == SAS_OK && cfg->gate_mode != SAS_GATE_SELECT_ONLY) return SAS_ERR_UNSUPPORTED;
   if (st != SAS_OK) return st;
   if (batch < 0 || seq_len < 0) return SAS_ERR_INVALID_ARG;
   if (batch == 0 || seq_len == 0) return SAS_OK;

@@ -130,6 +130,9 @@ __global__ void __launch_bounds__(kThreads, 4)
   uint32_t* selbits = reinterpret_cast<uint32_t*>(base + p.sm.r_selbits);
   int* scan = reinterpret_cast<int*>(base + p.sm.r_scan);
   float* po = reinterpret_cast<float*>(slots);  // [4][G][128], after the last tile
+  // gated mode: log-sigmoid gate of list entry j for head g at gbias[j * G + g]
+  float* gbias = reinterpret_cast<float*>(base + p.sm.gbias);
+  const bool gated = (MODE == kModeFused) && p.gated != 0;
 
   // ------------------------------------------------------------ prologue copies
   // Thread 0 loads the sequence length first (one request per CTA: every CTA
@@ -227,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 4)
       if (rank == 0)
         mbar_arrive_expect_tx(bar_sc, static_cast<uint32_t>(n * 4));
       else
-        mbar_arrive_expect_tx(bar_sel, static_cast<uint32_t>(m * 4));
+        mbar_arrive_expect_tx(bar_sel, static_cast<uint32_t>(m * 4 * (gated ? 1 + G : 1)));
     }
     if (do_pool) {
       mbar_arrive_expect_tx(bar_p, kPool * 4);
@@ -237,12 +240,12 @@ __global__ void __launch_bounds__(kThreads, 4)
   }
 
   // list entry e of this CTA -> block id (the current block first if owned)
+  auto entry_index = [&](int e) -> int {
+    if (own_cur) return (e == 0) ? (m - 1) : rank + (e - 1) * CS;
+    return rank + e * CS;
+  };
   auto entry_block = [&](int e) -> int {
-    int j;
-    if (own_cur)
-      j = (e == 0) ? (m - 1) : rank + (e - 1) * CS;
-    else
-      j = rank + e * CS;
+    const int j = entry_index(e);
     return (j == m - 1) ? c : sel[j];
   };
 
@@ -465,6 +468,29 @@ __global__ void __launch_bounds__(kThreads, 4)
           for (int j = tid; j < m; j += kThreads) sel[j] = c;
           __syncthreads();
         }
+        if (gated) {
+          // gate of every list entry and head: log(sigmoid(s_gb)), s_gb =
+          // (q~_g . k~_b) * gate_scale from q~ (v, rotated in place) and the
+          // block's gate key; 0 for the current block and a stand-in list
+          for (int w = warp; w < m * G; w += kWarps) {
+            const int j = w / G, g = w - j * G;
+            float beta = 0.f;
+            if (list_ok && j < m - 1) {
+              const float4 k4 = *reinterpret_cast<const float4*>(
+                  p.gate_keys + (static_cast<size_t>(pair) * p.mg + sel[j]) * kDim + 4 * lane);
+              const float4 q4 = *reinterpret_cast<const float4*>(qv + g * kDim + 4 * lane);
+              float a = fmaf(q4.x, k4.x, fmaf(q4.y, k4.y, fmaf(q4.z, k4.z, q4.w * k4.w)));
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+              const float sg = a * p.gate_scale;
+              beta = (sg >= 0.f) ? -log1pf(expf(-sg)) : sg - log1pf(expf(sg));
+            }
+            if (lane == 0) gbias[w] = beta;
+          }
+          __syncthreads();
+          for (int w = tid; w < m * G; w += kThreads)
+            for (int r = 1; r < CS; ++r) st_async_f32(dsmem_addr(gbias + w, r), gbias[w], dsmem_addr(bar_sel, r));
+        }
         SAS_TRACE(18);  // rank 0: list ready
         for (int j = tid; j < m; j += kThreads) {
           const int b = sel[j];
@@ -486,6 +512,8 @@ __global__ void __launch_bounds__(kThreads, 4)
     // read: the current block, always valid, stands in for every entry
     if (__syncthreads_and(list_ok) == 0) {
       for (int j = tid; j < m; j += kThreads) sel[j] = c;
+      if (gated)
+        for (int w = tid; w < m * G; w += kThreads) gbias[w] = 0.f;
       __syncthreads();
     }
     known = nchunks + kTilesPerBlock * cnt_mine;
@@ -564,6 +592,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 
   for (int e = 0; e < cnt_mine; ++e) {
     const int b = entry_block(e);
+    const int jg = entry_index(e) * G;  // gated mode: this entry's gates at gbias[jg + g]
     const int nvalid = (b == c) ? (L - b * kBlock) : kBlock;
     const int t0 = nchunks + e * kTilesPerBlock;
     if constexpr (!kF32) {
@@ -587,7 +616,9 @@ __global__ void __launch_bounds__(kThreads, 4)
       }
       __syncthreads();
       pump(t0 + 1, known);
-      // ---- online softmax (per warp, head gq)
+      // ---- online softmax (per warp, head gq); gated mode: + the entry's
+      // log-sigmoid gate, in log2 units like the scaled logits
+      const float beta2 = (gated && gq < G) ? gbias[jg + gq] * kLog2e : 0.f;
       float x[2][2];
       float mx = -INFINITY;
 #pragma unroll
@@ -595,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int tl = 16 * warp + 8 * nt + 2 * tq + q;
-          x[nt][q] = (tl < nvalid) ? sacc[nt][q] * sl2 : -INFINITY;
+          x[nt][q] = (tl < nvalid) ? fmaf(sacc[nt][q], sl2, beta2) : -INFINITY;
           mx = fmaxf(mx, x[nt][q]);
         }
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -683,7 +714,8 @@ __global__ void __launch_bounds__(kThreads, 4)
 #pragma unroll
       for (int g = 0; g < kMaxGroup; ++g) {
         float xv = lg[g] + __shfl_xor_sync(0xffffffffu, lg[g], 1);
-        xv = (tl < nvalid) ? xv * sl2 : -INFINITY;
+        const float bg = (gated && g < G) ? gbias[jg + g] * kLog2e : 0.f;
+        xv = (tl < nvalid) ? fmaf(xv, sl2, bg) : -INFINITY;
         float mx = xv;
 #pragma unroll
         for (int o = 2; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));

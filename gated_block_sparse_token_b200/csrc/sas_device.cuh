@@ -21,6 +21,7 @@ constexpr int kMaxGroup = 8;       // largest GQA group (Hq / Hkv) handled
 constexpr int kTileBytes = 16384;  // one stage slot: a 64x128 bf16 tile
 constexpr int kGkChunk = kTileBytes / (kDim * 4);  // gate keys per slot (32)
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;  // 1 s
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e): natural-log terms -> log2 logits
 
 // Bits of the device status word (first 4 bytes of the workspace).
 constexpr uint32_t kStatusBounds = 1u;

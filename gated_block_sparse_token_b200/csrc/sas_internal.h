@@ -30,6 +30,7 @@ constexpr int kSelCand = 256;   // candidates ranked exactly in the boundary buc
 struct DecodeSmem {
   int slots;     // NST stage slots of 16 KiB (gate-key chunks, then K/V tiles)
   int sel;       // int32 [max_sel] selected blocks (phases 2-3)
+  int gbias;     // fp32 [max_sel][G] gated mode: log-sigmoid gate per entry and head
   int qraw;      // T [G][128] query as stored (bf16 or fp32), bulk copy
   int qbar;      // fp32 [128] group-mean gate query (fused mode)
   int pml;       // fp32 m[4][8], l[4][8] per-warp softmax state
@@ -49,7 +50,8 @@ struct DecodeSmem {
   int total;     // bytes to request, including alignment slack
 };
 
-inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, bool f32_kv) {
+inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, bool f32_kv,
+                                   bool gated = false) {
   DecodeSmem p{};
   int off = 0;
   auto take = [&](int bytes, int align) {
@@ -63,6 +65,7 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
   mg = std::max(mg, 1);
   p.slots = take(nst * kTileBytes, 1024);
   p.sel = take(max_sel * 4, 16);
+  p.gbias = take(gated ? max_sel * G * 4 : 0, 16);
   p.qraw = take(G * kDim * (f32_kv ? 4 : 2), 16);
   p.qbar = take(kDim * 4, 16);
   p.pml = take(2 * kWarps * kMaxGroup * 4, 16);
@@ -107,6 +110,7 @@ struct DecodeParams {
   int max_sel;  // budget/64
   int mg;       // rows of the gate-key cache per (seq, head)
   float rope_base, eps, attn_scale_log2, gate_scale;
+  int gated;    // 1: log-sigmoid gate bias on the selected historical blocks
   const void* q;
   const __nv_bfloat16* w_q;
   const float* gamma_q;

@@ -27,6 +27,9 @@ SAS_ERR_CUDA = 4
 SAS_ERR_DEVICE_BOUNDS = 5
 SAS_ERR_TIMEOUT = 6
 
+GATE_SELECT_ONLY = 0       # selected blocks weighted 1
+GATE_LOGSIGMOID_BIAS = 1   # + log(sigmoid(gate score)) on a selected historical block's logits
+
 DTYPE_BF16 = 0
 DTYPE_F32 = 1
 _DT = {"bf16": DTYPE_BF16, "f32": DTYPE_F32}
@@ -45,7 +48,8 @@ class _Config(ctypes.Structure):
                 ("gate_hidden", ctypes.c_int32), ("token_budget", ctypes.c_int32),
                 ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float),
                 ("attn_scale", ctypes.c_float), ("gate_scale", ctypes.c_float),
-                ("kv_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+                ("kv_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
+                ("gate_mode", ctypes.c_int32)]
 
 
 class _Kv(ctypes.Structure):
@@ -124,11 +128,13 @@ class Config:
     head_dim: int = 128
     block_size: int = 64
     gate_hidden: int = 128
+    gate_mode: int = 0        # GATE_SELECT_ONLY or GATE_LOGSIGMOID_BIAS
 
     def c(self) -> _Config:
         return _Config(self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
                        self.gate_hidden, self.token_budget, self.rope_base, self.norm_eps,
-                       self.attn_scale, self.gate_scale, _DT[self.kv_dtype], _DT[self.out_dtype])
+                       self.attn_scale, self.gate_scale, _DT[self.kv_dtype], _DT[self.out_dtype],
+                       self.gate_mode)
 
     @property
     def group(self) -> int:

@@ -82,6 +82,16 @@ typedef enum {
 
 typedef enum { SAS_DTYPE_BF16 = 0, SAS_DTYPE_F32 = 1 } sas_dtype;
 
+/* How the selected blocks enter the decode attention.
+ *   SAS_GATE_SELECT_ONLY: every selected block weighs 1 (the gate only
+ *     selects).
+ *   SAS_GATE_LOGSIGMOID_BIAS: the attention logits of every token of a
+ *     selected historical block b, for query head g, get + log(sigmoid(s_gb)),
+ *     s_gb = (q~_g . k~_b) * gate_scale the head's gate score; the current
+ *     block gets 0.  One plain reading of the pages' "continuous gates act on
+ *     the selected blocks" (aigc.news release paragraph of 2026-09-14). */
+typedef enum { SAS_GATE_SELECT_ONLY = 0, SAS_GATE_LOGSIGMOID_BIAS = 1 } sas_gate_mode;
+
 typedef struct {
   int32_t num_q_heads;   /* Hq >= 1 */
   int32_t num_kv_heads;  /* Hkv >= 1, Hq % Hkv == 0, 1 <= Hq/Hkv <= 8 */
@@ -95,6 +105,11 @@ typedef struct {
   float gate_scale;      /* gate score scale, > 0; default 1/sqrt(128) */
   int32_t kv_dtype;      /* sas_dtype of q, K and V (and of prefill Q) */
   int32_t out_dtype;     /* sas_dtype of the attention output */
+  int32_t gate_mode;     /* sas_gate_mode; default SAS_GATE_SELECT_ONLY.  Only
+                            sas_decode_step(_static) implement the gated mode;
+                            sas_sparse_decode and sas_prefill_block_sparse
+                            return SAS_ERR_UNSUPPORTED for it, the gate-score,
+                            Top-K and pooling calls ignore it. */
 } sas_config;
 
 /* KV cache description (device pointers, caller-owned). */

@@ -11,14 +11,16 @@ int main() {
   for (int G = 1; G <= sas::kMaxGroup; ++G)
     for (int mg : mgs)
       for (int b : budgets)
-        for (int f32 = 0; f32 < 2; ++f32) {
-          const sas::DecodeSmem p = sas::plan_decode_smem(G, mg, 8, 2, b / 64, f32 != 0);
-          std::printf(
-              "G=%d mg=%d budget=%d f32=%d slots=%d sel=%d qraw=%d qbar=%d pml=%d gam=%d bars=%d "
-              "r_qv=%d r_wq=%d r_inbox=%d r_keys=%d r_hist=%d r_selbits=%d r_scan=%d total=%d ok=%d\n",
-              G, mg, b, f32, p.slots, p.sel, p.qraw, p.qbar, p.pml, p.gam, p.bars, p.r_qv, p.r_wq,
-              p.r_inbox, p.r_keys, p.r_hist, p.r_selbits, p.r_scan, p.total,
-              sas::decode_smem_aligned(p, G, sas::kDim / 8) ? 1 : 0);
-        }
+        for (int f32 = 0; f32 < 2; ++f32)
+          for (int gated = 0; gated < 2; ++gated) {
+            const sas::DecodeSmem p = sas::plan_decode_smem(G, mg, 8, 2, b / 64, f32 != 0, gated != 0);
+            std::printf(
+                "G=%d mg=%d budget=%d f32=%d gated=%d slots=%d sel=%d gbias=%d qraw=%d qbar=%d pml=%d "
+                "gam=%d bars=%d r_qv=%d r_wq=%d r_inbox=%d r_keys=%d r_hist=%d r_selbits=%d r_scan=%d "
+                "total=%d ok=%d\n",
+                G, mg, b, f32, gated, p.slots, p.sel, p.gbias, p.qraw, p.qbar, p.pml, p.gam, p.bars, p.r_qv,
+                p.r_wq, p.r_inbox, p.r_keys, p.r_hist, p.r_selbits, p.r_scan, p.total,
+                sas::decode_smem_aligned(p, G, sas::kDim / 8) ? 1 : 0);
+          }
   return 0;
 }

@@ -19,9 +19,9 @@ SCORE_FLOOR = 1e-3     # ... to max(|x|, 1e-3 * max|x|): the pure relative form 
 TIE_RTOL = 1e-3        # K-th vs (K+1)-th oracle score window for set mismatches
 
 
-def config_for(spec, budget, out_dtype="bf16"):
+def config_for(spec, budget, out_dtype="bf16", gate_mode=sas.GATE_SELECT_ONLY):
     return sas.Config(spec.hq, spec.hkv, token_budget=budget, kv_dtype=spec.kv_dtype,
-                      out_dtype=out_dtype)
+                      out_dtype=out_dtype, gate_mode=gate_mode)
 
 
 def kv_of(inputs):
@@ -58,7 +58,7 @@ def run_decode_step(inputs, cfg, ws, gate_keys, pool=False):
     return {"out": out, "sel_idx": sel_idx, "sel_count": sel_count, "group_scores": group_scores}
 
 
-def oracle_pairs(inputs, budget, pairs):
+def oracle_pairs(inputs, budget, pairs, gate_mode=O.GATE_SELECT_ONLY):
     """Oracle decode step (gate keys recomputed from K) for the listed pairs."""
     spec = inputs["spec"]
     G = spec.hq // spec.hkv
@@ -74,7 +74,7 @@ def oracle_pairs(inputs, budget, pairs):
         c = (L - 1) // BLOCK
         keys = O.gate_keys_for_sequence(ks, c, wk[h], gk)
         r = O.decode_one_group(q[s, h * G:(h + 1) * G], ks, vs, L, keys, wq[h * G:(h + 1) * G],
-                               np.tile(gq, (G, 1)), budget)
+                               np.tile(gq, (G, 1)), budget, gate_mode=gate_mode)
         r["gate_keys"] = keys
         r["k"], r["v"], r["L"] = ks, vs, L
         res[(s, h)] = r
@@ -136,8 +136,11 @@ def check_pairs(inputs, cfg, gpu, oracle, gate_keys=None, out_atol=OUT_ATOL):
         if swapped:  # an accepted tie swap: attend over the GPU's set
             toks = O.selected_token_ids(sel, r["L"])
             qg = inputs["q"][s, h * G:(h + 1) * G].double().cpu().numpy()
-            want = np.stack([O.attention_over_tokens(qg[g], r["k"], r["v"], toks, cfg.attn_scale)
-                             for g in range(G)])
+            cur = (r["L"] - 1) // BLOCK
+            want = np.stack([O.attention_over_tokens(
+                qg[g], r["k"], r["v"], toks, cfg.attn_scale,
+                O.gated_token_bias(r["s"][g], sel, r["L"], cur) if cfg.gate_mode else None)
+                for g in range(G)])
         got = out[s, h * G:(h + 1) * G]
         err = float(np.max(np.abs(got - want)))
         assert np.all(np.isfinite(got)) and err <= out_atol, f"{tag}: out max-abs err {err}"

@@ -60,7 +60,7 @@ def test_struct_layout_matches_header():
 int main(void) {
   printf("sizeof.sas_config %zu\nsizeof.sas_kv %zu\n", sizeof(sas_config), sizeof(sas_kv));
   O(sas_config, token_budget); O(sas_config, rope_base); O(sas_config, gate_scale);
-  O(sas_config, kv_dtype); O(sas_config, out_dtype);
+  O(sas_config, kv_dtype); O(sas_config, out_dtype); O(sas_config, gate_mode);
   O(sas_kv, block_table); O(sas_kv, seq_lens); O(sas_kv, batch); O(sas_kv, capacity);
   O(sas_kv, num_pages); O(sas_kv, max_blocks_per_seq);
   return 0;
@@ -84,7 +84,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(L):
-    assert sas.abi_version() >= 1
+    assert sas.abi_version() >= 3
     for st in range(7):
         assert len(sas.status_string(st)) > 0
     assert sas.status_string(sas.SAS_OK) == "ok"
@@ -132,6 +132,8 @@ def _decode(L, cfg, kv=None, ws_bytes=256, ws=FAKE, q=FAKE, out=FAKE, mg=64):
     (dict(gate_scale=float("nan")), sas.SAS_ERR_INVALID_ARG),
     (dict(norm_eps=-1.0), sas.SAS_ERR_INVALID_ARG),
     (dict(rope_base=-5.0), sas.SAS_ERR_INVALID_ARG),
+    (dict(gate_mode=2), sas.SAS_ERR_INVALID_ARG),
+    (dict(gate_mode=-1), sas.SAS_ERR_INVALID_ARG),
 ])
 def test_config_validation(L, kw, status):
     assert _decode(L, _cfg(**kw)) == status
@@ -184,3 +186,16 @@ def test_other_entry_points_validate(L):
     st = ctypes.c_int(0)
     assert L.sas_get_device_status(None, None, ctypes.byref(st)) == sas.SAS_ERR_INVALID_ARG
     assert L.sas_reset_device_status(None, None) == sas.SAS_ERR_WORKSPACE
+
+
+@nogpu
+def test_gated_mode_only_in_the_fused_decode_step(L):
+    """The gated mode needs the gate query and keys: sas_sparse_decode and the
+    prefill refuse it on the host, before any CUDA call."""
+    c = _cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS).c()
+    kv = _kv()
+    assert L.sas_sparse_decode(ctypes.byref(c), FAKE, ctypes.byref(kv), FAKE, FAKE, FAKE, FAKE,
+                               256, None) == sas.SAS_ERR_UNSUPPORTED
+    assert L.sas_prefill_block_sparse(ctypes.byref(c), FAKE, FAKE, FAKE, 2, 4096, FAKE, FAKE, FAKE, FAKE,
+                                      FAKE, 64, FAKE, None, None, FAKE, 1 << 30,
+                                      None) == sas.SAS_ERR_UNSUPPORTED

@@ -28,7 +28,7 @@ def plans():
 
 def test_plan_alignment_and_overlap(plans):
     CS, dpc = 8, 16
-    assert len(plans) == 8 * 8 * 5 * 2
+    assert len(plans) == 8 * 8 * 5 * 2 * 2
     for p in plans:
         G, mg, ms = p["G"], max(p["mg"], 1), p["budget"] // 64
         tag = str(p)
@@ -36,12 +36,13 @@ def test_plan_alignment_and_overlap(plans):
         assert p["slots"] % 1024 == 0 and p["r_wq"] % 128 == 0, tag
         assert p["qraw"] % 16 == 0 and p["gam"] % 16 == 0 and p["bars"] % 8 == 0, tag
         # fixed regions, in order, disjoint
-        fixed = [("slots", 2 * 16384), ("sel", 4 * ms), ("qraw", G * 128 * (4 if p["f32"] else 2)),
-                 ("qbar", 512), ("pml", 256), ("gam", 512), ("bars", 24)]
+        fixed = [("slots", 2 * 16384), ("sel", 4 * ms), ("gbias", 4 * ms * G * p["gated"]),
+                 ("qraw", G * 128 * (4 if p["f32"] else 2)), ("qbar", 512), ("pml", 256), ("gam", 512),
+                 ("bars", 8 * (2 + 8))]
         for (a, sa), (b, _) in zip(fixed, fixed[1:]):
             assert p[a] + sa <= p[b], (tag, a, b)
         r = p["r_qv"]
-        assert p["bars"] + 24 <= r, tag
+        assert p["bars"] + 8 * (2 + 8) <= r, tag
         # phase 0-1 layout: qv then the W_q slice
         qv_end = r + G * 128 * 4
         assert qv_end <= p["r_wq"], tag
@@ -59,5 +60,7 @@ def test_plan_alignment_and_overlap(plans):
 
 def test_plan_fits_four_ctas_per_sm_at_the_benchmark_shape(plans):
     # Qwen3-4B, 32k context: G = 4, 512 gate-key rows, budget 2,048, bf16
-    p = next(q for q in plans if q["G"] == 4 and q["mg"] == 512 and q["budget"] == 2048 and q["f32"] == 0)
-    assert 4 * (p["total"] + 1024) <= 228 * 1024
+    for gated in (0, 1):
+        p = next(q for q in plans if q["G"] == 4 and q["mg"] == 512 and q["budget"] == 2048 and q["f32"] == 0
+                 and q["gated"] == gated)
+        assert 4 * (p["total"] + 1024) <= 228 * 1024
