@@ -20,7 +20,7 @@ namespace {
 
 using sas::kDim;
 
-constexpr int32_t kAbiVersion = 3;
+constexpr int32_t kAbiVersion = 4;
 constexpr size_t kStatusBytes = 256;  // status word + padding
 constexpr int kMaxBudget = 16384;
 constexpr int kMaxGateBlocks = 16384;
@@ -113,6 +113,8 @@ sas::KvView make_view(const sas_config* cfg, const sas_kv* kv) {
   v.capacity = kv->capacity;
   v.num_pages = kv->num_pages;
   v.max_blocks_per_seq = kv->max_blocks_per_seq;
+  v.token_budgets = kv->token_budgets;
+  v.max_budget = cfg->token_budget;
   return v;
 }
 
@@ -352,9 +354,9 @@ sas_status sas_gate_scores(const sas_config* cfg, const void* q, const int32_t* 
 }
 
 sas_status sas_topk_blocks(const sas_config* cfg, const float* group_scores,
-                           const int32_t* seq_lens, int32_t batch, int32_t max_gate_blocks,
-                           int32_t* sel_idx, int32_t* sel_count, void* ws, size_t ws_bytes,
-                           sas_stream_t stream) {
+                           const int32_t* seq_lens, const int32_t* token_budgets, int32_t batch,
+                           int32_t max_gate_blocks, int32_t* sel_idx, int32_t* sel_count, void* ws,
+                           size_t ws_bytes, sas_stream_t stream) {
   sas_status st = check_config(cfg);
   if (st != SAS_OK) return st;
   if ((st = check_ws(cfg, ws, ws_bytes)) != SAS_OK) return st;
@@ -363,7 +365,7 @@ sas_status sas_topk_blocks(const sas_config* cfg, const float* group_scores,
   if (group_scores == nullptr || seq_lens == nullptr || sel_idx == nullptr || sel_count == nullptr)
     return SAS_ERR_INVALID_ARG;
   if (!aligned(group_scores, 4) || !aligned(seq_lens, 4) || !aligned(sel_idx, 4) ||
-      !aligned(sel_count, 4))
+      !aligned(sel_count, 4) || !aligned(token_budgets, 4))
     return SAS_ERR_INVALID_ARG;
   if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
   sas::TopkParams p{};
@@ -373,6 +375,7 @@ sas_status sas_topk_blocks(const sas_config* cfg, const float* group_scores,
   p.mg = max_gate_blocks;
   p.group_scores = group_scores;
   p.seq_lens = seq_lens;
+  p.token_budgets = token_budgets;
   p.sel_idx = sel_idx;
   p.sel_count = sel_count;
   p.status = static_cast<uint32_t*>(ws);

@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   int* len_s = reinterpret_cast<int*>(qbar);  // qbar is written only after the validation
   if (tid == 0) {
     const int L0 = p.kv.seq_lens[s];
+    const int topk0 = (MODE == kModeFused) ? p.kv.topk_of(s) : 0;  // this sequence's budget
     // the descriptors of the maps this mode uses are fetched while the plain
     // copies go out
     if (MODE != kModeAttend) prefetch_tensormap(&tmw);
@@ -167,7 +168,8 @@ __global__ void __launch_bounds__(kThreads, 4)
         tma_load_2d(wq_s + static_cast<size_t>(g) * kDim * kDpc, &tmw, rank * kDpc, (h * G + g) * kDim,
                     bar_pro);
     }
-    *len_s = L0;
+    len_s[0] = L0;
+    len_s[1] = topk0;
   }
   SAS_TRACE(16);  // thread 0: prologue copies requested
   // thread 0 arrives after its barrier initialisation: no CTA of the cluster
@@ -181,8 +183,9 @@ __global__ void __launch_bounds__(kThreads, 4)
 
   // ------------------------------------------------------------ validation
   __syncthreads();
-  const int L = *len_s;
-  bool err = (L < 1);
+  const int L = len_s[0];
+  const int topk = len_s[1];  // fused mode: historical blocks kept for this sequence
+  bool err = (L < 1) || topk < 0;
   const int c = err ? 0 : (L - 1) / kBlock;  // current block
   if (MODE != kModeAttend && c > p.mg) err = true;
   if (MODE == kModeFused && !err) {
@@ -213,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   const int n = bad ? 0 : c;  // historical blocks
   // the decoded token completes block c: pool it into gate-key row c
   const bool do_pool = pool_on && !bad && (L % kBlock == 0) && (c < p.mg);
-  if (MODE == kModeFused) m = bad ? 0 : min(p.topk, n) + 1;
+  if (MODE == kModeFused) m = bad ? 0 : min(topk, n) + 1;
   if (MODE == kModeAttend && bad) m = 0;
 
   const int nb_per = (n + CS - 1) / CS;
@@ -463,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 #endif
         list_ok = __syncthreads_and(list_ok) != 0;
         if (list_ok) {
-          select_blocks(keys, n, p.topk, c, sel, hist, selbits, scan, tr);
+          select_blocks(keys, n, topk, c, sel, hist, selbits, scan, tr);
         } else {  // scores missing (timeout, in the status word): a valid stand-in list
           for (int j = tid; j < m; j += kThreads) sel[j] = c;
           __syncthreads();
@@ -916,7 +919,12 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
   q += ((p.mg + 31) / 32 * 4 + 15) / 16 * 16;
   int* scan = reinterpret_cast<int*>(q);
   const int L = p.seq_lens[s];
-  if (L < 1 || (L - 1) / kBlock > p.mg) {
+  int topk = p.topk;
+  if (p.token_budgets != nullptr) {
+    const int b = p.token_budgets[s];
+    topk = (b >= kBlock && b <= (p.topk + 1) * kBlock && b % kBlock == 0) ? b / kBlock - 1 : -1;
+  }
+  if (L < 1 || (L - 1) / kBlock > p.mg || topk < 0) {
     if (tid == 0) {
       raise_status(p.status, kStatusBounds);
       p.sel_count[pair] = 0;
@@ -926,7 +934,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
   const int c = (L - 1) / kBlock;
   for (int b = tid; b < c; b += kThreads) vals[b] = p.group_scores[static_cast<size_t>(pair) * p.mg + b];
   __syncthreads();
-  const int m = select_blocks(vals, c, p.topk, c, sel, hist, selbits, scan);
+  const int m = select_blocks(vals, c, topk, c, sel, hist, selbits, scan);
   for (int j = tid; j < m; j += kThreads) p.sel_idx[static_cast<size_t>(pair) * p.max_sel + j] = sel[j];
   if (tid == 0) p.sel_count[pair] = m;
 }

@@ -448,6 +448,16 @@ struct KvView {
   int32_t capacity;
   int32_t num_pages;
   int32_t max_blocks_per_seq;
+  const int32_t* token_budgets;  // null: max_budget for every sequence
+  int32_t max_budget;            // the configured budget (sizes the block lists)
+
+  // Historical blocks kept for sequence s (budget/64 - 1), or -1 for a
+  // budget that is not a multiple of 64 in 64 .. max_budget.
+  __device__ __forceinline__ int topk_of(int s) const {
+    const int b = (token_budgets != nullptr) ? token_budgets[s] : max_budget;
+    if (b < kBlock || b > max_budget || b % kBlock != 0) return -1;
+    return b / kBlock - 1;
+  }
 
   __device__ __forceinline__ long long block_row(int s, int h, int b) const {
     if (b < 0) return -1;

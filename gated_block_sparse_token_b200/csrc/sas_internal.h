@@ -131,6 +131,7 @@ struct TopkParams {
   int hkv, topk, max_sel, mg;
   const float* group_scores;
   const int32_t* seq_lens;
+  const int32_t* token_budgets;  // null: topk for every sequence
   int32_t* sel_idx;
   int32_t* sel_count;
   uint32_t* status;

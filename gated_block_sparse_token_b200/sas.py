@@ -56,7 +56,8 @@ class _Kv(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
                 ("block_table", ctypes.c_void_p), ("seq_lens", ctypes.c_void_p),
                 ("batch", ctypes.c_int32), ("capacity", ctypes.c_int32),
-                ("num_pages", ctypes.c_int32), ("max_blocks_per_seq", ctypes.c_int32)]
+                ("num_pages", ctypes.c_int32), ("max_blocks_per_seq", ctypes.c_int32),
+                ("token_budgets", ctypes.c_void_p)]
 
 
 _lib = None
@@ -80,7 +81,7 @@ def lib() -> ctypes.CDLL:
             "sas_get_device_status": (ctypes.c_int, [vp, vp, ctypes.POINTER(ctypes.c_int)]),
             "sas_pool_keys": (ctypes.c_int, [cfgp, kvp, vp, i32, vp, vp, vp, i32, vp, vp, sz, vp]),
             "sas_gate_scores": (ctypes.c_int, [cfgp, vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, sz, vp]),
-            "sas_topk_blocks": (ctypes.c_int, [cfgp, vp, vp, i32, i32, vp, vp, vp, sz, vp]),
+            "sas_topk_blocks": (ctypes.c_int, [cfgp, vp, vp, vp, i32, i32, vp, vp, vp, sz, vp]),
             "sas_sparse_decode": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step_static": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]),
@@ -153,6 +154,7 @@ class KvCache:
     v: torch.Tensor
     seq_lens: torch.Tensor
     block_table: Optional[torch.Tensor] = None
+    token_budgets: Optional[torch.Tensor] = None   # int32 [B]; None: the config's budget
     _c: Optional[_Kv] = field(default=None, repr=False)
 
     @property
@@ -162,9 +164,10 @@ class KvCache:
     def c(self) -> _Kv:
         if self.block_table is None:
             return _Kv(_ptr(self.k), _ptr(self.v), None, _ptr(self.seq_lens), self.batch,
-                       int(self.k.shape[2]), 0, 0)
+                       int(self.k.shape[2]), 0, 0, _ptr(self.token_budgets))
         return _Kv(_ptr(self.k), _ptr(self.v), _ptr(self.block_table), _ptr(self.seq_lens),
-                   self.batch, 0, int(self.k.shape[0]), int(self.block_table.shape[1]))
+                   self.batch, 0, int(self.k.shape[0]), int(self.block_table.shape[1]),
+                   _ptr(self.token_budgets))
 
 
 def abi_version() -> int:
@@ -212,9 +215,10 @@ def gate_scores(cfg: Config, q, seq_lens, w_q, gamma_q, gate_keys, group_scores,
                                  _stream(stream)), "sas_gate_scores")
 
 
-def topk_blocks(cfg: Config, group_scores, seq_lens, sel_idx, sel_count, ws, stream=None) -> None:
+def topk_blocks(cfg: Config, group_scores, seq_lens, sel_idx, sel_count, ws, stream=None,
+                token_budgets=None) -> None:
     c = cfg.c()
-    _check(lib().sas_topk_blocks(ctypes.byref(c), _ptr(group_scores), _ptr(seq_lens),
+    _check(lib().sas_topk_blocks(ctypes.byref(c), _ptr(group_scores), _ptr(seq_lens), _ptr(token_budgets),
                                  int(seq_lens.shape[0]), int(group_scores.shape[2]), _ptr(sel_idx),
                                  _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),
            "sas_topk_blocks")

@@ -127,6 +127,14 @@ typedef struct {
                                   of 64; paged: ignored */
   int32_t num_pages;           /* paged: pages in the pool; contiguous: ignored */
   int32_t max_blocks_per_seq;  /* paged: row length of block_table */
+  const int32_t* token_budgets; /* NULL: cfg->token_budget for every sequence.
+                                   Else [B] per-sequence budgets (pages: 1,024,
+                                   2,048 or 4,096 usable without retraining),
+                                   each a multiple of 64 in 64 ..
+                                   cfg->token_budget; cfg->token_budget sizes
+                                   the block lists.  A sequence with a bad
+                                   budget is skipped and reported as
+                                   SAS_ERR_DEVICE_BOUNDS. */
 } sas_kv;
 
 /* Bytes of device workspace `ws` every entry point below needs for this
@@ -190,13 +198,14 @@ SAS_API sas_status sas_gate_scores(const sas_config* cfg, const void* q, const i
  * Top-K block selection under the token budget (pages: training Top-K 31,
  * default budget 2,048; 1,024 and 4,096 usable without retraining).
  *   group_scores fp32 [B][Hkv][MG]
- *   sel_idx   int32 [B][Hkv][budget/64]: ascending block ids, the current
+ *   token_budgets: NULL (cfg->token_budget for all) or int32 [B], as in sas_kv
+ *   sel_idx   int32 [B][Hkv][cfg budget/64]: ascending block ids, the current
  *             block c_s last; entries past sel_count are left untouched
- *   sel_count int32 [B][Hkv] = min(budget/64, c_s + 1)
+ *   sel_count int32 [B][Hkv] = min(budget_s/64, c_s + 1)
  */
 SAS_API sas_status sas_topk_blocks(const sas_config* cfg, const float* group_scores,
-                           const int32_t* seq_lens, int32_t batch, int32_t max_gate_blocks,
-                           int32_t* sel_idx, int32_t* sel_count,
+                           const int32_t* seq_lens, const int32_t* token_budgets, int32_t batch,
+                           int32_t max_gate_blocks, int32_t* sel_idx, int32_t* sel_count,
                            void* ws, size_t ws_bytes, sas_stream_t stream);
 
 /*

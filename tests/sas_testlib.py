@@ -113,18 +113,20 @@ def assert_selection(gpu_sel, oracle_sel, S, topk, what=""):
     return True
 
 
-def check_pairs(inputs, cfg, gpu, oracle, gate_keys=None, out_atol=OUT_ATOL):
-    """Compare a fused decode step's outputs with the oracle on the given pairs."""
+def check_pairs(inputs, cfg, gpu, oracle, gate_keys=None, out_atol=OUT_ATOL, budgets=None):
+    """Compare a fused decode step's outputs with the oracle on the given pairs
+    (budgets: per-sequence token budgets, else the config's)."""
     spec = inputs["spec"]
     G = spec.hq // spec.hkv
-    topk = cfg.max_sel - 1
     out = gpu["out"].float().cpu().numpy()
     sel_idx = gpu["sel_idx"].cpu().numpy()
     sel_count = gpu["sel_count"].cpu().numpy()
     gs = gpu["group_scores"].cpu().numpy()
     gkeys = None if gate_keys is None else gate_keys.cpu().numpy()
     for (s, h), r in oracle.items():
-        tag = f"{spec.name} s={s} h={h} budget={cfg.token_budget}"
+        budget = cfg.token_budget if budgets is None else int(budgets[s])
+        topk = budget // 64 - 1
+        tag = f"{spec.name} s={s} h={h} budget={budget}"
         c = len(r["S"])
         if gkeys is not None:
             assert_close_rel(gkeys[s, h, :c], r["gate_keys"], tag + " gate keys")

@@ -62,7 +62,7 @@ int main(void) {
   O(sas_config, token_budget); O(sas_config, rope_base); O(sas_config, gate_scale);
   O(sas_config, kv_dtype); O(sas_config, out_dtype); O(sas_config, gate_mode);
   O(sas_kv, block_table); O(sas_kv, seq_lens); O(sas_kv, batch); O(sas_kv, capacity);
-  O(sas_kv, num_pages); O(sas_kv, max_blocks_per_seq);
+  O(sas_kv, num_pages); O(sas_kv, max_blocks_per_seq); O(sas_kv, token_budgets);
   return 0;
 }
 '''
@@ -84,7 +84,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(L):
-    assert sas.abi_version() >= 3
+    assert sas.abi_version() >= 4
     for st in range(7):
         assert len(sas.status_string(st)) > 0
     assert sas.status_string(sas.SAS_OK) == "ok"
@@ -179,8 +179,10 @@ def test_other_entry_points_validate(L):
                            FAKE, 256, None) == sas.SAS_ERR_INVALID_ARG
     assert L.sas_gate_scores(ctypes.byref(c), FAKE, FAKE, 2, FAKE, FAKE, FAKE, 64, None, None,
                              FAKE, 256, None) == sas.SAS_ERR_INVALID_ARG
-    assert L.sas_topk_blocks(ctypes.byref(c), FAKE, FAKE, 2, 64, FAKE, None, FAKE, 256,
+    assert L.sas_topk_blocks(ctypes.byref(c), FAKE, FAKE, None, 2, 64, FAKE, None, FAKE, 256,
                              None) == sas.SAS_ERR_INVALID_ARG
+    assert L.sas_topk_blocks(ctypes.byref(c), FAKE, FAKE, FAKE + 2, 2, 64, FAKE, FAKE, FAKE, 256,
+                             None) == sas.SAS_ERR_INVALID_ARG  # misaligned budgets
     assert L.sas_sparse_decode(ctypes.byref(c), FAKE, ctypes.byref(kv), None, FAKE, FAKE, FAKE,
                                256, None) == sas.SAS_ERR_INVALID_ARG
     st = ctypes.c_int(0)
