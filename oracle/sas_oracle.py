@@ -65,6 +65,11 @@ R18 Gated inference mode (a variant of R12; "continuous gates act on the
     token of a selected historical block b, for query head g, get the
     additive bias log(sigmoid(s_{g,b})) with s_{g,b} the head's gate score
     (R7); the current block gets 0.  Gates equal to 1 reduce it to R12.
+R19 bf16 gate-key cache (a storage option, not a change of the method): the
+    gate key k~_b is computed as before and stored rounded to the nearest
+    bf16 value (ties to even); scores use the stored value.  The release
+    ships its gate weights in bf16 ([lmw-en] table: the printed checkpoint
+    sizes fit bf16 weights).
 
 Parity status: the gate formula as a whole (R1-R8) is pinned only by the
 invariants and hand-derived closed forms in tests/test_oracle.py, not by any
@@ -201,6 +206,24 @@ def topk_for_budget(token_budget: int) -> int:
 # --------------------------------------------------------------------------
 # Step 4: attention over the selected blocks (R12, R14).
 # --------------------------------------------------------------------------
+def round_to_bf16(x) -> np.ndarray:
+    """Round to the nearest bfloat16 value, ties to even (R19).  bfloat16 is
+    the upper half of an IEEE binary32: 1 sign, 8 exponent, 7 fraction bits.
+    The value is first rounded to binary32 (float64 -> float32 is itself
+    round-to-nearest-even), then the low 16 bits of the binary32 pattern are
+    rounded away: add 0x7FFF plus the lowest kept bit, clear the low half.
+    Infinities stay, NaN stays NaN."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    keep_lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + keep_lsb) & 0xFFFF0000).astype(np.uint32)
+    out = r.view(np.float32).astype(np.float64)
+    nan = np.isnan(f)
+    if np.any(nan):
+        out = np.where(nan, np.nan, out)
+    return out
+
+
 GATE_SELECT_ONLY = 0       # R12: selected blocks weighted 1
 GATE_LOGSIGMOID_BIAS = 1   # R18: + log(sigmoid(s_{g,b})) on block b's logits
 

@@ -387,6 +387,43 @@ def test_log_sigmoid_values():
     assert -1e-300 < O.log_sigmoid(800.0) <= 0.0
 
 
+# ---------------------------------------------------------------- bf16 gate-key storage (R19)
+def test_round_to_bf16_worked_values():
+    """Hand-worked bfloat16 roundings: 8 significant bits (1 implicit + 7)."""
+    cases = [
+        (1.0, 1.0),
+        (1.0 + 2 ** -8, 1.0),                  # exactly half an ulp above 1: tie, 1.0 is even
+        (1.0 + 3 * 2 ** -8, 1.0 + 2 ** -6),    # tie between 1+2^-7 (odd) and 1+2^-6 (even)
+        (1.0 + 2 ** -8 + 2 ** -20, 1.0 + 2 ** -7),   # just above the tie: up
+        (1.0 + 2 ** -7, 1.0 + 2 ** -7),        # representable
+        (-2.5, -2.5),
+        (3.0e38, 1.765625 * 2.0 ** 127),       # 1.11000011..b * 2^127 rounds up to 1.1100010b
+        (1.0e-40, 9.99e-41),                   # binary32 subnormal, kept to 7 fraction bits
+        (0.1, 0.10009765625),                  # 0x3DCD
+        (65504.0, 65536.0),
+    ]
+    for x, want in cases:
+        got = float(O.round_to_bf16(x))
+        assert got == pytest.approx(want, rel=2 ** -9), (x, got, want)
+    assert float(O.round_to_bf16(0.1)) == 0.10009765625
+    assert float(O.round_to_bf16(1.0 + 2 ** -8)) == 1.0
+    assert float(O.round_to_bf16(1.0 + 3 * 2 ** -8)) == 1.0 + 2 ** -6
+    assert np.isinf(O.round_to_bf16(np.inf)) and np.isnan(O.round_to_bf16(np.nan))
+
+
+def test_round_to_bf16_is_idempotent_and_within_half_ulp():
+    x = np.random.default_rng(9).standard_normal(10000) * 10.0 ** np.random.default_rng(10).integers(-6, 6, 10000)
+    r = O.round_to_bf16(x)
+    assert np.array_equal(O.round_to_bf16(r), r)
+    # |x - r| <= 2^-8 |x|: unit roundoff of an 8-bit significand (float32 step aside)
+    assert np.all(np.abs(x - r) <= 2.0 ** -8 * np.abs(x) * (1 + 2 ** -14) + 1e-300)
+    # an independent implementation: torch's float32 -> bfloat16 conversion
+    import torch
+    assert np.array_equal(torch.tensor(x).float().bfloat16().double().numpy(), r)
+    # the bf16 pattern has a zero low half
+    assert np.all((r.astype(np.float32).view(np.uint32) & 0xFFFF) == 0)
+
+
 # ---------------------------------------------------------------- planted mistakes
 def test_pins_catch_planted_mistakes(monkeypatch):
     """Plant plausible mistakes in the oracle (CPU) and show a pin fails."""
