@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--prefill-steps", type=int, default=5)
     ap.add_argument("--skip-prefill", action="store_true")
     ap.add_argument("--prefill-only", action="store_true")
+    ap.add_argument("--variant-steps", type=int, default=4000)
+    ap.add_argument("--skip-variants", action="store_true")
     return ap.parse_args()
 
 
@@ -174,20 +176,22 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- algorithmic bytes
-def decode_bytes(seq_lens, hq, hkv, budget, kv_elem=2, pool=True):
+def decode_bytes(seq_lens, hq, hkv, budget, kv_elem=2, pool=True, gk_elem=4):
     """Bytes one fused decode step must move: the selected K/V tokens, the fp32
     gate key of every historical block, q and out of every head and W_q once;
     with pooling of the completed current block also W_k once and the new
-    gate keys (the block's K is already among the selected tokens)."""
+    gate keys (the block's K is already among the selected tokens).  budget:
+    one for the batch, or one per sequence."""
     G = hq // hkv
     tot = 0
-    for L in seq_lens:
+    budgets = budget if isinstance(budget, (list, tuple)) else [budget] * len(seq_lens)
+    for L, budget in zip(seq_lens, budgets):
         c = (L - 1) // 64
         m = min(budget // 64 - 1, c)
         cur_tokens = L - 64 * c
-        per_pair = (m * 64 + cur_tokens) * 128 * kv_elem * 2 + c * 128 * 4 + 2 * G * 128 * 2
+        per_pair = (m * 64 + cur_tokens) * 128 * kv_elem * 2 + c * 128 * gk_elem + 2 * G * 128 * 2
         if pool and L % 64 == 0:
-            per_pair += 128 * 4
+            per_pair += 128 * gk_elem
         tot += hkv * per_pair
     tot += hq * 128 * 128 * 2
     if pool:
@@ -293,19 +297,21 @@ def profiled_traffic():
 
 
 # ---------------------------------------------------------------- our arm
-def build_layers(R, rank, device):
+def build_layers(R, rank, device, gate_mode=0, budgets=None, gk16=0):
     import torch
     from gated_block_sparse_token_b200 import sas
     from gated_block_sparse_token_b200.workloads import make_decode_inputs, qwen3_4b_32k
 
-    cfg = sas.Config(HQ, HKV, token_budget=BUDGET)
+    cfg = sas.Config(HQ, HKV, token_budget=BUDGET if budgets is None else max(budgets), gate_mode=gate_mode,
+                     gate_keys_bf16=gk16)
+    tb = None if budgets is None else torch.tensor(budgets, dtype=torch.int32, device=device)
     layers = []
     for li in range(R):
         spec = qwen3_4b_32k(batch=BATCH, seq_len=CTX, seed=1000 * (rank + 1) + li)
         inp = make_decode_inputs(spec, device)
-        kv = sas.KvCache(inp["k"], inp["v"], inp["seq_lens"])
+        kv = sas.KvCache(inp["k"], inp["v"], inp["seq_lens"], token_budgets=tb)
         mg = spec.cap // 64
-        gk = torch.zeros(BATCH, HKV, mg, 128, dtype=torch.float32, device=device)
+        gk = torch.zeros(BATCH, HKV, mg, 128, dtype=sas.gate_key_dtype(cfg), device=device)
         ws = sas.make_workspace(cfg, device)
         sas.pool_keys(cfg, kv, inp["w_k"], inp["gamma_k"], gk, ws)  # prefill-time keys (untimed)
         cur = torch.full((BATCH,), (CTX - 1) // 64, dtype=torch.int32, device=device)
@@ -366,6 +372,47 @@ def timed(graphs, world, stream):
     torch.cuda.synchronize()
     barrier(world)
     return max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+
+
+MIXED_BUDGETS = [1024, 2048, 4096, 2048, 1024, 4096, 2048, 2048]
+
+
+def run_variant(args, rank, world, device, name, gate_mode=0, budgets=None, gk16=0):
+    """The same decode workload in one of the widened modes (the gated
+    inference mode, or mixed per-sequence budgets), timed like the main line
+    on a shorter run; reports steps/s and the kernel's HBM roofline."""
+    import torch
+    from gated_block_sparse_token_b200 import sas
+    cfg, layers = build_layers(args.layers, rank, device, gate_mode=gate_mode, budgets=budgets, gk16=gk16)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for L in layers:
+            step(cfg, L, stream)
+    torch.cuda.synchronize()
+    fn = lambda L, st: step(cfg, L, st)  # noqa: E731
+    warm = plan(fn, max(args.warmup // 4, 3 * len(layers)), layers, stream)
+    main = plan(fn, args.variant_steps, layers, stream)
+    with torch.cuda.stream(stream):
+        run_graphs(warm)
+    torch.cuda.synchronize()
+    t = timed(main, world, stream)
+    for L in layers:
+        if sas.get_device_status(L["ws"], stream) != sas.SAS_OK:
+            raise RuntimeError(f"device status not OK after the {name} run")
+    del layers, main, warm
+    torch.cuda.empty_cache()
+    peak, peak_kind = measured_peaks()
+    dbytes = decode_bytes([CTX] * BATCH, HQ, HKV, budgets if budgets is not None else BUDGET,
+                          gk_elem=2 if gk16 else 4)
+    dec_s = t / args.variant_steps
+    achieved = dbytes / dec_s / 1e9
+    return {"mode": name, "token_budgets": budgets if budgets is not None else [BUDGET] * BATCH,
+            "gate_mode": gate_mode, "gate_keys": "bf16" if gk16 else "fp32", "steps": args.variant_steps,
+            "value": round(job_throughput(args.variant_steps, world, t), 2), "unit": UNIT,
+            "ms_per_step": round(dec_s * 1e3, 5),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+                         "bytes_per_launch": dbytes, "avg_launch_us": round(dec_s * 1e6, 3)}}
 
 
 def cpu_baseline(seconds):
@@ -445,6 +492,11 @@ def run_ours(args):
 
     del layers, main, warm
     torch.cuda.empty_cache()
+    variants = []
+    if not args.skip_variants:
+        variants.append(run_variant(args, rank, world, device, "gated (log-sigmoid bias)", gate_mode=1))
+        variants.append(run_variant(args, rank, world, device, "mixed budgets", budgets=MIXED_BUDGETS))
+        variants.append(run_variant(args, rank, world, device, "bf16 gate keys", gk16=1))
     pf = None if args.skip_prefill else run_prefill(args, device, world)
 
     if rank != 0:
@@ -479,6 +531,8 @@ def run_ours(args):
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if variants:
+        line["variants"] = variants
     if pf is not None:
         line["prefill"] = pf
     print(json.dumps(line), flush=True)

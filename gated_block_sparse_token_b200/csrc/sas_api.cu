@@ -20,7 +20,7 @@ namespace {
 
 using sas::kDim;
 
-constexpr int32_t kAbiVersion = 4;
+constexpr int32_t kAbiVersion = 5;
 constexpr size_t kStatusBytes = 256;  // status word + padding
 constexpr int kMaxBudget = 16384;
 constexpr int kMaxGateBlocks = 16384;
@@ -74,6 +74,7 @@ sas_status check_config(const sas_config* c) {
   if (c->out_dtype != SAS_DTYPE_BF16 && c->out_dtype != SAS_DTYPE_F32) return SAS_ERR_INVALID_ARG;
   if (c->gate_mode != SAS_GATE_SELECT_ONLY && c->gate_mode != SAS_GATE_LOGSIGMOID_BIAS)
     return SAS_ERR_INVALID_ARG;
+  if (c->gate_keys_bf16 != 0 && c->gate_keys_bf16 != 1) return SAS_ERR_INVALID_ARG;
   return SAS_OK;
 }
 
@@ -183,6 +184,7 @@ void fill_common(sas::DecodeParams& p, const sas_config* cfg, int mg) {
   p.attn_scale_log2 = cfg->attn_scale * 1.4426950408889634f;
   p.gate_scale = cfg->gate_scale;
   p.gated = cfg->gate_mode == SAS_GATE_LOGSIGMOID_BIAS ? 1 : 0;
+  p.gk16 = cfg->gate_keys_bf16;
   p.sm = sas::plan_decode_smem(p.G, mg, kClusterSize, kStages, p.max_sel,
                                cfg->kv_dtype == SAS_DTYPE_F32, p.gated != 0);
   sas::fill_rope_table(p.rope, cfg->rope_base);
@@ -280,7 +282,7 @@ sas_status sas_get_device_status(const void* ws, sas_stream_t stream, sas_status
 
 sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv, const int32_t* blk_begin,
                          int32_t num_blocks, const void* w_k, const float* gamma_k,
-                         float* gate_keys, int32_t max_gate_blocks, float* pooled_raw, void* ws,
+                         void* gate_keys, int32_t max_gate_blocks, float* pooled_raw, void* ws,
                          size_t ws_bytes, sas_stream_t stream) {
   sas_status st = check_config(cfg);
   if (st != SAS_OK) return st;
@@ -308,6 +310,7 @@ sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv, const int32_t*
   p.w_k = static_cast<const __nv_bfloat16*>(w_k);
   p.gamma_k = gamma_k;
   p.gate_keys = gate_keys;
+  p.gk16 = cfg->gate_keys_bf16;
   p.pooled_raw = pooled_raw;
   p.status = static_cast<uint32_t*>(ws);
   return launch_result(sas::launch_pool(cfg->kv_dtype == SAS_DTYPE_F32, p, kv->batch,
@@ -316,7 +319,7 @@ sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv, const int32_t*
 
 sas_status sas_gate_scores(const sas_config* cfg, const void* q, const int32_t* seq_lens,
                            int32_t batch, const void* w_q, const float* gamma_q,
-                           const float* gate_keys, int32_t max_gate_blocks, float* head_scores,
+                           const void* gate_keys, int32_t max_gate_blocks, float* head_scores,
                            float* group_scores, void* ws, size_t ws_bytes, sas_stream_t stream) {
   sas_status st = check_config(cfg);
   if (st != SAS_OK) return st;
@@ -384,7 +387,7 @@ sas_status sas_topk_blocks(const sas_config* cfg, const float* group_scores,
 
 static sas_status attention_call(int mode, const sas_config* cfg, const void* q, const sas_kv* kv,
                                  const void* w_q, const float* gamma_q, const void* w_k,
-                                 const float* gamma_k, float* gate_keys, int32_t max_gate_blocks,
+                                 const float* gamma_k, void* gate_keys, int32_t max_gate_blocks,
                                  void* out, int32_t* sel_idx, int32_t* sel_count,
                                  float* group_scores, void* ws, size_t ws_bytes,
                                  sas_stream_t stream) {
@@ -448,7 +451,7 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
 sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const void* k,
                                     const void* v, int32_t batch, int32_t seq_len,
                                     const void* w_q, const float* gamma_q, const void* w_k,
-                                    const float* gamma_k, float* gate_keys,
+                                    const float* gamma_k, void* gate_keys,
                                     int32_t max_gate_blocks, void* out, int32_t* sel_idx,
                                     int32_t* sel_count, void* ws, size_t ws_bytes,
                                     sas_stream_t stream) {
@@ -502,6 +505,7 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
   pp.w_k = static_cast<const __nv_bfloat16*>(w_k);
   pp.gamma_k = gamma_k;
   pp.gate_keys = gate_keys;
+  pp.gk16 = cfg->gate_keys_bf16;
   pp.pooled_raw = nullptr;
   pp.status = static_cast<uint32_t*>(ws);
   cudaError_t e = sas::launch_pool(false, pp, batch, s);
@@ -526,6 +530,7 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
   p.w_q = static_cast<const __nv_bfloat16*>(w_q);
   p.gamma_q = gamma_q;
   p.gate_keys = gate_keys;
+  p.gk16 = cfg->gate_keys_bf16;
   uint8_t* scratch = static_cast<uint8_t*>(ws) + ws_header_bytes();
   p.qt = reinterpret_cast<float*>(scratch);
   scratch += up256(static_cast<size_t>(batch) * p.hq * nblk * kDim * 4);
@@ -555,7 +560,7 @@ sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const sas_kv*
 
 sas_status sas_decode_step(const sas_config* cfg, const void* q, const sas_kv* kv, const void* w_q,
                            const float* gamma_q, const void* w_k, const float* gamma_k,
-                           float* gate_keys, int32_t max_gate_blocks, void* out,
+                           void* gate_keys, int32_t max_gate_blocks, void* out,
                            int32_t* sel_idx, int32_t* sel_count, float* group_scores, void* ws,
                            size_t ws_bytes, sas_stream_t stream) {
   return attention_call(sas::kModeFused, cfg, q, kv, w_q, gamma_q, w_k, gamma_k, gate_keys,

@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   uint64_t* bar_v = bars + NST + 5;   // the gate query v (a slice from each CTA)
   uint64_t* bar_m = bars + NST + 6;   // attention partials of this CTA's columns
   uint64_t* bar_u = bars + NST + 7;   // rank 0: projected pooled slices
+  uint64_t* bar_gb = bars + NST + 8;  // ranks > 0, gated mode: the gates of the list
   float* pool_p = reinterpret_cast<float*>(base + p.sm.r_pool_p);
   float* pool_u = reinterpret_cast<float*>(base + p.sm.r_pool_u);
   __nv_bfloat16* wk_s = reinterpret_cast<__nv_bfloat16*>(base + p.sm.r_wk);
@@ -152,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 4)
       prefetch_tensormap(&tmv);
     }
     if (pool_on) prefetch_tensormap(&tmwk);
-    for (int i = 0; i < NST + 8; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < NST + 9; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
     const uint32_t qbytes = static_cast<uint32_t>(G * kDim * sizeof(T));
     uint32_t tx = qbytes;
@@ -222,7 +223,11 @@ __global__ void __launch_bounds__(kThreads, 4)
   const int nb_per = (n + CS - 1) / CS;
   const int b_lo = min(n, rank * nb_per);
   const int b_hi = min(n, b_lo + nb_per);
-  const int nchunks = (MODE == kModeAttend) ? 0 : (b_hi - b_lo + kGkChunk - 1) / kGkChunk;
+  // gate-key rows per 16 KiB ring slot: 32 fp32 rows or 64 bf16 rows
+  const int gk_rows = p.gk16 ? 2 * kGkChunk : kGkChunk;
+  const uint32_t gk_row_bytes = p.gk16 ? kDim * 2u : kDim * 4u;
+  const uint8_t* gk_pair = static_cast<const uint8_t*>(p.gate_keys) + static_cast<size_t>(pair) * p.mg * gk_row_bytes;
+  const int nchunks = (MODE == kModeAttend) ? 0 : (b_hi - b_lo + gk_rows - 1) / gk_rows;
   const int cnt_mine = (rank < m) ? (m - 1 - rank) / CS + 1 : 0;
   const bool own_cur = (m > 0) && ((m - 1) % CS == rank);
 
@@ -232,8 +237,10 @@ __global__ void __launch_bounds__(kThreads, 4)
     if (MODE == kModeFused && !bad) {
       if (rank == 0)
         mbar_arrive_expect_tx(bar_sc, static_cast<uint32_t>(n * 4));
-      else
-        mbar_arrive_expect_tx(bar_sel, static_cast<uint32_t>(m * 4 * (gated ? 1 + G : 1)));
+      else {
+        mbar_arrive_expect_tx(bar_sel, static_cast<uint32_t>(m * 4));
+        if (gated) mbar_arrive_expect_tx(bar_gb, static_cast<uint32_t>(m * G * 4));
+      }
     }
     if (do_pool) {
       mbar_arrive_expect_tx(bar_p, kPool * 4);
@@ -261,12 +268,11 @@ __global__ void __launch_bounds__(kThreads, 4)
     const int slot = t % NST;
     uint8_t* dst = slots + slot * kTileBytes;
     if (t < nchunks) {
-      const int b0 = b_lo + t * kGkChunk;
-      const int cntb = min(kGkChunk, b_hi - b0);
-      const uint32_t bytes = static_cast<uint32_t>(cntb) * kDim * 4u;
+      const int b0 = b_lo + t * gk_rows;
+      const int cntb = min(gk_rows, b_hi - b0);
+      const uint32_t bytes = static_cast<uint32_t>(cntb) * gk_row_bytes;
       mbar_arrive_expect_tx(&bars[slot], bytes);
-      bulk_g2s(dst, p.gate_keys + (static_cast<size_t>(pair) * p.mg + b0) * kDim, bytes,
-               &bars[slot]);
+      bulk_g2s(dst, gk_pair + static_cast<size_t>(b0) * gk_row_bytes, bytes, &bars[slot]);
       return;
     }
     const int k = t - nchunks;
@@ -296,9 +302,8 @@ __global__ void __launch_bounds__(kThreads, 4)
   pump(0, known);
   if (tid == 0 && nchunks > NST) {
     // the ring holds NST chunks: ask L2 for the rest of this CTA's gate keys now
-    const int b0 = b_lo + NST * kGkChunk;
-    prefetch_l2(p.gate_keys + (static_cast<size_t>(pair) * p.mg + b0) * kDim,
-                static_cast<uint32_t>(b_hi - b0) * kDim * 4u);
+    const int b0 = b_lo + NST * gk_rows;
+    prefetch_l2(gk_pair + static_cast<size_t>(b0) * gk_row_bytes, static_cast<uint32_t>(b_hi - b0) * gk_row_bytes);
   }
   SAS_TRACE(1);
 
@@ -373,7 +378,9 @@ __global__ void __launch_bounds__(kThreads, 4)
     // ---------------------------------------------------------- phase 1: scores
     const int grp = lane >> 3;  // 4 blocks per warp at a time, 8 lanes per block
     const int sub = lane & 7;   // lane covers dims sub*16 .. sub*16+15
-    const int rot = sub >> 1;   // chunk rotation: conflict-free 16-byte loads
+    // fp32 keys: chunk rotation for conflict-free 16-byte loads; bf16 keys:
+    // natural order (each lane reads 32 contiguous bytes)
+    const int rot = p.gk16 ? 0 : sub >> 1;
     float4 qr[4];
     if (MODE == kModeFused) {
 #pragma unroll
@@ -383,21 +390,27 @@ __global__ void __launch_bounds__(kThreads, 4)
     for (int ci = 0; ci < nchunks; ++ci) {
       const int slot = ci % NST;
       const bool ok = mbar_wait(&bars[slot], (ci / NST) & 1, p.status);
-      const int b0 = b_lo + ci * kGkChunk;
-      const int cntb = min(kGkChunk, b_hi - b0);
+      const int b0 = b_lo + ci * gk_rows;
+      const int cntb = min(gk_rows, b_hi - b0);
       const float* gk = reinterpret_cast<const float*>(slots + slot * kTileBytes);
-#pragma unroll
-      for (int it = 0; it < kGkChunk / 16; ++it) {
+      const uint8_t* gk16 = slots + slot * kTileBytes;
+      for (int it = 0; it < gk_rows / 16; ++it) {
         const int bb = it * 16 + warp * 4 + grp;
         const bool act = ok && bb < cntb;
         const float* row = gk + bb * kDim + sub * 16;
+        const uint8_t* row16 = gk16 + bb * (kDim * 2) + sub * 32;
         float S = 0.f;
         if (MODE == kModeFused) {
           float acc = 0.f;
           if (act) {
+            if (p.gk16) {
+              acc = dot8_bf16(qr[0], qr[1], *reinterpret_cast<const uint4*>(row16), acc);
+              acc = dot8_bf16(qr[2], qr[3], *reinterpret_cast<const uint4*>(row16 + 16), acc);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              acc = dot4(qr[i], *reinterpret_cast<const float4*>(row + ((i + rot) & 3) * 4), acc);
+              for (int i = 0; i < 4; ++i)
+                acc = dot4(qr[i], *reinterpret_cast<const float4*>(row + ((i + rot) & 3) * 4), acc);
+            }
           }
           acc += __shfl_xor_sync(0xffffffffu, acc, 1);
           acc += __shfl_xor_sync(0xffffffffu, acc, 2);
@@ -410,11 +423,17 @@ __global__ void __launch_bounds__(kThreads, 4)
             float acc = 0.f;
             if (act) {
               const float* qrow = qv + g * kDim + sub * 16;
+              if (p.gk16) {
+                const float4* q4 = reinterpret_cast<const float4*>(qrow);
+                acc = dot8_bf16(q4[0], q4[1], *reinterpret_cast<const uint4*>(row16), acc);
+                acc = dot8_bf16(q4[2], q4[3], *reinterpret_cast<const uint4*>(row16 + 16), acc);
+              } else {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int ch = ((i + rot) & 3) * 4;
-                acc = dot4(*reinterpret_cast<const float4*>(qrow + ch),
-                           *reinterpret_cast<const float4*>(row + ch), acc);
+                for (int i = 0; i < 4; ++i) {
+                  const int ch = ((i + rot) & 3) * 4;
+                  acc = dot4(*reinterpret_cast<const float4*>(qrow + ch),
+                             *reinterpret_cast<const float4*>(row + ch), acc);
+                }
               }
             }
             acc += __shfl_xor_sync(0xffffffffu, acc, 1);
@@ -471,29 +490,6 @@ __global__ void __launch_bounds__(kThreads, 4)
           for (int j = tid; j < m; j += kThreads) sel[j] = c;
           __syncthreads();
         }
-        if (gated) {
-          // gate of every list entry and head: log(sigmoid(s_gb)), s_gb =
-          // (q~_g . k~_b) * gate_scale from q~ (v, rotated in place) and the
-          // block's gate key; 0 for the current block and a stand-in list
-          for (int w = warp; w < m * G; w += kWarps) {
-            const int j = w / G, g = w - j * G;
-            float beta = 0.f;
-            if (list_ok && j < m - 1) {
-              const float4 k4 = *reinterpret_cast<const float4*>(
-                  p.gate_keys + (static_cast<size_t>(pair) * p.mg + sel[j]) * kDim + 4 * lane);
-              const float4 q4 = *reinterpret_cast<const float4*>(qv + g * kDim + 4 * lane);
-              float a = fmaf(q4.x, k4.x, fmaf(q4.y, k4.y, fmaf(q4.z, k4.z, q4.w * k4.w)));
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-              const float sg = a * p.gate_scale;
-              beta = (sg >= 0.f) ? -log1pf(expf(-sg)) : sg - log1pf(expf(sg));
-            }
-            if (lane == 0) gbias[w] = beta;
-          }
-          __syncthreads();
-          for (int w = tid; w < m * G; w += kThreads)
-            for (int r = 1; r < CS; ++r) st_async_f32(dsmem_addr(gbias + w, r), gbias[w], dsmem_addr(bar_sel, r));
-        }
         SAS_TRACE(18);  // rank 0: list ready
         for (int j = tid; j < m; j += kThreads) {
           const int b = sel[j];
@@ -503,6 +499,68 @@ __global__ void __launch_bounds__(kThreads, 4)
         }
         if (p.sel_count != nullptr && tid == 0) p.sel_count[pair] = list_ok ? m : 0;
         SAS_TRACE(19);  // rank 0: list sent
+        if (gated) {
+          // this CTA's K/V copies go out first; the gates are computed while
+          // they (and the other CTAs' copies) are in flight
+          __syncthreads();
+          known = nchunks + kTilesPerBlock * cnt_mine;
+          pump(nchunks, known);
+          // gate of every list entry and head: log(sigmoid(s_gb)), s_gb =
+          // (q~_g . k~_b) * gate_scale from q~ (v, rotated in place) and the
+          // block's gate key; 0 for the current block and a stand-in list.
+          // As in the score phase: 8 lanes per key row (16 dimensions each),
+          // 4 rows per warp, two 16-row steps per round with every load of
+          // the round in flight, one 8-lane reduction per (row, head).
+          const int nh = list_ok ? m - 1 : 0;  // historical entries
+          const int grp = lane >> 3, sub = lane & 7;
+          for (int j0 = 0; j0 < nh; j0 += 32) {
+            uint4 kr[2][4];
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              const int j = j0 + 16 * v + 4 * warp + grp;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) kr[v][i] = make_uint4(0u, 0u, 0u, 0u);
+              if (j < nh) {
+                const uint8_t* krow = gk_pair + static_cast<size_t>(sel[j]) * gk_row_bytes;
+                if (p.gk16) {
+                  kr[v][0] = *reinterpret_cast<const uint4*>(krow + 32 * sub);
+                  kr[v][1] = *reinterpret_cast<const uint4*>(krow + 32 * sub + 16);
+                } else {
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) kr[v][i] = *reinterpret_cast<const uint4*>(krow + 64 * sub + 16 * i);
+                }
+              }
+            }
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              const int j = j0 + 16 * v + 4 * warp + grp;
+              for (int g = 0; g < G; ++g) {
+                const float4* q4 = reinterpret_cast<const float4*>(qv + g * kDim + 16 * sub);
+                float a = 0.f;
+                if (p.gk16) {
+                  a = dot8_bf16(q4[0], q4[1], kr[v][0], a);
+                  a = dot8_bf16(q4[2], q4[3], kr[v][1], a);
+                } else {
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    const uint4 k = kr[v][i];
+                    a = dot4(q4[i], make_float4(__uint_as_float(k.x), __uint_as_float(k.y),
+                                                __uint_as_float(k.z), __uint_as_float(k.w)), a);
+                  }
+                }
+                a += __shfl_xor_sync(0xffffffffu, a, 1);
+                a += __shfl_xor_sync(0xffffffffu, a, 2);
+                a += __shfl_xor_sync(0xffffffffu, a, 4);
+                const float sg = a * p.gate_scale;
+                if (sub == 0 && j < nh) gbias[j * G + g] = (sg >= 0.f) ? -log1pf(expf(-sg)) : sg - log1pf(expf(sg));
+              }
+            }
+          }
+          for (int w = nh * G + tid; w < m * G; w += kThreads) gbias[w] = 0.f;  // current block, stand-in
+          __syncthreads();
+          for (int w = tid; w < m * G; w += kThreads)
+            for (int r = 1; r < CS; ++r) st_async_f32(dsmem_addr(gbias + w, r), gbias[w], dsmem_addr(bar_gb, r));
+        }
         issue_wk();
       } else {
         issue_wk();
@@ -522,6 +580,13 @@ __global__ void __launch_bounds__(kThreads, 4)
     known = nchunks + kTilesPerBlock * cnt_mine;
     SAS_TRACE(20);  // list in hand
     pump(nchunks, known);
+    if (gated && rank != 0 && !bad) {
+      // the gates follow the list; the K/V copies just issued overlap the wait
+      if (__syncthreads_and(mbar_wait_cluster(bar_gb, 0, p.status)) == 0) {
+        for (int w = tid; w < m * G; w += kThreads) gbias[w] = 0.f;
+      }
+      __syncthreads();
+    }
     SAS_TRACE(5);
   }
 
@@ -898,7 +963,11 @@ __global__ void __launch_bounds__(kThreads, 4)
     float cs, sn;
     rope_cos_sin(p.rope.theta_over_pi[d & 63], c, cs, sn);
     const float y = (d < 64) ? qbar[d] * cs - qbar[d + 64] * sn : qbar[d] * cs + qbar[d - 64] * sn;
-    p.gate_keys_out[(static_cast<size_t>(pair) * p.mg + c) * kDim + d] = y;
+    const size_t gi = (static_cast<size_t>(pair) * p.mg + c) * kDim + d;
+    if (p.gk16)
+      static_cast<__nv_bfloat16*>(p.gate_keys_out)[gi] = __float2bfloat16_rn(y);
+    else
+      static_cast<float*>(p.gate_keys_out)[gi] = y;
   }
   SAS_TRACE(8);
 }

@@ -398,6 +398,23 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 }
 
 // ---------------------------------------------------------------- conversions
+// The two bf16 values packed in a 32-bit word (first in the low half) as fp32.
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// acc + a . (8 bf16 values packed in k), a given as two float4.
+__device__ __forceinline__ float dot8_bf16(float4 a0, float4 a1, uint4 k, float acc) {
+  acc = fmaf(a0.x, bf16_lo(k.x), acc);
+  acc = fmaf(a0.y, bf16_hi(k.x), acc);
+  acc = fmaf(a0.z, bf16_lo(k.y), acc);
+  acc = fmaf(a0.w, bf16_hi(k.y), acc);
+  acc = fmaf(a1.x, bf16_lo(k.z), acc);
+  acc = fmaf(a1.y, bf16_hi(k.z), acc);
+  acc = fmaf(a1.z, bf16_lo(k.w), acc);
+  acc = fmaf(a1.w, bf16_hi(k.w), acc);
+  return acc;
+}
+
 __device__ __forceinline__ float to_float(float x) { return x; }
 __device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
 

@@ -72,8 +72,8 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
   p.gam = take(kDim * 4, 16);
   p.gamk = take(kDim * 4, 16);
   // ring slots, prologue, pooled P, W_k slice, scores (rank 0), list, v,
-  // attention partials, pooled slices (rank 0)
-  p.bars = take((nst + 8) * 8, 8);
+  // attention partials, pooled slices (rank 0), gates of the list
+  p.bars = take((nst + 9) * 8, 8);
   auto up128 = [](int x) { return (x + 127) / 128 * 128; };
   const int r = up128(off);
   // phases 0-1 (the W_q slice is a tensor-TMA destination: 128-byte aligned)
@@ -114,9 +114,10 @@ struct DecodeParams {
   const void* q;
   const __nv_bfloat16* w_q;
   const float* gamma_q;
-  const float* gate_keys;
+  const void* gate_keys;  // fp32, or bf16 when gk16 [B][Hkv][mg][128]
   const float* gamma_k;  // fused pooling of a completed current block (null: off)
-  float* gate_keys_out;  // same array as gate_keys, written at row c when pooling
+  void* gate_keys_out;   // same array as gate_keys, written at row c when pooling
+  int gk16;              // gate keys stored as bf16
   KvView kv;
   float* head_scores;
   float* group_scores;
@@ -145,7 +146,8 @@ struct PoolParams {
   const int32_t* blk_begin;
   const __nv_bfloat16* w_k;
   const float* gamma_k;
-  float* gate_keys;
+  void* gate_keys;  // fp32, or bf16 when gk16
+  int gk16;
   float* pooled_raw;
   uint32_t* status;
 };
@@ -157,7 +159,8 @@ struct PrefillParams {
   const __nv_bfloat16* q;     // [B][Hq][T][128]
   const __nv_bfloat16* w_q;   // [Hq][128][128]
   const float* gamma_q;       // [128]
-  const float* gate_keys;     // [B][Hkv][mg][128]
+  const void* gate_keys;      // [B][Hkv][mg][128], fp32 or bf16 (gk16)
+  int gk16;
   float* qt;                  // workspace: gate queries [B][Hq][nblk][128]
   int32_t* sel;               // workspace: block lists [B][Hkv][nblk][max_sel]
   int32_t* cnt;               // workspace: list lengths [B][Hkv][nblk]

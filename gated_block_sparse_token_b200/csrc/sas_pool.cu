@@ -172,7 +172,11 @@ __global__ void __launch_bounds__(kThreads) pool_keys_kernel(const __grid_consta
       float cs, sn;
       rope_cos_sin(p.rope.theta_over_pi[j], b, cs, sn);
       const float y = (d < 64) ? xn[d] * cs - xn[d + 64] * sn : xn[d] * cs + xn[d - 64] * sn;
-      p.gate_keys[((static_cast<size_t>(s) * p.hkv + h) * p.mg + b) * kDim + d] = y;
+      const size_t gi = ((static_cast<size_t>(s) * p.hkv + h) * p.mg + b) * kDim + d;
+      if (p.gk16)
+        static_cast<__nv_bfloat16*>(p.gate_keys)[gi] = __float2bfloat16_rn(y);
+      else
+        static_cast<float*>(p.gate_keys)[gi] = y;
     }
     __syncthreads();
   }

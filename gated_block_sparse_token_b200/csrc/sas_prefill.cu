@@ -131,19 +131,26 @@ __global__ void __launch_bounds__(kThreads) prefill_select_kernel(const __grid_c
   float4 qr[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) qr[k] = *reinterpret_cast<const float4*>(qbar + sub * 16 + 4 * k);
-  const float* gk = p.gate_keys + (static_cast<size_t>(s) * p.hkv + h) * p.mg * kDim;
+  const size_t gk_base = (static_cast<size_t>(s) * p.hkv + h) * p.mg * kDim;  // elements
   for (int b0 = 0; b0 < i; b0 += 16) {
     const int b = b0 + warp * 4 + grp;
     float acc = 0.f;
     if (b < i) {
-      const float4* row = reinterpret_cast<const float4*>(gk + static_cast<size_t>(b) * kDim + sub * 16);
+      const size_t off = gk_base + static_cast<size_t>(b) * kDim + sub * 16;
+      if (p.gk16) {
+        const uint4* row = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.gate_keys) + off);
+        acc = dot8_bf16(qr[0], qr[1], row[0], acc);
+        acc = dot8_bf16(qr[2], qr[3], row[1], acc);
+      } else {
+        const float4* row = reinterpret_cast<const float4*>(static_cast<const float*>(p.gate_keys) + off);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 kv = row[k];
-        acc = fmaf(qr[k].x, kv.x, acc);
-        acc = fmaf(qr[k].y, kv.y, acc);
-        acc = fmaf(qr[k].z, kv.z, acc);
-        acc = fmaf(qr[k].w, kv.w, acc);
+        for (int k = 0; k < 4; ++k) {
+          const float4 kv = row[k];
+          acc = fmaf(qr[k].x, kv.x, acc);
+          acc = fmaf(qr[k].y, kv.y, acc);
+          acc = fmaf(qr[k].z, kv.z, acc);
+          acc = fmaf(qr[k].w, kv.w, acc);
+        }
       }
     }
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);

@@ -60,7 +60,7 @@ sas_status scratch_for_current_device(void** out) {
 extern "C" sas_status sas_decode_step_static(const sas_config* cfg, const void* q,
                                              const sas_kv* kv, const void* w_q,
                                              const float* gamma_q, const void* w_k,
-                                             const float* gamma_k, float* gate_keys,
+                                             const float* gamma_k, void* gate_keys,
                                              int32_t max_gate_blocks, void* out,
                                              int32_t* sel_idx, int32_t* sel_count,
                                              float* group_scores, uint32_t* status_out,

@@ -49,7 +49,7 @@ class _Config(ctypes.Structure):
                 ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float),
                 ("attn_scale", ctypes.c_float), ("gate_scale", ctypes.c_float),
                 ("kv_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
-                ("gate_mode", ctypes.c_int32)]
+                ("gate_mode", ctypes.c_int32), ("gate_keys_bf16", ctypes.c_int32)]
 
 
 class _Kv(ctypes.Structure):
@@ -130,12 +130,13 @@ class Config:
     block_size: int = 64
     gate_hidden: int = 128
     gate_mode: int = 0        # GATE_SELECT_ONLY or GATE_LOGSIGMOID_BIAS
+    gate_keys_bf16: int = 0   # 1: the gate-key cache is bf16 (else fp32)
 
     def c(self) -> _Config:
         return _Config(self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
                        self.gate_hidden, self.token_budget, self.rope_base, self.norm_eps,
                        self.attn_scale, self.gate_scale, _DT[self.kv_dtype], _DT[self.out_dtype],
-                       self.gate_mode)
+                       self.gate_mode, self.gate_keys_bf16)
 
     @property
     def group(self) -> int:
@@ -198,6 +199,7 @@ def get_device_status(ws: torch.Tensor, stream=None) -> int:
 def pool_keys(cfg: Config, kv: KvCache, w_k, gamma_k, gate_keys, ws, blk_begin=None,
               num_blocks: Optional[int] = None, pooled_raw=None, stream=None) -> None:
     """sas_pool_keys.  num_blocks defaults to gate_keys.shape[2] (all rows)."""
+    _check_gk(cfg, gate_keys)
     mg = int(gate_keys.shape[2])
     nb = mg if num_blocks is None else int(num_blocks)
     c, k = cfg.c(), kv.c()
@@ -208,6 +210,7 @@ def pool_keys(cfg: Config, kv: KvCache, w_k, gamma_k, gate_keys, ws, blk_begin=N
 
 def gate_scores(cfg: Config, q, seq_lens, w_q, gamma_q, gate_keys, group_scores, ws,
                 head_scores=None, stream=None) -> None:
+    _check_gk(cfg, gate_keys)
     c = cfg.c()
     _check(lib().sas_gate_scores(ctypes.byref(c), _ptr(q), _ptr(seq_lens), int(seq_lens.shape[0]),
                                  _ptr(w_q), _ptr(gamma_q), _ptr(gate_keys), int(gate_keys.shape[2]),
@@ -235,6 +238,7 @@ def decode_step(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out, ws, s
                 sel_count=None, group_scores=None, w_k=None, gamma_k=None, stream=None) -> None:
     """sas_decode_step.  With w_k / gamma_k the step also pools the block the
     decoded token completes into gate_keys (see include/sas.h)."""
+    _check_gk(cfg, gate_keys)
     c, k = cfg.c(), kv.c()
     _check(lib().sas_decode_step(ctypes.byref(c), _ptr(q), ctypes.byref(k), _ptr(w_q),
                                  _ptr(gamma_q), _ptr(w_k), _ptr(gamma_k), _ptr(gate_keys),
@@ -247,6 +251,7 @@ def decode_step_static(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out
                        sel_count=None, group_scores=None, w_k=None, gamma_k=None, status_out=None,
                        stream=None) -> None:
     """sas_decode_step_static: the same step with no workspace argument, for
+    _check_gk(cfg, gate_keys)
     callers that cannot allocate; status_out (optional device uint32/int32
     tensor) receives the call's status bits."""
     c, k = cfg.c(), kv.c()
@@ -262,6 +267,7 @@ def prefill_block_sparse(cfg: Config, q, k, v, w_q, gamma_q, w_k, gamma_k, gate_
     """sas_prefill_block_sparse: q [B][Hq][T][128], k / v [B][Hkv][T][128] (bf16),
     out like q; writes gate_keys [B][Hkv][MG][128]; ws from
     make_workspace(cfg, device, batch=B, max_seq_len=T)."""
+    _check_gk(cfg, gate_keys)
     c = cfg.c()
     B, T = int(q.shape[0]), int(q.shape[2])
     _check(lib().sas_prefill_block_sparse(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), B, T, _ptr(w_q),
@@ -273,6 +279,16 @@ def prefill_block_sparse(cfg: Config, q, k, v, w_q, gamma_q, w_k, gamma_k, gate_
 
 def out_dtype(cfg: Config) -> torch.dtype:
     return _TORCH_DT[_DT[cfg.out_dtype]]
+
+
+def gate_key_dtype(cfg: Config) -> torch.dtype:
+    """Element type of the gate-key cache under cfg (bf16 or fp32)."""
+    return torch.bfloat16 if cfg.gate_keys_bf16 else torch.float32
+
+
+def _check_gk(cfg: Config, gate_keys) -> None:
+    if gate_keys is not None and gate_keys.dtype != gate_key_dtype(cfg):
+        raise ValueError(f"gate_keys is {gate_keys.dtype}, the config wants {gate_key_dtype(cfg)}")
 
 
 def kv_dtype(cfg: Config) -> torch.dtype:

@@ -110,6 +110,11 @@ typedef struct {
                             sas_sparse_decode and sas_prefill_block_sparse
                             return SAS_ERR_UNSUPPORTED for it, the gate-score,
                             Top-K and pooling calls ignore it. */
+  int32_t gate_keys_bf16;  /* 0 (default): the gate-key cache is fp32
+                              [B][Hkv][MG][128].  1: it is bf16, keys rounded to
+                              nearest-even when written (half the bytes the
+                              scores stream).  Every call that reads or writes
+                              gate keys follows it. */
 } sas_config;
 
 /* KV cache description (device pointers, caller-owned). */
@@ -174,7 +179,7 @@ SAS_API int32_t sas_abi_version(void);
 SAS_API sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv,
                          const int32_t* blk_begin, int32_t num_blocks,
                          const void* w_k, const float* gamma_k,
-                         float* gate_keys, int32_t max_gate_blocks,
+                         void* gate_keys, int32_t max_gate_blocks,
                          float* pooled_raw, void* ws, size_t ws_bytes,
                          sas_stream_t stream);
 
@@ -190,7 +195,7 @@ SAS_API sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv,
  */
 SAS_API sas_status sas_gate_scores(const sas_config* cfg, const void* q, const int32_t* seq_lens,
                            int32_t batch, const void* w_q, const float* gamma_q,
-                           const float* gate_keys, int32_t max_gate_blocks,
+                           const void* gate_keys, int32_t max_gate_blocks,
                            float* head_scores, float* group_scores,
                            void* ws, size_t ws_bytes, sas_stream_t stream);
 
@@ -237,7 +242,7 @@ SAS_API sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const
  */
 SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const sas_kv* kv,
                                    const void* w_q, const float* gamma_q, const void* w_k,
-                                   const float* gamma_k, float* gate_keys,
+                                   const float* gamma_k, void* gate_keys,
                                    int32_t max_gate_blocks, void* out, int32_t* sel_idx,
                                    int32_t* sel_count, float* group_scores, void* ws,
                                    size_t ws_bytes, sas_stream_t stream);
@@ -268,7 +273,7 @@ SAS_API sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q
                                             const void* v, int32_t batch, int32_t seq_len,
                                             const void* w_q, const float* gamma_q,
                                             const void* w_k, const float* gamma_k,
-                                            float* gate_keys, int32_t max_gate_blocks, void* out,
+                                            void* gate_keys, int32_t max_gate_blocks, void* out,
                                             int32_t* sel_idx, int32_t* sel_count, void* ws,
                                             size_t ws_bytes, sas_stream_t stream);
 
@@ -292,7 +297,7 @@ SAS_API sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q
  */
 SAS_API sas_status sas_decode_step_static(const sas_config* cfg, const void* q, const sas_kv* kv,
                                           const void* w_q, const float* gamma_q, const void* w_k,
-                                          const float* gamma_k, float* gate_keys,
+                                          const float* gamma_k, void* gate_keys,
                                           int32_t max_gate_blocks, void* out, int32_t* sel_idx,
                                           int32_t* sel_count, float* group_scores,
                                           uint32_t* status_out, sas_stream_t stream);

@@ -17,6 +17,7 @@ OUT_ATOL = 1e-2        # attention outputs, bf16 storage / fp32 accumulate
 SCORE_RTOL = 1e-3      # gate scores and gate keys, relative ...
 SCORE_FLOOR = 1e-3     # ... to max(|x|, 1e-3 * max|x|): the pure relative form is ill-posed near 0
 TIE_RTOL = 1e-3        # K-th vs (K+1)-th oracle score window for set mismatches
+BF16_ULP = 2.0 ** -7   # one bf16 ulp, relative: stored keys vs the oracle's rounded keys
 
 
 def config_for(spec, budget, out_dtype="bf16", gate_mode=sas.GATE_SELECT_ONLY):

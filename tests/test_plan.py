@@ -38,11 +38,11 @@ def test_plan_alignment_and_overlap(plans):
         # fixed regions, in order, disjoint
         fixed = [("slots", 2 * 16384), ("sel", 4 * ms), ("gbias", 4 * ms * G * p["gated"]),
                  ("qraw", G * 128 * (4 if p["f32"] else 2)), ("qbar", 512), ("pml", 256), ("gam", 512),
-                 ("bars", 8 * (2 + 8))]
+                 ("bars", 8 * (2 + 9))]
         for (a, sa), (b, _) in zip(fixed, fixed[1:]):
             assert p[a] + sa <= p[b], (tag, a, b)
         r = p["r_qv"]
-        assert p["bars"] + 8 * (2 + 8) <= r, tag
+        assert p["bars"] + 8 * (2 + 9) <= r, tag
         # phase 0-1 layout: qv then the W_q slice
         qv_end = r + G * 128 * 4
         assert qv_end <= p["r_wq"], tag

@@ -18,13 +18,13 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _run(spec):
+def _run(spec, gk16=0):
     inp = make_prefill_inputs(spec, DEV)
     B, Tn = spec.batch, spec.seq_len
     nblk = Tn // 64
-    cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget)
+    cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget, gate_keys_bf16=gk16)
     ws = sas.make_workspace(cfg, DEV, batch=B, max_seq_len=Tn)
-    gk = torch.zeros(B, spec.hkv, nblk, 128, dtype=torch.float32, device=DEV)
+    gk = torch.zeros(B, spec.hkv, nblk, 128, dtype=sas.gate_key_dtype(cfg), device=DEV)
     out = torch.full((B, spec.hq, Tn, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
     sel = torch.full((B, spec.hkv, nblk, cfg.max_sel), -1, dtype=torch.int32, device=DEV)
     cnt = torch.full((B, spec.hkv, nblk), -1, dtype=torch.int32, device=DEV)
@@ -41,14 +41,22 @@ def _check(spec, inp, cfg, gk, out, sel, cnt, triples):
     wq = inp["w_q"].double().cpu().numpy()
     wk = inp["w_k"].double().cpu().numpy()
     ones = np.ones(128)
-    gk_h, out_h, sel_h, cnt_h = gk.cpu().numpy(), out.float().cpu().numpy(), sel.cpu().numpy(), cnt.cpu().numpy()
+    gk_h = gk.double().cpu().numpy()
+    out_h, sel_h, cnt_h = out.float().cpu().numpy(), sel.cpu().numpy(), cnt.cpu().numpy()
     cache = {}
     for (s, h, i) in triples:
         if (s, h) not in cache:
             ks = inp["k"][s, h].double().cpu().numpy()
             vs = inp["v"][s, h].double().cpu().numpy()
             keys = O.gate_keys_for_sequence(ks, spec.seq_len // 64, wk[h], ones)
-            T.assert_close_rel(gk_h[s, h], keys, f"prefill gate keys s={s} h={h}")
+            if cfg.gate_keys_bf16:
+                # stored keys within one bf16 ulp of the oracle's rounded keys; the
+                # scores are then checked from the stored keys themselves
+                T.assert_close_rel(gk_h[s, h], O.round_to_bf16(keys), f"prefill bf16 gate keys s={s} h={h}",
+                                   rtol=T.BF16_ULP)
+                keys = gk_h[s, h]
+            else:
+                T.assert_close_rel(gk_h[s, h], keys, f"prefill gate keys s={s} h={h}")
             cache[(s, h)] = (ks, vs, keys)
         ks, vs, keys = cache[(s, h)]
         qb = inp["q"][s, h * G:(h + 1) * G, 64 * i:64 * (i + 1)].double().cpu().numpy()
@@ -70,6 +78,13 @@ def _check(spec, inp, cfg, gk, out, sel, cnt, triples):
 def test_prefill_small_all_blocks():
     spec = PrefillSpec("pf_small", 1, 4, 2, 1024, token_budget=256, seed=41)
     res = _run(spec)
+    triples = [(0, h, i) for h in range(2) for i in range(16)]
+    _check(spec, *res, triples)
+
+
+def test_prefill_small_bf16_gate_keys():
+    spec = PrefillSpec("pf_small_bf16", 1, 4, 2, 1024, token_budget=256, seed=41)
+    res = _run(spec, gk16=1)
     triples = [(0, h, i) for h in range(2) for i in range(16)]
     _check(spec, *res, triples)
 
