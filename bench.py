@@ -377,6 +377,54 @@ def timed(graphs, world, stream):
 MIXED_BUDGETS = [1024, 2048, 4096, 2048, 1024, 4096, 2048, 2048]
 
 
+def run_long_context(args, rank, world, device, layers=2, steps=1000):
+    """Long-context decode: the Qwen3-14B layer (40 query / 8 KV heads), batch
+    16, 131,072 tokens in 64-token pages behind a random block table, budget
+    4,096; the step pools the block its token completes.  Two layers of
+    8.6 GB caches rotate (far above L2)."""
+    import torch
+    from gated_block_sparse_token_b200 import sas
+    from gated_block_sparse_token_b200.workloads import make_decode_inputs, qwen3_14b_paged_128k
+    spec0 = qwen3_14b_paged_128k()
+    cfg = sas.Config(spec0.hq, spec0.hkv, token_budget=4096)
+    Ls = []
+    for li in range(layers):
+        spec = qwen3_14b_paged_128k(seed=2000 * (rank + 1) + li)
+        inp = make_decode_inputs(spec, device)
+        kv = sas.KvCache(inp["k"], inp["v"], inp["seq_lens"], inp["block_table"])
+        gk = torch.zeros(spec.batch, spec.hkv, spec.cap // 64, 128, dtype=torch.float32, device=device)
+        ws = sas.make_workspace(cfg, device)
+        sas.pool_keys(cfg, kv, inp["w_k"], inp["gamma_k"], gk, ws)
+        out = torch.empty(spec.batch, spec.hq, 128, dtype=torch.bfloat16, device=device)
+        Ls.append(dict(inp=inp, kv=kv, gk=gk, ws=ws, out=out))
+    stream = torch.cuda.Stream(device)
+    fn = lambda L, st: step(cfg, L, st)  # noqa: E731
+    with torch.cuda.stream(stream):
+        for L in Ls:
+            step(cfg, L, stream)
+    torch.cuda.synchronize()
+    warm = plan(fn, 20 * layers, Ls, stream)
+    main = plan(fn, steps, Ls, stream)
+    with torch.cuda.stream(stream):
+        run_graphs(warm)
+    torch.cuda.synchronize()
+    t = timed(main, world, stream)
+    for L in Ls:
+        if sas.get_device_status(L["ws"], stream) != sas.SAS_OK:
+            raise RuntimeError("device status not OK after the long-context run")
+    del Ls, main, warm
+    torch.cuda.empty_cache()
+    peak, peak_kind = measured_peaks()
+    dbytes = decode_bytes(spec0.seq_lens, spec0.hq, spec0.hkv, 4096)
+    dec_s = t / steps
+    achieved = dbytes / dec_s / 1e9
+    return {"mode": "long context", "workload": "qwen3_14b_paged_b16_128k_budget4096", "steps": steps,
+            "value": round(job_throughput(steps, world, t), 2), "unit": UNIT, "ms_per_step": round(dec_s * 1e3, 5),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+                         "bytes_per_launch": dbytes, "avg_launch_us": round(dec_s * 1e6, 3)}}
+
+
 def run_variant(args, rank, world, device, name, gate_mode=0, budgets=None, gk16=0):
     """The same decode workload in one of the widened modes (the gated
     inference mode, or mixed per-sequence budgets), timed like the main line
@@ -497,6 +545,7 @@ def run_ours(args):
         variants.append(run_variant(args, rank, world, device, "gated (log-sigmoid bias)", gate_mode=1))
         variants.append(run_variant(args, rank, world, device, "mixed budgets", budgets=MIXED_BUDGETS))
         variants.append(run_variant(args, rank, world, device, "bf16 gate keys", gk16=1))
+        variants.append(run_long_context(args, rank, world, device))
     pf = None if args.skip_prefill else run_prefill(args, device, world)
 
     if rank != 0:

@@ -17,7 +17,8 @@ CSRC = os.path.join(ROOT, "gated_block_sparse_token_b200", "csrc")
 def plans():
     with tempfile.TemporaryDirectory() as d:
         exe = os.path.join(d, "plan_check")
-        subprocess.run(["/usr/local/cuda/bin/nvcc", "-std=c++17", "-I", CSRC, "-I", os.path.join(ROOT, "include"),
+        subprocess.run(["/usr/local/cuda/bin/nvcc", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+                        "-I", CSRC, "-I", os.path.join(ROOT, "include"),
                         os.path.join(ROOT, "tests", "native", "plan_check.cu"), "-o", exe], check=True)
         out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
     rows = []
