@@ -14,6 +14,10 @@ selected working set (R x ~85 MB) is far larger than the 126 MB L2.
 Metric: decode steps/s per layer (whole job: summed over ranks), achieved
 HBM GB/s of the dominant kernel against the measured B200 copy bandwidth.
 
+The layers share one sequence-length vector (a model's decode step reads
+the same lengths in every layer); K/V caches, gate keys, queries and gate
+weights are per layer.
+
 Multi-GPU: one process per GPU (torchrun); every rank decodes its own
 independent batch (weak scaling, no collective on the data path); the only
 collectives are the barrier and the max-reduce of the timings.
@@ -306,9 +310,13 @@ def build_layers(R, rank, device, gate_mode=0, budgets=None, gk16=0):
                      gate_keys_bf16=gk16)
     tb = None if budgets is None else torch.tensor(budgets, dtype=torch.int32, device=device)
     layers = []
+    lens = None  # one length vector for every layer, as in a model's decode step
     for li in range(R):
         spec = qwen3_4b_32k(batch=BATCH, seq_len=CTX, seed=1000 * (rank + 1) + li)
         inp = make_decode_inputs(spec, device)
+        if lens is None:
+            lens = inp["seq_lens"]
+        inp["seq_lens"] = lens
         kv = sas.KvCache(inp["k"], inp["v"], inp["seq_lens"], token_budgets=tb)
         mg = spec.cap // 64
         gk = torch.zeros(BATCH, HKV, mg, 128, dtype=sas.gate_key_dtype(cfg), device=device)
@@ -388,9 +396,13 @@ def run_long_context(args, rank, world, device, layers=2, steps=1000):
     spec0 = qwen3_14b_paged_128k()
     cfg = sas.Config(spec0.hq, spec0.hkv, token_budget=4096)
     Ls = []
+    lens = None  # one length vector for every layer
     for li in range(layers):
         spec = qwen3_14b_paged_128k(seed=2000 * (rank + 1) + li)
         inp = make_decode_inputs(spec, device)
+        if lens is None:
+            lens = inp["seq_lens"]
+        inp["seq_lens"] = lens
         kv = sas.KvCache(inp["k"], inp["v"], inp["seq_lens"], inp["block_table"])
         gk = torch.zeros(spec.batch, spec.hkv, spec.cap // 64, 128, dtype=torch.float32, device=device)
         ws = sas.make_workspace(cfg, device)
