@@ -198,7 +198,7 @@ def decode_bytes(seq_lens, hq, hkv, budget, kv_elem=2, pool=True, gk_elem=4):
             per_pair += 128 * gk_elem
         tot += hkv * per_pair
     tot += hq * 128 * 128 * 2
-    if pool:
+    if pool and any(L % 64 == 0 for L in seq_lens):  # W_k is read only when a block completes
         tot += hkv * 384 * 128 * 2
     return tot
 
