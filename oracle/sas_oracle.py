@@ -317,28 +317,35 @@ def dense_causal_decode(q_group, k_seq, v_seq, seq_len,
 # --------------------------------------------------------------------------
 def prefill_query_block(q_blk_group, k_seq, v_seq, i, gate_keys, w_q_group,
                         gamma_q_group, topk, attn_scale=1.0 / math.sqrt(128.0),
-                        gate_scale=1.0 / math.sqrt(128.0), eps=1e-6, base=10000.0):
+                        gate_scale=1.0 / math.sqrt(128.0), eps=1e-6, base=10000.0,
+                        gate_mode=GATE_SELECT_ONLY):
     """One (sequence, KV head, query block i) of block-sparse causal prefill.
 
     q_blk_group [G][64][128]: queries of block i for the G heads.
     Gate query of head g = mean over the block's 64 queries (R13), placed at
     position i; historical blocks 0..i-1 scored; top-min(topk, i) kept plus
     the diagonal block i; token t of block i attends to all tokens of the
-    kept historical blocks and to tokens 64i..t of block i.
-    Returns dict(out [G][64][128], sel, S).
+    kept historical blocks and to tokens 64i..t of block i.  Gated mode
+    (R18): the tokens of a kept historical block b get + log(sigmoid(s_gb))
+    on head g's logits, the diagonal block 0.
+    Returns dict(out [G][64][128], sel, S, s).
     """
     G = q_blk_group.shape[0]
     qbar = q_blk_group.astype(np.float64).mean(axis=1)
-    _, S = gate_scores(qbar, w_q_group, gamma_q_group, gate_keys, i, i,
+    s, S = gate_scores(qbar, w_q_group, gamma_q_group, gate_keys, i, i,
                        gate_scale, eps, base)
     sel = select_blocks(S, i, topk)
     hist_toks = selected_token_ids(sel[:-1], (i + 1) * BLOCK)
     out = np.zeros((G, BLOCK, HEAD_DIM))
     for g in range(G):
+        hist_bias = None
+        if gate_mode == GATE_LOGSIGMOID_BIAS:
+            hist_bias = gated_token_bias(s[g], sel[:-1], (i + 1) * BLOCK, i)
         for t in range(BLOCK):
             toks = hist_toks + list(range(i * BLOCK, i * BLOCK + t + 1))
-            out[g, t] = attention_over_tokens(q_blk_group[g, t], k_seq, v_seq, toks, attn_scale)
-    return {"out": out, "sel": sel, "S": S}
+            bias = None if hist_bias is None else hist_bias + [0.0] * (t + 1)
+            out[g, t] = attention_over_tokens(q_blk_group[g, t], k_seq, v_seq, toks, attn_scale, bias)
+    return {"out": out, "sel": sel, "S": S, "s": s}
 
 
 def dense_causal_prefill(q_seq, k_seq, v_seq, attn_scale=1.0 / math.sqrt(128.0)):

@@ -378,6 +378,38 @@ def test_gated_mode_saturated_gates():
     assert np.allclose(res[O.GATE_LOGSIGMOID_BIAS]["out"][1], v1, rtol=1e-12, atol=1e-12)
 
 
+def test_gated_prefill_closed_form():
+    """Query block 1 of a 128-token sequence: block 0's keys a*e1 (gate key
+    sqrt(128)-ish e0 as in the decode case), block 1's keys 0, every query of
+    head g equal to +-b e0 (so the block-mean gate query is the same vector,
+    at position 1).  All attention logits are 0, so token t of block 1 gives
+    (64 sigmoid(s_g) v0 + (t + 1) v1) / (64 sigmoid(s_g) + t + 1)."""
+    a, b = 1.5, 2.0
+    rng = np.random.default_rng(4)
+    k = np.zeros((128, 128))
+    k[:64, 1] = a
+    v = np.zeros((128, 128))
+    v0, v1 = rng.standard_normal(128), rng.standard_normal(128)
+    v[:64], v[64:] = v0, v1
+    w_k = np.zeros((384, 128))
+    w_k[1, 0] = w_k[129, 0] = w_k[257, 0] = 1.0
+    gk = O.gate_keys_for_sequence(k, 2, w_k, np.ones(128))
+    q = np.zeros((2, 64, 128))
+    q[0, :, 0], q[1, :, 0] = b, -b
+    w_q = np.stack([np.eye(128)] * 2)
+    r = O.prefill_query_block(q, k, v, 1, gk, w_q, np.ones((2, 128)), 31, gate_mode=O.GATE_LOGSIGMOID_BIAS)
+    eps = 1e-6
+    kn = 3 * a / math.sqrt((3 * a) ** 2 / 128 + eps)
+    qn = b / math.sqrt(b ** 2 / 128 + eps)
+    s = np.array([1.0, -1.0]) * qn * math.cos(1.0) * kn * SCALE
+    assert r["sel"] == [0, 1]
+    for g in range(2):
+        w = 64.0 / (1.0 + math.exp(-s[g]))
+        for t in (0, 17, 63):
+            want = (w * v0 + (t + 1) * v1) / (w + t + 1)
+            assert np.allclose(r["out"][g, t], want, rtol=1e-12, atol=1e-12), (g, t)
+
+
 def test_log_sigmoid_values():
     assert O.log_sigmoid(0.0) == pytest.approx(-math.log(2.0), abs=1e-15)
     for x in (-50.0, -3.0, -0.5, 0.25, 4.0):
@@ -489,4 +521,8 @@ def test_pins_catch_planted_mistakes(monkeypatch):
     monkeypatch.setattr(O, "gated_token_bias", bias_on_current_too)
     with pytest.raises(AssertionError):
         test_gated_mode_closed_form()
+    monkeypatch.setattr(O, "log_sigmoid", lambda x: good_ls(-x))
+    with pytest.raises(AssertionError):
+        test_gated_prefill_closed_form()
+    monkeypatch.setattr(O, "log_sigmoid", good_ls)
     monkeypatch.setattr(O, "gated_token_bias", good_bias)
