@@ -224,7 +224,7 @@ def measured_tensor_peak():
 def run_prefill(args, device, world):
     """Block-sparse chunked prefill, Qwen3-8B heads, 32,768 tokens per sequence,
     Top-K 31 + diagonal: one sas_prefill_block_sparse call per step (pooling,
-    gate queries, selection, tcgen05 attention)."""
+    gate queries, selection, tcgen05 attention), in both gate modes."""
     import torch
     from gated_block_sparse_token_b200 import sas
     from gated_block_sparse_token_b200.workloads import make_prefill_inputs, qwen3_8b_prefill_32k
@@ -233,33 +233,39 @@ def run_prefill(args, device, world):
     inp = make_prefill_inputs(spec, device)
     B, T = spec.batch, spec.seq_len
     nblk = T // 64
-    cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget)
-    ws = sas.make_workspace(cfg, device, batch=B, max_seq_len=T)
-    gk = torch.zeros(B, spec.hkv, nblk, 128, dtype=torch.float32, device=device)
     out = torch.empty(B, spec.hq, T, 128, dtype=torch.bfloat16, device=device)
+    gk = torch.zeros(B, spec.hkv, nblk, 128, dtype=torch.float32, device=device)
     stream = torch.cuda.Stream(device)
 
-    def call():
-        sas.prefill_block_sparse(cfg, inp["q"], inp["k"], inp["v"], inp["w_q"], inp["gamma_q"], inp["w_k"],
-                                 inp["gamma_k"], gk, out, ws, stream=stream)
+    def time_mode(gate_mode):
+        cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget, gate_mode=gate_mode)
+        ws = sas.make_workspace(cfg, device, batch=B, max_seq_len=T)
 
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            call()
-    torch.cuda.synchronize()
-    barrier(world)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(args.prefill_steps):
-            call()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.prefill_steps, world)
-    if sas.get_device_status(ws, stream) != sas.SAS_OK:
-        raise RuntimeError("device status not OK after the prefill run")
+        def call():
+            sas.prefill_block_sparse(cfg, inp["q"], inp["k"], inp["v"], inp["w_q"], inp["gamma_q"], inp["w_k"],
+                                     inp["gamma_k"], gk, out, ws, stream=stream)
+
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                call()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.prefill_steps):
+                call()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.prefill_steps, world)
+        if sas.get_device_status(ws, stream) != sas.SAS_OK:
+            raise RuntimeError("device status not OK after the prefill run")
+        return t
+
+    t = time_mode(sas.GATE_SELECT_ONLY)
+    t_gated = time_mode(sas.GATE_LOGSIGMOID_BIAS)
     flops = prefill_flops(nblk, spec.hq, spec.hkv, spec.token_budget, B)
     peak, kind = measured_tensor_peak()
     achieved = flops / t / 1e12
@@ -267,6 +273,7 @@ def run_prefill(args, device, world):
             "kv_heads": spec.hkv, "token_budget": spec.token_budget, "steps": args.prefill_steps,
             "ms_per_step": round(t * 1e3, 4), "tokens_per_s": round(job_throughput(B * T, world, t), 1),
             "launches_per_step": 4,
+            "gated_mode_ms_per_step": round(t_gated * 1e3, 4),
             "roofline": {"kernel": "prefill_attn_kernel (tcgen05)", "bound": "tensor",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "peak_kind": kind,

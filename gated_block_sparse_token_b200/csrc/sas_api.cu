@@ -213,9 +213,10 @@ size_t ws_header_bytes() {
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
-size_t prefill_scratch_bytes(size_t batch, int hq, int hkv, size_t nblk, int max_sel) {
+// gate queries, block lists, list lengths (+ gated mode: the gates of the lists)
+size_t prefill_scratch_bytes(size_t batch, int hq, int hkv, size_t nblk, int max_sel, bool gated) {
   return up256(batch * hq * nblk * kDim * 4) + up256(batch * hkv * nblk * max_sel * 4) +
-         up256(batch * hkv * nblk * 4);
+         up256(batch * hkv * nblk * 4) + (gated ? up256(batch * hq * nblk * max_sel * 4) : 0);
 }
 
 sas_status launch_result(cudaError_t e) {
@@ -252,7 +253,7 @@ size_t sas_workspace_bytes(const sas_config* cfg, int32_t batch, int32_t max_seq
     // prefill scratch: gate queries, block lists and their lengths
     const size_t nblk = static_cast<size_t>((max_seq_len + 63) / 64);
     bytes += prefill_scratch_bytes(batch, cfg->num_q_heads, cfg->num_kv_heads, nblk,
-                                   cfg->token_budget / 64);
+                                   cfg->token_budget / 64, cfg->gate_mode == SAS_GATE_LOGSIGMOID_BIAS);
   }
   return bytes;
 }
@@ -456,7 +457,6 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
                                     int32_t* sel_count, void* ws, size_t ws_bytes,
                                     sas_stream_t stream) {
   sas_status st = check_config(cfg);
-  if (st == SAS_OK && cfg->gate_mode != SAS_GATE_SELECT_ONLY) return SAS_ERR_UNSUPPORTED;
   if (st != SAS_OK) return st;
   if (batch < 0 || seq_len < 0) return SAS_ERR_INVALID_ARG;
   if (batch == 0 || seq_len == 0) return SAS_OK;
@@ -537,6 +537,8 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
   p.sel = reinterpret_cast<int32_t*>(scratch);
   scratch += up256(static_cast<size_t>(batch) * p.hkv * nblk * p.max_sel * 4);
   p.cnt = reinterpret_cast<int32_t*>(scratch);
+  scratch += up256(static_cast<size_t>(batch) * p.hkv * nblk * 4);
+  p.gb = (cfg->gate_mode == SAS_GATE_LOGSIGMOID_BIAS) ? reinterpret_cast<float*>(scratch) : nullptr;
   p.sel_out = sel_idx;
   p.cnt_out = sel_count;
   p.out = static_cast<__nv_bfloat16*>(out);

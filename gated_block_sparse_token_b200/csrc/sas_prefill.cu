@@ -161,6 +161,35 @@ __global__ void __launch_bounds__(kThreads) prefill_select_kernel(const __grid_c
   __syncthreads();
   const int m = select_blocks(vals, i, p.topk, i, sel, hist, selbits, scan);
   const size_t base = (static_cast<size_t>(s) * p.hkv + h) * p.nblk + i;
+  if (p.gb != nullptr) {
+    // gated mode: gate of every kept historical block and head of the group,
+    // log(sigmoid(q~_g(i) . k~_b * gate_scale)); one (entry, head) per thread
+    for (int w = tid; w < (m - 1) * G; w += kThreads) {
+      const int j = w / G, g = w - j * G;
+      const float4* qg = reinterpret_cast<const float4*>(
+          p.qt + ((static_cast<size_t>(s) * p.hq + h * G + g) * p.nblk + i) * kDim);
+      const size_t koff = gk_base + static_cast<size_t>(sel[j]) * kDim;
+      float a0 = 0.f, a1 = 0.f;
+      if (p.gk16) {
+        const uint4* kr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.gate_keys) + koff);
+#pragma unroll 4
+        for (int c = 0; c < kDim / 8; c += 2) {
+          a0 = dot8_bf16(qg[2 * c], qg[2 * c + 1], kr[c], a0);
+          a1 = dot8_bf16(qg[2 * c + 2], qg[2 * c + 3], kr[c + 1], a1);
+        }
+      } else {
+        const float4* kr = reinterpret_cast<const float4*>(static_cast<const float*>(p.gate_keys) + koff);
+#pragma unroll 8
+        for (int c = 0; c < kDim / 4; c += 2) {
+          const float4 k0 = kr[c], k1 = kr[c + 1], q0 = qg[c], q1 = qg[c + 1];
+          a0 = fmaf(q0.x, k0.x, fmaf(q0.y, k0.y, fmaf(q0.z, k0.z, fmaf(q0.w, k0.w, a0))));
+          a1 = fmaf(q1.x, k1.x, fmaf(q1.y, k1.y, fmaf(q1.z, k1.z, fmaf(q1.w, k1.w, a1))));
+        }
+      }
+      const float sg = (a0 + a1) * p.gate_scale;
+      p.gb[(base * p.max_sel + j) * G + g] = (sg >= 0.f) ? -log1pf(expf(-sg)) : sg - log1pf(expf(sg));
+    }
+  }
   for (int j = tid; j < m; j += kThreads) {
     p.sel[base * p.max_sel + j] = sel[j];
     if (p.sel_out != nullptr) p.sel_out[base * p.max_sel + j] = sel[j];
@@ -201,7 +230,8 @@ enum { kBarQ = 0, kBarK0 = 1, kBarV0 = kBarK0 + kPfKStages, kBarS0 = kBarV0 + kP
        kBarP0 = kBarS0 + 2, kBarO = kBarP0 + 2, kNumPfBars = kBarO + 1 };
 
 size_t prefill_attn_smem_bytes(int max_sel) {
-  return static_cast<size_t>(kPfSmemBars + kNumPfBars * 8 + 16 + max_sel * 4);
+  // barriers, TMEM slot, block list, gates of the list for the CTA's 2 heads
+  return static_cast<size_t>(kPfSmemBars + kNumPfBars * 8 + 16 + max_sel * 4 + max_sel * 2 * 4);
 }
 
 // Tracing builds: the issuer and softmax thread 0 add up the SM cycles they
@@ -246,6 +276,7 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + kPfSmemBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumPfBars);
   int* sel_s = reinterpret_cast<int*>(tmem_slot + 4);
+  float* gb_s = reinterpret_cast<float*>(sel_s + p.max_sel);  // gated mode: [entry][2 heads]
   // the plan assumes a 1024-byte aligned dynamic shared window (swizzled
   // TMA boxes and UMMA descriptors); anything else is reported, not used
   const bool misaligned = (smem_u32(base) & 1023u) != 0;
@@ -263,6 +294,13 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
       const int b = sl[j];
       sel_s[j] = b;
       if (b < 0 || b > i || (j == m - 1 && b != i) || (j > 0 && sl[j - 1] >= b)) err = true;
+    }
+    if (p.gb != nullptr) {
+      const float* gl = p.gb + lbase * p.max_sel * p.G;
+      for (int w = tid; w < 2 * m; w += kPfAttnThreads) {
+        const int j = w >> 1;
+        gb_s[w] = (j < m - 1) ? gl[j * p.G + 2 * pair + (w & 1)] : 0.f;  // the diagonal block: 0
+      }
     }
   }
   if (tid == 0 && !misaligned) {
@@ -408,7 +446,9 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
         mx0 = fmax3(mx0, sv[j], sv[j + 1]);
         mx1 = fmax3(mx1, sv[j + 2], sv[j + 3]);
       }
-      const float mx = fmax3(mx0, mx1, fmaxf(sv[62], sv[63])) * sl2;
+      // gated mode: + the block's gate for this row's head, in log2 units
+      const float beta2 = (p.gb != nullptr) ? gb_s[2 * e + (r >> 6)] * kLog2e : 0.f;
+      const float mx = fmaf(fmax3(mx0, mx1, fmaxf(sv[62], sv[63])), sl2, beta2);
       const float m_new = fmaxf(m_run, mx);
       // rescale O only when the running maximum grows by more than 2^8:
       // probabilities stay below 256 in between, exact after normalisation
@@ -418,8 +458,8 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
       uint32_t pk[32];
 #pragma unroll
       for (int j = 0; j < 64; j += 2) {
-        const float p0 = exp2_approx(fmaf(sv[j], sl2, -m_use));
-        const float p1 = exp2_approx(fmaf(sv[j + 1], sl2, -m_use));
+        const float p0 = exp2_approx(fmaf(sv[j], sl2, beta2 - m_use));
+        const float p1 = exp2_approx(fmaf(sv[j + 1], sl2, beta2 - m_use));
         rs[(j >> 1) & 3] += p0 + p1;
         pk[j >> 1] = pack_bf16x2(p0, p1);
       }

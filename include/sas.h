@@ -105,11 +105,13 @@ typedef struct {
   float gate_scale;      /* gate score scale, > 0; default 1/sqrt(128) */
   int32_t kv_dtype;      /* sas_dtype of q, K and V (and of prefill Q) */
   int32_t out_dtype;     /* sas_dtype of the attention output */
-  int32_t gate_mode;     /* sas_gate_mode; default SAS_GATE_SELECT_ONLY.  Only
-                            sas_decode_step(_static) implement the gated mode;
-                            sas_sparse_decode and sas_prefill_block_sparse
-                            return SAS_ERR_UNSUPPORTED for it, the gate-score,
-                            Top-K and pooling calls ignore it. */
+  int32_t gate_mode;     /* sas_gate_mode; default SAS_GATE_SELECT_ONLY.
+                            sas_decode_step(_static) and sas_prefill_block_sparse
+                            implement the gated mode (prefill: gates of each
+                            query block's gate query; a larger workspace, see
+                            sas_workspace_bytes); sas_sparse_decode returns
+                            SAS_ERR_UNSUPPORTED for it (it has no gate inputs);
+                            the gate-score, Top-K and pooling calls ignore it. */
   int32_t gate_keys_bf16;  /* 0 (default): the gate-key cache is fp32
                               [B][Hkv][MG][128].  1: it is bf16, keys rounded to
                               nearest-even when written (half the bytes the

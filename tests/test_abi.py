@@ -192,13 +192,17 @@ def test_other_entry_points_validate(L):
 
 
 @nogpu
-def test_gated_mode_only_in_the_fused_decode_step(L):
-    """The gated mode needs the gate query and keys: sas_sparse_decode and the
-    prefill refuse it on the host, before any CUDA call."""
+def test_gated_mode_not_in_sparse_decode(L):
+    """The gated mode needs the gate query and keys: sas_sparse_decode, which
+    has neither, refuses it on the host, before any CUDA call."""
     c = _cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS).c()
     kv = _kv()
     assert L.sas_sparse_decode(ctypes.byref(c), FAKE, ctypes.byref(kv), FAKE, FAKE, FAKE, FAKE,
                                256, None) == sas.SAS_ERR_UNSUPPORTED
-    assert L.sas_prefill_block_sparse(ctypes.byref(c), FAKE, FAKE, FAKE, 2, 4096, FAKE, FAKE, FAKE, FAKE,
-                                      FAKE, 64, FAKE, None, None, FAKE, 1 << 30,
-                                      None) == sas.SAS_ERR_UNSUPPORTED
+
+
+def test_gated_prefill_needs_a_larger_workspace(L):
+    plain = sas.workspace_bytes(_cfg(), 2, 4096)
+    gated = sas.workspace_bytes(_cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS), 2, 4096)
+    # gates of every (sequence, query head, query block, list entry): 2 * 32 * 64 * 32 floats
+    assert gated - plain >= 2 * 32 * 64 * 32 * 4

@@ -18,11 +18,12 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _run(spec, gk16=0):
+def _run(spec, gk16=0, gate_mode=sas.GATE_SELECT_ONLY):
     inp = make_prefill_inputs(spec, DEV)
     B, Tn = spec.batch, spec.seq_len
     nblk = Tn // 64
-    cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget, gate_keys_bf16=gk16)
+    cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget, gate_keys_bf16=gk16,
+                     gate_mode=gate_mode)
     ws = sas.make_workspace(cfg, DEV, batch=B, max_seq_len=Tn)
     gk = torch.zeros(B, spec.hkv, nblk, 128, dtype=sas.gate_key_dtype(cfg), device=DEV)
     out = torch.full((B, spec.hq, Tn, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
@@ -60,16 +61,23 @@ def _check(spec, inp, cfg, gk, out, sel, cnt, triples):
             cache[(s, h)] = (ks, vs, keys)
         ks, vs, keys = cache[(s, h)]
         qb = inp["q"][s, h * G:(h + 1) * G, 64 * i:64 * (i + 1)].double().cpu().numpy()
-        r = O.prefill_query_block(qb, ks, vs, i, keys, wq[h * G:(h + 1) * G], np.tile(ones, (G, 1)), topk)
+        r = O.prefill_query_block(qb, ks, vs, i, keys, wq[h * G:(h + 1) * G], np.tile(ones, (G, 1)), topk,
+                                  gate_mode=cfg.gate_mode)
         m = int(cnt_h[s, h, i])
         got_sel = list(sel_h[s, h, i, :m])
         tag = f"{spec.name} s={s} h={h} i={i}"
         swapped = T.assert_selection(got_sel, r["sel"], r["S"], topk, tag)
         want = r["out"]
         if swapped:
+            # the kernel kept a tie-window swap: attend over its list, gates from the oracle's scores
             hist = O.selected_token_ids(got_sel[:-1], 64 * (i + 1))
-            want = np.stack([np.stack([O.attention_over_tokens(qb[g, t], ks, vs, hist + list(range(64 * i, 64 * i + t + 1)),
-                                                                 cfg.attn_scale) for t in range(64)]) for g in range(G)])
+            want = np.zeros((G, 64, 128))
+            for g in range(G):
+                hb = O.gated_token_bias(r["s"][g], got_sel[:-1], 64 * (i + 1), i) if cfg.gate_mode else None
+                for t in range(64):
+                    bias = None if hb is None else hb + [0.0] * (t + 1)
+                    want[g, t] = O.attention_over_tokens(qb[g, t], ks, vs, hist + list(range(64 * i, 64 * i + t + 1)),
+                                                         cfg.attn_scale, bias)
         got = out_h[s, h * G:(h + 1) * G, 64 * i:64 * (i + 1)]
         err = float(np.max(np.abs(got - want)))
         assert np.all(np.isfinite(got)) and err <= T.OUT_ATOL, f"{tag}: out max-abs err {err}"
@@ -87,6 +95,24 @@ def test_prefill_small_bf16_gate_keys():
     res = _run(spec, gk16=1)
     triples = [(0, h, i) for h in range(2) for i in range(16)]
     _check(spec, *res, triples)
+
+
+def test_prefill_gated_mode():
+    spec = PrefillSpec("pf_gated", 1, 4, 2, 1024, token_budget=256, seed=44)
+    res = _run(spec, gate_mode=sas.GATE_LOGSIGMOID_BIAS)
+    _check(spec, *res, [(0, h, i) for h in range(2) for i in range(16)])
+
+
+def test_prefill_gated_mode_bf16_keys_eight_heads_per_group():
+    spec = PrefillSpec("pf_gated_g8", 1, 8, 1, 768, token_budget=320, seed=45)
+    res = _run(spec, gk16=1, gate_mode=sas.GATE_LOGSIGMOID_BIAS)
+    _check(spec, *res, [(0, 0, i) for i in range(12)])
+
+
+def test_prefill_gated_mode_full_size_sampled():
+    spec = qwen3_8b_prefill_32k()
+    res = _run(spec, gate_mode=sas.GATE_LOGSIGMOID_BIAS)
+    _check(spec, *res, [(0, 1, 1), (1, 6, 100), (3, 4, 511)])
 
 
 def test_prefill_budget_covering_context_is_dense_causal():
