@@ -224,7 +224,8 @@ def measured_tensor_peak():
 def run_prefill(args, device, world):
     """Block-sparse chunked prefill, Qwen3-8B heads, 32,768 tokens per sequence,
     Top-K 31 + diagonal: one sas_prefill_block_sparse call per step (pooling,
-    gate queries, selection, tcgen05 attention), in both gate modes."""
+    gate queries, selection, tcgen05 attention), in both gate modes and with
+    per-sequence budgets."""
     import torch
     from gated_block_sparse_token_b200 import sas
     from gated_block_sparse_token_b200.workloads import make_prefill_inputs, qwen3_8b_prefill_32k
@@ -237,35 +238,49 @@ def run_prefill(args, device, world):
     gk = torch.zeros(B, spec.hkv, nblk, 128, dtype=torch.float32, device=device)
     stream = torch.cuda.Stream(device)
 
-    def time_mode(gate_mode):
-        cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget, gate_mode=gate_mode)
+    def make_call(gate_mode, budgets=None):
+        cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget if budgets is None else max(budgets),
+                         gate_mode=gate_mode)
         ws = sas.make_workspace(cfg, device, batch=B, max_seq_len=T)
+        tb = None if budgets is None else torch.tensor(budgets, dtype=torch.int32, device=device)
 
         def call():
             sas.prefill_block_sparse(cfg, inp["q"], inp["k"], inp["v"], inp["w_q"], inp["gamma_q"], inp["w_k"],
-                                     inp["gamma_k"], gk, out, ws, stream=stream)
+                                     inp["gamma_k"], gk, out, ws, stream=stream, token_budgets=tb)
+        return call, ws
 
-        with torch.cuda.stream(stream):
-            for _ in range(2):
+    mixed = [1024, 2048, 4096, 2048][:B] if B <= 4 else None
+    modes = [make_call(sas.GATE_SELECT_ONLY), make_call(sas.GATE_LOGSIGMOID_BIAS)]
+    if mixed:
+        modes.append(make_call(sas.GATE_SELECT_ONLY, mixed))
+    # the modes take turns, call by call, so that all of them see the same
+    # clocks (a long tensor-core run settles under the power cap)
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            for call, _ws in modes:
                 call()
-        torch.cuda.synchronize()
-        barrier(world)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(args.prefill_steps):
+    torch.cuda.synchronize()
+    barrier(world)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.prefill_steps)] for _ in modes]
+    clk = ClockSampler(torch.device(device).index or 0)
+    clk.start()
+    time.sleep(0.3)  # nvidia-smi's first sample
+    with torch.cuda.stream(stream):
+        for k in range(args.prefill_steps):
+            for (call, _ws), evm in zip(modes, ev):
+                evm[k][0].record(stream)
                 call()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        t = max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.prefill_steps, world)
+                evm[k][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = clk.stop()
+    barrier(world)
+    times = [max_over_ranks(sum(a.elapsed_time(b) for a, b in evm) / 1e3 / args.prefill_steps, world) for evm in ev]
+    for _call, ws in modes:
         if sas.get_device_status(ws, stream) != sas.SAS_OK:
             raise RuntimeError("device status not OK after the prefill run")
-        return t
-
-    t = time_mode(sas.GATE_SELECT_ONLY)
-    t_gated = time_mode(sas.GATE_LOGSIGMOID_BIAS)
+    t, t_gated = times[0], times[1]
+    t_mixed = times[2] if mixed else None
     flops = prefill_flops(nblk, spec.hq, spec.hkv, spec.token_budget, B)
     peak, kind = measured_tensor_peak()
     achieved = flops / t / 1e12
@@ -273,7 +288,10 @@ def run_prefill(args, device, world):
             "kv_heads": spec.hkv, "token_budget": spec.token_budget, "steps": args.prefill_steps,
             "ms_per_step": round(t * 1e3, 4), "tokens_per_s": round(job_throughput(B * T, world, t), 1),
             "launches_per_step": 4,
+            "clocks": clocks,
             "gated_mode_ms_per_step": round(t_gated * 1e3, 4),
+            "mixed_budgets": None if t_mixed is None else {"token_budgets": mixed,
+                                                          "ms_per_step": round(t_mixed * 1e3, 4)},
             "roofline": {"kernel": "prefill_attn_kernel (tcgen05)", "bound": "tensor",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "peak_kind": kind,

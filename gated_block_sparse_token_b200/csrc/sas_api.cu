@@ -20,7 +20,7 @@ namespace {
 
 using sas::kDim;
 
-constexpr int32_t kAbiVersion = 5;
+constexpr int32_t kAbiVersion = 6;
 constexpr size_t kStatusBytes = 256;  // status word + padding
 constexpr int kMaxBudget = 16384;
 constexpr int kMaxGateBlocks = 16384;
@@ -213,10 +213,10 @@ size_t ws_header_bytes() {
 
 size_t up256(size_t x) { return (x + 255) / 256 * 256; }
 
-// gate queries, block lists, list lengths (+ gated mode: the gates of the lists)
-size_t prefill_scratch_bytes(size_t batch, int hq, int hkv, size_t nblk, int max_sel, bool gated) {
+// gate queries, block lists, list lengths
+size_t prefill_scratch_bytes(size_t batch, int hq, int hkv, size_t nblk, int max_sel) {
   return up256(batch * hq * nblk * kDim * 4) + up256(batch * hkv * nblk * max_sel * 4) +
-         up256(batch * hkv * nblk * 4) + (gated ? up256(batch * hq * nblk * max_sel * 4) : 0);
+         up256(batch * hkv * nblk * 4);
 }
 
 sas_status launch_result(cudaError_t e) {
@@ -253,7 +253,7 @@ size_t sas_workspace_bytes(const sas_config* cfg, int32_t batch, int32_t max_seq
     // prefill scratch: gate queries, block lists and their lengths
     const size_t nblk = static_cast<size_t>((max_seq_len + 63) / 64);
     bytes += prefill_scratch_bytes(batch, cfg->num_q_heads, cfg->num_kv_heads, nblk,
-                                   cfg->token_budget / 64, cfg->gate_mode == SAS_GATE_LOGSIGMOID_BIAS);
+                                   cfg->token_budget / 64);
   }
   return bytes;
 }
@@ -451,7 +451,7 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
 
 sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const void* k,
                                     const void* v, int32_t batch, int32_t seq_len,
-                                    const void* w_q, const float* gamma_q, const void* w_k,
+                                    const int32_t* token_budgets, const void* w_q, const float* gamma_q, const void* w_k,
                                     const float* gamma_k, void* gate_keys,
                                     int32_t max_gate_blocks, void* out, int32_t* sel_idx,
                                     int32_t* sel_count, void* ws, size_t ws_bytes,
@@ -473,7 +473,7 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(w_q, 16) ||
       !aligned(gamma_q, 16) || !aligned(w_k, 16) || !aligned(gamma_k, 16) ||
       !aligned(gate_keys, 16) || !aligned(out, 16) || (sel_idx != nullptr && !aligned(sel_idx, 4)) ||
-      (sel_count != nullptr && !aligned(sel_count, 4)))
+      (sel_count != nullptr && !aligned(sel_count, 4)) || !aligned(token_budgets, 4))
     return SAS_ERR_INVALID_ARG;
   if (ws == nullptr || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
   if (ws_bytes < sas_workspace_bytes(cfg, batch, seq_len)) return SAS_ERR_WORKSPACE;
@@ -537,8 +537,8 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
   p.sel = reinterpret_cast<int32_t*>(scratch);
   scratch += up256(static_cast<size_t>(batch) * p.hkv * nblk * p.max_sel * 4);
   p.cnt = reinterpret_cast<int32_t*>(scratch);
-  scratch += up256(static_cast<size_t>(batch) * p.hkv * nblk * 4);
-  p.gb = (cfg->gate_mode == SAS_GATE_LOGSIGMOID_BIAS) ? reinterpret_cast<float*>(scratch) : nullptr;
+  p.gated = (cfg->gate_mode == SAS_GATE_LOGSIGMOID_BIAS) ? 1 : 0;
+  p.token_budgets = token_budgets;
   p.sel_out = sel_idx;
   p.cnt_out = sel_count;
   p.out = static_cast<__nv_bfloat16*>(out);

@@ -393,6 +393,11 @@ __device__ __forceinline__ float exp2_approx(float x) {
 }
 
 // Arrive on a local mbarrier (one arrival, no transaction bytes).
+// barrier `id` (1..15) among the first `n` threads of the CTA (n a multiple of 32)
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }

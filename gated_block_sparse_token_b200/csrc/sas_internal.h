@@ -166,7 +166,8 @@ struct PrefillParams {
   int32_t* cnt;               // workspace: list lengths [B][Hkv][nblk]
   int32_t* sel_out;           // optional copies of the lists
   int32_t* cnt_out;
-  float* gb;                  // gated mode: gates [B][Hkv][nblk][max_sel][G] (workspace), else null
+  int gated;                  // gated mode: + log(sigmoid(gate score)) on kept historical blocks
+  const int32_t* token_budgets;  // [B] per-sequence budgets, or null (topk for every sequence)
   __nv_bfloat16* out;         // [B][Hq][T][128]
   uint32_t* status;
   unsigned long long* trace;  // per-CTA timings (tracing builds only), else null

@@ -8,10 +8,10 @@
 //
 // One CTA handles up to kPoolBlocksPerCta consecutive blocks of one (s, h).
 // W_k[h] (96 KiB bf16) comes into shared memory with one TMA bulk copy that
-// overlaps the pooling; the block's K rows are read with 16-byte loads (all
-// rows of a block in flight at once), reduced per row group in registers and
-// across row groups in shared memory.  The 384x128 projection then runs out
-// of shared memory, thread d owning output dimension d.
+// overlaps the pooling; each warp pools whole blocks (16-byte loads, 16 rows
+// in flight per lane, reduced in registers and across the lanes that share
+// a column chunk).  The 384x128 projection of all the CTA's blocks then runs
+// out of shared memory at once, thread d owning output dimension d.
 #include <cmath>
 
 #include "sas_internal.h"
@@ -22,9 +22,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads) pool_keys_kernel(const __grid_constant__ PoolParams p) {
   constexpr int NB = kPoolBlocksPerCta;
   constexpr int VEC = 16 / static_cast<int>(sizeof(T));  // elements per 16-byte load
-  constexpr int TPR = kDim / VEC;                       // threads per K row
-  constexpr int RG = kThreads / TPR;                    // row groups
-  constexpr int RPT = kBlock / RG;                      // rows per thread
+  constexpr int TPR = kDim / VEC;                       // lanes per K row
   const int s = blockIdx.z;
   const int h = blockIdx.y;
   const int tid = threadIdx.x;
@@ -33,10 +31,10 @@ __global__ void __launch_bounds__(kThreads) pool_keys_kernel(const __grid_consta
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __nv_bfloat16* wk_s = reinterpret_cast<__nv_bfloat16*>(smem_raw);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + kPoolWkBytes);
-  __shared__ float P[NB][kPool];
-  __shared__ float red[RG][3][kDim];
-  __shared__ float xn[kDim];
-  __shared__ float ssq[kWarps];
+  // pooled blocks, [pooled dim][block]; reused for the normalised u, [block][dim]
+  __shared__ __align__(16) float Pt[kPool][NB];
+  float (*xs)[kDim] = reinterpret_cast<float (*)[kDim]>(&Pt[0][0]);
+  __shared__ float ssq[kWarps][NB];
 
   const int L = (p.kv.seq_lens != nullptr) ? p.kv.seq_lens[s] : p.kv.capacity;  // prefill: full length
   const int first = p.blk_begin != nullptr ? p.blk_begin[s] : 0;
@@ -66,73 +64,77 @@ __global__ void __launch_bounds__(kThreads) pool_keys_kernel(const __grid_consta
   if (tid == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
-  }
-  __syncthreads();
-  if (tid == 0) {
     mbar_arrive_expect_tx(bar, kPoolWkBytes);
     bulk_g2s(wk_s, p.w_k + static_cast<size_t>(h) * kPool * kDim, kPoolWkBytes, bar);
   }
 
-  // ---- pooling: max, min, mean over the 64 tokens, per dimension
-  const T* kbase = static_cast<const T*>(p.kv.k);
-  const int cvec = tid % TPR;  // dims cvec*VEC .. +VEC
-  const int rg = tid / TPR;    // rows rg, rg+RG, ...
-  for (int i = 0; i < nb; ++i) {
-    if (rows[i] < 0) continue;  // uniform
-    const T* blk = kbase + rows[i] * kDim + cvec * VEC;
-    uint4 raw[RPT];
-#pragma unroll
-    for (int r = 0; r < RPT; ++r)
-      raw[r] = *reinterpret_cast<const uint4*>(blk + static_cast<size_t>(rg + r * RG) * kDim);
-    float mx[VEC], mn[VEC], sm[VEC];
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) {
-      mx[v] = -INFINITY;
-      mn[v] = INFINITY;
-      sm[v] = 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-      const T* e = reinterpret_cast<const T*>(&raw[r]);
+  // ---- pooling: max, min, mean over the 64 tokens, per dimension.  Warp w
+  // pools blocks w, w + 4, ...: lane l reads the 16-byte chunk l % TPR of
+  // rows l / TPR, l / TPR + RPW, ... (16 rows' loads in flight per lane)
+  {
+    constexpr int RPW = 32 / TPR;          // rows per warp step (2 bf16, 1 fp32)
+    constexpr int ROWS = kBlock / RPW;     // rows per lane
+    const T* kbase = static_cast<const T*>(p.kv.k);
+    const int cvec = lane % TPR, par = lane / TPR;
+    for (int i = warp; i < NB; i += kWarps) {  // warp-uniform
+      float mx[VEC], mn[VEC], sm[VEC];
 #pragma unroll
       for (int v = 0; v < VEC; ++v) {
-        const float x = to_float(e[v]);
-        mx[v] = fmaxf(mx[v], x);
-        mn[v] = fminf(mn[v], x);
-        sm[v] += x;
+        mx[v] = -INFINITY;
+        mn[v] = INFINITY;
+        sm[v] = 0.f;
       }
-    }
+      if (rows[i] >= 0) {
+        const T* blk = kbase + (rows[i] + par) * kDim + cvec * VEC;
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) {
-      red[rg][0][cvec * VEC + v] = mx[v];
-      red[rg][1][cvec * VEC + v] = mn[v];
-      red[rg][2][cvec * VEC + v] = sm[v];
-    }
-    __syncthreads();
-    {
-      const int d = tid;
-      float a = red[0][0][d], b = red[0][1][d], c = red[0][2][d];
+        for (int part = 0; part < ROWS / 16; ++part) {
+          uint4 raw[16];
 #pragma unroll
-      for (int g = 1; g < RG; ++g) {
-        a = fmaxf(a, red[g][0][d]);
-        b = fminf(b, red[g][1][d]);
-        c += red[g][2][d];
+          for (int r = 0; r < 16; ++r)
+            raw[r] = *reinterpret_cast<const uint4*>(blk + static_cast<size_t>(RPW * (16 * part + r)) * kDim);
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            const T* e = reinterpret_cast<const T*>(&raw[r]);
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+              const float x = to_float(e[v]);
+              mx[v] = fmaxf(mx[v], x);
+              mn[v] = fminf(mn[v], x);
+              sm[v] += x;
+            }
+          }
+        }
       }
-      c *= (1.f / kBlock);
-      P[i][d] = a;
-      P[i][kDim + d] = b;
-      P[i][2 * kDim + d] = c;
-      if (p.pooled_raw != nullptr) {
-        float* pr = p.pooled_raw + ((static_cast<size_t>(s) * p.hkv + h) * p.mg + (b0 + i)) * kPool;
-        pr[d] = a;
-        pr[kDim + d] = b;
-        pr[2 * kDim + d] = c;
+#pragma unroll
+      for (int o = TPR; o < 32; o <<= 1) {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          mx[v] = fmaxf(mx[v], __shfl_xor_sync(0xffffffffu, mx[v], o));
+          mn[v] = fminf(mn[v], __shfl_xor_sync(0xffffffffu, mn[v], o));
+          sm[v] += __shfl_xor_sync(0xffffffffu, sm[v], o);
+        }
+      }
+      if (par == 0) {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          const int dd = cvec * VEC + v;
+          const float mean = sm[v] * (1.f / kBlock);
+          Pt[dd][i] = rows[i] >= 0 ? mx[v] : 0.f;
+          Pt[kDim + dd][i] = rows[i] >= 0 ? mn[v] : 0.f;
+          Pt[2 * kDim + dd][i] = mean;
+          if (p.pooled_raw != nullptr && rows[i] >= 0) {
+            float* pr = p.pooled_raw + ((static_cast<size_t>(s) * p.hkv + h) * p.mg + (b0 + i)) * kPool;
+            pr[dd] = mx[v];
+            pr[kDim + dd] = mn[v];
+            pr[2 * kDim + dd] = mean;
+          }
+        }
       }
     }
-    __syncthreads();
   }
+  __syncthreads();
 
-  // ---- u = P @ W_k[h] from shared memory
+  // ---- u = P @ W_k[h] from shared memory, thread d owning output dimension d
   const bool ok = mbar_wait(bar, 0, p.status);
   const int d = tid;
   float u[NB];
@@ -142,43 +144,46 @@ __global__ void __launch_bounds__(kThreads) pool_keys_kernel(const __grid_consta
 #pragma unroll 4
     for (int r = 0; r < kPool; ++r) {
       const float w = __bfloat162float(wk_s[r * kDim + d]);
+      const float4* p4 = reinterpret_cast<const float4*>(&Pt[r][0]);
 #pragma unroll
-      for (int i = 0; i < NB; ++i)
-        if (i < nb) u[i] = fmaf(P[i][r], w, u[i]);
+      for (int c = 0; c < NB / 4; ++c) {
+        const float4 x = p4[c];
+        u[4 * c] = fmaf(x.x, w, u[4 * c]);
+        u[4 * c + 1] = fmaf(x.y, w, u[4 * c + 1]);
+        u[4 * c + 2] = fmaf(x.z, w, u[4 * c + 2]);
+        u[4 * c + 3] = fmaf(x.w, w, u[4 * c + 3]);
+      }
     }
   }
 
   // ---- RMSNorm (gain gamma_k) and gate RoPE at the block index, per block
-  const float gk = p.gamma_k[d];
-  const int j = d & 63;
-  for (int i = 0; i < nb; ++i) {
-    float sq = u[0] * u[0];
 #pragma unroll
-    for (int k = 1; k < NB; ++k)
-      if (k == i) sq = u[k] * u[k];
-    float ui = u[0];
-#pragma unroll
-    for (int k = 1; k < NB; ++k)
-      if (k == i) ui = u[k];
+  for (int i = 0; i < NB; ++i) {
+    float sq = u[i] * u[i];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    if (lane == 0) ssq[warp] = sq;
-    __syncthreads();
-    const float tot = ssq[0] + ssq[1] + ssq[2] + ssq[3];
-    xn[d] = ui * (1.f / sqrtf(tot / kDim + p.eps)) * gk;
-    __syncthreads();
-    if (rows[i] >= 0) {
-      const int b = b0 + i;
-      float cs, sn;
-      rope_cos_sin(p.rope.theta_over_pi[j], b, cs, sn);
-      const float y = (d < 64) ? xn[d] * cs - xn[d + 64] * sn : xn[d] * cs + xn[d - 64] * sn;
-      const size_t gi = ((static_cast<size_t>(s) * p.hkv + h) * p.mg + b) * kDim + d;
-      if (p.gk16)
-        static_cast<__nv_bfloat16*>(p.gate_keys)[gi] = __float2bfloat16_rn(y);
-      else
-        static_cast<float*>(p.gate_keys)[gi] = y;
-    }
-    __syncthreads();
+    if (lane == 0) ssq[warp][i] = sq;
+  }
+  __syncthreads();  // every Pt read is done: xs may overwrite it
+  const float gk = p.gamma_k[d];
+#pragma unroll
+  for (int i = 0; i < NB; ++i) {
+    const float tot = ssq[0][i] + ssq[1][i] + ssq[2][i] + ssq[3][i];
+    xs[i][d] = u[i] * (1.f / sqrtf(tot / kDim + p.eps)) * gk;
+  }
+  __syncthreads();
+  const int j = d & 63;
+  for (int i = 0; i < nb; ++i) {
+    if (rows[i] < 0) continue;
+    const int b = b0 + i;
+    float cs, sn;
+    rope_cos_sin(p.rope.theta_over_pi[j], b, cs, sn);
+    const float y = (d < 64) ? xs[i][d] * cs - xs[i][d + 64] * sn : xs[i][d] * cs + xs[i][d - 64] * sn;
+    const size_t gi = ((static_cast<size_t>(s) * p.hkv + h) * p.mg + b) * kDim + d;
+    if (p.gk16)
+      static_cast<__nv_bfloat16*>(p.gate_keys)[gi] = __float2bfloat16_rn(y);
+    else
+      static_cast<float*>(p.gate_keys)[gi] = y;
   }
 }
 

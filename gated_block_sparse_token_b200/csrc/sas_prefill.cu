@@ -27,75 +27,118 @@
 namespace sas {
 
 // ------------------------------------------------------------ gate queries
-// grid (ceil(nblk / kPfQb), Hq, B), 128 threads.  Thread d owns dimension d.
+// grid (ceil(nblk / kPfQb), Hq, B), 128 threads; one CTA per kPfQb query
+// blocks of one (sequence, query head).
+//   A. block sums: warp w sums the 64 queries of blocks w, w + 4, ... (lane:
+//      16-byte column chunk lane % 16, rows of parity lane / 16; 16 rows'
+//      loads in flight per lane), into qm[dim][block];
+//   B. u = mean @ W_q[g] for all the CTA's blocks at once, thread d owning
+//      output dimension d (W_q read from shared memory once per CTA);
+//   C. RMSNorm (gain gamma_q) and gate RoPE at each block's index.
 __global__ void __launch_bounds__(kThreads) prefill_gate_query_kernel(const __grid_constant__ PrefillParams p) {
+  constexpr int NB = kPfQb;
   const int g = blockIdx.y;
   const int s = blockIdx.z;
-  const int i0 = blockIdx.x * kPfQb;
+  const int i0 = blockIdx.x * NB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __nv_bfloat16* wq = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // [128][128]
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw + kDim * kDim * 2);
-  __shared__ float red[8][kDim];
-  __shared__ float qbar[kDim];
-  __shared__ float xn[kDim];
-  __shared__ float ssq[kWarps];
+  __shared__ __align__(16) float qm[kDim][NB];  // block sums, [dim][block]
+  __shared__ float xs[NB][kDim];                // normalised u, [block][dim]
+  __shared__ float ssq[kWarps][NB];
   if (tid == 0) {
     mbar_init(bar, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(bar, kDim * kDim * 2);
     bulk_g2s(wq, p.w_q + static_cast<size_t>(g) * kDim * kDim, kDim * kDim * 2, bar);
   }
+  const int nb = min(NB, p.nblk - i0);  // blocks of this CTA (>= 1)
+
+  // ---- A. sums of the 64 queries of each block
+  {
+    const int cvec = lane & 15, par = lane >> 4;
+    for (int bi = warp; bi < NB; bi += kWarps) {  // warp-uniform
+      float acc[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) acc[v] = 0.f;
+      if (bi < nb) {
+        const __nv_bfloat16* qb =
+            p.q + ((static_cast<size_t>(s) * p.hq + g) * p.T + static_cast<size_t>(i0 + bi) * kBlock + par) * kDim +
+            cvec * 8;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint4 raw[16];
+#pragma unroll
+          for (int r = 0; r < 16; ++r)
+            raw[r] = *reinterpret_cast<const uint4*>(qb + static_cast<size_t>(2 * (16 * half + r)) * kDim);
+#pragma unroll
+          for (int r = 0; r < 16; ++r) {
+            const uint32_t u[4] = {raw[r].x, raw[r].y, raw[r].z, raw[r].w};
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              acc[2 * v] += bf16_lo(u[v]);
+              acc[2 * v + 1] += bf16_hi(u[v]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < 8; ++v) acc[v] += __shfl_xor_sync(0xffffffffu, acc[v], 16);
+      if (par == 0) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) qm[cvec * 8 + v][bi] = acc[v];
+      }
+    }
+  }
   __syncthreads();
   const bool ok = mbar_wait(bar, 0, p.status);
-  const float gam = p.gamma_q[tid];
-  const int cvec = tid & 15, rg = tid >> 4;  // 8 dims x rows rg, rg+8, ...
-  const int i1 = min(p.nblk, i0 + kPfQb);
-  for (int i = i0; i < i1; ++i) {
-    const __nv_bfloat16* qb = p.q + ((static_cast<size_t>(s) * p.hq + g) * p.T + static_cast<size_t>(i) * kBlock) * kDim;
-    uint4 raw[8];
+
+  // ---- B. u_b[d] = (sum_b / 64) . W_q[:, d]
+  const int d = tid;
+  float u[NB];
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
-      raw[r] = *reinterpret_cast<const uint4*>(qb + static_cast<size_t>(rg + 8 * r) * kDim + cvec * 8);
-    float acc[8];
+  for (int b = 0; b < NB; ++b) u[b] = 0.f;
+  if (ok) {
+#pragma unroll 4
+    for (int r = 0; r < kDim; ++r) {
+      const float w = __bfloat162float(wq[r * kDim + d]);
+      const float4* m4 = reinterpret_cast<const float4*>(&qm[r][0]);
 #pragma unroll
-    for (int v = 0; v < 8; ++v) acc[v] = 0.f;
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw[r]);
-#pragma unroll
-      for (int v = 0; v < 8; ++v) acc[v] += __bfloat162float(e[v]);
+      for (int c = 0; c < NB / 4; ++c) {
+        const float4 x = m4[c];
+        u[4 * c] = fmaf(x.x, w, u[4 * c]);
+        u[4 * c + 1] = fmaf(x.y, w, u[4 * c + 1]);
+        u[4 * c + 2] = fmaf(x.z, w, u[4 * c + 2]);
+        u[4 * c + 3] = fmaf(x.w, w, u[4 * c + 3]);
+      }
     }
+  }
 #pragma unroll
-    for (int v = 0; v < 8; ++v) red[rg][cvec * 8 + v] = acc[v];
-    __syncthreads();
-    {
-      float sm = 0.f;
+  for (int b = 0; b < NB; ++b) u[b] *= (1.f / kBlock);  // a power of two: exact
+
+  // ---- C. RMSNorm and RoPE per block
 #pragma unroll
-      for (int r = 0; r < 8; ++r) sm += red[r][tid];
-      qbar[tid] = sm * (1.f / kBlock);  // per-head mean of the block's 64 queries
-    }
-    __syncthreads();
-    float u = 0.f;
-    if (ok) {
-      float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 16
-      for (int r = 0; r < kDim; ++r) a4[r & 3] = fmaf(qbar[r], __bfloat162float(wq[r * kDim + tid]), a4[r & 3]);
-      u = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-    }
-    float sq = u * u;
+  for (int b = 0; b < NB; ++b) {
+    float sq = u[b] * u[b];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-    if (lane == 0) ssq[warp] = sq;
-    __syncthreads();
-    const float tot = ssq[0] + ssq[1] + ssq[2] + ssq[3];
-    xn[tid] = u * (1.f / sqrtf(tot / kDim + p.eps)) * gam;
-    __syncthreads();
+    if (lane == 0) ssq[warp][b] = sq;
+  }
+  __syncthreads();
+  const float gam = p.gamma_q[d];
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const float tot = ssq[0][b] + ssq[1][b] + ssq[2][b] + ssq[3][b];
+    xs[b][d] = u[b] * (1.f / sqrtf(tot / kDim + p.eps)) * gam;
+  }
+  __syncthreads();
+  for (int b = 0; b < nb; ++b) {
+    const int i = i0 + b;
     float cs, sn;
-    rope_cos_sin(p.rope.theta_over_pi[tid & 63], i, cs, sn);
-    const float y = (tid < 64) ? xn[tid] * cs - xn[tid + 64] * sn : xn[tid] * cs + xn[tid - 64] * sn;
-    p.qt[((static_cast<size_t>(s) * p.hq + g) * p.nblk + i) * kDim + tid] = y;
-    __syncthreads();  // red / qbar / xn / ssq are reused by the next block
+    rope_cos_sin(p.rope.theta_over_pi[d & 63], i, cs, sn);
+    const float y = (d < 64) ? xs[b][d] * cs - xs[b][d + 64] * sn : xs[b][d] * cs + xs[b][d - 64] * sn;
+    p.qt[((static_cast<size_t>(s) * p.hq + g) * p.nblk + i) * kDim + d] = y;
   }
 }
 
@@ -107,6 +150,22 @@ __global__ void __launch_bounds__(kThreads) prefill_select_kernel(const __grid_c
   const int s = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.G;
+  const size_t base = (static_cast<size_t>(s) * p.hkv + h) * p.nblk + i;
+  // this sequence's Top-K: budget / 64 - 1; a bad budget skips the sequence
+  // (empty lists, which the attention kernel reports and skips as well)
+  int topk = p.topk;
+  if (p.token_budgets != nullptr) {
+    const int b = p.token_budgets[s];
+    topk = (b >= kBlock && b <= p.max_sel * kBlock && b % kBlock == 0) ? b / kBlock - 1 : -1;
+  }
+  if (topk < 0) {
+    if (tid == 0) {
+      raise_status(p.status, kStatusBounds);
+      p.cnt[base] = 0;
+      if (p.cnt_out != nullptr) p.cnt_out[base] = 0;
+    }
+    return;
+  }
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* vals = reinterpret_cast<float*>(smem_raw);
   uint8_t* q = smem_raw + (p.nblk * 4 + 15) / 16 * 16;
@@ -159,37 +218,7 @@ __global__ void __launch_bounds__(kThreads) prefill_select_kernel(const __grid_c
     if (b < i && sub == 0) vals[b] = acc;
   }
   __syncthreads();
-  const int m = select_blocks(vals, i, p.topk, i, sel, hist, selbits, scan);
-  const size_t base = (static_cast<size_t>(s) * p.hkv + h) * p.nblk + i;
-  if (p.gb != nullptr) {
-    // gated mode: gate of every kept historical block and head of the group,
-    // log(sigmoid(q~_g(i) . k~_b * gate_scale)); one (entry, head) per thread
-    for (int w = tid; w < (m - 1) * G; w += kThreads) {
-      const int j = w / G, g = w - j * G;
-      const float4* qg = reinterpret_cast<const float4*>(
-          p.qt + ((static_cast<size_t>(s) * p.hq + h * G + g) * p.nblk + i) * kDim);
-      const size_t koff = gk_base + static_cast<size_t>(sel[j]) * kDim;
-      float a0 = 0.f, a1 = 0.f;
-      if (p.gk16) {
-        const uint4* kr = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.gate_keys) + koff);
-#pragma unroll 4
-        for (int c = 0; c < kDim / 8; c += 2) {
-          a0 = dot8_bf16(qg[2 * c], qg[2 * c + 1], kr[c], a0);
-          a1 = dot8_bf16(qg[2 * c + 2], qg[2 * c + 3], kr[c + 1], a1);
-        }
-      } else {
-        const float4* kr = reinterpret_cast<const float4*>(static_cast<const float*>(p.gate_keys) + koff);
-#pragma unroll 8
-        for (int c = 0; c < kDim / 4; c += 2) {
-          const float4 k0 = kr[c], k1 = kr[c + 1], q0 = qg[c], q1 = qg[c + 1];
-          a0 = fmaf(q0.x, k0.x, fmaf(q0.y, k0.y, fmaf(q0.z, k0.z, fmaf(q0.w, k0.w, a0))));
-          a1 = fmaf(q1.x, k1.x, fmaf(q1.y, k1.y, fmaf(q1.z, k1.z, fmaf(q1.w, k1.w, a1))));
-        }
-      }
-      const float sg = (a0 + a1) * p.gate_scale;
-      p.gb[(base * p.max_sel + j) * G + g] = (sg >= 0.f) ? -log1pf(expf(-sg)) : sg - log1pf(expf(sg));
-    }
-  }
+  const int m = select_blocks(vals, i, topk, i, sel, hist, selbits, scan);
   for (int j = tid; j < m; j += kThreads) {
     p.sel[base * p.max_sel + j] = sel[j];
     if (p.sel_out != nullptr) p.sel_out[base * p.max_sel + j] = sel[j];
@@ -276,7 +305,7 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + kPfSmemBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumPfBars);
   int* sel_s = reinterpret_cast<int*>(tmem_slot + 4);
-  float* gb_s = reinterpret_cast<float*>(sel_s + p.max_sel);  // gated mode: [entry][2 heads]
+  float* gb_s = reinterpret_cast<float*>(sel_s + p.max_sel);  // gated mode: gates [entry][2 heads]
   // the plan assumes a 1024-byte aligned dynamic shared window (swizzled
   // TMA boxes and UMMA descriptors); anything else is reported, not used
   const bool misaligned = (smem_u32(base) & 1023u) != 0;
@@ -294,13 +323,6 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
       const int b = sl[j];
       sel_s[j] = b;
       if (b < 0 || b > i || (j == m - 1 && b != i) || (j > 0 && sl[j - 1] >= b)) err = true;
-    }
-    if (p.gb != nullptr) {
-      const float* gl = p.gb + lbase * p.max_sel * p.G;
-      for (int w = tid; w < 2 * m; w += kPfAttnThreads) {
-        const int j = w >> 1;
-        gb_s[w] = (j < m - 1) ? gl[j * p.G + 2 * pair + (w & 1)] : 0.f;  // the diagonal block: 0
-      }
     }
   }
   if (tid == 0 && !misaligned) {
@@ -425,6 +447,74 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
     const int t = r & 63;
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * warp) << 16);
     float m_run = -INFINITY, l_run = 0.f;  // running maximum in log2 units, row sum
+    if (p.gated && m > 0) {
+      // gated mode: gate log(sigmoid(q~_g(i) . k~_b * gate_scale)) of every kept
+      // historical block b for the CTA's two heads, computed while the first
+      // Q / K copies and S tile are in flight.  Eight lanes per block (16
+      // dimensions each), 16 blocks per pass; the diagonal block gets 0.
+      const int grp = lane >> 3, sub = lane & 7;
+      const float4* qa = reinterpret_cast<const float4*>(
+          p.qt + ((static_cast<size_t>(s) * p.hq + g0) * p.nblk + i) * kDim + sub * 16);
+      const float4* qb = qa + static_cast<size_t>(p.nblk) * (kDim / 4);  // head g0 + 1
+      float4 q0[4], q1[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        q0[c] = qa[c];
+        q1[c] = qb[c];
+      }
+      const size_t gk_base = (static_cast<size_t>(s) * p.hkv + h) * p.mg * kDim + sub * 16;  // elements
+      for (int j0 = 0; j0 < m - 1; j0 += 16) {
+        const int j = j0 + 4 * warp + grp;
+        const bool ok = j < m - 1;
+        float kr[16];
+#pragma unroll
+        for (int x = 0; x < 16; ++x) kr[x] = 0.f;
+        if (ok) {
+          const size_t off = gk_base + static_cast<size_t>(sel_s[j]) * kDim;
+          if (p.gk16) {
+            const uint4* row = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.gate_keys) + off);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const uint4 w = row[c];
+              const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int x = 0; x < 4; ++x) {
+                kr[8 * c + 2 * x] = bf16_lo(u[x]);
+                kr[8 * c + 2 * x + 1] = bf16_hi(u[x]);
+              }
+            }
+          } else {
+            const float4* row = reinterpret_cast<const float4*>(static_cast<const float*>(p.gate_keys) + off);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float4 w = row[c];
+              kr[4 * c] = w.x;
+              kr[4 * c + 1] = w.y;
+              kr[4 * c + 2] = w.z;
+              kr[4 * c + 3] = w.w;
+            }
+          }
+        }
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          a0 = fmaf(q0[c].x, kr[4 * c], fmaf(q0[c].y, kr[4 * c + 1], fmaf(q0[c].z, kr[4 * c + 2], fmaf(q0[c].w, kr[4 * c + 3], a0))));
+          a1 = fmaf(q1[c].x, kr[4 * c], fmaf(q1[c].y, kr[4 * c + 1], fmaf(q1[c].z, kr[4 * c + 2], fmaf(q1[c].w, kr[4 * c + 3], a1))));
+        }
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+          a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+          a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+        }
+        if (ok && sub == 0) {
+          const float s0 = a0 * p.gate_scale, s1 = a1 * p.gate_scale;
+          gb_s[2 * j] = (s0 >= 0.f) ? -log1pf(expf(-s0)) : s0 - log1pf(expf(s0));
+          gb_s[2 * j + 1] = (s1 >= 0.f) ? -log1pf(expf(-s1)) : s1 - log1pf(expf(s1));
+        }
+      }
+      if (tid < 2) gb_s[2 * (m - 1) + tid] = 0.f;
+      named_bar_sync(1, 128);  // the four softmax warps
+    }
     for (int e = 0; e < m; ++e) {
       PF_TIC(ts);
       mbar_wait(&bars[kBarS0 + (e & 1)], (e >> 1) & 1, p.status);
@@ -447,7 +537,7 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
         mx1 = fmax3(mx1, sv[j + 2], sv[j + 3]);
       }
       // gated mode: + the block's gate for this row's head, in log2 units
-      const float beta2 = (p.gb != nullptr) ? gb_s[2 * e + (r >> 6)] * kLog2e : 0.f;
+      const float beta2 = p.gated ? gb_s[2 * e + (r >> 6)] * kLog2e : 0.f;
       const float mx = fmaf(fmax3(mx0, mx1, fmaxf(sv[62], sv[63])), sl2, beta2);
       const float m_new = fmaxf(m_run, mx);
       // rescale O only when the running maximum grows by more than 2^8:

@@ -18,6 +18,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 # SAS_LIBRARY selects another build of the same ABI (e.g. the phase-trace build).
 LIB_PATH = os.environ.get("SAS_LIBRARY", os.path.join(_HERE, "libsas.so"))
+ABI_VERSION = 6             # the include/sas.h this binding marshals for
 
 SAS_OK = 0
 SAS_ERR_INVALID_ARG = 1
@@ -85,12 +86,15 @@ def lib() -> ctypes.CDLL:
             "sas_sparse_decode": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step_static": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]),
-            "sas_prefill_block_sparse": (ctypes.c_int, [cfgp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
+            "sas_prefill_block_sparse": (ctypes.c_int, [cfgp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
+        if L.sas_abi_version() != ABI_VERSION:
+            raise RuntimeError(f"{LIB_PATH} has ABI {L.sas_abi_version()}, this binding wants {ABI_VERSION}: "
+                               "rebuild it")
         _lib = L
     return _lib
 
@@ -263,14 +267,16 @@ def decode_step_static(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out
 
 
 def prefill_block_sparse(cfg: Config, q, k, v, w_q, gamma_q, w_k, gamma_k, gate_keys, out, ws,
-                         sel_idx=None, sel_count=None, stream=None) -> None:
+                         sel_idx=None, sel_count=None, stream=None, token_budgets=None) -> None:
     """sas_prefill_block_sparse: q [B][Hq][T][128], k / v [B][Hkv][T][128] (bf16),
     out like q; writes gate_keys [B][Hkv][MG][128]; ws from
-    make_workspace(cfg, device, batch=B, max_seq_len=T)."""
+    make_workspace(cfg, device, batch=B, max_seq_len=T); token_budgets: None or
+    int32 [B] on the device (each a multiple of 64, at most cfg.token_budget)."""
     _check_gk(cfg, gate_keys)
     c = cfg.c()
     B, T = int(q.shape[0]), int(q.shape[2])
-    _check(lib().sas_prefill_block_sparse(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), B, T, _ptr(w_q),
+    _check(lib().sas_prefill_block_sparse(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), B, T,
+                                          _ptr(token_budgets), _ptr(w_q),
                                           _ptr(gamma_q), _ptr(w_k), _ptr(gamma_k), _ptr(gate_keys),
                                           int(gate_keys.shape[2]), _ptr(out), _ptr(sel_idx),
                                           _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),

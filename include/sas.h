@@ -107,9 +107,8 @@ typedef struct {
   int32_t out_dtype;     /* sas_dtype of the attention output */
   int32_t gate_mode;     /* sas_gate_mode; default SAS_GATE_SELECT_ONLY.
                             sas_decode_step(_static) and sas_prefill_block_sparse
-                            implement the gated mode (prefill: gates of each
-                            query block's gate query; a larger workspace, see
-                            sas_workspace_bytes); sas_sparse_decode returns
+                            implement the gated mode (prefill: gates from each
+                            query block's gate query); sas_sparse_decode returns
                             SAS_ERR_UNSUPPORTED for it (it has no gate inputs);
                             the gate-score, Top-K and pooling calls ignore it. */
   int32_t gate_keys_bf16;  /* 0 (default): the gate-key cache is fp32
@@ -258,11 +257,17 @@ SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const s
  * gate keys of blocks b < i; the min(budget/64 - 1, i) best blocks plus block
  * i; token t of block i attends to all tokens of the kept blocks and to
  * tokens 64i..t of its own block.
+ *   token_budgets: NULL (cfg->token_budget for every sequence) or int32 [B]
+ *   per-sequence budgets, each a multiple of 64 in 64 .. cfg->token_budget
+ *   (cfg->token_budget sizes the lists and the workspace).  A sequence with
+ *   a bad budget is skipped (its out rows set to 0, sel_count 0) and reported as
+ *   SAS_ERR_DEVICE_BOUNDS.
  *   q      bf16 [B][Hq][T][128]      k, v bf16 [B][Hkv][T][128]
  *   out    bf16 [B][Hq][T][128]      (all 16-byte aligned)
  *   w_q, gamma_q, w_k, gamma_k as for the decode entry points.
- *   gate_keys fp32 [B][Hkv][MG][128] (output): rows 0..T/64-1 are written, so
- *   decoding can continue from them.  MG >= T/64.
+ *   gate_keys [B][Hkv][MG][128] (output; fp32, bf16 when cfg->gate_keys_bf16):
+ *   rows 0..T/64-1 are written, so decoding can continue from them.
+ *   MG >= T/64.
  *   sel_idx int32 [B][Hkv][T/64][budget/64], sel_count int32 [B][Hkv][T/64]:
  *   optional outputs (NULL to skip), the block list of every query block.
  *   ws: 256-byte aligned, at least sas_workspace_bytes(cfg, B, T) bytes
@@ -273,6 +278,7 @@ SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const s
  */
 SAS_API sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const void* k,
                                             const void* v, int32_t batch, int32_t seq_len,
+                                            const int32_t* token_budgets,
                                             const void* w_q, const float* gamma_q,
                                             const void* w_k, const float* gamma_k,
                                             void* gate_keys, int32_t max_gate_blocks, void* out,

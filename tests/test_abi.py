@@ -84,7 +84,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(L):
-    assert sas.abi_version() >= 5
+    assert sas.abi_version() == sas.ABI_VERSION == 6
     for st in range(7):
         assert len(sas.status_string(st)) > 0
     assert sas.status_string(sas.SAS_OK) == "ok"
@@ -201,8 +201,26 @@ def test_gated_mode_not_in_sparse_decode(L):
                                256, None) == sas.SAS_ERR_UNSUPPORTED
 
 
-def test_gated_prefill_needs_a_larger_workspace(L):
-    plain = sas.workspace_bytes(_cfg(), 2, 4096)
-    gated = sas.workspace_bytes(_cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS), 2, 4096)
-    # gates of every (sequence, query head, query block, list entry): 2 * 32 * 64 * 32 floats
-    assert gated - plain >= 2 * 32 * 64 * 32 * 4
+def test_gated_mode_needs_no_more_workspace(L):
+    # the gates live in shared memory (decode and prefill alike)
+    for b, t in ((8, 32768), (2, 4096)):
+        assert sas.workspace_bytes(_cfg(), b, t) == sas.workspace_bytes(_cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS), b, t)
+
+
+def _prefill(L, c, budgets=None, batch=2, seq_len=4096, mg=64, ws=FAKE, ws_bytes=1 << 30, sel_count=None):
+    return L.sas_prefill_block_sparse(ctypes.byref(c), FAKE, FAKE, FAKE, batch, seq_len, budgets, FAKE, FAKE,
+                                      FAKE, FAKE, FAKE, mg, FAKE, None, sel_count, ws, ws_bytes, None)
+
+
+@nogpu
+def test_prefill_validates_on_the_host(L):
+    c = _cfg().c()
+    assert _prefill(L, c, budgets=FAKE + 2) == sas.SAS_ERR_INVALID_ARG     # misaligned budgets
+    assert _prefill(L, c, seq_len=4000) == sas.SAS_ERR_UNSUPPORTED        # not a multiple of 64
+    assert _prefill(L, c, mg=63) == sas.SAS_ERR_INVALID_ARG                # gate-key rows < T/64
+    assert _prefill(L, c, ws=FAKE + 16) == sas.SAS_ERR_WORKSPACE           # not 256-byte aligned
+    assert _prefill(L, c, ws_bytes=1024) == sas.SAS_ERR_WORKSPACE
+    assert _prefill(L, c, sel_count=FAKE + 1) == sas.SAS_ERR_INVALID_ARG
+    assert _prefill(L, _cfg(num_q_heads=24).c()) == sas.SAS_ERR_UNSUPPORTED  # odd group size (3)
+    assert _prefill(L, _cfg(token_budget=8192).c()) == sas.SAS_ERR_UNSUPPORTED
+    assert _prefill(L, c, batch=0) == sas.SAS_OK

@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _run(spec, gk16=0, gate_mode=sas.GATE_SELECT_ONLY):
+def _run(spec, gk16=0, gate_mode=sas.GATE_SELECT_ONLY, budgets=None, want_status=sas.SAS_OK):
     inp = make_prefill_inputs(spec, DEV)
     B, Tn = spec.batch, spec.seq_len
     nblk = Tn // 64
@@ -29,16 +29,16 @@ def _run(spec, gk16=0, gate_mode=sas.GATE_SELECT_ONLY):
     out = torch.full((B, spec.hq, Tn, 128), float("nan"), dtype=torch.bfloat16, device=DEV)
     sel = torch.full((B, spec.hkv, nblk, cfg.max_sel), -1, dtype=torch.int32, device=DEV)
     cnt = torch.full((B, spec.hkv, nblk), -1, dtype=torch.int32, device=DEV)
+    tb = None if budgets is None else torch.tensor(budgets, dtype=torch.int32, device=DEV)
     sas.prefill_block_sparse(cfg, inp["q"], inp["k"], inp["v"], inp["w_q"], inp["gamma_q"], inp["w_k"],
-                             inp["gamma_k"], gk, out, ws, sel_idx=sel, sel_count=cnt)
+                             inp["gamma_k"], gk, out, ws, sel_idx=sel, sel_count=cnt, token_budgets=tb)
     torch.cuda.synchronize()
-    assert sas.get_device_status(ws) == sas.SAS_OK
+    assert sas.get_device_status(ws) == want_status
     return inp, cfg, gk, out, sel, cnt
 
 
-def _check(spec, inp, cfg, gk, out, sel, cnt, triples):
+def _check(spec, inp, cfg, gk, out, sel, cnt, triples, budgets=None):
     G = spec.hq // spec.hkv
-    topk = cfg.max_sel - 1
     wq = inp["w_q"].double().cpu().numpy()
     wk = inp["w_k"].double().cpu().numpy()
     ones = np.ones(128)
@@ -61,6 +61,7 @@ def _check(spec, inp, cfg, gk, out, sel, cnt, triples):
             cache[(s, h)] = (ks, vs, keys)
         ks, vs, keys = cache[(s, h)]
         qb = inp["q"][s, h * G:(h + 1) * G, 64 * i:64 * (i + 1)].double().cpu().numpy()
+        topk = (cfg.max_sel if budgets is None else budgets[s] // 64) - 1
         r = O.prefill_query_block(qb, ks, vs, i, keys, wq[h * G:(h + 1) * G], np.tile(ones, (G, 1)), topk,
                                   gate_mode=cfg.gate_mode)
         m = int(cnt_h[s, h, i])
@@ -113,6 +114,31 @@ def test_prefill_gated_mode_full_size_sampled():
     spec = qwen3_8b_prefill_32k()
     res = _run(spec, gate_mode=sas.GATE_LOGSIGMOID_BIAS)
     _check(spec, *res, [(0, 1, 1), (1, 6, 100), (3, 4, 511)])
+
+
+def test_prefill_per_sequence_budgets():
+    spec = PrefillSpec("pf_budgets", 3, 4, 2, 1024, token_budget=512, seed=46)
+    res = _run(spec, budgets=[128, 512, 256])
+    _check(spec, *res, [(s, h, i) for s in range(3) for h in range(2) for i in (1, 2, 5, 9, 15)],
+           budgets=[128, 512, 256])
+    cnt = res[-1].cpu().numpy()
+    for s, kmax in enumerate((1, 7, 3)):
+        assert list(cnt[s, 0]) == [min(i, kmax) + 1 for i in range(16)]
+
+
+def test_prefill_per_sequence_budgets_gated():
+    spec = PrefillSpec("pf_budgets_gated", 2, 4, 1, 768, token_budget=384, seed=47)
+    res = _run(spec, gate_mode=sas.GATE_LOGSIGMOID_BIAS, budgets=[384, 192])
+    _check(spec, *res, [(s, 0, i) for s in range(2) for i in range(12)], budgets=[384, 192])
+
+
+def test_prefill_bad_budget_skips_that_sequence():
+    spec = PrefillSpec("pf_bad_budget", 2, 4, 1, 512, token_budget=256, seed=48)
+    inp, cfg, gk, out, sel, cnt = _run(spec, budgets=[256, 100], want_status=sas.SAS_ERR_DEVICE_BOUNDS)
+    assert torch.all(cnt[1] == 0)
+    assert torch.all(out[1] == 0)  # skipped: rows zeroed
+    assert not torch.isnan(out[0].float()).any()
+    _check(spec, inp, cfg, gk, out, sel, cnt, [(0, 0, i) for i in range(8)])
 
 
 def test_prefill_budget_covering_context_is_dense_causal():
