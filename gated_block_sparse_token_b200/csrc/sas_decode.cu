@@ -118,7 +118,6 @@ __global__ void __launch_bounds__(kThreads, 4)
   uint64_t* bar_v = bars + NST + 5;   // the gate query v (a slice from each CTA)
   uint64_t* bar_m = bars + NST + 6;   // attention partials of this CTA's columns
   uint64_t* bar_u = bars + NST + 7;   // rank 0: projected pooled slices
-  uint64_t* bar_gb = bars + NST + 8;  // ranks > 0, gated mode: the gates of the list
   float* pool_p = reinterpret_cast<float*>(base + p.sm.r_pool_p);
   float* pool_u = reinterpret_cast<float*>(base + p.sm.r_pool_u);
   __nv_bfloat16* wk_s = reinterpret_cast<__nv_bfloat16*>(base + p.sm.r_wk);
@@ -153,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 4)
       prefetch_tensormap(&tmv);
     }
     if (pool_on) prefetch_tensormap(&tmwk);
-    for (int i = 0; i < NST + 9; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < NST + 8; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
     const uint32_t qbytes = static_cast<uint32_t>(G * kDim * sizeof(T));
     uint32_t tx = qbytes;
@@ -237,10 +236,8 @@ __global__ void __launch_bounds__(kThreads, 4)
     if (MODE == kModeFused && !bad) {
       if (rank == 0)
         mbar_arrive_expect_tx(bar_sc, static_cast<uint32_t>(n * 4));
-      else {
+      else
         mbar_arrive_expect_tx(bar_sel, static_cast<uint32_t>(m * 4));
-        if (gated) mbar_arrive_expect_tx(bar_gb, static_cast<uint32_t>(m * G * 4));
-      }
     }
     if (do_pool) {
       mbar_arrive_expect_tx(bar_p, kPool * 4);
@@ -499,68 +496,6 @@ __global__ void __launch_bounds__(kThreads, 4)
         }
         if (p.sel_count != nullptr && tid == 0) p.sel_count[pair] = list_ok ? m : 0;
         SAS_TRACE(19);  // rank 0: list sent
-        if (gated) {
-          // this CTA's K/V copies go out first; the gates are computed while
-          // they (and the other CTAs' copies) are in flight
-          __syncthreads();
-          known = nchunks + kTilesPerBlock * cnt_mine;
-          pump(nchunks, known);
-          // gate of every list entry and head: log(sigmoid(s_gb)), s_gb =
-          // (q~_g . k~_b) * gate_scale from q~ (v, rotated in place) and the
-          // block's gate key; 0 for the current block and a stand-in list.
-          // As in the score phase: 8 lanes per key row (16 dimensions each),
-          // 4 rows per warp, two 16-row steps per round with every load of
-          // the round in flight, one 8-lane reduction per (row, head).
-          const int nh = list_ok ? m - 1 : 0;  // historical entries
-          const int grp = lane >> 3, sub = lane & 7;
-          for (int j0 = 0; j0 < nh; j0 += 32) {
-            uint4 kr[2][4];
-#pragma unroll
-            for (int v = 0; v < 2; ++v) {
-              const int j = j0 + 16 * v + 4 * warp + grp;
-#pragma unroll
-              for (int i = 0; i < 4; ++i) kr[v][i] = make_uint4(0u, 0u, 0u, 0u);
-              if (j < nh) {
-                const uint8_t* krow = gk_pair + static_cast<size_t>(sel[j]) * gk_row_bytes;
-                if (p.gk16) {
-                  kr[v][0] = *reinterpret_cast<const uint4*>(krow + 32 * sub);
-                  kr[v][1] = *reinterpret_cast<const uint4*>(krow + 32 * sub + 16);
-                } else {
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) kr[v][i] = *reinterpret_cast<const uint4*>(krow + 64 * sub + 16 * i);
-                }
-              }
-            }
-#pragma unroll
-            for (int v = 0; v < 2; ++v) {
-              const int j = j0 + 16 * v + 4 * warp + grp;
-              for (int g = 0; g < G; ++g) {
-                const float4* q4 = reinterpret_cast<const float4*>(qv + g * kDim + 16 * sub);
-                float a = 0.f;
-                if (p.gk16) {
-                  a = dot8_bf16(q4[0], q4[1], kr[v][0], a);
-                  a = dot8_bf16(q4[2], q4[3], kr[v][1], a);
-                } else {
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    const uint4 k = kr[v][i];
-                    a = dot4(q4[i], make_float4(__uint_as_float(k.x), __uint_as_float(k.y),
-                                                __uint_as_float(k.z), __uint_as_float(k.w)), a);
-                  }
-                }
-                a += __shfl_xor_sync(0xffffffffu, a, 1);
-                a += __shfl_xor_sync(0xffffffffu, a, 2);
-                a += __shfl_xor_sync(0xffffffffu, a, 4);
-                const float sg = a * p.gate_scale;
-                if (sub == 0 && j < nh) gbias[j * G + g] = (sg >= 0.f) ? -log1pf(expf(-sg)) : sg - log1pf(expf(sg));
-              }
-            }
-          }
-          for (int w = nh * G + tid; w < m * G; w += kThreads) gbias[w] = 0.f;  // current block, stand-in
-          __syncthreads();
-          for (int w = tid; w < m * G; w += kThreads)
-            for (int r = 1; r < CS; ++r) st_async_f32(dsmem_addr(gbias + w, r), gbias[w], dsmem_addr(bar_gb, r));
-        }
         issue_wk();
       } else {
         issue_wk();
@@ -573,17 +508,59 @@ __global__ void __launch_bounds__(kThreads, 4)
     // read: the current block, always valid, stands in for every entry
     if (__syncthreads_and(list_ok) == 0) {
       for (int j = tid; j < m; j += kThreads) sel[j] = c;
-      if (gated)
-        for (int w = tid; w < m * G; w += kThreads) gbias[w] = 0.f;
       __syncthreads();
     }
     known = nchunks + kTilesPerBlock * cnt_mine;
     SAS_TRACE(20);  // list in hand
     pump(nchunks, known);
-    if (gated && rank != 0 && !bad) {
-      // the gates follow the list; the K/V copies just issued overlap the wait
-      if (__syncthreads_and(mbar_wait_cluster(bar_gb, 0, p.status)) == 0) {
-        for (int w = tid; w < m * G; w += kThreads) gbias[w] = 0.f;
+    if (gated && !bad) {
+      // gated mode: each CTA computes the gates of its own list entries,
+      // log(sigmoid(s_gb)), s_gb = (q~_g . k~_b) * gate_scale, while its K/V
+      // copies are in flight; q~ (v, rotated in place) is still intact (the
+      // gated plan keeps every later region clear of it).  The current block
+      // (and a stand-in list, all entries the current block) gets 0.  As in
+      // the score phase: 8 lanes per key row (16 dimensions each), 4 rows per
+      // warp; one 8-lane reduction per (row, head).
+      const int grp = lane >> 3, sub = lane & 7;
+      for (int e0 = 0; e0 < cnt_mine; e0 += 4 * kWarps) {
+        const int e = e0 + 4 * warp + grp;
+        const bool live = e < cnt_mine;
+        const int b = live ? entry_block(e) : c;
+        uint4 kr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) kr[i] = make_uint4(0u, 0u, 0u, 0u);
+        if (b != c) {
+          const uint8_t* krow = gk_pair + static_cast<size_t>(b) * gk_row_bytes;
+          if (p.gk16) {
+            kr[0] = *reinterpret_cast<const uint4*>(krow + 32 * sub);
+            kr[1] = *reinterpret_cast<const uint4*>(krow + 32 * sub + 16);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) kr[i] = *reinterpret_cast<const uint4*>(krow + 64 * sub + 16 * i);
+          }
+        }
+        const int jg = live ? entry_index(e) * G : 0;
+        for (int g = 0; g < G; ++g) {
+          const float4* q4 = reinterpret_cast<const float4*>(qv + g * kDim + 16 * sub);
+          float a = 0.f;
+          if (p.gk16) {
+            a = dot8_bf16(q4[0], q4[1], kr[0], a);
+            a = dot8_bf16(q4[2], q4[3], kr[1], a);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const uint4 k = kr[i];
+              a = dot4(q4[i], make_float4(__uint_as_float(k.x), __uint_as_float(k.y),
+                                          __uint_as_float(k.z), __uint_as_float(k.w)), a);
+            }
+          }
+          a += __shfl_xor_sync(0xffffffffu, a, 1);
+          a += __shfl_xor_sync(0xffffffffu, a, 2);
+          a += __shfl_xor_sync(0xffffffffu, a, 4);
+          const float sg = a * p.gate_scale;
+          if (sub == 0 && live)
+            gbias[jg + g] = (b == c) ? 0.f : ((sg >= 0.f) ? -log1pf(expf(-sg)) : sg - log1pf(expf(sg)));
+        }
       }
       __syncthreads();
     }

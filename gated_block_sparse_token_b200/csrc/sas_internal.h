@@ -72,17 +72,17 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
   p.gam = take(kDim * 4, 16);
   p.gamk = take(kDim * 4, 16);
   // ring slots, prologue, pooled P, W_k slice, scores (rank 0), list, v,
-  // attention partials, pooled slices (rank 0), gates of the list
-  p.bars = take((nst + 9) * 8, 8);
+  // attention partials, pooled slices (rank 0)
+  p.bars = take((nst + 8) * 8, 8);
   auto up128 = [](int x) { return (x + 127) / 128 * 128; };
   const int r = up128(off);
   // phases 0-1 (the W_q slice is a tensor-TMA destination: 128-byte aligned)
   p.r_qv = r;
   p.r_wq = up128(r + G * kDim * 4);
   const int end01 = p.r_wq + up16(G * kDim * dpc * 2);
-  // phases 2-4
-  p.r_inbox = r;
-  p.r_pool_p = r + up16(cs * G * (dpc + 2) * 4);
+  // phases 2-4 (gated mode: clear of q~, which the gates read after the list)
+  p.r_inbox = gated ? up16(r + G * kDim * 4) : r;
+  p.r_pool_p = p.r_inbox + up16(cs * G * (dpc + 2) * 4);
   p.r_pool_u = p.r_pool_p + up16(kPool * 4);
   p.r_keys = up128(p.r_pool_u + up16(cs * 17 * 4));
   p.r_wk = p.r_keys;
