@@ -133,6 +133,11 @@ __global__ void __launch_bounds__(kThreads, 4)
   // gated mode: log-sigmoid gate of list entry j for head g at gbias[j * G + g]
   float* gbias = reinterpret_cast<float*>(base + p.sm.gbias);
   const bool gated = (MODE == kModeFused) && p.gated != 0;
+  // paged cache: rows of this CTA's list entries, looked up once in parallel
+  // when the list is in hand (the issuer then needs no page-table load per tile)
+  long long* rows_s = reinterpret_cast<long long*>(base + p.sm.rows);
+  const bool paged = p.kv.block_table != nullptr;
+  bool rows_cached = false;  // meaningful in thread 0 only
 
   // ------------------------------------------------------------ prologue copies
   // Thread 0 loads the sequence length first (one request per CTA: every CTA
@@ -189,8 +194,27 @@ __global__ void __launch_bounds__(kThreads, 4)
   const int c = err ? 0 : (L - 1) / kBlock;  // current block
   if (MODE != kModeAttend && c > p.mg) err = true;
   if (MODE == kModeFused && !err) {
-    for (int b = tid; b <= c; b += kThreads)
-      if (p.kv.block_row(s, h, b) < 0) err = true;
+    // every block 0..c must map to cache rows.  Contiguous: one bound (rows
+    // grow with the block index).  Paged: every page id of the sequence in
+    // the pool, 16 independent loads in flight per thread.
+    if (p.kv.block_table == nullptr) {
+      if (p.kv.block_row(s, h, c) < 0) err = true;
+    } else if (c >= p.kv.max_blocks_per_seq) {
+      err = true;
+    } else {
+      const int32_t* trow = p.kv.block_table + static_cast<long long>(s) * p.kv.max_blocks_per_seq;
+      for (int b0 = tid; b0 <= c; b0 += 16 * kThreads) {
+        int pg[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int b = b0 + u * kThreads;
+          pg[u] = (b <= c) ? trow[b] : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (pg[u] < 0 || pg[u] >= p.kv.num_pages) err = true;
+      }
+    }
   }
   int m = 0;  // entries of the block list (current block last)
   if (MODE == kModeAttend && !err) {
@@ -275,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     const int k = t - nchunks;
     const int e = k / kTilesPerBlock;
     const int part = k - e * kTilesPerBlock;
-    const long long row0 = p.kv.block_row(s, h, entry_block(e));
+    const long long row0 = rows_cached ? rows_s[e] : p.kv.block_row(s, h, entry_block(e));
     mbar_arrive_expect_tx(&bars[slot], kTileBytes);
     if constexpr (kF32) {
       const float* src = static_cast<const float*>(part < 2 ? p.kv.k : p.kv.v) +
@@ -513,6 +537,11 @@ __global__ void __launch_bounds__(kThreads, 4)
     known = nchunks + kTilesPerBlock * cnt_mine;
     SAS_TRACE(20);  // list in hand
     pump(nchunks, known);
+    if (paged) {
+      // every later issue follows a block-wide barrier, which publishes these
+      for (int e = tid; e < cnt_mine; e += kThreads) rows_s[e] = p.kv.block_row(s, h, entry_block(e));
+      rows_cached = true;
+    }
     if (gated && !bad) {
       // gated mode: each CTA computes the gates of its own list entries,
       // log(sigmoid(s_gb)), s_gb = (q~_g . k~_b) * gate_scale, while its K/V
@@ -950,6 +979,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 }
 
 // ------------------------------------------------------------ Top-K kernel
+template <bool kMedium>
 __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ TopkParams p) {
   const int pair = blockIdx.x;
   const int s = pair / p.hkv;
@@ -980,7 +1010,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
   const int c = (L - 1) / kBlock;
   for (int b = tid; b < c; b += kThreads) vals[b] = p.group_scores[static_cast<size_t>(pair) * p.mg + b];
   __syncthreads();
-  const int m = select_blocks(vals, c, topk, c, sel, hist, selbits, scan);
+  const int m = select_blocks<kMedium>(vals, c, topk, c, sel, hist, selbits, scan);
   for (int j = tid; j < m; j += kThreads) p.sel_idx[static_cast<size_t>(pair) * p.max_sel + j] = sel[j];
   if (tid == 0) p.sel_count[pair] = m;
 }
@@ -1062,7 +1092,10 @@ cudaError_t launch_decode(int mode, bool f32_kv, bool f32_out, int cs, int nst,
 
 cudaError_t launch_topk(const TopkParams& p, int batch, cudaStream_t stream) {
   const size_t smem = topk_smem_bytes(p.mg, p.max_sel);
-  topk_kernel<<<static_cast<unsigned>(batch * p.hkv), kThreads, smem, stream>>>(p);
+  if (p.mg > 4 * kThreads)  // more than 512 historical blocks can occur
+    topk_kernel<true><<<static_cast<unsigned>(batch * p.hkv), kThreads, smem, stream>>>(p);
+  else
+    topk_kernel<false><<<static_cast<unsigned>(batch * p.hkv), kThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -1071,7 +1104,10 @@ cudaError_t prepare_decode_kernels() {
   if ((e = attrs_for_mode<kModeGate>()) != cudaSuccess) return e;
   if ((e = attrs_for_mode<kModeAttend>()) != cudaSuccess) return e;
   if ((e = attrs_for_mode<kModeFused>()) != cudaSuccess) return e;
-  return cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if ((e = cudaFuncSetAttribute(topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024)) !=
+      cudaSuccess)
+    return e;
+  return cudaFuncSetAttribute(topk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
 }
 
 }  // namespace sas

@@ -30,6 +30,7 @@ constexpr int kSelCand = 256;   // candidates ranked exactly in the boundary buc
 struct DecodeSmem {
   int slots;     // NST stage slots of 16 KiB (gate-key chunks, then K/V tiles)
   int sel;       // int32 [max_sel] selected blocks (phases 2-3)
+  int rows;      // int64 [ceil(max_sel / CS)] cache rows of this CTA's entries (paged)
   int gbias;     // fp32 [max_sel][G] gated mode: log-sigmoid gate per entry and head
   int qraw;      // T [G][128] query as stored (bf16 or fp32), bulk copy
   int qbar;      // fp32 [128] group-mean gate query (fused mode)
@@ -65,6 +66,7 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
   mg = std::max(mg, 1);
   p.slots = take(nst * kTileBytes, 1024);
   p.sel = take(max_sel * 4, 16);
+  p.rows = take((max_sel + cs - 1) / cs * 8, 16);
   p.gbias = take(gated ? max_sel * G * 4 : 0, 16);
   p.qraw = take(G * kDim * (f32_kv ? 4 : 2), 16);
   p.qbar = take(kDim * 4, 16);

@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(kThreads) prefill_gate_query_kernel(const __gr
 
 // ------------------------------------------------------------ selection
 // grid (nblk, Hkv, B), 128 threads.
+template <bool kMedium>
 __global__ void __launch_bounds__(kThreads) prefill_select_kernel(const __grid_constant__ PrefillParams p) {
   const int i = blockIdx.x;
   const int h = blockIdx.y;
@@ -218,7 +219,7 @@ __global__ void __launch_bounds__(kThreads) prefill_select_kernel(const __grid_c
     if (b < i && sub == 0) vals[b] = acc;
   }
   __syncthreads();
-  const int m = select_blocks(vals, i, topk, i, sel, hist, selbits, scan);
+  const int m = select_blocks<kMedium>(vals, i, topk, i, sel, hist, selbits, scan);
   for (int j = tid; j < m; j += kThreads) {
     p.sel[base * p.max_sel + j] = sel[j];
     if (p.sel_out != nullptr) p.sel_out[base * p.max_sel + j] = sel[j];
@@ -635,7 +636,11 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmq, const
   }
   {
     const dim3 grid(static_cast<unsigned>(p.nblk), static_cast<unsigned>(p.hkv), static_cast<unsigned>(p.batch));
-    prefill_select_kernel<<<grid, kThreads, prefill_select_smem_bytes(p.nblk, p.max_sel), stream>>>(p);
+    const size_t smem = prefill_select_smem_bytes(p.nblk, p.max_sel);
+    if (p.nblk - 1 > 4 * kThreads)  // more than 512 historical blocks can occur
+      prefill_select_kernel<true><<<grid, kThreads, smem, stream>>>(p);
+    else
+      prefill_select_kernel<false><<<grid, kThreads, smem, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -648,7 +653,9 @@ cudaError_t prepare_prefill_kernels() {
   cudaError_t e = cudaFuncSetAttribute(prefill_gate_query_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kDim * kDim * 2 + 16);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(prefill_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  e = cudaFuncSetAttribute(prefill_select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(prefill_select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   if (e != cudaSuccess) return e;
   return cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(prefill_attn_smem_bytes(kPfMaxSel)));

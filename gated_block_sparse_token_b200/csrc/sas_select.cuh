@@ -14,32 +14,39 @@ namespace {
 #define SEL_TRACE(k, v)
 #endif
 
-// Exact Top-K of n <= 4 * kThreads scores (every decode context up to 32,768
-// tokens), the short path: each thread keeps the keys of indices
-// 4t .. 4t+3 in registers; buckets are linear in the score value between the
-// finite minimum and maximum (monotone in key order: NaN and -inf fall in
-// bucket 0, +inf in the last), so the boundary bucket holds few members; the
-// kept set is a bit mask, turned into the ascending list by one warp.
-// Requires topk >= 1 and n > topk; same result as the general path.
-__device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
-                            uint32_t* selmask, int* scan, unsigned long long* tr) {
+// Exact Top-K of n <= PER * kThreads scores, the register path (PER = 4:
+// every decode context up to 32,768 tokens; PER = 16: up to 131,072): each
+// thread keeps the keys of indices PER t .. PER t + PER - 1 in registers;
+// buckets are linear in the score value between the finite minimum and
+// maximum (monotone in key order: NaN and -inf fall in bucket 0, +inf in
+// the last), so the boundary bucket holds few members; the kept set is a bit
+// mask, turned into the ascending list by one warp.  Requires topk >= 1 and
+// n > topk; same result as the general path.
+template <int PER>
+__device__ __forceinline__ int select_regs(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
+                                           uint32_t* selmask, int* scan, unsigned long long* tr) {
+  static_assert(PER == 4 || PER == 8 || PER == 16, "4, 8 or 16 keys per thread");
+  constexpr int TPW = 32 / PER;                     // threads per 32-bit mask word
+  constexpr int WPL = (PER * kThreads / 32 + 31) / 32;  // mask words per lane of warp 0
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned full = 0xffffffffu;
   uint32_t* keys = reinterpret_cast<uint32_t*>(vals);
-  const int i0 = 4 * tid;
-  float x[4];
-  uint32_t k[4];
-  bool valid[4];
-  {
-    const float4 v = (i0 < n) ? *reinterpret_cast<const float4*>(vals + i0) : make_float4(0.f, 0.f, 0.f, 0.f);
-    x[0] = v.x;
-    x[1] = v.y;
-    x[2] = v.z;
-    x[3] = v.w;
+  const int i0 = PER * tid;
+  float x[PER];
+  uint32_t k[PER];
+  bool valid[PER];
+#pragma unroll
+  for (int q = 0; q < PER / 4; ++q) {
+    const float4 v = (i0 + 4 * q < n) ? *reinterpret_cast<const float4*>(vals + i0 + 4 * q)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    x[4 * q] = v.x;
+    x[4 * q + 1] = v.y;
+    x[4 * q + 2] = v.z;
+    x[4 * q + 3] = v.w;
   }
   float fmn = INFINITY, fmx = -INFINITY;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
+  for (int u = 0; u < PER; ++u) {
     valid[u] = (i0 + u) < n;
     k[u] = order_key(x[u]);
     if (valid[u] && isfinite(x[u])) {
@@ -47,12 +54,17 @@ __device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uin
       fmx = fmaxf(fmx, x[u]);
     }
   }
-  if (i0 + 3 < n) {
-    *reinterpret_cast<uint4*>(keys + i0) = make_uint4(k[0], k[1], k[2], k[3]);
-  } else {
+  // keys over the scores: each thread rewrites only its own range
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (valid[u]) keys[i0 + u] = k[u];
+  for (int q = 0; q < PER / 4; ++q) {
+    const int b = i0 + 4 * q;
+    if (b + 3 < n) {
+      *reinterpret_cast<uint4*>(keys + b) = make_uint4(k[4 * q], k[4 * q + 1], k[4 * q + 2], k[4 * q + 3]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (b + u < n) keys[b + u] = k[4 * q + u];
+    }
   }
   *reinterpret_cast<uint4*>(hist + 8 * tid) = make_uint4(0u, 0u, 0u, 0u);
   *reinterpret_cast<uint4*>(hist + 8 * tid + 4) = make_uint4(0u, 0u, 0u, 0u);
@@ -74,9 +86,9 @@ __device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uin
   SEL_TRACE(0, global_timer_ns());
   const float span = fmx - fmn;
   const float scale = (span > 0.f && isfinite(span)) ? static_cast<float>(kSelBins - 1) / span : 0.f;
-  int bk[4];
+  int bk[PER];
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
+  for (int u = 0; u < PER; ++u) {
     int b = 0;
     if (isfinite(x[u]))
       b = min(kSelBins - 1, static_cast<int>((x[u] - fmn) * scale));
@@ -124,21 +136,20 @@ __device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uin
   const int take = scan[9];
   SEL_TRACE(2, global_timer_ns());
 
-  // ---- kept-above bits (one 32-bit word per 8 threads) and boundary members
+  // ---- kept-above bits (one 32-bit word per TPW threads) and boundary members
   int* cand = reinterpret_cast<int*>(hist);
   uint32_t* candk = hist + kSelCand;
   {
     uint32_t bits = 0u;
     int cnt = 0;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (valid[u] && bk[u] > bstar) bits |= 1u << (4 * (tid & 7) + u);
+    for (int u = 0; u < PER; ++u) {
+      if (valid[u] && bk[u] > bstar) bits |= 1u << (PER * (tid % TPW) + u);
       cnt += (valid[u] && bk[u] == bstar) ? 1 : 0;
     }
-    bits |= __shfl_xor_sync(full, bits, 1);
-    bits |= __shfl_xor_sync(full, bits, 2);
-    bits |= __shfl_xor_sync(full, bits, 4);
-    if ((tid & 7) == 0 && (tid >> 3) < words) selmask[tid >> 3] = bits;
+#pragma unroll
+    for (int o = 1; o < TPW; o <<= 1) bits |= __shfl_xor_sync(full, bits, o);
+    if ((tid % TPW) == 0 && (tid / TPW) < words) selmask[tid / TPW] = bits;
     int inc = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -150,7 +161,7 @@ __device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uin
     base = __shfl_sync(full, base, 31);
     int pos = base + inc - cnt;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < PER; ++u) {
       if (valid[u] && bk[u] == bstar) {
         if (pos < kSelCand) {
           cand[pos] = i0 + u;
@@ -180,7 +191,7 @@ __device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uin
   } else {
     // a crowded boundary bucket (many equal scores): rank against all members
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < PER; ++u) {
       if (!(valid[u] && bk[u] == bstar)) continue;
       const int i = i0 + u;
       int r = 0;
@@ -205,10 +216,17 @@ __device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uin
   __syncthreads();
   SEL_TRACE(4, global_timer_ns());
 
-  // ---- ascending list from the mask (one warp: lane w owns word w)
+  // ---- ascending list from the mask (one warp: lane l owns words
+  // WPL l .. WPL l + WPL - 1)
   if (warp == 0) {
-    const uint32_t wmask = (lane < words) ? selmask[lane] : 0u;
-    const int c = __popc(wmask);
+    uint32_t wmask[WPL];
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < WPL; ++w) {
+      const int wi = WPL * lane + w;
+      wmask[w] = (wi < words) ? selmask[wi] : 0u;
+      c += __popc(wmask[w]);
+    }
     int inc = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -216,16 +234,31 @@ __device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uin
       if (lane >= o) inc += y;
     }
     int pos = inc - c;
-    uint32_t mm = wmask;
-    while (mm != 0u) {
-      const int b = __ffs(mm) - 1;
-      sel[pos++] = 32 * lane + b;
-      mm &= mm - 1u;
+#pragma unroll
+    for (int w = 0; w < WPL; ++w) {
+      uint32_t mm = wmask[w];
+      while (mm != 0u) {
+        const int b = __ffs(mm) - 1;
+        sel[pos++] = 32 * (WPL * lane + w) + b;
+        mm &= mm - 1u;
+      }
     }
     if (lane == 0) sel[topk] = cur;
   }
   __syncthreads();
   return topk + 1;
+}
+
+__device__ int select_small(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist, uint32_t* selmask,
+                            int* scan, unsigned long long* tr) {
+  return select_regs<4>(vals, n, topk, cur, sel, hist, selmask, scan, tr);
+}
+
+// contexts of 513 .. 2,048 blocks; out of line so that its 16 keys per
+// thread do not weigh on the registers of the kernels that inline the rest
+__device__ __noinline__ int select_medium(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
+                                          uint32_t* selmask, int* scan, unsigned long long* tr) {
+  return select_regs<16>(vals, n, topk, cur, sel, hist, selmask, scan, tr);
 }
 
 // Top-K selection, general path (pages: training Top-K 31 under the 2,048-token budget).
@@ -430,8 +463,11 @@ __device__ __noinline__ int select_large(float* vals, int n, int topk, int cur, 
 
 
 // Entry point: trivial budgets, then the short path (n <= 512) inline, the
-// general path out of line (it is rare, and keeping its code out of the
-// caller keeps the caller's instruction footprint small).
+// 16-keys-per-thread path (n <= 2,048) and the general path out of line
+// (keeping their code out of the caller keeps its instruction footprint
+// small).  kMedium = false leaves the 16-key path out, for kernels that never
+// see more than 512 blocks and should not carry its registers.
+template <bool kMedium = true>
 __device__ __forceinline__ int select_blocks(float* vals, int n, int topk, int cur, int* sel, uint32_t* hist,
                                              uint32_t* selbits, int* scan, unsigned long long* tr = nullptr) {
   const int tid = threadIdx.x;
@@ -447,6 +483,7 @@ __device__ __forceinline__ int select_blocks(float* vals, int n, int topk, int c
     return n + 1;
   }
   if (n <= 4 * kThreads) return select_small(vals, n, topk, cur, sel, hist, selbits, scan, tr);
+  if (kMedium && n <= 16 * kThreads) return select_medium(vals, n, topk, cur, sel, hist, selbits, scan, tr);
   return select_large(vals, n, topk, cur, sel, hist, selbits, scan, tr);
 }
 

@@ -269,6 +269,41 @@ def test_topk_exact_up_to_512_blocks(budget):
             assert list(sel[s, h, :len(want)]) == want, (s, h)
 
 
+@pytest.mark.parametrize("budget", [1024, 4096, 16384])
+def test_topk_exact_513_to_2048_blocks(budget):
+    """513 .. 2,048 historical blocks (contexts to 128k) take the 16-keys-per-
+    thread path, 2,049 and more the general one; ties, equal scores,
+    infinities and a span that overflows fp32 must give the full-sort rule
+    exactly on both sides of each boundary."""
+    g = torch.Generator().manual_seed(budget + 11)
+    B, hkv, mg = 5, 4, 2100
+    nblocks = [513, 1024, 1999, 2048, 2049]
+    lens = torch.tensor([64 * n + 1 for n in nblocks], dtype=torch.int32)
+    scores = torch.randn(B, hkv, mg, generator=g)
+    scores[:, 0] = torch.randint(-4, 5, (B, mg), generator=g).float() * 0.25   # 9 values, many ties
+    scores[:, 1] = -1.25                                                     # all equal
+    scores[0, 2, 3] = float("inf")
+    scores[2, 2, 50:60] = float("-inf")
+    scores[3, 2, 10] = 3.0e38
+    scores[3, 2, 11] = -3.0e38                                               # max - min overflows
+    scores[1, 3, 700:720] = 2.0                                              # a tied plateau at the top
+    cfg = sas.Config(4 * hkv, hkv, token_budget=budget)
+    ws = sas.make_workspace(cfg, DEV)
+    sel = torch.full((B, hkv, budget // 64), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.full((B, hkv), -1, dtype=torch.int32, device=DEV)
+    sas.topk_blocks(cfg, scores.to(DEV), lens.to(DEV), sel, cnt, ws)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    sel, cnt = sel.cpu().numpy(), cnt.cpu().numpy()
+    for s in range(B):
+        c = (int(lens[s]) - 1) // 64
+        assert c == nblocks[s]
+        for h in range(hkv):
+            want = O.select_blocks(scores[s, h, :c].double().numpy(), c, budget // 64 - 1)
+            assert int(cnt[s, h]) == len(want)
+            assert list(sel[s, h, :len(want)]) == want, (s, h)
+
+
 def test_sparse_decode_given_blocks():
     spec = DecodeSpec("given", 2, 8, 2, [3000, 2100], (512,), capacity=4096, seed=19)
     inp = make_decode_inputs(spec, DEV)

@@ -37,7 +37,8 @@ def test_plan_alignment_and_overlap(plans):
         assert p["slots"] % 1024 == 0 and p["r_wq"] % 128 == 0, tag
         assert p["qraw"] % 16 == 0 and p["gam"] % 16 == 0 and p["bars"] % 8 == 0, tag
         # fixed regions, in order, disjoint
-        fixed = [("slots", 2 * 16384), ("sel", 4 * ms), ("gbias", 4 * ms * G * p["gated"]),
+        fixed = [("slots", 2 * 16384), ("sel", 4 * ms), ("rows", 8 * ((ms + 7) // 8)),
+                 ("gbias", 4 * ms * G * p["gated"]),
                  ("qraw", G * 128 * (4 if p["f32"] else 2)), ("qbar", 512), ("pml", 256), ("gam", 512),
                  ("bars", 8 * (2 + 8))]
         for (a, sa), (b, _) in zip(fixed, fixed[1:]):

@@ -162,6 +162,14 @@ def test_prefill_eight_query_heads_per_kv_head():
     _check(spec, *res, [(0, 0, i) for i in range(12)])
 
 
+def test_prefill_beyond_512_blocks():
+    """33,920 tokens: query blocks past 512 historical blocks take the
+    16-keys-per-thread selection."""
+    spec = PrefillSpec("pf_530_blocks", 1, 2, 1, 64 * 530, token_budget=1024, seed=49)
+    res = _run(spec)
+    _check(spec, *res, [(0, 0, i) for i in (5, 512, 513, 520, 529)])
+
+
 def test_prefill_qwen3_8b_32k_full_size():
     spec = qwen3_8b_prefill_32k()
     res = _run(spec)
