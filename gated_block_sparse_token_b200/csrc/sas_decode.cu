@@ -118,6 +118,8 @@ __global__ void __launch_bounds__(kThreads, 4)
   uint64_t* bar_v = bars + NST + 5;   // the gate query v (a slice from each CTA)
   uint64_t* bar_m = bars + NST + 6;   // attention partials of this CTA's columns
   uint64_t* bar_u = bars + NST + 7;   // rank 0: projected pooled slices
+  uint64_t* bar_wq2 = bars + NST + 8; // second pass of the W_q slice (large groups)
+  const int wq_heads = p.sm.wq_heads;  // heads of the W_q slice resident at once
   float* pool_p = reinterpret_cast<float*>(base + p.sm.r_pool_p);
   float* pool_u = reinterpret_cast<float*>(base + p.sm.r_pool_u);
   __nv_bfloat16* wk_s = reinterpret_cast<__nv_bfloat16*>(base + p.sm.r_wk);
@@ -157,11 +159,11 @@ __global__ void __launch_bounds__(kThreads, 4)
       prefetch_tensormap(&tmv);
     }
     if (pool_on) prefetch_tensormap(&tmwk);
-    for (int i = 0; i < NST + 8; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < NST + 9; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
     const uint32_t qbytes = static_cast<uint32_t>(G * kDim * sizeof(T));
     uint32_t tx = qbytes;
-    if (MODE != kModeAttend) tx += static_cast<uint32_t>(G * kDim * kDpc * 2 + kDim * 4);
+    if (MODE != kModeAttend) tx += static_cast<uint32_t>(wq_heads * kDim * kDpc * 2 + kDim * 4);
     if (pool_on) tx += kDim * 4;
     mbar_arrive_expect_tx(bar_pro, tx);
     bulk_g2s(qraw, static_cast<const T*>(p.q) + (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim,
@@ -169,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     if (MODE != kModeAttend) bulk_g2s(gam_s, p.gamma_q, kDim * 4, bar_pro);
     if (pool_on) bulk_g2s(gamk_s, p.gamma_k, kDim * 4, bar_pro);
     if (MODE != kModeAttend) {
-      for (int g = 0; g < G; ++g)
+      for (int g = 0; g < wq_heads; ++g)
         tma_load_2d(wq_s + static_cast<size_t>(g) * kDim * kDpc, &tmw, rank * kDpc, (h * G + g) * kDim,
                     bar_pro);
     }
@@ -333,26 +335,44 @@ __global__ void __launch_bounds__(kThreads, 4)
   cluster_wait();  // every CTA of the cluster is running
   if (MODE != kModeAttend && !bad) {
     // two threads per output column (rows 0..63 and 64..127), combined by
-    // shuffle; every CTA of the cluster receives every column
-    for (int o = tid; o < 2 * G * kDpc; o += kThreads) {
-      const int half = o & 1;
-      const int oc = o >> 1;
-      const int g = oc / kDpc;
-      const int j = oc - g * kDpc;
-      const T* qrow = qraw + g * kDim + half * 64;
-      const __nv_bfloat16* wcol = wq_s + (static_cast<size_t>(g) * kDim + half * 64) * kDpc + j;
-      float a4[4] = {0.f, 0.f, 0.f, 0.f};
-      if (pro_ok) {
-#pragma unroll 16
-        for (int i = 0; i < 64; ++i)
-          a4[i & 3] = fmaf(to_float(qrow[i]), __bfloat162float(wcol[i * kDpc]), a4[i & 3]);
+    // shuffle; every CTA of the cluster receives every column.  Large groups
+    // take the W_q slice in two passes through the same region (the second
+    // copy is requested once every read of the first is done).
+    bool wq_ok = pro_ok;
+    for (int g0 = 0; g0 < G; g0 += wq_heads) {
+      const int gn = min(wq_heads, G - g0);
+      if (g0 > 0) {
+        __syncthreads();
+        if (tid == 0) {
+          fence_proxy_async_smem();  // the slice's generic reads before the async-proxy overwrite
+          mbar_arrive_expect_tx(bar_wq2, static_cast<uint32_t>(gn * kDim * kDpc * 2));
+          for (int g = 0; g < gn; ++g)
+            tma_load_2d(wq_s + static_cast<size_t>(g) * kDim * kDpc, &tmw, rank * kDpc,
+                        (h * G + g0 + g) * kDim, bar_wq2);
+        }
+        wq_ok = mbar_wait(bar_wq2, 0, p.status) && wq_ok;
       }
-      float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      if (half == 0) {
+      for (int o = tid; o < 2 * gn * kDpc; o += kThreads) {
+        const int half = o & 1;
+        const int oc = o >> 1;
+        const int gl = oc / kDpc;  // head within this pass
+        const int j = oc - gl * kDpc;
+        const int g = g0 + gl;
+        const T* qrow = qraw + g * kDim + half * 64;
+        const __nv_bfloat16* wcol = wq_s + (static_cast<size_t>(gl) * kDim + half * 64) * kDpc + j;
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (wq_ok) {
+#pragma unroll 16
+          for (int i = 0; i < 64; ++i)
+            a4[i & 3] = fmaf(to_float(qrow[i]), __bfloat162float(wcol[i * kDpc]), a4[i & 3]);
+        }
+        float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        if (half == 0) {
 #pragma unroll
-        for (int r = 0; r < CS; ++r)
-          st_async_f32(dsmem_addr(qv + g * kDim + rank * kDpc + j, r), acc, dsmem_addr(bar_v, r));
+          for (int r = 0; r < CS; ++r)
+            st_async_f32(dsmem_addr(qv + g * kDim + rank * kDpc + j, r), acc, dsmem_addr(bar_v, r));
+        }
       }
     }
     mbar_wait_cluster(bar_v, 0, p.status);  // every column of v is here

@@ -37,7 +37,8 @@ struct DecodeSmem {
   int pml;       // fp32 m[4][8], l[4][8] per-warp softmax state
   int bars;      // uint64 [NST] mbarriers
   int r_qv;      // fp32 [G][128] gate query v, then q~ in place   (phases 0-1)
-  int r_wq;      // bf16 [G][128][dpc] W_q column slice (TMA)       (phase 0)
+  int r_wq;      // bf16 [wq_heads][128][dpc] W_q column slice (TMA) (phase 0)
+  int wq_heads;  // heads of the slice resident at once (G, or ceil(G / 2): two passes)
   int gam;       // fp32 [128] gamma_q (bulk copy)
   int r_inbox;   // fp32 [CS][G][dpc] o, then [CS][G][2] (m, l)     (phases 3-4)
   int r_pool_p;  // fp32 [384] pooled current block (fused pooling)  (phases 3-4)
@@ -51,8 +52,14 @@ struct DecodeSmem {
   int total;     // bytes to request, including alignment slack
 };
 
-inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, bool f32_kv,
-                                   bool gated = false) {
+// Shared memory a CTA may take for four to fit on one SM (228 KiB per SM,
+// 1 KiB of it reserved per CTA).
+constexpr int kFourPerSmBytes = 228 * 1024 / 4 - 1024;
+
+// wq_heads: heads of the W_q slice resident at once (G: one pass; fewer:
+// phase 0 loads the slice in two passes through the same region).
+inline DecodeSmem plan_decode_smem_heads(int G, int mg, int cs, int nst, int max_sel, bool f32_kv, bool gated,
+                                         int wq_heads) {
   DecodeSmem p{};
   int off = 0;
   auto take = [&](int bytes, int align) {
@@ -64,6 +71,7 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
   auto up16 = [](int x) { return (x + 15) / 16 * 16; };
   const int dpc = kDim / cs;
   mg = std::max(mg, 1);
+  p.wq_heads = wq_heads;
   p.slots = take(nst * kTileBytes, 1024);
   p.sel = take(max_sel * 4, 16);
   p.rows = take((max_sel + cs - 1) / cs * 8, 16);
@@ -74,14 +82,14 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
   p.gam = take(kDim * 4, 16);
   p.gamk = take(kDim * 4, 16);
   // ring slots, prologue, pooled P, W_k slice, scores (rank 0), list, v,
-  // attention partials, pooled slices (rank 0)
-  p.bars = take((nst + 8) * 8, 8);
+  // attention partials, pooled slices (rank 0), second W_q pass
+  p.bars = take((nst + 9) * 8, 8);
   auto up128 = [](int x) { return (x + 127) / 128 * 128; };
   const int r = up128(off);
   // phases 0-1 (the W_q slice is a tensor-TMA destination: 128-byte aligned)
   p.r_qv = r;
   p.r_wq = up128(r + G * kDim * 4);
-  const int end01 = p.r_wq + up16(G * kDim * dpc * 2);
+  const int end01 = p.r_wq + up16(wq_heads * kDim * dpc * 2);
   // phases 2-4 (gated mode: clear of q~, which the gates read after the list)
   p.r_inbox = gated ? up16(r + G * kDim * 4) : r;
   p.r_pool_p = p.r_inbox + up16(cs * G * (dpc + 2) * 4);
@@ -94,6 +102,16 @@ inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, 
   const int end24 = std::max(p.r_scan + 16 * 4, p.r_wk + kPool * dpc * 2);
   p.total = std::max(end01, end24) + 1024;
   return p;
+}
+
+// One pass over W_q when four CTAs fit on an SM that way (or two passes
+// would not make them fit); else two passes of ceil(G / 2) heads.
+inline DecodeSmem plan_decode_smem(int G, int mg, int cs, int nst, int max_sel, bool f32_kv,
+                                   bool gated = false) {
+  const DecodeSmem one = plan_decode_smem_heads(G, mg, cs, nst, max_sel, f32_kv, gated, G);
+  if (one.total <= kFourPerSmBytes || G < 2) return one;
+  const DecodeSmem two = plan_decode_smem_heads(G, mg, cs, nst, max_sel, f32_kv, gated, (G + 1) / 2);
+  return two.total <= kFourPerSmBytes ? two : one;
 }
 
 // TMA destinations of the plan: tensor boxes need 128-byte (swizzled: 1024-

@@ -40,11 +40,11 @@ def test_plan_alignment_and_overlap(plans):
         fixed = [("slots", 2 * 16384), ("sel", 4 * ms), ("rows", 8 * ((ms + 7) // 8)),
                  ("gbias", 4 * ms * G * p["gated"]),
                  ("qraw", G * 128 * (4 if p["f32"] else 2)), ("qbar", 512), ("pml", 256), ("gam", 512),
-                 ("bars", 8 * (2 + 8))]
+                 ("bars", 8 * (2 + 9))]
         for (a, sa), (b, _) in zip(fixed, fixed[1:]):
             assert p[a] + sa <= p[b], (tag, a, b)
         r = p["r_qv"]
-        assert p["bars"] + 8 * (2 + 8) <= r, tag
+        assert p["bars"] + 8 * (2 + 9) <= r, tag
         # phase 0-1 layout: qv then the W_q slice
         qv_end = r + G * 128 * 4
         assert qv_end <= p["r_wq"], tag
@@ -61,8 +61,24 @@ def test_plan_alignment_and_overlap(plans):
         assert p["r_hist"] >= p["r_keys"] + 4 * mg, tag
         assert p["r_selbits"] >= p["r_hist"] + 4 * 1024, tag
         assert p["r_scan"] >= p["r_selbits"] + 4 * ((mg + 31) // 32), tag
-        end = max(p["r_wq"] + G * 128 * dpc * 2, p["r_scan"] + 64)
+        assert p["wq_heads"] in (G, (G + 1) // 2), tag
+        end = max(p["r_wq"] + p["wq_heads"] * 128 * dpc * 2, p["r_scan"] + 64)
         assert p["total"] >= end + 1024, tag
+
+
+def test_w_q_in_two_passes_only_where_it_buys_the_fourth_cta(plans):
+    four = 228 * 1024 // 4 - 1024
+    for p in plans:
+        if p["wq_heads"] < p["G"]:
+            assert p["total"] <= four, p
+    # Qwen3-14B, 128k context: G = 5, 2,048 gate-key rows, budget 4,096, bf16
+    p = next(q for q in plans if q["G"] == 5 and q["mg"] == 2048 and q["budget"] == 4096 and q["f32"] == 0
+             and q["gated"] == 0)
+    assert p["wq_heads"] == 3 and p["total"] <= four, p
+    # Qwen3-4B, 32k: one pass
+    p = next(q for q in plans if q["G"] == 4 and q["mg"] == 512 and q["budget"] == 2048 and q["f32"] == 0
+             and q["gated"] == 0)
+    assert p["wq_heads"] == 4, p
 
 
 def test_plan_fits_four_ctas_per_sm_at_the_benchmark_shape(plans):
