@@ -279,6 +279,9 @@ size_t prefill_attn_smem_bytes(int max_sel) {
   } while (0)
 #endif
 
+// kGated: the gated mode (a separate instance, so that the select-only
+// softmax loop carries no gate load)
+template <bool kGated>
 __global__ void __launch_bounds__(kPfAttnThreads, 2)
     prefill_attn_kernel(const __grid_constant__ PrefillParams p,
                         const __grid_constant__ CUtensorMap tmq,
@@ -448,7 +451,7 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
     const int t = r & 63;
     const uint32_t tl = tmem + (static_cast<uint32_t>(32 * warp) << 16);
     float m_run = -INFINITY, l_run = 0.f;  // running maximum in log2 units, row sum
-    if (p.gated && m > 0) {
+    if (kGated && m > 0) {
       // gated mode: gate log(sigmoid(q~_g(i) . k~_b * gate_scale)) of every kept
       // historical block b for the CTA's two heads, computed while the first
       // Q / K copies and S tile are in flight.  Eight lanes per block (16
@@ -538,7 +541,7 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
         mx1 = fmax3(mx1, sv[j + 2], sv[j + 3]);
       }
       // gated mode: + the block's gate for this row's head, in log2 units
-      const float beta2 = p.gated ? gb_s[2 * e + (r >> 6)] * kLog2e : 0.f;
+      const float beta2 = kGated ? gb_s[2 * e + (r >> 6)] * kLog2e : 0.f;
       const float mx = fmaf(fmax3(mx0, mx1, fmaxf(sv[62], sv[63])), sl2, beta2);
       const float m_new = fmaxf(m_run, mx);
       // rescale O only when the running maximum grows by more than 2^8:
@@ -645,7 +648,11 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmq, const
     if (e != cudaSuccess) return e;
   }
   const unsigned ctas = static_cast<unsigned>(p.batch) * p.hkv * p.nblk * (p.G / 2);
-  prefill_attn_kernel<<<ctas, kPfAttnThreads, prefill_attn_smem_bytes(p.max_sel), stream>>>(p, tmq, tmk, tmv);
+  const size_t smem = prefill_attn_smem_bytes(p.max_sel);
+  if (p.gated)
+    prefill_attn_kernel<true><<<ctas, kPfAttnThreads, smem, stream>>>(p, tmq, tmk, tmv);
+  else
+    prefill_attn_kernel<false><<<ctas, kPfAttnThreads, smem, stream>>>(p, tmq, tmk, tmv);
   return cudaGetLastError();
 }
 
@@ -657,7 +664,10 @@ cudaError_t prepare_prefill_kernels() {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(prefill_select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(prefill_attn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(prefill_attn_smem_bytes(kPfMaxSel)));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(prefill_attn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(prefill_attn_smem_bytes(kPfMaxSel)));
 }
 
