@@ -33,6 +33,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -301,16 +302,24 @@ def run_prefill(args, device, world):
 
 
 # the sources the fused decode kernel is built and launched from (its ncu
-# counters stay valid while none of these changes)
+# counters stay valid while the code in these does not change)
 DECODE_SOURCES = ("sas_api.cu", "sas_decode.cu", "sas_device.cuh", "sas_internal.h", "sas_select.cuh")
+
+
+def code_only(text):
+    """C++ source without its comments, trailing blanks and empty lines, so
+    that a comment edit leaves the digest alone."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines())
+    return "\n".join(ln for ln in lines if ln)
 
 
 def source_digest():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_block_sparse_token_b200", "csrc")
     for f in DECODE_SOURCES:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(csrc, f)) as fh:
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -12,25 +12,33 @@
 //
 // Work split of one cluster of CS CTAs (128 threads each) for (s, h):
 //   start    every load that does not depend on the sequence length (q, the
-//            CTA's W_q column slice, gains, RoPE frequencies) is issued first.
+//            CTA's W_q column slice, gains, RoPE frequencies) is issued first;
+//            then the length, and for a paged cache every page id of the
+//            sequence, is validated.
 //   phase 0  each CTA computes 128/CS columns of v_g = q_g @ W_q[g] for the G
-//            query heads of the group and stores them into every CTA of the
-//            cluster (distributed shared memory); RMSNorm + RoPE -> q~_g.
+//            query heads of the group (large groups: the W_q slice in two
+//            passes of ceil(G/2) heads) and stores them into every CTA of the
+//            cluster (st.async into distributed shared memory, bytes counted
+//            on the receiver's mbarrier); RMSNorm + RoPE -> q~_g.
 //   phase 1  each CTA streams 1/CS of the gate keys k~_b (TMA bulk copies
 //            into a ring of 16 KiB stage slots), scores its blocks and stores
-//            each score into every CTA of the cluster.
-//   phase 2  every CTA runs the same exact selection on the full score list
-//            (value buckets, exact ranking inside the boundary bucket, ties to
-//            the lower index), so all CTAs hold the same ascending block list.
+//            each score into CTA 0.
+//   phase 2  CTA 0 runs the exact selection once for the cluster (value
+//            buckets, exact ranking inside the boundary bucket, ties to the
+//            lower index) and sends the ascending block list to the others.
+//            Gated mode: each CTA then computes the gates of its own entries.
 //   phase 3  CTA r attends to list entries j = r (mod CS): K and V tiles come
 //            in by 2-D TMA (128-byte swizzle); each warp runs flash-decoding
 //            over 16 tokens of every tile on bf16 mma.sync (the GQA group as
 //            the M=16 rows, fp32 accumulate, online softmax).
 //   phase 4  each CTA folds its 4 warps' partials (m, l, o) and stores the
-//            128/CS-column slices into the owning CTAs; after one cluster
-//            barrier CTA r merges the CS partials of its columns locally.
+//            128/CS-column slices into the owning CTAs (st.async, counted on
+//            the owner's barrier); CTA r merges the CS partials of its columns
+//            once all have arrived.
 // The CTA that owns the current block (always selected) prefetches its
-// tiles before the selection finishes.
+// tiles before the selection finishes and, when the decoded token completes
+// the block, pools it into the block's gate key.  No cluster barrier follows
+// the start, and every wait is bounded.
 #include <cooperative_groups.h>
 
 #include <type_traits>

@@ -43,3 +43,12 @@ def test_prefill_flops_qwen3_8b_32k():
     pairs = sum(min(31, i) + 1 for i in range(512))
     assert pairs == 15_888
     assert bench.prefill_flops(512, 32, 8, 2048, 4) == 4 * 32 * 15_888 * 4 * 64 * 64 * 128
+
+
+def test_traffic_digest_ignores_comments_but_not_code():
+    src = "int f(int x) {  // doubles\n  /* the\n     rule */\n  return 2 * x;\n}\n"
+    base = bench.code_only(src)
+    assert base == "int f(int x) {\n  return 2 * x;\n}"
+    assert bench.code_only(src.replace("doubles", "twice")) == base
+    assert bench.code_only("\n\n" + src.replace("/* the", "/* a")) == base
+    assert bench.code_only(src.replace("2 * x", "3 * x")) != base
