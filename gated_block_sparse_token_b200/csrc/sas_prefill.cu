@@ -7,15 +7,20 @@
 // sequence and every KV head h,
 //   q~_g = RoPE(RMSNorm(mean_t q_{g,t} @ W_q[g]) * gamma_q, i)   (g in the group)
 //   S_b  = mean_g(q~_g . k~_b) * gate_scale                    (b < i)
-//   keep the min(topk, i) blocks of largest S_b (ties: lower index) + block i;
-//   token t of block i attends to every token of the kept blocks and to the
-//   tokens of block i up to t (causal).
+//   keep the min(topk_s, i) blocks of largest S_b (ties: lower index) + block
+//   i, topk_s = budget_s / 64 - 1 (one budget per sequence, or the
+//   configured one); token t of block i attends to every token of the kept
+//   blocks and to the tokens of block i up to t (causal); gated mode: the
+//   logits of a kept historical block b for head g get + log(sigmoid(s_gb)),
+//   s_gb = q~_g . k~_b * gate_scale.
 //
 // Kernels:
 //   prefill_gate_query_kernel  q~ for every (sequence, query head, block):
-//                              W_q[g] staged in shared memory once per CTA.
+//                              W_q[g] staged in shared memory once per CTA,
+//                              16 blocks projected at once.
 //   prefill_select_kernel      scores and exact Top-K per (seq, head, block).
-//   prefill_attn_kernel        tcgen05 block-sparse attention: one CTA per
+//   prefill_attn_kernel        tcgen05 block-sparse attention (gated mode: a
+//                              second instance): one CTA per
 //                              (seq, KV head, query block, pair of query
 //                              heads); the 128 query rows (2 heads x 64
 //                              tokens) are the M dimension of
