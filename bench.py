@@ -514,12 +514,37 @@ def run_variant(args, rank, world, device, name, gate_mode=0, budgets=None, gk16
                          "bytes_per_launch": dbytes, "avg_launch_us": round(dec_s * 1e6, 3)}}
 
 
-def cpu_baseline(seconds):
+def cpu_baseline(seconds, all_cores_workers=None):
     """The oracle as it stands, single-threaded, on a bounded sample of the
-    workload: decode steps of individual (sequence, KV head) pairs."""
+    workload: decode steps of individual (sequence, KV head) pairs; plus the
+    same over the host's cores (independent pairs in spawned processes)."""
     r = reference_sample(seconds_budget=seconds)
-    return {"value": r["value"], "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": r["sample"]}
+    out = {"value": r["value"], "unit": UNIT, "cores": 1, "kind": "oracle", "sample": r["sample"]}
+    if all_cores_workers != 0:
+        out["all_cores"] = cpu_baseline_all_cores(seconds, all_cores_workers)
+    return out
+
+
+def _oracle_worker(job):
+    seconds, h = job
+    r = reference_sample(seconds_budget=seconds, heads=(h,))
+    return r["pairs"], r["elapsed"]
+
+
+def cpu_baseline_all_cores(seconds, workers=None, max_workers=32):
+    """Oracle decode steps on every host core at once: one spawned process per
+    core (at most max_workers, each ~0.3 GB), each timing its own KV head's
+    pairs single-threaded; steps/s = pairs per second over all of them / 64.
+    Runs before any CUDA use of the parent process."""
+    import multiprocessing as mp
+    n = workers or min(os.cpu_count() or 1, max_workers)
+    with mp.get_context("spawn").Pool(n) as pool:
+        res = pool.map(_oracle_worker, [(seconds, i % HKV) for i in range(n)])
+    rate = sum(p / e for p, e in res)
+    pairs = sum(p for p, _ in res)
+    return {"value": rate / (BATCH * HKV), "unit": UNIT, "cores": n, "kind": "oracle",
+            "sample": f"{pairs} (sequence, KV head) decode steps in {n} processes of {seconds:.0f} s each, "
+                      f"1 thread each; a full step is {BATCH * HKV} pairs"}
 
 
 def run_ours(args):
@@ -639,10 +664,11 @@ def run_ours(args):
 
 
 # ---------------------------------------------------------------- reference arm (CPU oracle)
-def reference_sample(seconds_budget=None, steps=None):
+def reference_sample(seconds_budget=None, steps=None, heads=None):
     """Time oracle decode steps of single (sequence, KV head) pairs of the
     workload (gate keys of the historical blocks precomputed by the oracle,
-    untimed; the step pools the current block, gates, selects and attends)."""
+    untimed; the step pools the current block, gates, selects and attends).
+    heads: the KV heads to take turns over (all by default)."""
     import numpy as np
     import torch
     from threadpoolctl import threadpool_limits
@@ -660,7 +686,7 @@ def reference_sample(seconds_budget=None, steps=None):
     ones = np.ones(128)
     c = (CTX - 1) // 64
     pairs = []
-    for h in range(HKV):
+    for h in (range(HKV) if heads is None else heads):
         ks, vs = logical_kv(inp, 0, h, CTX)
         keys = O.gate_keys_for_sequence(ks, c, wk[h], ones)
         pairs.append((h, ks, vs, keys))
@@ -668,7 +694,7 @@ def reference_sample(seconds_budget=None, steps=None):
     t0 = time.perf_counter()
     with threadpool_limits(limits=1):
         while True:
-            h, ks, vs, keys = pairs[done % HKV]
+            h, ks, vs, keys = pairs[done % len(pairs)]
             O.gate_key(O.pool_block(ks[64 * c:64 * c + 64]), wk[h], ones, c)
             O.decode_one_group(q[0, h * G:(h + 1) * G], ks, vs, CTX, keys, wq[h * G:(h + 1) * G],
                                np.tile(ones, (G, 1)), BUDGET)

@@ -52,3 +52,9 @@ def test_traffic_digest_ignores_comments_but_not_code():
     assert bench.code_only(src.replace("doubles", "twice")) == base
     assert bench.code_only("\n\n" + src.replace("/* the", "/* a")) == base
     assert bench.code_only(src.replace("2 * x", "3 * x")) != base
+
+
+def test_all_cores_oracle_baseline_runs_in_spawned_processes():
+    r = bench.cpu_baseline_all_cores(0.3, workers=2)
+    assert r["cores"] == 2 and r["kind"] == "oracle" and r["value"] > 0
+    assert "2 processes" in r["sample"]
