@@ -87,3 +87,20 @@ def test_plan_fits_four_ctas_per_sm_at_the_benchmark_shape(plans):
         p = next(q for q in plans if q["G"] == 4 and q["mg"] == 512 and q["budget"] == 2048 and q["f32"] == 0
                  and q["gated"] == gated)
         assert 4 * (p["total"] + 1024) <= 228 * 1024
+
+
+def test_prefill_attention_keeps_two_ctas_per_sm():
+    """The block list and its gates sit beside the Q tile and the K/V rings:
+    at every accepted list length (budgets to 4,096 tokens) two CTAs of the
+    tcgen05 attention kernel must still fit in an SM's 228 KiB (1 KiB of it
+    reserved per CTA)."""
+    with tempfile.TemporaryDirectory() as d:
+        exe = os.path.join(d, "prefill_plan_check")
+        subprocess.run(["/usr/local/cuda/bin/nvcc", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+                        "-I", CSRC, "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "native", "prefill_plan_check.cu"), "-o", exe],
+                       check=True, capture_output=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    sizes = [int(line.split("bytes=")[1]) for line in out.splitlines()]
+    assert len(sizes) == 64
+    assert all(2 * (b + 1024) <= 228 * 1024 for b in sizes), max(sizes)
