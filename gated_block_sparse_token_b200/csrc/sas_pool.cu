@@ -1,7 +1,7 @@
 // SAS key-block pooling and gate keys.
 //
-// Method (release pages, "key block pooling max + min + average", "Q/K
-// normalization enabled", "gate RoPE enabled", gate hidden size 128): for a
+// Method (release pages: keys pooled per block by max, min and average, Q/K
+// normalisation and gate RoPE on, gate hidden size 128): for a
 // complete 64-token block b of (sequence s, KV head h)
 //   P_b  = [max_j K_j ; min_j K_j ; mean_j K_j]          (384 = 3 x 128)
 //   k~_b = RoPE(RMSNorm(P_b @ W_k[h]) * gamma_k, position b)

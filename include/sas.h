@@ -88,8 +88,9 @@ typedef enum { SAS_DTYPE_BF16 = 0, SAS_DTYPE_F32 = 1 } sas_dtype;
  *   SAS_GATE_LOGSIGMOID_BIAS: the attention logits of every token of a
  *     selected historical block b, for query head g, get + log(sigmoid(s_gb)),
  *     s_gb = (q~_g . k~_b) * gate_scale the head's gate score; the current
- *     block gets 0.  One plain reading of the pages' "continuous gates act on
- *     the selected blocks" (aigc.news release paragraph of 2026-09-14). */
+ *     block gets 0.  One plain reading of the continuous gates that the
+ *     pages say weight the selected blocks (aigc.news release paragraph of
+ *     2026-09-14). */
 typedef enum { SAS_GATE_SELECT_ONLY = 0, SAS_GATE_LOGSIGMOID_BIAS = 1 } sas_gate_mode;
 
 typedef struct {
@@ -162,8 +163,8 @@ SAS_API const char* sas_status_string(sas_status s);
 SAS_API int32_t sas_abi_version(void);
 
 /*
- * Pooling and gate keys (pages: "key block pooling max + min + average",
- * "Q/K normalization", "gate RoPE"; gate hidden 128).
+ * Pooling and gate keys (pages: keys pooled per block by max, min and
+ * average; Q/K normalisation and gate RoPE on; gate hidden size 128).
  *
  * For each sequence s and KV head h, pools blocks
  *   b = blk_begin[s] .. blk_begin[s] + num_blocks - 1
@@ -185,8 +186,8 @@ SAS_API sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv,
                          sas_stream_t stream);
 
 /*
- * Gate scores of every historical block (pages: gate "learns to rank and
- * select KV blocks"; query projection Qproj).
+ * Gate scores of every historical block (pages: the gate ranks the KV
+ * blocks so that the best can be selected; query projection Qproj).
  *   q            kv_dtype [B][Hq][128]  query of token L_s - 1
  *   w_q          bf16 [Hq][128][128]    gamma_q fp32 [128]
  *   gate_keys    fp32 [B][Hkv][MG][128] (from sas_pool_keys)

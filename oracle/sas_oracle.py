@@ -60,8 +60,8 @@ R12 Inference weights every selected block 1 (the continuous gate is the
 R13 Prefill gate query for query block i is the mean over the block's 64
     token queries, per query head.
 R14 Attention logits use scale 1/sqrt(128); softmax in float64.
-R18 Gated inference mode (a variant of R12; "continuous gates act on the
-    selected blocks", [aigc-0914] release paragraph): the logits of every
+R18 Gated inference mode (a variant of R12; the release paragraph of
+    [aigc-0914] has continuous gates on the chosen blocks): the logits of every
     token of a selected historical block b, for query head g, get the
     additive bias log(sigmoid(s_{g,b})) with s_{g,b} the head's gate score
     (R7); the current block gets 0.  Gates equal to 1 reduce it to R12.
@@ -162,8 +162,9 @@ def gate_keys_for_sequence(k_seq: np.ndarray, num_blocks: int, w_k: np.ndarray,
 
 
 # --------------------------------------------------------------------------
-# Steps 2-3: gate scores and Top-K selection ([aigc-0914] "learns to rank
-# and select KV blocks", training Top-K 31, budget 2,048; [nedoborov] list).
+# Steps 2-3: gate scores and Top-K selection ([aigc-0914]: the gate ranks
+# the KV blocks and the best are kept, training Top-K 31, budget 2,048;
+# [nedoborov] list).
 # --------------------------------------------------------------------------
 def gate_scores(q_group: np.ndarray, w_q_group: np.ndarray, gamma_q_group: np.ndarray,
                 gate_keys: np.ndarray, n_hist: int, q_pos: int,
