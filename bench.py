@@ -718,7 +718,9 @@ def run_reference(args):
         return
     warm = reference_sample(steps=max(1, min(args.warmup, 3)))
     del warm
-    r = reference_sample(steps=args.steps)
+    # K (sequence, KV head) samples, or as many as fit in 150 s: the run stays
+    # within a few minutes whatever K the caller picks
+    r = reference_sample(steps=args.steps, seconds_budget=150.0)
     value = r["value"]
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
