@@ -20,6 +20,17 @@ def test_decode_bytes_qwen3_4b_32k():
     assert bench.decode_bytes([32768] * 8, 32, 8, 2048) == want
 
 
+def test_decode_bytes_qwen3_14b_paged_128k():
+    """Batch 16, 40/8 heads, 131,072 tokens, budget 4,096: per (sequence, KV
+    head) 63 historical blocks plus the full current block (64 tokens) of K
+    and V, 2,047 fp32 gate keys, q and out of 5 heads, the new gate key (the
+    token completes block 2,047); per launch W_q of 40 heads and W_k of 8."""
+    per_pair = 64 * 64 * 128 * 2 * 2 + 2047 * 128 * 4 + 2 * 5 * 128 * 2 + 128 * 4
+    want = 16 * 8 * per_pair + 40 * 128 * 128 * 2 + 8 * 384 * 128 * 2
+    assert want == 405_078_016
+    assert bench.decode_bytes([131072] * 16, 40, 8, 4096) == want
+
+
 def test_decode_bytes_bf16_keys_and_mixed_budgets():
     per_pair16 = 32 * 64 * 128 * 4 + 511 * 128 * 2 + 2 * 4 * 128 * 2 + 128 * 2
     assert bench.decode_bytes([32768] * 8, 32, 8, 2048, gk_elem=2) == \
