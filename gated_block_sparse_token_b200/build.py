@@ -9,6 +9,7 @@ so loading the library needs no GPU and no libcuda.
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
@@ -36,14 +37,21 @@ def build(force: bool = False, verbose: bool = False, trace: bool = False) -> st
         return lib
     bdir = os.path.join(ROOT, "_build", "trace" if trace else "release")
     os.makedirs(bdir, exist_ok=True)
-    objs = []
+    objs, cmds = [], []
     for src in SOURCES:
         obj = os.path.join(bdir, src.replace(".cu", ".o"))
         cmd = [NVCC] + FLAGS + (["-DSAS_PHASE_TRACE"] if trace else []) + ["-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
-        subprocess.run(cmd, check=True)
+        cmds.append(cmd)
         objs.append(obj)
+    # the translation units compile independently: run them side by side
+    with ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 1)) as ex:
+        for r in ex.map(lambda c: subprocess.run(c, capture_output=True, text=True), cmds):
+            if verbose or r.returncode != 0:
+                sys.stderr.write(r.stdout + r.stderr)
+            if r.returncode != 0:
+                raise subprocess.CalledProcessError(r.returncode, r.args)
     tmp = lib + ".tmp"
     subprocess.run([NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp] + objs
                    + ["-cudart", "static"], check=True)

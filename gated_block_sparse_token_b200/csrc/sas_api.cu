@@ -386,16 +386,20 @@ sas_status sas_topk_blocks(const sas_config* cfg, const float* group_scores,
   return launch_result(sas::launch_topk(p, batch, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-static sas_status attention_call(int mode, const sas_config* cfg, const void* q, const sas_kv* kv,
-                                 const void* w_q, const float* gamma_q, const void* w_k,
-                                 const float* gamma_k, void* gate_keys, int32_t max_gate_blocks,
-                                 void* out, int32_t* sel_idx, int32_t* sel_count,
-                                 float* group_scores, void* ws, size_t ws_bytes,
-                                 sas_stream_t stream) {
+// Host checks of a decode-attention call (everything attention_call checks
+// before it enqueues anything).  *launch is false when there is nothing to do.
+static sas_status check_attention_args(int mode, const sas_config* cfg, const void* q,
+                                       const sas_kv* kv, const void* w_q, const float* gamma_q,
+                                       const void* w_k, const float* gamma_k,
+                                       const void* gate_keys, int32_t max_gate_blocks,
+                                       const void* out, const int32_t* sel_idx,
+                                       const int32_t* sel_count, const float* group_scores,
+                                       const void* ws, size_t ws_bytes, bool* launch) {
+  *launch = false;
   sas_status st = check_config(cfg);
   if (st != SAS_OK) return st;
   if ((st = check_kv(cfg, kv)) != SAS_OK) return st;
-  if ((st = check_ws(cfg, ws, ws_bytes)) != SAS_OK) return st;
+  if ((st = check_ws(cfg, const_cast<void*>(ws), ws_bytes)) != SAS_OK) return st;
   if (kv->batch == 0) return SAS_OK;
   if (q == nullptr || out == nullptr || !aligned(q, 16) || !aligned(out, 4)) return SAS_ERR_INVALID_ARG;
   if (mode == sas::kModeFused) {
@@ -415,10 +419,28 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
     max_gate_blocks = 1;
   }
   if (static_cast<long long>(kv->batch) * cfg->num_kv_heads > 65535) return SAS_ERR_UNSUPPORTED;
-  if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
   sas::DecodeParams p{};
   fill_common(p, cfg, max_gate_blocks);
   if (!plan_ok(p)) return SAS_ERR_UNSUPPORTED;
+  *launch = true;
+  return SAS_OK;
+}
+
+static sas_status attention_call(int mode, const sas_config* cfg, const void* q, const sas_kv* kv,
+                                 const void* w_q, const float* gamma_q, const void* w_k,
+                                 const float* gamma_k, void* gate_keys, int32_t max_gate_blocks,
+                                 void* out, int32_t* sel_idx, int32_t* sel_count,
+                                 float* group_scores, void* ws, size_t ws_bytes,
+                                 sas_stream_t stream) {
+  bool launch = false;
+  sas_status st = check_attention_args(mode, cfg, q, kv, w_q, gamma_q, w_k, gamma_k, gate_keys,
+                                       max_gate_blocks, out, sel_idx, sel_count, group_scores, ws,
+                                       ws_bytes, &launch);
+  if (st != SAS_OK || !launch) return st;
+  if (mode != sas::kModeFused) max_gate_blocks = 1;
+  if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
+  sas::DecodeParams p{};
+  fill_common(p, cfg, max_gate_blocks);
   p.q = q;
   p.w_q = static_cast<const __nv_bfloat16*>(w_q);
   p.gamma_q = gamma_q;
@@ -559,6 +581,23 @@ sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const sas_kv*
                         0, out, const_cast<int32_t*>(sel_idx), const_cast<int32_t*>(sel_count),
                         nullptr, ws, ws_bytes, stream);
 }
+
+}  // extern "C"
+
+namespace sas {
+sas_status check_decode_step_args(const sas_config* cfg, const void* q, const sas_kv* kv,
+                                  const void* w_q, const float* gamma_q, const void* w_k,
+                                  const float* gamma_k, const void* gate_keys,
+                                  int32_t max_gate_blocks, const void* out, const int32_t* sel_idx,
+                                  const int32_t* sel_count, const float* group_scores,
+                                  const void* ws, size_t ws_bytes, bool* launch) {
+  return check_attention_args(kModeFused, cfg, q, kv, w_q, gamma_q, w_k, gamma_k, gate_keys,
+                              max_gate_blocks, out, sel_idx, sel_count, group_scores, ws, ws_bytes,
+                              launch);
+}
+}  // namespace sas
+
+extern "C" {
 
 sas_status sas_decode_step(const sas_config* cfg, const void* q, const sas_kv* kv, const void* w_q,
                            const float* gamma_q, const void* w_k, const float* gamma_k,

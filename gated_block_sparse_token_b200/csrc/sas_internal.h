@@ -222,3 +222,19 @@ size_t prefill_attn_smem_bytes(int max_sel);
 cudaError_t prepare_kernels();
 
 }  // namespace sas
+
+#include "sas.h"
+
+namespace sas {
+
+// Every host check sas_decode_step makes before it enqueues anything (the
+// workspace check against ws / ws_bytes included); *launch is false when the
+// call has nothing to do (batch 0).
+sas_status check_decode_step_args(const sas_config* cfg, const void* q, const sas_kv* kv,
+                                  const void* w_q, const float* gamma_q, const void* w_k,
+                                  const float* gamma_k, const void* gate_keys,
+                                  int32_t max_gate_blocks, const void* out, const int32_t* sel_idx,
+                                  const int32_t* sel_count, const float* group_scores,
+                                  const void* ws, size_t ws_bytes, bool* launch);
+
+}  // namespace sas

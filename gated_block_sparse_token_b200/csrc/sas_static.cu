@@ -29,11 +29,39 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
+// Driver calls that identify the current context (looked up through the
+// runtime, like the library's other driver entry points).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
 std::mutex g_scratch_mu;
+std::once_flag g_ctx_fn_once;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+// per device: the context the address was looked up in, and the address
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_decode_scratch on the current device, looked up once per
-// device (the host-side symbol is only a stand-in, never a device address).
+void load_ctx_fns() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q) ==
+          cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+  fn = nullptr;
+  if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) ==
+          cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(fn);
+  (void)cudaGetLastError();
+}
+
+// Device address of g_decode_scratch in the current device's context.  The
+// host-side symbol is only a stand-in, never a device address.  The address
+// is looked up once per device and looked up again when the device's context
+// has changed since (after cudaDeviceReset the module is loaded anew and the
+// array may sit elsewhere).
 sas_status scratch_for_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -41,15 +69,29 @@ sas_status scratch_for_current_device(void** out) {
     return SAS_ERR_CUDA;
   }
   if (dev < 0 || dev >= kMaxDevices) return SAS_ERR_UNSUPPORTED;
+  std::call_once(g_ctx_fn_once, load_ctx_fns);
+  if (g_ctx_get_current == nullptr || g_ctx_get_id == nullptr) return SAS_ERR_CUDA;
+  // id of the current context; 0 while none is bound yet (first call)
+  auto current_ctx_id = [](unsigned long long* id) -> bool {
+    CUcontext ctx = nullptr;
+    *id = 0;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return false;
+    return ctx == nullptr || g_ctx_get_id(ctx, id) == CUDA_SUCCESS;
+  };
+  unsigned long long ctx_id = 0;
+  if (!current_ctx_id(&ctx_id)) return SAS_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (ctx_id == 0 || g_scratch_addr[dev] == nullptr || g_scratch_ctx[dev] != ctx_id) {
     void* p = nullptr;
+    // binds (or creates) the device's primary context if none is current
     const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess || p == nullptr) {
       (void)cudaGetLastError();
       return SAS_ERR_CUDA;
     }
+    if (!current_ctx_id(&ctx_id) || ctx_id == 0) return SAS_ERR_CUDA;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = ctx_id;
   }
   *out = g_scratch_addr[dev];
   return SAS_OK;
@@ -69,18 +111,27 @@ extern "C" sas_status sas_decode_step_static(const sas_config* cfg, const void* 
   if (sas_workspace_bytes(cfg, kv->batch, 0) > kStaticScratchBytes) return SAS_ERR_WORKSPACE;
   if (status_out != nullptr && (reinterpret_cast<uintptr_t>(status_out) % 4) != 0)
     return SAS_ERR_INVALID_ARG;
-  void* scratch = nullptr;
-  sas_status st = scratch_for_current_device(&scratch);
+  // every host check of the step first (any 256-aligned stand-in passes the
+  // workspace check), so that a refused call enqueues nothing at all
+  bool launch = false;
+  sas_status st = sas::check_decode_step_args(
+      cfg, q, kv, w_q, gamma_q, w_k, gamma_k, gate_keys, max_gate_blocks, out, sel_idx, sel_count,
+      group_scores, reinterpret_cast<const void*>(static_cast<uintptr_t>(256)), kStaticScratchBytes,
+      &launch);
   if (st != SAS_OK) return st;
+  void* scratch = nullptr;
+  if ((st = scratch_for_current_device(&scratch)) != SAS_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // the array keeps the last call's contents: the status word starts at zero
   if (cudaMemsetAsync(scratch, 0, sizeof(uint32_t), s) != cudaSuccess) {
     (void)cudaGetLastError();
     return SAS_ERR_CUDA;
   }
-  st = sas_decode_step(cfg, q, kv, w_q, gamma_q, w_k, gamma_k, gate_keys, max_gate_blocks, out,
-                       sel_idx, sel_count, group_scores, scratch, kStaticScratchBytes, stream);
-  if (st != SAS_OK) return st;
+  if (launch) {
+    st = sas_decode_step(cfg, q, kv, w_q, gamma_q, w_k, gamma_k, gate_keys, max_gate_blocks, out,
+                         sel_idx, sel_count, group_scores, scratch, kStaticScratchBytes, stream);
+    if (st != SAS_OK) return st;
+  }
   if (status_out != nullptr &&
       cudaMemcpyAsync(status_out, scratch, sizeof(uint32_t), cudaMemcpyDeviceToDevice, s) !=
           cudaSuccess) {

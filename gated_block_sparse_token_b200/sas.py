@@ -255,9 +255,9 @@ def decode_step_static(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out
                        sel_count=None, group_scores=None, w_k=None, gamma_k=None, status_out=None,
                        stream=None) -> None:
     """sas_decode_step_static: the same step with no workspace argument, for
-    _check_gk(cfg, gate_keys)
     callers that cannot allocate; status_out (optional device uint32/int32
     tensor) receives the call's status bits."""
+    _check_gk(cfg, gate_keys)
     c, k = cfg.c(), kv.c()
     _check(lib().sas_decode_step_static(ctypes.byref(c), _ptr(q), ctypes.byref(k), _ptr(w_q),
                                         _ptr(gamma_q), _ptr(w_k), _ptr(gamma_k), _ptr(gate_keys),

@@ -13,7 +13,10 @@ layout, plus, when ``block_offset_std`` > 0, a per-(seq, head, block) offset
 vector N(0, std^2) added to all 64 tokens of the block (K's offsets drawn
 right after K, V's after V); paged caches take a random permutation of the
 page ids as block table; W_q ~ N(0, 1/128) [Hq][128][128] and W_k ~
-N(0, 1/384) [Hkv][384][128], rounded to bf16; gains gamma_q = gamma_k = 1.
+N(0, 1/384) [Hkv][384][128], rounded to bf16; then the RMSNorm gains
+gamma_q = 1 + gain_std * N(0,1) and gamma_k = 1 + gain_std * N(0,1), [128]
+fp32 each (gain_std 0.25; the tiny fp32 workload keeps gain 1, as its
+description states, but still draws them so the draw order is the same).
 Values are rounded to the storage dtype (bf16 or fp32) once.
 """
 from __future__ import annotations
@@ -42,6 +45,7 @@ class DecodeSpec:
     block_offset_std: float = 0.0
     appended: int = 0                       # tokens appended incrementally
     seed: int = 0
+    gain_std: float = 0.25                  # RMSNorm gains 1 + gain_std * N(0,1)
 
     @property
     def cap(self) -> int:
@@ -52,7 +56,8 @@ class DecodeSpec:
 
 def tiny_decode(seed: int = 0) -> DecodeSpec:
     """One sequence, one KV head, G = 4, context 4,096, budget 1,024, fp32."""
-    return DecodeSpec("tiny_1x4q1kv_4k_f32", 1, 4, 1, [4096], (1024,), kv_dtype="f32", seed=seed)
+    return DecodeSpec("tiny_1x4q1kv_4k_f32", 1, 4, 1, [4096], (1024,), kv_dtype="f32", seed=seed,
+                      gain_std=0.0)
 
 
 def qwen3_4b_32k(batch: int = 8, seq_len: int = 32768, seed: int = 1) -> DecodeSpec:
@@ -78,6 +83,14 @@ def qwen3_14b_paged_128k(batch: int = 16, seq_len: int = 131072, appended: int =
     added (and their blocks pooled) incrementally."""
     return DecodeSpec(f"qwen3_14b_paged_b{batch}_{seq_len // 1024}k", batch, 40, 8,
                       [seq_len] * batch, (4096,), paged=True, appended=appended, seed=seed)
+
+
+def _gains(g, device, std):
+    """RMSNorm gains of the gate query and key: 1 + std * N(0,1), [128] fp32
+    each (drawn even when std is 0, so later draws do not move)."""
+    gq = _randn((DIM,), g, device)
+    gk = _randn((DIM,), g, device)
+    return 1.0 + std * gq, 1.0 + std * gk
 
 
 def _randn(shape, g, device, std=1.0):
@@ -120,8 +133,7 @@ def make_decode_inputs(spec: DecodeSpec, device="cpu") -> dict:
         out["block_table"] = None
     out["w_q"] = _randn((hq, DIM, DIM), g, device, 1.0 / math.sqrt(DIM)).to(torch.bfloat16)
     out["w_k"] = _randn((hkv, 3 * DIM, DIM), g, device, 1.0 / math.sqrt(3 * DIM)).to(torch.bfloat16)
-    out["gamma_q"] = torch.ones(DIM, dtype=torch.float32, device=device)
-    out["gamma_k"] = torch.ones(DIM, dtype=torch.float32, device=device)
+    out["gamma_q"], out["gamma_k"] = _gains(g, device, spec.gain_std)
     out["seq_lens"] = torch.tensor(spec.seq_lens, dtype=torch.int32, device=device)
     return out
 
@@ -150,6 +162,7 @@ class PrefillSpec:
     seq_len: int
     token_budget: int = 2048
     seed: int = 4
+    gain_std: float = 0.25   # RMSNorm gains 1 + gain_std * N(0,1)
 
 
 def qwen3_8b_prefill_32k(batch: int = 4, seq_len: int = 32768, seed: int = 4) -> PrefillSpec:
@@ -159,8 +172,8 @@ def qwen3_8b_prefill_32k(batch: int = 4, seq_len: int = 32768, seed: int = 4) ->
 
 
 def make_prefill_inputs(spec: PrefillSpec, device="cpu") -> dict:
-    """q [B][Hq][T][128], k / v [B][Hkv][T][128] ~ N(0,1) in bf16; gate weights as
-    for decode.  Draw order: q, K, V, W_q, W_k."""
+    """q [B][Hq][T][128], k / v [B][Hkv][T][128] ~ N(0,1) in bf16; gate weights and
+    gains as for decode.  Draw order: q, K, V, W_q, W_k, gamma_q, gamma_k."""
     g = torch.Generator(device=device).manual_seed(spec.seed)
     B, hq, hkv, T = spec.batch, spec.hq, spec.hkv, spec.seq_len
     out = {"spec": spec}
@@ -169,6 +182,5 @@ def make_prefill_inputs(spec: PrefillSpec, device="cpu") -> dict:
     out["v"] = _randn((B, hkv, T, DIM), g, device).to(torch.bfloat16)
     out["w_q"] = _randn((hq, DIM, DIM), g, device, 1.0 / math.sqrt(DIM)).to(torch.bfloat16)
     out["w_k"] = _randn((hkv, 3 * DIM, DIM), g, device, 1.0 / math.sqrt(3 * DIM)).to(torch.bfloat16)
-    out["gamma_q"] = torch.ones(DIM, dtype=torch.float32, device=device)
-    out["gamma_k"] = torch.ones(DIM, dtype=torch.float32, device=device)
+    out["gamma_q"], out["gamma_k"] = _gains(g, device, spec.gain_std)
     return out

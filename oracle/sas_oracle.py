@@ -16,11 +16,12 @@ formula below is a reading, flagged ``ASSUMPTION``):
 
 * [aigc-0914] "Tencent released Simple-Attention-Sparsification, a method for
   efficient sparse attention in Qwen3 models" (aigc.news, 2026-09-14), release
-  paragraph: KV block size 64 tokens, training Top-K 31 historical blocks,
-  gate hidden size 128, query projection Qproj, key block pooling
-  max + min + average, Q/K normalization enabled, gate RoPE enabled, training
-  length 32,768, default sparse decode budget 2,048 tokens (1,024 and 4,096
-  also usable); continuous gates act on the selected blocks.
+  paragraph: 64-token KV blocks; 31 historical blocks kept in training; a
+  128-wide gate; the query goes through a projection called Qproj; each key
+  block is summarised by its maximum, minimum and average; queries and keys
+  are normalised and the gate applies RoPE; training sequences of 32,768
+  tokens; a 2,048-token decode budget by default, 1,024 and 4,096 also
+  usable; continuous gates weight the blocks that were selected.
 * [lmw-en] "Simple-Attention-Sparsification Text Generation Model: 12GB+
   VRAM" (localmodelwatch, English), "Specifications and Configuration Table":
   the same settings, and gate parameter counts 33.0M / 33.0M / 42.0M.
@@ -38,8 +39,8 @@ R1  W_q is [128][128] per query head, W_k is [384][128] per KV head, no bias,
     head layouts.
 R2  The query fed to Qproj is the per-head attention query (head_dim 128).
 R3  The pooled keys are the K cache values attention reads.
-R4  Pooled vector order is [max; min; avg] (word order of "max + min +
-    average").
+R4  Pooled vector order is [max; min; avg] (the order in which the release
+    paragraph lists the three poolings).
 R5  Q/K normalization is RMSNorm x / sqrt(mean(x^2) + eps) * gamma, eps 1e-6,
     applied after the projection and before RoPE.  The gain is one
     128-vector per layer for q and one for k, shared by all heads: with
@@ -88,8 +89,8 @@ POOL_DIM = 3 * HEAD_DIM   # max, min, avg stacked  (R4)
 
 
 # --------------------------------------------------------------------------
-# Step 1: key-block pooling ([aigc-0914] "key block pooling max + min +
-# average"; R3, R4).
+# Step 1: key-block pooling (release paragraph of [aigc-0914]: every key
+# block is summarised by its maximum, minimum and average; R3, R4).
 # --------------------------------------------------------------------------
 def pool_block(k_block: np.ndarray) -> np.ndarray:
     """Pooled key of one complete 64-token block.
@@ -106,8 +107,8 @@ def pool_block(k_block: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
-# Step 2 pieces: Q/K normalisation and gate RoPE ([aigc-0914] "Q/K
-# normalization enabled", "gate RoPE enabled"; R5, R6).
+# Step 2 pieces: Q/K normalisation and gate RoPE (release paragraph of
+# [aigc-0914]: queries and keys are normalised, the gate applies RoPE; R5, R6).
 # --------------------------------------------------------------------------
 def rms_norm(x: np.ndarray, gamma: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     """x / sqrt(mean(x^2) + eps) * gamma.  ASSUMPTION R5."""

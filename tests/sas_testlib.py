@@ -59,8 +59,13 @@ def run_decode_step(inputs, cfg, ws, gate_keys, pool=False):
     return {"out": out, "sel_idx": sel_idx, "sel_count": sel_count, "group_scores": group_scores}
 
 
-def oracle_pairs(inputs, budget, pairs, gate_mode=O.GATE_SELECT_ONLY):
-    """Oracle decode step (gate keys recomputed from K) for the listed pairs."""
+def oracle_pairs(inputs, budget, pairs, gate_mode=O.GATE_SELECT_ONLY, keys_cache=None,
+                 budgets=None):
+    """Oracle decode step (gate keys recomputed from K with the workload's
+    gain gamma_k; gate queries with gamma_q) for the listed pairs.
+    keys_cache: optional dict (s, h) -> oracle gate keys, filled and reused
+    (the keys do not depend on the budget).  budgets: per-sequence token
+    budgets, else `budget` for all."""
     spec = inputs["spec"]
     G = spec.hq // spec.hkv
     q = inputs["q"].double().cpu().numpy()
@@ -73,9 +78,15 @@ def oracle_pairs(inputs, budget, pairs, gate_mode=O.GATE_SELECT_ONLY):
         L = int(spec.seq_lens[s])
         ks, vs = logical_kv(inputs, s, h, L)
         c = (L - 1) // BLOCK
-        keys = O.gate_keys_for_sequence(ks, c, wk[h], gk)
+        if keys_cache is not None and (s, h) in keys_cache:
+            keys = keys_cache[(s, h)]
+        else:
+            keys = O.gate_keys_for_sequence(ks, c, wk[h], gk)
+            if keys_cache is not None:
+                keys_cache[(s, h)] = keys
+        bud = budget if budgets is None else int(budgets[s])
         r = O.decode_one_group(q[s, h * G:(h + 1) * G], ks, vs, L, keys, wq[h * G:(h + 1) * G],
-                               np.tile(gq, (G, 1)), budget, gate_mode=gate_mode)
+                               np.tile(gq, (G, 1)), bud, gate_mode=gate_mode)
         r["gate_keys"] = keys
         r["k"], r["v"], r["L"] = ks, vs, L
         res[(s, h)] = r
@@ -131,10 +142,28 @@ def check_pairs(inputs, cfg, gpu, oracle, gate_keys=None, out_atol=OUT_ATOL, bud
         c = len(r["S"])
         if gkeys is not None:
             assert_close_rel(gkeys[s, h, :c], r["gate_keys"], tag + " gate keys")
-        assert_close_rel(gs[s, h, :c], r["S"], tag + " group scores")
+        # bf16 key cache: rows whose stored key lies one ulp off the oracle's
+        # rounded key (see oracle_on_rounded_keys) are scored from the stored key
+        flipped = sorted(r.get("flipped_blocks", ()))
+        S_want = np.array(r["S"], np.float64)
+        if flipped:
+            S_want[flipped] = r["alt"]["S"][flipped]
+        assert_close_rel(gs[s, h, :c], S_want, tag + " group scores")
         m = int(sel_count[s, h])
         sel = list(sel_idx[s, h, :m])
-        swapped = assert_selection(sel, r["sel"], r["S"], topk, tag)
+        try:
+            swapped = assert_selection(sel, r["sel"], r["S"], topk, tag)
+        except AssertionError:
+            # accepted only when traced to a one-ulp key flip: a block whose
+            # membership differs has a flipped stored key, and the oracle on the
+            # stored keys selects the GPU's set (up to its own tie window)
+            if not flipped:
+                raise
+            diff = set(int(b) for b in sel) ^ set(r["sel"])
+            assert diff & set(flipped), f"{tag}: set mismatch not traceable to a one-ulp key flip"
+            swapped = assert_selection(sel, r["alt"]["sel"], r["alt"]["S"], topk, tag + " (stored keys)")
+            swapped = swapped or sel != r["sel"]
+            r = dict(r, s=r["alt"]["s"])
         want = r["out"]
         if swapped:  # an accepted tie swap: attend over the GPU's set
             toks = O.selected_token_ids(sel, r["L"])
@@ -147,3 +176,41 @@ def check_pairs(inputs, cfg, gpu, oracle, gate_keys=None, out_atol=OUT_ATOL, bud
         got = out[s, h * G:(h + 1) * G]
         err = float(np.max(np.abs(got - want)))
         assert np.all(np.isfinite(got)) and err <= out_atol, f"{tag}: out max-abs err {err}"
+
+
+def oracle_on_rounded_keys(inputs, cfg, gk_dev, pairs):
+    """Oracle decode step for a bf16 gate-key cache: the oracle's own keys,
+    rounded to bf16 (R19), feed its scores, selection and output.  The GPU's
+    stored keys must lie within one bf16 ulp of them and be equal for more
+    than 99 % of the elements (the two sides differ below fp32 precision, so
+    a value on a rounding boundary may land one ulp apart).  Blocks whose
+    stored key differs are listed as "flipped_blocks", and "alt" holds the
+    oracle run on the stored keys, which check_pairs consults only for them."""
+    spec = inputs["spec"]
+    G = spec.hq // spec.hkv
+    q = inputs["q"].double().cpu().numpy()
+    wq = inputs["w_q"].double().cpu().numpy()
+    wk = inputs["w_k"].double().cpu().numpy()
+    gq = np.tile(inputs["gamma_q"].double().cpu().numpy(), (G, 1))
+    gkn = inputs["gamma_k"].double().cpu().numpy()
+    gk_h = gk_dev.double().cpu().numpy()
+    res = {}
+    for (s, h) in pairs:
+        L = int(spec.seq_lens[s])
+        c = (L - 1) // BLOCK
+        ks, vs = logical_kv(inputs, s, h, L)
+        want_keys = O.round_to_bf16(O.gate_keys_for_sequence(ks, c, wk[h], gkn))
+        stored = gk_h[s, h, :c]
+        assert_close_rel(stored, want_keys, f"bf16 keys s={s} h={h}", rtol=BF16_ULP)
+        exact = float(np.mean(stored == want_keys)) if c else 1.0
+        assert exact > 0.99, f"only {exact:.4f} of the stored keys equal the rounded oracle keys"
+        qg, wg = q[s, h * G:(h + 1) * G], wq[h * G:(h + 1) * G]
+        r = O.decode_one_group(qg, ks, vs, L, want_keys, wg, gq, cfg.token_budget, gate_mode=cfg.gate_mode)
+        flipped = [b for b in range(c) if not np.array_equal(stored[b], want_keys[b])]
+        if flipped:
+            r["alt"] = O.decode_one_group(qg, ks, vs, L, stored, wg, gq, cfg.token_budget,
+                                          gate_mode=cfg.gate_mode)
+        r["flipped_blocks"] = flipped
+        r["k"], r["v"], r["L"] = ks, vs, L
+        res[(s, h)] = r
+    return res

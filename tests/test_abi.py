@@ -224,3 +224,30 @@ def test_prefill_validates_on_the_host(L):
     assert _prefill(L, _cfg(num_q_heads=24).c()) == sas.SAS_ERR_UNSUPPORTED  # odd group size (3)
     assert _prefill(L, _cfg(token_budget=8192).c()) == sas.SAS_ERR_UNSUPPORTED
     assert _prefill(L, c, batch=0) == sas.SAS_OK
+
+
+@pytest.mark.parametrize("gk16", [0, 1])
+def test_every_gate_key_entry_point_checks_the_dtype_first(monkeypatch, gk16):
+    """A gate-key tensor whose dtype disagrees with cfg.gate_keys_bf16 is refused
+    by the binding before any library call (a bf16 array read as fp32 would be
+    over-run by the kernels)."""
+    def no_library():
+        raise AssertionError("the library was called before the dtype check")
+
+    monkeypatch.setattr(sas, "lib", no_library)
+    cfg = sas.Config(8, 2, gate_keys_bf16=gk16)
+    wrong = torch.zeros(1, 2, 4, 128, dtype=torch.float32 if gk16 else torch.bfloat16)
+    kv = sas.KvCache(torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16),
+                     torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16), torch.ones(1, dtype=torch.int32))
+    q = torch.zeros(1, 8, 128, dtype=torch.bfloat16)
+    ws = torch.zeros(256, dtype=torch.uint8)
+    calls = [
+        lambda: sas.decode_step_static(cfg, q, kv, None, None, wrong, q),
+        lambda: sas.decode_step(cfg, q, kv, None, None, wrong, q, ws),
+        lambda: sas.pool_keys(cfg, kv, None, None, wrong, ws),
+        lambda: sas.gate_scores(cfg, q, kv.seq_lens, None, None, wrong, None, ws),
+        lambda: sas.prefill_block_sparse(cfg, q, q, q, None, None, None, None, wrong, q, ws),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError):
+            call()

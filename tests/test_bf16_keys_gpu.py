@@ -3,7 +3,9 @@ and stored rounded to nearest-even bf16; every reader scores from the stored
 value.  Parity: stored keys within one bf16 ulp of the oracle's keys rounded
 the same way (the two sides differ below fp32 precision, so a value on a
 rounding boundary may land one ulp apart), then scores, block sets and
-outputs against the oracle run on the stored keys."""
+outputs against the oracle run on its own rounded keys; a set difference is
+accepted only where a block involved has a stored key one ulp off and the
+oracle run on the stored keys agrees with the GPU."""
 import numpy as np
 import pytest
 import torch
@@ -27,27 +29,7 @@ def _pool(inp, cfg, ws):
 
 
 def _oracle_on_stored_keys(inp, cfg, gk, pairs):
-    spec = inp["spec"]
-    G = spec.hq // spec.hkv
-    q = inp["q"].double().cpu().numpy()
-    wq = inp["w_q"].double().cpu().numpy()
-    wk = inp["w_k"].double().cpu().numpy()
-    ones = np.ones(128)
-    gk_h = gk.double().cpu().numpy()
-    res = {}
-    for (s, h) in pairs:
-        L = int(spec.seq_lens[s])
-        c = (L - 1) // 64
-        ks, vs = logical_kv(inp, s, h, L)
-        want_keys = O.round_to_bf16(O.gate_keys_for_sequence(ks, c, wk[h], ones))
-        T.assert_close_rel(gk_h[s, h, :c], want_keys, f"bf16 keys s={s} h={h}", rtol=T.BF16_ULP)
-        exact = float(np.mean(gk_h[s, h, :c] == want_keys)) if c else 1.0
-        assert exact > 0.99, f"only {exact:.4f} of the stored keys equal the rounded oracle keys"
-        r = O.decode_one_group(q[s, h * G:(h + 1) * G], ks, vs, L, gk_h[s, h, :c], wq[h * G:(h + 1) * G],
-                               np.tile(ones, (G, 1)), cfg.token_budget, gate_mode=cfg.gate_mode)
-        r["k"], r["v"], r["L"] = ks, vs, L
-        res[(s, h)] = r
-    return res
+    return T.oracle_on_rounded_keys(inp, cfg, gk, pairs)
 
 
 @pytest.mark.parametrize("gate_mode", [sas.GATE_SELECT_ONLY, sas.GATE_LOGSIGMOID_BIAS])
@@ -96,7 +78,7 @@ def test_bf16_keys_qwen3_4b_32k_full_size():
     gpu = T.run_decode_step(inp, cfg, ws, gk)
     torch.cuda.synchronize()
     assert sas.get_device_status(ws) == sas.SAS_OK
-    pairs = [(0, 0), (3, 5), (7, 7)]
+    pairs = [(s, h) for s in range(spec.batch) for h in range(spec.hkv)]
     T.check_pairs(inp, cfg, gpu, _oracle_on_stored_keys(inp, cfg, gk, pairs))
 
 

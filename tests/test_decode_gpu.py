@@ -2,8 +2,10 @@
 
 Small shapes span several gate-key chunks, several selected blocks per CTA
 and ragged current blocks; the full-size workloads (Qwen3-4B 32k batch 8,
-Qwen3-8B ragged batch 32, Qwen3-14B paged 128k) are checked on sampled
-(sequence, KV head) pairs the oracle computes one by one."""
+Qwen3-8B ragged batch 32 at three budgets, Qwen3-14B paged 128k) are checked
+on every (sequence, KV head) pair, which the oracle computes one by one.  The
+workloads carry non-unit RMSNorm gains, so every kernel's use of gamma_q and
+gamma_k is compared too."""
 import math
 
 import numpy as np
@@ -118,12 +120,14 @@ def test_pool_keys_vs_oracle_and_raw_pooling():
     torch.cuda.synchronize()
     gk, raw = gk.cpu().numpy(), raw.cpu().numpy()
     wk = inp["w_k"].double().cpu().numpy()
+    gam_k = inp["gamma_k"].double().cpu().numpy()
+    assert not np.allclose(gam_k, 1.0)   # the gain is exercised
     for s in range(2):
         for h in range(2):
             L = spec.seq_lens[s]
             ks, _ = logical_kv(inp, s, h, L)
             nfull = L // 64
-            want = O.gate_keys_for_sequence(ks, nfull, wk[h], np.ones(128))
+            want = O.gate_keys_for_sequence(ks, nfull, wk[h], gam_k)
             T.assert_close_rel(gk[s, h, :nfull], want, f"gate keys s={s} h={h}")
             assert np.all(gk[s, h, nfull:] == 0), "incomplete blocks must not be pooled"
             for b in range(nfull):
@@ -149,13 +153,14 @@ def test_decode_step_pools_the_completed_block(dt):
     torch.cuda.synchronize()
     assert sas.get_device_status(ws) == sas.SAS_OK
     wk = inp["w_k"].double().cpu().numpy()
+    gam_k = inp["gamma_k"].double().cpu().numpy()
     for s, L in enumerate(spec.seq_lens):
         c = (L - 1) // 64
         for h in range(2):
             row = gk[s, h, c].cpu().numpy()
             if L % 64 == 0:
                 ks, _ = logical_kv(inp, s, h, L)
-                want = O.gate_key(O.pool_block(ks[64 * c:64 * c + 64]), wk[h], np.ones(128), c)
+                want = O.gate_key(O.pool_block(ks[64 * c:64 * c + 64]), wk[h], gam_k, c)
                 T.assert_close_rel(row, want, f"fused pooled key s={s} h={h}")
                 # same fp32 arithmetic in another accumulation order (384-term dot products)
                 T.assert_close_rel(row, ref[s, h, c].cpu().numpy(), "fused vs pooling kernel",
@@ -359,15 +364,31 @@ def test_device_bounds_are_reported_not_faulted():
 
 
 # ------------------------------------------------------------ full-size workloads
+# Gate keys, group scores, block sets and outputs are compared with the
+# oracle on EVERY (sequence, KV head) pair of the workload.
+
+
 def test_qwen3_4b_32k_full_size():
     spec = qwen3_4b_32k()
-    _run_and_check(spec, 2048, pairs=[(0, 0), (3, 5), (7, 7), (5, 2)])
+    inp, *_ = _run_and_check(spec, 2048)
+    assert not torch.allclose(inp["gamma_q"], torch.ones_like(inp["gamma_q"]))
 
 
-@pytest.mark.parametrize("budget", [1024, 2048, 4096])
-def test_qwen3_8b_ragged_full_size(budget):
+def test_qwen3_8b_ragged_full_size():
+    """Batch 32, contexts uniform in [8,192, 65,536]: every pair at each of the
+    budgets 1,024 / 2,048 / 4,096 (one set of gate keys, as in serving)."""
     spec = qwen3_8b_ragged()
-    _run_and_check(spec, budget, pairs=[(0, 0), (13, 4), (31, 7)])
+    inp = make_decode_inputs(spec, DEV)
+    keys = {}
+    for budget in (1024, 2048, 4096):
+        cfg = T.config_for(spec, budget)
+        ws = sas.make_workspace(cfg, DEV)
+        gk = T.run_pool(inp, cfg, ws)
+        gpu = T.run_decode_step(inp, cfg, ws, gk)
+        torch.cuda.synchronize()
+        assert sas.get_device_status(ws) == sas.SAS_OK
+        orc = T.oracle_pairs(inp, budget, _all_pairs(spec), keys_cache=keys)
+        T.check_pairs(inp, cfg, gpu, orc, gate_keys=gk)
 
 
 def test_qwen3_14b_paged_128k_incremental():
@@ -394,5 +415,5 @@ def test_qwen3_14b_paged_128k_incremental():
     gpu = T.run_decode_step(inp, cfg, ws, gk)
     torch.cuda.synchronize()
     assert sas.get_device_status(ws) == sas.SAS_OK
-    orc = T.oracle_pairs(inp, 4096, [(0, 0), (9, 3), (15, 7)])
+    orc = T.oracle_pairs(inp, 4096, _all_pairs(spec))
     T.check_pairs(inp, cfg, gpu, orc, gate_keys=gk)

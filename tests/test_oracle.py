@@ -9,8 +9,9 @@ catch them.
 Sources: "Tencent released Simple-Attention-Sparsification ..." (aigc.news,
 2026-09-14), release paragraph, and "Simple-Attention-Sparsification Text
 Generation Model: 12GB+ VRAM" (localmodelwatch), "Specifications and
-Configuration Table": block 64, Top-K 31, gate hidden 128, Qproj, max + min +
-average pooling, Q/K normalization, gate RoPE, budgets 1,024/2,048/4,096.
+Configuration Table": 64-token blocks, Top-K 31, a 128-wide gate, the Qproj
+query projection, keys pooled by maximum, minimum and average, normalised
+queries and keys, RoPE in the gate, budgets of 1,024 / 2,048 / 4,096 tokens.
 """
 import itertools
 import math
@@ -132,6 +133,93 @@ def test_gate_scores_closed_form():
         assert S[b] == s[0, b]
 
 
+# Asymmetric projection, non-unit gains.  q = e3; head 0's W_q has a single 1
+# at row 3, column 0, so q @ W_q = e0, while W_q @ q (the transposed
+# reading) would give e64 from the 1 at row 64, column 3.  Head 1's W_q sends
+# q to e64.  Gains: gamma_q[0] = 2, gamma_q[64] = 0.5, gamma_k[0] = 1.5,
+# gamma_k[1] = 0.25, gamma_k[64] = 3, every other entry 1 + (i mod 5)/10 (so
+# a gain read at the wrong index, dropped, or taken from the other vector
+# changes the value).
+def _gains():
+    i = np.arange(128)
+    g_q = 1.0 + (i % 5) / 10.0
+    g_k = 1.0 + ((i + 2) % 5) / 10.0
+    g_q[0], g_q[64] = 2.0, 0.5
+    g_k[0], g_k[1], g_k[64] = 1.5, 0.25, 3.0
+    return g_q, g_k
+
+
+def _asym_w_q():
+    w0 = np.zeros((128, 128))
+    w0[3, 0] = 1.0      # q @ W_q = e0
+    w0[64, 3] = 1.0     # W_q @ q = e64 (must not be used)
+    w1 = np.zeros((128, 128))
+    w1[3, 64] = 1.0     # q @ W_q = e64
+    w1[0, 3] = 1.0      # W_q @ q = e0 (must not be used)
+    return np.stack([w0, w1])
+
+
+def _asym_closed_form(c):
+    """Hand-derived scores of the two heads for the blocks of
+    _closed_form_inputs(c) (u = e64 - 3 e0 - e1 before the gain):
+      k^ = kn (3 e64 - 4.5 e0 - 0.25 e1),  kn = 1/sqrt(11/128 + eps);
+      q~_0 = 2a (cos c e0 + sin c e64),  q~_1 = 0.5a (-sin c e0 + cos c e64),
+      a = 1/sqrt(1/128 + eps);  RoPE turns pair (0, 64) by the position, so
+      s_0b = 2a kn (-4.5 cos(c-b) + 3 sin(c-b)) scale
+      s_1b = 0.5a kn (4.5 sin(c-b) + 3 cos(c-b)) scale
+    (pair (1, 65) meets zeros in both queries)."""
+    a = 1.0 / math.sqrt(1.0 / 128 + EPS)
+    kn = 1.0 / math.sqrt(11.0 / 128 + EPS)
+    s0 = [2 * a * kn * (-4.5 * math.cos(c - b) + 3 * math.sin(c - b)) * SCALE for b in range(c)]
+    s1 = [0.5 * a * kn * (4.5 * math.sin(c - b) + 3 * math.cos(c - b)) * SCALE for b in range(c)]
+    return np.array(s0), np.array(s1)
+
+
+def test_gate_scores_closed_form_asymmetric_projection_and_gains():
+    c = 11
+    n, k, w_k, _, _ = _closed_form_inputs(c)
+    g_q, g_k = _gains()
+    q = np.zeros((2, 128))
+    q[:, 3] = 1.0
+    gk = O.gate_keys_for_sequence(k, n, w_k, g_k, EPS)
+    s, S = O.gate_scores(q, _asym_w_q(), np.stack([g_q, g_q]), gk, n, c, SCALE, EPS)
+    s0, s1 = _asym_closed_form(c)
+    assert np.allclose(s[0], s0, rtol=0, atol=1e-12)
+    assert np.allclose(s[1], s1, rtol=0, atol=1e-12)
+    # group score: the mean of the two heads' closed forms (not their max)
+    assert np.allclose(S, 0.5 * (s0 + s1), rtol=0, atol=1e-12)
+    assert not np.allclose(S, np.maximum(s0, s1))
+
+
+def test_decode_step_driver_closed_form_gains():
+    """The batched driver gives gamma_q to the queries and gamma_k to the keys:
+    the same closed form through O.decode_step (one sequence, one KV head,
+    G = 2)."""
+    c = 11
+    _, k, w_k, _, _ = _closed_form_inputs(c)
+    g_q, g_k = _gains()
+    L = 64 * c + 5
+    kc = np.zeros((1, 1, L, 128))
+    kc[0, 0] = k[:L]
+    q = np.zeros((1, 2, 128))
+    q[0, :, 3] = 1.0
+    res = O.decode_step(q, kc, np.zeros_like(kc), [L], _asym_w_q(), g_q, w_k[None], g_k, 64 * 4)
+    s0, s1 = _asym_closed_form(c)
+    assert np.allclose(res[(0, 0)]["S"], 0.5 * (s0 + s1), rtol=0, atol=1e-12)
+
+
+def test_rms_norm_closed_form_with_gain():
+    # x = 3 e0 + 4 e1: mean(x^2) = 25/128; gain 2 at 0, -1 at 1
+    x = np.zeros(128)
+    x[0], x[1] = 3.0, 4.0
+    g = np.full(128, 7.0)
+    g[0], g[1] = 2.0, -1.0
+    r = math.sqrt(25.0 / 128 + EPS)
+    want = np.zeros(128)
+    want[0], want[1] = 6.0 / r, -4.0 / r
+    assert np.allclose(O.rms_norm(x, g, EPS), want, rtol=0, atol=1e-12)
+
+
 def test_gate_group_score_is_mean_over_heads():
     rng = np.random.default_rng(4)
     G, c = 4, 12
@@ -141,10 +229,11 @@ def test_gate_group_score_is_mean_over_heads():
     q = rng.standard_normal((G, 128))
     w_q = rng.standard_normal((G, 128, 128)) / math.sqrt(128)
     s, S = O.gate_scores(q, w_q, np.ones((G, 128)), gk, c, c, SCALE, EPS)
+    # each head scored alone gives the same row (heads do not interact)
     for g in range(G):
-        s1, _ = O.gate_scores(q[g:g + 1], w_q[g:g + 1], np.ones((1, 128)), gk, c, c, SCALE, EPS)
+        s1, S1 = O.gate_scores(q[g:g + 1], w_q[g:g + 1], np.ones((1, 128)), gk, c, c, SCALE, EPS)
         assert np.allclose(s1[0], s[g], atol=1e-14)
-    assert np.allclose(S, s.mean(axis=0), atol=1e-14)
+        assert np.allclose(S1, s1[0], atol=1e-14)   # one head: the group score is that head's
 
 
 def test_gate_scores_invariant_to_positive_key_scale():
@@ -526,3 +615,49 @@ def test_pins_catch_planted_mistakes(monkeypatch):
         test_gated_prefill_closed_form()
     monkeypatch.setattr(O, "log_sigmoid", good_ls)
     monkeypatch.setattr(O, "gated_token_bias", good_bias)
+
+    # projection read transposed (W_q @ q instead of q @ W_q)
+    good_gq = O.gate_query
+
+    def gate_query_transposed(q, w_q, gamma_q, pos, eps=1e-6, base=10000.0):
+        return good_gq(q, np.asarray(w_q).T, gamma_q, pos, eps, base)
+
+    monkeypatch.setattr(O, "gate_query", gate_query_transposed)
+    with pytest.raises(AssertionError):
+        test_gate_scores_closed_form_asymmetric_projection_and_gains()
+    monkeypatch.setattr(O, "gate_query", good_gq)
+
+    # gain read at the wrong index (rotate-half partner), or dropped
+    good_rms = O.rms_norm
+    monkeypatch.setattr(O, "rms_norm", lambda x, g, eps=1e-6: good_rms(x, np.roll(g, 64), eps))
+    with pytest.raises(AssertionError):
+        test_gate_scores_closed_form_asymmetric_projection_and_gains()
+    monkeypatch.setattr(O, "rms_norm", lambda x, g, eps=1e-6: good_rms(x, np.ones(128), eps))
+    with pytest.raises(AssertionError):
+        test_gate_scores_closed_form_asymmetric_projection_and_gains()
+    with pytest.raises(AssertionError):
+        test_rms_norm_closed_form_with_gain()
+    monkeypatch.setattr(O, "rms_norm", good_rms)
+
+    # the key gain given to the queries (driver level)
+    good_step = O.decode_step
+
+    def step_gains_swapped(q, kc, vc, lens, w_q, gamma_q, w_k, gamma_k, budget, **kw):
+        return good_step(q, kc, vc, lens, w_q, gamma_k, w_k, gamma_k, budget, **kw)
+
+    monkeypatch.setattr(O, "decode_step", step_gains_swapped)
+    with pytest.raises(AssertionError):
+        test_decode_step_driver_closed_form_gains()
+    monkeypatch.setattr(O, "decode_step", good_step)
+
+    # group score as the max over heads instead of the mean
+    good_gs = O.gate_scores
+
+    def gate_scores_max(*a, **kw):
+        s, S = good_gs(*a, **kw)
+        return s, (s.max(axis=0) if s.shape[1] else S)
+
+    monkeypatch.setattr(O, "gate_scores", gate_scores_max)
+    with pytest.raises(AssertionError):
+        test_gate_scores_closed_form_asymmetric_projection_and_gains()
+    monkeypatch.setattr(O, "gate_scores", good_gs)

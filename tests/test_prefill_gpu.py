@@ -37,37 +37,62 @@ def _run(spec, gk16=0, gate_mode=sas.GATE_SELECT_ONLY, budgets=None, want_status
     return inp, cfg, gk, out, sel, cnt
 
 
-def _check(spec, inp, cfg, gk, out, sel, cnt, triples, budgets=None):
+def _check(spec, inp, cfg, gk, out, sel, cnt, triples, budgets=None, sets_only=()):
+    """Compare the listed (sequence, KV head, query block) triples with the
+    oracle: gate keys of the pair, the block list, and the 64 x G outputs
+    (only the block list for the triples also listed in sets_only)."""
     G = spec.hq // spec.hkv
     wq = inp["w_q"].double().cpu().numpy()
     wk = inp["w_k"].double().cpu().numpy()
-    ones = np.ones(128)
+    gq = np.tile(inp["gamma_q"].double().cpu().numpy(), (G, 1))
+    gkn = inp["gamma_k"].double().cpu().numpy()
     gk_h = gk.double().cpu().numpy()
     out_h, sel_h, cnt_h = out.float().cpu().numpy(), sel.cpu().numpy(), cnt.cpu().numpy()
+    sets_only = set(sets_only)
     cache = {}
     for (s, h, i) in triples:
         if (s, h) not in cache:
             ks = inp["k"][s, h].double().cpu().numpy()
             vs = inp["v"][s, h].double().cpu().numpy()
-            keys = O.gate_keys_for_sequence(ks, spec.seq_len // 64, wk[h], ones)
+            keys = O.gate_keys_for_sequence(ks, spec.seq_len // 64, wk[h], gkn)
+            stored, flipped = None, set()
             if cfg.gate_keys_bf16:
-                # stored keys within one bf16 ulp of the oracle's rounded keys; the
-                # scores are then checked from the stored keys themselves
-                T.assert_close_rel(gk_h[s, h], O.round_to_bf16(keys), f"prefill bf16 gate keys s={s} h={h}",
-                                   rtol=T.BF16_ULP)
-                keys = gk_h[s, h]
+                # the oracle scores from its own rounded keys; stored keys lie within
+                # one bf16 ulp of them (> 99 % equal), and a row one ulp off is
+                # consulted only to trace a set difference to it
+                keys = O.round_to_bf16(keys)
+                T.assert_close_rel(gk_h[s, h], keys, f"prefill bf16 gate keys s={s} h={h}", rtol=T.BF16_ULP)
+                assert float(np.mean(gk_h[s, h] == keys)) > 0.99
+                stored = gk_h[s, h]
+                flipped = {b for b in range(keys.shape[0]) if not np.array_equal(stored[b], keys[b])}
             else:
                 T.assert_close_rel(gk_h[s, h], keys, f"prefill gate keys s={s} h={h}")
-            cache[(s, h)] = (ks, vs, keys)
-        ks, vs, keys = cache[(s, h)]
+            cache[(s, h)] = (ks, vs, keys, stored, flipped)
+        ks, vs, keys, stored, flipped = cache[(s, h)]
         qb = inp["q"][s, h * G:(h + 1) * G, 64 * i:64 * (i + 1)].double().cpu().numpy()
         topk = (cfg.max_sel if budgets is None else budgets[s] // 64) - 1
-        r = O.prefill_query_block(qb, ks, vs, i, keys, wq[h * G:(h + 1) * G], np.tile(ones, (G, 1)), topk,
-                                  gate_mode=cfg.gate_mode)
         m = int(cnt_h[s, h, i])
         got_sel = list(sel_h[s, h, i, :m])
         tag = f"{spec.name} s={s} h={h} i={i}"
-        swapped = T.assert_selection(got_sel, r["sel"], r["S"], topk, tag)
+        if (s, h, i) in sets_only:
+            qbar = qb.mean(axis=1)
+            sg, S = O.gate_scores(qbar, wq[h * G:(h + 1) * G], gq, keys, i, i)
+            r = {"sel": O.select_blocks(S, i, topk), "S": S, "s": sg}
+        else:
+            r = O.prefill_query_block(qb, ks, vs, i, keys, wq[h * G:(h + 1) * G], gq, topk,
+                                      gate_mode=cfg.gate_mode)
+        try:
+            swapped = T.assert_selection(got_sel, r["sel"], r["S"], topk, tag)
+        except AssertionError:
+            if not flipped:
+                raise
+            assert (set(int(b) for b in got_sel) ^ set(r["sel"])) & flipped, \
+                f"{tag}: set mismatch not traceable to a one-ulp key flip"
+            sg, S = O.gate_scores(qb.mean(axis=1), wq[h * G:(h + 1) * G], gq, stored, i, i)
+            T.assert_selection(got_sel, O.select_blocks(S, i, topk), S, topk, tag + " (stored keys)")
+            swapped, r = True, dict(r, s=sg)
+        if (s, h, i) in sets_only:
+            continue
         want = r["out"]
         if swapped:
             # the kernel kept a tie-window swap: attend over its list, gates from the oracle's scores
@@ -171,7 +196,13 @@ def test_prefill_beyond_512_blocks():
 
 
 def test_prefill_qwen3_8b_32k_full_size():
+    """Block lists of every query block of two (sequence, KV head) pairs and of
+    a spread of query blocks over all pairs; outputs on a sample."""
     spec = qwen3_8b_prefill_32k()
     res = _run(spec)
-    triples = [(0, 0, 0), (0, 0, 30), (1, 3, 31), (2, 5, 200), (3, 7, 511), (3, 2, 64)]
-    _check(spec, *res, triples)
+    nblk = spec.seq_len // 64
+    every = [(0, 0, i) for i in range(nblk)] + [(3, 7, i) for i in range(nblk)]
+    spread = [(s, h, (37 * (8 * s + h) + 11) % nblk) for s in range(spec.batch) for h in range(spec.hkv)]
+    outs = [(0, 0, 0), (0, 0, 30), (1, 3, 31), (2, 5, 200), (3, 7, 511), (3, 2, 64)]
+    sets = [t for t in every + spread if t not in outs]
+    _check(spec, *res, sets + outs, sets_only=sets)
