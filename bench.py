@@ -311,6 +311,112 @@ def run_prefill(args, device, world):
                                  "attention launches): a lower bound on the attention kernel's rate"}}
 
 
+def run_backward(args, rank, world, device):
+    """Gradient through the gates on the main workload (Qwen3-4B layer, batch 8,
+    32k context, budget 2,048, gated mode): one sas_gate_backward call per
+    step with the block lists of the forward step held fixed and a seeded
+    upstream gradient.  Algorithmic bytes: the selected K and V blocks, W_q
+    and W_k once, q and dL/dout, and the fp32 gradients of W_q and W_k
+    written once."""
+    import torch
+    from gated_block_sparse_token_b200 import sas
+    cfg, layers = build_layers(2, rank, device, gate_mode=sas.GATE_LOGSIGMOID_BIAS)
+    stream = torch.cuda.Stream(device)
+    for L in layers:
+        L["sel"] = torch.zeros(BATCH, HKV, cfg.max_sel, dtype=torch.int32, device=device)
+        L["cnt"] = torch.zeros(BATCH, HKV, dtype=torch.int32, device=device)
+        L["dout"] = torch.randn(BATCH, HQ, 128, generator=torch.Generator(device=device).manual_seed(9),
+                                device=device)
+    grads = [torch.zeros(HQ, 128, 128, device=device), torch.zeros(HKV, 384, 128, device=device),
+             torch.zeros(128, device=device), torch.zeros(128, device=device)]
+    torch.cuda.synchronize()   # the tensors above come from torch's stream
+    for L in layers:          # the forward step that fixes the block lists
+        inp = L["inp"]
+        sas.decode_step(cfg, inp["q"], L["kv"], inp["w_q"], inp["gamma_q"], L["gk"], L["out"], L["ws"],
+                        sel_idx=L["sel"], sel_count=L["cnt"], stream=stream)
+    torch.cuda.synchronize()
+
+    def bwd(L, st):
+        inp = L["inp"]
+        sas.gate_backward(cfg, inp["q"], L["kv"], inp["w_q"], inp["gamma_q"], inp["w_k"], inp["gamma_k"],
+                          L["sel"], L["cnt"], L["dout"], *grads, L["ws"], stream=st)
+
+    with torch.cuda.stream(stream):
+        for L in layers:
+            bwd(L, stream)
+    torch.cuda.synchronize()
+    steps = 200
+    main = plan(bwd, steps, layers, stream)
+    with torch.cuda.stream(stream):
+        run_graphs(main)
+    torch.cuda.synchronize()
+    med, lo, hi, ts = timed_repeats(main, world, stream, args.repeats)
+    for L in layers:
+        if sas.get_device_status(L["ws"], stream) != sas.SAS_OK:
+            raise RuntimeError("device status not OK after the backward run")
+    del layers, main
+    torch.cuda.empty_cache()
+    G = HQ // HKV
+    kv_bytes = BATCH * HKV * (BUDGET // 64) * 64 * 128 * 2 * 2
+    dbytes = (kv_bytes + HQ * 128 * 128 * 2 + HKV * 384 * 128 * 2 + 2 * BATCH * HQ * 128 * 2
+              + HQ * 128 * 128 * 4 + HKV * 384 * 128 * 4)
+    call_s = med / steps
+    peak, peak_kind = measured_peaks()
+    return {"workload": f"{WORKLOAD} gated-mode gradient (W_q, W_k, gains)", "steps": steps,
+            "value": round(job_throughput(steps, world, med), 2), "unit": "backward steps/s",
+            "ms_per_step": round(call_s * 1e3, 5), "timing": spread(ts, steps),
+            "roofline": dict(roofline_of(dbytes, call_s, peak, peak_kind),
+                             kernel="gate_backward_kernel (sas_gate_backward)")}
+
+
+def run_pooling(args, device, world):
+    """Pooled keys and gate keys of a whole prefill-shaped cache (the Qwen3-8B
+    head layout, batch 4 x 32,768 tokens, 8 KV heads: 16,384 blocks) in one
+    sas_pool_keys call: each block's K is read once, [max; min; mean] pooled,
+    projected by W_k on the tensor cores, normalised, rotated and stored.
+    Algorithmic bytes: K once, the gate keys written, W_k once per KV head."""
+    import torch
+    from gated_block_sparse_token_b200 import sas
+    from gated_block_sparse_token_b200.workloads import make_prefill_inputs, qwen3_8b_prefill_32k
+
+    spec = qwen3_8b_prefill_32k(batch=args.prefill_batch)
+    inp = make_prefill_inputs(spec, device)
+    B, T = spec.batch, spec.seq_len
+    nblk = T // 64
+    cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget)
+    lens = torch.full((B,), T, dtype=torch.int32, device=device)
+    # two copies of the cache alternate, so the timed calls read K from HBM
+    caches = [inp["k"], inp["k"].clone()]
+    kvs = [sas.KvCache(k, inp["v"], lens) for k in caches]
+    gk = torch.zeros(B, spec.hkv, nblk, 128, dtype=torch.float32, device=device)
+    ws = sas.make_workspace(cfg, device)
+    stream = torch.cuda.Stream(device)
+    with torch.cuda.stream(stream):
+        for kv in kvs:
+            sas.pool_keys(cfg, kv, inp["w_k"], inp["gamma_k"], gk, ws, stream=stream)
+    torch.cuda.synchronize()
+    n = 20
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            sas.pool_keys(cfg, kvs[i % 2], inp["w_k"], inp["gamma_k"], gk, ws, stream=stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    med, lo, hi, ts = timed_repeats([(g, 1)], world, stream, args.repeats)
+    if sas.get_device_status(ws, stream) != sas.SAS_OK:
+        raise RuntimeError("device status not OK after the pooling run")
+    del g, kvs, caches
+    torch.cuda.empty_cache()
+    dbytes = B * spec.hkv * T * 128 * 2 + B * spec.hkv * nblk * 128 * 4 + spec.hkv * 384 * 128 * 2
+    call_s = med / n
+    peak, peak_kind = measured_peaks()
+    return {"workload": f"{spec.name} (all {B * spec.hkv * nblk} blocks)", "calls": n,
+            "ms_per_call": round(call_s * 1e3, 4), "timing": spread(ts, n),
+            "roofline": dict(roofline_of(dbytes, call_s, peak, peak_kind),
+                             kernel="pool_project_kernel (tcgen05 projection)")}
+
+
 # the sources the fused decode kernel is built and launched from (its ncu
 # counters stay valid while the code in these does not change)
 DECODE_SOURCES = ("sas_api.cu", "sas_decode.cu", "sas_device.cuh", "sas_internal.h", "sas_select.cuh")
@@ -728,7 +834,9 @@ def run_ours(args):
         variants.append(run_variant(args, rank, world, device, "bf16 gate keys", gk16=1))
         variants.extend(run_ragged(args, rank, world, device))
         variants.append(run_long_context(args, rank, world, device))
+    bwd = None if args.skip_variants else run_backward(args, rank, world, device)
     pf = None if args.skip_prefill else run_prefill(args, device, world)
+    pool = None if args.skip_prefill else run_pooling(args, device, world)
 
     if rank != 0:
         return
@@ -767,6 +875,10 @@ def run_ours(args):
         line["variants"] = variants
     if pf is not None:
         line["prefill"] = pf
+    if pool is not None:
+        line["pooling"] = pool
+    if bwd is not None:
+        line["gate_backward"] = bwd
     print(json.dumps(line), flush=True)
 
 

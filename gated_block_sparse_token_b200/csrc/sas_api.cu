@@ -14,13 +14,14 @@ namespace sas {
 cudaError_t prepare_decode_kernels();
 cudaError_t prepare_pool_kernels();
 cudaError_t prepare_prefill_kernels();
+cudaError_t prepare_backward_kernels();
 }
 
 namespace {
 
 using sas::kDim;
 
-constexpr int32_t kAbiVersion = 6;
+constexpr int32_t kAbiVersion = 7;
 constexpr size_t kStatusBytes = 256;  // status word + padding
 constexpr int kMaxBudget = 16384;
 constexpr int kMaxGateBlocks = 16384;
@@ -50,6 +51,7 @@ cudaError_t prepare() {
     g_prep_err = sas::prepare_decode_kernels();
     if (g_prep_err == cudaSuccess) g_prep_err = sas::prepare_pool_kernels();
     if (g_prep_err == cudaSuccess) g_prep_err = sas::prepare_prefill_kernels();
+    if (g_prep_err == cudaSuccess) g_prep_err = sas::prepare_backward_kernels();
   });
   return g_prep_err;
 }
@@ -314,8 +316,11 @@ sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv, const int32_t*
   p.gk16 = cfg->gate_keys_bf16;
   p.pooled_raw = pooled_raw;
   p.status = static_cast<uint32_t*>(ws);
-  return launch_result(sas::launch_pool(cfg->kv_dtype == SAS_DTYPE_F32, p, kv->batch,
-                                        reinterpret_cast<cudaStream_t>(stream)));
+  if (cfg->kv_dtype == SAS_DTYPE_F32)
+    return launch_result(sas::launch_pool(true, p, kv->batch, reinterpret_cast<cudaStream_t>(stream)));
+  CUtensorMap tmwk;
+  if (!encode_kv_map(&tmwk, w_k, static_cast<long long>(cfg->num_kv_heads) * sas::kPool)) return SAS_ERR_CUDA;
+  return launch_result(sas::launch_pool_project(p, tmwk, kv->batch, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_gate_scores(const sas_config* cfg, const void* q, const int32_t* seq_lens,
@@ -484,7 +489,6 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
   if (batch == 0 || seq_len == 0) return SAS_OK;
   if (cfg->kv_dtype != SAS_DTYPE_BF16 || cfg->out_dtype != SAS_DTYPE_BF16) return SAS_ERR_UNSUPPORTED;
   const int G = cfg->num_q_heads / cfg->num_kv_heads;
-  if (G % 2 != 0) return SAS_ERR_UNSUPPORTED;  // the tensor-core tile pairs two query heads
   if (seq_len % 64 != 0) return SAS_ERR_UNSUPPORTED;
   if (cfg->token_budget / 64 > sas::kPfMaxSel) return SAS_ERR_UNSUPPORTED;
   const int nblk = seq_len / 64;
@@ -501,7 +505,7 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
   if (ws_bytes < sas_workspace_bytes(cfg, batch, seq_len)) return SAS_ERR_WORKSPACE;
   const long long qrows = static_cast<long long>(batch) * cfg->num_q_heads * seq_len;
   if (qrows > 0x7fffffffLL) return SAS_ERR_UNSUPPORTED;
-  if (static_cast<long long>(batch) * cfg->num_kv_heads * nblk * (G / 2) > 0x7fffffffLL)
+  if (static_cast<long long>(batch) * cfg->num_kv_heads * nblk * ((G + 1) / 2) > 0x7fffffffLL)
     return SAS_ERR_UNSUPPORTED;
   if (batch > 65535 || cfg->num_q_heads > 65535) return SAS_ERR_UNSUPPORTED;
   if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
@@ -530,7 +534,9 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
   pp.gk16 = cfg->gate_keys_bf16;
   pp.pooled_raw = nullptr;
   pp.status = static_cast<uint32_t*>(ws);
-  cudaError_t e = sas::launch_pool(false, pp, batch, s);
+  CUtensorMap tmwk;
+  if (!encode_kv_map(&tmwk, w_k, static_cast<long long>(cfg->num_kv_heads) * sas::kPool)) return SAS_ERR_CUDA;
+  cudaError_t e = sas::launch_pool_project(pp, tmwk, batch, s);
   if (e != cudaSuccess) return launch_result(e);
 
   // 2-4. gate queries, selection, tensor-core block-sparse attention
@@ -572,6 +578,64 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
       !encode_kv_map(&tmv, v, static_cast<long long>(batch) * p.hkv * seq_len))
     return SAS_ERR_CUDA;
   return launch_result(sas::launch_prefill(p, tmq, tmk, tmv, s));
+}
+
+sas_status sas_gate_backward(const sas_config* cfg, const void* q, const sas_kv* kv,
+                             const void* w_q, const float* gamma_q, const void* w_k,
+                             const float* gamma_k, const int32_t* sel_idx,
+                             const int32_t* sel_count, const float* d_out, float* dw_q,
+                             float* dw_k, float* dgamma_q, float* dgamma_k, void* ws,
+                             size_t ws_bytes, sas_stream_t stream) {
+  sas_status st = check_config(cfg);
+  if (st != SAS_OK) return st;
+  if ((st = check_kv(cfg, kv)) != SAS_OK) return st;
+  if ((st = check_ws(cfg, ws, ws_bytes)) != SAS_OK) return st;
+  if (kv->batch == 0) return SAS_OK;
+  if (q == nullptr || w_q == nullptr || gamma_q == nullptr || w_k == nullptr || gamma_k == nullptr ||
+      sel_idx == nullptr || sel_count == nullptr || d_out == nullptr || dw_q == nullptr ||
+      dw_k == nullptr || dgamma_q == nullptr || dgamma_k == nullptr)
+    return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 4) || !aligned(w_q, 2) || !aligned(gamma_q, 4) || !aligned(w_k, 2) ||
+      !aligned(gamma_k, 4) || !aligned(sel_idx, 4) || !aligned(sel_count, 4) ||
+      !aligned(d_out, 4) || !aligned(dw_q, 4) || !aligned(dw_k, 4) || !aligned(dgamma_q, 4) ||
+      !aligned(dgamma_k, 4))
+    return SAS_ERR_INVALID_ARG;
+  if (cfg->kv_dtype != SAS_DTYPE_BF16) return SAS_ERR_UNSUPPORTED;
+  const int G = cfg->num_q_heads / cfg->num_kv_heads;
+  const int max_sel = cfg->token_budget / 64;
+  // two K/V stages when they fit beside the list's pooled keys, else one
+  const int stages = sas::gate_bwd_smem_bytes(G, max_sel, 2) <= 227 * 1024 ? 2 : 1;
+  if (max_sel > sas::kBwMaxSel || sas::gate_bwd_smem_bytes(G, max_sel, stages) > 227 * 1024)
+    return SAS_ERR_UNSUPPORTED;
+  if (static_cast<long long>(kv->batch) * cfg->num_kv_heads > 0x7fffffffLL) return SAS_ERR_UNSUPPORTED;
+  // the select-only mode gives the gate parameters no gradient
+  if (cfg->gate_mode == SAS_GATE_SELECT_ONLY) return SAS_OK;
+  if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
+  sas::GateBwdParams p{};
+  sas::fill_rope_table(p.rope, cfg->rope_base);
+  p.hq = cfg->num_q_heads;
+  p.hkv = cfg->num_kv_heads;
+  p.G = G;
+  p.max_sel = max_sel;
+  p.eps = cfg->norm_eps;
+  p.attn_scale = cfg->attn_scale;
+  p.gate_scale = cfg->gate_scale;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kv = make_view(cfg, kv);
+  p.w_q = static_cast<const __nv_bfloat16*>(w_q);
+  p.gamma_q = gamma_q;
+  p.w_k = static_cast<const __nv_bfloat16*>(w_k);
+  p.gamma_k = gamma_k;
+  p.sel_idx = sel_idx;
+  p.sel_count = sel_count;
+  p.d_out = d_out;
+  p.stages = stages;
+  p.dw_q = dw_q;
+  p.dw_k = dw_k;
+  p.dgamma_q = dgamma_q;
+  p.dgamma_k = dgamma_k;
+  p.status = static_cast<uint32_t*>(ws);
+  return launch_result(sas::launch_gate_backward(p, kv->batch, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const sas_kv* kv,

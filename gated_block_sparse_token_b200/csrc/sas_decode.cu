@@ -82,6 +82,102 @@ __device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc)
 
 }  // namespace
 
+// Distributed exact Top-K of one cluster (the fused step's selection when
+// the sequence keeps at most kFastTopk historical blocks).  Every CTA holds
+// the (score, block) keys of its own gate-key rows in lkeys (plen[rank] of
+// them kept; keys are distinct, the block index breaks score ties toward the
+// lower block).  (1) each CTA ranks its keys by counting and sends its best
+// plen[rank], in descending order, to every CTA of the cluster (st.async into
+// gather[rank][.], bytes counted on bar); (2) every CTA ranks each received
+// candidate in the union -- its position in its own list plus, for each
+// other list, how many keys of that list beat it (binary search) -- and marks
+// the topk best in fmask (zeroed by the caller); (3) warp 0 turns the mask
+// into the ascending list sel[0 .. topk), then sel[topk] = cur.  The global
+// best topk always lie in the union (each is among its own CTA's best topk),
+// and a candidate outside them has at least topk union keys above it.
+// Returns false if the candidates did not all arrive (bounded wait; the
+// timeout bit is then set).  Ends with a block-wide barrier.
+template <int CS>
+__device__ __noinline__ bool distributed_topk(const unsigned long long* lkeys, unsigned long long* gather,
+                                              uint32_t* fmask, const int* plen, int n, int topk, int cur,
+                                              int rank, int* sel, uint64_t* bar, uint32_t* status) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // rows this CTA holds (the caller's plen is min(topk, rows)); the counting
+  // ranks only need the first plen[rank] positions, over all of its rows
+  const int nl = plen[CS];  // passed in plen[CS]: this CTA's row count
+  const int P = plen[rank];
+  const int split = (nl <= 32) ? 4 : ((nl <= 64) ? 2 : 1);  // threads per key
+  for (int base0 = 0; base0 < nl * split; base0 += kThreads) {
+    const int idx = base0 + tid;
+    const int i = idx / split, part = idx - i * split;
+    const bool live = i < nl;
+    const unsigned long long x = live ? lkeys[i] : 0ull;
+    int r = 0;
+    if (live)
+      for (int jj = part; jj < nl; jj += split) r += (lkeys[jj] > x) ? 1 : 0;
+    if (split >= 2) r += __shfl_xor_sync(0xffffffffu, r, 1);
+    if (split >= 4) r += __shfl_xor_sync(0xffffffffu, r, 2);
+    if (live && part == 0 && r < P) {
+#pragma unroll
+      for (int dst = 0; dst < CS; ++dst)
+        st_async_u64(dsmem_addr(gather + rank * kFastTopk + r, dst), x, dsmem_addr(bar, dst));
+    }
+  }
+  bool ok = mbar_wait_cluster(bar, 0, status);  // every CTA's candidates
+  ok = __syncthreads_and(ok) != 0;
+  if (!ok) return false;
+  for (int e = tid; e < CS * kFastTopk; e += kThreads) {
+    const int src = e / kFastTopk, pos = e - src * kFastTopk;
+    if (pos >= plen[src]) continue;
+    const unsigned long long x = gather[e];
+    int rk = pos;
+#pragma unroll
+    for (int r = 0; r < CS; ++r) {
+      if (r == src) continue;
+      const unsigned long long* lst = gather + r * kFastTopk;
+      int lo = 0;  // keys lst[0 .. lo) beat x (lists are descending)
+#pragma unroll
+      for (int step = kFastTopk; step > 0; step >>= 1)
+        if (lo + step <= plen[r] && lst[lo + step - 1] > x) lo += step;
+      rk += lo;
+    }
+    if (rk < topk) {
+      const uint32_t b = ~static_cast<uint32_t>(x & 0xFFFFFFFFull);
+      atomicOr(&fmask[b >> 5], 1u << (b & 31));
+    }
+  }
+  __syncthreads();
+  // ascending list from the mask (warp 0; lane l owns words wpl*l ..)
+  if (warp == 0) {
+    const int words = (n + 31) / 32;
+    const int wpl = (words + 31) / 32;
+    int cnt = 0;
+    for (int w = 0; w < wpl; ++w) {
+      const int wi = wpl * lane + w;
+      cnt += (wi < words) ? __popc(fmask[wi]) : 0;
+    }
+    int inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    int pos = inc - cnt;
+    for (int w = 0; w < wpl; ++w) {
+      const int wi = wpl * lane + w;
+      uint32_t mm = (wi < words) ? fmask[wi] : 0u;
+      while (mm != 0u) {
+        if (pos < topk) sel[pos] = 32 * wi + __ffs(mm) - 1;  // exactly topk bits are set
+        ++pos;
+        mm &= mm - 1u;
+      }
+    }
+    if (lane == 0) sel[topk] = cur;
+  }
+  __syncthreads();
+  return true;
+}
+
 template <typename T, typename OutT, int CS, int NST, int MODE>
 __global__ void __launch_bounds__(kThreads, 4)
     decode_cluster_kernel(const __grid_constant__ DecodeParams p,
@@ -149,12 +245,25 @@ __global__ void __launch_bounds__(kThreads, 4)
   const bool paged = p.kv.block_table != nullptr;
   bool rows_cached = false;  // meaningful in thread 0 only
 
+  // ------------------------------------------------------------ gate-key partition
+  // The gate-key rows of (s, h) are split over the cluster in chunks of one
+  // 16 KiB ring slot (32 fp32 or 64 bf16 rows): chunk j goes to CTA j % CS.
+  // The split does not depend on the sequence length, so each CTA requests
+  // its first NST chunks that lie inside the gate-key cache before the length
+  // is known (a chunk past the historical blocks is then not scored).
+  const int gk_rows = p.gk16 ? 2 * kGkChunk : kGkChunk;
+  const uint32_t gk_row_bytes = p.gk16 ? kDim * 2u : kDim * 4u;
+  const uint8_t* gk_pair = static_cast<const uint8_t*>(p.gate_keys) + static_cast<size_t>(pair) * p.mg * gk_row_bytes;
+  int nspec = 0;  // chunks requested before the length is known (tiles 0 .. nspec-1)
+  if (MODE != kModeAttend)
+    while (nspec < NST && (rank + nspec * CS) * gk_rows < p.mg) ++nspec;
+
   // ------------------------------------------------------------ prologue copies
   // Thread 0 loads the sequence length first (one request per CTA: every CTA
   // of the grid reads the same few bytes) and, while it is in flight,
   // requests everything that does not depend on it, asynchronously: q of the
-  // group (bulk), gamma_q (bulk) and the W_q column slice of this CTA (one 2-D
-  // TMA box per head).
+  // group (bulk), gamma_q (bulk), the W_q column slice of this CTA (one 2-D
+  // TMA box per head) and its first gate-key chunks.
   int* len_s = reinterpret_cast<int*>(qbar);  // qbar is written only after the validation
   if (tid == 0) {
     const int L0 = p.kv.seq_lens[s];
@@ -182,6 +291,14 @@ __global__ void __launch_bounds__(kThreads, 4)
       for (int g = 0; g < wq_heads; ++g)
         tma_load_2d(wq_s + static_cast<size_t>(g) * kDim * kDpc, &tmw, rank * kDpc, (h * G + g) * kDim,
                     bar_pro);
+      // the gate query v arrives from every CTA whatever the length holds
+      mbar_arrive_expect_tx(bar_v, static_cast<uint32_t>(G * kDim * 4));
+    }
+    for (int k = 0; k < nspec; ++k) {
+      const int r0 = (rank + k * CS) * gk_rows;
+      const uint32_t bytes = static_cast<uint32_t>(min(gk_rows, p.mg - r0)) * gk_row_bytes;
+      mbar_arrive_expect_tx(&bars[k], bytes);
+      bulk_g2s(slots + k * kTileBytes, gk_pair + static_cast<size_t>(r0) * gk_row_bytes, bytes, &bars[k]);
     }
     len_s[0] = L0;
     len_s[1] = topk0;
@@ -195,6 +312,59 @@ __global__ void __launch_bounds__(kThreads, 4)
     th0 = p.rope.theta_over_pi[lane];
     th1 = p.rope.theta_over_pi[lane + 32];
   }
+
+  // ------------------------------------------------------------ phase 0: gate query projection
+  // v_g = q_g @ W_q[g] needs no length: it runs while the length load is in
+  // flight.  Two threads per output column (rows 0..63 and 64..127),
+  // combined by shuffle; every CTA of the cluster receives every column.
+  // Large groups take the W_q slice in two passes through the same region
+  // (the second copy is requested once every read of the first is done).
+  // the cluster barrier first: every thread of the cluster has arrived, so
+  // thread 0's barrier initialisation (fenced before its arrival) is visible
+  // before any thread waits on those barriers, and every CTA runs before
+  // stores reach it
+  cluster_wait();
+  const bool pro_ok = mbar_wait(bar_pro, 0, p.status);
+  if (MODE != kModeAttend) {
+    bool wq_ok = pro_ok;
+    for (int g0 = 0; g0 < G; g0 += wq_heads) {
+      const int gn = min(wq_heads, G - g0);
+      if (g0 > 0) {
+        __syncthreads();
+        if (tid == 0) {
+          fence_proxy_async_smem();  // the slice's generic reads before the async-proxy overwrite
+          mbar_arrive_expect_tx(bar_wq2, static_cast<uint32_t>(gn * kDim * kDpc * 2));
+          for (int g = 0; g < gn; ++g)
+            tma_load_2d(wq_s + static_cast<size_t>(g) * kDim * kDpc, &tmw, rank * kDpc,
+                        (h * G + g0 + g) * kDim, bar_wq2);
+        }
+        wq_ok = mbar_wait(bar_wq2, 0, p.status) && wq_ok;
+      }
+      for (int o = tid; o < 2 * gn * kDpc; o += kThreads) {
+        const int half = o & 1;
+        const int oc = o >> 1;
+        const int gl = oc / kDpc;  // head within this pass
+        const int j = oc - gl * kDpc;
+        const int g = g0 + gl;
+        const T* qrow = qraw + g * kDim + half * 64;
+        const __nv_bfloat16* wcol = wq_s + (static_cast<size_t>(gl) * kDim + half * 64) * kDpc + j;
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (wq_ok) {
+#pragma unroll 16
+          for (int i = 0; i < 64; ++i)
+            a4[i & 3] = fmaf(to_float(qrow[i]), __bfloat162float(wcol[i * kDpc]), a4[i & 3]);
+        }
+        float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        if (half == 0) {
+#pragma unroll
+          for (int r = 0; r < CS; ++r)
+            st_async_f32(dsmem_addr(qv + g * kDim + rank * kDpc + j, r), acc, dsmem_addr(bar_v, r));
+        }
+      }
+    }
+  }
+  SAS_TRACE(1);
 
   // ------------------------------------------------------------ validation
   __syncthreads();
@@ -253,25 +423,47 @@ __global__ void __launch_bounds__(kThreads, 4)
   if (MODE == kModeFused) m = bad ? 0 : min(topk, n) + 1;
   if (MODE == kModeAttend && bad) m = 0;
 
-  const int nb_per = (n + CS - 1) / CS;
-  const int b_lo = min(n, rank * nb_per);
-  const int b_hi = min(n, b_lo + nb_per);
-  // gate-key rows per 16 KiB ring slot: 32 fp32 rows or 64 bf16 rows
-  const int gk_rows = p.gk16 ? 2 * kGkChunk : kGkChunk;
-  const uint32_t gk_row_bytes = p.gk16 ? kDim * 2u : kDim * 4u;
-  const uint8_t* gk_pair = static_cast<const uint8_t*>(p.gate_keys) + static_cast<size_t>(pair) * p.mg * gk_row_bytes;
-  const int nchunks = (MODE == kModeAttend) ? 0 : (b_hi - b_lo + gk_rows - 1) / gk_rows;
+  // gate-key chunks of this CTA: global chunks rank, rank + CS, ... below
+  // ceil(n / gk_rows); the speculative ones are tiles 0 .. nspec-1 whatever
+  // the length turned out to be
+  const int nch_all = (n + gk_rows - 1) / gk_rows;
+  const int nch_need = (MODE == kModeAttend || nch_all <= rank) ? 0 : (nch_all - rank + CS - 1) / CS;
+  const int nchunks = (MODE == kModeAttend) ? 0 : max(nch_need, nspec);
+  // historical blocks (gate-key rows) CTA r scores: its full chunks plus the
+  // partial last chunk if it owns it
+  auto rows_of = [&](int r) -> int {
+    const int full = n / gk_rows, rem = n - full * gk_rows;
+    const int nf = (full > r) ? (full - r + CS - 1) / CS : 0;
+    return nf * gk_rows + ((rem > 0 && full % CS == r) ? rem : 0);
+  };
+  // Top-K route: nothing to choose (a 64-token budget, or every historical
+  // block kept); the distributed selection; or every score to rank 0, which
+  // selects for the cluster (budgets above kFastTopk + 1 blocks, very long
+  // contexts)
+  const bool sel_local = (MODE == kModeFused) && (topk <= 0 || n <= topk);
+  const bool sel_fast = (MODE == kModeFused) && !sel_local && topk <= kFastTopk &&
+                        ((nch_all + CS - 1) / CS) * gk_rows <= kFastRows;
   const int cnt_mine = (rank < m) ? (m - 1 - rank) / CS + 1 : 0;
   const bool own_cur = (m > 0) && ((m - 1) % CS == rank);
+  unsigned long long* lkeys = reinterpret_cast<unsigned long long*>(base + p.sm.r_lkeys);
+  unsigned long long* gather = reinterpret_cast<unsigned long long*>(base + p.sm.r_gather);
+  uint32_t* fmask = reinterpret_cast<uint32_t*>(base + p.sm.r_fmask);
 
   // bytes this CTA will receive from the cluster (bad is uniform over it)
   if (tid == 0) {
-    if (MODE != kModeAttend && !bad) mbar_arrive_expect_tx(bar_v, static_cast<uint32_t>(G * kDim * 4));
     if (MODE == kModeFused && !bad) {
-      if (rank == 0)
-        mbar_arrive_expect_tx(bar_sc, static_cast<uint32_t>(n * 4));
-      else
-        mbar_arrive_expect_tx(bar_sel, static_cast<uint32_t>(m * 4));
+      if (sel_fast) {
+        uint32_t bytes = 0;
+        for (int r = 0; r < CS; ++r) bytes += static_cast<uint32_t>(min(topk, rows_of(r))) * 8u;
+        mbar_arrive_expect_tx(bar_sc, bytes);
+      } else if (!sel_local) {
+        if (rank == 0)
+          mbar_arrive_expect_tx(bar_sc, static_cast<uint32_t>(n * 4));
+        else
+          mbar_arrive_expect_tx(bar_sel, static_cast<uint32_t>(m * 4));
+      } else {
+        mbar_arrive_expect_tx(bar_sc, static_cast<uint32_t>(CS * 4));  // one token per CTA
+      }
     }
     if (do_pool) {
       mbar_arrive_expect_tx(bar_p, kPool * 4);
@@ -279,6 +471,8 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
     if (MODE != kModeGate) mbar_arrive_expect_tx(bar_m, static_cast<uint32_t>(CS * G * (kDpc + 2) * 4));
   }
+  if (sel_fast && !bad)
+    for (int w = tid; w < (n + 31) / 32; w += kThreads) fmask[w] = 0u;  // W_q reads are done
 
   // list entry e of this CTA -> block id (the current block first if owned)
   auto entry_index = [&](int e) -> int {
@@ -294,13 +488,13 @@ __global__ void __launch_bounds__(kThreads, 4)
   // Tile t lives in slot t % NST, phase (t / NST) & 1.  Tiles 0..nchunks-1
   // are gate-key chunks, then kTilesPerBlock tiles per list entry.  Thread 0
   // issues tile t once tile t - NST has been released by every thread.
-  int issued = 0;  // meaningful in thread 0 only
+  int issued = nspec;  // meaningful in thread 0 only
   auto issue = [&](int t) {
     const int slot = t % NST;
     uint8_t* dst = slots + slot * kTileBytes;
     if (t < nchunks) {
-      const int b0 = b_lo + t * gk_rows;
-      const int cntb = min(gk_rows, b_hi - b0);
+      const int b0 = (rank + t * CS) * gk_rows;
+      const int cntb = min(gk_rows, n - b0);
       const uint32_t bytes = static_cast<uint32_t>(cntb) * gk_row_bytes;
       mbar_arrive_expect_tx(&bars[slot], bytes);
       bulk_g2s(dst, gk_pair + static_cast<size_t>(b0) * gk_row_bytes, bytes, &bars[slot]);
@@ -331,60 +525,17 @@ __global__ void __launch_bounds__(kThreads, 4)
   int known = nchunks + ((MODE == kModeAttend) ? kTilesPerBlock * cnt_mine
                                                : (own_cur ? kTilesPerBlock : 0));
   pump(0, known);
-  if (tid == 0 && nchunks > NST) {
-    // the ring holds NST chunks: ask L2 for the rest of this CTA's gate keys now
-    const int b0 = b_lo + NST * gk_rows;
-    prefetch_l2(gk_pair + static_cast<size_t>(b0) * gk_row_bytes, static_cast<uint32_t>(b_hi - b0) * gk_row_bytes);
-  }
-  SAS_TRACE(1);
-
-  // ------------------------------------------------------------ phase 0: gate query
-  const bool pro_ok = mbar_wait(bar_pro, 0, p.status);
-  cluster_wait();  // every CTA of the cluster is running
-  if (MODE != kModeAttend && !bad) {
-    // two threads per output column (rows 0..63 and 64..127), combined by
-    // shuffle; every CTA of the cluster receives every column.  Large groups
-    // take the W_q slice in two passes through the same region (the second
-    // copy is requested once every read of the first is done).
-    bool wq_ok = pro_ok;
-    for (int g0 = 0; g0 < G; g0 += wq_heads) {
-      const int gn = min(wq_heads, G - g0);
-      if (g0 > 0) {
-        __syncthreads();
-        if (tid == 0) {
-          fence_proxy_async_smem();  // the slice's generic reads before the async-proxy overwrite
-          mbar_arrive_expect_tx(bar_wq2, static_cast<uint32_t>(gn * kDim * kDpc * 2));
-          for (int g = 0; g < gn; ++g)
-            tma_load_2d(wq_s + static_cast<size_t>(g) * kDim * kDpc, &tmw, rank * kDpc,
-                        (h * G + g0 + g) * kDim, bar_wq2);
-        }
-        wq_ok = mbar_wait(bar_wq2, 0, p.status) && wq_ok;
-      }
-      for (int o = tid; o < 2 * gn * kDpc; o += kThreads) {
-        const int half = o & 1;
-        const int oc = o >> 1;
-        const int gl = oc / kDpc;  // head within this pass
-        const int j = oc - gl * kDpc;
-        const int g = g0 + gl;
-        const T* qrow = qraw + g * kDim + half * 64;
-        const __nv_bfloat16* wcol = wq_s + (static_cast<size_t>(gl) * kDim + half * 64) * kDpc + j;
-        float a4[4] = {0.f, 0.f, 0.f, 0.f};
-        if (wq_ok) {
-#pragma unroll 16
-          for (int i = 0; i < 64; ++i)
-            a4[i & 3] = fmaf(to_float(qrow[i]), __bfloat162float(wcol[i * kDpc]), a4[i & 3]);
-        }
-        float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        if (half == 0) {
-#pragma unroll
-          for (int r = 0; r < CS; ++r)
-            st_async_f32(dsmem_addr(qv + g * kDim + rank * kDpc + j, r), acc, dsmem_addr(bar_v, r));
-        }
-      }
+  if (tid == 0) {
+    // the ring holds NST chunks: ask L2 for this CTA's later chunks now
+    for (int t = NST; t < nch_need; ++t) {
+      const int b0 = (rank + t * CS) * gk_rows;
+      prefetch_l2(gk_pair + static_cast<size_t>(b0) * gk_row_bytes,
+                  static_cast<uint32_t>(min(gk_rows, n - b0)) * gk_row_bytes);
     }
-    mbar_wait_cluster(bar_v, 0, p.status);  // every column of v is here
   }
+
+  // ------------------------------------------------------------ gate query: norm and RoPE
+  if (MODE != kModeAttend) mbar_wait_cluster(bar_v, 0, p.status);  // every column of v is here
   SAS_TRACE(2);
 
   if (MODE != kModeAttend) {
@@ -439,8 +590,8 @@ __global__ void __launch_bounds__(kThreads, 4)
     for (int ci = 0; ci < nchunks; ++ci) {
       const int slot = ci % NST;
       const bool ok = mbar_wait(&bars[slot], (ci / NST) & 1, p.status);
-      const int b0 = b_lo + ci * gk_rows;
-      const int cntb = min(gk_rows, b_hi - b0);
+      const int b0 = (rank + ci * CS) * gk_rows;
+      const int cntb = max(0, min(gk_rows, n - b0));  // 0 for a speculative chunk past n
       const float* gk = reinterpret_cast<const float*>(slots + slot * kTileBytes);
       const uint8_t* gk16 = slots + slot * kTileBytes;
       for (int it = 0; it < gk_rows / 16; ++it) {
@@ -465,8 +616,16 @@ __global__ void __launch_bounds__(kThreads, 4)
           acc += __shfl_xor_sync(0xffffffffu, acc, 2);
           acc += __shfl_xor_sync(0xffffffffu, acc, 4);
           S = acc;
-          // rank 0 of the cluster receives every score and selects
-          if (sub == 0 && bb < cntb) st_async_f32(dsmem_addr(keys + b0 + bb, 0), S, dsmem_addr(bar_sc, 0));
+          if (sub == 0 && bb < cntb) {
+            if (sel_fast) {
+              // (score, block) key: larger score first, then the lower block
+              lkeys[ci * gk_rows + bb] = (static_cast<unsigned long long>(order_key(S)) << 32) |
+                                         static_cast<unsigned long long>(~static_cast<uint32_t>(b0 + bb));
+            } else if (!sel_local) {
+              // rank 0 of the cluster receives every score and selects
+              st_async_f32(dsmem_addr(keys + b0 + bb, 0), S, dsmem_addr(bar_sc, 0));
+            }
+          }
         } else {
           for (int g = 0; g < G; ++g) {
             float acc = 0.f;
@@ -506,22 +665,63 @@ __global__ void __launch_bounds__(kThreads, 4)
   if (MODE == kModeGate) return;  // everything sent to this CTA (v) has arrived
 
   // ------------------------------------------------------------ phase 2: Top-K
-  // Rank 0 selects once for the cluster: every CTA signals rank 0 when its
-  // scores are in (release / acquire at cluster scope), rank 0 ranks them
-  // and sends the block list to every other CTA the same way.
   if (MODE == kModeFused) {
     SAS_TRACE(4);
     auto issue_wk = [&]() {
       // this CTA's 16 columns of W_k[h] (384 rows as three 128-row boxes);
       // they land over the key region, unused from here on
       if (do_pool && tid == 0) {
+        fence_proxy_async_smem();  // the key region's generic accesses before the async-proxy overwrite
         mbar_arrive_expect_tx(bar_wk, kPool * kDpc * 2);
         for (int part = 0; part < 3; ++part)
           tma_load_2d(wk_s + part * 128 * kDpc, &tmwk, rank * kDpc, h * kPool + part * 128, bar_wk);
       }
     };
     bool list_ok = true;
-    if (!bad) {
+    if (bad) {
+      if (rank == 0 && tid == 0 && p.sel_count != nullptr) p.sel_count[pair] = 0;
+    } else if (sel_local) {
+      // every historical block kept (or none): the list needs no scores.  A
+      // token from every CTA still marks the end of its scores, so that no
+      // CTA's merge partials reach another's inbox (over its gate query)
+      // while that CTA is still scoring.
+      if (tid < CS) st_async_u32(dsmem_addr(scan + rank, tid), 1u, dsmem_addr(bar_sc, tid));
+      list_ok = mbar_wait_cluster(bar_sc, 0, p.status);
+      const int kept = m - 1;
+      for (int j = tid; j < kept; j += kThreads) sel[j] = j;
+      if (tid == 0) sel[kept] = c;
+      __syncthreads();
+      if (rank == 0) {
+        for (int j = tid; j < m; j += kThreads)
+          if (p.sel_idx != nullptr) p.sel_idx[static_cast<size_t>(pair) * p.max_sel + j] = sel[j];
+        if (p.sel_count != nullptr && tid == 0) p.sel_count[pair] = m;
+      }
+      issue_wk();
+    } else if (sel_fast) {
+      // Distributed exact Top-K.  (1) each CTA ranks its own (score, block)
+      // keys by counting (keys are distinct: the block index breaks ties) and
+      // sends its best min(topk, rows) in descending order to every CTA;
+      // (2) every CTA ranks each received candidate in the union -- its
+      // position in its own list plus, for each other list, how many keys of
+      // that list beat it (binary search) -- and keeps the topk best as a
+      // bit mask; (3) the mask gives the ascending list.  The global best
+      // topk always lie in the union: each is among its own CTA's best topk.
+      int plen[CS + 1];  // kept candidates of every CTA, then this CTA's row count
+#pragma unroll
+      for (int r = 0; r < CS; ++r) plen[r] = min(topk, rows_of(r));
+      plen[CS] = rows_of(rank);
+      list_ok = distributed_topk<CS>(lkeys, gather, fmask, plen, n, topk, c, rank, sel, bar_sc, p.status);
+      __syncthreads();
+      SAS_TRACE(18);
+      if (rank == 0) {
+        if (p.sel_idx != nullptr)
+          for (int j = tid; j < m; j += kThreads) p.sel_idx[static_cast<size_t>(pair) * p.max_sel + j] = sel[j];
+        if (p.sel_count != nullptr && tid == 0) p.sel_count[pair] = list_ok ? m : 0;
+      }
+      issue_wk();
+    } else {
+      // Rank 0 selects once for the cluster: it waits for every score, ranks
+      // them and sends the block list to every other CTA the same way.
       if (rank == 0) {
         list_ok = mbar_wait_cluster(bar_sc, 0, p.status);
         SAS_TRACE(9);  // rank 0: every score of the cluster is in
@@ -553,8 +753,6 @@ __global__ void __launch_bounds__(kThreads, 4)
         issue_wk();
         list_ok = mbar_wait_cluster(bar_sel, 0, p.status);
       }
-    } else if (rank == 0 && tid == 0 && p.sel_count != nullptr) {
-      p.sel_count[pair] = 0;
     }
     // a list that never came (timeout, already in the status word) is not
     // read: the current block, always valid, stands in for every entry

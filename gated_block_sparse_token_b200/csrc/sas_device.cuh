@@ -136,6 +136,12 @@ __device__ __forceinline__ void st_async_u32(uint32_t raddr, uint32_t v, uint32_
                : "memory");
 }
 
+__device__ __forceinline__ void st_async_u64(uint32_t raddr, unsigned long long v, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(raddr), "l"(v),
+               "r"(rbar)
+               : "memory");
+}
+
 __device__ __forceinline__ void fence_acq_rel_cluster() {
   asm volatile("fence.acq_rel.cluster;" ::: "memory");
 }

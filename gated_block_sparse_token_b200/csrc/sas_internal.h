@@ -26,6 +26,12 @@ enum DecodeMode : int { kModeGate = 0, kModeAttend = 1, kModeFused = 2 };
 // this CTA still reads.
 constexpr int kSelBins = 1024;  // value buckets of the Top-K selection
 constexpr int kSelCand = 256;   // candidates ranked exactly in the boundary bucket
+// Distributed Top-K of the fused step (every CTA ranks its own gate-key rows,
+// the clusters' CTAs exchange their sorted local candidates, every CTA ranks
+// the union): taken when the sequence keeps at most kFastTopk historical
+// blocks and no CTA holds more than kFastRows of them.
+constexpr int kFastTopk = 64;
+constexpr int kFastRows = 256;
 
 struct DecodeSmem {
   int slots;     // NST stage slots of 16 KiB (gate-key chunks, then K/V tiles)
@@ -49,6 +55,10 @@ struct DecodeSmem {
   int r_hist;    // uint32 [kSelBins], then int32 candidates        (phase 2)
   int r_selbits; // uint32 [(mg + 31) / 32]                         (phase 2)
   int r_scan;    // int32 [16]                                      (phase 2)
+  // distributed Top-K (phases 1-2; over keys.., like the rank-0 selection)
+  int r_lkeys;   // uint64 [kFastRows] this CTA's (score, block) keys
+  int r_gather;  // uint64 [CS][kFastTopk] sorted local candidates of every CTA
+  int r_fmask;   // uint32 [(mg + 31) / 32] selected blocks
   int total;     // bytes to request, including alignment slack
 };
 
@@ -99,7 +109,11 @@ inline DecodeSmem plan_decode_smem_heads(int G, int mg, int cs, int nst, int max
   p.r_hist = p.r_keys + up16(mg * 4);
   p.r_selbits = p.r_hist + up16(std::max(kSelBins, kSelCand) * 4);
   p.r_scan = p.r_selbits + up16((mg + 31) / 32 * 4);
-  const int end24 = std::max(p.r_scan + 16 * 4, p.r_wk + kPool * dpc * 2);
+  p.r_lkeys = p.r_keys;
+  p.r_gather = p.r_lkeys + kFastRows * 8;
+  p.r_fmask = p.r_gather + cs * kFastTopk * 8;
+  const int end_fast = p.r_fmask + up16((mg + 31) / 32 * 4);
+  const int end24 = std::max(std::max(p.r_scan + 16 * 4, end_fast), p.r_wk + kPool * dpc * 2);
   p.total = std::max(end01, end24) + 1024;
   return p;
 }
@@ -193,8 +207,51 @@ struct PrefillParams {
   unsigned long long* trace;  // per-CTA timings (tracing builds only), else null
 };
 
+// Gradient through the gates of the gated decode step (one CTA per
+// (sequence, KV head), the block list held fixed).
+constexpr int kBwThreads = 256;
+constexpr int kBwMaxSel = 64;  // block lists of up to 64 entries (4,096 tokens)
+
+struct GateBwdParams {
+  RopeTable rope;
+  int hq, hkv, G, max_sel;
+  float eps, attn_scale, gate_scale;
+  const __nv_bfloat16* q;     // [B][Hq][128]
+  KvView kv;
+  const __nv_bfloat16* w_q;   // [Hq][128][128]
+  const float* gamma_q;       // [128]
+  const __nv_bfloat16* w_k;   // [Hkv][384][128]
+  const float* gamma_k;       // [128]
+  const int32_t* sel_idx;     // [B][Hkv][max_sel]
+  const int32_t* sel_count;   // [B][Hkv]
+  const float* d_out;         // [B][Hq][128]
+  int stages;                 // K/V ring stages (2, or 1 when two do not fit)
+  float* dw_q;                // [Hq][128][128]  (accumulated)
+  float* dw_k;                // [Hkv][384][128] (accumulated)
+  float* dgamma_q;            // [128]           (accumulated)
+  float* dgamma_k;            // [128]           (accumulated)
+  uint32_t* status;
+};
+
+// Shared-memory bytes of the backward kernel for a group of G heads and
+// block lists of max_sel entries.
+inline int gate_bwd_smem_bytes(int G, int max_sel, int stages = 2) {
+  return stages * 2 * kTileBytes       // K and V tiles, one or two stages
+         + max_sel * kPool * 4         // pooled keys of the list
+         + max_sel * kDim * 4          // u, then dL/du, per entry
+         + 4 * G * kDim * 4            // q, d_out, v (then dL/dv), q~
+         + 3 * max_sel * G * 4         // per-entry softmax statistics
+         + 2 * max_sel * G * 4         // gate scores and their gradients
+         + 2 * G * kBlock * 4          // logits and d_out . v of one block
+         + 2 * max_sel * 4             // list, RMS of u
+         + 3 * kDim * 4                // spare
+         + G * kDim * 4                // dL/dq~ per head
+         + 2 * kDim * 4                // dL/dgamma_q, dL/dgamma_k partial sums
+         + 4 * 8 + 1024;               // barriers, alignment slack
+}
+
 constexpr int kPfQb = 16;      // query blocks per gate-query CTA
-constexpr int kPfMaxSel = 64;  // prefill budget up to 4,096 tokens (two CTAs per SM)
+constexpr int kPfMaxSel = 256;  // prefill budget up to 16,384 tokens (two CTAs per SM up to 4,096)
 
 constexpr int kPoolBlocksPerCta = 8;
 constexpr int kPoolWkBytes = kPool * kDim * 2;  // W_k of one KV head, bf16 (96 KiB)
@@ -211,12 +268,16 @@ cudaError_t launch_decode(int mode, bool f32_kv, bool f32_out, int cs, int nst,
                           cudaStream_t stream);
 cudaError_t launch_topk(const TopkParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_pool(bool f32_kv, const PoolParams& p, int batch, cudaStream_t stream);
+// bf16 caches: pooling on the CUDA cores, projection on the tensor cores
+// (tmwk: W_k as a [Hkv*384][128] bf16 map, 64x64 boxes, 128-byte swizzle)
+cudaError_t launch_pool_project(const PoolParams& p, const CUtensorMap& tmwk, int batch, cudaStream_t stream);
 size_t topk_smem_bytes(int mg, int max_sel);
 size_t pool_smem_bytes();
 void fill_rope_table(RopeTable& t, float base);
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmq, const CUtensorMap& tmk,
                            const CUtensorMap& tmv, cudaStream_t stream);
 size_t prefill_attn_smem_bytes(int max_sel);
+cudaError_t launch_gate_backward(const GateBwdParams& p, int batch, cudaStream_t stream);
 
 // One-time per-process set-up of kernel attributes.
 cudaError_t prepare_kernels();

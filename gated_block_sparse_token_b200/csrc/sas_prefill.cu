@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
                         const __grid_constant__ CUtensorMap tmk,
                         const __grid_constant__ CUtensorMap tmv) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int npair = p.G / 2;
+  const int npair = (p.G + 1) / 2;
   int idx = static_cast<int>(blockIdx.x);
   const int pair = idx % npair;
   idx /= npair;
@@ -302,6 +302,9 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
   const int s = idx % p.batch;
   const int i = p.nblk - 1 - idx / p.batch;  // longest block lists first
   const int g0 = h * p.G + 2 * pair;
+  // an odd group's last tile holds one head: rows 64..127 repeat it and are
+  // not stored
+  const bool lone = 2 * pair + 1 >= p.G;
 #ifdef SAS_PHASE_TRACE
   unsigned long long* trc =
       (p.trace != nullptr && blockIdx.x < static_cast<unsigned>(kTraceCtas)) ? p.trace + blockIdx.x * kTraceSlots : nullptr;
@@ -369,7 +372,7 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
       const uint64_t dK = umma_desc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dV = umma_desc_sw128(smem_u32(sV), 8192, 1024);
       const int rowq0 = static_cast<int>((static_cast<size_t>(s) * p.hq + g0) * p.T) + kBlock * i;
-      const int rowq1 = rowq0 + p.T;
+      const int rowq1 = lone ? rowq0 : rowq0 + p.T;
       const int rowkv = static_cast<int>((static_cast<size_t>(s) * p.hkv + h) * p.T);
       mbar_arrive_expect_tx(&bars[kBarQ], 32768);
       tma_load_2d(sQ + 0, &tmq, 0, rowq0, &bars[kBarQ]);
@@ -464,7 +467,7 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
       const int grp = lane >> 3, sub = lane & 7;
       const float4* qa = reinterpret_cast<const float4*>(
           p.qt + ((static_cast<size_t>(s) * p.hq + g0) * p.nblk + i) * kDim + sub * 16);
-      const float4* qb = qa + static_cast<size_t>(p.nblk) * (kDim / 4);  // head g0 + 1
+      const float4* qb = qa + (lone ? 0 : static_cast<size_t>(p.nblk) * (kDim / 4));  // head g0 + 1
       float4 q0[4], q1[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -609,10 +612,10 @@ __global__ void __launch_bounds__(kPfAttnThreads, 2)
           pk.y = pack_bf16x2(o[8 * k + 2] * inv, o[8 * k + 3] * inv);
           pk.z = pack_bf16x2(o[8 * k + 4] * inv, o[8 * k + 5] * inv);
           pk.w = pack_bf16x2(o[8 * k + 6] * inv, o[8 * k + 7] * inv);
-          *reinterpret_cast<uint4*>(dst + 32 * c + 8 * k) = pk;
+          if (!(lone && r >= kBlock)) *reinterpret_cast<uint4*>(dst + 32 * c + 8 * k) = pk;
         }
       }
-    } else {
+    } else if (!(lone && r >= kBlock)) {
       for (int c = 0; c < kDim / 8; ++c) *reinterpret_cast<uint4*>(dst + 8 * c) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
@@ -652,7 +655,7 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmq, const
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  const unsigned ctas = static_cast<unsigned>(p.batch) * p.hkv * p.nblk * (p.G / 2);
+  const unsigned ctas = static_cast<unsigned>(p.batch) * p.hkv * p.nblk * ((p.G + 1) / 2);
   const size_t smem = prefill_attn_smem_bytes(p.max_sel);
   if (p.gated)
     prefill_attn_kernel<true><<<ctas, kPfAttnThreads, smem, stream>>>(p, tmq, tmk, tmv);

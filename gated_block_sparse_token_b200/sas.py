@@ -18,7 +18,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 # SAS_LIBRARY selects another build of the same ABI (e.g. the phase-trace build).
 LIB_PATH = os.environ.get("SAS_LIBRARY", os.path.join(_HERE, "libsas.so"))
-ABI_VERSION = 6             # the include/sas.h this binding marshals for
+ABI_VERSION = 7             # the include/sas.h this binding marshals for
 
 SAS_OK = 0
 SAS_ERR_INVALID_ARG = 1
@@ -86,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "sas_sparse_decode": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step_static": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]),
+            "sas_gate_backward": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "sas_prefill_block_sparse": (ctypes.c_int, [cfgp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
         }
         for name, (res, args) in sigs.items():
@@ -264,6 +265,17 @@ def decode_step_static(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out
                                         int(gate_keys.shape[2]), _ptr(out), _ptr(sel_idx),
                                         _ptr(sel_count), _ptr(group_scores), _ptr(status_out),
                                         _stream(stream)), "sas_decode_step_static")
+
+
+def gate_backward(cfg: Config, q, kv: KvCache, w_q, gamma_q, w_k, gamma_k, sel_idx, sel_count, d_out,
+                  dw_q, dw_k, dgamma_q, dgamma_k, ws, stream=None) -> None:
+    """sas_gate_backward: adds dL/dW_q, dL/dW_k, dL/dgamma_q, dL/dgamma_k (fp32)
+    of the gated decode step, block lists held fixed, for d_out = dL/dout."""
+    c, k = cfg.c(), kv.c()
+    _check(lib().sas_gate_backward(ctypes.byref(c), _ptr(q), ctypes.byref(k), _ptr(w_q), _ptr(gamma_q),
+                                   _ptr(w_k), _ptr(gamma_k), _ptr(sel_idx), _ptr(sel_count), _ptr(d_out),
+                                   _ptr(dw_q), _ptr(dw_k), _ptr(dgamma_q), _ptr(dgamma_k), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "sas_gate_backward")
 
 
 def prefill_block_sparse(cfg: Config, q, k, v, w_q, gamma_q, w_k, gamma_k, gate_keys, out, ws,

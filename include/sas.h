@@ -8,10 +8,11 @@
  * in Qwen3 models", aigc.news 2026-09-14, release paragraph; "Simple-Attention-
  * Sparsification Text Generation Model: 12GB+ VRAM", localmodelwatch,
  * "Specifications and Configuration Table"):
- *   KV block size 64 tokens; gate hidden size 128; query projection "Qproj";
- *   key block pooling max + min + average; Q/K normalization; gate RoPE;
- *   Top-K of historical blocks under a 1,024 / 2,048 (default) / 4,096-token
- *   budget, the current block always kept (31 + 1 = 2,048 / 64).
+ *   64-token KV blocks; a 128-wide gate; the query goes through a projection
+ *   the pages call Qproj; each key block is summarised by its maximum,
+ *   minimum and average; queries and keys are normalised and the gate applies
+ *   RoPE; the top historical blocks are kept under a 1,024, 2,048 (default)
+ *   or 4,096-token budget, the current block always kept (31 + 1 = 2,048/64).
  *
  * Readings of what the pages leave open (one per item, used by every entry
  * point):
@@ -273,9 +274,10 @@ SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const s
  *   optional outputs (NULL to skip), the block list of every query block.
  *   ws: 256-byte aligned, at least sas_workspace_bytes(cfg, B, T) bytes
  *   (gate queries and block lists live there).
- * This build requires bf16 inputs and output, an even GQA group size
- * (the tensor-core tile holds two query heads), T a multiple of 64 and a
- * budget of at most 4,096 tokens; other requests return SAS_ERR_UNSUPPORTED.
+ * This build requires bf16 inputs and output and T a multiple of 64; other
+ * requests return SAS_ERR_UNSUPPORTED.  Budgets up to the configuration's
+ * limit of 16,384 tokens and GQA groups of 1 to 8 heads are handled (the
+ * tensor-core tile holds two query heads; an odd group's last tile one).
  */
 SAS_API sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const void* k,
                                             const void* v, int32_t batch, int32_t seq_len,
@@ -285,6 +287,42 @@ SAS_API sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q
                                             void* gate_keys, int32_t max_gate_blocks, void* out,
                                             int32_t* sel_idx, int32_t* sel_count, void* ws,
                                             size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * Gradient through the gates (pages: the continuous gates on the selected
+ * blocks give a differentiable path through the discrete Top-K selection;
+ * aigc.news release paragraph of 2026-09-14).  For the gated decode step
+ * (cfg->gate_mode = SAS_GATE_LOGSIGMOID_BIAS) with the block lists held fixed
+ * and an upstream gradient d_out of its output, ADDS to
+ *   dw_q     fp32 [Hq][128][128]   dL/dW_q
+ *   dw_k     fp32 [Hkv][384][128]  dL/dW_k
+ *   dgamma_q fp32 [128]            dL/dgamma_q
+ *   dgamma_k fp32 [128]            dL/dgamma_k
+ * (zero them first for a fresh gradient; the sums over sequences use atomic
+ * adds, so the last bits depend on their order).  The gate of a selected
+ * historical block b for query head g is log(sigmoid(s_gb)) on its tokens'
+ * logits; its gradient reaches W_q and gamma_q through the gate query (q_g
+ * @ W_q[g], RMSNorm, gain, RoPE at the current block) and W_k and gamma_k
+ * through the gate key of b (pooled block @ W_k, RMSNorm, gain, RoPE at b),
+ * recomputed here from the cache.  The Top-K itself has no gradient.  In the
+ * select-only mode the gate parameters get no gradient: the call returns
+ * SAS_OK and enqueues nothing.
+ *   q        bf16 [B][Hq][128], the step's queries
+ *   kv       the cache the step read (bf16)
+ *   sel_idx, sel_count: the block lists of the step (as sas_decode_step
+ *            returns them); a list that is not ascending, does not end with
+ *            the current block or names a block outside the cache skips its
+ *            (sequence, KV head) and sets SAS_ERR_DEVICE_BOUNDS's bit
+ *   d_out    fp32 [B][Hq][128]  dL/dout
+ * This build handles budgets up to 4,096 tokens (lists of up to 64 blocks)
+ * and bf16 caches; others return SAS_ERR_UNSUPPORTED.
+ */
+SAS_API sas_status sas_gate_backward(const sas_config* cfg, const void* q, const sas_kv* kv,
+                                     const void* w_q, const float* gamma_q, const void* w_k,
+                                     const float* gamma_k, const int32_t* sel_idx,
+                                     const int32_t* sel_count, const float* d_out, float* dw_q,
+                                     float* dw_k, float* dgamma_q, float* dgamma_k, void* ws,
+                                     size_t ws_bytes, sas_stream_t stream);
 
 /*
  * Allocation-free variant of sas_decode_step.  The release pages have no

@@ -72,6 +72,15 @@ R19 bf16 gate-key cache (a storage option, not a change of the method): the
     ships its gate weights in bf16 ([lmw-en] table: the printed checkpoint
     sizes fit bf16 weights).
 
+R20 Gradient through the gates (the release paragraph of [aigc-0914] says the
+    continuous gates on the selected blocks give a differentiable path
+    through the discrete Top-K; second paragraph of [nedoborov] likewise):
+    in the gated mode (R18), for an upstream gradient dL/dout, the gradients
+    of the gate parameters W_q, W_k, gamma_q and gamma_k flow through
+    log(sigmoid(s_gb)) of every selected historical block; the selected set
+    is held fixed (the Top-K itself has no gradient).  In the select-only
+    mode (R12) the gate parameters get no gradient.
+
 Parity status: the gate formula as a whole (R1-R8) is pinned only by the
 invariants and hand-derived closed forms in tests/test_oracle.py, not by any
 value the pages print ("parity unpinned" against the pages for the exact gate
@@ -397,3 +406,129 @@ def decode_step(q, k_cache, v_cache, seq_lens, w_q, gamma_q, w_k, gamma_k,
                                        w_q[heads], np.tile(gamma_q, (G, 1)), token_budget,
                                        eps=eps, base=base, gate_mode=gate_mode)
     return res
+
+
+# --------------------------------------------------------------------------
+# Gradient of the gated decode step with respect to the gate parameters
+# (R20): the continuous gates on the selected blocks make the gate
+# differentiable; the Top-K set is held fixed.
+# --------------------------------------------------------------------------
+def rms_norm_backward(x, gamma, dy, eps: float = 1e-6):
+    """Backward of y = x / r * gamma, r = sqrt(mean(x^2) + eps): returns
+    (dL/dx, dL/dgamma) for dL/dy = dy.  From dy_i/dx_k = gamma_i (delta_ik / r
+    - x_i x_k / (n r^3))."""
+    x = np.asarray(x, np.float64)
+    gamma = np.asarray(gamma, np.float64)
+    dy = np.asarray(dy, np.float64)
+    n = x.shape[-1]
+    r = math.sqrt(float(np.mean(x * x)) + eps)
+    gdy = gamma * dy
+    dx = gdy / r - x * float(np.dot(gdy, x)) / (n * r ** 3)
+    dgamma = dy * x / r
+    return dx, dgamma
+
+
+def log_sigmoid_grad(x: float) -> float:
+    """d log(sigmoid(x)) / dx = 1 - sigmoid(x) = sigmoid(-x)."""
+    return math.exp(log_sigmoid(-x))
+
+
+def matmul_weight_grad(x, dy):
+    """Gradient of W in y = x @ W (row vector x): dL/dW[i][j] = x_i dL/dy_j."""
+    return np.outer(np.asarray(x, np.float64), np.asarray(dy, np.float64))
+
+
+def rope_backward(dy, pos: int, base: float = 10000.0):
+    """Backward of the gate RoPE at `pos`: each (i, i+64) pair is a plane
+    rotation, so its transpose is the rotation by -pos."""
+    return rope_rotate_half(dy, -pos, base)
+
+
+def decode_gate_grads(q_group, k_seq, v_seq, seq_len, w_q_group, gamma_q, w_k, gamma_k,
+                      token_budget, d_out, attn_scale=1.0 / math.sqrt(128.0),
+                      gate_scale=1.0 / math.sqrt(128.0), eps=1e-6, base=10000.0, sel=None):
+    """Gated-mode decode step of one (sequence, KV head) and the gradients of
+    L = sum_g d_out[g] . out[g] with respect to the gate parameters (R20).
+
+    q_group [G][128]; k_seq, v_seq [>= L][128]; w_q_group [G][128][128];
+    gamma_q [128]; w_k [384][128]; gamma_k [128]; d_out [G][128].
+    sel: the block list to hold fixed (None: the gate's own Top-K).
+    Returns dict(out, sel, s, dw_q [G][128][128], dw_k [384][128],
+    dgamma_q [128], dgamma_k [128]).
+
+    Forward, in the method's order: pooled keys P_b, u_b = P_b @ W_k,
+    k^_b = RMSNorm(u_b) * gamma_k, k~_b = RoPE(k^_b, b); v_g = q_g @ W_q[g],
+    q^_g = RMSNorm(v_g) * gamma_q, q~_g = RoPE(q^_g, c); s_gb = q~_g . k~_b *
+    gate_scale; logits q_g . k_j * attn_scale + log(sigmoid(s_gb)) on the
+    tokens j of a selected historical block b (0 on the current block);
+    softmax; out_g = sum_j p_gj v_j.  Backward in reverse order."""
+    q_group = np.asarray(q_group, np.float64)
+    d_out = np.asarray(d_out, np.float64)
+    G = q_group.shape[0]
+    c = (seq_len - 1) // BLOCK
+    # forward
+    P = [pool_block(k_seq[b * BLOCK:(b + 1) * BLOCK]) for b in range(c)]
+    u = [P[b] @ np.asarray(w_k, np.float64) for b in range(c)]
+    kt = np.array([rope_rotate_half(rms_norm(u[b], gamma_k, eps), b, base) for b in range(c)]).reshape(c, HEAD_DIM)
+    v = [q_group[g] @ np.asarray(w_q_group[g], np.float64) for g in range(G)]
+    qt = np.array([rope_rotate_half(rms_norm(v[g], gamma_q, eps), c, base) for g in range(G)])
+    s = (qt @ kt.T) * gate_scale if c else np.zeros((G, 0))
+    if sel is None:
+        sel = select_blocks(s.mean(axis=0) if c else np.zeros(0), c, topk_for_budget(token_budget))
+    toks = selected_token_ids(sel, seq_len)
+    blk = [t // BLOCK for t in toks]
+    out = np.zeros((G, HEAD_DIM))
+    dw_q = np.zeros((G, HEAD_DIM, HEAD_DIM))
+    dgamma_q = np.zeros(HEAD_DIM)
+    dkt = np.zeros((c, HEAD_DIM))
+    ds_all = np.zeros((G, c))
+    for g in range(G):
+        bias = np.array([0.0 if b == c else log_sigmoid(s[g, b]) for b in blk])
+        logits = (k_seq[toks].astype(np.float64) @ q_group[g]) * attn_scale + bias
+        w = np.exp(logits - logits.max())
+        p = w / w.sum()
+        out[g] = p @ v_seq[toks].astype(np.float64)
+        # softmax backward: dL/dlogit_j = p_j (d_out . v_j - d_out . out)
+        dv_dot = v_seq[toks].astype(np.float64) @ d_out[g]
+        dlogit = p * (dv_dot - float(np.dot(d_out[g], out[g])))
+        # the bias of block b is shared by its tokens; d log(sigmoid(s))/ds = 1 - sigmoid(s)
+        dq_t = np.zeros(HEAD_DIM)
+        for b in sel[:-1]:
+            dbias = sum(dl for dl, bj in zip(dlogit, blk) if bj == b)
+            ds = dbias * log_sigmoid_grad(s[g, b])
+            ds_all[g, b] = ds
+            dq_t += ds * gate_scale * kt[b]
+            dkt[b] += ds * gate_scale * qt[g]
+        dq_hat = rope_backward(dq_t, c, base)
+        dvg, dgq = rms_norm_backward(v[g], gamma_q, dq_hat, eps)
+        dgamma_q += dgq
+        dw_q[g] = matmul_weight_grad(q_group[g], dvg)
+    dw_k = np.zeros((POOL_DIM, HEAD_DIM))
+    dgamma_k = np.zeros(HEAD_DIM)
+    for b in sel[:-1]:
+        dk_hat = rope_backward(dkt[b], b, base)
+        dub, dgk = rms_norm_backward(u[b], gamma_k, dk_hat, eps)
+        dgamma_k += dgk
+        dw_k += matmul_weight_grad(P[b], dub)
+    return {"out": out, "sel": sel, "s": s, "ds": ds_all, "dw_q": dw_q, "dw_k": dw_k,
+            "dgamma_q": dgamma_q, "dgamma_k": dgamma_k}
+
+
+def gated_decode_loss(q_group, k_seq, v_seq, seq_len, w_q_group, gamma_q, w_k, gamma_k,
+                      d_out, sel, attn_scale=1.0 / math.sqrt(128.0),
+                      gate_scale=1.0 / math.sqrt(128.0), eps=1e-6, base=10000.0):
+    """L = sum_g d_out[g] . out[g] of the gated decode step over the fixed
+    block list `sel` (the scalar whose gradient decode_gate_grads returns),
+    through the forward functions above (gate_keys_for_sequence,
+    gate_scores, attention_over_tokens)."""
+    G = len(q_group)
+    c = (seq_len - 1) // BLOCK
+    keys = gate_keys_for_sequence(k_seq, c, w_k, gamma_k, eps, base)
+    s, _ = gate_scores(q_group, w_q_group, np.tile(gamma_q, (G, 1)), keys, c, c, gate_scale, eps, base)
+    toks = selected_token_ids(sel, seq_len)
+    tot = 0.0
+    for g in range(G):
+        o = attention_over_tokens(q_group[g], k_seq, v_seq, toks, attn_scale,
+                                  gated_token_bias(s[g], sel, seq_len, c))
+        tot += float(np.dot(d_out[g], o))
+    return tot

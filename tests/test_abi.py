@@ -33,7 +33,7 @@ def test_header_declares_all_entry_points():
     names = set(declared_functions())
     want = {"sas_pool_keys", "sas_gate_scores", "sas_topk_blocks", "sas_sparse_decode",
             "sas_decode_step", "sas_workspace_bytes", "sas_get_device_status",
-            "sas_reset_device_status", "sas_status_string", "sas_abi_version"}
+            "sas_reset_device_status", "sas_status_string", "sas_abi_version", "sas_gate_backward"}
     assert want <= names
 
 
@@ -84,7 +84,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(L):
-    assert sas.abi_version() == sas.ABI_VERSION == 6
+    assert sas.abi_version() == sas.ABI_VERSION == 7
     for st in range(7):
         assert len(sas.status_string(st)) > 0
     assert sas.status_string(sas.SAS_OK) == "ok"
@@ -221,9 +221,28 @@ def test_prefill_validates_on_the_host(L):
     assert _prefill(L, c, ws=FAKE + 16) == sas.SAS_ERR_WORKSPACE           # not 256-byte aligned
     assert _prefill(L, c, ws_bytes=1024) == sas.SAS_ERR_WORKSPACE
     assert _prefill(L, c, sel_count=FAKE + 1) == sas.SAS_ERR_INVALID_ARG
-    assert _prefill(L, _cfg(num_q_heads=24).c()) == sas.SAS_ERR_UNSUPPORTED  # odd group size (3)
-    assert _prefill(L, _cfg(token_budget=8192).c()) == sas.SAS_ERR_UNSUPPORTED
+    assert _prefill(L, _cfg(kv_dtype="f32").c()) == sas.SAS_ERR_UNSUPPORTED  # bf16 only
     assert _prefill(L, c, batch=0) == sas.SAS_OK
+
+
+@nogpu
+def test_gate_backward_validates_on_the_host(L):
+    def bwd(c, **kw):
+        a = dict(q=FAKE, w_q=FAKE, g_q=FAKE, w_k=FAKE, g_k=FAKE, sel=FAKE, cnt=FAKE, dout=FAKE, dwq=FAKE,
+                 dwk=FAKE, dgq=FAKE, dgk=FAKE, ws=FAKE, ws_bytes=256)
+        a.update(kw)
+        kv = sas._Kv(FAKE, FAKE, None, FAKE, 2, 4096, 0, 0, None)
+        return L.sas_gate_backward(ctypes.byref(c), a["q"], ctypes.byref(kv), a["w_q"], a["g_q"], a["w_k"],
+                                   a["g_k"], a["sel"], a["cnt"], a["dout"], a["dwq"], a["dwk"], a["dgq"],
+                                   a["dgk"], a["ws"], a["ws_bytes"], None)
+    gated = _cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS)
+    assert bwd(gated.c(), dout=None) == sas.SAS_ERR_INVALID_ARG
+    assert bwd(gated.c(), dwq=FAKE + 2) == sas.SAS_ERR_INVALID_ARG
+    assert bwd(gated.c(), ws=None) == sas.SAS_ERR_WORKSPACE
+    assert bwd(_cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS, token_budget=8192).c()) == sas.SAS_ERR_UNSUPPORTED
+    assert bwd(_cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS, kv_dtype="f32").c()) == sas.SAS_ERR_UNSUPPORTED
+    # the select-only mode gives the gate parameters no gradient: nothing to do
+    assert bwd(_cfg().c()) == sas.SAS_OK
 
 
 @pytest.mark.parametrize("gk16", [0, 1])

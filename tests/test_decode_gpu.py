@@ -136,6 +136,40 @@ def test_pool_keys_vs_oracle_and_raw_pooling():
                 assert np.allclose(raw[s, h, b, 256:], p[256:], rtol=1e-6, atol=1e-7)
 
 
+@pytest.mark.parametrize("gk16", [0, 1])
+def test_pool_keys_tiles_offsets_and_ragged_ends(gk16):
+    """Pooling calls that start mid-cache and cross the 128-block tiles of the
+    tensor-core projection: blocks blk_begin[s] .. blk_begin[s] + 199 that are
+    complete, every other row left alone."""
+    spec = DecodeSpec("pool_tiles", 2, 8, 2, [64 * 300, 64 * 250 + 17], (512,), capacity=64 * 300,
+                      block_offset_std=0.5, seed=19)
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, 512)
+    cfg.gate_keys_bf16 = gk16
+    ws = sas.make_workspace(cfg, DEV)
+    mg = T.gate_key_rows(spec)
+    gk = torch.full((2, 2, mg, 128), 7.0, dtype=sas.gate_key_dtype(cfg), device=DEV)
+    begin = torch.tensor([5, 130], dtype=torch.int32, device=DEV)
+    sas.pool_keys(cfg, T.kv_of(inp), inp["w_k"], inp["gamma_k"], gk, ws, blk_begin=begin, num_blocks=200)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    got = gk.double().cpu().numpy()
+    wk = inp["w_k"].double().cpu().numpy()
+    gam_k = inp["gamma_k"].double().cpu().numpy()
+    for s, L in enumerate(spec.seq_lens):
+        lo, hi = int(begin[s]), min(int(begin[s]) + 200, L // 64)
+        for h in range(2):
+            ks, _ = logical_kv(inp, s, h, L)
+            want = np.stack([O.gate_key(O.pool_block(ks[64 * b:64 * b + 64]), wk[h], gam_k, b) for b in range(lo, hi)])
+            if gk16:
+                want = O.round_to_bf16(want)
+                T.assert_close_rel(got[s, h, lo:hi], want, f"pooled s={s} h={h}", rtol=T.BF16_ULP)
+            else:
+                T.assert_close_rel(got[s, h, lo:hi], want, f"pooled s={s} h={h}")
+            keep = [b for b in range(mg) if not lo <= b < hi]
+            assert np.all(got[s, h, keep] == 7.0), "rows outside the range must be left alone"
+
+
 @pytest.mark.parametrize("dt", ["bf16", "f32"])
 def test_decode_step_pools_the_completed_block(dt):
     """With W_k / gamma_k the fused step writes the gate key of the block the

@@ -206,3 +206,40 @@ def test_prefill_qwen3_8b_32k_full_size():
     outs = [(0, 0, 0), (0, 0, 30), (1, 3, 31), (2, 5, 200), (3, 7, 511), (3, 2, 64)]
     sets = [t for t in every + spread if t not in outs]
     _check(spec, *res, sets + outs, sets_only=sets)
+
+
+def test_prefill_odd_group_small():
+    """Five query heads per KV head (the Qwen3-14B grouping): the last tile of
+    each group holds one head."""
+    spec = PrefillSpec("pf_g5", 1, 10, 2, 768, token_budget=320, seed=51)
+    res = _run(spec)
+    _check(spec, *res, [(0, h, i) for h in range(2) for i in range(12)])
+
+
+def test_prefill_odd_group_gated():
+    spec = PrefillSpec("pf_g5_gated", 2, 5, 1, 640, token_budget=256, seed=52)
+    res = _run(spec, gate_mode=sas.GATE_LOGSIGMOID_BIAS)
+    _check(spec, *res, [(s, 0, i) for s in range(2) for i in range(10)])
+
+
+def test_prefill_qwen3_14b_heads_8k():
+    """Qwen3-14B head layout (40 query / 8 KV heads), 8,192 tokens, budget
+    2,048: block lists of every query block of two pairs, outputs sampled."""
+    spec = PrefillSpec("pf_qwen3_14b_8k", 1, 40, 8, 8192, token_budget=2048, seed=53)
+    res = _run(spec)
+    nblk = spec.seq_len // 64
+    outs = [(0, 0, 5), (0, 7, 127), (0, 3, 64)]
+    sets = [t for t in [(0, 0, i) for i in range(nblk)] + [(0, 7, i) for i in range(nblk)] if t not in outs]
+    _check(spec, *res, sets + outs, sets_only=sets)
+
+
+@pytest.mark.parametrize("budget", [8192, 16384])
+def test_prefill_budgets_beyond_4096(budget):
+    """Budgets above 4,096 tokens (lists of up to 256 blocks; one attention
+    CTA per SM)."""
+    spec = PrefillSpec(f"pf_budget{budget}", 1, 4, 1, 64 * 300, token_budget=budget, seed=54)
+    res = _run(spec)
+    nblk = spec.seq_len // 64
+    outs = [(0, 0, 3), (0, 0, 200), (0, 0, nblk - 1)]
+    sets = [(0, 0, i) for i in range(nblk) if (0, 0, i) not in outs]
+    _check(spec, *res, sets + outs, sets_only=sets)
