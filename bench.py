@@ -461,7 +461,7 @@ def build_layers(R, rank, device, gate_mode=0, budgets=None, gk16=0):
     from gated_block_sparse_token_b200.workloads import make_decode_inputs, qwen3_4b_32k
 
     cfg = sas.Config(HQ, HKV, token_budget=BUDGET if budgets is None else max(budgets), gate_mode=gate_mode,
-                     gate_keys_bf16=gk16)
+                     gate_keys_bf16=gk16, static_weights=1)
     tb = None if budgets is None else torch.tensor(budgets, dtype=torch.int32, device=device)
     layers = []
     lens = None  # one length vector for every layer, as in a model's decode step
@@ -576,7 +576,7 @@ def run_long_context(args, rank, world, device, layers=2):
     n_app = spec0.appended
     full = spec0.seq_lens[0]
     start = full - n_app
-    cfg = sas.Config(spec0.hq, spec0.hkv, token_budget=4096)
+    cfg = sas.Config(spec0.hq, spec0.hkv, token_budget=4096, static_weights=1)
     Ls = []
     # one length vector per appended token, shared by the layers
     lens = [torch.full((spec0.batch,), start + t + 1, dtype=torch.int32, device=device) for t in range(n_app)]
@@ -655,7 +655,7 @@ def run_ragged(args, rank, world, device, layers=2):
     peak, peak_kind = measured_peaks()
     res = []
     for budget in (1024, 2048, 4096):
-        cfg = sas.Config(spec0.hq, spec0.hkv, token_budget=budget)
+        cfg = sas.Config(spec0.hq, spec0.hkv, token_budget=budget, static_weights=1)
         fn = lambda L, st: step(cfg, L, st)  # noqa: E731
         with torch.cuda.stream(stream):
             for L in Ls:

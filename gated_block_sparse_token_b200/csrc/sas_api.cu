@@ -21,7 +21,7 @@ namespace {
 
 using sas::kDim;
 
-constexpr int32_t kAbiVersion = 7;
+constexpr int32_t kAbiVersion = 8;
 constexpr size_t kStatusBytes = 256;  // status word + padding
 constexpr int kMaxBudget = 16384;
 constexpr int kMaxGateBlocks = 16384;
@@ -77,6 +77,7 @@ sas_status check_config(const sas_config* c) {
   if (c->gate_mode != SAS_GATE_SELECT_ONLY && c->gate_mode != SAS_GATE_LOGSIGMOID_BIAS)
     return SAS_ERR_INVALID_ARG;
   if (c->gate_keys_bf16 != 0 && c->gate_keys_bf16 != 1) return SAS_ERR_INVALID_ARG;
+  if (c->static_weights != 0 && c->static_weights != 1) return SAS_ERR_INVALID_ARG;
   return SAS_OK;
 }
 
@@ -187,6 +188,7 @@ void fill_common(sas::DecodeParams& p, const sas_config* cfg, int mg) {
   p.gate_scale = cfg->gate_scale;
   p.gated = cfg->gate_mode == SAS_GATE_LOGSIGMOID_BIAS ? 1 : 0;
   p.gk16 = cfg->gate_keys_bf16;
+  p.static_weights = cfg->static_weights;
   p.sm = sas::plan_decode_smem(p.G, mg, kClusterSize, kStages, p.max_sel,
                                cfg->kv_dtype == SAS_DTYPE_F32, p.gated != 0);
   sas::fill_rope_table(p.rope, cfg->rope_base);

@@ -11,15 +11,19 @@
 // plus the current block are attended.
 //
 // Work split of one cluster of CS CTAs (128 threads each) for (s, h):
-//   start    every load that does not depend on the sequence length (q, the
-//            CTA's W_q column slice, gains, RoPE frequencies) is issued first;
-//            then the length, and for a paged cache every page id of the
+//   start    the launch may overlap the kernel ahead on the stream
+//            (programmatic dependent launch): barriers are set up, and with
+//            static weights the W_q column slice and gains requested, before
+//            waiting for it; then every load that does not depend on the
+//            sequence length (q, the first gate-key chunks) is issued;
+//            the length, and for a paged cache every page id of the
 //            sequence, is validated.
 //   phase 0  each CTA computes 128/CS columns of v_g = q_g @ W_q[g] for the G
-//            query heads of the group (large groups: the W_q slice in two
-//            passes of ceil(G/2) heads) and stores them into every CTA of the
-//            cluster (st.async into distributed shared memory, bytes counted
-//            on the receiver's mbarrier); RMSNorm + RoPE -> q~_g.
+//            query heads of the group, one warp per head (large groups: the
+//            W_q slice in two passes of ceil(G/2) heads), and stores them into
+//            every CTA of the cluster (st.async into distributed shared
+//            memory, bytes counted on the receiver's mbarrier); RMSNorm +
+//            RoPE -> q~_g.
 //   phase 1  each CTA streams 1/CS of the gate keys k~_b (TMA bulk copies
 //            into a ring of 16 KiB stage slots), scores its blocks and stores
 //            each score into CTA 0.
@@ -53,11 +57,22 @@ namespace sas {
 // Phase-trace hook: thread 0 of each CTA stamps the global timer at phase
 // boundaries (tracing builds only).
 #ifdef SAS_PHASE_TRACE
+// Slot 0 holds the global timer at the CTA's start (for alignment across
+// CTAs) and slot 23 the SM clock there; slot 22 the global timer at the end;
+// every other slot the SM clock.
 #define SAS_TRACE(k)                                                                        \
   do {                                                                                      \
     const unsigned cta_ = blockIdx.y * gridDim.x + blockIdx.x;                              \
-    if (p.trace != nullptr && threadIdx.x == 0 && cta_ < static_cast<unsigned>(kTraceCtas)) \
-      p.trace[cta_ * kTraceSlots + (k)] = global_timer_ns();                               \
+    if (p.trace != nullptr && threadIdx.x == 0 && cta_ < static_cast<unsigned>(kTraceCtas)) { \
+      unsigned long long* t_ = p.trace + cta_ * kTraceSlots;                                \
+      if ((k) == 0) {                                                                       \
+        t_[0] = global_timer_ns();                                                          \
+        t_[23] = clock64();                                                                 \
+      } else {                                                                              \
+        t_[(k)] = clock64();                                                                \
+        if ((k) == 8) t_[22] = global_timer_ns();                                           \
+      }                                                                                     \
+    }                                                                                       \
   } while (0)
 #else
 #define SAS_TRACE(k) \
@@ -82,29 +97,110 @@ __device__ __forceinline__ float dot4(const float4 a, const float4 b, float acc)
 
 }  // namespace
 
-// Distributed exact Top-K of one cluster (the fused step's selection when
-// the sequence keeps at most kFastTopk historical blocks).  Every CTA holds
-// the (score, block) keys of its own gate-key rows in lkeys (plen[rank] of
-// them kept; keys are distinct, the block index breaks score ties toward the
-// lower block).  (1) each CTA ranks its keys by counting and sends its best
-// plen[rank], in descending order, to every CTA of the cluster (st.async into
-// gather[rank][.], bytes counted on bar); (2) every CTA ranks each received
-// candidate in the union -- its position in its own list plus, for each
-// other list, how many keys of that list beat it (binary search) -- and marks
-// the topk best in fmask (zeroed by the caller); (3) warp 0 turns the mask
-// into the ascending list sel[0 .. topk), then sel[topk] = cur.  The global
-// best topk always lie in the union (each is among its own CTA's best topk),
-// and a candidate outside them has at least topk union keys above it.
+// Bitonic merge of two descending lists of 32*E keys held by one warp (lane l
+// holds elements l + 32 i, i < E): the elementwise maximum of A and reversed B
+// holds the 32*E largest keys of both as a bitonic sequence, which the
+// cleaning stages sort descending.  Returns them in the same layout.
+template <int E>
+__device__ __forceinline__ void merge_desc(unsigned long long (&a)[E], const unsigned long long (&b)[E]) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long c[E];
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    // reversed B: element 32E-1-(l+32i) = lane 31-l, slot E-1-i
+    const unsigned long long br = __shfl_sync(0xffffffffu, b[E - 1 - i], 31 - lane);
+    c[i] = a[i] > br ? a[i] : br;
+  }
+#pragma unroll
+  for (int j = 16 * E; j > 0; j >>= 1) {
+    if (j >= 32) {  // partner in another slot of the same lane
+      const int js = j / 32;
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        if ((i & js) == 0) {
+          const unsigned long long x = c[i], y = c[i | js];
+          c[i] = x > y ? x : y;
+          c[i | js] = x > y ? y : x;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        const unsigned long long y = __shfl_xor_sync(0xffffffffu, c[i], j);
+        const bool keep_max = (lane & j) == 0;
+        c[i] = keep_max ? (c[i] > y ? c[i] : y) : (c[i] > y ? y : c[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < E; ++i) a[i] = c[i];
+}
+
+// Distributed exact Top-K of one cluster of 8 CTAs (the fused step's
+// selection when the sequence keeps at most kFastTopk historical blocks).
+// Every CTA holds the (score, block) keys of its own gate-key rows in lkeys
+// (keys are distinct: the block index breaks score ties toward the lower
+// block; key 0 sorts below every key).  (1) each CTA ranks its keys by
+// counting and sends its best plen[rank], in descending order, to every CTA
+// of the cluster (st.async into gather[rank][.], bytes counted on bar);
+// (2) every CTA merges the 8 sorted lists with a bitonic merge tree (four
+// warps, then two, then one; lists of 32*E keys, E = 1 or 2) -- the global
+// best topk always lie among them, each being among its own CTA's best topk
+// -- whose first topk are the kept blocks; (3) warp 0 sorts their block
+// ids ascending (a bitonic network over the warp) into sel[0 .. topk), then
+// sel[topk] = cur.  lkeys and gather are scratch from step (2) on.
 // Returns false if the candidates did not all arrive (bounded wait; the
 // timeout bit is then set).  Ends with a block-wide barrier.
-template <int CS>
-__device__ __noinline__ bool distributed_topk(const unsigned long long* lkeys, unsigned long long* gather,
-                                              uint32_t* fmask, const int* plen, int n, int topk, int cur,
-                                              int rank, int* sel, uint64_t* bar, uint32_t* status) {
+// Ascending bitonic sort of 32*E values held by one warp (lane l holds
+// elements l + 32 i, i < E).
+template <int E>
+__device__ __forceinline__ void warp_sort_asc(uint32_t (&x)[E]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32 * E; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {  // partner in another slot of the same lane
+        const int js = j / 32;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          if ((i & js) == 0) {
+            const bool asc = ((lane + 32 * i) & k) == 0;
+            const uint32_t lo = min(x[i], x[i | js]), hi = max(x[i], x[i | js]);
+            x[i] = asc ? lo : hi;
+            x[i | js] = asc ? hi : lo;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const uint32_t y = __shfl_xor_sync(0xffffffffu, x[i], j);
+          const bool asc = ((lane + 32 * i) & k) == 0;
+          const bool lower = (lane & j) == 0;
+          x[i] = (lower == asc) ? min(x[i], y) : max(x[i], y);
+        }
+      }
+    }
+  }
+}
+
+template <int E>
+__device__ __forceinline__ void load_list(unsigned long long (&v)[E], const unsigned long long* lst, int len) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < E; ++i) v[i] = (lane + 32 * i < len) ? lst[lane + 32 * i] : 0ull;
+}
+
+template <int CS, int E>
+__device__ __noinline__ bool distributed_topk(unsigned long long* lkeys, unsigned long long* gather,
+                                              const int* plen, int topk, int cur,
+                                              int rank, int* sel, uint64_t* bar, uint32_t* status,
+                                              unsigned long long* tr) {
+  static_assert(CS == 8, "the merge tree has three levels");
+  constexpr int LEN = 32 * E;  // list length of the merge
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // rows this CTA holds (the caller's plen is min(topk, rows)); the counting
-  // ranks only need the first plen[rank] positions, over all of its rows
-  const int nl = plen[CS];  // passed in plen[CS]: this CTA's row count
+  // rows this CTA holds (plen[CS]); only the first plen[rank] ranks are sent
+  const int nl = plen[CS];
   const int P = plen[rank];
   const int split = (nl <= 32) ? 4 : ((nl <= 64) ? 2 : 1);  // threads per key
   for (int base0 = 0; base0 < nl * split; base0 += kThreads) {
@@ -113,8 +209,10 @@ __device__ __noinline__ bool distributed_topk(const unsigned long long* lkeys, u
     const bool live = i < nl;
     const unsigned long long x = live ? lkeys[i] : 0ull;
     int r = 0;
-    if (live)
+    if (live) {
+#pragma unroll 8
       for (int jj = part; jj < nl; jj += split) r += (lkeys[jj] > x) ? 1 : 0;
+    }
     if (split >= 2) r += __shfl_xor_sync(0xffffffffu, r, 1);
     if (split >= 4) r += __shfl_xor_sync(0xffffffffu, r, 2);
     if (live && part == 0 && r < P) {
@@ -123,55 +221,44 @@ __device__ __noinline__ bool distributed_topk(const unsigned long long* lkeys, u
         st_async_u64(dsmem_addr(gather + rank * kFastTopk + r, dst), x, dsmem_addr(bar, dst));
     }
   }
+  if (tr != nullptr && tid == 0) tr[0] = clock64();  // candidates sent
   bool ok = mbar_wait_cluster(bar, 0, status);  // every CTA's candidates
-  ok = __syncthreads_and(ok) != 0;
+  ok = __syncthreads_and(ok) != 0;             // (and every read of lkeys is done)
   if (!ok) return false;
-  for (int e = tid; e < CS * kFastTopk; e += kThreads) {
-    const int src = e / kFastTopk, pos = e - src * kFastTopk;
-    if (pos >= plen[src]) continue;
-    const unsigned long long x = gather[e];
-    int rk = pos;
+  if (tr != nullptr && tid == 0) tr[1] = clock64();  // candidates in
+  // merge tree: level 1 into lkeys (4 lists), level 2 into gather (2 lists)
+  unsigned long long a[E], b[E];
+  {
+    load_list<E>(a, gather + (2 * warp) * kFastTopk, plen[2 * warp]);
+    load_list<E>(b, gather + (2 * warp + 1) * kFastTopk, plen[2 * warp + 1]);
+    merge_desc<E>(a, b);
 #pragma unroll
-    for (int r = 0; r < CS; ++r) {
-      if (r == src) continue;
-      const unsigned long long* lst = gather + r * kFastTopk;
-      int lo = 0;  // keys lst[0 .. lo) beat x (lists are descending)
-#pragma unroll
-      for (int step = kFastTopk; step > 0; step >>= 1)
-        if (lo + step <= plen[r] && lst[lo + step - 1] > x) lo += step;
-      rk += lo;
-    }
-    if (rk < topk) {
-      const uint32_t b = ~static_cast<uint32_t>(x & 0xFFFFFFFFull);
-      atomicOr(&fmask[b >> 5], 1u << (b & 31));
-    }
+    for (int i = 0; i < E; ++i) lkeys[warp * LEN + lane + 32 * i] = a[i];
   }
   __syncthreads();
-  // ascending list from the mask (warp 0; lane l owns words wpl*l ..)
-  if (warp == 0) {
-    const int words = (n + 31) / 32;
-    const int wpl = (words + 31) / 32;
-    int cnt = 0;
-    for (int w = 0; w < wpl; ++w) {
-      const int wi = wpl * lane + w;
-      cnt += (wi < words) ? __popc(fmask[wi]) : 0;
-    }
-    int inc = cnt;
+  if (warp < 2) {
+    load_list<E>(a, lkeys + (2 * warp) * LEN, LEN);
+    load_list<E>(b, lkeys + (2 * warp + 1) * LEN, LEN);
+    merge_desc<E>(a, b);
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
-    }
-    int pos = inc - cnt;
-    for (int w = 0; w < wpl; ++w) {
-      const int wi = wpl * lane + w;
-      uint32_t mm = (wi < words) ? fmask[wi] : 0u;
-      while (mm != 0u) {
-        if (pos < topk) sel[pos] = 32 * wi + __ffs(mm) - 1;  // exactly topk bits are set
-        ++pos;
-        mm &= mm - 1u;
-      }
-    }
+    for (int i = 0; i < E; ++i) gather[warp * LEN + lane + 32 * i] = a[i];
+  }
+  __syncthreads();
+  if (warp == 0) {
+    load_list<E>(a, gather, LEN);
+    load_list<E>(b, gather + LEN, LEN);
+    merge_desc<E>(a, b);
+    if (tr != nullptr && lane == 0) tr[2] = clock64();  // merged
+    // the first topk of the merged list are the kept blocks: their ids,
+    // sorted ascending (the rest sort last), give the list
+    uint32_t blk[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i)
+      blk[i] = (lane + 32 * i < topk) ? ~static_cast<uint32_t>(a[i] & 0xFFFFFFFFull) : 0xFFFFFFFFu;
+    warp_sort_asc<E>(blk);
+#pragma unroll
+    for (int i = 0; i < E; ++i)
+      if (lane + 32 * i < topk) sel[lane + 32 * i] = static_cast<int>(blk[i]);
     if (lane == 0) sel[topk] = cur;
   }
   __syncthreads();
@@ -188,7 +275,8 @@ __global__ void __launch_bounds__(kThreads, 4)
   constexpr bool kF32 = std::is_same<T, float>::value;
   constexpr int kDpc = kDim / CS;               // output / W_q columns per CTA
   constexpr int kTilesPerBlock = kF32 ? 4 : 2;  // 16 KiB tiles per K+V block
-  static_assert(kDpc % 8 == 0, "cluster size must divide 128 into 16-byte slices");
+  static_assert(kDpc == 16, "the gate-query GEMV maps 8 row groups x 4 column quads to a warp");
+  static_assert((CS & (CS - 1)) == 0, "power-of-two clusters");
 
   cg::cluster_group cluster = cg::this_cluster();
   SAS_TRACE(0);
@@ -252,6 +340,8 @@ __global__ void __launch_bounds__(kThreads, 4)
   // its first NST chunks that lie inside the gate-key cache before the length
   // is known (a chunk past the historical blocks is then not scored).
   const int gk_rows = p.gk16 ? 2 * kGkChunk : kGkChunk;
+  const int gk_shift = p.gk16 ? 6 : 5;  // log2(gk_rows)
+  static_assert(kGkChunk == 32, "gate-key chunks of 32 fp32 or 64 bf16 rows");
   const uint32_t gk_row_bytes = p.gk16 ? kDim * 2u : kDim * 4u;
   const uint8_t* gk_pair = static_cast<const uint8_t*>(p.gate_keys) + static_cast<size_t>(pair) * p.mg * gk_row_bytes;
   int nspec = 0;  // chunks requested before the length is known (tiles 0 .. nspec-1)
@@ -259,17 +349,25 @@ __global__ void __launch_bounds__(kThreads, 4)
     while (nspec < NST && (rank + nspec * CS) * gk_rows < p.mg) ++nspec;
 
   // ------------------------------------------------------------ prologue copies
-  // Thread 0 loads the sequence length first (one request per CTA: every CTA
-  // of the grid reads the same few bytes) and, while it is in flight,
-  // requests everything that does not depend on it, asynchronously: q of the
-  // group (bulk), gamma_q (bulk), the W_q column slice of this CTA (one 2-D
-  // TMA box per head) and its first gate-key chunks.
+  // The launch may overlap the kernels ahead on the stream (programmatic
+  // dependent launch).  Thread 0 initialises the barriers before waiting for
+  // them; when the caller declares the weights static, it also requests
+  // gamma_q, gamma_k and the CTA's W_q column slice (one 2-D TMA box per
+  // head) before the wait.  q, the length, the budget, the gate keys and
+  // the cache are always read after it.
   int* len_s = reinterpret_cast<int*>(qbar);  // qbar is written only after the validation
+  auto issue_weights = [&]() {
+    if (MODE != kModeAttend) {
+      bulk_g2s(gam_s, p.gamma_q, kDim * 4, bar_pro);
+      for (int g = 0; g < wq_heads; ++g)
+        tma_load_2d(wq_s + static_cast<size_t>(g) * kDim * kDpc, &tmw, rank * kDpc, (h * G + g) * kDim, bar_pro);
+    }
+    if (pool_on) bulk_g2s(gamk_s, p.gamma_k, kDim * 4, bar_pro);
+  };
   if (tid == 0) {
-    const int L0 = p.kv.seq_lens[s];
-    const int topk0 = (MODE == kModeFused) ? p.kv.topk_of(s) : 0;  // this sequence's budget
-    // the descriptors of the maps this mode uses are fetched while the plain
-    // copies go out
+    // the kernel behind this one may be scheduled from now on: it reads
+    // nothing this grid writes before this grid has completed
+    griddep_launch_dependents();
     if (MODE != kModeAttend) prefetch_tensormap(&tmw);
     if constexpr (!kF32 && MODE != kModeGate) {
       prefetch_tensormap(&tmk);
@@ -283,17 +381,17 @@ __global__ void __launch_bounds__(kThreads, 4)
     if (MODE != kModeAttend) tx += static_cast<uint32_t>(wq_heads * kDim * kDpc * 2 + kDim * 4);
     if (pool_on) tx += kDim * 4;
     mbar_arrive_expect_tx(bar_pro, tx);
+    // the gate query v arrives from every CTA whatever the length holds
+    if (MODE != kModeAttend) mbar_arrive_expect_tx(bar_v, static_cast<uint32_t>(G * kDim * 4));
+    if (p.static_weights) issue_weights();
+  }
+  griddep_wait();
+  if (tid == 0) {
+    const int L0 = p.kv.seq_lens[s];
+    const int topk0 = (MODE == kModeFused) ? p.kv.topk_of(s) : 0;  // this sequence's budget
     bulk_g2s(qraw, static_cast<const T*>(p.q) + (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim,
-             qbytes, bar_pro);
-    if (MODE != kModeAttend) bulk_g2s(gam_s, p.gamma_q, kDim * 4, bar_pro);
-    if (pool_on) bulk_g2s(gamk_s, p.gamma_k, kDim * 4, bar_pro);
-    if (MODE != kModeAttend) {
-      for (int g = 0; g < wq_heads; ++g)
-        tma_load_2d(wq_s + static_cast<size_t>(g) * kDim * kDpc, &tmw, rank * kDpc, (h * G + g) * kDim,
-                    bar_pro);
-      // the gate query v arrives from every CTA whatever the length holds
-      mbar_arrive_expect_tx(bar_v, static_cast<uint32_t>(G * kDim * 4));
-    }
+             G * kDim * static_cast<uint32_t>(sizeof(T)), bar_pro);
+    if (!p.static_weights) issue_weights();
     for (int k = 0; k < nspec; ++k) {
       const int r0 = (rank + k * CS) * gk_rows;
       const uint32_t bytes = static_cast<uint32_t>(min(gk_rows, p.mg - r0)) * gk_row_bytes;
@@ -315,8 +413,9 @@ __global__ void __launch_bounds__(kThreads, 4)
 
   // ------------------------------------------------------------ phase 0: gate query projection
   // v_g = q_g @ W_q[g] needs no length: it runs while the length load is in
-  // flight.  Two threads per output column (rows 0..63 and 64..127),
-  // combined by shuffle; every CTA of the cluster receives every column.
+  // flight.  One warp per head: each lane accumulates 16 rows (8 apart) of
+  // 4 columns, shuffles sum the 8 row groups, and every CTA of the cluster
+  // receives every column (one 16-byte asynchronous store per lane).
   // Large groups take the W_q slice in two passes through the same region
   // (the second copy is requested once every read of the first is done).
   // the cluster barrier first: every thread of the cluster has arrived, so
@@ -325,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   // stores reach it
   cluster_wait();
   const bool pro_ok = mbar_wait(bar_pro, 0, p.status);
+  SAS_TRACE(21);  // prologue copies in
   if (MODE != kModeAttend) {
     bool wq_ok = pro_ok;
     for (int g0 = 0; g0 < G; g0 += wq_heads) {
@@ -340,27 +440,38 @@ __global__ void __launch_bounds__(kThreads, 4)
         }
         wq_ok = mbar_wait(bar_wq2, 0, p.status) && wq_ok;
       }
-      for (int o = tid; o < 2 * gn * kDpc; o += kThreads) {
-        const int half = o & 1;
-        const int oc = o >> 1;
-        const int gl = oc / kDpc;  // head within this pass
-        const int j = oc - gl * kDpc;
+      // warp w: heads w, w + 4, ..; lane (rg, cq): rows rg, rg + 8, .., rg +
+      // 120 of columns 4 cq .. 4 cq + 3 of the CTA's slice (one load step
+      // reads 8 consecutive 32-byte rows: no bank conflicts)
+      const int cq = lane & 3, rg = lane >> 2;
+      for (int gl = warp; gl < gn; gl += kWarps) {
         const int g = g0 + gl;
-        const T* qrow = qraw + g * kDim + half * 64;
-        const __nv_bfloat16* wcol = wq_s + (static_cast<size_t>(gl) * kDim + half * 64) * kDpc + j;
-        float a4[4] = {0.f, 0.f, 0.f, 0.f};
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         if (wq_ok) {
-#pragma unroll 16
-          for (int i = 0; i < 64; ++i)
-            a4[i & 3] = fmaf(to_float(qrow[i]), __bfloat162float(wcol[i * kDpc]), a4[i & 3]);
-        }
-        float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        if (half == 0) {
+          const __nv_bfloat16* wrow = wq_s + (static_cast<size_t>(gl) * kDim + rg) * kDpc + 4 * cq;
+          const T* qcol = qraw + g * kDim + rg;
 #pragma unroll
-          for (int r = 0; r < CS; ++r)
-            st_async_f32(dsmem_addr(qv + g * kDim + rank * kDpc + j, r), acc, dsmem_addr(bar_v, r));
+          for (int u = 0; u < 16; ++u) {
+            const float x = to_float(qcol[8 * u]);
+            const uint2 w = *reinterpret_cast<const uint2*>(wrow + 8 * u * kDpc);
+            a0 = fmaf(x, __uint_as_float(w.x << 16), a0);
+            a1 = fmaf(x, __uint_as_float(w.x & 0xffff0000u), a1);
+            a2 = fmaf(x, __uint_as_float(w.y << 16), a2);
+            a3 = fmaf(x, __uint_as_float(w.y & 0xffff0000u), a3);
+          }
         }
+        if (gl == 0) SAS_TRACE(24);  // thread 0: products summed
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+          a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+          a2 += __shfl_xor_sync(0xffffffffu, a2, o);
+          a3 += __shfl_xor_sync(0xffffffffu, a3, o);
+        }
+        if (gl == 0) SAS_TRACE(25);  // thread 0: row groups combined
+        // the lanes of row group r deliver the four columns to CTA r
+        st_async_v4_f32(dsmem_addr(qv + g * kDim + rank * kDpc + 4 * cq, rg), a0, a1, a2, a3,
+                        dsmem_addr(bar_v, rg));
       }
     }
   }
@@ -426,15 +537,15 @@ __global__ void __launch_bounds__(kThreads, 4)
   // gate-key chunks of this CTA: global chunks rank, rank + CS, ... below
   // ceil(n / gk_rows); the speculative ones are tiles 0 .. nspec-1 whatever
   // the length turned out to be
-  const int nch_all = (n + gk_rows - 1) / gk_rows;
+  const int nch_all = (n + gk_rows - 1) >> gk_shift;
   const int nch_need = (MODE == kModeAttend || nch_all <= rank) ? 0 : (nch_all - rank + CS - 1) / CS;
   const int nchunks = (MODE == kModeAttend) ? 0 : max(nch_need, nspec);
   // historical blocks (gate-key rows) CTA r scores: its full chunks plus the
   // partial last chunk if it owns it
   auto rows_of = [&](int r) -> int {
-    const int full = n / gk_rows, rem = n - full * gk_rows;
+    const int full = n >> gk_shift, rem = n & (gk_rows - 1);
     const int nf = (full > r) ? (full - r + CS - 1) / CS : 0;
-    return nf * gk_rows + ((rem > 0 && full % CS == r) ? rem : 0);
+    return nf * gk_rows + ((rem > 0 && (full & (CS - 1)) == r) ? rem : 0);
   };
   // Top-K route: nothing to choose (a 64-token budget, or every historical
   // block kept); the distributed selection; or every score to rank 0, which
@@ -447,7 +558,6 @@ __global__ void __launch_bounds__(kThreads, 4)
   const bool own_cur = (m > 0) && ((m - 1) % CS == rank);
   unsigned long long* lkeys = reinterpret_cast<unsigned long long*>(base + p.sm.r_lkeys);
   unsigned long long* gather = reinterpret_cast<unsigned long long*>(base + p.sm.r_gather);
-  uint32_t* fmask = reinterpret_cast<uint32_t*>(base + p.sm.r_fmask);
 
   // bytes this CTA will receive from the cluster (bad is uniform over it)
   if (tid == 0) {
@@ -471,8 +581,6 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
     if (MODE != kModeGate) mbar_arrive_expect_tx(bar_m, static_cast<uint32_t>(CS * G * (kDpc + 2) * 4));
   }
-  if (sel_fast && !bad)
-    for (int w = tid; w < (n + 31) / 32; w += kThreads) fmask[w] = 0u;  // W_q reads are done
 
   // list entry e of this CTA -> block id (the current block first if owned)
   auto entry_index = [&](int e) -> int {
@@ -489,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 4)
   // are gate-key chunks, then kTilesPerBlock tiles per list entry.  Thread 0
   // issues tile t once tile t - NST has been released by every thread.
   int issued = nspec;  // meaningful in thread 0 only
-  auto issue = [&](int t) {
+  auto issue = [&](int t, bool traced) {
     const int slot = t % NST;
     uint8_t* dst = slots + slot * kTileBytes;
     if (t < nchunks) {
@@ -504,7 +612,9 @@ __global__ void __launch_bounds__(kThreads, 4)
     const int e = k / kTilesPerBlock;
     const int part = k - e * kTilesPerBlock;
     const long long row0 = rows_cached ? rows_s[e] : p.kv.block_row(s, h, entry_block(e));
+    if (traced) SAS_TRACE(9);
     mbar_arrive_expect_tx(&bars[slot], kTileBytes);
+    if (traced) SAS_TRACE(19);
     if constexpr (kF32) {
       const float* src = static_cast<const float*>(part < 2 ? p.kv.k : p.kv.v) +
                          (row0 + (part & 1) * 32) * kDim;
@@ -512,13 +622,21 @@ __global__ void __launch_bounds__(kThreads, 4)
     } else {
       const CUtensorMap* map = (part == 0) ? &tmk : &tmv;
       tma_load_2d(dst, map, 0, static_cast<int>(row0), &bars[slot]);
+      if (traced) SAS_TRACE(26);
       tma_load_2d(dst + 8192, map, 64, static_cast<int>(row0), &bars[slot]);
     }
   };
-  auto pump = [&](int consumed, int known) {
+  auto pump = [&](int consumed, int known, bool traced = false) {
     if (tid != 0) return;
+    if (traced) SAS_TRACE(27);
     fence_proxy_async_smem();
-    while (issued < known && issued < consumed + NST) issue(issued++);
+    if (traced) SAS_TRACE(28);
+    bool first = traced;
+    while (issued < known && issued < consumed + NST) {
+      issue(issued++, first);
+      first = false;
+    }
+    if (traced) SAS_TRACE(29);
   };
 
   // before the selection only the gate-key chunks and the current block are known
@@ -535,15 +653,19 @@ __global__ void __launch_bounds__(kThreads, 4)
   }
 
   // ------------------------------------------------------------ gate query: norm and RoPE
+  // the rotation at position c needs only the length: computed while v is
+  // still on its way
+  float c0 = 1.f, s0 = 0.f, c1 = 1.f, s1 = 0.f;
+  if (MODE != kModeAttend && !bad) {
+    rope_cos_sin(th0, c, c0, s0);
+    rope_cos_sin(th1, c, c1, s1);
+  }
   if (MODE != kModeAttend) mbar_wait_cluster(bar_v, 0, p.status);  // every column of v is here
   SAS_TRACE(2);
 
   if (MODE != kModeAttend) {
     if (!bad) {
       // Q normalisation (RMSNorm, gain gamma_q) and gate RoPE at position c.
-      float c0, s0, c1, s1;
-      rope_cos_sin(th0, c, c0, s0);
-      rope_cos_sin(th1, c, c1, s1);
       for (int g = warp; g < G; g += kWarps) {
         float x[4];
         float ss = 0.f;
@@ -587,9 +709,11 @@ __global__ void __launch_bounds__(kThreads, 4)
       for (int i = 0; i < 4; ++i)
         qr[i] = *reinterpret_cast<const float4*>(qbar + sub * 16 + ((i + rot) & 3) * 4);
     }
+    SAS_TRACE(14);  // q~ and the head mean ready
     for (int ci = 0; ci < nchunks; ++ci) {
       const int slot = ci % NST;
       const bool ok = mbar_wait(&bars[slot], (ci / NST) & 1, p.status);
+      if (ci == 0) SAS_TRACE(15);  // first gate-key chunk in
       const int b0 = (rank + ci * CS) * gk_rows;
       const int cntb = max(0, min(gk_rows, n - b0));  // 0 for a speculative chunk past n
       const float* gk = reinterpret_cast<const float*>(slots + slot * kTileBytes);
@@ -657,8 +781,14 @@ __global__ void __launch_bounds__(kThreads, 4)
         if (act && sub == 0 && p.group_scores != nullptr)
           p.group_scores[static_cast<size_t>(pair) * p.mg + b0 + bb] = S;
       }
-      __syncthreads();
-      pump(ci + 1, known);
+      if (ci == 0) SAS_TRACE(30);  // first chunk scored (thread 0)
+      // chunks that all fit the ring (requested up front) need no slot
+      // recycling: one barrier after the last
+      if (nchunks > NST || ci == nchunks - 1) {
+        __syncthreads();
+        if (ci == 0) SAS_TRACE(31);
+        pump(ci + 1, known);
+      }
     }
   }
   SAS_TRACE(3);
@@ -701,16 +831,25 @@ __global__ void __launch_bounds__(kThreads, 4)
       // Distributed exact Top-K.  (1) each CTA ranks its own (score, block)
       // keys by counting (keys are distinct: the block index breaks ties) and
       // sends its best min(topk, rows) in descending order to every CTA;
-      // (2) every CTA ranks each received candidate in the union -- its
-      // position in its own list plus, for each other list, how many keys of
-      // that list beat it (binary search) -- and keeps the topk best as a
-      // bit mask; (3) the mask gives the ascending list.  The global best
-      // topk always lie in the union: each is among its own CTA's best topk.
+      // (2) every CTA merges the sorted lists (bitonic merge tree) and keeps
+      // the topk best; (3) their block ids, sorted, give the ascending list.
+      // The global best topk always lie in the union: each is among its own
+      // CTA's best topk.
       int plen[CS + 1];  // kept candidates of every CTA, then this CTA's row count
 #pragma unroll
       for (int r = 0; r < CS; ++r) plen[r] = min(topk, rows_of(r));
       plen[CS] = rows_of(rank);
-      list_ok = distributed_topk<CS>(lkeys, gather, fmask, plen, n, topk, c, rank, sel, bar_sc, p.status);
+      SAS_TRACE(10);  // scores of this CTA done
+#ifdef SAS_PHASE_TRACE
+      unsigned long long* ttr = (p.trace != nullptr && blockIdx.y * gridDim.x + blockIdx.x < kTraceCtas)
+                                    ? p.trace + (blockIdx.y * gridDim.x + blockIdx.x) * kTraceSlots + 11
+                                    : nullptr;
+#else
+      unsigned long long* ttr = nullptr;
+#endif
+      list_ok = (topk <= 32)
+                    ? distributed_topk<CS, 1>(lkeys, gather, plen, topk, c, rank, sel, bar_sc, p.status, ttr)
+                    : distributed_topk<CS, 2>(lkeys, gather, plen, topk, c, rank, sel, bar_sc, p.status, ttr);
       __syncthreads();
       SAS_TRACE(18);
       if (rank == 0) {
@@ -762,12 +901,12 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
     known = nchunks + kTilesPerBlock * cnt_mine;
     SAS_TRACE(20);  // list in hand
-    pump(nchunks, known);
-    if (paged) {
-      // every later issue follows a block-wide barrier, which publishes these
-      for (int e = tid; e < cnt_mine; e += kThreads) rows_s[e] = p.kv.block_row(s, h, entry_block(e));
-      rows_cached = true;
-    }
+    // the cache rows of this CTA's entries, looked up in parallel (paged:
+    // one page-table read each), so that issuing a tile reads one word
+    for (int e = tid; e < cnt_mine; e += kThreads) rows_s[e] = p.kv.block_row(s, h, entry_block(e));
+    __syncthreads();
+    rows_cached = true;
+    pump(nchunks, known, true);
     if (gated && !bad) {
       // gated mode: each CTA computes the gates of its own list entries,
       // log(sigmoid(s_gb)), s_gb = (q~_g . k~_b) * gate_scale, while its K/V
@@ -1258,13 +1397,17 @@ cudaError_t launch_cluster(const DecodeParams& p, const CUtensorMap& tmk, const 
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = static_cast<size_t>(p.sm.total);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CS;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the CTAs may start while the kernel ahead
+  // on the stream drains; the kernel waits for it before reading its inputs
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, decode_cluster_kernel<T, OutT, CS, NST, MODE>, p, tmk, tmv, tmw,
                             tmwk);
 }

@@ -142,6 +142,26 @@ __device__ __forceinline__ void st_async_u64(uint32_t raddr, unsigned long long 
                : "memory");
 }
 
+// Four consecutive fp32 values (a 16-byte aligned remote address) in one
+// asynchronous store, 16 bytes completed on the receiver's barrier.
+__device__ __forceinline__ void st_async_v4_f32(uint32_t raddr, float a, float b, float c, float d, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   raddr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
+               : "memory");
+}
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before
+// the kernel ahead of it on the stream has finished.  griddep_wait() returns
+// once every such prerequisite grid has completed and its memory operations
+// are visible (at once when there is none); griddep_launch_dependents() lets
+// the kernel behind this one on the stream be scheduled from here on.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void fence_acq_rel_cluster() {
   asm volatile("fence.acq_rel.cluster;" ::: "memory");
 }

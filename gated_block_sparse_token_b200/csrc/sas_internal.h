@@ -58,7 +58,6 @@ struct DecodeSmem {
   // distributed Top-K (phases 1-2; over keys.., like the rank-0 selection)
   int r_lkeys;   // uint64 [kFastRows] this CTA's (score, block) keys
   int r_gather;  // uint64 [CS][kFastTopk] sorted local candidates of every CTA
-  int r_fmask;   // uint32 [(mg + 31) / 32] selected blocks
   int total;     // bytes to request, including alignment slack
 };
 
@@ -111,8 +110,7 @@ inline DecodeSmem plan_decode_smem_heads(int G, int mg, int cs, int nst, int max
   p.r_scan = p.r_selbits + up16((mg + 31) / 32 * 4);
   p.r_lkeys = p.r_keys;
   p.r_gather = p.r_lkeys + kFastRows * 8;
-  p.r_fmask = p.r_gather + cs * kFastTopk * 8;
-  const int end_fast = p.r_fmask + up16((mg + 31) / 32 * 4);
+  const int end_fast = p.r_gather + cs * kFastTopk * 8;
   const int end24 = std::max(std::max(p.r_scan + 16 * 4, end_fast), p.r_wk + kPool * dpc * 2);
   p.total = std::max(end01, end24) + 1024;
   return p;
@@ -152,6 +150,10 @@ struct DecodeParams {
   const float* gamma_k;  // fused pooling of a completed current block (null: off)
   void* gate_keys_out;   // same array as gate_keys, written at row c when pooling
   int gk16;              // gate keys stored as bf16
+  // 1: W_q, gamma_q and gamma_k are read before the kernels ahead on the
+  // stream have finished (the caller guarantees that none writes them);
+  // 0: every input is read after they have finished
+  int static_weights;
   KvView kv;
   float* head_scores;
   float* group_scores;
@@ -258,7 +260,7 @@ constexpr int kPoolWkBytes = kPool * kDim * 2;  // W_k of one KV head, bf16 (96 
 
 // Phase-trace builds (-DSAS_PHASE_TRACE) record per-CTA timestamps after the
 // status word; ordinary builds compile the hooks out.
-constexpr int kTraceSlots = 24;
+constexpr int kTraceSlots = 32;
 constexpr int kTraceCtas = 4096;
 
 // Launchers (return the cudaError_t of the launch).

@@ -18,7 +18,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 # SAS_LIBRARY selects another build of the same ABI (e.g. the phase-trace build).
 LIB_PATH = os.environ.get("SAS_LIBRARY", os.path.join(_HERE, "libsas.so"))
-ABI_VERSION = 7             # the include/sas.h this binding marshals for
+ABI_VERSION = 8             # the include/sas.h this binding marshals for
 
 SAS_OK = 0
 SAS_ERR_INVALID_ARG = 1
@@ -50,7 +50,8 @@ class _Config(ctypes.Structure):
                 ("rope_base", ctypes.c_float), ("norm_eps", ctypes.c_float),
                 ("attn_scale", ctypes.c_float), ("gate_scale", ctypes.c_float),
                 ("kv_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
-                ("gate_mode", ctypes.c_int32), ("gate_keys_bf16", ctypes.c_int32)]
+                ("gate_mode", ctypes.c_int32), ("gate_keys_bf16", ctypes.c_int32),
+                ("static_weights", ctypes.c_int32)]
 
 
 class _Kv(ctypes.Structure):
@@ -136,12 +137,16 @@ class Config:
     gate_hidden: int = 128
     gate_mode: int = 0        # GATE_SELECT_ONLY or GATE_LOGSIGMOID_BIAS
     gate_keys_bf16: int = 0   # 1: the gate-key cache is bf16 (else fp32)
+    # 1: w_q, gamma_q, w_k and gamma_k are never written while decode kernels
+    # may run, so the kernels read them before the kernels ahead of them on
+    # the stream have finished; 0: every input after those have finished
+    static_weights: int = 0
 
     def c(self) -> _Config:
         return _Config(self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
                        self.gate_hidden, self.token_budget, self.rope_base, self.norm_eps,
                        self.attn_scale, self.gate_scale, _DT[self.kv_dtype], _DT[self.out_dtype],
-                       self.gate_mode, self.gate_keys_bf16)
+                       self.gate_mode, self.gate_keys_bf16, self.static_weights)
 
     @property
     def group(self) -> int:

@@ -118,6 +118,16 @@ typedef struct {
                               nearest-even when written (half the bytes the
                               scores stream).  Every call that reads or writes
                               gate keys follows it. */
+  int32_t static_weights; /* 0 (default) or 1.  The decode kernels are launched
+                            with programmatic stream serialization: they may
+                            start while kernels ahead of them on the stream
+                            are still running, and read their inputs and
+                            write their outputs only once those have
+                            finished.  With 1, the caller guarantees that
+                            w_q, gamma_q, w_k and gamma_k are not written by
+                            any kernel that may still be running (weights of
+                            an inference model never are), and the kernels
+                            read them before that point. */
 } sas_config;
 
 /* KV cache description (device pointers, caller-owned). */

@@ -17,9 +17,9 @@ int main() {
             std::printf(
                 "G=%d mg=%d budget=%d f32=%d gated=%d wq_heads=%d slots=%d sel=%d rows=%d gbias=%d qraw=%d qbar=%d pml=%d "
                 "gam=%d bars=%d r_qv=%d r_wq=%d r_inbox=%d r_keys=%d r_hist=%d r_selbits=%d r_scan=%d "
-                "r_lkeys=%d r_gather=%d r_fmask=%d total=%d ok=%d\n",
+                "r_lkeys=%d r_gather=%d total=%d ok=%d\n",
                 G, mg, b, f32, gated, p.wq_heads, p.slots, p.sel, p.rows, p.gbias, p.qraw, p.qbar, p.pml, p.gam, p.bars, p.r_qv,
-                p.r_wq, p.r_inbox, p.r_keys, p.r_hist, p.r_selbits, p.r_scan, p.r_lkeys, p.r_gather, p.r_fmask, p.total,
+                p.r_wq, p.r_inbox, p.r_keys, p.r_hist, p.r_selbits, p.r_scan, p.r_lkeys, p.r_gather, p.total,
                 sas::decode_smem_aligned(p, G, sas::kDim / 8) ? 1 : 0);
           }
   return 0;

@@ -61,6 +61,7 @@ int main(void) {
   printf("sizeof.sas_config %zu\nsizeof.sas_kv %zu\n", sizeof(sas_config), sizeof(sas_kv));
   O(sas_config, token_budget); O(sas_config, rope_base); O(sas_config, gate_scale);
   O(sas_config, kv_dtype); O(sas_config, out_dtype); O(sas_config, gate_mode); O(sas_config, gate_keys_bf16);
+  O(sas_config, static_weights);
   O(sas_kv, block_table); O(sas_kv, seq_lens); O(sas_kv, batch); O(sas_kv, capacity);
   O(sas_kv, num_pages); O(sas_kv, max_blocks_per_seq); O(sas_kv, token_budgets);
   return 0;
@@ -84,7 +85,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(L):
-    assert sas.abi_version() == sas.ABI_VERSION == 7
+    assert sas.abi_version() == sas.ABI_VERSION == 8
     for st in range(7):
         assert len(sas.status_string(st)) > 0
     assert sas.status_string(sas.SAS_OK) == "ok"
@@ -135,6 +136,7 @@ def _decode(L, cfg, kv=None, ws_bytes=256, ws=FAKE, q=FAKE, out=FAKE, mg=64):
     (dict(gate_mode=2), sas.SAS_ERR_INVALID_ARG),
     (dict(gate_mode=-1), sas.SAS_ERR_INVALID_ARG),
     (dict(gate_keys_bf16=2), sas.SAS_ERR_INVALID_ARG),
+    (dict(static_weights=2), sas.SAS_ERR_INVALID_ARG),
 ])
 def test_config_validation(L, kw, status):
     assert _decode(L, _cfg(**kw)) == status

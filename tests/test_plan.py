@@ -65,11 +65,10 @@ def test_plan_alignment_and_overlap(plans):
         # after their phase 1 (past the inbox and qv, clear of the local keys)
         assert p["r_lkeys"] >= inbox_end and p["r_lkeys"] >= qv_end, tag
         assert p["r_gather"] >= p["r_lkeys"] + 8 * 256, tag
-        assert p["r_fmask"] >= p["r_gather"] + 8 * CS * 64, tag
         assert p["r_gather"] % 16 == 0 and p["r_lkeys"] % 16 == 0, tag
         assert p["wq_heads"] in (G, (G + 1) // 2), tag
         end = max(p["r_wq"] + p["wq_heads"] * 128 * dpc * 2, p["r_scan"] + 64,
-                  p["r_fmask"] + 4 * ((mg + 31) // 32))
+                  p["r_gather"] + 8 * CS * 64)
         assert p["total"] >= end + 1024, tag
 
 
