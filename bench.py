@@ -323,6 +323,7 @@ def run_backward(args, rank, world, device):
     cfg, layers = build_layers(2, rank, device, gate_mode=sas.GATE_LOGSIGMOID_BIAS)
     stream = torch.cuda.Stream(device)
     for L in layers:
+        L["ws"] = sas.make_workspace(cfg, device, batch=BATCH)   # the per-pair terms of the reduction
         L["sel"] = torch.zeros(BATCH, HKV, cfg.max_sel, dtype=torch.int32, device=device)
         L["cnt"] = torch.zeros(BATCH, HKV, dtype=torch.int32, device=device)
         L["dout"] = torch.randn(BATCH, HQ, 128, generator=torch.Generator(device=device).manual_seed(9),
@@ -366,7 +367,7 @@ def run_backward(args, rank, world, device):
             "value": round(job_throughput(steps, world, med), 2), "unit": "backward steps/s",
             "ms_per_step": round(call_s * 1e3, 5), "timing": spread(ts, steps),
             "roofline": dict(roofline_of(dbytes, call_s, peak, peak_kind),
-                             kernel="gate_backward_kernel (sas_gate_backward)")}
+                             kernel="gate_backward_kernel + gate_grad_reduce_kernel (sas_gate_backward)")}
 
 
 def run_pooling(args, device, world):

@@ -250,8 +250,17 @@ const char* sas_status_string(sas_status s) {
   return "unknown status";
 }
 
+// Workspace layout: status header, then (batch > 0) the gate backward's
+// per-pair terms, then (batch > 0 and max_seq_len > 0) the prefill scratch.
+size_t bwd_scratch_bytes(const sas_config* cfg, int32_t batch) {
+  if (cfg == nullptr || batch <= 0 || cfg->num_kv_heads <= 0 || cfg->num_q_heads <= 0 || cfg->token_budget < 64)
+    return 0;
+  return sas::gate_bwd_scratch_bytes(static_cast<size_t>(batch), cfg->num_q_heads, cfg->num_kv_heads,
+                                     cfg->token_budget / 64);
+}
+
 size_t sas_workspace_bytes(const sas_config* cfg, int32_t batch, int32_t max_seq_len) {
-  size_t bytes = ws_header_bytes();
+  size_t bytes = ws_header_bytes() + bwd_scratch_bytes(cfg, batch);
   if (cfg != nullptr && batch > 0 && max_seq_len > 0 && cfg->num_kv_heads > 0 &&
       cfg->num_q_heads > 0 && cfg->token_budget >= 64) {
     // prefill scratch: gate queries, block lists and their lengths
@@ -561,7 +570,7 @@ sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q, const 
   p.gamma_q = gamma_q;
   p.gate_keys = gate_keys;
   p.gk16 = cfg->gate_keys_bf16;
-  uint8_t* scratch = static_cast<uint8_t*>(ws) + ws_header_bytes();
+  uint8_t* scratch = static_cast<uint8_t*>(ws) + ws_header_bytes() + bwd_scratch_bytes(cfg, batch);
   p.qt = reinterpret_cast<float*>(scratch);
   scratch += up256(static_cast<size_t>(batch) * p.hq * nblk * kDim * 4);
   p.sel = reinterpret_cast<int32_t*>(scratch);
@@ -597,7 +606,7 @@ sas_status sas_gate_backward(const sas_config* cfg, const void* q, const sas_kv*
       sel_idx == nullptr || sel_count == nullptr || d_out == nullptr || dw_q == nullptr ||
       dw_k == nullptr || dgamma_q == nullptr || dgamma_k == nullptr)
     return SAS_ERR_INVALID_ARG;
-  if (!aligned(q, 4) || !aligned(w_q, 2) || !aligned(gamma_q, 4) || !aligned(w_k, 2) ||
+  if (!aligned(q, 4) || !aligned(w_q, 4) || !aligned(gamma_q, 4) || !aligned(w_k, 16) ||
       !aligned(gamma_k, 4) || !aligned(sel_idx, 4) || !aligned(sel_count, 4) ||
       !aligned(d_out, 4) || !aligned(dw_q, 4) || !aligned(dw_k, 4) || !aligned(dgamma_q, 4) ||
       !aligned(dgamma_k, 4))
@@ -605,13 +614,17 @@ sas_status sas_gate_backward(const sas_config* cfg, const void* q, const sas_kv*
   if (cfg->kv_dtype != SAS_DTYPE_BF16) return SAS_ERR_UNSUPPORTED;
   const int G = cfg->num_q_heads / cfg->num_kv_heads;
   const int max_sel = cfg->token_budget / 64;
-  // two K/V stages when they fit beside the list's pooled keys, else one
-  const int stages = sas::gate_bwd_smem_bytes(G, max_sel, 2) <= 227 * 1024 ? 2 : 1;
+  // as many K/V stages (up to 4) as fit beside the list's pooled keys
+  int stages = 4;
+  while (stages > 1 && sas::gate_bwd_smem_bytes(G, max_sel, stages) > 227 * 1024) --stages;
   if (max_sel > sas::kBwMaxSel || sas::gate_bwd_smem_bytes(G, max_sel, stages) > 227 * 1024)
     return SAS_ERR_UNSUPPORTED;
   if (static_cast<long long>(kv->batch) * cfg->num_kv_heads > 0x7fffffffLL) return SAS_ERR_UNSUPPORTED;
+  if (kv_rows(cfg, kv) > 0x7fffffffLL) return SAS_ERR_UNSUPPORTED;  // TMA row coordinates are int32
   // the select-only mode gives the gate parameters no gradient
   if (cfg->gate_mode == SAS_GATE_SELECT_ONLY) return SAS_OK;
+  // the per-pair terms the reduction sums live in the workspace
+  if (ws_bytes < sas_workspace_bytes(cfg, kv->batch, 0)) return SAS_ERR_WORKSPACE;
   if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
   sas::GateBwdParams p{};
   sas::fill_rope_table(p.rope, cfg->rope_base);
@@ -632,12 +645,32 @@ sas_status sas_gate_backward(const sas_config* cfg, const void* q, const sas_kv*
   p.sel_count = sel_count;
   p.d_out = d_out;
   p.stages = stages;
+  p.batch = kv->batch;
   p.dw_q = dw_q;
   p.dw_k = dw_k;
   p.dgamma_q = dgamma_q;
   p.dgamma_k = dgamma_k;
   p.status = static_cast<uint32_t*>(ws);
-  return launch_result(sas::launch_gate_backward(p, kv->batch, reinterpret_cast<cudaStream_t>(stream)));
+  {
+    const size_t B = static_cast<size_t>(kv->batch), pairs = B * cfg->num_kv_heads;
+    uint8_t* w = static_cast<uint8_t*>(ws) + ws_header_bytes();
+    p.ws_dv = reinterpret_cast<float*>(w);
+    w += up256(B * cfg->num_q_heads * kDim * 4);
+    p.ws_p = reinterpret_cast<float*>(w);
+    w += up256(pairs * max_sel * sas::kPool * 4);
+    p.ws_du = reinterpret_cast<float*>(w);
+    w += up256(pairs * max_sel * kDim * 4);
+    p.ws_dg = reinterpret_cast<float*>(w);
+    w += up256(pairs * 2 * kDim * 4);
+    p.ws_nh = reinterpret_cast<int32_t*>(w);
+  }
+  p.trace = trace_region(ws);
+  CUtensorMap tmk, tmv, tmwk;
+  const long long rows = kv_rows(cfg, kv);
+  if (!encode_kv_map(&tmk, kv->k, rows) || !encode_kv_map(&tmv, kv->v, rows)) return SAS_ERR_CUDA;
+  // W_k as [Hkv * 384][128] in 64 x 64 boxes (64-row chunks of the projection)
+  if (!encode_kv_map(&tmwk, w_k, static_cast<long long>(cfg->num_kv_heads) * sas::kPool)) return SAS_ERR_CUDA;
+  return launch_result(sas::launch_gate_backward(p, tmk, tmv, tmwk, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const sas_kv* kv,

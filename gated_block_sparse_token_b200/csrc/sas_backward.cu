@@ -12,29 +12,55 @@
 // then back through the score, the gate RoPE, the RMSNorms and the two
 // projections.  The block list is held fixed (the Top-K has no gradient).
 //
-// One CTA (256 threads) per (sequence, KV head):
+// Two kernels.  gate_backward_kernel, one CTA (256 threads) per (sequence,
+// KV head):
 //   1. q, dout and the gains into shared memory; v_g = q_g @ W_q[g]; RMSNorm,
 //      gain, RoPE -> q~_g.
-//   2. one pass over the block list, K and V blocks by TMA bulk copy into a
-//      two-stage ring (one stage for 8-head groups at lists of 64 blocks,
-//      where two do not fit): the pooled key [max; min; mean] of every historical
-//      entry, and per (entry, head) the softmax statistics of the block
-//      without its bias -- max m', sum z' of exp(logit - m'), sum y' of
-//      exp(logit - m') (dout . v_j).  A bias constant over the block only
-//      shifts m', so the biased statistics follow once the gates are known.
-//   3. u_e = P_e @ W_k[h] for every historical entry (W_k read once, each
-//      element used for all entries); RMSNorm, gain, RoPE -> k~_e; s_ge.
+//   2. one pass over the block list, K and V blocks by 2-D TMA (128-byte
+//      swizzle) into a ring of as many stages (up to 4) as shared memory
+//      holds beside the list's terms: the pooled key [max; min; mean]
+//      of every historical entry; the logits q_g . k_j (warps 0-3) and
+//      dout_g . v_j (warps 4-7, dout split into two bf16 terms) on bf16
+//      mma.sync with fp32 accumulation; per (entry, head) the softmax
+//      statistics of the block without its bias -- max m', sum z' of
+//      exp(logit - m'), sum y' of exp(logit - m') (dout . v_j).  A bias
+//      constant over the block only shifts m', so the biased statistics
+//      follow once the gates are known.
+//   3. u_e = P_e @ W_k[h] for every historical entry on the tensor cores
+//      (W_k read once through the idle ring, P split into two bf16 terms);
+//      RMSNorm, gain, RoPE -> k~_e; s_ge.
 //   4. per head: the global max, sum and D_g = dout_g . out_g from the
 //      per-entry statistics with the biases; dL/dbias_ge and dL/ds_ge.
 //   5. dL/dq~_g and dL/dk~_e; RoPE transposed (rotation by -pos); RMSNorm
 //      backward; dL/dv_g, dL/du_e and the gain gradients.
-//   6. dL/dW_q[g] += q_g (x) dL/dv_g, dL/dW_k[h] += sum_e P_e (x) dL/du_e and
-//      the gain gradients, added to the caller's arrays with atomics.
+//   6. dL/dv_g, the pooled keys P_e, dL/du_e and the pair's gain gradients
+//      into the workspace.
+// gate_grad_reduce_kernel then adds, with no atomics (a fixed summation
+// order, so the result is reproducible bit for bit),
+//   dL/dW_q[g] = sum over sequences of q_g (x) dL/dv_g,
+//   dL/dW_k[h] = sum over sequences and historical entries of P_e (x) dL/du_e,
+// and the gain gradients summed over the pairs, to the caller's arrays.
 #include <cmath>
 
 #include "sas_internal.h"
 
 namespace sas {
+
+// Step-trace hook: thread 0 of each CTA stamps the SM clock at step
+// boundaries (tracing builds only; slot 0 is the global timer).
+#ifdef SAS_PHASE_TRACE
+#define BWD_TRACE(k)                                                                         \
+  do {                                                                                       \
+    if (p.trace != nullptr && threadIdx.x == 0 && blockIdx.x < static_cast<unsigned>(kTraceCtas)) { \
+      p.trace[blockIdx.x * kTraceSlots + (k)] = ((k) == 0) ? global_timer_ns() : clock64();  \
+      if ((k) == 0) p.trace[blockIdx.x * kTraceSlots + 23] = clock64();                      \
+    }                                                                                        \
+  } while (0)
+#else
+#define BWD_TRACE(k) \
+  do {               \
+  } while (0)
+#endif
 
 namespace {
 
@@ -61,7 +87,9 @@ __device__ __forceinline__ float sigmoid_f(float x) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __grid_constant__ GateBwdParams p) {
+__global__ void __launch_bounds__(kBwThreads, 1)
+    gate_backward_kernel(const __grid_constant__ GateBwdParams p, const __grid_constant__ CUtensorMap tmk,
+                         const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmwk) {
   constexpr int kW = kBwThreads / 32;  // warps
   const int pair = blockIdx.x;
   const int s = pair / p.hkv;
@@ -69,14 +97,16 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
   const int G = p.G;
   const int MS = p.max_sel;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  BWD_TRACE(0);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // carve (the order of gate_bwd_smem_bytes)
   const int NS = p.stages;                                            // K/V ring stages (1 or 2)
   uint8_t* tiles = base;                                              // [NS stages][K, V] bf16 [64][128]
-  float* P = reinterpret_cast<float*>(tiles + 2 * NS * kTileBytes);   // [MS][384]
-  float* U = P + MS * kPool;                                          // [MS][128] u, then dL/du
+  constexpr int kPs = kBwPoolStride;
+  float* P = reinterpret_cast<float*>(tiles + 2 * NS * kTileBytes);   // [MS][kPs] pooled keys
+  float* U = P + MS * kPs;                                            // [MS][128] u, then dL/du
   float* qf = U + MS * kDim;                                          // [G][128] q
   float* dof = qf + G * kDim;                                         // [G][128] dout
   float* vq = dof + G * kDim;                                         // [G][128] v, then dL/dv
@@ -90,11 +120,15 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
   float* wg = lg + G * kBlock;                                        // [G][64] dout . v_j
   int* sel = reinterpret_cast<int*>(wg + G * kBlock);                 // [MS]
   float* ru = reinterpret_cast<float*>(sel + MS);                     // [MS] RMS of u_e
-  float* scratch = ru + MS;                                           // [3][128] (unused slack)
-  float* dqt = scratch + 3 * kDim;                                    // [G][128] dL/dq~
+  __nv_bfloat16* qb = reinterpret_cast<__nv_bfloat16*>(ru + MS);     // [G][128] q as bf16
+  float* dqt = reinterpret_cast<float*>(qb + G * kDim);               // [G][128] dL/dq~
   float* dgq = dqt + G * kDim;                                        // [128]
   float* dgk = dgq + kDim;                                            // [128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(dgk + kDim) + 7) & ~uintptr_t(7));
+  float* red = dgk + kDim;                                            // [2][warps][128] gain partials
+  uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(red + 2 * kW * kDim) + 7) & ~uintptr_t(7));
+  // k~ of every historical entry (steps 3-5), over the K/V ring, idle by then
+  float* ktl = reinterpret_cast<float*>(tiles);                       // [MS][128]
+  static_assert(kBwMaxSel * kDim * 4 <= 2 * kTileBytes, "k~ of a full list fits one ring stage");
 
   // ---- the block list, checked like the attention call checks it
   const int L = p.kv.seq_lens[s];
@@ -113,7 +147,10 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
     }
   }
   if (__syncthreads_or(err)) {
-    if (tid == 0) raise_status(p.status, kStatusBounds);
+    if (tid == 0) {
+      raise_status(p.status, kStatusBounds);
+      p.ws_nh[pair] = -1;
+    }
     return;
   }
   const int nh = m - 1;  // historical entries (the current block, last, has no gate)
@@ -121,41 +158,55 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
   // ---- K/V ring: entry e in stage e % NS (16 KiB K then 16 KiB V)
   auto issue = [&](int e) {
     const int st = e % NS;
-    const long long row0 = p.kv.block_row(s, h, sel[e]);
-    const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(p.kv.k) + row0 * kDim;
-    const __nv_bfloat16* vb = static_cast<const __nv_bfloat16*>(p.kv.v) + row0 * kDim;
+    const int row0 = static_cast<int>(p.kv.block_row(s, h, sel[e]));
+    uint8_t* kd = tiles + (2 * st) * kTileBytes;
+    uint8_t* vd = kd + kTileBytes;
     mbar_arrive_expect_tx(&bars[st], 2 * kTileBytes);
-    bulk_g2s(tiles + (2 * st) * kTileBytes, kb, kTileBytes, &bars[st]);
-    bulk_g2s(tiles + (2 * st + 1) * kTileBytes, vb, kTileBytes, &bars[st]);
+    tma_load_2d(kd, &tmk, 0, row0, &bars[st]);
+    tma_load_2d(kd + 8192, &tmk, 64, row0, &bars[st]);
+    tma_load_2d(vd, &tmv, 0, row0, &bars[st]);
+    tma_load_2d(vd + 8192, &tmv, 64, row0, &bars[st]);
   };
+  uint64_t* bar_w = &bars[4];  // W_k chunks (step 3)
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+    prefetch_tensormap(&tmwk);
+    for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
+    mbar_init(bar_w, 1);
     fence_mbar_init();
-    issue(0);
-    if (m > 1 && NS > 1) issue(1);
+    for (int e = 0; e < NS && e < m; ++e) issue(e);
   }
 
+  BWD_TRACE(1);  // list checked, ring started
   // ---- 1. gate query: v_g = q_g @ W_q[g], RMSNorm, gain, RoPE at c
   const size_t qoff = (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim;
   for (int i = tid; i < G * kDim; i += kBwThreads) {
-    qf[i] = __bfloat162float(p.q[qoff + i]);
+    const __nv_bfloat16 x = p.q[qoff + i];
+    qb[i] = x;
+    qf[i] = __bfloat162float(x);
     dof[i] = p.d_out[qoff + i];
   }
-  if (tid < kDim) {
-    dgq[tid] = 0.f;
-    dgk[tid] = 0.f;
-  }
-  for (int i = tid; i < G * kDim; i += kBwThreads) dqt[i] = 0.f;
   __syncthreads();
-  for (int o = tid; o < G * kDim; o += kBwThreads) {
-    const int g = o >> 7, j = o & (kDim - 1);
-    const __nv_bfloat16* wcol = p.w_q + (static_cast<size_t>(h * G + g) * kDim) * kDim + j;
+  // two adjacent columns per thread (one 4-byte load per row, 256 bytes per
+  // warp and row)
+  for (int o = tid; o < G * (kDim / 2); o += kBwThreads) {
+    const int g = o / (kDim / 2), j = 2 * (o - g * (kDim / 2));
+    const uint32_t* wcol =
+        reinterpret_cast<const uint32_t*>(p.w_q + (static_cast<size_t>(h * G + g) * kDim) * kDim + j);
     const float* qrow = qf + g * kDim;
-    float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int i = 0; i < kDim; ++i) a4[i & 3] = fmaf(qrow[i], __bfloat162float(wcol[static_cast<size_t>(i) * kDim]), a4[i & 3]);
-    vq[o] = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll 16
+    for (int i = 0; i < kDim; i += 2) {
+      const uint32_t w0 = wcol[static_cast<size_t>(i) * (kDim / 2)];
+      const uint32_t w1 = wcol[static_cast<size_t>(i + 1) * (kDim / 2)];
+      a0 = fmaf(qrow[i], bf16_lo(w0), a0);
+      a1 = fmaf(qrow[i], bf16_hi(w0), a1);
+      b0 = fmaf(qrow[i + 1], bf16_lo(w1), b0);
+      b1 = fmaf(qrow[i + 1], bf16_hi(w1), b1);
+    }
+    vq[g * kDim + j] = a0 + b0;
+    vq[g * kDim + j + 1] = a1 + b1;
   }
   __syncthreads();
   for (int g = warp; g < G; g += kW) {
@@ -178,6 +229,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
     qt[g * kDim + lane + 96] = x[3] * c1 + x[1] * s1;
   }
 
+  BWD_TRACE(2);  // gate query done
   // ---- 2. pass over the list: pooled keys and unbiased block statistics
   const float alpha = p.attn_scale;
   for (int e = 0; e < m; ++e) {
@@ -190,43 +242,67 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
     if (b != c && tid < kDim) {
       float mx = -INFINITY, mn = INFINITY, sm = 0.f;
       if (ok) {
+        const uint8_t* kt8 = reinterpret_cast<const uint8_t*>(kt) + (tid & 7) * 2;
 #pragma unroll 8
         for (int t = 0; t < kBlock; ++t) {
-          const float x = __bfloat162float(kt[t * kDim + tid]);
+          const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kt8 + swz_tile_offset(t, tid >> 3)));
           mx = fmaxf(mx, x);
           mn = fminf(mn, x);
           sm += x;
         }
       }
-      P[e * kPool + tid] = mx;
-      P[e * kPool + kDim + tid] = mn;
-      P[e * kPool + 2 * kDim + tid] = sm * (1.f / kBlock);
+      P[e * kPs + tid] = mx;
+      P[e * kPs + kDim + tid] = mn;
+      P[e * kPs + 2 * kDim + tid] = sm * (1.f / kBlock);
     }
-    // logits and dout . v_j: warp w takes tokens w, w + 8, ...; lane l holds
-    // dimensions 4l .. 4l + 3
-    for (int j = warp; j < kBlock; j += kW) {
-      if (j >= nvalid) {
-        if (lane < G) {
-          lg[lane * kBlock + j] = -INFINITY;
-          wg[lane * kBlock + j] = 0.f;
+    // logits q_g . k_j (warps 0-3) and dout_g . v_j (warps 4-7) on the
+    // tensor cores: the group's heads are rows 0..G-1 of the A operand, each
+    // warp takes 16 tokens as two 8-column tiles; dout enters as hi + lo
+    // bf16 terms (its fp32 value to about 2^-16)
+    {
+      const bool is_w = warp >= 4;
+      const int wt = warp & 3;
+      const int tq = lane & 3, gq = lane >> 2;
+      const int mat = lane >> 3;
+      const int tok = 16 * wt + (mat >> 1) * 8 + (lane & 7);
+      const uint32_t tb = smem_u32(tiles + (2 * st + (is_w ? 1 : 0)) * kTileBytes);
+      const int gr = min(gq, G - 1);
+      float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+      if (ok) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4(tb + swz_tile_offset(tok, 2 * ks + (mat & 1)), r0, r1, r2, r3);
+          if (!is_w) {
+            const uint32_t* q2 = reinterpret_cast<const uint32_t*>(qb + gr * kDim + 16 * ks + 2 * tq);
+            const uint32_t a0 = q2[0], a2 = q2[4];
+            mma_rows0_7(acc[0][0], acc[0][1], a0, a2, r0, r1);
+            mma_rows0_7(acc[1][0], acc[1][1], a0, a2, r2, r3);
+          } else {
+            const float* d = dof + gr * kDim + 16 * ks + 2 * tq;
+            const float x0 = d[0], x1 = d[1], x8 = d[8], x9 = d[9];
+            const uint32_t h0 = pack_bf16x2(x0, x1), h2 = pack_bf16x2(x8, x9);
+            const uint32_t l0 = pack_bf16x2(x0 - bf16_lo(h0), x1 - bf16_hi(h0));
+            const uint32_t l2 = pack_bf16x2(x8 - bf16_lo(h2), x9 - bf16_hi(h2));
+            mma_rows0_7(acc[0][0], acc[0][1], h0, h2, r0, r1);
+            mma_rows0_7(acc[0][0], acc[0][1], l0, l2, r0, r1);
+            mma_rows0_7(acc[1][0], acc[1][1], h0, h2, r2, r3);
+            mma_rows0_7(acc[1][0], acc[1][1], l0, l2, r2, r3);
+          }
         }
-        continue;
       }
-      const uint2 kr = *reinterpret_cast<const uint2*>(kt + j * kDim + 4 * lane);
-      const uint2 vr = *reinterpret_cast<const uint2*>(vt + j * kDim + 4 * lane);
-      const float k0 = bf16_lo(kr.x), k1 = bf16_hi(kr.x), k2 = bf16_lo(kr.y), k3 = bf16_hi(kr.y);
-      const float v0 = bf16_lo(vr.x), v1 = bf16_hi(vr.x), v2 = bf16_lo(vr.y), v3 = bf16_hi(vr.y);
-      for (int g = 0; g < G; ++g) {
-        const float4 q4 = *reinterpret_cast<const float4*>(qf + g * kDim + 4 * lane);
-        const float4 d4 = *reinterpret_cast<const float4*>(dof + g * kDim + 4 * lane);
-        float a = q4.x * k0 + q4.y * k1 + q4.z * k2 + q4.w * k3;
-        float w = d4.x * v0 + d4.y * v1 + d4.z * v2 + d4.w * v3;
-        a = warp_sum(a);
-        w = warp_sum(w);
-        if (lane == 0) {
-          lg[g * kBlock + j] = ok ? a * alpha : -INFINITY;
-          wg[g * kBlock + j] = ok ? w : 0.f;
-        }
+      if (gq < G) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int j = 16 * wt + 8 * nt + 2 * tq + q;
+            const bool live = ok && j < nvalid;  // rows past the context may hold anything
+            if (!is_w)
+              lg[gq * kBlock + j] = live ? acc[nt][q] * alpha : -INFINITY;
+            else
+              wg[gq * kBlock + j] = live ? acc[nt][q] : 0.f;
+          }
       }
     }
     __syncthreads();  // every read of this stage is done, the block's values are in
@@ -255,27 +331,81 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
     __syncthreads();  // lg / wg are rewritten by the next entry
   }
 
-  // ---- 3. gate keys of the historical entries: u_e = P_e @ W_k[h]
+  BWD_TRACE(3);  // list pass done
+  // ---- 3. gate keys of the historical entries: u_e = P_e @ W_k[h], on the
+  // tensor cores.  W_k[h] streams through the idle K/V ring in 64-row
+  // chunks (2-D TMA, 128-byte swizzle, two chunks per round); warp w owns
+  // output columns 16w .. 16w + 15 of every 16-entry tile; P enters as hi +
+  // lo bf16 terms (its fp32 value to about 2^-16), W_k is bf16 already.
   {
-    const int j = tid & (kDim - 1);
-    const int half = tid >> 7;  // entries half, half + 2, ...
-    const __nv_bfloat16* wk = p.w_k + static_cast<size_t>(h) * kPool * kDim + j;
-    constexpr int kMaxRows = kBwMaxSel / 2;
-    float acc[kMaxRows];
+    const int tq = lane & 3, gq = lane >> 2, mat = lane >> 3;
+    const int nmt = (nh + 15) >> 4;  // 16-entry tiles
+    float acc[kBwMaxSel / 16][2][4];
 #pragma unroll
-    for (int r = 0; r < kMaxRows; ++r) acc[r] = 0.f;
-    const int nrows = (nh - half + 1) / 2;  // entries of this thread
-    for (int i = 0; i < kPool; ++i) {
-      const float w = __bfloat162float(wk[static_cast<size_t>(i) * kDim]);
+    for (int mt = 0; mt < kBwMaxSel / 16; ++mt)
 #pragma unroll
-      for (int r = 0; r < kMaxRows; ++r)
-        if (r < nrows) acc[r] = fmaf(P[(half + 2 * r) * kPool + i], w, acc[r]);
+      for (int nt = 0; nt < 2; ++nt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] = acc[mt][nt][3] = 0.f;
+    constexpr int kChunks = kPool / 64;
+    constexpr int kPerRound = 2;  // one ring stage holds two 16 KiB tiles
+    for (int c0 = 0; c0 < kChunks; c0 += kPerRound) {
+      __syncthreads();  // every read of the region (list pass, last round) is done
+      if (tid == 0) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(bar_w, kPerRound * kTileBytes);
+        for (int cc = 0; cc < kPerRound; ++cc) {
+          const int y = h * kPool + (c0 + cc) * 64;
+          tma_load_2d(tiles + cc * kTileBytes, &tmwk, 0, y, bar_w);
+          tma_load_2d(tiles + cc * kTileBytes + 8192, &tmwk, 64, y, bar_w);
+        }
+      }
+      if (!mbar_wait(bar_w, (c0 / kPerRound) & 1, p.status)) continue;
+      for (int cc = 0; cc < kPerRound; ++cc) {
+        const uint32_t tb = smem_u32(tiles + cc * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // 16 rows of the chunk
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4_trans(tb + swz_tile_offset(16 * kk + (mat & 1) * 8 + (lane & 7), 2 * warp + (mat >> 1)), r0,
+                        r1, r2, r3);
+          const int k0 = (c0 + cc) * 64 + 16 * kk + 2 * tq;  // pooled dimension
+#pragma unroll
+          for (int mt = 0; mt < kBwMaxSel / 16; ++mt) {
+            if (mt < nmt) {
+              const int e0 = 16 * mt + gq, e1 = e0 + 8;
+              const float2 z = make_float2(0.f, 0.f);
+              const float2 x00 = e0 < nh ? *reinterpret_cast<const float2*>(P + e0 * kPs + k0) : z;
+              const float2 x02 = e0 < nh ? *reinterpret_cast<const float2*>(P + e0 * kPs + k0 + 8) : z;
+              const float2 x10 = e1 < nh ? *reinterpret_cast<const float2*>(P + e1 * kPs + k0) : z;
+              const float2 x12 = e1 < nh ? *reinterpret_cast<const float2*>(P + e1 * kPs + k0 + 8) : z;
+              const uint32_t h0 = pack_bf16x2(x00.x, x00.y), h1 = pack_bf16x2(x10.x, x10.y);
+              const uint32_t h2 = pack_bf16x2(x02.x, x02.y), h3 = pack_bf16x2(x12.x, x12.y);
+              const uint32_t l0 = pack_bf16x2(x00.x - bf16_lo(h0), x00.y - bf16_hi(h0));
+              const uint32_t l1 = pack_bf16x2(x10.x - bf16_lo(h1), x10.y - bf16_hi(h1));
+              const uint32_t l2 = pack_bf16x2(x02.x - bf16_lo(h2), x02.y - bf16_hi(h2));
+              const uint32_t l3 = pack_bf16x2(x12.x - bf16_lo(h3), x12.y - bf16_hi(h3));
+              mma_bf16_16816(acc[mt][0], h0, h1, h2, h3, r0, r1);
+              mma_bf16_16816(acc[mt][0], l0, l1, l2, l3, r0, r1);
+              mma_bf16_16816(acc[mt][1], h0, h1, h2, h3, r2, r3);
+              mma_bf16_16816(acc[mt][1], l0, l1, l2, l3, r2, r3);
+            }
+          }
+        }
+      }
     }
 #pragma unroll
-    for (int r = 0; r < kMaxRows; ++r)
-      if (r < nrows) U[(half + 2 * r) * kDim + j] = acc[r];
+    for (int mt = 0; mt < kBwMaxSel / 16; ++mt) {
+      if (mt < nmt) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int j = 16 * warp + 8 * nt + 2 * tq;
+          const int e0 = 16 * mt + gq, e1 = e0 + 8;
+          if (e0 < nh) *reinterpret_cast<float2*>(U + e0 * kDim + j) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+          if (e1 < nh) *reinterpret_cast<float2*>(U + e1 * kDim + j) = make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+        }
+      }
+    }
   }
   __syncthreads();
+  BWD_TRACE(4);  // u = P W_k done
   // RMS, k~_e and the gate scores s_ge (warp per entry)
   auto key_of = [&](int e, float* kk, float& inv) {
     float ss = 0.f;
@@ -302,6 +432,8 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
     float kk[4], inv;
     key_of(e, kk, inv);
     if (lane == 0) ru[e] = inv;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) ktl[e * kDim + lane + 32 * k] = kk[k];
     for (int g = 0; g < G; ++g) {
       float a = 0.f;
 #pragma unroll
@@ -312,6 +444,7 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
   }
   __syncthreads();
 
+  BWD_TRACE(5);  // gate keys and scores done
   // ---- 4. biased statistics per head; dL/dbias and dL/ds per entry
   for (int g = warp; g < G; g += kW) {
     float mx = -INFINITY;
@@ -341,18 +474,28 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
   }
   __syncthreads();
 
-  // ---- 5. dL/dq~_g (summed over entries), dL/dk~_e -> dL/du_e, dL/dgamma_k
+  BWD_TRACE(6);  // gate gradients done
+  // ---- 5. dL/dq~_g = sum_e dL/ds_ge * gate_scale * k~_e: warp g owns head g
+  // (entries in order)
+  for (int g = warp; g < G; g += kW) {
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int e = 0; e < nh; ++e) {
+      const float d = dsg[e * G + g] * p.gate_scale;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) a[k] = fmaf(d, ktl[e * kDim + lane + 32 * k], a[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dqt[g * kDim + lane + 32 * k] = a[k];
+  }
+  // dL/dk~_e -> dL/du_e (in place of u); dL/dgamma_k per warp
+  float pgk[4] = {0.f, 0.f, 0.f, 0.f};
   for (int e = warp; e < nh; e += kW) {
-    float kk[4], inv;
-    key_of(e, kk, inv);
+    const float inv = ru[e];
     float dk[4] = {0.f, 0.f, 0.f, 0.f};
     for (int g = 0; g < G; ++g) {
       const float d = dsg[e * G + g] * p.gate_scale;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        atomicAdd(&dqt[g * kDim + lane + 32 * k], d * kk[k]);
-        dk[k] = fmaf(d, qt[g * kDim + lane + 32 * k], dk[k]);
-      }
+      for (int k = 0; k < 4; ++k) dk[k] = fmaf(d, qt[g * kDim + lane + 32 * k], dk[k]);
     }
     // RoPE transposed: rotation by -b
     float c0, s0, c1, s1;
@@ -375,12 +518,13 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int d = lane + 32 * k;
-      atomicAdd(&dgk[d], dh[k] * u[k] * inv);
+      pgk[k] = fmaf(dh[k] * u[k], inv, pgk[k]);
       U[e * kDim + d] = p.gamma_k[d] * dh[k] * inv - u[k] * dot * inv3 / kDim;
     }
   }
-  __syncthreads();
-  // dL/dq^_g -> dL/dv_g (in place of v), dL/dgamma_q
+  __syncthreads();  // dqt complete
+  // dL/dq^_g -> dL/dv_g (in place of v); dL/dgamma_q per warp
+  float pgq[4] = {0.f, 0.f, 0.f, 0.f};
   for (int g = warp; g < G; g += kW) {
     float c0, s0, c1, s1;
     rope_cos_sin(p.rope.theta_over_pi[lane], c, c0, s0);
@@ -406,36 +550,121 @@ __global__ void __launch_bounds__(kBwThreads, 1) gate_backward_kernel(const __gr
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const int d = lane + 32 * k;
-      atomicAdd(&dgq[d], dh[k] * x[k] * inv);
+      pgq[k] = fmaf(dh[k] * x[k], inv, pgq[k]);
       vq[g * kDim + d] = p.gamma_q[d] * dh[k] * inv - x[k] * dot * inv3 / kDim;
     }
   }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    red[warp * kDim + lane + 32 * k] = pgq[k];
+    red[(kW + warp) * kDim + lane + 32 * k] = pgk[k];
+  }
+  __syncthreads();
+  // the gain gradients: warps summed in order
+  {
+    const int d = tid & (kDim - 1), which = tid >> 7;  // 0: gamma_q, 1: gamma_k
+    float a = 0.f;
+    for (int w = 0; w < kW; ++w) a += red[(which * kW + w) * kDim + d];
+    (which == 0 ? dgq : dgk)[d] = a;
+  }
   __syncthreads();
 
-  // ---- 6. weight and gain gradients into the caller's arrays
-  for (int o = tid; o < G * kDim * kDim; o += kBwThreads) {
-    const int g = o / (kDim * kDim);
-    const int r = o - g * kDim * kDim;
-    const int i = r >> 7, j = r & (kDim - 1);
-    atomicAdd(&p.dw_q[(static_cast<size_t>(h * G + g) * kDim + i) * kDim + j], qf[g * kDim + i] * vq[g * kDim + j]);
-  }
+  BWD_TRACE(7);  // back through the norms done
+  // ---- 6. the pair's terms into the workspace (the reduction adds them up)
+  for (int i = tid; i < G * kDim; i += kBwThreads) p.ws_dv[qoff + i] = vq[i];
   {
-    const int j = tid & (kDim - 1);
-    for (int i = tid >> 7; i < kPool; i += kBwThreads / kDim) {
-      float a = 0.f;
-      for (int e = 0; e < nh; ++e) a = fmaf(P[e * kPool + i], U[e * kDim + j], a);
-      if (nh > 0) atomicAdd(&p.dw_k[(static_cast<size_t>(h) * kPool + i) * kDim + j], a);
-    }
+    float* wp = p.ws_p + static_cast<size_t>(pair) * MS * kPool;
+    float* wu = p.ws_du + static_cast<size_t>(pair) * MS * kDim;
+    for (int i = tid; i < nh * kPool; i += kBwThreads) wp[i] = P[(i / kPool) * kPs + i % kPool];
+    for (int i = tid; i < nh * kDim; i += kBwThreads) wu[i] = U[i];
   }
   if (tid < kDim) {
-    atomicAdd(&p.dgamma_q[tid], dgq[tid]);
-    atomicAdd(&p.dgamma_k[tid], dgk[tid]);
+    p.ws_dg[(static_cast<size_t>(pair) * 2) * kDim + tid] = dgq[tid];
+    p.ws_dg[(static_cast<size_t>(pair) * 2 + 1) * kDim + tid] = dgk[tid];
+  }
+  if (tid == 0) p.ws_nh[pair] = nh;
+  BWD_TRACE(8);
+}
+
+// Sums of the per-pair terms, added to the caller's gradient arrays.  Blocks
+// [0, Hq * 8): 16 rows of dW_q[hq] each; then Hkv * 24 blocks of 16 rows of
+// dW_k[h]; the last block the two gain gradients.  Thread (rp, j) owns
+// column j of rows rp, rp + 2, .. of its block's 16 and sums in a fixed order
+// (sequences, then entries).  A pair the kernel skipped (a bad block list)
+// contributes nothing.
+constexpr int kRedRows = 16;
+
+__global__ void __launch_bounds__(kBwThreads) gate_grad_reduce_kernel(const __grid_constant__ GateBwdParams p) {
+  const int tid = threadIdx.x;
+  const int j = tid & (kDim - 1), rp = tid >> 7;
+  constexpr int kPer = kRedRows / (kBwThreads / kDim);  // rows per thread
+  const int nq = p.hq * (kDim / kRedRows);
+  const int nk = p.hkv * (kPool / kRedRows);
+  const int blk = blockIdx.x;
+  const int MS = p.max_sel;
+  float acc[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
+  if (blk < nq) {
+    const int hq = blk / (kDim / kRedRows);
+    const int i0 = (blk - hq * (kDim / kRedRows)) * kRedRows + rp;
+    const int h = hq / p.G;
+    for (int s = 0; s < p.batch; ++s) {
+      if (p.ws_nh[s * p.hkv + h] < 0) continue;
+      const float dv = p.ws_dv[(static_cast<size_t>(s) * p.hq + hq) * kDim + j];
+      const __nv_bfloat16* qr = p.q + (static_cast<size_t>(s) * p.hq + hq) * kDim;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) acc[k] = fmaf(__bfloat162float(qr[i0 + 2 * k]), dv, acc[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) p.dw_q[(static_cast<size_t>(hq) * kDim + i0 + 2 * k) * kDim + j] += acc[k];
+  } else if (blk < nq + nk) {
+    // rounds of up to 32 entries: dL/du rows and this block's 16 pooled
+    // columns staged in shared memory by every thread, then summed in order
+    __shared__ float sdu[32][kDim];
+    __shared__ float sp[32][kRedRows];
+    const int b = blk - nq;
+    const int h = b / (kPool / kRedRows);
+    const int r0 = (b - h * (kPool / kRedRows)) * kRedRows;
+    for (int s = 0; s < p.batch; ++s) {
+      const size_t pair = static_cast<size_t>(s) * p.hkv + h;
+      const int nh = p.ws_nh[pair];
+      const float* pp = p.ws_p + pair * MS * kPool;
+      const float* du = p.ws_du + pair * MS * kDim;
+      for (int e0 = 0; e0 < nh; e0 += 32) {
+        const int ne = min(32, nh - e0);
+        __syncthreads();  // the previous round's reads are done
+        for (int i = tid; i < ne * kDim; i += kBwThreads)
+          sdu[i / kDim][i % kDim] = du[static_cast<size_t>(e0) * kDim + i];
+        for (int i = tid; i < ne * kRedRows; i += kBwThreads)
+          sp[i / kRedRows][i % kRedRows] = pp[static_cast<size_t>(e0 + i / kRedRows) * kPool + r0 + i % kRedRows];
+        __syncthreads();
+        for (int e = 0; e < ne; ++e) {
+          const float d = sdu[e][j];
+#pragma unroll
+          for (int k = 0; k < kPer; ++k) acc[k] = fmaf(sp[e][rp + 2 * k], d, acc[k]);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) p.dw_k[(static_cast<size_t>(h) * kPool + r0 + rp + 2 * k) * kDim + j] += acc[k];
+  } else {
+    // thread (rp, j): gamma_q (rp = 0) or gamma_k (rp = 1), element j
+    float a = 0.f;
+    for (int pair = 0; pair < p.batch * p.hkv; ++pair)
+      if (p.ws_nh[pair] >= 0) a += p.ws_dg[(static_cast<size_t>(pair) * 2 + rp) * kDim + j];
+    (rp == 0 ? p.dgamma_q : p.dgamma_k)[j] += a;
   }
 }
 
-cudaError_t launch_gate_backward(const GateBwdParams& p, int batch, cudaStream_t stream) {
+cudaError_t launch_gate_backward(const GateBwdParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                                 const CUtensorMap& tmwk, cudaStream_t stream) {
   const int smem = gate_bwd_smem_bytes(p.G, p.max_sel, p.stages);
-  gate_backward_kernel<<<static_cast<unsigned>(batch * p.hkv), kBwThreads, smem, stream>>>(p);
+  gate_backward_kernel<<<static_cast<unsigned>(p.batch * p.hkv), kBwThreads, smem, stream>>>(p, tmk, tmv, tmwk);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const unsigned nblk = static_cast<unsigned>(p.hq * (kDim / kRedRows) + p.hkv * (kPool / kRedRows) + 1);
+  gate_grad_reduce_kernel<<<nblk, kBwThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -247,6 +247,19 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
                : "r"(addr));
 }
 
+// D(16x8, f32) += A(16x16 bf16, row) * B(16x8 bf16, col): lane (g, t) =
+// (lane / 4, lane % 4) holds a0 = A[g][2t..], a1 = A[g + 8][2t..], a2 =
+// A[g][2t + 8..], a3 = A[g + 8][2t + 8..] and d = D[g][2t], D[g][2t + 1],
+// D[g + 8][2t], D[g + 8][2t + 1].
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // D(16x8, f32) = A(16x16 bf16, row) * B(16x8 bf16, col) + C, keeping only the
 // rows 0..7 of the result (rows 8..15 enter as zero and are dropped): the
 // callers pad a GQA group of <= 8 heads to the 16 rows of the instruction.

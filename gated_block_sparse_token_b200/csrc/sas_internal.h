@@ -228,28 +228,50 @@ struct GateBwdParams {
   const int32_t* sel_count;   // [B][Hkv]
   const float* d_out;         // [B][Hq][128]
   int stages;                 // K/V ring stages (2, or 1 when two do not fit)
+  int batch;                  // B
   float* dw_q;                // [Hq][128][128]  (accumulated)
   float* dw_k;                // [Hkv][384][128] (accumulated)
   float* dgamma_q;            // [128]           (accumulated)
   float* dgamma_k;            // [128]           (accumulated)
+  // per-pair terms the reduction kernel sums (workspace)
+  float* ws_dv;               // [B][Hq][128]        dL/dv_g
+  float* ws_p;                // [B*Hkv][max_sel][384] pooled keys of the historical entries
+  float* ws_du;               // [B*Hkv][max_sel][128] dL/du_e
+  float* ws_dg;               // [B*Hkv][2][128]     gain gradients (q, k)
+  int32_t* ws_nh;             // [B*Hkv]             historical entries (-1: pair skipped)
   uint32_t* status;
+  unsigned long long* trace;  // per-CTA step timings (tracing builds only), else null
 };
+
+// Workspace bytes of the backward's per-pair terms (after the status header).
+inline size_t gate_bwd_scratch_bytes(size_t batch, int hq, int hkv, int max_sel) {
+  auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t pairs = batch * static_cast<size_t>(hkv);
+  return up256(batch * hq * kDim * 4) + up256(pairs * max_sel * kPool * 4) + up256(pairs * max_sel * kDim * 4) +
+         up256(pairs * 2 * kDim * 4) + up256(pairs * 4);
+}
 
 // Shared-memory bytes of the backward kernel for a group of G heads and
 // block lists of max_sel entries.
+// Row stride (floats) of the pooled keys in the backward's shared memory:
+// 8 floats of padding put the 8 rows of one tensor-core fragment load in
+// different banks.
+constexpr int kBwPoolStride = kPool + 8;
+
 inline int gate_bwd_smem_bytes(int G, int max_sel, int stages = 2) {
-  return stages * 2 * kTileBytes       // K and V tiles, one or two stages
-         + max_sel * kPool * 4         // pooled keys of the list
+  return stages * 2 * kTileBytes       // K and V tiles, 1 to 4 stages
+         + max_sel * kBwPoolStride * 4 // pooled keys of the list
          + max_sel * kDim * 4          // u, then dL/du, per entry
          + 4 * G * kDim * 4            // q, d_out, v (then dL/dv), q~
          + 3 * max_sel * G * 4         // per-entry softmax statistics
          + 2 * max_sel * G * 4         // gate scores and their gradients
          + 2 * G * kBlock * 4          // logits and d_out . v of one block
          + 2 * max_sel * 4             // list, RMS of u
-         + 3 * kDim * 4                // spare
+         + G * kDim * 2                // q as bf16 (the tensor-core operand)
          + G * kDim * 4                // dL/dq~ per head
-         + 2 * kDim * 4                // dL/dgamma_q, dL/dgamma_k partial sums
-         + 4 * 8 + 1024;               // barriers, alignment slack
+         + 2 * kDim * 4                // dL/dgamma_q, dL/dgamma_k
+         + 2 * (kBwThreads / 32) * kDim * 4  // their per-warp partial sums
+         + 8 * 8 + 1024;               // barriers, alignment slack
 }
 
 constexpr int kPfQb = 16;      // query blocks per gate-query CTA
@@ -279,7 +301,8 @@ void fill_rope_table(RopeTable& t, float base);
 cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmq, const CUtensorMap& tmk,
                            const CUtensorMap& tmv, cudaStream_t stream);
 size_t prefill_attn_smem_bytes(int max_sel);
-cudaError_t launch_gate_backward(const GateBwdParams& p, int batch, cudaStream_t stream);
+cudaError_t launch_gate_backward(const GateBwdParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
+                                 const CUtensorMap& tmwk, cudaStream_t stream);
 
 // One-time per-process set-up of kernel attributes.
 cudaError_t prepare_kernels();

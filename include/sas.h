@@ -156,8 +156,10 @@ typedef struct {
 } sas_kv;
 
 /* Bytes of device workspace `ws` every entry point below needs for this
- * configuration (status word plus any scratch).  max_seq_len is the largest
- * L_s (decode) or T (prefill) of the calls that will use it. */
+ * configuration (status word plus any scratch).  batch and max_seq_len are
+ * the largest B and L_s (decode) or T (prefill) of the calls that will use
+ * it; decode steps need neither (0, 0), sas_gate_backward the batch,
+ * sas_prefill_block_sparse both. */
 SAS_API size_t sas_workspace_bytes(const sas_config* cfg, int32_t batch, int32_t max_seq_len);
 
 /* Zero the status word at the start of ws (cudaMemsetAsync on `stream`). */
@@ -308,8 +310,9 @@ SAS_API sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q
  *   dw_k     fp32 [Hkv][384][128]  dL/dW_k
  *   dgamma_q fp32 [128]            dL/dgamma_q
  *   dgamma_k fp32 [128]            dL/dgamma_k
- * (zero them first for a fresh gradient; the sums over sequences use atomic
- * adds, so the last bits depend on their order).  The gate of a selected
+ * (zero them first for a fresh gradient; the sums over sequences and block
+ * list entries run in a fixed order, so repeated calls add identical values).
+ * The gate of a selected
  * historical block b for query head g is log(sigmoid(s_gb)) on its tokens'
  * logits; its gradient reaches W_q and gamma_q through the gate query (q_g
  * @ W_q[g], RMSNorm, gain, RoPE at the current block) and W_k and gamma_k
@@ -324,6 +327,9 @@ SAS_API sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q
  *            the current block or names a block outside the cache skips its
  *            (sequence, KV head) and sets SAS_ERR_DEVICE_BOUNDS's bit
  *   d_out    fp32 [B][Hq][128]  dL/dout
+ *   ws       at least sas_workspace_bytes(cfg, B, 0) bytes (per-pair terms
+ *            that a second kernel sums into the gradients), else
+ *            SAS_ERR_WORKSPACE
  * This build handles budgets up to 4,096 tokens (lists of up to 64 blocks)
  * and bf16 caches; others return SAS_ERR_UNSUPPORTED.
  */

@@ -241,6 +241,10 @@ def test_gate_backward_validates_on_the_host(L):
     assert bwd(gated.c(), dout=None) == sas.SAS_ERR_INVALID_ARG
     assert bwd(gated.c(), dwq=FAKE + 2) == sas.SAS_ERR_INVALID_ARG
     assert bwd(gated.c(), ws=None) == sas.SAS_ERR_WORKSPACE
+    # the per-pair terms of the reduction need sas_workspace_bytes(cfg, B, 0)
+    need = L.sas_workspace_bytes(ctypes.byref(gated.c()), 2, 0)
+    assert need > L.sas_workspace_bytes(ctypes.byref(gated.c()), 0, 0)
+    assert bwd(gated.c(), ws_bytes=need - 1) == sas.SAS_ERR_WORKSPACE
     assert bwd(_cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS, token_budget=8192).c()) == sas.SAS_ERR_UNSUPPORTED
     assert bwd(_cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS, kv_dtype="f32").c()) == sas.SAS_ERR_UNSUPPORTED
     # the select-only mode gives the gate parameters no gradient: nothing to do

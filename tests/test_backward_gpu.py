@@ -6,9 +6,11 @@ Simple-Attention-Sparsification ..." (aigc.news, 2026-09-14), release
 paragraph.
 
 Tolerance: every gradient tensor within 1e-3 of its largest magnitude (max-abs
-error / max |oracle|): the kernel accumulates in fp32 (dot products of 128,
-softmax sums over up to 4,096 tokens, 384-term projections, atomic sums over
-sequences), whose rounding stays orders of magnitude below that."""
+error / max |oracle|): the kernels accumulate in fp32 (dot products of 128 --
+dL/dout entering the tensor cores as two bf16 terms, exact to about 2^-16 --,
+softmax sums over up to 4,096 tokens, 384-term projections, fixed-order sums
+over sequences and entries), whose rounding stays orders of magnitude below
+that."""
 import numpy as np
 import pytest
 import torch
@@ -27,7 +29,7 @@ GRAD_RTOL = 1e-3
 def _forward(inp, budget, gate_mode=sas.GATE_LOGSIGMOID_BIAS):
     spec = inp["spec"]
     cfg = T.config_for(spec, budget, gate_mode=gate_mode)
-    ws = sas.make_workspace(cfg, DEV)
+    ws = sas.make_workspace(cfg, DEV, batch=spec.batch)  # the backward's per-pair terms
     gk = T.run_pool(inp, cfg, ws)
     gpu = T.run_decode_step(inp, cfg, ws, gk)
     torch.cuda.synchronize()
@@ -141,3 +143,17 @@ def test_gate_backward_bad_list_is_reported_and_skipped():
     d_out = torch.randn(2, 8, 128, generator=torch.Generator(device=DEV).manual_seed(7), device=DEV)
     _backward(inp, cfg, ws, gpu, d_out)
     assert sas.get_device_status(ws) == sas.SAS_ERR_DEVICE_BOUNDS
+
+
+def test_gate_backward_is_reproducible_bit_for_bit():
+    """The sums over sequences and entries run in a fixed order: two calls on
+    the same inputs add exactly the same values."""
+    spec = DecodeSpec("bwd_repro", 4, 16, 4, [3000, 1000, 2500, 4096], (1024,), block_offset_std=0.5, seed=74)
+    inp = make_decode_inputs(spec, DEV)
+    cfg, ws, gk, gpu = _forward(inp, 1024)
+    d_out = torch.randn(4, 16, 128, generator=torch.Generator(device=DEV).manual_seed(8), device=DEV)
+    a = _backward(inp, cfg, ws, gpu, d_out)
+    b = _backward(inp, cfg, ws, gpu, d_out)
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
