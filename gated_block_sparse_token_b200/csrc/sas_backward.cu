@@ -125,7 +125,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   float* dgq = dqt + G * kDim;                                        // [128]
   float* dgk = dgq + kDim;                                            // [128]
   float* red = dgk + kDim;                                            // [2][warps][128] gain partials
-  uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(red + 2 * kW * kDim) + 7) & ~uintptr_t(7));
+  float* poolp = red + 2 * kW * kDim;                                 // [4][384] pooling partials
+  uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(poolp + 4 * kPool) + 7) & ~uintptr_t(7));
   // k~ of every historical entry (steps 3-5), over the K/V ring, idle by then
   float* ktl = reinterpret_cast<float*>(tiles);                       // [MS][128]
   static_assert(kBwMaxSel * kDim * 4 <= 2 * kTileBytes, "k~ of a full list fits one ring stage");
@@ -232,29 +233,52 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   BWD_TRACE(2);  // gate query done
   // ---- 2. pass over the list: pooled keys and unbiased block statistics
   const float alpha = p.attn_scale;
+#ifdef SAS_PHASE_TRACE
+  unsigned long long seg[6] = {0, 0, 0, 0, 0, 0}, tseg = clock64();
+#define BWD_SEG(i)                      \
+  do {                                  \
+    const unsigned long long t_ = clock64(); \
+    seg[i] += t_ - tseg;                \
+    tseg = t_;                          \
+  } while (0)
+#else
+#define BWD_SEG(i) \
+  do {             \
+  } while (0)
+#endif
   for (int e = 0; e < m; ++e) {
     const int st = e % NS;
     const bool ok = mbar_wait(&bars[st], (e / NS) & 1, p.status);
+    BWD_SEG(0);
     const int b = sel[e];
     const int nvalid = (b == c) ? (L - b * kBlock) : kBlock;
     const __nv_bfloat16* kt = reinterpret_cast<const __nv_bfloat16*>(tiles + (2 * st) * kTileBytes);
     const __nv_bfloat16* vt = reinterpret_cast<const __nv_bfloat16*>(tiles + (2 * st + 1) * kTileBytes);
-    if (b != c && tid < kDim) {
-      float mx = -INFINITY, mn = INFINITY, sm = 0.f;
+    // pooling partials: thread (quarter, pair) takes dimensions 2 pr, 2 pr + 1
+    // over tokens 16 quarter .. + 15 (4-byte loads; every warp shares it)
+    if (b != c) {
+      const int pr = tid & 63, qt4 = tid >> 6;
+      float mx0 = -INFINITY, mx1 = -INFINITY, mn0 = INFINITY, mn1 = INFINITY, s0 = 0.f, s1 = 0.f;
       if (ok) {
-        const uint8_t* kt8 = reinterpret_cast<const uint8_t*>(kt) + (tid & 7) * 2;
-#pragma unroll 8
-        for (int t = 0; t < kBlock; ++t) {
-          const float x = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kt8 + swz_tile_offset(t, tid >> 3)));
-          mx = fmaxf(mx, x);
-          mn = fminf(mn, x);
-          sm += x;
+        const uint8_t* kt8 = reinterpret_cast<const uint8_t*>(kt) + (pr & 3) * 4;
+#pragma unroll
+        for (int t = 16 * qt4; t < 16 * qt4 + 16; ++t) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(kt8 + swz_tile_offset(t, pr >> 2));
+          const float x0 = bf16_lo(w), x1 = bf16_hi(w);
+          mx0 = fmaxf(mx0, x0);
+          mx1 = fmaxf(mx1, x1);
+          mn0 = fminf(mn0, x0);
+          mn1 = fminf(mn1, x1);
+          s0 += x0;
+          s1 += x1;
         }
       }
-      P[e * kPs + tid] = mx;
-      P[e * kPs + kDim + tid] = mn;
-      P[e * kPs + 2 * kDim + tid] = sm * (1.f / kBlock);
+      float* pp = poolp + qt4 * kPool;
+      *reinterpret_cast<float2*>(pp + 2 * pr) = make_float2(mx0, mx1);
+      *reinterpret_cast<float2*>(pp + kDim + 2 * pr) = make_float2(mn0, mn1);
+      *reinterpret_cast<float2*>(pp + 2 * kDim + 2 * pr) = make_float2(s0, s1);
     }
+    BWD_SEG(1);
     // logits q_g . k_j (warps 0-3) and dout_g . v_j (warps 4-7) on the
     // tensor cores: the group's heads are rows 0..G-1 of the A operand, each
     // warp takes 16 tokens as two 8-column tiles; dout enters as hi + lo
@@ -305,10 +329,25 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           }
       }
     }
+    BWD_SEG(2);
     __syncthreads();  // every read of this stage is done, the block's values are in
     if (tid == 0 && e + NS < m) {
       fence_proxy_async_smem();
       issue(e + NS);
+    }
+    BWD_SEG(3);
+    if (b != c) {  // the pooled key: quarters combined in order
+      for (int i = tid; i < kPool; i += kBwThreads) {
+        const float a0 = poolp[i], a1 = poolp[kPool + i], a2 = poolp[2 * kPool + i], a3 = poolp[3 * kPool + i];
+        float r;
+        if (i < kDim)
+          r = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+        else if (i < 2 * kDim)
+          r = fminf(fminf(a0, a1), fminf(a2, a3));
+        else
+          r = ((a0 + a1) + (a2 + a3)) * (1.f / kBlock);
+        P[e * kPs + i] = r;
+      }
     }
     for (int g = warp; g < G; g += kW) {
       const float l0 = lg[g * kBlock + lane], l1 = lg[g * kBlock + lane + 32];
@@ -328,8 +367,14 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         st_y[e * G + g] = y;
       }
     }
+    BWD_SEG(4);
     __syncthreads();  // lg / wg are rewritten by the next entry
+    BWD_SEG(5);
   }
+#ifdef SAS_PHASE_TRACE
+  if (p.trace != nullptr && tid == 0 && blockIdx.x < static_cast<unsigned>(kTraceCtas))
+    for (int i = 0; i < 6; ++i) p.trace[blockIdx.x * kTraceSlots + 10 + i] = seg[i];
+#endif
 
   BWD_TRACE(3);  // list pass done
   // ---- 3. gate keys of the historical entries: u_e = P_e @ W_k[h], on the
@@ -609,9 +654,10 @@ __global__ void __launch_bounds__(kBwThreads) gate_grad_reduce_kernel(const __gr
     const int hq = blk / (kDim / kRedRows);
     const int i0 = (blk - hq * (kDim / kRedRows)) * kRedRows + rp;
     const int h = hq / p.G;
+#pragma unroll 4
     for (int s = 0; s < p.batch; ++s) {
-      if (p.ws_nh[s * p.hkv + h] < 0) continue;
-      const float dv = p.ws_dv[(static_cast<size_t>(s) * p.hq + hq) * kDim + j];
+      const bool live = p.ws_nh[s * p.hkv + h] >= 0;
+      const float dv = live ? p.ws_dv[(static_cast<size_t>(s) * p.hq + hq) * kDim + j] : 0.f;
       const __nv_bfloat16* qr = p.q + (static_cast<size_t>(s) * p.hq + hq) * kDim;
 #pragma unroll
       for (int k = 0; k < kPer; ++k) acc[k] = fmaf(__bfloat162float(qr[i0 + 2 * k]), dv, acc[k]);
@@ -651,8 +697,11 @@ __global__ void __launch_bounds__(kBwThreads) gate_grad_reduce_kernel(const __gr
   } else {
     // thread (rp, j): gamma_q (rp = 0) or gamma_k (rp = 1), element j
     float a = 0.f;
-    for (int pair = 0; pair < p.batch * p.hkv; ++pair)
-      if (p.ws_nh[pair] >= 0) a += p.ws_dg[(static_cast<size_t>(pair) * 2 + rp) * kDim + j];
+#pragma unroll 16
+    for (int pair = 0; pair < p.batch * p.hkv; ++pair) {
+      const float x = p.ws_dg[(static_cast<size_t>(pair) * 2 + rp) * kDim + j];
+      a += (p.ws_nh[pair] >= 0) ? x : 0.f;
+    }
     (rp == 0 ? p.dgamma_q : p.dgamma_k)[j] += a;
   }
 }

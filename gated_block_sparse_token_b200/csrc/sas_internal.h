@@ -271,6 +271,7 @@ inline int gate_bwd_smem_bytes(int G, int max_sel, int stages = 2) {
          + G * kDim * 4                // dL/dq~ per head
          + 2 * kDim * 4                // dL/dgamma_q, dL/dgamma_k
          + 2 * (kBwThreads / 32) * kDim * 4  // their per-warp partial sums
+         + 4 * kPool * 4               // pooling partials of one block (4 token quarters)
          + 8 * 8 + 1024;               // barriers, alignment slack
 }
 
