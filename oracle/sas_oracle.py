@@ -532,3 +532,113 @@ def gated_decode_loss(q_group, k_seq, v_seq, seq_len, w_q_group, gamma_q, w_k, g
                                   gated_token_bias(s[g], sel, seq_len, c))
         tot += float(np.dot(d_out[g], o))
     return tot
+
+
+# --------------------------------------------------------------------------
+# Gradient of the gated prefill with respect to the gate parameters (R20 for
+# the chunked prefill: every query block i has its own gate query, its own
+# block list and its own gates log(sigmoid(s_{g,i,b}))).
+# --------------------------------------------------------------------------
+def prefill_gate_grads(q_seq_group, k_seq, v_seq, w_q_group, gamma_q, w_k, gamma_k, sels, d_out,
+                       attn_scale=1.0 / math.sqrt(128.0), gate_scale=1.0 / math.sqrt(128.0),
+                       eps=1e-6, base=10000.0):
+    """Gated-mode prefill of one (sequence, KV head) over the fixed block lists
+    `sels` (sels[i]: ascending historical blocks of query block i, then i) and
+    the gradients of L = sum_{g,t} d_out[g][t] . out[g][t] with respect to the
+    gate parameters (R20).
+
+    q_seq_group, d_out [G][T][128]; k_seq, v_seq [T][128]; T a multiple of 64;
+    w_q_group [G][128][128]; gamma_q, gamma_k [128]; w_k [384][128].
+    Returns dict(out [G][T][128], s (dict (g, i) -> scores over blocks < i),
+    dw_q [G][128][128], dw_k [384][128], dgamma_q, dgamma_k).
+
+    Forward as prefill_query_block (R13, R18): gate query of head g for block
+    i = RoPE(RMSNorm(mean_t q[g][t] @ W_q[g]) * gamma_q, i); gate key of block
+    b as decode; token t of block i attends to the kept historical blocks'
+    tokens (+ log(sigmoid(s_{g,i,b}))) and causally to block i (+ 0).
+    Backward: dL/dlogit_j = p_j (d_out_t . v_j - d_out_t . out_t); a block's
+    bias is shared by all (t, j) of query block i and key block b."""
+    q_seq_group = np.asarray(q_seq_group, np.float64)
+    d_out = np.asarray(d_out, np.float64)
+    k_seq = np.asarray(k_seq, np.float64)
+    v_seq = np.asarray(v_seq, np.float64)
+    G, T = q_seq_group.shape[0], q_seq_group.shape[1]
+    nblk = T // BLOCK
+    P = [pool_block(k_seq[b * BLOCK:(b + 1) * BLOCK]) for b in range(nblk)]
+    u = [P[b] @ np.asarray(w_k, np.float64) for b in range(nblk)]
+    kt = np.array([rope_rotate_half(rms_norm(u[b], gamma_k, eps), b, base) for b in range(nblk)])
+    out = np.zeros((G, T, HEAD_DIM))
+    dw_q = np.zeros((G, HEAD_DIM, HEAD_DIM))
+    dgamma_q = np.zeros(HEAD_DIM)
+    dkt = np.zeros((nblk, HEAD_DIM))
+    s_all = {}
+    for i in range(nblk):
+        sel = list(sels[i])
+        hist = sel[:-1]
+        toks_hist = selected_token_ids(hist, (i + 1) * BLOCK)
+        blk_hist = [t // BLOCK for t in toks_hist]
+        for g in range(G):
+            qbar = q_seq_group[g, i * BLOCK:(i + 1) * BLOCK].mean(axis=0)
+            v = qbar @ np.asarray(w_q_group[g], np.float64)
+            qt = rope_rotate_half(rms_norm(v, gamma_q, eps), i, base)
+            s = np.array([float(qt @ kt[b]) * gate_scale for b in range(i)])
+            s_all[(g, i)] = s
+            dbias = {b: 0.0 for b in hist}
+            for t in range(BLOCK):
+                tok = i * BLOCK + t
+                toks = toks_hist + list(range(i * BLOCK, tok + 1))
+                bias = np.array([log_sigmoid(s[b]) for b in blk_hist] + [0.0] * (t + 1))
+                logits = (k_seq[toks] @ q_seq_group[g, tok]) * attn_scale + bias
+                w = np.exp(logits - logits.max())
+                p = w / w.sum()
+                out[g, tok] = p @ v_seq[toks]
+                dlogit = p * (v_seq[toks] @ d_out[g, tok] - float(np.dot(d_out[g, tok], out[g, tok])))
+                for dl, b in zip(dlogit[:len(toks_hist)], blk_hist):
+                    dbias[b] += dl
+            dq_t = np.zeros(HEAD_DIM)
+            for b in hist:
+                ds = dbias[b] * log_sigmoid_grad(s[b])
+                dq_t += ds * gate_scale * kt[b]
+                dkt[b] += ds * gate_scale * qt
+            dq_hat = rope_backward(dq_t, i, base)
+            dvg, dgq = rms_norm_backward(v, gamma_q, dq_hat, eps)
+            dgamma_q += dgq
+            dw_q[g] += matmul_weight_grad(qbar, dvg)
+    dw_k = np.zeros((POOL_DIM, HEAD_DIM))
+    dgamma_k = np.zeros(HEAD_DIM)
+    for b in range(nblk):
+        if not np.any(dkt[b]):
+            continue
+        dk_hat = rope_backward(dkt[b], b, base)
+        dub, dgk = rms_norm_backward(u[b], gamma_k, dk_hat, eps)
+        dgamma_k += dgk
+        dw_k += matmul_weight_grad(P[b], dub)
+    return {"out": out, "s": s_all, "dw_q": dw_q, "dw_k": dw_k, "dgamma_q": dgamma_q, "dgamma_k": dgamma_k}
+
+
+def gated_prefill_loss(q_seq_group, k_seq, v_seq, w_q_group, gamma_q, w_k, gamma_k, sels, d_out,
+                       attn_scale=1.0 / math.sqrt(128.0), gate_scale=1.0 / math.sqrt(128.0),
+                       eps=1e-6, base=10000.0):
+    """L = sum_{g,t} d_out[g][t] . out[g][t] of the gated prefill over the
+    fixed block lists `sels` (the scalar whose gradient prefill_gate_grads
+    returns), through the forward functions above (gate_keys_for_sequence,
+    gate_scores, gated_token_bias, attention_over_tokens)."""
+    q_seq_group = np.asarray(q_seq_group, np.float64)
+    G, T = q_seq_group.shape[0], q_seq_group.shape[1]
+    nblk = T // BLOCK
+    keys = gate_keys_for_sequence(k_seq, nblk, w_k, gamma_k, eps, base)
+    tot = 0.0
+    for i in range(nblk):
+        qbar = q_seq_group[:, i * BLOCK:(i + 1) * BLOCK].mean(axis=1)
+        s, _ = gate_scores(qbar, w_q_group, np.tile(gamma_q, (G, 1)), keys, i, i, gate_scale, eps, base)
+        hist = list(sels[i])[:-1]
+        toks_hist = selected_token_ids(hist, (i + 1) * BLOCK)
+        for g in range(G):
+            hb = gated_token_bias(s[g], hist, (i + 1) * BLOCK, i)
+            for t in range(BLOCK):
+                tok = i * BLOCK + t
+                toks = toks_hist + list(range(i * BLOCK, tok + 1))
+                o = attention_over_tokens(q_seq_group[g, tok], k_seq, v_seq, toks, attn_scale,
+                                          hb + [0.0] * (t + 1))
+                tot += float(np.dot(d_out[g, tok], o))
+    return tot

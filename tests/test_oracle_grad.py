@@ -163,3 +163,82 @@ def test_rms_norm_backward_matches_finite_differences():
         assert dx[i] == pytest.approx(fd, rel=1e-6, abs=1e-9)
         fdg = (np.dot(dy, O.rms_norm(x, g + e)) - np.dot(dy, O.rms_norm(x, g - e))) / 2e-6
         assert dg[i] == pytest.approx(fdg, rel=1e-6, abs=1e-9)
+
+
+# ---------------------------------------------------------------- prefill shape
+def _tiny_prefill(seed=5, T=256, G=2):
+    rng = np.random.default_rng(seed)
+    k = rng.standard_normal((T, 128))
+    k += np.repeat(0.5 * rng.standard_normal((T // 64, 128)), 64, axis=0)  # distinct blocks
+    v = rng.standard_normal((T, 128))
+    q = rng.standard_normal((G, T, 128))
+    w_q = rng.standard_normal((G, 128, 128)) / math.sqrt(128)
+    w_k = rng.standard_normal((384, 128)) / math.sqrt(384)
+    g_q = 1.0 + 0.25 * rng.standard_normal(128)
+    g_k = 1.0 + 0.25 * rng.standard_normal(128)
+    d_out = rng.standard_normal((G, T, 128))
+    # fixed block lists (any ascending lists ending with the query block are
+    # valid: the Top-K is held fixed); block 1 is chosen by two query blocks
+    sels = [[0], [0, 1], [1, 2], [0, 1, 3]]
+    return dict(q=q, k=k, v=v, w_q=w_q, w_k=w_k, g_q=g_q, g_k=g_k, d_out=d_out, sels=sels)
+
+
+def _pf_grads(t):
+    return O.prefill_gate_grads(t["q"], t["k"], t["v"], t["w_q"], t["g_q"], t["w_k"], t["g_k"], t["sels"],
+                                t["d_out"])
+
+
+def _pf_fd(t, name, idx, h=1e-5):
+    arr = t[name]
+    old = arr[idx]
+    loss = lambda: O.gated_prefill_loss(t["q"], t["k"], t["v"], t["w_q"], t["g_q"], t["w_k"], t["g_k"],  # noqa: E731
+                                        t["sels"], t["d_out"])
+    arr[idx] = old + h
+    lp = loss()
+    arr[idx] = old - h
+    lm = loss()
+    arr[idx] = old
+    return (lp - lm) / (2 * h)
+
+
+def test_prefill_gate_grads_match_finite_differences():
+    """Every parameter tensor of the prefill-shaped gradient against central
+    differences of the gated prefill's loss (built from the forward
+    functions), on 4 query blocks of 2 heads with block 1 kept by two query
+    blocks (its gate key's gradient sums over both)."""
+    t = _tiny_prefill()
+    r = _pf_grads(t)
+    checks = [("w_q", "dw_q", (0, 3, 5)), ("w_q", "dw_q", (1, 100, 7)), ("w_q", "dw_q", (1, 64, 64)),
+              ("w_k", "dw_k", (2, 9)), ("w_k", "dw_k", (130, 0)), ("w_k", "dw_k", (300, 77)),
+              ("g_q", "dgamma_q", (4,)), ("g_q", "dgamma_q", (90,)),
+              ("g_k", "dgamma_k", (11,)), ("g_k", "dgamma_k", (127,))]
+    for name, key, idx in checks:
+        want = _pf_fd(t, name, idx)
+        got = r[key][idx]
+        assert abs(got - want) <= 1e-6 * max(1.0, abs(want)), (key, idx, got, want)
+    # the forward part is the prefill the GPU is compared with
+    for i in range(4):
+        fwd = O.prefill_query_block(t["q"][:, 64 * i:64 * (i + 1)], t["k"], t["v"], i,
+                                    O.gate_keys_for_sequence(t["k"], 4, t["w_k"], t["g_k"]), t["w_q"],
+                                    np.tile(t["g_q"], (2, 1)), topk=len(t["sels"][i]) - 1,
+                                    gate_mode=O.GATE_LOGSIGMOID_BIAS)
+        if list(fwd["sel"]) == t["sels"][i]:
+            assert np.allclose(fwd["out"], r["out"][:, 64 * i:64 * (i + 1)], atol=1e-12)
+
+
+def test_prefill_gradient_planted_mistakes(monkeypatch):
+    t = _tiny_prefill(seed=6)
+    idx = (1, 100, 7)
+
+    def fd_ok():
+        return abs(_pf_grads(t)["dw_q"][idx] - _pf_fd(t, "w_q", idx)) <= 1e-6 * max(1.0, abs(_pf_fd(t, "w_q", idx)))
+
+    assert fd_ok()
+    good = O.log_sigmoid_grad
+    monkeypatch.setattr(O, "log_sigmoid_grad", lambda x: 1.0 - good(x))
+    assert not fd_ok()
+    monkeypatch.setattr(O, "log_sigmoid_grad", good)
+    good_rope = O.rope_backward
+    monkeypatch.setattr(O, "rope_backward", lambda dy, pos, base=10000.0: O.rope_rotate_half(dy, pos, base))
+    assert not fd_ok()
+    monkeypatch.setattr(O, "rope_backward", good_rope)

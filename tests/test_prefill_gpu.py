@@ -233,6 +233,21 @@ def test_prefill_qwen3_14b_heads_8k():
     _check(spec, *res, sets + outs, sets_only=sets)
 
 
+def test_prefill_qwen3_14b_32k_full_size_sampled():
+    """The Qwen3-14B head layout (40 query / 8 KV heads, five heads per group)
+    at the full 32,768-token training length, budget 2,048: block lists of
+    every query block of one pair and of a spread over the other pairs,
+    outputs on a sample."""
+    spec = PrefillSpec("pf_qwen3_14b_32k", 1, 40, 8, 32768, token_budget=2048, seed=55)
+    res = _run(spec)
+    nblk = spec.seq_len // 64
+    every = [(0, 5, i) for i in range(nblk)]
+    spread = [(0, h, (97 * h + 13) % nblk) for h in range(spec.hkv) if h != 5]
+    outs = [(0, 5, 0), (0, 5, 31), (0, 0, 300), (0, 7, 511)]
+    sets = [t for t in every + spread if t not in outs]
+    _check(spec, *res, sets + outs, sets_only=sets)
+
+
 @pytest.mark.parametrize("budget", [8192, 16384])
 def test_prefill_budgets_beyond_4096(budget):
     """Budgets above 4,096 tokens (lists of up to 256 blocks; one attention
