@@ -370,6 +370,73 @@ def run_backward(args, rank, world, device):
                              kernel="gate_backward_kernel + gate_grad_reduce_kernel (sas_gate_backward)")}
 
 
+def run_prefill_backward(args, device, world):
+    """Gradient through the gates of the gated prefill (Qwen3-8B heads, batch
+    --prefill-batch x 32,768 tokens, Top-K 31 + diagonal): one
+    sas_prefill_gate_backward call per step over the block lists of a gated
+    forward call, with a seeded upstream gradient.  Tensor FLOPs counted like
+    the forward's: per tile pair 2*64*64*128 for q K^T and as much for
+    dout V^T."""
+    import torch
+    from gated_block_sparse_token_b200 import sas
+    from gated_block_sparse_token_b200.workloads import make_prefill_inputs, qwen3_8b_prefill_32k
+
+    spec = qwen3_8b_prefill_32k(batch=args.prefill_batch)
+    inp = make_prefill_inputs(spec, device)
+    B, T = spec.batch, spec.seq_len
+    nblk = T // 64
+    cfg = sas.Config(spec.hq, spec.hkv, token_budget=spec.token_budget, gate_mode=sas.GATE_LOGSIGMOID_BIAS)
+    ws = sas.make_workspace(cfg, device, batch=B, max_seq_len=T)
+    gk = torch.zeros(B, spec.hkv, nblk, 128, dtype=torch.float32, device=device)
+    out = torch.empty(B, spec.hq, T, 128, dtype=torch.bfloat16, device=device)
+    sel = torch.zeros(B, spec.hkv, nblk, cfg.max_sel, dtype=torch.int32, device=device)
+    cnt = torch.zeros(B, spec.hkv, nblk, dtype=torch.int32, device=device)
+    d_out = torch.randn(B, spec.hq, T, 128, generator=torch.Generator(device=device).manual_seed(12), device=device)
+    grads = [torch.zeros(spec.hq, 128, 128, device=device), torch.zeros(spec.hkv, 384, 128, device=device),
+             torch.zeros(128, device=device), torch.zeros(128, device=device)]
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        sas.prefill_block_sparse(cfg, inp["q"], inp["k"], inp["v"], inp["w_q"], inp["gamma_q"], inp["w_k"],
+                                 inp["gamma_k"], gk, out, ws, sel_idx=sel, sel_count=cnt, stream=stream)
+
+    def call():
+        sas.prefill_gate_backward(cfg, inp["q"], inp["k"], inp["v"], inp["w_q"], inp["gamma_q"], inp["w_k"],
+                                  inp["gamma_k"], gk, sel, cnt, d_out, *grads, ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        call()
+    torch.cuda.synchronize()
+    steps = max(1, args.prefill_steps)
+    ts = []
+    for _ in range(max(3, min(args.repeats, 7))):
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps):
+                call()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(max_over_ranks(e0.elapsed_time(e1) / 1e3 / steps, world))
+    if sas.get_device_status(ws, stream) != sas.SAS_OK:
+        raise RuntimeError("device status not OK after the prefill backward run")
+    del inp, out, d_out, grads, ws
+    torch.cuda.empty_cache()
+    t = statistics.median(ts)
+    flops = prefill_flops(nblk, spec.hq, spec.hkv, spec.token_budget, B)
+    peak, kind = measured_tensor_peak()
+    return {"workload": f"{spec.name} gated-mode gradient (W_q, W_k, gains)", "batch_per_gpu": B,
+            "calls_per_repeat": steps, "ms_per_step": round(t * 1e3, 4),
+            "timing": {"repeats": len(ts), "median_ms": round(t * 1e3, 4), "min_ms": round(min(ts) * 1e3, 4),
+                       "max_ms": round(max(ts) * 1e3, 4)},
+            "roofline": {"kernel": "prefill_bwd_attn_kernel (mma.sync) + key, reduction kernels",
+                         "bound": "tensor", "achieved": round(flops / t / 1e12, 1), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(flops / t / 1e12 / peak, 4), "peak_kind": kind,
+                         "flops_per_step": flops}}
+
+
 def run_pooling(args, device, world):
     """Pooled keys and gate keys of a whole prefill-shaped cache (the Qwen3-8B
     head layout, batch 4 x 32,768 tokens, 8 KV heads: 16,384 blocks) in one
@@ -838,6 +905,7 @@ def run_ours(args):
     bwd = None if args.skip_variants else run_backward(args, rank, world, device)
     pf = None if args.skip_prefill else run_prefill(args, device, world)
     pool = None if args.skip_prefill else run_pooling(args, device, world)
+    pf_bwd = None if (args.skip_prefill or args.skip_variants) else run_prefill_backward(args, device, world)
 
     if rank != 0:
         return
@@ -880,6 +948,8 @@ def run_ours(args):
         line["pooling"] = pool
     if bwd is not None:
         line["gate_backward"] = bwd
+    if pf_bwd is not None:
+        line["prefill_gate_backward"] = pf_bwd
     print(json.dumps(line), flush=True)
 
 

@@ -17,7 +17,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsas.so")
 TRACE_LIB = os.path.join(PKG, "libsas_trace.so")  # phase-trace build (-DSAS_PHASE_TRACE)
-SOURCES = ["sas_api.cu", "sas_decode.cu", "sas_pool.cu", "sas_prefill.cu", "sas_static.cu", "sas_backward.cu"]
+SOURCES = ["sas_api.cu", "sas_decode.cu", "sas_pool.cu", "sas_prefill.cu", "sas_static.cu", "sas_backward.cu",
+           "sas_prefill_backward.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-I" + INCLUDE]

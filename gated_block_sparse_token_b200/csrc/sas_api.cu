@@ -15,13 +15,14 @@ cudaError_t prepare_decode_kernels();
 cudaError_t prepare_pool_kernels();
 cudaError_t prepare_prefill_kernels();
 cudaError_t prepare_backward_kernels();
+cudaError_t prepare_prefill_backward_kernels();
 }
 
 namespace {
 
 using sas::kDim;
 
-constexpr int32_t kAbiVersion = 8;
+constexpr int32_t kAbiVersion = 9;
 constexpr size_t kStatusBytes = 256;  // status word + padding
 constexpr int kMaxBudget = 16384;
 constexpr int kMaxGateBlocks = 16384;
@@ -52,6 +53,7 @@ cudaError_t prepare() {
     if (g_prep_err == cudaSuccess) g_prep_err = sas::prepare_pool_kernels();
     if (g_prep_err == cudaSuccess) g_prep_err = sas::prepare_prefill_kernels();
     if (g_prep_err == cudaSuccess) g_prep_err = sas::prepare_backward_kernels();
+    if (g_prep_err == cudaSuccess) g_prep_err = sas::prepare_prefill_backward_kernels();
   });
   return g_prep_err;
 }
@@ -251,7 +253,8 @@ const char* sas_status_string(sas_status s) {
 }
 
 // Workspace layout: status header, then (batch > 0) the gate backward's
-// per-pair terms, then (batch > 0 and max_seq_len > 0) the prefill scratch.
+// per-pair terms, then (batch > 0 and max_seq_len > 0) the prefill scratch
+// and the prefill gate backward's terms.
 size_t bwd_scratch_bytes(const sas_config* cfg, int32_t batch) {
   if (cfg == nullptr || batch <= 0 || cfg->num_kv_heads <= 0 || cfg->num_q_heads <= 0 || cfg->token_budget < 64)
     return 0;
@@ -267,6 +270,9 @@ size_t sas_workspace_bytes(const sas_config* cfg, int32_t batch, int32_t max_seq
     const size_t nblk = static_cast<size_t>((max_seq_len + 63) / 64);
     bytes += prefill_scratch_bytes(batch, cfg->num_q_heads, cfg->num_kv_heads, nblk,
                                    cfg->token_budget / 64);
+    // the prefill gate backward's per-(sequence, head, block) terms
+    bytes += sas::prefill_bwd_scratch_bytes(static_cast<size_t>(batch), cfg->num_q_heads, cfg->num_kv_heads,
+                                            nblk, cfg->token_budget / 64);
   }
   return bytes;
 }
@@ -671,6 +677,102 @@ sas_status sas_gate_backward(const sas_config* cfg, const void* q, const sas_kv*
   // W_k as [Hkv * 384][128] in 64 x 64 boxes (64-row chunks of the projection)
   if (!encode_kv_map(&tmwk, w_k, static_cast<long long>(cfg->num_kv_heads) * sas::kPool)) return SAS_ERR_CUDA;
   return launch_result(sas::launch_gate_backward(p, tmk, tmv, tmwk, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sas_status sas_prefill_gate_backward(const sas_config* cfg, const void* q, const void* k, const void* v,
+                                     int32_t batch, int32_t seq_len, const void* w_q, const float* gamma_q,
+                                     const void* w_k, const float* gamma_k, const void* gate_keys,
+                                     int32_t max_gate_blocks, const int32_t* sel_idx, const int32_t* sel_count,
+                                     const float* d_out, float* dw_q, float* dw_k, float* dgamma_q,
+                                     float* dgamma_k, void* ws, size_t ws_bytes, sas_stream_t stream) {
+  sas_status st = check_config(cfg);
+  if (st != SAS_OK) return st;
+  if (batch < 0 || seq_len < 0) return SAS_ERR_INVALID_ARG;
+  if (batch == 0 || seq_len == 0) return SAS_OK;
+  if (q == nullptr || k == nullptr || v == nullptr || w_q == nullptr || gamma_q == nullptr || w_k == nullptr ||
+      gamma_k == nullptr || gate_keys == nullptr || sel_idx == nullptr || sel_count == nullptr ||
+      d_out == nullptr || dw_q == nullptr || dw_k == nullptr || dgamma_q == nullptr || dgamma_k == nullptr)
+    return SAS_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(w_q, 2) || !aligned(gamma_q, 4) ||
+      !aligned(w_k, 2) || !aligned(gamma_k, 4) || !aligned(gate_keys, 16) || !aligned(sel_idx, 4) ||
+      !aligned(sel_count, 4) || !aligned(d_out, 16) || !aligned(dw_q, 4) || !aligned(dw_k, 4) ||
+      !aligned(dgamma_q, 4) || !aligned(dgamma_k, 4))
+    return SAS_ERR_INVALID_ARG;
+  if (cfg->kv_dtype != SAS_DTYPE_BF16 || cfg->gate_keys_bf16 != 0) return SAS_ERR_UNSUPPORTED;
+  if (seq_len % 64 != 0) return SAS_ERR_UNSUPPORTED;
+  const int nblk = seq_len / 64;
+  const int max_sel = cfg->token_budget / 64;
+  if (max_gate_blocks < nblk || max_gate_blocks > kMaxGateBlocks) return SAS_ERR_INVALID_ARG;
+  if (max_sel > sas::kPbMaxSel) return SAS_ERR_UNSUPPORTED;
+  const int stages = sas::prefill_bwd_smem_bytes(max_sel, 2) <= 113 * 1024 ? 2 : 1;
+  if (sas::prefill_bwd_smem_bytes(max_sel, stages) > 227 * 1024) return SAS_ERR_UNSUPPORTED;
+  if (static_cast<long long>(nblk) * (sas::kPbChunk / 32 + 1) * 4 > 227 * 1024) return SAS_ERR_UNSUPPORTED;
+  if (static_cast<long long>(batch) * cfg->num_q_heads * seq_len > 0x7fffffffLL) return SAS_ERR_UNSUPPORTED;
+  if (batch > 65535 || cfg->num_q_heads > 65535 || nblk > 0x7fffffff) return SAS_ERR_UNSUPPORTED;
+  if (ws == nullptr || !aligned(ws, 256)) return SAS_ERR_WORKSPACE;
+  // the select-only mode gives the gate parameters no gradient
+  if (cfg->gate_mode == SAS_GATE_SELECT_ONLY) return SAS_OK;
+  if (ws_bytes < sas_workspace_bytes(cfg, batch, seq_len)) return SAS_ERR_WORKSPACE;
+  if (prepare() != cudaSuccess) return SAS_ERR_CUDA;
+  sas::PrefillBwdParams p{};
+  sas::fill_rope_table(p.rope, cfg->rope_base);
+  p.batch = batch;
+  p.hq = cfg->num_q_heads;
+  p.hkv = cfg->num_kv_heads;
+  p.G = cfg->num_q_heads / cfg->num_kv_heads;
+  p.T = seq_len;
+  p.nblk = nblk;
+  p.max_sel = max_sel;
+  p.mg = max_gate_blocks;
+  p.stages = stages;
+  p.eps = cfg->norm_eps;
+  p.attn_scale = cfg->attn_scale;
+  p.gate_scale = cfg->gate_scale;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.w_q = static_cast<const __nv_bfloat16*>(w_q);
+  p.gamma_q = gamma_q;
+  p.w_k = static_cast<const __nv_bfloat16*>(w_k);
+  p.gamma_k = gamma_k;
+  p.gate_keys = static_cast<const float*>(gate_keys);
+  p.sel_idx = sel_idx;
+  p.sel_count = sel_count;
+  p.d_out = d_out;
+  p.dw_q = dw_q;
+  p.dw_k = dw_k;
+  p.dgamma_q = dgamma_q;
+  p.dgamma_k = dgamma_k;
+  p.status = static_cast<uint32_t*>(ws);
+  {
+    // after the header, the decode backward's terms and the prefill scratch
+    const size_t B = static_cast<size_t>(batch);
+    uint8_t* w = static_cast<uint8_t*>(ws) + ws_header_bytes() + bwd_scratch_bytes(cfg, batch) +
+                 prefill_scratch_bytes(B, p.hq, p.hkv, nblk, max_sel);
+    const size_t qh = B * p.hq * nblk, kh = B * p.hkv * nblk;
+    p.ws_qbar = reinterpret_cast<float*>(w);
+    w += up256(qh * kDim * 4);
+    p.ws_qt = reinterpret_cast<float*>(w);
+    w += up256(qh * kDim * 4);
+    p.ws_dv = reinterpret_cast<float*>(w);
+    w += up256(qh * kDim * 4);
+    p.ws_dgq = reinterpret_cast<float*>(w);
+    w += up256(qh * kDim * 4);
+    p.ws_ds = reinterpret_cast<float*>(w);
+    w += up256(qh * max_sel * 4);
+    p.ws_p = reinterpret_cast<float*>(w);
+    w += up256(kh * sas::kPool * 4);
+    p.ws_du = reinterpret_cast<float*>(w);
+    w += up256(kh * kDim * 4);
+    p.ws_dgk = reinterpret_cast<float*>(w);
+    w += up256(kh * kDim * 4);
+    p.ws_gpart = reinterpret_cast<float*>(w);
+  }
+  CUtensorMap tmq, tmk, tmv;
+  const long long qrows = static_cast<long long>(batch) * p.hq * seq_len;
+  const long long krows = static_cast<long long>(batch) * p.hkv * seq_len;
+  if (!encode_kv_map(&tmq, q, qrows) || !encode_kv_map(&tmk, k, krows) || !encode_kv_map(&tmv, v, krows))
+    return SAS_ERR_CUDA;
+  return launch_result(sas::launch_prefill_gate_backward(p, tmq, tmk, tmv, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const sas_kv* kv,

@@ -251,6 +251,58 @@ inline size_t gate_bwd_scratch_bytes(size_t batch, int hq, int hkv, int max_sel)
          up256(pairs * 2 * kDim * 4) + up256(pairs * 4);
 }
 
+// Gradient through the gates of the gated prefill (block lists held fixed).
+constexpr int kPbThreads = 128;  // attention pass: 4 warps of 16 query tokens
+constexpr int kPbMaxSel = 64;    // block lists of up to 64 entries (4,096 tokens)
+constexpr int kPbChunk = 128;    // key blocks per CTA of the gate-key pass
+
+struct PrefillBwdParams {
+  RopeTable rope;
+  int batch, hq, hkv, G, T, nblk, max_sel, mg, stages;
+  float eps, attn_scale, gate_scale;
+  const __nv_bfloat16* q;      // [B][Hq][T][128]
+  const __nv_bfloat16* k;      // [B][Hkv][T][128]
+  const __nv_bfloat16* w_q;    // [Hq][128][128]
+  const float* gamma_q;        // [128]
+  const __nv_bfloat16* w_k;    // [Hkv][384][128]
+  const float* gamma_k;        // [128]
+  const float* gate_keys;      // [B][Hkv][mg][128] fp32 (the forward's)
+  const int32_t* sel_idx;      // [B][Hkv][nblk][max_sel]
+  const int32_t* sel_count;    // [B][Hkv][nblk]
+  const float* d_out;          // [B][Hq][T][128]
+  float* dw_q;                 // [Hq][128][128]  (accumulated)
+  float* dw_k;                 // [Hkv][384][128] (accumulated)
+  float* dgamma_q;             // [128]           (accumulated)
+  float* dgamma_k;             // [128]           (accumulated)
+  // per-(sequence, head, block) terms (workspace)
+  float* ws_qbar;   // [B][Hq][nblk][128] block-mean gate query
+  float* ws_qt;     // [B][Hq][nblk][128] q~
+  float* ws_dv;     // [B][Hq][nblk][128] dL/dv
+  float* ws_dgq;    // [B][Hq][nblk][128] dL/dgamma_q terms
+  float* ws_ds;     // [B][Hq][nblk][max_sel] dL/ds of each list entry
+  float* ws_p;      // [B][Hkv][nblk][384] pooled keys
+  float* ws_du;     // [B][Hkv][nblk][128] dL/du
+  float* ws_dgk;    // [B][Hkv][nblk][128] dL/dgamma_k terms
+  float* ws_gpart;  // [Hq + Hkv][128] gain sums per head
+  uint32_t* status;
+};
+
+inline size_t prefill_bwd_scratch_bytes(size_t batch, int hq, int hkv, size_t nblk, int max_sel) {
+  auto up256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t qh = batch * hq * nblk, kh = batch * hkv * nblk;
+  return 4 * up256(qh * kDim * 4) + up256(qh * max_sel * 4) + up256(kh * kPool * 4) + 2 * up256(kh * kDim * 4) +
+         up256(static_cast<size_t>(hq + hkv) * kDim * 4);
+}
+
+// Shared memory of the prefill backward's attention pass: the K/V ring, the
+// per-(entry, token) statistics (the Q tile first lands in the same region),
+// the list and its gate terms, the gate-query vectors.
+inline int prefill_bwd_smem_bytes(int max_sel, int stages) {
+  const int stats = 3 * max_sel * 64 * 4;
+  return stages * 2 * kTileBytes + (stats > kTileBytes ? stats : kTileBytes) + 4 * max_sel * 4 + 6 * kDim * 4 +
+         64 + 1024;
+}
+
 // Shared-memory bytes of the backward kernel for a group of G heads and
 // block lists of max_sel entries.
 // Row stride (floats) of the pooled keys in the backward's shared memory:
@@ -304,6 +356,8 @@ cudaError_t launch_prefill(const PrefillParams& p, const CUtensorMap& tmq, const
 size_t prefill_attn_smem_bytes(int max_sel);
 cudaError_t launch_gate_backward(const GateBwdParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                  const CUtensorMap& tmwk, cudaStream_t stream);
+cudaError_t launch_prefill_gate_backward(const PrefillBwdParams& p, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                                         const CUtensorMap& tmv, cudaStream_t stream);
 
 // One-time per-process set-up of kernel attributes.
 cudaError_t prepare_kernels();

@@ -18,7 +18,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 # SAS_LIBRARY selects another build of the same ABI (e.g. the phase-trace build).
 LIB_PATH = os.environ.get("SAS_LIBRARY", os.path.join(_HERE, "libsas.so"))
-ABI_VERSION = 8             # the include/sas.h this binding marshals for
+ABI_VERSION = 9             # the include/sas.h this binding marshals for
 
 SAS_OK = 0
 SAS_ERR_INVALID_ARG = 1
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
             "sas_decode_step_static": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]),
             "sas_gate_backward": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "sas_prefill_block_sparse": (ctypes.c_int, [cfgp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
+            "sas_prefill_gate_backward": (ctypes.c_int, [cfgp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, i32, vp, vp, vp,
+                                                         vp, vp, vp, vp, vp, sz, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -298,6 +300,22 @@ def prefill_block_sparse(cfg: Config, q, k, v, w_q, gamma_q, w_k, gamma_k, gate_
                                           int(gate_keys.shape[2]), _ptr(out), _ptr(sel_idx),
                                           _ptr(sel_count), _ptr(ws), ws.numel(), _stream(stream)),
            "sas_prefill_block_sparse")
+
+
+def prefill_gate_backward(cfg: Config, q, k, v, w_q, gamma_q, w_k, gamma_k, gate_keys, sel_idx, sel_count,
+                          d_out, dw_q, dw_k, dgamma_q, dgamma_k, ws, stream=None) -> None:
+    """sas_prefill_gate_backward: adds dL/dW_q, dL/dW_k, dL/dgamma_q, dL/dgamma_k
+    (fp32) of the gated prefill, its block lists held fixed, for d_out =
+    dL/dout [B][Hq][T][128] fp32; ws from make_workspace(cfg, device, batch=B,
+    max_seq_len=T)."""
+    _check_gk(cfg, gate_keys)
+    c = cfg.c()
+    B, T = int(q.shape[0]), int(q.shape[2])
+    _check(lib().sas_prefill_gate_backward(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), B, T, _ptr(w_q),
+                                           _ptr(gamma_q), _ptr(w_k), _ptr(gamma_k), _ptr(gate_keys),
+                                           int(gate_keys.shape[2]), _ptr(sel_idx), _ptr(sel_count), _ptr(d_out),
+                                           _ptr(dw_q), _ptr(dw_k), _ptr(dgamma_q), _ptr(dgamma_k), _ptr(ws),
+                                           ws.numel(), _stream(stream)), "sas_prefill_gate_backward")
 
 
 def out_dtype(cfg: Config) -> torch.dtype:

@@ -159,7 +159,7 @@ typedef struct {
  * configuration (status word plus any scratch).  batch and max_seq_len are
  * the largest B and L_s (decode) or T (prefill) of the calls that will use
  * it; decode steps need neither (0, 0), sas_gate_backward the batch,
- * sas_prefill_block_sparse both. */
+ * sas_prefill_block_sparse and sas_prefill_gate_backward both. */
 SAS_API size_t sas_workspace_bytes(const sas_config* cfg, int32_t batch, int32_t max_seq_len);
 
 /* Zero the status word at the start of ws (cudaMemsetAsync on `stream`). */
@@ -339,6 +339,44 @@ SAS_API sas_status sas_gate_backward(const sas_config* cfg, const void* q, const
                                      const int32_t* sel_count, const float* d_out, float* dw_q,
                                      float* dw_k, float* dgamma_q, float* dgamma_k, void* ws,
                                      size_t ws_bytes, sas_stream_t stream);
+
+/*
+ * Gradient through the gates of the gated block-sparse prefill (pages: the
+ * continuous gates on the selected blocks give a differentiable path through
+ * the discrete Top-K selection; aigc.news release paragraph of 2026-09-14).
+ * For sas_prefill_block_sparse in the gated mode (cfg->gate_mode =
+ * SAS_GATE_LOGSIGMOID_BIAS), its block lists held fixed, and an upstream
+ * gradient d_out of its output, ADDS to dw_q, dw_k, dgamma_q and dgamma_k
+ * (shapes as for sas_gate_backward; zero them first for a fresh gradient;
+ * every sum runs in a fixed order, so repeated calls add identical values).
+ * Query block i of head g carries the gate log(sigmoid(s_gib)) on the tokens
+ * of each selected historical block b, s_gib = q~_gi . k~_b * gate_scale with
+ * q~_gi from the mean of the block's 64 queries (q_bar @ W_q[g], RMSNorm,
+ * gain, RoPE at i); the gradient reaches W_q and gamma_q through every
+ * query block's gate query and W_k and gamma_k through the gate keys (pooled
+ * block @ W_k, RMSNorm, gain, RoPE at b, recomputed from the cache), summed
+ * over the query blocks that kept each key block.  The select-only mode
+ * gives no gradient: the call returns SAS_OK and enqueues nothing.
+ *   q, k, v     bf16, as for sas_prefill_block_sparse (16-byte aligned)
+ *   gate_keys   fp32 [B][Hkv][max_gate_blocks][128], the keys the forward
+ *               wrote (scores are recomputed from them); cfg->gate_keys_bf16
+ *               must be 0
+ *   sel_idx, sel_count: the forward's block lists [B][Hkv][T/64][budget/64]
+ *               and lengths [B][Hkv][T/64]; a list that is not ascending or
+ *               does not end with its query block skips that query block
+ *               and sets SAS_ERR_DEVICE_BOUNDS's bit
+ *   d_out       fp32 [B][Hq][T][128]  dL/dout (16-byte aligned)
+ *   ws          at least sas_workspace_bytes(cfg, B, T) bytes
+ * This build handles bf16 inputs, T a multiple of 64 and budgets up to
+ * 4,096 tokens; others return SAS_ERR_UNSUPPORTED.
+ */
+SAS_API sas_status sas_prefill_gate_backward(const sas_config* cfg, const void* q, const void* k, const void* v,
+                                             int32_t batch, int32_t seq_len, const void* w_q,
+                                             const float* gamma_q, const void* w_k, const float* gamma_k,
+                                             const void* gate_keys, int32_t max_gate_blocks,
+                                             const int32_t* sel_idx, const int32_t* sel_count,
+                                             const float* d_out, float* dw_q, float* dw_k, float* dgamma_q,
+                                             float* dgamma_k, void* ws, size_t ws_bytes, sas_stream_t stream);
 
 /*
  * Allocation-free variant of sas_decode_step.  The release pages have no

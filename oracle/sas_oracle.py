@@ -575,29 +575,31 @@ def prefill_gate_grads(q_seq_group, k_seq, v_seq, w_q_group, gamma_q, w_k, gamma
     for i in range(nblk):
         sel = list(sels[i])
         hist = sel[:-1]
-        toks_hist = selected_token_ids(hist, (i + 1) * BLOCK)
-        blk_hist = [t // BLOCK for t in toks_hist]
+        toks_hist = selected_token_ids(hist, (i + 1) * BLOCK)  # 64 tokens per kept block, in list order
+        k_hist, v_hist = k_seq[toks_hist], v_seq[toks_hist]
         for g in range(G):
             qbar = q_seq_group[g, i * BLOCK:(i + 1) * BLOCK].mean(axis=0)
             v = qbar @ np.asarray(w_q_group[g], np.float64)
             qt = rope_rotate_half(rms_norm(v, gamma_q, eps), i, base)
             s = np.array([float(qt @ kt[b]) * gate_scale for b in range(i)])
             s_all[(g, i)] = s
-            dbias = {b: 0.0 for b in hist}
+            bias_hist = np.repeat([log_sigmoid(s[b]) for b in hist], BLOCK)
+            dbias = np.zeros(len(hist))
             for t in range(BLOCK):
                 tok = i * BLOCK + t
-                toks = toks_hist + list(range(i * BLOCK, tok + 1))
-                bias = np.array([log_sigmoid(s[b]) for b in blk_hist] + [0.0] * (t + 1))
-                logits = (k_seq[toks] @ q_seq_group[g, tok]) * attn_scale + bias
+                k_diag, v_diag = k_seq[i * BLOCK:tok + 1], v_seq[i * BLOCK:tok + 1]
+                logits = np.concatenate([k_hist @ q_seq_group[g, tok] * attn_scale + bias_hist,
+                                         k_diag @ q_seq_group[g, tok] * attn_scale])
                 w = np.exp(logits - logits.max())
                 p = w / w.sum()
-                out[g, tok] = p @ v_seq[toks]
-                dlogit = p * (v_seq[toks] @ d_out[g, tok] - float(np.dot(d_out[g, tok], out[g, tok])))
-                for dl, b in zip(dlogit[:len(toks_hist)], blk_hist):
-                    dbias[b] += dl
+                vv = np.concatenate([v_hist, v_diag])
+                out[g, tok] = p @ vv
+                dlogit = p * (vv @ d_out[g, tok] - float(np.dot(d_out[g, tok], out[g, tok])))
+                # a kept block's bias is shared by its 64 tokens
+                dbias += dlogit[:len(toks_hist)].reshape(len(hist), BLOCK).sum(axis=1)
             dq_t = np.zeros(HEAD_DIM)
-            for b in hist:
-                ds = dbias[b] * log_sigmoid_grad(s[b])
+            for n, b in enumerate(hist):
+                ds = dbias[n] * log_sigmoid_grad(s[b])
                 dq_t += ds * gate_scale * kt[b]
                 dkt[b] += ds * gate_scale * qt
             dq_hat = rope_backward(dq_t, i, base)

@@ -33,7 +33,8 @@ def test_header_declares_all_entry_points():
     names = set(declared_functions())
     want = {"sas_pool_keys", "sas_gate_scores", "sas_topk_blocks", "sas_sparse_decode",
             "sas_decode_step", "sas_workspace_bytes", "sas_get_device_status",
-            "sas_reset_device_status", "sas_status_string", "sas_abi_version", "sas_gate_backward"}
+            "sas_reset_device_status", "sas_status_string", "sas_abi_version", "sas_gate_backward",
+            "sas_prefill_gate_backward"}
     assert want <= names
 
 
@@ -85,7 +86,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(L):
-    assert sas.abi_version() == sas.ABI_VERSION == 8
+    assert sas.abi_version() == sas.ABI_VERSION == 9
     for st in range(7):
         assert len(sas.status_string(st)) > 0
     assert sas.status_string(sas.SAS_OK) == "ok"
@@ -249,6 +250,25 @@ def test_gate_backward_validates_on_the_host(L):
     assert bwd(_cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS, kv_dtype="f32").c()) == sas.SAS_ERR_UNSUPPORTED
     # the select-only mode gives the gate parameters no gradient: nothing to do
     assert bwd(_cfg().c()) == sas.SAS_OK
+
+
+@nogpu
+def test_prefill_gate_backward_validates_on_the_host(L):
+    def bwd(c, seq_len=4096, mg=64, ws_bytes=1 << 34, dout=FAKE, batch=2):
+        return L.sas_prefill_gate_backward(ctypes.byref(c), FAKE, FAKE, FAKE, batch, seq_len, FAKE, FAKE, FAKE,
+                                           FAKE, FAKE, mg, FAKE, FAKE, dout, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                           ws_bytes, None)
+    gated = _cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS)
+    assert bwd(gated.c(), dout=None) == sas.SAS_ERR_INVALID_ARG
+    assert bwd(gated.c(), dout=FAKE + 4) == sas.SAS_ERR_INVALID_ARG               # d_out not 16-byte aligned
+    assert bwd(gated.c(), mg=63) == sas.SAS_ERR_INVALID_ARG                       # gate-key rows < T/64
+    assert bwd(gated.c(), seq_len=4000) == sas.SAS_ERR_UNSUPPORTED                # not a multiple of 64
+    assert bwd(_cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS, gate_keys_bf16=1).c()) == sas.SAS_ERR_UNSUPPORTED
+    assert bwd(_cfg(gate_mode=sas.GATE_LOGSIGMOID_BIAS, token_budget=8192).c()) == sas.SAS_ERR_UNSUPPORTED
+    need = L.sas_workspace_bytes(ctypes.byref(gated.c()), 2, 4096)
+    assert bwd(gated.c(), ws_bytes=need - 1) == sas.SAS_ERR_WORKSPACE
+    assert bwd(gated.c(), batch=0) == sas.SAS_OK
+    assert bwd(_cfg().c(), ws_bytes=256) == sas.SAS_OK  # select-only: no gradient, nothing enqueued
 
 
 @pytest.mark.parametrize("gk16", [0, 1])
