@@ -108,7 +108,8 @@ extern "C" sas_status sas_decode_step_static(const sas_config* cfg, const void* 
                                              float* group_scores, uint32_t* status_out,
                                              sas_stream_t stream) {
   if (cfg == nullptr || kv == nullptr) return SAS_ERR_INVALID_ARG;
-  if (sas_workspace_bytes(cfg, kv->batch, 0) > kStaticScratchBytes) return SAS_ERR_WORKSPACE;
+  // a decode step needs the workspace of no batch and no prefill length
+  if (sas_workspace_bytes(cfg, 0, 0) > kStaticScratchBytes) return SAS_ERR_WORKSPACE;
   if (status_out != nullptr && (reinterpret_cast<uintptr_t>(status_out) % 4) != 0)
     return SAS_ERR_INVALID_ARG;
   // every host check of the step first (any 256-aligned stand-in passes the

@@ -253,6 +253,19 @@ def test_gate_backward_validates_on_the_host(L):
 
 
 @nogpu
+def test_static_step_needs_no_batch_workspace(L):
+    """The allocation-free step's 256-byte scratch covers a decode step of any
+    batch (the workspace a decode step needs is sas_workspace_bytes(cfg, 0, 0));
+    its host checks then refuse a missing q before anything is enqueued."""
+    c = _cfg().c()
+    for batch in (1, 8, 64):
+        kv = _kv(batch=batch)
+        st = L.sas_decode_step_static(ctypes.byref(c), None, ctypes.byref(kv), FAKE, FAKE, None, None, FAKE, 64,
+                                      FAKE, None, None, None, None, None)
+        assert st == sas.SAS_ERR_INVALID_ARG, (batch, st)
+
+
+@nogpu
 def test_prefill_gate_backward_validates_on_the_host(L):
     def bwd(c, seq_len=4096, mg=64, ws_bytes=1 << 34, dout=FAKE, batch=2):
         return L.sas_prefill_gate_backward(ctypes.byref(c), FAKE, FAKE, FAKE, batch, seq_len, FAKE, FAKE, FAKE,
