@@ -200,7 +200,8 @@ SAS_API sas_status sas_pool_keys(const sas_config* cfg, const sas_kv* kv,
 
 /*
  * Gate scores of every historical block (pages: the gate ranks the KV
- * blocks so that the best can be selected; query projection Qproj).
+ * blocks so that the best can be selected; the query side goes through
+ * the projection the pages name Qproj).
  *   q            kv_dtype [B][Hq][128]  query of token L_s - 1
  *   w_q          bf16 [Hq][128][128]    gamma_q fp32 [128]
  *   gate_keys    fp32 [B][Hkv][MG][128] (from sas_pool_keys)
@@ -302,7 +303,7 @@ SAS_API sas_status sas_prefill_block_sparse(const sas_config* cfg, const void* q
 
 /*
  * Gradient through the gates (pages: the continuous gates on the selected
- * blocks give a differentiable path through the discrete Top-K selection;
+ * blocks let a gradient reach the gate despite the discrete Top-K;
  * aigc.news release paragraph of 2026-09-14).  For the gated decode step
  * (cfg->gate_mode = SAS_GATE_LOGSIGMOID_BIAS) with the block lists held fixed
  * and an upstream gradient d_out of its output, ADDS to
@@ -342,7 +343,7 @@ SAS_API sas_status sas_gate_backward(const sas_config* cfg, const void* q, const
 
 /*
  * Gradient through the gates of the gated block-sparse prefill (pages: the
- * continuous gates on the selected blocks give a differentiable path through
+ * continuous gates on the selected blocks let a gradient reach the gate past
  * the discrete Top-K selection; aigc.news release paragraph of 2026-09-14).
  * For sas_prefill_block_sparse in the gated mode (cfg->gate_mode =
  * SAS_GATE_LOGSIGMOID_BIAS), its block lists held fixed, and an upstream

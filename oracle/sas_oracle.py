@@ -73,7 +73,7 @@ R19 bf16 gate-key cache (a storage option, not a change of the method): the
     sizes fit bf16 weights).
 
 R20 Gradient through the gates (the release paragraph of [aigc-0914] says the
-    continuous gates on the selected blocks give a differentiable path
+    continuous gates on the selected blocks let a gradient reach the gate
     through the discrete Top-K; second paragraph of [nedoborov] likewise):
     in the gated mode (R18), for an upstream gradient dL/dout, the gradients
     of the gate parameters W_q, W_k, gamma_q and gamma_k flow through
@@ -152,7 +152,8 @@ def gate_key(pooled: np.ndarray, w_k: np.ndarray, gamma_k: np.ndarray, pos: int,
 
 def gate_query(q: np.ndarray, w_q: np.ndarray, gamma_q: np.ndarray, pos: int,
                eps: float = 1e-6, base: float = 10000.0) -> np.ndarray:
-    """q~ = RoPE(RMSNorm(q @ W_q), pos) ("query projection Qproj").  W_q: [128][128].
+    """q~ = RoPE(RMSNorm(q @ W_q), pos): the gate's query projection, which the
+    pages name Qproj.  W_q: [128][128].
     R1, R2, R5, R6."""
     v = np.asarray(q, np.float64) @ np.asarray(w_q, np.float64)
     return rope_rotate_half(rms_norm(v, gamma_q, eps), pos, base)
