@@ -41,8 +41,12 @@
 //            once all have arrived.
 // The CTA that owns the current block (always selected) prefetches its
 // tiles before the selection finishes and, when the decoded token completes
-// the block, pools it into the block's gate key.  No cluster barrier follows
-// the start, and every wait is bounded.
+// the block, pools it and sends the pooled vector to every CTA; each CTA
+// projects it on its 16 W_k columns inside its attention loop (after its
+// second list entry, while its warps mostly wait on tiles) and CTA 0
+// normalises and rotates the result into the block's gate key before it
+// waits for the attention partials.  No cluster barrier follows the start,
+// and every wait is bounded.
 #include <cooperative_groups.h>
 
 #include <type_traits>
@@ -1029,6 +1033,43 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
   }
 
+  // u = P @ W_k[h] for this CTA's 16 columns; slices and their sums of
+  // squares go to CTA 0, which normalises and rotates once all have come.
+  // Run inside the attention loop (after the CTA's second list entry), where
+  // the warps mostly wait on tiles; qbar (dead since the scores) is scratch.
+  bool pooled_done = false;
+  auto project_pooled = [&]() {
+    // u = P @ W_k[h] for this CTA's 16 columns; slices and their sums of
+    // squares go to CTA 0, which normalises and rotates once all have come
+    const bool okp = mbar_wait_cluster(bar_p, 0, p.status);  // the pooled block
+    const bool okw = mbar_wait(bar_wk, 0, p.status);
+    const int j = tid & (kDpc - 1);
+    const int rg = tid / kDpc;  // kThreads / kDpc row groups
+    constexpr int kRowsPer = kPool / (kThreads / kDpc);
+    float acc = 0.f;
+    if (okp && okw) {
+      float a2[2] = {0.f, 0.f};
+#pragma unroll 16
+      for (int r = 0; r < kRowsPer; ++r)
+        a2[r & 1] = fmaf(pool_p[rg * kRowsPer + r], __bfloat162float(wk_s[(rg * kRowsPer + r) * kDpc + j]),
+                         a2[r & 1]);
+      acc = a2[0] + a2[1];
+    }
+    qbar[tid] = acc;  // qbar (dead since the scores) holds the row-group sums
+    __syncthreads();
+    if (tid < kDpc) {
+      float u = 0.f;
+      for (int g = 0; g < kThreads / kDpc; ++g) u += qbar[g * kDpc + tid];
+      float sq = u * u;
+#pragma unroll
+      for (int o = kDpc / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0x0000ffffu, sq, o);
+      const uint32_t rb = dsmem_addr(bar_u, 0);
+      st_async_f32(dsmem_addr(pool_u + rank * 17 + tid, 0), u, rb);
+      if (tid == 0) st_async_f32(dsmem_addr(pool_u + rank * 17 + 16, 0), sq, rb);
+    }
+    pooled_done = true;
+  };
+
   for (int e = 0; e < cnt_mine; ++e) {
     const int b = entry_block(e);
     const int jg = entry_index(e) * G;  // gated mode: this entry's gates at gbias[jg + g]
@@ -1203,6 +1244,7 @@ __global__ void __launch_bounds__(kThreads, 4)
       __syncthreads();
       pump(t0 + 4, known);
     }
+    if (do_pool && e == min(1, cnt_mine - 1)) project_pooled();
   }
   SAS_TRACE(6);
 
@@ -1262,35 +1304,25 @@ __global__ void __launch_bounds__(kThreads, 4)
       }
     }
   }
-  if (do_pool) {
-    // u = P @ W_k[h] for this CTA's 16 columns; slices and their sums of
-    // squares go to CTA 0, which normalises and rotates once all have come
-    const bool okp = mbar_wait_cluster(bar_p, 0, p.status);  // the pooled block
-    const bool okw = mbar_wait(bar_wk, 0, p.status);
-    const int j = tid & (kDpc - 1);
-    const int rg = tid / kDpc;  // kThreads / kDpc row groups
-    constexpr int kRowsPer = kPool / (kThreads / kDpc);
-    float acc = 0.f;
-    if (okp && okw) {
-      float a2[2] = {0.f, 0.f};
-#pragma unroll 16
-      for (int r = 0; r < kRowsPer; ++r)
-        a2[r & 1] = fmaf(pool_p[rg * kRowsPer + r], __bfloat162float(wk_s[(rg * kRowsPer + r) * kDpc + j]),
-                         a2[r & 1]);
-      acc = a2[0] + a2[1];
-    }
-    qbar[tid] = acc;  // qbar (dead since the scores) holds the row-group sums
-    __syncthreads();
-    if (tid < kDpc) {
-      float u = 0.f;
-      for (int g = 0; g < kThreads / kDpc; ++g) u += qbar[g * kDpc + tid];
-      float sq = u * u;
+  if (do_pool && !pooled_done) project_pooled();
+  if (do_pool && rank == 0) {
+    // RMSNorm (gain gamma_k) and gate RoPE at position c of the pooled block
+    mbar_wait_cluster(bar_u, 0, p.status);
+    const int d = tid;
+    float ss = 0.f;
 #pragma unroll
-      for (int o = kDpc / 2; o > 0; o >>= 1) sq += __shfl_xor_sync(0x0000ffffu, sq, o);
-      const uint32_t rb = dsmem_addr(bar_u, 0);
-      st_async_f32(dsmem_addr(pool_u + rank * 17 + tid, 0), u, rb);
-      if (tid == 0) st_async_f32(dsmem_addr(pool_u + rank * 17 + 16, 0), sq, rb);
-    }
+    for (int r = 0; r < CS; ++r) ss += pool_u[r * 17 + 16];
+    const float x = pool_u[(d / kDpc) * 17 + (d % kDpc)] * (1.f / sqrtf(ss / kDim + p.eps)) * gamk_s[d];
+    qbar[d] = x;
+    __syncthreads();
+    float cs, sn;
+    rope_cos_sin(p.rope.theta_over_pi[d & 63], c, cs, sn);
+    const float y = (d < 64) ? qbar[d] * cs - qbar[d + 64] * sn : qbar[d] * cs + qbar[d - 64] * sn;
+    const size_t gi = (static_cast<size_t>(pair) * p.mg + c) * kDim + d;
+    if (p.gk16)
+      static_cast<__nv_bfloat16*>(p.gate_keys_out)[gi] = __float2bfloat16_rn(y);
+    else
+      static_cast<float*>(p.gate_keys_out)[gi] = y;
   }
   mbar_wait_cluster(bar_m, 0, p.status);  // every partial of this CTA's columns
   __syncthreads();                         // qbar is reused below
@@ -1320,25 +1352,6 @@ __global__ void __launch_bounds__(kThreads, 4)
       out[(static_cast<size_t>(s) * p.hq + h * G + g) * kDim + rank * kDpc + dd] =
           from_float<OutT>(res);
     }
-  }
-  if (do_pool && rank == 0) {
-    // RMSNorm (gain gamma_k) and gate RoPE at position c of the pooled block
-    mbar_wait_cluster(bar_u, 0, p.status);
-    const int d = tid;
-    float ss = 0.f;
-#pragma unroll
-    for (int r = 0; r < CS; ++r) ss += pool_u[r * 17 + 16];
-    const float x = pool_u[(d / kDpc) * 17 + (d % kDpc)] * (1.f / sqrtf(ss / kDim + p.eps)) * gamk_s[d];
-    qbar[d] = x;
-    __syncthreads();
-    float cs, sn;
-    rope_cos_sin(p.rope.theta_over_pi[d & 63], c, cs, sn);
-    const float y = (d < 64) ? qbar[d] * cs - qbar[d + 64] * sn : qbar[d] * cs + qbar[d - 64] * sn;
-    const size_t gi = (static_cast<size_t>(pair) * p.mg + c) * kDim + d;
-    if (p.gk16)
-      static_cast<__nv_bfloat16*>(p.gate_keys_out)[gi] = __float2bfloat16_rn(y);
-    else
-      static_cast<float*>(p.gate_keys_out)[gi] = y;
   }
   SAS_TRACE(8);
 }
