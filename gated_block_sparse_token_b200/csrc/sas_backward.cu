@@ -667,8 +667,8 @@ __global__ void __launch_bounds__(kBwThreads) gate_grad_reduce_kernel(const __gr
   } else if (blk < nq + nk) {
     // rounds of up to 32 entries: dL/du rows and this block's 16 pooled
     // columns staged in shared memory by every thread, then summed in order
-    __shared__ float sdu[32][kDim];
-    __shared__ float sp[32][kRedRows];
+    __shared__ __align__(16) float sdu[32][kDim];
+    __shared__ __align__(16) float sp[32][kRedRows];
     const int b = blk - nq;
     const int h = b / (kPool / kRedRows);
     const int r0 = (b - h * (kPool / kRedRows)) * kRedRows;
@@ -680,10 +680,18 @@ __global__ void __launch_bounds__(kBwThreads) gate_grad_reduce_kernel(const __gr
       for (int e0 = 0; e0 < nh; e0 += 32) {
         const int ne = min(32, nh - e0);
         __syncthreads();  // the previous round's reads are done
-        for (int i = tid; i < ne * kDim; i += kBwThreads)
-          sdu[i / kDim][i % kDim] = du[static_cast<size_t>(e0) * kDim + i];
-        for (int i = tid; i < ne * kRedRows; i += kBwThreads)
-          sp[i / kRedRows][i % kRedRows] = pp[static_cast<size_t>(e0 + i / kRedRows) * kPool + r0 + i % kRedRows];
+        // 16-byte loads, all of a thread's in flight at once
+        {
+          const float4* src = reinterpret_cast<const float4*>(du + static_cast<size_t>(e0) * kDim);
+          float4* dst = reinterpret_cast<float4*>(&sdu[0][0]);
+#pragma unroll 4
+          for (int i = tid; i < ne * (kDim / 4); i += kBwThreads) dst[i] = src[i];
+          if (tid < ne * (kRedRows / 4)) {
+            const int e = tid / (kRedRows / 4), c4 = tid % (kRedRows / 4);
+            reinterpret_cast<float4*>(&sp[e][0])[c4] =
+                reinterpret_cast<const float4*>(pp + static_cast<size_t>(e0 + e) * kPool + r0)[c4];
+          }
+        }
         __syncthreads();
         for (int e = 0; e < ne; ++e) {
           const float d = sdu[e][j];

@@ -540,9 +540,9 @@ __global__ void __launch_bounds__(256) prefill_bwd_keys_kernel(const __grid_cons
 constexpr int kPbRed = 16;
 
 __global__ void __launch_bounds__(256) prefill_grad_reduce_kernel(const __grid_constant__ PrefillBwdParams p) {
-  __shared__ float sx[32][kDim];
-  __shared__ float sv[32][kPbRed];
-  __shared__ float sg[32][kDim];
+  __shared__ __align__(16) float sx[32][kDim];
+  __shared__ __align__(16) float sv[32][kPbRed];
+  __shared__ __align__(16) float sg[32][kDim];
   const int tid = threadIdx.x, j = tid & (kDim - 1), rp = tid >> 7;
   constexpr int kPer = kPbRed / 2;
   const int nq = p.hq * (kDim / kPbRed);
@@ -572,13 +572,20 @@ __global__ void __launch_bounds__(256) prefill_grad_reduce_kernel(const __grid_c
   for (int n0 = 0; n0 < N; n0 += 32) {
     const int nn = min(32, N - n0);
     __syncthreads();
-    for (int x = tid; x < nn * kDim; x += 256) sx[x / kDim][x % kDim] = right(n0 + x / kDim)[x % kDim];
-    for (int x = tid; x < nn * kPbRed; x += 256) sv[x / kPbRed][x % kPbRed] = left(n0 + x / kPbRed)[r0 + x % kPbRed];
+    // 16-byte loads, all of a thread's in flight at once
+#pragma unroll 4
+    for (int x = tid; x < nn * (kDim / 4); x += 256)
+      reinterpret_cast<float4*>(&sx[x / (kDim / 4)][0])[x % (kDim / 4)] =
+          reinterpret_cast<const float4*>(right(n0 + x / (kDim / 4)))[x % (kDim / 4)];
+    if (tid < nn * (kPbRed / 4))
+      reinterpret_cast<float4*>(&sv[tid / (kPbRed / 4)][0])[tid % (kPbRed / 4)] =
+          reinterpret_cast<const float4*>(left(n0 + tid / (kPbRed / 4)) + r0)[tid % (kPbRed / 4)];
     if (gains) {
-      for (int x = tid; x < nn * kDim; x += 256) {
-        const int n = n0 + x / kDim, s = n / p.nblk, b = n - s * p.nblk;
-        sg[x / kDim][x % kDim] =
-            gterm[((static_cast<size_t>(s) * (is_q ? p.hq : p.hkv) + head) * p.nblk + b) * kDim + x % kDim];
+#pragma unroll 4
+      for (int x = tid; x < nn * (kDim / 4); x += 256) {
+        const int n = n0 + x / (kDim / 4), s = n / p.nblk, b = n - s * p.nblk;
+        reinterpret_cast<float4*>(&sg[x / (kDim / 4)][0])[x % (kDim / 4)] = reinterpret_cast<const float4*>(
+            gterm + ((static_cast<size_t>(s) * (is_q ? p.hq : p.hkv) + head) * p.nblk + b) * kDim)[x % (kDim / 4)];
       }
     }
     __syncthreads();
