@@ -22,7 +22,7 @@ namespace {
 
 using sas::kDim;
 
-constexpr int32_t kAbiVersion = 9;
+constexpr int32_t kAbiVersion = 10;
 constexpr size_t kStatusBytes = 256;  // status word + padding
 constexpr int kMaxBudget = 16384;
 constexpr int kMaxGateBlocks = 16384;
@@ -808,6 +808,31 @@ sas_status sas_decode_step(const sas_config* cfg, const void* q, const sas_kv* k
   return attention_call(sas::kModeFused, cfg, q, kv, w_q, gamma_q, w_k, gamma_k, gate_keys,
                         max_gate_blocks, out, sel_idx, sel_count, group_scores, ws, ws_bytes,
                         stream);
+}
+
+sas_status sas_decode_step_host(const sas_config* cfg, const void* q_host, void* q_dev,
+                                const sas_kv* kv, const void* w_q, const float* gamma_q,
+                                const void* w_k, const float* gamma_k, void* gate_keys,
+                                int32_t max_gate_blocks, void* out_dev, void* out_host,
+                                int32_t* sel_idx, int32_t* sel_count, float* group_scores,
+                                void* ws, size_t ws_bytes, sas_stream_t stream) {
+  bool launch = false;
+  sas_status st = check_attention_args(sas::kModeFused, cfg, q_dev, kv, w_q, gamma_q, w_k, gamma_k,
+                                       gate_keys, max_gate_blocks, out_dev, sel_idx, sel_count,
+                                       group_scores, ws, ws_bytes, &launch);
+  if (st != SAS_OK || !launch) return st;
+  if (q_host == nullptr || out_host == nullptr) return SAS_ERR_INVALID_ARG;
+  const size_t elems = static_cast<size_t>(kv->batch) * cfg->num_q_heads * kDim;
+  const size_t q_bytes = elems * (cfg->kv_dtype == SAS_DTYPE_F32 ? 4 : 2);
+  const size_t out_bytes = elems * (cfg->out_dtype == SAS_DTYPE_F32 ? 4 : 2);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = launch_result(cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s));
+  if (st != SAS_OK) return st;
+  st = attention_call(sas::kModeFused, cfg, q_dev, kv, w_q, gamma_q, w_k, gamma_k, gate_keys,
+                      max_gate_blocks, out_dev, sel_idx, sel_count, group_scores, ws, ws_bytes,
+                      stream);
+  if (st != SAS_OK) return st;
+  return launch_result(cudaMemcpyAsync(out_host, out_dev, out_bytes, cudaMemcpyDeviceToHost, s));
 }
 
 }  // extern "C"

@@ -18,7 +18,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 # SAS_LIBRARY selects another build of the same ABI (e.g. the phase-trace build).
 LIB_PATH = os.environ.get("SAS_LIBRARY", os.path.join(_HERE, "libsas.so"))
-ABI_VERSION = 9             # the include/sas.h this binding marshals for
+ABI_VERSION = 10            # the include/sas.h this binding marshals for
 
 SAS_OK = 0
 SAS_ERR_INVALID_ARG = 1
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
             "sas_sparse_decode": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]),
             "sas_decode_step_static": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp]),
+            "sas_decode_step_host": (ctypes.c_int, [cfgp, vp, vp, kvp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp,
+                                                    sz, vp]),
             "sas_gate_backward": (ctypes.c_int, [cfgp, vp, kvp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "sas_prefill_block_sparse": (ctypes.c_int, [cfgp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, sz, vp]),
             "sas_prefill_gate_backward": (ctypes.c_int, [cfgp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, i32, vp, vp, vp,
@@ -257,6 +259,22 @@ def decode_step(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out, ws, s
                                  int(gate_keys.shape[2]), _ptr(out), _ptr(sel_idx), _ptr(sel_count),
                                  _ptr(group_scores), _ptr(ws), ws.numel(), _stream(stream)),
            "sas_decode_step")
+
+
+def decode_step_host(cfg: Config, q_host, q_dev, kv: KvCache, w_q, gamma_q, gate_keys, out_dev, out_host, ws,
+                     sel_idx=None, sel_count=None, group_scores=None, w_k=None, gamma_k=None,
+                     stream=None) -> None:
+    """sas_decode_step_host: the step with q and out in host memory (pinned
+    CPU tensors keep the copies asynchronous); q_dev / out_dev are device
+    staging buffers of the same shapes.  out_host holds the output once the
+    stream has passed the call."""
+    _check_gk(cfg, gate_keys)
+    c, k = cfg.c(), kv.c()
+    _check(lib().sas_decode_step_host(ctypes.byref(c), _ptr(q_host), _ptr(q_dev), ctypes.byref(k), _ptr(w_q),
+                                      _ptr(gamma_q), _ptr(w_k), _ptr(gamma_k), _ptr(gate_keys),
+                                      int(gate_keys.shape[2]), _ptr(out_dev), _ptr(out_host), _ptr(sel_idx),
+                                      _ptr(sel_count), _ptr(group_scores), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "sas_decode_step_host")
 
 
 def decode_step_static(cfg: Config, q, kv: KvCache, w_q, gamma_q, gate_keys, out, sel_idx=None,

@@ -264,6 +264,33 @@ SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const s
                                    size_t ws_bytes, sas_stream_t stream);
 
 /*
+ * The fused decode step with the query and the output in host memory, for a
+ * serving loop that makes one call per step: enqueues on `stream`, in this
+ * order, the copy of q_host into q_dev, sas_decode_step on q_dev and out_dev,
+ * and the copy of out_dev into out_host.  out_host holds the step's output
+ * once the stream has passed this call (synchronise on the stream, or on an
+ * event recorded after the call).
+ *   q_host   host memory, kv_dtype [B][Hq][128]
+ *   q_dev    device memory of the same size, 16-byte aligned (overwritten)
+ *   out_dev  device memory, out_dtype [B][Hq][128] (overwritten)
+ *   out_host host memory of the same size
+ * Page-locked host memory (cudaHostAlloc, cudaHostRegister) keeps both
+ * copies asynchronous; with pageable memory the CUDA runtime stages them and
+ * the call may block until a copy is done.  The host buffers are the
+ * caller's and must stay valid until the stream has passed the call.  Every
+ * other argument is that of sas_decode_step.  All arguments are checked
+ * before anything is enqueued (a bad one enqueues nothing); SAS_ERR_CUDA
+ * from a copy or the launch leaves what was enqueued before it in place.
+ */
+SAS_API sas_status sas_decode_step_host(const sas_config* cfg, const void* q_host, void* q_dev,
+                                        const sas_kv* kv, const void* w_q, const float* gamma_q,
+                                        const void* w_k, const float* gamma_k, void* gate_keys,
+                                        int32_t max_gate_blocks, void* out_dev, void* out_host,
+                                        int32_t* sel_idx, int32_t* sel_count,
+                                        float* group_scores, void* ws, size_t ws_bytes,
+                                        sas_stream_t stream);
+
+/*
  * Block-sparse chunked prefill (pages: training Top-K 31 historical blocks
  * over 32,768-token sequences, 64-token blocks, gate with Qproj, Q/K
  * normalisation and gate RoPE).  For every 64-token query block i of every

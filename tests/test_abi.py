@@ -34,7 +34,7 @@ def test_header_declares_all_entry_points():
     want = {"sas_pool_keys", "sas_gate_scores", "sas_topk_blocks", "sas_sparse_decode",
             "sas_decode_step", "sas_workspace_bytes", "sas_get_device_status",
             "sas_reset_device_status", "sas_status_string", "sas_abi_version", "sas_gate_backward",
-            "sas_prefill_gate_backward"}
+            "sas_prefill_gate_backward", "sas_decode_step_host"}
     assert want <= names
 
 
@@ -86,7 +86,7 @@ int main(void) {
 
 
 def test_abi_version_and_status_strings(L):
-    assert sas.abi_version() == sas.ABI_VERSION == 9
+    assert sas.abi_version() == sas.ABI_VERSION == 10
     for st in range(7):
         assert len(sas.status_string(st)) > 0
     assert sas.status_string(sas.SAS_OK) == "ok"
@@ -170,6 +170,28 @@ def test_workspace_and_pointer_validation(L):
 @nogpu
 def test_empty_batch_is_a_no_op(L):
     assert _decode(L, _cfg(), kv=_kv(batch=0)) == sas.SAS_OK
+
+
+def _decode_host(L, cfg, kv=None, q_host=FAKE, q_dev=FAKE, out_dev=FAKE, out_host=FAKE, ws_bytes=256):
+    c = cfg.c()
+    kv = kv or _kv()
+    return L.sas_decode_step_host(ctypes.byref(c), q_host, q_dev, ctypes.byref(kv), FAKE, FAKE, None, None,
+                                  FAKE, 64, out_dev, out_host, None, None, None, FAKE, ws_bytes, None)
+
+
+@nogpu
+def test_host_buffer_step_validates_before_any_copy(L):
+    """sas_decode_step_host checks every argument, the host buffers included,
+    before it enqueues its first copy; an empty batch enqueues nothing."""
+    cfg = _cfg()
+    assert _decode_host(L, cfg, q_host=None) == sas.SAS_ERR_INVALID_ARG
+    assert _decode_host(L, cfg, out_host=None) == sas.SAS_ERR_INVALID_ARG
+    assert _decode_host(L, cfg, q_dev=None) == sas.SAS_ERR_INVALID_ARG
+    assert _decode_host(L, cfg, q_dev=FAKE + 4) == sas.SAS_ERR_INVALID_ARG    # bulk-copied: 16 bytes
+    assert _decode_host(L, cfg, out_dev=None) == sas.SAS_ERR_INVALID_ARG
+    assert _decode_host(L, cfg, ws_bytes=8) == sas.SAS_ERR_WORKSPACE
+    assert _decode_host(L, _cfg(gate_mode=3)) == sas.SAS_ERR_INVALID_ARG
+    assert _decode_host(L, cfg, kv=_kv(batch=0), q_host=None, out_host=None) == sas.SAS_OK
 
 
 @nogpu
