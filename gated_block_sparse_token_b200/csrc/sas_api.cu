@@ -453,7 +453,7 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
                                  const float* gamma_k, void* gate_keys, int32_t max_gate_blocks,
                                  void* out, int32_t* sel_idx, int32_t* sel_count,
                                  float* group_scores, void* ws, size_t ws_bytes,
-                                 sas_stream_t stream) {
+                                 sas_stream_t stream, bool q_mapped = false) {
   bool launch = false;
   sas_status st = check_attention_args(mode, cfg, q, kv, w_q, gamma_q, w_k, gamma_k, gate_keys,
                                        max_gate_blocks, out, sel_idx, sel_count, group_scores, ws,
@@ -464,6 +464,7 @@ static sas_status attention_call(int mode, const sas_config* cfg, const void* q,
   sas::DecodeParams p{};
   fill_common(p, cfg, max_gate_blocks);
   p.q = q;
+  p.q_mapped = q_mapped ? 1 : 0;
   p.w_q = static_cast<const __nv_bfloat16*>(w_q);
   p.gamma_q = gamma_q;
   p.gate_keys = gate_keys;
@@ -810,6 +811,18 @@ sas_status sas_decode_step(const sas_config* cfg, const void* q, const sas_kv* k
                         stream);
 }
 
+// The device address of page-locked host memory (cudaHostAlloc,
+// cudaHostRegister) that this context can reach, else nullptr (pageable
+// memory).
+static void* mapped_host(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
 sas_status sas_decode_step_host(const sas_config* cfg, const void* q_host, void* q_dev,
                                 const sas_kv* kv, const void* w_q, const float* gamma_q,
                                 const void* w_k, const float* gamma_k, void* gate_keys,
@@ -826,12 +839,20 @@ sas_status sas_decode_step_host(const sas_config* cfg, const void* q_host, void*
   const size_t q_bytes = elems * (cfg->kv_dtype == SAS_DTYPE_F32 ? 4 : 2);
   const size_t out_bytes = elems * (cfg->out_dtype == SAS_DTYPE_F32 ? 4 : 2);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  st = launch_result(cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s));
-  if (st != SAS_OK) return st;
-  st = attention_call(sas::kModeFused, cfg, q_dev, kv, w_q, gamma_q, w_k, gamma_k, gate_keys,
-                      max_gate_blocks, out_dev, sel_idx, sel_count, group_scores, ws, ws_bytes,
-                      stream);
-  if (st != SAS_OK) return st;
+  // page-locked buffers move over the host link inside the step kernel (no
+  // copy engine next to the launch); pageable ones take a runtime copy
+  const void* q_src = mapped_host(q_host);
+  void* out_dst = mapped_host(out_host);
+  const bool q_mapped = q_src != nullptr && aligned(q_src, 16);
+  if (!q_mapped) {
+    st = launch_result(cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s));
+    if (st != SAS_OK) return st;
+  }
+  void* out_target = (out_dst != nullptr && aligned(out_dst, 4)) ? out_dst : out_dev;
+  st = attention_call(sas::kModeFused, cfg, q_mapped ? q_src : q_dev, kv, w_q, gamma_q, w_k, gamma_k,
+                      gate_keys, max_gate_blocks, out_target, sel_idx, sel_count, group_scores, ws,
+                      ws_bytes, stream, q_mapped);
+  if (st != SAS_OK || out_target != out_dev) return st;
   return launch_result(cudaMemcpyAsync(out_host, out_dev, out_bytes, cudaMemcpyDeviceToHost, s));
 }
 

@@ -389,12 +389,27 @@ __global__ void __launch_bounds__(kThreads, 4)
     if (MODE != kModeAttend) mbar_arrive_expect_tx(bar_v, static_cast<uint32_t>(G * kDim * 4));
     if (p.static_weights) issue_weights();
   }
+  // q in page-locked host memory: each CTA loads one eighth of the cluster's
+  // query over the host link (16 bytes a lane of warp 1) and, after the
+  // cluster barrier, stores it into every CTA's q buffer, so the link carries
+  // each byte once.  The caller guarantees that no earlier device work writes
+  // that memory, so the loads go out before the wait.
+  constexpr int kQWords = kDim * static_cast<int>(sizeof(T)) / (16 * CS);  // words per head and CTA
+  static_assert(kQWords * 16 * CS == kDim * static_cast<int>(sizeof(T)), "q rows split evenly over the cluster");
+  const bool q_sender = p.q_mapped && warp == 1 && lane < G * kQWords;
+  uint4 q_word = make_uint4(0u, 0u, 0u, 0u);
+  if (q_sender)
+    q_word = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) +
+                                            (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) *
+                                                kDim)[rank * G * kQWords + lane];
   griddep_wait();
   if (tid == 0) {
     const int L0 = p.kv.seq_lens[s];
     const int topk0 = (MODE == kModeFused) ? p.kv.topk_of(s) : 0;  // this sequence's budget
-    bulk_g2s(qraw, static_cast<const T*>(p.q) + (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim,
-             G * kDim * static_cast<uint32_t>(sizeof(T)), bar_pro);
+    if (!p.q_mapped)
+      bulk_g2s(qraw,
+               static_cast<const T*>(p.q) + (static_cast<size_t>(s) * p.hq + static_cast<size_t>(h) * G) * kDim,
+               G * kDim * static_cast<uint32_t>(sizeof(T)), bar_pro);
     if (!p.static_weights) issue_weights();
     for (int k = 0; k < nspec; ++k) {
       const int r0 = (rank + k * CS) * gk_rows;
@@ -427,6 +442,14 @@ __global__ void __launch_bounds__(kThreads, 4)
   // before any thread waits on those barriers, and every CTA runs before
   // stores reach it
   cluster_wait();
+  if (q_sender) {
+    const uint32_t off = static_cast<uint32_t>(rank * G * kQWords + lane) * 16u;
+#pragma unroll 1
+    for (int r = 0; r < CS; ++r)
+      st_async_v4_f32(dsmem_addr(reinterpret_cast<const char*>(qraw) + off, r), __uint_as_float(q_word.x),
+                      __uint_as_float(q_word.y), __uint_as_float(q_word.z), __uint_as_float(q_word.w),
+                      dsmem_addr(bar_pro, r));
+  }
   const bool pro_ok = mbar_wait(bar_pro, 0, p.status);
   SAS_TRACE(21);  // prologue copies in
   if (MODE != kModeAttend) {

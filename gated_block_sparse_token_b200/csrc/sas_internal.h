@@ -154,6 +154,8 @@ struct DecodeParams {
   // stream have finished (the caller guarantees that none writes them);
   // 0: every input is read after they have finished
   int static_weights;
+  int q_mapped;          // q is page-locked host memory at its device address:
+                         // the cluster's CTAs each load a share and broadcast it
   KvView kv;
   float* head_scores;
   float* group_scores;

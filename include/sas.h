@@ -33,7 +33,8 @@
  *     the selected blocks, each selected block weighted 1.
  *
  * Conventions for every entry point:
- *   - All tensor pointers are caller-owned DEVICE memory; the library never
+ *   - All tensor pointers are caller-owned DEVICE memory (sas_decode_step_host
+ *     also takes two host buffers); the library never
  *     allocates, frees or synchronises (except sas_get_device_status, which
  *     synchronises the given stream).
  *   - Every call validates its arguments on the host, enqueues its kernels on
@@ -265,22 +266,30 @@ SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const s
 
 /*
  * The fused decode step with the query and the output in host memory, for a
- * serving loop that makes one call per step: enqueues on `stream`, in this
- * order, the copy of q_host into q_dev, sas_decode_step on q_dev and out_dev,
- * and the copy of out_dev into out_host.  out_host holds the step's output
- * once the stream has passed this call (synchronise on the stream, or on an
- * event recorded after the call).
+ * serving loop that makes one call per step: enqueues on `stream` the move of
+ * q_host into q_dev, sas_decode_step on q_dev, and the move of the output
+ * into out_host.  out_host holds the step's output once the stream has
+ * passed this call (synchronise on the stream, or on an event recorded after
+ * the call).
  *   q_host   host memory, kv_dtype [B][Hq][128]
- *   q_dev    device memory of the same size, 16-byte aligned (overwritten)
- *   out_dev  device memory, out_dtype [B][Hq][128] (overwritten)
+ *   q_dev    device memory of the same size, 16-byte aligned (overwritten
+ *            when q_host is pageable, else untouched)
+ *   out_dev  device memory, out_dtype [B][Hq][128] (overwritten when
+ *            out_host is pageable, else untouched)
  *   out_host host memory of the same size
- * Page-locked host memory (cudaHostAlloc, cudaHostRegister) keeps both
- * copies asynchronous; with pageable memory the CUDA runtime stages them and
- * the call may block until a copy is done.  The host buffers are the
- * caller's and must stay valid until the stream has passed the call.  Every
- * other argument is that of sas_decode_step.  All arguments are checked
- * before anything is enqueued (a bad one enqueues nothing); SAS_ERR_CUDA
- * from a copy or the launch leaves what was enqueued before it in place.
+ * Page-locked host memory (cudaHostAlloc, cudaHostRegister) that the
+ * stream's device can address moves without the copy engine: the step
+ * kernel reads q_host over the host link (a 16-byte aligned q_host; each
+ * byte crosses the link once) and writes its output rows straight into
+ * out_host.  It may read q_host before kernels ahead of it on the stream
+ * have finished, so q_host must hold the query when the call is made and
+ * must not be written by device work enqueued before the call.  Pageable
+ * memory takes a runtime copy instead (the CUDA runtime stages it; the call
+ * may block until the copy is done).  The host buffers are the caller's and must stay valid
+ * until the stream has passed the call.  Every other argument is that of
+ * sas_decode_step.  All arguments are checked before anything is enqueued
+ * (a bad one enqueues nothing); SAS_ERR_CUDA from a copy or a launch leaves
+ * what was enqueued before it in place.
  */
 SAS_API sas_status sas_decode_step_host(const sas_config* cfg, const void* q_host, void* q_dev,
                                         const sas_kv* kv, const void* w_q, const float* gamma_q,
