@@ -324,6 +324,7 @@ def test_every_gate_key_entry_point_checks_the_dtype_first(monkeypatch, gk16):
     calls = [
         lambda: sas.decode_step_static(cfg, q, kv, None, None, wrong, q),
         lambda: sas.decode_step(cfg, q, kv, None, None, wrong, q, ws),
+        lambda: sas.decode_step_host(cfg, q, q, kv, None, None, wrong, q, q, ws),
         lambda: sas.pool_keys(cfg, kv, None, None, wrong, ws),
         lambda: sas.gate_scores(cfg, q, kv.seq_lens, None, None, wrong, None, ws),
         lambda: sas.prefill_block_sparse(cfg, q, q, q, None, None, None, None, wrong, q, ws),
