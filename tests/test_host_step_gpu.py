@@ -110,3 +110,46 @@ def test_pageable_host_buffers_give_the_same_step():
     assert sas.get_device_status(ws) == sas.SAS_OK
     assert torch.equal(pinned, pageable)
     assert torch.isfinite(pinned.float()).all()
+
+
+def _host_vs_device(spec, out_dtype, q_pinned=True, out_pinned=True):
+    """One step through sas_decode_step_host against sas_decode_step on the
+    same inputs: outputs and block lists bit-identical."""
+    inp = make_decode_inputs(spec, DEV)
+    cfg = T.config_for(spec, 512, out_dtype=out_dtype)
+    ws = sas.make_workspace(cfg, DEV)
+    gk = T.run_pool(inp, cfg, ws)
+    want = T.run_decode_step(inp, cfg, ws, gk.clone())
+    torch.cuda.synchronize()
+    q_host = inp["q"].cpu()
+    out_host = torch.full(tuple(want["out"].shape), float("nan"), dtype=want["out"].dtype)
+    if q_pinned:
+        q_host = q_host.pin_memory()
+    if out_pinned:
+        out_host = out_host.pin_memory()
+    q_dev = torch.empty_like(inp["q"])
+    out_dev = torch.empty_like(want["out"])
+    sel = torch.full_like(want["sel_idx"], -1)
+    cnt = torch.full_like(want["sel_count"], -1)
+    sas.decode_step_host(cfg, q_host, q_dev, T.kv_of(inp), inp["w_q"], inp["gamma_q"], gk.clone(), out_dev,
+                         out_host, ws, sel_idx=sel, sel_count=cnt)
+    torch.cuda.synchronize()
+    assert sas.get_device_status(ws) == sas.SAS_OK
+    assert torch.equal(cnt, want["sel_count"]) and torch.equal(sel, want["sel_idx"])
+    assert torch.equal(out_host, want["out"].cpu())
+
+
+@pytest.mark.parametrize("name,kv_dtype,out_dtype,hq,hkv", [
+    ("f32_in_f32_out_g4", "f32", "f32", 8, 2),     # four 16-byte words of q per head and CTA
+    ("f32_in_bf16_out_g4", "f32", "bf16", 8, 2),
+    ("bf16_g5", "bf16", "bf16", 10, 2),            # an odd group: ten words per CTA
+])
+def test_host_step_query_types_and_groups(name, kv_dtype, out_dtype, hq, hkv):
+    spec = DecodeSpec("host_" + name, 2, hq, hkv, [3001, 1500], (512,), kv_dtype=kv_dtype, capacity=4096, seed=64)
+    _host_vs_device(spec, out_dtype)
+
+
+@pytest.mark.parametrize("q_pinned,out_pinned", [(True, False), (False, True)])
+def test_host_step_mixed_pinned_and_pageable(q_pinned, out_pinned):
+    spec = DecodeSpec("host_mixed", 2, 8, 2, [3001, 1500], (512,), capacity=4096, seed=65)
+    _host_vs_device(spec, "bf16", q_pinned, out_pinned)
