@@ -91,7 +91,12 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     gate_backward_kernel(const __grid_constant__ GateBwdParams p, const __grid_constant__ CUtensorMap tmk,
                          const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmwk) {
   constexpr int kW = kBwThreads / 32;  // warps
-  const int pair = blockIdx.x;
+  // a cluster of two CTAs per (sequence, KV head) pair: CTA 1 streams and
+  // pools every other list entry and hands its rows to CTA 0, which carries
+  // the rest of the pass alone
+  uint32_t crank;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
+  const int pair = static_cast<int>(blockIdx.x >> 1);
   const int s = pair / p.hkv;
   const int h = pair - s * p.hkv;
   const int G = p.G;
@@ -147,19 +152,25 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       if (p.kv.block_row(s, h, b) < 0) err = true;
     }
   }
-  if (__syncthreads_or(err)) {
-    if (tid == 0) {
+  if (__syncthreads_or(err)) {  // both CTAs see the same list and leave together
+    if (tid == 0 && crank == 0) {
       raise_status(p.status, kStatusBounds);
       p.ws_nh[pair] = -1;
     }
     return;
   }
   const int nh = m - 1;  // historical entries (the current block, last, has no gate)
+  // entries e = crank, crank + 2, ...; CTA 1's rows reach CTA 0 as
+  // (pooled row unless e is the current block) + 3 G statistics each
+  const int n1 = m >> 1;
+  const int hist1 = n1 - (((m - 1) & 1) ? 1 : 0);
+  const uint32_t x_bytes = static_cast<uint32_t>(n1 * 3 * G * 4 + hist1 * kPool * 4);
 
-  // ---- K/V ring: entry e in stage e % NS (16 KiB K then 16 KiB V)
-  auto issue = [&](int e) {
-    const int st = e % NS;
-    const int row0 = static_cast<int>(p.kv.block_row(s, h, sel[e]));
+  // ---- K/V ring: the CTA's k-th entry (e = crank + 2k) in stage k % NS
+  // (16 KiB K then 16 KiB V)
+  auto issue = [&](int k) {
+    const int st = k % NS;
+    const int row0 = static_cast<int>(p.kv.block_row(s, h, sel[static_cast<int>(crank) + 2 * k]));
     uint8_t* kd = tiles + (2 * st) * kTileBytes;
     uint8_t* vd = kd + kTileBytes;
     mbar_arrive_expect_tx(&bars[st], 2 * kTileBytes);
@@ -169,15 +180,22 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     tma_load_2d(vd + 8192, &tmv, 64, row0, &bars[st]);
   };
   uint64_t* bar_w = &bars[4];  // W_k chunks (step 3)
+  uint64_t* bar_x = &bars[5];  // CTA 0: the rows CTA 1 hands over
+  const int mine = (m - static_cast<int>(crank) + 1) >> 1;  // entries of this CTA
   if (tid == 0) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
     prefetch_tensormap(&tmwk);
     for (int i = 0; i < NS; ++i) mbar_init(&bars[i], 1);
     mbar_init(bar_w, 1);
+    mbar_init(bar_x, 1);
     fence_mbar_init();
-    for (int e = 0; e < NS && e < m; ++e) issue(e);
+    if (crank == 0) mbar_arrive_expect_tx(bar_x, x_bytes);
+    for (int k = 0; k < NS && k < mine; ++k) issue(k);
   }
+  // thread 0 arrives after its barrier initialisation: CTA 1 stores into
+  // CTA 0 only after the wait that follows its list pass
+  cluster_arrive_relaxed();
 
   BWD_TRACE(1);  // list checked, ring started
   // ---- 1. gate query: v_g = q_g @ W_q[g], RMSNorm, gain, RoPE at c
@@ -246,9 +264,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   do {             \
   } while (0)
 #endif
-  for (int e = 0; e < m; ++e) {
-    const int st = e % NS;
-    const bool ok = mbar_wait(&bars[st], (e / NS) & 1, p.status);
+  for (int k = 0; k < mine; ++k) {
+    const int e = static_cast<int>(crank) + 2 * k;
+    const int st = k % NS;
+    const bool ok = mbar_wait(&bars[st], (k / NS) & 1, p.status);
     BWD_SEG(0);
     const int b = sel[e];
     const int nvalid = (b == c) ? (L - b * kBlock) : kBlock;
@@ -331,9 +350,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     }
     BWD_SEG(2);
     __syncthreads();  // every read of this stage is done, the block's values are in
-    if (tid == 0 && e + NS < m) {
+    if (tid == 0 && k + NS < mine) {
       fence_proxy_async_smem();
-      issue(e + NS);
+      issue(k + NS);
     }
     BWD_SEG(3);
     if (b != c) {  // the pooled key: quarters combined in order
@@ -375,6 +394,32 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   if (p.trace != nullptr && tid == 0 && blockIdx.x < static_cast<unsigned>(kTraceCtas))
     for (int i = 0; i < 6; ++i) p.trace[blockIdx.x * kTraceSlots + 10 + i] = seg[i];
 #endif
+
+  // ---- hand-over: CTA 1's pooled rows and statistics into CTA 0's arrays
+  // (the same places CTA 0 would have written them), 16-byte and 4-byte
+  // asynchronous stores completing bar_x's bytes; CTA 1 then leaves
+  cluster_wait();
+  if (crank == 1) {
+    const uint32_t rbar = dsmem_addr(bar_x, 0);
+    for (int i = tid; i < hist1 * (kPool / 4); i += kBwThreads) {
+      const int e = 1 + 2 * (i / (kPool / 4)), q4 = i - (i / (kPool / 4)) * (kPool / 4);
+      const float4 v = *reinterpret_cast<const float4*>(P + e * kPs + 4 * q4);
+      st_async_v4_f32(dsmem_addr(P + e * kPs + 4 * q4, 0), v.x, v.y, v.z, v.w, rbar);
+    }
+    for (int i = tid; i < n1 * G; i += kBwThreads) {
+      const int e = 1 + 2 * (i / G), g = i - (i / G) * G;
+      const int o = e * G + g;
+      st_async_f32(dsmem_addr(st_m + o, 0), st_m[o], rbar);
+      st_async_f32(dsmem_addr(st_z + o, 0), st_z[o], rbar);
+      st_async_f32(dsmem_addr(st_y + o, 0), st_y[o], rbar);
+    }
+  } else if (x_bytes > 0) {
+    mbar_wait_cluster(bar_x, 0, p.status);  // acquire at cluster scope: stores of CTA 1
+  }
+  // CTA 1 stays until CTA 0 holds every row
+  cluster_arrive_relaxed();
+  cluster_wait();
+  if (crank == 1) return;
 
   BWD_TRACE(3);  // list pass done
   // ---- 3. gate keys of the historical entries: u_e = P_e @ W_k[h], on the
@@ -717,8 +762,19 @@ __global__ void __launch_bounds__(kBwThreads) gate_grad_reduce_kernel(const __gr
 cudaError_t launch_gate_backward(const GateBwdParams& p, const CUtensorMap& tmk, const CUtensorMap& tmv,
                                  const CUtensorMap& tmwk, cudaStream_t stream) {
   const int smem = gate_bwd_smem_bytes(p.G, p.max_sel, p.stages);
-  gate_backward_kernel<<<static_cast<unsigned>(p.batch * p.hkv), kBwThreads, smem, stream>>>(p, tmk, tmv, tmwk);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * p.batch * p.hkv), 1, 1);
+  cfg.blockDim = dim3(kBwThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gate_backward_kernel, p, tmk, tmv, tmwk);
   if (e != cudaSuccess) return e;
   const unsigned nblk = static_cast<unsigned>(p.hq * (kDim / kRedRows) + p.hkv * (kPool / kRedRows) + 1);
   gate_grad_reduce_kernel<<<nblk, kBwThreads, 0, stream>>>(p);
