@@ -710,40 +710,66 @@ __global__ void __launch_bounds__(kBwThreads) gate_grad_reduce_kernel(const __gr
 #pragma unroll
     for (int k = 0; k < kPer; ++k) p.dw_q[(static_cast<size_t>(hq) * kDim + i0 + 2 * k) * kDim + j] += acc[k];
   } else if (blk < nq + nk) {
-    // rounds of up to 32 entries: dL/du rows and this block's 16 pooled
-    // columns staged in shared memory by every thread, then summed in order
-    __shared__ __align__(16) float sdu[32][kDim];
-    __shared__ __align__(16) float sp[32][kRedRows];
+    // rounds of up to 32 entries of one sequence (sequences ascending, then
+    // entries): the dL/du rows and this block's 16 pooled columns staged in
+    // shared memory, double-buffered -- the next round's 16-byte loads are
+    // in flight in registers while this round is summed in order
+    __shared__ __align__(16) float sdu[2][32][kDim];
+    __shared__ __align__(16) float sp[2][32][kRedRows];
     const int b = blk - nq;
     const int h = b / (kPool / kRedRows);
     const int r0 = (b - h * (kPool / kRedRows)) * kRedRows;
-    for (int s = 0; s < p.batch; ++s) {
-      const size_t pair = static_cast<size_t>(s) * p.hkv + h;
-      const int nh = p.ws_nh[pair];
-      const float* pp = p.ws_p + pair * MS * kPool;
-      const float* du = p.ws_du + pair * MS * kDim;
-      for (int e0 = 0; e0 < nh; e0 += 32) {
-        const int ne = min(32, nh - e0);
-        __syncthreads();  // the previous round's reads are done
-        // 16-byte loads, all of a thread's in flight at once
-        {
-          const float4* src = reinterpret_cast<const float4*>(du + static_cast<size_t>(e0) * kDim);
-          float4* dst = reinterpret_cast<float4*>(&sdu[0][0]);
-#pragma unroll 4
-          for (int i = tid; i < ne * (kDim / 4); i += kBwThreads) dst[i] = src[i];
-          if (tid < ne * (kRedRows / 4)) {
-            const int e = tid / (kRedRows / 4), c4 = tid % (kRedRows / 4);
-            reinterpret_cast<float4*>(&sp[e][0])[c4] =
-                reinterpret_cast<const float4*>(pp + static_cast<size_t>(e0 + e) * kPool + r0)[c4];
-          }
-        }
-        __syncthreads();
-        for (int e = 0; e < ne; ++e) {
-          const float d = sdu[e][j];
+    constexpr int kDuVec = 32 * (kDim / 4) / kBwThreads;  // float4 of dL/du per thread and round
+    auto nh_of = [&](int s) { return max(p.ws_nh[s * p.hkv + h], 0); };
+    float4 rdu[kDuVec];
+    float4 rsp = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto fetch = [&](int s, int e0, int ne) {
+      const size_t pr = static_cast<size_t>(s) * p.hkv + h;
+      const float4* src = reinterpret_cast<const float4*>(p.ws_du + (pr * MS + e0) * kDim);
 #pragma unroll
-          for (int k = 0; k < kPer; ++k) acc[k] = fmaf(sp[e][rp + 2 * k], d, acc[k]);
-        }
+      for (int q = 0; q < kDuVec; ++q) {
+        const int i = tid + q * kBwThreads;
+        rdu[q] = (i < ne * (kDim / 4)) ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      if (tid < ne * (kRedRows / 4)) {
+        const int e = tid / (kRedRows / 4), c4 = tid % (kRedRows / 4);
+        rsp = reinterpret_cast<const float4*>(p.ws_p + (pr * MS + e0 + e) * kPool + r0)[c4];
+      }
+    };
+    auto stash = [&](int buf, int ne) {
+#pragma unroll
+      for (int q = 0; q < kDuVec; ++q) {
+        const int i = tid + q * kBwThreads;
+        if (i < ne * (kDim / 4)) reinterpret_cast<float4*>(&sdu[buf][0][0])[i] = rdu[q];
+      }
+      if (tid < ne * (kRedRows / 4))
+        reinterpret_cast<float4*>(&sp[buf][tid / (kRedRows / 4)][0])[tid % (kRedRows / 4)] = rsp;
+    };
+    int s = 0, e0 = 0;
+    while (s < p.batch && nh_of(s) == 0) ++s;
+    int ne = (s < p.batch) ? min(32, nh_of(s)) : 0;
+    if (s < p.batch) fetch(s, e0, ne);
+    for (int buf = 0; s < p.batch; buf ^= 1) {
+      // the reads of this buffer two rounds ago ended before the barrier of
+      // the last round
+      stash(buf, ne);
+      __syncthreads();
+      int s2 = s, e2 = e0 + 32;
+      if (e2 >= nh_of(s2)) {
+        e2 = 0;
+        ++s2;
+        while (s2 < p.batch && nh_of(s2) == 0) ++s2;
+      }
+      const int ne2 = (s2 < p.batch) ? min(32, nh_of(s2) - e2) : 0;
+      if (s2 < p.batch) fetch(s2, e2, ne2);
+      for (int e = 0; e < ne; ++e) {
+        const float d = sdu[buf][e][j];
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) acc[k] = fmaf(sp[buf][e][rp + 2 * k], d, acc[k]);
+      }
+      s = s2;
+      e0 = e2;
+      ne = ne2;
     }
 #pragma unroll
     for (int k = 0; k < kPer; ++k) p.dw_k[(static_cast<size_t>(h) * kPool + r0 + rp + 2 * k) * kDim + j] += acc[k];
