@@ -267,8 +267,15 @@ def decode_step_host(cfg: Config, q_host, q_dev, kv: KvCache, w_q, gamma_q, gate
     """sas_decode_step_host: the step with q and out in host memory (pinned
     CPU tensors keep the copies asynchronous); q_dev / out_dev are device
     staging buffers of the same shapes.  out_host holds the output once the
-    stream has passed the call."""
+    stream has passed the call.  The library sizes both transfers from the
+    config, so each host tensor must be a contiguous CPU tensor of its
+    staging buffer's shape and dtype (checked here)."""
     _check_gk(cfg, gate_keys)
+    for name, h, d in (("q_host", q_host, q_dev), ("out_host", out_host, out_dev)):
+        if h.device.type != "cpu" or not h.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU tensor")
+        if h.shape != d.shape or h.dtype != d.dtype:
+            raise ValueError(f"{name} is {tuple(h.shape)} {h.dtype}, its device buffer {tuple(d.shape)} {d.dtype}")
     c, k = cfg.c(), kv.c()
     _check(lib().sas_decode_step_host(ctypes.byref(c), _ptr(q_host), _ptr(q_dev), ctypes.byref(k), _ptr(w_q),
                                       _ptr(gamma_q), _ptr(w_k), _ptr(gamma_k), _ptr(gate_keys),

@@ -194,6 +194,28 @@ def test_host_buffer_step_validates_before_any_copy(L):
     assert _decode_host(L, cfg, kv=_kv(batch=0), q_host=None, out_host=None) == sas.SAS_OK
 
 
+def test_host_step_binding_refuses_mismatched_host_buffers(monkeypatch):
+    """The library sizes the host transfers from the config: the binding
+    refuses a host tensor whose shape, dtype or placement disagrees with its
+    staging buffer before any library call."""
+    def no_library():
+        raise AssertionError("the library was called before the buffer check")
+
+    monkeypatch.setattr(sas, "lib", no_library)
+    cfg = sas.Config(8, 2)
+    kv = sas.KvCache(torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16),
+                     torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16), torch.ones(1, dtype=torch.int32))
+    gk = torch.zeros(1, 2, 4, 128)
+    ws = torch.zeros(256, dtype=torch.uint8)
+    dev = torch.zeros(1, 8, 128, dtype=torch.bfloat16)   # stands for a device buffer
+    good = torch.zeros(1, 8, 128, dtype=torch.bfloat16)
+    for q_host, out_host in ((torch.zeros(1, 4, 128, dtype=torch.bfloat16), good),
+                             (good, torch.zeros(1, 8, 128, dtype=torch.float32)),
+                             (torch.zeros(1, 8, 256, dtype=torch.bfloat16)[..., :128], good)):
+        with pytest.raises(ValueError):
+            sas.decode_step_host(cfg, q_host, dev, kv, None, None, gk, dev, out_host, ws)
+
+
 @nogpu
 def test_other_entry_points_validate(L):
     c = _cfg(token_budget=96).c()
