@@ -243,7 +243,11 @@ SAS_API sas_status sas_sparse_decode(const sas_config* cfg, const void* q, const
                              void* out, void* ws, size_t ws_bytes, sas_stream_t stream);
 
 /*
- * Fused decode step: gate query, scores, Top-K and block-sparse attention in
+ * Fused decode step (pages: for each decoded token the gate ranks the
+ * historical blocks, the best are kept under the token budget with the
+ * current block, and attention runs over those blocks only; aigc.news
+ * release paragraph of 2026-09-14): gate query, scores, Top-K and
+ * block-sparse attention in
  * one launch (one thread-block cluster per (sequence, KV head); the cluster's
  * CTAs split the gate keys and the selected blocks and merge through
  * distributed shared memory).
@@ -265,8 +269,9 @@ SAS_API sas_status sas_decode_step(const sas_config* cfg, const void* q, const s
                                    size_t ws_bytes, sas_stream_t stream);
 
 /*
- * The fused decode step with the query and the output in host memory, for a
- * serving loop that makes one call per step: enqueues on `stream` the move of
+ * The fused decode step with the query and the output in host memory.  The
+ * release pages have no counterpart: the operation is sas_decode_step's, for
+ * a serving loop that makes one call per step: enqueues on `stream` the move of
  * q_host into q_dev, sas_decode_step on q_dev, and the move of the output
  * into out_host.  out_host holds the step's output once the stream has
  * passed this call (synchronise on the stream, or on an event recorded after
