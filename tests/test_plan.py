@@ -112,3 +112,29 @@ def test_prefill_attention_keeps_two_ctas_per_sm():
     # two CTAs per SM up to the 4,096-token budget, one beyond
     assert all(2 * (b + 1024) <= 228 * 1024 for b in sizes[:64]), max(sizes[:64])
     assert all(b <= 227 * 1024 for b in sizes), max(sizes)
+
+
+def test_gate_backward_ring_fits_every_accepted_shape():
+    """The gate backward (a cluster of two CTAs per pair, one CTA per SM)
+    takes as many K/V ring stages as fit: every group of 1 to 8 heads and
+    every list of up to 64 blocks (budgets to 4,096 tokens) gets at least one
+    within 227 KiB, the benchmark shape (4 heads, 32 blocks) the full four,
+    and the second CTA's hand-over (a pooled row of 384 floats per
+    historical entry, 3 statistics per head and entry, for half the list)
+    stays far inside an mbarrier's transaction count."""
+    with tempfile.TemporaryDirectory() as d:
+        exe = os.path.join(d, "bwd_plan_check")
+        subprocess.run(["/usr/local/cuda/bin/nvcc", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
+                        "-I", CSRC, "-I", os.path.join(ROOT, "include"),
+                        os.path.join(ROOT, "tests", "native", "bwd_plan_check.cu"), "-o", exe],
+                       check=True, capture_output=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    rows = [{k: int(v) for k, v in (f.split("=") for f in line.split())} for line in out.splitlines()]
+    assert len(rows) == 8 * 64
+    for r in rows:
+        assert 1 <= r["stages"] <= 4 and r["bytes"] <= 227 * 1024, r
+        m = r["max_sel"]
+        handover = (m // 2) * 3 * r["G"] * 4 + (m // 2) * 384 * 4
+        assert handover < (1 << 20) - 1
+    bench = next(r for r in rows if r["G"] == 4 and r["max_sel"] == 32)
+    assert bench["stages"] == 4
